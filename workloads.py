@@ -1,0 +1,209 @@
+"""Seeded synthetic workloads for QSA (shared by the tests and the benchmark).
+
+This module only draws inputs.  It computes no output of the method: no
+pooling, scoring, selection or attention.  The one piece of arithmetic it
+carries is the inverse position rotation used to plant "needles" whose
+direction must survive the rotation the method applies; it builds inputs and
+is written here on its own, independent of the oracle and of the CUDA path.
+
+Workload shapes follow the pages ("Qwen3.8-Flash-Next: Day-0 Support in
+SGLang", "Qwen Sparse Attention: Retrieve Coarsely, Attend Precisely";
+"Qwen3.8-Flash-Next, Layer by Layer", "Token mixing"): an indexer of 4 query
+heads and one shared 128-dim key head, blocks of 4 tokens, top-512 blocks.
+
+Conventions
+  * indexer inputs are RAW (before RoPE): the method rotates them itself;
+  * attention q and k are given AFTER the attention layer's RoPE (the sparse
+    attention consumes rotated q/k, as a paged KV cache stores them);
+  * all tensors are contiguous: q_idx [B][T][4][128], k_idx [B][T][128],
+    q [B][T][Hq][d], k/v [B][T][Hkv][d].
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import torch
+
+IDX_HEADS = 4
+IDX_DIM = 128
+BLOCK = 4
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    kind: str                 # "prefill" or "decode"
+    B: int
+    T: int                    # prefill tokens, or decode cache length before the new token
+    top_k: int
+    Hq: int
+    Hkv: int
+    d: int
+    dtype: str                # "bf16" or "fp32"
+    seed: int
+    rope_base: float = 10000.0
+    pos_scale: float = 1.0
+    needles: int = 0
+    heavy_tail: bool = False
+    extra: dict = field(default_factory=dict)
+
+
+WORKLOADS = {
+    "tiny_prefill_t1k_fp32": Workload("tiny_prefill_t1k_fp32", "prefill", 1, 1024, 64, 8, 1, 128,
+                                      "fp32", 1001),
+    "prefill_t32k_needles": Workload("prefill_t32k_needles", "prefill", 1, 32768, 512, 16, 2, 128,
+                                     "bf16", 1002, needles=64),
+    "decode_b64_l128k": Workload("decode_b64_l128k", "decode", 64, 131072, 512, 16, 2, 128,
+                                 "bf16", 1003),
+    "prefill_t128k_heavytail": Workload("prefill_t128k_heavytail", "prefill", 1, 131072, 512, 16, 2,
+                                        128, "bf16", 1004, heavy_tail=True),
+    "decode_b8_l1m_scale4": Workload("decode_b8_l1m_scale4", "decode", 8, 1048576, 512, 16, 2, 128,
+                                     "bf16", 1005, pos_scale=4.0),
+}
+
+
+def torch_dtype(w: Workload):
+    return torch.bfloat16 if w.dtype == "bf16" else torch.float32
+
+
+def _gen(device, seed):
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return g
+
+
+def _randn(shape, g, device, dtype=torch.float32):
+    return torch.randn(shape, generator=g, device=device, dtype=dtype)
+
+
+def _heavy_scale(n, g, device):
+    """Per-vector norm multiplier s = u^(-1/1.5), u ~ U(0,1], clipped at 64
+    (a Pareto tail with alpha = 1.5)."""
+    u = torch.rand(n, generator=g, device=device, dtype=torch.float32)
+    u = 1.0 - u                      # (0, 1]
+    return torch.clamp(u.pow(-1.0 / 1.5), max=64.0)
+
+
+def _inverse_rotation(u: torch.Tensor, pos: float, base: float, pos_scale: float) -> torch.Tensor:
+    """Return x with rotate-half rotation R(pos) x == u (fp64).  Pairs
+    (i, i + 64) turn by (pos / pos_scale) * base^(-2i/128); the inverse turns
+    by the negative angle."""
+    half = IDX_DIM // 2
+    i = torch.arange(half, dtype=torch.float64, device=u.device)
+    ang = (pos / pos_scale) * torch.pow(torch.tensor(base, dtype=torch.float64, device=u.device),
+                                        -(2.0 * i) / IDX_DIM)
+    c, s = torch.cos(-ang), torch.sin(-ang)
+    a, b = u[..., :half], u[..., half:]
+    return torch.cat([a * c - b * s, b * c + a * s], dim=-1)
+
+
+def make_prefill(w: Workload, device="cuda", T: int | None = None):
+    """Inputs of a prefill workload (optionally truncated to T tokens).
+
+    Returns dict(q_idx, k_idx, q, k, v, needles) with needles a list of
+    (block, [query positions]) when the workload plants them.
+    """
+    assert w.kind == "prefill"
+    T = T or w.T
+    g = _gen(device, w.seed)
+    B = w.B
+    dt = torch_dtype(w)
+    q_idx = _randn((B, T, IDX_HEADS, IDX_DIM), g, device)
+    k_idx = _randn((B, T, IDX_DIM), g, device)
+    q = _randn((B, T, w.Hq, w.d), g, device)
+    k = _randn((B, T, w.Hkv, w.d), g, device)
+    v = _randn((B, T, w.Hkv, w.d), g, device)
+    needles = []
+    if w.heavy_tail:
+        k_idx *= _heavy_scale(B * T, g, device).view(B, T, 1)
+        k *= _heavy_scale(B * T * w.Hkv, g, device).view(B, T, w.Hkv, 1)
+    if w.needles:
+        needles = _plant_needles(w, T, g, device, q_idx, k_idx, q, k)
+    return dict(q_idx=q_idx.to(dt).contiguous(), k_idx=k_idx.to(dt).contiguous(),
+                q=q.to(dt).contiguous(), k=k.to(dt).contiguous(), v=v.to(dt).contiguous(),
+                needles=needles)
+
+
+def _plant_needles(w, T, g, device, q_idx, k_idx, q, k, alpha=8.0, beta=8.0, per_needle=16,
+                   min_query=2048):
+    """Plant `w.needles` blocks whose indexer keys (after the method's pooling
+    and rotation) point along a unit direction u_j, and add beta * u_j (in
+    the rotated frame) to the indexer queries of 16 later positions per
+    needle, drawn from [max(min_query, 4b+4), T).  The attention keys of the
+    block and the queries at those positions get the same direction, so the
+    attention mass follows the needle too.  Needles need T > min_query + 4."""
+    nblk = T // BLOCK
+    B = w.B
+    hi = min(nblk, (T - 4) // BLOCK)
+    perm = torch.randperm(hi, generator=g, device=device)[: w.needles]
+    out = []
+    for j in range(w.needles):
+        b = int(perm[j])
+        u = _randn((IDX_DIM,), g, device).double()
+        u = u / u.norm()
+        ua = _randn((w.d,), g, device).double()
+        ua = ua / ua.norm()
+        lo = max(min_query, BLOCK * b + BLOCK)
+        if lo >= T:
+            continue
+        ts = torch.randint(lo, T, (per_needle,), generator=g, device=device).tolist()
+        for bi in range(B):
+            for i in range(BLOCK):
+                tok = BLOCK * b + i
+                k_idx[bi, tok] = (alpha * _inverse_rotation(u, BLOCK * b, w.rope_base, w.pos_scale)
+                                  + 0.1 * _randn((IDX_DIM,), g, device).double()).float()
+                k[bi, tok] = (alpha * ua + 0.1 * _randn((w.Hkv, w.d), g, device).double()).float()
+            for t in ts:
+                add = beta * _inverse_rotation(u, t, w.rope_base, w.pos_scale)
+                q_idx[bi, t] += add.float().view(1, IDX_DIM)
+                q[bi, t] += (beta * ua).float().view(1, w.d)
+        out.append((b, sorted(set(ts))))
+    return out
+
+
+def make_decode(w: Workload, device="cuda", L: int | None = None, B: int | None = None,
+                ragged: bool = False):
+    """Inputs of a decode workload.
+
+    Each sequence i has a cache of L_i tokens before the new one (L, or with
+    ragged=True L - (i mod 4), which covers tails 0..3 and in-step pooling).
+    Returns dict(k_idx [B][Lmax][128] raw indexer keys of the cache,
+                 q_idx [B][4][128], k_idx_new [B][128] raw indexer key of the
+                 new token, q [B][Hq][d], k, v [B][Lmax+1][Hkv][d] caches that
+                 already hold the new token at position L_i, seq_len [B]
+                 int32 = L_i + 1).
+    """
+    assert w.kind == "decode"
+    L = L or w.T
+    B = B or w.B
+    g = _gen(device, w.seed)
+    dt = torch_dtype(w)
+    lens = [L - (i % 4 if ragged else 0) for i in range(B)]
+    Lmax = max(lens)
+    k_idx = _randn((B, Lmax, IDX_DIM), g, device, dt)
+    q_idx = _randn((B, IDX_HEADS, IDX_DIM), g, device, dt)
+    k_idx_new = _randn((B, IDX_DIM), g, device, dt)
+    q = _randn((B, w.Hq, w.d), g, device, dt)
+    k = _randn((B, Lmax + 1, w.Hkv, w.d), g, device, dt)
+    v = _randn((B, Lmax + 1, w.Hkv, w.d), g, device, dt)
+    seq_len = torch.tensor([x + 1 for x in lens], dtype=torch.int32, device=device)
+    return dict(k_idx=k_idx, q_idx=q_idx, k_idx_new=k_idx_new, q=q, k=k, v=v, seq_len=seq_len,
+                lens=lens)
+
+
+def sample_rows(T: int, needles=(), n_uniform: int = 2048, seed: int = 7) -> list[int]:
+    """Query rows checked at full size: the first and last 16, four around
+    every multiple of 2048, all needle queries, and n_uniform uniform rows."""
+    rows = set(range(min(16, T))) | set(range(max(0, T - 16), T))
+    for m in range(2048, T, 2048):
+        rows |= {m - 2, m - 1, m, m + 1}
+    for _, ts in needles:
+        rows |= set(ts)
+    g = torch.Generator().manual_seed(seed)
+    rows |= set(torch.randint(0, T, (n_uniform,), generator=g).tolist())
+    return sorted(r for r in rows if 0 <= r < T)
+
+
+def scale_default(d: int) -> float:
+    return 1.0 / math.sqrt(d)
