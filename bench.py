@@ -1,0 +1,453 @@
+"""Benchmark of the QSA hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole hot path over one batch of synthetic input:
+  prefill workloads: compressed-key pooling + indexer (query rotation, block
+    scores, per-row top-k) + sparse attention over the selected K/V;
+  decode workloads: ring pooling + decode indexer (scan + merge) + split-KV
+    sparse attention + combine.
+The default workload is the 32K-token prefill with planted needles (B=1,
+T=32768, top-512, 16 q / 2 kv heads, bf16).  One JSON line is printed by
+rank 0.  With N > 1 (torchrun) every rank runs its own replica of the
+workload (QSA has no exchange step: replicas only), the timed region is
+bracketed by barriers and the max over ranks is reported; value is the whole
+job's throughput.
+
+--impl reference times the CPU oracle (the only reference this method has) on
+a bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 1024 * 1024
+
+
+def peaks():
+    try:
+        with open(PEAKS_PATH) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except Exception:
+        return dict(FALLBACK), "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- workload plumbing
+
+class PrefillRunner:
+    """Device buffers and one step of the prefill hot path."""
+
+    def __init__(self, w, dev):
+        import block_sparse_attention_11_b200 as qsa
+        self.qsa = qsa
+        self.w = w
+        self.dev = dev
+        self.x = workloads.make_prefill(w, device=dev)
+        B, T = w.B, w.T
+        dt = workloads.torch_dtype(w)
+        self.rope = qsa.Rope(base=w.rope_base, pos_scale=w.pos_scale, rotary_dim=128)
+        self.k_pool = torch.zeros(B, max(T // 4, 1), 128, dtype=dt, device=dev)
+        self.sel = torch.empty(B, T, w.top_k, dtype=torch.int32, device=dev)
+        self.nsel = torch.empty(B, T, dtype=torch.int32, device=dev)
+        self.out = torch.empty_like(self.x["q"])
+        ws = qsa.qsa_index_topk_prefill_workspace(B, T, 0, w.top_k, 0, 0 if w.dtype == "bf16" else 1)
+        self.ws = torch.empty(ws, dtype=torch.uint8, device=dev)
+        # per-stage timing events (on the launching stream)
+        self.ev = None
+
+    def step(self, x=None, events=None):
+        qsa, w = self.qsa, self.w
+        x = x or self.x
+        if events is not None:
+            events[0].record()
+        qsa.qsa_pool_keys_prefill(x["k_idx"], self.k_pool, rope=self.rope)
+        if events is not None:
+            events[1].record()
+        qsa.qsa_index_topk_prefill(x["q_idx"], self.k_pool, self.sel, self.nsel, top_k=w.top_k, rope=self.rope,
+                                   workspace=self.ws)
+        if events is not None:
+            events[2].record()
+        qsa.qsa_sparse_attn_prefill(x["q"], x["k"], x["v"], self.sel, self.nsel, self.out)
+        if events is not None:
+            events[3].record()
+        return self.out
+
+    def launches_per_step(self):
+        return 5   # pool, query rotation, score GEMM, row select, attention
+
+    def units(self):
+        return self.w.B * self.w.T   # tokens
+
+    def stage_names(self):
+        return ["pool", "index_topk", "sparse_attn"]
+
+    # algorithmic work (see the design notes): per-query gathered K/V bytes and flops
+    def algorithmic(self):
+        w = self.w
+        T, K = w.T, w.top_k
+        t = torch.arange(T, dtype=torch.float64)
+        nb = torch.floor((t + 1) / 4)
+        npos = torch.minimum(nb, torch.tensor(float(K))) * 4 + (t + 1 - 4 * nb)
+        gather = float(npos.sum()) * w.Hkv * w.d * 2 * 2 * w.B        # K and V bytes gathered
+        qo = 2.0 * T * w.Hq * w.d * 2 * w.B                            # q read + out write
+        attn_flops = float(npos.sum()) * 4 * w.d * w.Hq * w.B
+        pairs = float(nb.sum()) * w.B
+        idx_flops = pairs * 2 * 128                                    # head-sum form of the linear score
+        return dict(attn_bytes=gather + qo, attn_flops=attn_flops, idx_flops=idx_flops, pairs=pairs)
+
+    def host_inputs(self):
+        return {k: v.cpu().pin_memory() for k, v in self.x.items() if isinstance(v, torch.Tensor)}
+
+
+class DecodeRunner:
+    def __init__(self, w, dev):
+        import block_sparse_attention_11_b200 as qsa
+        self.qsa = qsa
+        self.w = w
+        self.dev = dev
+        x = workloads.make_decode(w, device=dev)
+        self.x = x
+        dt = workloads.torch_dtype(w)
+        B, L = w.B, w.T
+        self.rope = qsa.Rope(base=w.rope_base, pos_scale=w.pos_scale, rotary_dim=128)
+        self.cap = L // 4 + 1
+        self.k_pool = torch.zeros(B, self.cap, 128, dtype=dt, device=dev)
+        qsa.qsa_pool_keys_prefill(x["k_idx"], self.k_pool, rope=self.rope)      # the cache's compressed keys
+        self.ring = torch.zeros(B, 4, 128, dtype=dt, device=dev)
+        del x["k_idx"]
+        torch.cuda.empty_cache()
+        self.sel = torch.empty(B, w.top_k, dtype=torch.int32, device=dev)
+        self.nsel = torch.empty(B, dtype=torch.int32, device=dev)
+        self.out = torch.empty_like(x["q"])
+        self.max_blocks = (L + 1) // 4
+        self.ws_i = torch.empty(qsa.qsa_index_topk_decode_workspace(B, self.max_blocks, w.top_k), dtype=torch.uint8,
+                                device=dev)
+        self.ws_a = torch.empty(qsa.qsa_sparse_attn_decode_workspace(B, w.Hq, w.d, w.top_k), dtype=torch.uint8,
+                                device=dev)
+
+    def step(self, x=None, events=None):
+        qsa, w = self.qsa, self.w
+        x = x or self.x
+        if events is not None:
+            events[0].record()
+        qsa.qsa_pool_keys_decode(x["k_idx_new"], self.ring, self.k_pool, x["seq_len"], rope=self.rope)
+        if events is not None:
+            events[1].record()
+        qsa.qsa_index_topk_decode(x["q_idx"], self.k_pool, x["seq_len"], self.sel, self.nsel,
+                                  max_blocks=self.max_blocks, top_k=w.top_k, rope=self.rope, workspace=self.ws_i)
+        if events is not None:
+            events[2].record()
+        qsa.qsa_sparse_attn_decode(x["q"], x["k"], x["v"], x["seq_len"], self.sel, self.nsel, self.out,
+                                   workspace=self.ws_a)
+        if events is not None:
+            events[3].record()
+        return self.out
+
+    def launches_per_step(self):
+        return 5   # ring pool, decode scorer, merge, attention, combine
+
+    def units(self):
+        return self.w.B
+
+    def stage_names(self):
+        return ["pool_ring", "index_topk", "sparse_attn"]
+
+    def algorithmic(self):
+        w = self.w
+        nb = (w.T + 1) // 4
+        tail = (w.T + 1) - 4 * nb
+        npos = min(nb, w.top_k) * 4 + tail
+        idx_bytes = nb * 128 * 2 + 4 * 128 * 2                        # compressed keys + indexer query
+        kv_bytes = npos * w.Hkv * w.d * 2 * 2 + 2 * w.Hq * w.d * 2     # gathered K/V + q + out
+        return dict(idx_bytes=idx_bytes * w.B, attn_bytes=kv_bytes * w.B, step_bytes=(idx_bytes + kv_bytes) * w.B)
+
+    def host_inputs(self):
+        keys = ["q_idx", "k_idx_new", "q", "seq_len"]
+        return {k: self.x[k].cpu().pin_memory() for k in keys}
+
+
+# ----------------------------------------------------------------------------- measurement
+
+def flush_l2(buf):
+    buf.add_(1.0)
+
+
+def run_ours(args, rank, world):
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    w = workloads.WORKLOADS[args.workload]
+    runner = (PrefillRunner if w.kind == "prefill" else DecodeRunner)(w, dev)
+    flush = torch.zeros(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    qsa = runner.qsa
+    for _ in range(args.warmup):
+        runner.step()
+    torch.cuda.synchronize()
+    qsa.qsa_check_status()
+
+    nst = 3
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)] for _ in range(args.steps)]
+    sampler = ClockSampler(dev.index if "CUDA_VISIBLE_DEVICES" not in os.environ else 0)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    for i in range(args.steps):
+        flush_l2(flush)                 # untimed: inputs start cold in L2
+        runner.step(events=events[i])
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if world > 1:
+        torch.distributed.barrier()
+    qsa.qsa_check_status()
+    step_ms = [events[i][0].elapsed_time(events[i][nst]) for i in range(args.steps)]
+    stage_ms = [[events[i][s].elapsed_time(events[i][s + 1]) for i in range(args.steps)] for s in range(nst)]
+    total_ms = sum(step_ms)
+    # max over ranks
+    t = torch.tensor([total_ms], device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+
+    # end to end through the public API: pinned host inputs -> device -> QSA -> host result
+    host = runner.host_inputs()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    out_host = torch.empty(runner.out.shape, dtype=runner.out.dtype, pin_memory=True)
+    d2h = out_host.numel() * out_host.element_size()
+    e2e_steps = max(3, min(args.steps, 10))
+    dev_x = dict(runner.x)
+    for it in range(e2e_steps + 2):
+        if it == 2:
+            torch.cuda.synchronize()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+        for k, v in host.items():
+            dev_x[k] = v.to(dev, non_blocking=True)
+        out = runner.step(x=dev_x)
+        out_host.copy_(out, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+
+    pk, pk_kind = peaks()
+    alg = runner.algorithmic()
+    res = dict(n_gpus=world, steps=args.steps, warmup=args.warmup, ms_per_step=ms_per_step, dtype=w.dtype,
+               data="synthetic", scaling="weak", vs_baseline=None, clocks=clocks,
+               gpu_launches=runner.launches_per_step() * args.steps)
+    stage_avg = {n: sum(v) / len(v) for n, v in zip(runner.stage_names(), stage_ms)}
+    res["stage_ms"] = {k: round(v, 4) for k, v in stage_avg.items()}
+    if w.kind == "prefill":
+        tokens = runner.units() * world
+        res.update(metric="QSA prefill tokens/s", unit="tokens/s", higher_is_better=True,
+                   value=tokens / (ms_per_step / 1e3))
+        res["e2e"] = dict(value=tokens / (e2e_ms / 1e3), unit="tokens/s", h2d_bytes_per_step=h2d,
+                          d2h_bytes_per_step=d2h)
+        attn_ms = stage_avg["sparse_attn"]
+        achieved = alg["attn_bytes"] / (attn_ms / 1e3) / 1e9
+        res["roofline"] = dict(kernel="sparse_attn_prefill", bound="hbm", achieved=achieved, peak=pk["hbm_gbs"],
+                               unit="GB/s", frac=achieved / pk["hbm_gbs"], traffic=None, peak_kind=pk_kind,
+                               note="algorithmic bytes = K/V rows gathered per query (4*nsel+tail positions x "
+                                    "Hkv x d x 2 B x 2) + q read + out write; the unique K/V fits in L2, so "
+                                    "gathers are served from L2 and frac can exceed 1")
+        flops = alg["attn_flops"] + alg["idx_flops"]
+        tf = flops / (ms_per_step / 1e3) / 1e12
+        res["tensor_roofline"] = dict(achieved=tf, peak=pk["bf16_tflops"], unit="TFLOP/s",
+                                      frac=tf / pk["bf16_tflops"], peak_kind=pk_kind,
+                                      note="indexer (2*128 flop per visible (query, block) pair) + attention "
+                                           "(4*d*Hq flop per selected position) over the whole step")
+        res["config"] = dict(workload=w.name, B=w.B, T=w.T, top_k=w.top_k, Hq=w.Hq, Hkv=w.Hkv, d=w.d,
+                             needles=w.needles, l2="flushed between timed steps (256 MB write)",
+                             parallelism=f"replicas x{world}")
+    else:
+        res.update(metric="QSA decode us/step", unit="us/step", higher_is_better=False,
+                   value=ms_per_step * 1e3)
+        res["e2e"] = dict(value=e2e_ms * 1e3, unit="us/step", h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h)
+        achieved = alg["step_bytes"] / (ms_per_step / 1e3) / 1e9
+        res["roofline"] = dict(kernel="decode step (scorer dominant)", bound="hbm", achieved=achieved,
+                               peak=pk["hbm_gbs"], unit="GB/s", frac=achieved / pk["hbm_gbs"], traffic=None,
+                               peak_kind=pk_kind)
+        res["config"] = dict(workload=w.name, B=w.B, L=w.T, top_k=w.top_k, Hq=w.Hq, Hkv=w.Hkv, d=w.d,
+                             pos_scale=w.pos_scale, l2="flushed between timed steps (256 MB write)",
+                             parallelism=f"replicas x{world}")
+    return res
+
+
+# ----------------------------------------------------------------------------- CPU oracle arm
+
+def run_oracle_sample(w, budget_s=15.0, seed=0):
+    """Time the CPU oracle on a bounded sample of the workload; returns
+    (value in the workload's unit, sample description, threads)."""
+    import numpy as np
+
+    import oracle
+    nthreads = os.cpu_count() or 1
+    if w.kind == "prefill":
+        x = workloads.make_prefill(w, device="cpu")
+        q_idx = x["q_idx"][0].float().numpy()
+        k_raw = x["k_idx"][0].float().numpy()
+        q, k, v = (x[n][0].float().numpy() for n in ("q", "k", "v"))
+        t0 = time.perf_counter()
+        kp = oracle.pool_keys(k_raw, base=w.rope_base, pos_scale=w.pos_scale, store_bf16=w.dtype == "bf16")
+        t_pool = time.perf_counter() - t0
+        rng = np.random.default_rng(seed)
+        done, elapsed, n = 0, 0.0, 64
+        while elapsed < budget_s and done < w.T:
+            rows = rng.integers(0, w.T, n)
+            t0 = time.perf_counter()
+            oracle.prefill_rows(rows, q_idx=q_idx, k_pool=kp, top_k=w.top_k, base=w.rope_base,
+                                pos_scale=w.pos_scale, store_bf16=w.dtype == "bf16", q=q, k=k, v=v, Hq=w.Hq,
+                                Hkv=w.Hkv, d=w.d, nthreads=nthreads)
+            dt = time.perf_counter() - t0
+            elapsed += dt
+            done += n
+            n = min(4096, n * 2)
+        per_row = elapsed / done
+        total = t_pool + per_row * w.T * w.B
+        value = w.T * w.B / total
+        sample = (f"{done} uniformly drawn query rows of the {w.T}-token workload (full indexer scan, top-k, "
+                  f"attention per row) + pooling of all keys; extrapolated per row to all rows")
+        return value, sample, nthreads, "tokens/s"
+    # decode: a subset of sequences at full length
+    x = workloads.make_decode(w, device="cpu", B=1)
+    kr = x["k_idx"][0].float().numpy()
+    kp = oracle.pool_keys(kr, base=w.rope_base, pos_scale=w.pos_scale, store_bf16=True)
+    q, k, v = x["q"].float().numpy(), x["k"].float().numpy(), x["v"].float().numpy()
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        oracle.decode(x["q_idx"].float().numpy(), kp[None], x["seq_len"].numpy(), q=q, k=k, v=v, top_k=w.top_k,
+                      base=w.rope_base, pos_scale=w.pos_scale, Hq=w.Hq, Hkv=w.Hkv, d=w.d, nthreads=nthreads)
+        reps += 1
+        if time.perf_counter() - t0 > min(budget_s, 5.0):
+            break
+    per_seq = (time.perf_counter() - t0) / reps
+    value = per_seq * w.B * 1e6          # a decode step of all B sequences, us
+    sample = f"{reps} decode steps of one {w.T}-token sequence, scaled to B={w.B}"
+    return value, sample, nthreads, "us/step"
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="prefill_t32k_needles", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    w = workloads.WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        if rank == 0:
+            value, sample, threads, unit = run_oracle_sample(w, budget_s=args.cpu_budget)
+            line = dict(impl="reference", metric="QSA prefill tokens/s" if w.kind == "prefill" else
+                        "QSA decode us/step", value=value, unit=unit, higher_is_better=w.kind == "prefill",
+                        n_gpus=args.gpus, steps=args.steps, warmup=args.warmup, dtype=w.dtype, data="synthetic",
+                        config=dict(workload=w.name), vs_baseline=None,
+                        cpu_baseline=dict(value=value, unit=unit, cores=threads, kind="oracle", sample=sample),
+                        e2e=dict(value=value, unit=unit, h2d_bytes_per_step=0, d2h_bytes_per_step=0))
+            print(json.dumps(line), flush=True)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+
+    res = run_ours(args, rank, world)
+    if rank == 0 and not args.no_cpu_baseline:
+        value, sample, threads, unit = run_oracle_sample(w, budget_s=args.cpu_budget)
+        res["cpu_baseline"] = dict(value=value, unit=unit, cores=threads, kind="oracle", sample=sample)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        order = ["metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                 "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "tensor_roofline", "e2e",
+                 "cpu_baseline", "gpu_launches", "clocks", "stage_ms"]
+        line = {k: res[k] for k in order if k in res}
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,89 @@
+// internal.h -- host-side launchers shared between the kernel files and the
+// C-ABI layer (qsa_api.cu).  Nothing here is exported from libqsa.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace qsa {
+
+struct DeviceInfo {
+    int sm_count = 0;
+    int major = 0, minor = 0;
+    size_t smem_optin = 0;
+    unsigned *status = nullptr;   // device address of the library status word
+};
+
+// Per-device info of the current device (cached).  Returns nullptr on error.
+const DeviceInfo *device_info();
+
+// ---- pooling / rotation (k_rope.cu)
+cudaError_t launch_pool_prefill(const void *k_raw, void *k_pool, int B, int64_t nblk, int64_t pos0,
+                                int64_t raw_stride, int64_t pool_stride, Rope rope, bool rmsnorm, bool bf16,
+                                cudaStream_t s);
+cudaError_t launch_pool_decode(const void *k_new, void *ring, void *k_pool, const int32_t *seq_len, int B,
+                               int64_t pool_stride, Rope rope, bool rmsnorm, bool bf16, unsigned *status,
+                               cudaStream_t s);
+cudaError_t launch_rope_apply(void *x, int B, int64_t n, int H, int d, int64_t pos0, Rope rope, bool bf16,
+                              cudaStream_t s);
+// Indexer queries for prefill: mode 0 -> hi/lo bf16 planes of the head sum
+// ([rows][128] each); mode 1 -> per-head bf16 [rows][4][128]; mode 2 -> per-head fp32.
+cudaError_t launch_rotate_index_q(const void *q_idx, int B, int64_t n_q, int64_t q0, Rope rope, int mode,
+                                  void *out0, void *out1, cudaStream_t s);
+
+// ---- indexer scores (k_index.cu)
+struct ScoreGemmArgs {
+    int B;
+    int64_t n_q;          // query rows per sequence in this call
+    int64_t q0;           // position of query row 0
+    int64_t row_begin;    // first query row of this chunk (within each sequence)
+    int64_t row_count;    // rows of this chunk
+    int64_t pool_stride;
+    int64_t ld;           // score row stride (floats)
+    int per_head;         // 0: hi/lo head-sum operands, 1: per-head operands
+    int relu;
+    const float *head_w;  // [B][n_q][4] or null
+    float *scores;        // [B][row_count][ld]
+};
+cudaError_t launch_score_gemm(const ScoreGemmArgs &a, const void *qa0, const void *qa1, const void *k_pool,
+                              unsigned *status, cudaStream_t s);
+cudaError_t launch_score_simt_f32(const ScoreGemmArgs &a, const float *q_hat, const float *k_pool,
+                                  cudaStream_t s);
+cudaError_t launch_select_rows(const float *scores, int B, int64_t row_begin, int64_t row_count, int64_t n_q,
+                               int64_t q0, int64_t ld, int top_k, int32_t *sel, int32_t *nsel,
+                               unsigned *status, cudaStream_t s);
+
+// ---- decode indexer (k_decode_index.cu)
+struct DecodePlan {
+    int chunks;          // chunks per sequence
+    int64_t chunk;       // blocks per chunk
+};
+DecodePlan decode_index_plan(int B, int64_t max_blocks, bool bf16);
+size_t decode_index_ws_bytes(int B, int64_t max_blocks, int top_k, bool bf16);
+cudaError_t launch_decode_index(const void *q_idx, const void *k_pool, const float *head_w,
+                                const int32_t *seq_len, int B, int64_t pool_stride, int64_t max_blocks,
+                                int top_k, int32_t *sel, int32_t *nsel, void *ws, Rope rope, bool relu,
+                                bool bf16, unsigned *status, cudaStream_t s);
+
+// ---- sparse attention (k_attn.cu)
+struct AttnArgs {
+    const void *q, *k, *v;
+    const int32_t *sel, *nsel;
+    const int32_t *seq_len;   // decode: [B]; prefill: null
+    int B;
+    int64_t n_q, q0, kv_stride;
+    int Hq, Hkv, d, top_k;
+    float scale;
+    void *out;
+    float *lse;
+    bool decode;
+};
+size_t attn_decode_ws_bytes(int B, int Hq, int d, int top_k);
+cudaError_t launch_attn_bf16(const AttnArgs &a, void *ws, unsigned *status, cudaStream_t s);
+cudaError_t launch_attn_f32(const AttnArgs &a, unsigned *status, cudaStream_t s);
+
+}  // namespace qsa

@@ -1,0 +1,558 @@
+// k_attn.cu -- sparse attention over the selected original K/V.
+//
+// Page "Qwen3.8-Flash-Next: Day-0 Support in SGLang", section "Qwen Sparse
+// Attention: Retrieve Coarsely, Attend Precisely": the selected blocks expand
+// to 2048 positions, the 0-3 tokens of the query's own incomplete block are
+// appended (at most 2051 positions), and softmax and value aggregation use the
+// original uncompressed K/V.  One selection per query serves every head.
+//
+// bf16 kernel.  Each query gathers its own ~2 MB of K/V, so the stage is bound
+// by gather bandwidth (about 8 flop per byte), not by the tensor cores.  The
+// design keeps the gather engine busy and the math off the critical path:
+//   * a producer warp walks the selection and issues one bulk TMA copy per
+//     selected block and tensor (a block of all kv heads is one contiguous
+//     4 x Hkv x 256-byte span), 8 blocks per stage, 4 stages in flight;
+//   * each block lands in its own shared-memory slot, slots padded by 16 bytes
+//     so that token j of 8 different blocks fall in 8 different bank groups:
+//     every 8x8 ldmatrix tile reads 8 blocks' token j conflict-free;
+//   * consumers use swap-AB warp MMAs (m16n8k16): S^T = K Q^T with 16 keys as
+//     M and the 8 q heads of one kv head as N (no padding waste for GQA 8),
+//     an fp32 online softmax per head column, P^T re-laid out in registers
+//     with movmatrix, and O^T += V^T P;
+//   * two warps per kv head split each stage's 32 keys (tokens {0,1} and
+//     {2,3} of the 8 blocks) and merge their softmax states at the end.
+// A persistent grid walks the work items; the pipeline runs across item
+// boundaries.  Decode splits each sequence's key list over several items
+// (split-KV) and a small kernel combines the partial results.
+//
+// fp32 kernel.  A plain SIMT warp per (query, head): used for the fp32 mode.
+#include <algorithm>
+
+#include "internal.h"
+
+namespace qsa {
+
+namespace {
+
+constexpr int AT_BPS = 8;               // blocks per stage
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int HKV> struct AttnCfg {
+    static constexpr int kConsumers = 2 * HKV;
+    static constexpr int kThreads = (kConsumers + 1) * 32;
+    static constexpr int kSpan = kBlock * HKV * 128 * 2;      // bytes of one block, all kv heads
+    static constexpr int kSlot = kSpan + 16;                   // padded slot
+    static constexpr int kStage = 2 * AT_BPS * kSlot;          // K slots then V slots
+    static constexpr int kHq = 8 * HKV;
+    static constexpr int kQBytes = kHq * 128 * 2;
+    static constexpr int kNS = HKV >= 4 ? 2 : 4;               // stages in flight (smem bound)
+};
+
+struct AttnParams {
+    const __nv_bfloat16 *q, *k, *v;
+    const int32_t *sel, *nsel, *seq_len;
+    int B;
+    int64_t n_q, q0, kv_stride;
+    int top_k;
+    float scale_log2;
+    int decode;
+    int splits;            // decode: items per sequence
+    int split_blocks;      // decode: list entries per split (multiple of AT_BPS)
+    int64_t items;
+    __nv_bfloat16 *out;
+    float *lse;
+    float *part_o;         // decode: [B][splits][Hq][128]
+    float *part_lse;       // decode: [B][splits][Hq] (log2 domain)
+    unsigned *status;
+};
+
+// The key list of one work item: positions lbeg..lend of
+// [sel[0..nsel), tail block (if tail > 0)].
+struct Item {
+    int seq;
+    int64_t row;       // prefill: query row; decode: split index
+    int64_t t;         // query position
+    const int32_t *sel;
+    int nsel;
+    int64_t nb;
+    int tail;
+    int lbeg, lend;
+    const __nv_bfloat16 *qrow;
+};
+
+template <int HKV>
+__device__ __forceinline__ Item get_item(const AttnParams &p, int64_t i) {
+    Item it;
+    if (!p.decode) {
+        it.seq = (int)(i % p.B);
+        it.row = p.n_q - 1 - i / p.B;                       // longest rows first
+        it.t = p.q0 + it.row;
+        const int64_t qi = (int64_t)it.seq * p.n_q + it.row;
+        it.sel = p.sel + qi * p.top_k;
+        it.nsel = p.nsel[qi];
+        it.qrow = p.q + qi * (int64_t)AttnCfg<HKV>::kHq * 128;
+    } else {
+        it.seq = (int)(i / p.splits);
+        it.row = i % p.splits;
+        it.t = (int64_t)p.seq_len[it.seq] - 1;
+        it.sel = p.sel + (int64_t)it.seq * p.top_k;
+        it.nsel = p.nsel[it.seq];
+        it.qrow = p.q + (int64_t)it.seq * AttnCfg<HKV>::kHq * 128;
+    }
+    if (it.t < 0 || it.t >= p.kv_stride) {
+        if (it.t >= p.kv_stride) flag(p.status, QSA_DEV_BAD_LENGTH);
+        it.t = -1;   // nothing visible: the item attends to no position
+    }
+    it.nb = (it.t + 1) / kBlock;
+    it.tail = (int)(it.t + 1 - kBlock * it.nb);
+    it.nsel = max(0, min(it.nsel, p.top_k));
+    const int len = it.nsel + (it.tail > 0 ? 1 : 0);
+    if (!p.decode) {
+        it.lbeg = 0;
+        it.lend = len;
+    } else {
+        it.lbeg = min(len, (int)it.row * p.split_blocks);
+        it.lend = min(len, it.lbeg + p.split_blocks);
+    }
+    return it;
+}
+
+template <int HKV>
+struct __align__(128) AttnSmem {
+    using Cfg = AttnCfg<HKV>;
+    uint8_t stage[Cfg::kNS][AttnCfg<HKV>::kStage];
+    alignas(16) uint8_t qbuf[2][AttnCfg<HKV>::kQBytes];
+    float xbuf[HKV][32][36];
+    alignas(16) __nv_bfloat16 obuf[HKV][8][128];
+    uint32_t info[Cfg::kNS];
+    uint64_t full[Cfg::kNS], empty[Cfg::kNS], qfull[2], qempty[2];
+    uint64_t xready[HKV], xdone[HKV];   // pair merge handshake per kv head
+};
+
+template <int HKV>
+__global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, 1) attn_bf16_kernel(AttnParams p) {
+    using Cfg = AttnCfg<HKV>;
+    extern __shared__ uint8_t asm_raw[];
+    AttnSmem<HKV> &sm = *reinterpret_cast<AttnSmem<HKV> *>((reinterpret_cast<uintptr_t>(asm_raw) + 127) & ~uintptr_t(127));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    // zero the slots once: masked keys must read finite values (0 * NaN = NaN)
+    for (int i = threadIdx.x; i < (int)(sizeof(sm.stage) / 16); i += blockDim.x)
+        reinterpret_cast<uint4 *>(&sm.stage[0][0])[i] = make_uint4(0, 0, 0, 0);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < Cfg::kNS; ++s) { mbar_init(&sm.full[s], 1); mbar_init(&sm.empty[s], Cfg::kConsumers); }
+        for (int s = 0; s < 2; ++s) { mbar_init(&sm.qfull[s], 1); mbar_init(&sm.qempty[s], Cfg::kConsumers); }
+        for (int s = 0; s < HKV; ++s) { mbar_init(&sm.xready[s], 1); mbar_init(&sm.xdone[s], 1); }
+        fence_mbar_init();
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+
+    if (warp == Cfg::kConsumers) {
+        // ------------------------------------------------------------ producer
+        int64_t it_count = 0;   // stage counter across items
+        int64_t ic = 0;         // item counter
+        bool ok = true;
+        for (int64_t i = blockIdx.x; i < p.items && ok; i += gridDim.x, ++ic) {
+            const Item it = get_item<HKV>(p, i);
+            const int qs = (int)(ic & 1);
+            if (ic >= 2) ok = mbar_wait(&sm.qempty[qs], (int)(((ic >> 1) + 1) & 1), p.status);
+            if (!ok) break;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&sm.qfull[qs], Cfg::kQBytes);
+                bulk_g2s(sm.qbuf[qs], it.qrow, Cfg::kQBytes, &sm.qfull[qs]);
+            }
+            const int64_t kv0 = (int64_t)it.seq * p.kv_stride;
+            for (int pos = it.lbeg; pos < it.lend && ok; pos += AT_BPS, ++it_count) {
+                const int s = (int)(it_count % Cfg::kNS);
+                if (it_count >= Cfg::kNS) ok = mbar_wait(&sm.empty[s], (int)(((it_count / Cfg::kNS) + 1) & 1), p.status);
+                if (!ok) break;
+                // lane j < 8 handles list entry pos + j
+                int tokens = 0;
+                int64_t blk = 0;
+                const int e = pos + lane;
+                if (lane < AT_BPS && e < it.lend) {
+                    if (e < it.nsel) {
+                        blk = it.sel[e];
+                        if (blk >= 0 && blk < it.nb) tokens = kBlock;
+                        else flag(p.status, QSA_DEV_BAD_INDEX);
+                    } else {
+                        blk = it.nb;            // the incomplete tail block
+                        tokens = it.tail;
+                    }
+                }
+                uint32_t bytes = (uint32_t)tokens * HKV * 256u;
+                uint32_t info = (uint32_t)tokens << (3 * (lane & 7));
+                if (lane >= AT_BPS) info = 0;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    bytes += __shfl_xor_sync(0xffffffffu, bytes, o);
+                    info |= __shfl_xor_sync(0xffffffffu, info, o);
+                }
+                if (lane == 0) {
+                    sm.info[s] = info;
+                    mbar_arrive_expect_tx(&sm.full[s], 2 * bytes);
+                }
+                __syncwarp();
+                if (tokens > 0) {
+                    const int64_t off = (kv0 + blk * kBlock) * HKV * 128;
+                    const uint32_t nbytes = (uint32_t)tokens * HKV * 256u;
+                    bulk_g2s(sm.stage[s] + lane * Cfg::kSlot, p.k + off, nbytes, &sm.full[s]);
+                    bulk_g2s(sm.stage[s] + (AT_BPS + lane) * Cfg::kSlot, p.v + off, nbytes, &sm.full[s]);
+                }
+            }
+        }
+        // drain: wait until the copies of the last stages have landed
+        if (lane == 0) {
+            for (int64_t c = (it_count > Cfg::kNS ? it_count - Cfg::kNS : 0); c < it_count; ++c)
+                mbar_wait(&sm.full[c % Cfg::kNS], (int)((c / Cfg::kNS) & 1), p.status);
+            for (int64_t c = (ic > 2 ? ic - 2 : 0); c < ic; ++c) mbar_wait(&sm.qfull[c & 1], (int)((c >> 1) & 1), p.status);
+        }
+        return;
+    }
+
+    // ---------------------------------------------------------------- consumers
+    const int g = warp >> 1;        // kv head
+    const int hf = warp & 1;        // token pair {2hf, 2hf+1}
+    const int gr = lane >> 2, tq = lane & 3;
+    const uint32_t stage0 = smem_u32(&sm.stage[0][0]);
+    // ldmatrix row addresses (byte offsets inside a stage)
+    const int mi = lane >> 3, rr = lane & 7;
+    const uint32_t k_lane_off = (uint32_t)(rr * Cfg::kSlot + (2 * hf + (mi & 1)) * HKV * 256 + g * 256 + (mi >> 1) * 16);
+    const uint32_t v_lane_off = (uint32_t)(AT_BPS * Cfg::kSlot + rr * Cfg::kSlot + (2 * hf + (mi >> 1)) * HKV * 256 +
+                                           g * 256 + (mi & 1) * 16);
+    int64_t it_count = 0, ic = 0;
+    bool ok = true;
+    for (int64_t i = blockIdx.x; i < p.items && ok; i += gridDim.x, ++ic) {
+        const Item it = get_item<HKV>(p, i);
+        const int qs = (int)(ic & 1);
+        ok = mbar_wait(&sm.qfull[qs], (int)((ic >> 1) & 1), p.status);
+        if (!ok) break;
+        uint32_t qf[8][2];
+        {
+            const uint32_t *qw = reinterpret_cast<const uint32_t *>(sm.qbuf[qs]);
+            const int head = 8 * g + gr;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                qf[kk][0] = qw[(head * 128 + 16 * kk + 2 * tq) >> 1];
+                qf[kk][1] = qw[(head * 128 + 16 * kk + 8 + 2 * tq) >> 1];
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.qempty[qs]);
+        float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
+        float o[8][4];
+#pragma unroll
+        for (int a = 0; a < 8; ++a) o[a][0] = o[a][1] = o[a][2] = o[a][3] = 0.f;
+
+        for (int pos = it.lbeg; pos < it.lend; pos += AT_BPS, ++it_count) {
+            const int s = (int)(it_count % Cfg::kNS);
+            ok = mbar_wait(&sm.full[s], (int)((it_count / Cfg::kNS) & 1), p.status);
+            if (!ok) break;
+            const uint32_t info = sm.info[s];
+            const uint32_t sbase = stage0 + (uint32_t)s * Cfg::kStage;
+            // S^T (16 keys x 8 heads)
+            float sacc[4] = {0.f, 0.f, 0.f, 0.f}, sacc2[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int kk = 0; kk < 8; kk += 2) {
+                uint32_t a0, a1, a2, a3, c0, c1, c2, c3;
+                ldsm_x4(sbase + k_lane_off + kk * 32, a0, a1, a2, a3);
+                ldsm_x4(sbase + k_lane_off + (kk + 1) * 32, c0, c1, c2, c3);
+                mma16816(sacc, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
+                mma16816(sacc2, c0, c1, c2, c3, qf[kk + 1][0], qf[kk + 1][1]);
+            }
+#pragma unroll
+            for (int c = 0; c < 4; ++c) sacc[c] += sacc2[c];
+            const int ntok = (int)((info >> (3 * gr)) & 7u);
+            const bool v0 = ntok > 2 * hf, v1 = ntok > 2 * hf + 1;
+            float x0 = v0 ? sacc[0] * p.scale_log2 : -INFINITY;   // key (slot gr, tok 2hf),   head 2tq
+            float x1 = v0 ? sacc[1] * p.scale_log2 : -INFINITY;   //                           head 2tq+1
+            float x2 = v1 ? sacc[2] * p.scale_log2 : -INFINITY;   // key (slot gr, tok 2hf+1), head 2tq
+            float x3 = v1 ? sacc[3] * p.scale_log2 : -INFINITY;
+            float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+            for (int o2 = 4; o2 < 32; o2 <<= 1) {
+                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o2));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o2));
+            }
+            const float mn0 = fmaxf(mrow[0], mx0), mn1 = fmaxf(mrow[1], mx1);
+            const float mu0 = (mn0 == -INFINITY) ? 0.f : mn0, mu1 = (mn1 == -INFINITY) ? 0.f : mn1;
+            const float al0 = exp2f(mrow[0] - mu0), al1 = exp2f(mrow[1] - mu1);
+            mrow[0] = mn0;
+            mrow[1] = mn1;
+            const float p0 = exp2f(x0 - mu0), p1 = exp2f(x1 - mu1), p2 = exp2f(x2 - mu0), p3 = exp2f(x3 - mu1);
+            lrow[0] = lrow[0] * al0 + p0 + p2;
+            lrow[1] = lrow[1] * al1 + p1 + p3;
+            const uint32_t b0 = movm_t(pack_bf16(p0, p1));
+            const uint32_t b1 = movm_t(pack_bf16(p2, p3));
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+                o[mt][0] *= al0;
+                o[mt][1] *= al1;
+                o[mt][2] *= al0;
+                o[mt][3] *= al1;
+                uint32_t a0, a1, a2, a3;
+                ldsm_x4_t(sbase + v_lane_off + mt * 32, a0, a1, a2, a3);
+                mma16816(o[mt], a0, a1, a2, a3, b0, b1);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.empty[s]);
+        }
+        if (!ok) break;
+        // row sums across the 8 lane groups
+#pragma unroll
+        for (int o2 = 4; o2 < 32; o2 <<= 1) {
+            lrow[0] += __shfl_xor_sync(0xffffffffu, lrow[0], o2);
+            lrow[1] += __shfl_xor_sync(0xffffffffu, lrow[1], o2);
+        }
+        // merge the two warps of this kv head
+        float *xb = sm.xbuf[g][lane];
+        if (hf == 1) {
+            if (ic > 0) ok = mbar_wait(&sm.xdone[g], (int)((ic - 1) & 1), p.status);
+            if (!ok) break;
+            xb[0] = mrow[0]; xb[1] = mrow[1]; xb[2] = lrow[0]; xb[3] = lrow[1];
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) xb[4 + 4 * mt + c] = o[mt][c];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.xready[g]);
+        } else {
+            ok = mbar_wait(&sm.xready[g], (int)(ic & 1), p.status);
+            if (!ok) break;
+            float f0[2], f1[2], l[2], m[2];
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                const float mo = xb[c], lo = xb[2 + c];
+                m[c] = fmaxf(mrow[c], mo);
+                const float mu = (m[c] == -INFINITY) ? 0.f : m[c];
+                f0[c] = exp2f(mrow[c] - mu);
+                f1[c] = exp2f(mo - mu);
+                l[c] = lrow[c] * f0[c] + lo * f1[c];
+            }
+            const float inv0 = l[0] > 0.f ? 1.f / l[0] : 0.f, inv1 = l[1] > 0.f ? 1.f / l[1] : 0.f;
+            if (!p.decode) {
+#pragma unroll
+                for (int mt = 0; mt < 8; ++mt) {
+                    const float r0 = (o[mt][0] * f0[0] + xb[4 + 4 * mt + 0] * f1[0]) * inv0;
+                    const float r1 = (o[mt][1] * f0[1] + xb[4 + 4 * mt + 1] * f1[1]) * inv1;
+                    const float r2 = (o[mt][2] * f0[0] + xb[4 + 4 * mt + 2] * f1[0]) * inv0;
+                    const float r3 = (o[mt][3] * f0[1] + xb[4 + 4 * mt + 3] * f1[1]) * inv1;
+                    sm.obuf[g][2 * tq][16 * mt + gr] = __float2bfloat16_rn(r0);
+                    sm.obuf[g][2 * tq + 1][16 * mt + gr] = __float2bfloat16_rn(r1);
+                    sm.obuf[g][2 * tq][16 * mt + gr + 8] = __float2bfloat16_rn(r2);
+                    sm.obuf[g][2 * tq + 1][16 * mt + gr + 8] = __float2bfloat16_rn(r3);
+                }
+                __syncwarp();
+                const int64_t qi = (int64_t)it.seq * p.n_q + it.row;
+                uint4 *dst = reinterpret_cast<uint4 *>(p.out + (qi * Cfg::kHq + 8 * g) * 128);
+                const uint4 *src = reinterpret_cast<const uint4 *>(&sm.obuf[g][0][0]);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) dst[lane + 32 * c] = src[lane + 32 * c];
+                if (p.lse && gr == 0) {
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        const float v = (l[c] > 0.f) ? (m[c] + log2f(l[c])) / kLog2e : -INFINITY;
+                        p.lse[qi * Cfg::kHq + 8 * g + 2 * tq + c] = v;
+                    }
+                }
+                __syncwarp();
+            } else {
+                const int64_t pi = (int64_t)it.seq * p.splits + it.row;
+                float *po = p.part_o + (pi * Cfg::kHq + 8 * g) * 128;
+#pragma unroll
+                for (int mt = 0; mt < 8; ++mt) {
+                    po[(2 * tq) * 128 + 16 * mt + gr] = (o[mt][0] * f0[0] + xb[4 + 4 * mt + 0] * f1[0]) * inv0;
+                    po[(2 * tq + 1) * 128 + 16 * mt + gr] = (o[mt][1] * f0[1] + xb[4 + 4 * mt + 1] * f1[1]) * inv1;
+                    po[(2 * tq) * 128 + 16 * mt + gr + 8] = (o[mt][2] * f0[0] + xb[4 + 4 * mt + 2] * f1[0]) * inv0;
+                    po[(2 * tq + 1) * 128 + 16 * mt + gr + 8] = (o[mt][3] * f0[1] + xb[4 + 4 * mt + 3] * f1[1]) * inv1;
+                }
+                if (gr == 0) {
+#pragma unroll
+                    for (int c = 0; c < 2; ++c)
+                        p.part_lse[pi * Cfg::kHq + 8 * g + 2 * tq + c] = (l[c] > 0.f) ? m[c] + log2f(l[c]) : -INFINITY;
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.xdone[g]);
+        }
+    }
+}
+
+// Decode combine: one CTA of 128 threads per (sequence, q head).
+__global__ void attn_combine_kernel(const float *__restrict__ part_o, const float *__restrict__ part_lse, int splits,
+                                    int Hq, __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
+    const int seq = blockIdx.x / Hq, h = blockIdx.x % Hq, e = threadIdx.x;
+    float mx = -INFINITY;
+    for (int s = 0; s < splits; ++s) mx = fmaxf(mx, part_lse[((int64_t)seq * splits + s) * Hq + h]);
+    float acc = 0.f, den = 0.f;
+    if (mx != -INFINITY) {
+        for (int s = 0; s < splits; ++s) {
+            const float ls = part_lse[((int64_t)seq * splits + s) * Hq + h];
+            if (ls == -INFINITY) continue;
+            const float w = exp2f(ls - mx);
+            den += w;
+            acc += w * part_o[(((int64_t)seq * splits + s) * Hq + h) * 128 + e];
+        }
+    }
+    out[((int64_t)seq * Hq + h) * 128 + e] = __float2bfloat16_rn(den > 0.f ? acc / den : 0.f);
+    if (lse && e == 0) lse[(int64_t)seq * Hq + h] = den > 0.f ? (mx + log2f(den)) / kLog2e : -INFINITY;
+}
+
+// fp32 SIMT attention: one warp per (item, q head); lane owns 4 dims.
+__global__ void __launch_bounds__(256) attn_f32_kernel(const float *__restrict__ q, const float *__restrict__ k,
+                                                        const float *__restrict__ v, const int32_t *__restrict__ sel,
+                                                        const int32_t *__restrict__ nsel_p,
+                                                        const int32_t *__restrict__ seq_len, int B, int64_t n_q,
+                                                        int64_t q0, int64_t kv_stride, int Hq, int Hkv, int top_k,
+                                                        float scale, float *__restrict__ out, float *__restrict__ lse,
+                                                        int decode, unsigned *status) {
+    const int64_t wid = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    const int64_t items = decode ? (int64_t)B : (int64_t)B * n_q;
+    if (wid >= items * Hq) return;
+    const int h = (int)(wid % Hq);
+    const int64_t item = wid / Hq;
+    int seq;
+    int64_t t, qi;
+    if (decode) { seq = (int)item; t = (int64_t)seq_len[seq] - 1; qi = seq; }
+    else { seq = (int)(item / n_q); t = q0 + item % n_q; qi = item; }
+    const int g = (int)(((int64_t)h * Hkv) / Hq);
+    if (t >= kv_stride) {
+        if (lane == 0) flag(status, QSA_DEV_BAD_LENGTH);
+        t = -1;   // nothing visible
+    }
+    const int64_t nb = (t + 1) / kBlock;
+    const int tail = (int)(t + 1 - kBlock * nb);
+    const int32_t *sl = sel + qi * top_k;
+    const int nsel = max(0, min(nsel_p[qi], top_k));
+    const float4 qv = reinterpret_cast<const float4 *>(q + (qi * Hq + h) * 128)[lane];
+    float m = -INFINITY, l = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    const int len = nsel + (tail > 0 ? 1 : 0);
+    for (int e = 0; e < len; ++e) {
+        int64_t b;
+        int ntok;
+        if (e < nsel) {
+            b = sl[e];
+            ntok = kBlock;
+            if (b < 0 || b >= nb) {
+                if (lane == 0) flag(status, QSA_DEV_BAD_INDEX);
+                continue;
+            }
+        } else {
+            b = nb;
+            ntok = tail;
+        }
+        for (int j = 0; j < ntok; ++j) {
+            const int64_t row = ((int64_t)seq * kv_stride + b * kBlock + j) * Hkv + g;
+            const float4 kv = reinterpret_cast<const float4 *>(k + row * 128)[lane];
+            float d = qv.x * kv.x + qv.y * kv.y + qv.z * kv.z + qv.w * kv.w;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+            const float x = d * scale;
+            const float mn = fmaxf(m, x);
+            const float al = expf(m - mn);
+            const float pw = expf(x - mn);
+            m = mn;
+            l = l * al + pw;
+            const float4 vv = reinterpret_cast<const float4 *>(v + row * 128)[lane];
+            acc.x = acc.x * al + pw * vv.x;
+            acc.y = acc.y * al + pw * vv.y;
+            acc.z = acc.z * al + pw * vv.z;
+            acc.w = acc.w * al + pw * vv.w;
+        }
+    }
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    reinterpret_cast<float4 *>(out + (qi * Hq + h) * 128)[lane] =
+        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    if (lse && lane == 0) lse[qi * Hq + h] = l > 0.f ? m + logf(l) : -INFINITY;
+}
+
+template <int HKV>
+cudaError_t run_bf16(const AttnArgs &a, void *ws, unsigned *status, cudaStream_t s) {
+    using Cfg = AttnCfg<HKV>;
+    const DeviceInfo *di = device_info();
+    const int sms = di ? di->sm_count : 148;
+    AttnParams p{};
+    p.q = (const __nv_bfloat16 *)a.q;
+    p.k = (const __nv_bfloat16 *)a.k;
+    p.v = (const __nv_bfloat16 *)a.v;
+    p.sel = a.sel;
+    p.nsel = a.nsel;
+    p.seq_len = a.seq_len;
+    p.B = a.B;
+    p.n_q = a.n_q;
+    p.q0 = a.q0;
+    p.kv_stride = a.kv_stride;
+    p.top_k = a.top_k;
+    p.scale_log2 = a.scale * kLog2e;
+    p.decode = a.decode ? 1 : 0;
+    p.out = (__nv_bfloat16 *)a.out;
+    p.lse = a.lse;
+    p.status = status;
+    if (a.decode) {
+        const int list_max = a.top_k + 1;
+        int splits = max(1, (2 * sms + a.B - 1) / a.B);
+        int sb = (list_max + splits - 1) / splits;
+        sb = max(AT_BPS, (sb + AT_BPS - 1) / AT_BPS * AT_BPS);
+        splits = (list_max + sb - 1) / sb;
+        p.splits = splits;
+        p.split_blocks = sb;
+        p.items = (int64_t)a.B * splits;
+        float *w = static_cast<float *>(ws);
+        p.part_o = w;
+        p.part_lse = w + (size_t)a.B * splits * Cfg::kHq * 128;
+    } else {
+        p.splits = 1;
+        p.split_blocks = 0;
+        p.items = (int64_t)a.B * a.n_q;
+    }
+    if (p.items <= 0) return cudaSuccess;
+    const size_t smem = sizeof(AttnSmem<HKV>) + 128;
+    cudaError_t e = cudaFuncSetAttribute(attn_bf16_kernel<HKV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int64_t grid = std::min<int64_t>(p.items, (int64_t)sms);
+    attn_bf16_kernel<HKV><<<(unsigned)grid, Cfg::kThreads, smem, s>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess || !a.decode) return e;
+    attn_combine_kernel<<<(unsigned)(a.B * Cfg::kHq), 128, 0, s>>>(p.part_o, p.part_lse, p.splits, Cfg::kHq,
+                                                                   (__nv_bfloat16 *)a.out, a.lse);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t attn_decode_ws_bytes(int B, int Hq, int d, int top_k) {
+    // upper bound over the split plans of run_bf16: splits <= top_k + 1
+    const DeviceInfo *di = device_info();
+    const int sms = di ? di->sm_count : 148;
+    const int list_max = top_k + 1;
+    int splits = std::max(1, (2 * sms + B - 1) / B);
+    int sb = (list_max + splits - 1) / splits;
+    sb = std::max(AT_BPS, (sb + AT_BPS - 1) / AT_BPS * AT_BPS);
+    splits = (list_max + sb - 1) / sb;
+    size_t n = (size_t)B * splits * Hq;
+    return (n * d * sizeof(float) + n * sizeof(float) + 255) / 256 * 256;
+}
+
+cudaError_t launch_attn_bf16(const AttnArgs &a, void *ws, unsigned *status, cudaStream_t s) {
+    switch (a.Hkv) {
+    case 1: return run_bf16<1>(a, ws, status, s);
+    case 2: return run_bf16<2>(a, ws, status, s);
+    case 4: return run_bf16<4>(a, ws, status, s);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_attn_f32(const AttnArgs &a, unsigned *status, cudaStream_t s) {
+    const int64_t items = a.decode ? (int64_t)a.B : (int64_t)a.B * a.n_q;
+    const int64_t warps = items * a.Hq;
+    if (warps <= 0) return cudaSuccess;
+    attn_f32_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, s>>>(
+        (const float *)a.q, (const float *)a.k, (const float *)a.v, a.sel, a.nsel, a.seq_len, a.B, a.n_q, a.q0,
+        a.kv_stride, a.Hq, a.Hkv, a.top_k, a.scale, (float *)a.out, a.lse, a.decode ? 1 : 0, status);
+    return cudaGetLastError();
+}
+
+}  // namespace qsa

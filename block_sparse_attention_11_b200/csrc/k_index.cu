@@ -1,0 +1,336 @@
+// k_index.cu -- prefill indexer: block scores on the 5th-generation tensor
+// cores (tcgen05, accumulators in TMEM, operands fed by TMA), an fp32 SIMT
+// variant for the fp32 mode, and the per-row top-k select.
+//
+// Score (page "Qwen3.8-Flash-Next: Day-0 Support in SGLang", section "Qwen
+// Sparse Attention: Retrieve Coarsely, Attend Precisely", score equation):
+//     s_{t,b} = (1/sqrt(128)) * sum_h w_h * phi(<qhat_{t,h}, kbar_b>),  b < nb(t).
+// The positive factor 1/sqrt(128) does not change the ranking and is not
+// applied; only the ranking leaves this file.
+//
+// Two operand layouts:
+//   * head-sum ("hi/lo"): with phi = identity and w = 1 the score is
+//     <sum_h qhat_h, kbar_b>.  The FP32 head sum is split into two BF16 planes
+//     hi + lo (16 significant bits, exact for BF16 heads of similar
+//     magnitude), so one query row costs two K=128 MMAs instead of four and
+//     the ranking keeps FP32 accuracy.  A tile is 128 query rows.
+//   * per-head: rows are (query, head) pairs, 32 queries per 128-row tile;
+//     the epilogue applies phi and w and sums the 4 heads across 4 lanes.
+//
+// Tile shape: M = 128 (TMEM lanes), N = 128 key blocks, K = 128 (two
+// 64-element 128-byte-swizzled k-atoms).  The query tile is loaded once per
+// CTA and stays in shared memory; key tiles stream through a 4-stage TMA
+// ring; two TMEM accumulators (128 columns each) let the epilogue of tile j
+// overlap the MMAs of tile j+1.  Warp roles: 0 = TMA producer, 1 = MMA issuer
+// and TMEM owner, 2..5 = epilogue (warp w reads TMEM lanes 32*(w%4)..+31).
+#include "internal.h"
+#include "select.cuh"
+
+namespace qsa {
+
+namespace {
+
+constexpr int GM = 128;
+constexpr int GN = 128;
+constexpr int NST = 4;
+constexpr int KATOM_BYTES_A = GM * 128;            // 128 rows x 128 bytes
+constexpr int KATOM_BYTES_B = GN * 128;
+constexpr int A_BYTES = 2 * KATOM_BYTES_A;         // one operand plane, both k-atoms
+constexpr int B_STAGE_BYTES = 2 * KATOM_BYTES_B;
+constexpr int GEMM_THREADS = 192;
+constexpr int TMEM_COLS = 2 * GN;
+
+struct GemmSmem {
+    alignas(1024) uint8_t a0[A_BYTES];
+    alignas(1024) uint8_t a1[A_BYTES];
+    alignas(1024) uint8_t b[NST][B_STAGE_BYTES];
+    alignas(8) uint64_t a_full;
+    uint64_t b_full[NST];
+    uint64_t b_empty[NST];
+    uint64_t acc_full[2];
+    uint64_t acc_empty[2];
+    uint32_t tmem_base;
+};
+
+struct GemmParams {
+    int64_t n_q, q0, row_begin, row_count, pool_stride, ld;
+    int per_head, relu;
+    const float *head_w;
+    float *scores;
+    unsigned *status;
+};
+
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    score_gemm_kernel(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ CUtensorMap map_a1,
+                      const __grid_constant__ CUtensorMap map_b, GemmParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    GemmSmem &sm = *reinterpret_cast<GemmSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int seq = blockIdx.y;
+    const int rows_per_tile = p.per_head ? GM / kIdxHeads : GM;
+    const int m = gridDim.x - 1 - blockIdx.x;                 // heaviest (latest) tiles first
+    const int64_t r0 = p.row_begin + (int64_t)m * rows_per_tile;
+    const int64_t r_end = min(r0 + rows_per_tile, p.row_begin + p.row_count);
+    const int64_t t_last = p.q0 + r_end - 1;
+    const int64_t nb_tile = (t_last + 1) / kBlock;
+    const int ntiles = (int)((nb_tile + GN - 1) / GN);
+    const int kplanes = p.per_head ? 1 : 2;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&sm.a_full, 1);
+        for (int s = 0; s < NST; ++s) { mbar_init(&sm.b_full[s], 1); mbar_init(&sm.b_empty[s], 1); }
+        for (int s = 0; s < 2; ++s) { mbar_init(&sm.acc_full[s], 1); mbar_init(&sm.acc_empty[s], 4); }
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&sm.tmem_base, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+
+    if (warp == 0) {
+        // ---------------- TMA producer
+        if (lane == 0 && ntiles > 0) {
+            prefetch_tmap(&map_a0);
+            prefetch_tmap(&map_b);
+            const int ay = p.per_head ? (int)((seq * p.n_q + r0) * kIdxHeads) : (int)(seq * p.n_q + r0);
+            mbar_arrive_expect_tx(&sm.a_full, kplanes * A_BYTES);
+            tma_load_2d(sm.a0, &map_a0, 0, ay, &sm.a_full);
+            tma_load_2d(sm.a0 + KATOM_BYTES_A, &map_a0, 64, ay, &sm.a_full);
+            if (!p.per_head) {
+                tma_load_2d(sm.a1, &map_a1, 0, ay, &sm.a_full);
+                tma_load_2d(sm.a1 + KATOM_BYTES_A, &map_a1, 64, ay, &sm.a_full);
+            }
+            bool ok = true;
+            for (int j = 0; j < ntiles && ok; ++j) {
+                const int s = j % NST;
+                if (j >= NST) ok = mbar_wait(&sm.b_empty[s], ((j / NST) + 1) & 1, p.status);
+                if (!ok) break;
+                const int by = (int)(seq * p.pool_stride + (int64_t)j * GN);
+                mbar_arrive_expect_tx(&sm.b_full[s], B_STAGE_BYTES);
+                tma_load_2d(sm.b[s], &map_b, 0, by, &sm.b_full[s]);
+                tma_load_2d(sm.b[s] + KATOM_BYTES_B, &map_b, 64, by, &sm.b_full[s]);
+            }
+            // make sure no copy is still landing in shared memory when the CTA ends
+            mbar_wait(&sm.a_full, 0, p.status);
+            for (int j = max(0, ntiles - NST); j < ntiles; ++j) mbar_wait(&sm.b_full[j % NST], (j / NST) & 1, p.status);
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer (one thread)
+        if (lane == 0 && ntiles > 0) {
+            const uint32_t idesc = idesc_bf16_f32(GM, GN);
+            bool ok = mbar_wait(&sm.a_full, 0, p.status);
+            tc_fence_after();
+            const uint32_t a0 = smem_u32(sm.a0), a1 = smem_u32(sm.a1);
+            for (int j = 0; j < ntiles && ok; ++j) {
+                const int s = j % NST, ab = j & 1;
+                if (j >= 2) ok = mbar_wait(&sm.acc_empty[ab], ((j >> 1) + 1) & 1, p.status);
+                if (ok) ok = mbar_wait(&sm.b_full[s], (j / NST) & 1, p.status);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t d = tmem + (uint32_t)(ab * GN);
+                const uint32_t bs = smem_u32(sm.b[s]);
+                uint32_t acc = 0;
+                for (int pl = 0; pl < kplanes; ++pl) {
+                    const uint32_t abase = pl ? a1 : a0;
+#pragma unroll
+                    for (int ka = 0; ka < 2; ++ka)
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const uint64_t adesc = sw128_desc(abase + ka * KATOM_BYTES_A + kk * 32);
+                            const uint64_t bdesc = sw128_desc(bs + ka * KATOM_BYTES_B + kk * 32);
+                            tc_mma_f16(d, adesc, bdesc, idesc, acc);
+                            acc = 1;
+                        }
+                }
+                tc_commit(&sm.b_empty[s]);
+                tc_commit(&sm.acc_full[ab]);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ---------------- epilogue: TMEM -> registers -> global scores
+        const int quarter = warp & 3;
+        const int lrow = quarter * 32 + lane;   // TMEM lane = operand row in the tile
+        int64_t qrow;                           // query row (within the sequence)
+        int head = 0;
+        if (p.per_head) { qrow = r0 + lrow / kIdxHeads; head = lrow % kIdxHeads; }
+        else qrow = r0 + lrow;
+        const bool row_live = qrow < r_end;
+        float w = 1.0f;
+        if (p.per_head && p.head_w && row_live) w = p.head_w[(seq * p.n_q + qrow) * kIdxHeads + head];
+        float *dst = p.scores + ((int64_t)seq * p.row_count + (qrow - p.row_begin)) * p.ld;
+        for (int j = 0; j < ntiles; ++j) {
+            const int ab = j & 1;
+            if (!mbar_wait(&sm.acc_full[ab], (j >> 1) & 1, p.status)) break;
+            tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < GN / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(ab * GN + c * 32), r);
+                tc_wait_ld();
+                float v[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+                if (p.per_head) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        float x = v[i];
+                        if (p.relu) x = fmaxf(x, 0.0f);
+                        x *= w;
+                        x += __shfl_xor_sync(0xffffffffu, x, 1);
+                        x += __shfl_xor_sync(0xffffffffu, x, 2);
+                        v[i] = x;
+                    }
+                }
+                const bool writer = row_live && (!p.per_head || head == 0);
+                if (writer) {
+                    float4 *o = reinterpret_cast<float4 *>(dst + (int64_t)j * GN + c * 32);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) o[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.acc_empty[ab]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+// fp32 mode: plain SIMT scores.  One CTA per (query row, 128-block slab);
+// thread b owns one block.  q_hat [B][n_q][4][128] fp32 (rotated, rounded).
+__global__ void __launch_bounds__(128) score_simt_kernel(const float *__restrict__ q_hat,
+                                                          const float *__restrict__ k_pool, GemmParams p) {
+    __shared__ float qs[kIdxHeads][kIdxDim];
+    const int seq = blockIdx.z;
+    const int64_t row = p.row_begin + blockIdx.y;
+    const int64_t t = p.q0 + row;
+    const int64_t nb = (t + 1) / kBlock;
+    const int64_t b = (int64_t)blockIdx.x * 128 + threadIdx.x;
+    for (int i = threadIdx.x; i < kIdxHeads * kIdxDim; i += 128)
+        qs[i / kIdxDim][i % kIdxDim] = q_hat[((int64_t)seq * p.n_q + row) * kIdxHeads * kIdxDim + i];
+    __syncthreads();
+    if (b >= nb) return;
+    const float *kb = k_pool + ((int64_t)seq * p.pool_stride + b) * kIdxDim;
+    float acc = 0.0f;
+#pragma unroll
+    for (int h = 0; h < kIdxHeads; ++h) {
+        float dsum = 0.0f;
+        for (int i = 0; i < kIdxDim; ++i) dsum = fmaf(qs[h][i], kb[i], dsum);
+        if (p.relu) dsum = fmaxf(dsum, 0.0f);
+        const float w = p.head_w ? p.head_w[((int64_t)seq * p.n_q + row) * kIdxHeads + h] : 1.0f;
+        acc += w * dsum;
+    }
+    p.scores[((int64_t)seq * p.row_count + blockIdx.y) * p.ld + b] = acc;
+}
+
+// Per-row top-k over materialised scores: one CTA per (row, sequence).
+__global__ void __launch_bounds__(512) select_rows_kernel(const float *__restrict__ scores, int64_t row_begin,
+                                                          int64_t n_q, int64_t q0, int64_t ld, int top_k,
+                                                          int32_t *__restrict__ sel, int32_t *__restrict__ nsel,
+                                                          int64_t row_count) {
+    extern __shared__ uint32_t keys[];
+    __shared__ SelectSmem sm;
+    const int seq = blockIdx.y;
+    const int64_t rloc = blockIdx.x;
+    const int64_t row = row_begin + rloc;
+    const int64_t t = q0 + row;
+    const int n = (int)((t + 1) / kBlock);
+    const float *src = scores + ((int64_t)seq * row_count + rloc) * ld;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) keys[i] = score_key(src[i]);
+    __syncthreads();
+    int32_t *out = sel + ((int64_t)seq * n_q + row) * top_k;
+    const int cnt = cta_topk(keys, n, top_k, sm, [&](int pos, int i) { out[pos] = i; });
+    for (int i = cnt + threadIdx.x; i < top_k; i += blockDim.x) out[i] = -1;
+    if (threadIdx.x == 0) nsel[(int64_t)seq * n_q + row] = cnt;
+}
+
+// Driver-API tensor-map encoder obtained through the runtime (no -lcuda).
+using EncodeTiledFn = decltype(&cuTensorMapEncodeTiled);
+EncodeTiledFn get_encode() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+// 2-D bf16 map over [rows][128] with a 64 x box_rows box, 128-byte swizzle.
+bool make_map(CUtensorMap *map, const void *base, uint64_t rows, uint32_t box_rows) {
+    auto enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {128, rows};
+    cuuint64_t strides[1] = {128 * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_score_gemm(const ScoreGemmArgs &a, const void *qa0, const void *qa1, const void *k_pool,
+                              unsigned *status, cudaStream_t s) {
+    if (a.row_count <= 0) return cudaSuccess;
+    const int rows_per_tile = a.per_head ? GM / kIdxHeads : GM;
+    const uint64_t a_rows = (uint64_t)a.B * a.n_q * (a.per_head ? kIdxHeads : 1);
+    CUtensorMap ma0, ma1, mb;
+    if (!make_map(&ma0, qa0, a_rows, GM)) return cudaErrorInvalidValue;
+    if (!make_map(&ma1, a.per_head ? qa0 : qa1, a_rows, GM)) return cudaErrorInvalidValue;
+    if (!make_map(&mb, k_pool, (uint64_t)a.B * a.pool_stride, GN)) return cudaErrorInvalidValue;
+    GemmParams p{a.n_q, a.q0, a.row_begin, a.row_count, a.pool_stride, a.ld, a.per_head, a.relu, a.head_w,
+                 a.scores, status};
+    const size_t smem = sizeof(GemmSmem) + 1024;
+    static bool attr_done = false;
+    if (!attr_done) {
+        cudaError_t e = cudaFuncSetAttribute(score_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        attr_done = true;
+    }
+    dim3 grid((unsigned)((a.row_count + rows_per_tile - 1) / rows_per_tile), (unsigned)a.B);
+    score_gemm_kernel<<<grid, GEMM_THREADS, smem, s>>>(ma0, ma1, mb, p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_score_simt_f32(const ScoreGemmArgs &a, const float *q_hat, const float *k_pool, cudaStream_t s) {
+    if (a.row_count <= 0) return cudaSuccess;
+    const int64_t nb_max = (a.q0 + a.row_begin + a.row_count) / kBlock;
+    if (nb_max <= 0) return cudaSuccess;
+    GemmParams p{a.n_q, a.q0, a.row_begin, a.row_count, a.pool_stride, a.ld, 0, a.relu, a.head_w, a.scores,
+                 nullptr};
+    dim3 grid((unsigned)((nb_max + 127) / 128), (unsigned)a.row_count, (unsigned)a.B);
+    score_simt_kernel<<<grid, 128, 0, s>>>(q_hat, k_pool, p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_select_rows(const float *scores, int B, int64_t row_begin, int64_t row_count, int64_t n_q,
+                               int64_t q0, int64_t ld, int top_k, int32_t *sel, int32_t *nsel, unsigned *status,
+                               cudaStream_t s) {
+    (void)status;
+    if (row_count <= 0) return cudaSuccess;
+    const size_t smem = (size_t)ld * sizeof(uint32_t);
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(select_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    dim3 grid((unsigned)row_count, (unsigned)B);
+    select_rows_kernel<<<grid, 512, smem, s>>>(scores, row_begin, n_q, q0, ld, top_k, sel, nsel, row_count);
+    return cudaGetLastError();
+}
+
+}  // namespace qsa

@@ -1,0 +1,286 @@
+/*
+ * qsa.h -- C ABI of libqsa: Qwen Sparse Attention (QSA) on NVIDIA B200 (sm_100a).
+ *
+ * QSA (page "Qwen3.8-Flash-Next: Day-0 Support in SGLang", section "Qwen Sparse
+ * Attention: Retrieve Coarsely, Attend Precisely"; page "Qwen3.8-Flash-Next,
+ * Layer by Layer", section "Token mixing") runs in two stages per attention
+ * layer:
+ *   1. an indexer mean-pools every 4 consecutive raw indexer keys (in FP32),
+ *      rotates the mean with the first token's RoPE position, stores it as one
+ *      BF16 compressed key, scores every complete visible block for each query
+ *      with 4 indexer query heads against the one shared 128-dim key head, and
+ *      keeps the best 512 blocks;
+ *   2. softmax attention over the original (uncompressed) K/V at exactly the
+ *      selected blocks' 4*512 = 2048 positions plus the query's own 0-3 tail
+ *      tokens (at most 2051 positions).
+ *
+ * Conventions shared by every entry point
+ *   - Pointers named as device pointers are device memory owned by the
+ *     caller; host pointers are named so.  The library allocates nothing and
+ *     never synchronises the stream (qsa_check_status excepted).
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL = the legacy default stream).
+ *   - All tensors are dense, row-major, with the layouts stated per call.
+ *     Element type: `dtype` = QSA_BF16 (bfloat16) or QSA_FP32 (float) for
+ *     every floating-point tensor of the call, except head weights (always
+ *     float) and the fp32 scratch.
+ *   - Indexer geometry is fixed by the pages: 4 query heads, 1 key head,
+ *     128 dims, blocks of 4 tokens.  Attention head dim d = 128.
+ *   - Positions: token i of a sequence has RoPE position i.  Block b holds
+ *     positions 4b..4b+3 and is visible to the query at position t iff
+ *     4b + 3 <= t, so nb(t) = floor((t + 1) / 4) blocks are visible and the
+ *     tail is positions 4*nb(t)..t.  A query selects min(top_k, nb(t)) blocks.
+ *   - Selections are written as block ids sorted ascending, padded with -1
+ *     up to top_k, plus a count.  Ranking: higher score first, equal scores
+ *     go to the lower block id.
+ *   - Return value: QSA_OK or an error code.  Invalid arguments are rejected
+ *     before anything is launched and leave no state behind.  Kernels that
+ *     find an out-of-range index or run out of a bounded wait set the
+ *     library's device status word instead of trapping; qsa_check_status
+ *     reads it.
+ */
+#ifndef QSA_H
+#define QSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QSA_API __attribute__((visibility("default")))
+#else
+#define QSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ---- */
+#define QSA_OK 0
+#define QSA_ERR_INVALID_ARG 1   /* null pointer, bad size, bad stride, bad flag */
+#define QSA_ERR_UNSUPPORTED 2   /* shape/dtype/option this build does not implement, or not an sm_100 device */
+#define QSA_ERR_CUDA 3          /* a CUDA launch or runtime call failed */
+#define QSA_ERR_DEVICE 4        /* a kernel reported a bounds violation or a wait timeout */
+#define QSA_ERR_WORKSPACE 5     /* workspace pointer null or smaller than the size query returned */
+
+/* ---- element types ---- */
+#define QSA_BF16 0
+#define QSA_FP32 1
+
+/* ---- option flags ---- */
+/* Score with ReLU of each head's dot product, as in the score equation of
+ * "Qwen Sparse Attention: Retrieve Coarsely, Attend Precisely".  Off by
+ * default: the default score is the plain sum over heads. */
+#define QSA_SCORE_RELU 1u
+/* Normalise the FP32 block mean before rotation (unit-weight RMS norm,
+ * eps 1e-6); the same section says the mean is "normalized" without naming
+ * the norm.  Off by default. */
+#define QSA_POOL_RMSNORM 2u
+
+/* RoPE parameters.  Rotate-half convention (style 0): for i < rotary_dim/2
+ * the pair (x_i, x_{i + rotary_dim/2}) turns by the angle
+ * (pos / pos_scale) * base^(-2i / rotary_dim); dims >= rotary_dim are left
+ * alone.  rotary_dim: even, multiple of 16, 16..128.  pos_scale > 0 is a
+ * linear position scale (4 stands in for the 1M-token context extension). */
+typedef struct {
+    double base;
+    double pos_scale;
+    int32_t rotary_dim;
+    int32_t style;      /* 0 = rotate-half; other values -> QSA_ERR_UNSUPPORTED */
+} qsa_rope_t;
+
+/* Human-readable text of a status code (static storage). */
+QSA_API const char *qsa_strerror(int status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+QSA_API int qsa_version(void);
+
+/* Reads and clears the device status word of the current device after
+ * synchronising `stream`.  Returns QSA_OK, or QSA_ERR_DEVICE when a kernel
+ * flagged an out-of-range index or a wait timeout since the last call.  If
+ * detail != NULL it receives the raw status bits (host pointer). */
+QSA_API int qsa_check_status(void *stream, uint32_t *detail);
+
+/* ========================================================================= */
+/* a1. Compressed-key pooling, prefill                                        */
+/* ========================================================================= */
+/*
+ * For each sequence i < B and each complete block j < floor(n_tok / 4) of the
+ * raw keys k_raw[i][0..n_tok):
+ *     m   = (((k0 + k1) + k2) + k3) * 0.25            (FP32, the pages' "averaged in FP32")
+ *     m   = m / sqrt(mean(m^2) + 1e-6)                 (only with QSA_POOL_RMSNORM)
+ *     out = RoPE(m, position pos0 + 4j)                (the first token's position)
+ *     k_pool[i][pos0/4 + j] = round_to_dtype(out)      (BF16: round to nearest even)
+ * Source: "Qwen Sparse Attention: Retrieve Coarsely, Attend Precisely" (four raw
+ * index keys averaged in FP32, rotated with the first token's position, one
+ * BF16 compressed key per four tokens); flozi.net guide, "How a token moves
+ * through the model", item 2 (RoPE after pooling).
+ *
+ * k_raw   device, [B][raw_stride][128] dtype; tokens pos0 .. pos0+n_tok-1 of
+ *         each sequence sit at rows 0 .. n_tok-1.
+ * k_pool  device, [B][pool_stride][128] dtype; rows pos0/4 .. pos0/4 +
+ *         floor(n_tok/4) - 1 are written, nothing else.
+ * pos0    multiple of 4, >= 0.  Trailing n_tok mod 4 tokens are not pooled
+ *         (they belong in the decode ring); n_tok < 4 is a no-op (pointers
+ *         may then be NULL).
+ * Errors: QSA_ERR_INVALID_ARG for null pointers, B < 1, n_tok < 0,
+ *         raw_stride < n_tok, pos0 mod 4 != 0, pool_stride < pos0/4 +
+ *         floor(n_tok/4), bad flags or rope; QSA_ERR_UNSUPPORTED for a style
+ *         other than 0.
+ */
+QSA_API int qsa_pool_keys_prefill(const void *k_raw, void *k_pool, int32_t B, int64_t n_tok, int64_t pos0,
+                          int64_t raw_stride, int64_t pool_stride, qsa_rope_t rope, uint32_t flags,
+                          int32_t dtype, void *stream);
+
+/* ========================================================================= */
+/* a1d. Compressed-key pooling, decode (four-slot ring)                       */
+/* ========================================================================= */
+/*
+ * One new token per sequence.  seq_len[i] = s counts the tokens including the
+ * new one, whose position is p = s - 1.  The new raw key goes to ring slot
+ * p mod 4.  When s mod 4 == 0 the block is complete: ring slots 0..3 are
+ * pooled exactly as in qsa_pool_keys_prefill (position s - 4) into
+ * k_pool[i][s/4 - 1].
+ * Source: "Qwen Sparse Attention: Retrieve Coarsely, Attend Precisely" (the raw
+ * keys of the unfinished block live in a four-slot per-request ring).
+ *
+ * k_new    device, [B][128] dtype, raw indexer key of the new token.
+ * ring     device, [B][4][128] dtype, updated in place.
+ * k_pool   device, [B][pool_stride][128] dtype.
+ * seq_len  device, [B] int32, each >= 1.  A sequence whose s/4 > pool_stride
+ *          is skipped and flagged in the device status word.
+ */
+QSA_API int qsa_pool_keys_decode(const void *k_new, void *ring, void *k_pool, const int32_t *seq_len,
+                         int32_t B, int64_t pool_stride, qsa_rope_t rope, uint32_t flags,
+                         int32_t dtype, void *stream);
+
+/* ========================================================================= */
+/* a2-a4. Indexer scores and top-k, prefill                                    */
+/* ========================================================================= */
+/*
+ * For each sequence i and query row r < n_q (position t = q0 + r):
+ *     qhat_h = round_to_dtype(RoPE(q_idx[i][r][h], t))           h = 0..3
+ *     s_b    = (1/sqrt(128)) * sum_h w_h * phi(<qhat_h, k_pool[i][b]>),  b < nb(t)
+ * with phi = ReLU under QSA_SCORE_RELU and the identity otherwise, w_h =
+ * head_w[i][r][h] or 1 when head_w is NULL; then the min(top_k, nb(t)) best
+ * blocks are written to sel[i][r][0..top_k) ascending (padded with -1) and
+ * their count to nsel[i][r].
+ * Source: "Qwen Sparse Attention: Retrieve Coarsely, Attend Precisely" (score
+ * equation s_{t,b}; keeps the best 512 blocks); "Token mixing" (4 query
+ * heads, 1 key head, 128 dims).
+ *
+ * q_idx    device, [B][n_q][4][128] dtype, RAW (unrotated) indexer queries.
+ * k_pool   device, [B][pool_stride][128] dtype, compressed keys of positions
+ *          0 .. q0+n_q-1 (rows 0 .. nb(q0+n_q-1)-1 must be valid).
+ * head_w   device, [B][n_q][4] float, or NULL.
+ * sel      device, [B][n_q][top_k] int32.   nsel  device, [B][n_q] int32.
+ * workspace device scratch of at least qsa_index_topk_prefill_workspace()
+ *          bytes, 256-byte aligned; contents on entry are ignored.
+ * top_k    1..2048.
+ */
+QSA_API size_t qsa_index_topk_prefill_workspace(int32_t B, int64_t n_q, int64_t q0, int32_t top_k,
+                                        uint32_t flags, int32_t dtype);
+QSA_API int qsa_index_topk_prefill(const void *q_idx, const void *k_pool, const float *head_w, int32_t B,
+                           int64_t n_q, int64_t q0, int64_t pool_stride, int32_t top_k, int32_t *sel,
+                           int32_t *nsel, void *workspace, size_t ws_bytes, qsa_rope_t rope,
+                           uint32_t flags, int32_t dtype, void *stream);
+
+/* ========================================================================= */
+/* a2-a4 (decode). Indexer scores and top-k for one new token per sequence     */
+/* ========================================================================= */
+/*
+ * As qsa_index_topk_prefill for the single query at position t = seq_len[i]-1
+ * of each sequence, scanning all nb(t) = floor(seq_len[i]/4) compressed keys
+ * (run qsa_pool_keys_decode first so a block completed by the new token is
+ * visible).  Source: as above, and "IndexShare MTP" (the decode scorer scans
+ * all ceil(L/4) compressed blocks and dominates the layer's cost at long
+ * context).
+ *
+ * q_idx     device, [B][4][128] dtype, RAW indexer query of the new token.
+ * k_pool    device, [B][pool_stride][128] dtype.
+ * head_w    device, [B][4] float, or NULL.
+ * seq_len   device, [B] int32.
+ * max_blocks host bound on floor(seq_len[i]/4) for every i (sizes the grid;
+ *           a sequence beyond it or beyond pool_stride is flagged and gets
+ *           nsel = 0).
+ * sel       device, [B][top_k] int32;  nsel device, [B] int32.
+ * workspace at least qsa_index_topk_decode_workspace() bytes.
+ */
+QSA_API size_t qsa_index_topk_decode_workspace(int32_t B, int64_t max_blocks, int32_t top_k, uint32_t flags,
+                                       int32_t dtype);
+QSA_API int qsa_index_topk_decode(const void *q_idx, const void *k_pool, const float *head_w,
+                          const int32_t *seq_len, int32_t B, int64_t pool_stride, int64_t max_blocks,
+                          int32_t top_k, int32_t *sel, int32_t *nsel, void *workspace, size_t ws_bytes,
+                          qsa_rope_t rope, uint32_t flags, int32_t dtype, void *stream);
+
+/* ========================================================================= */
+/* a5-a6. Sparse attention, prefill                                           */
+/* ========================================================================= */
+/*
+ * For each sequence i, query row r (position t = q0 + r) and q head h
+ * (kv head g = floor(h * Hkv / Hq)):
+ *     P(t) = {4b .. 4b+3 : b in sel[i][r][0..nsel)}  U  {4*nb(t) .. t}
+ *     out[i][r][h] = sum_{j in P(t)} softmax_j(scale * <q[i][r][h], k[i][j][g]>) v[i][j][g]
+ *     lse[i][r][h] = log(sum_{j in P(t)} exp(scale * <q, k_j>))     (natural log)
+ * Softmax and accumulation in fp32; out rounded to dtype.
+ * Source: "Qwen Sparse Attention: Retrieve Coarsely, Attend Precisely" (expand
+ * the 512 blocks to 2048 positions, append the 0-3 tail tokens, softmax and
+ * value aggregation over the original uncompressed K/V; one selection per
+ * query shared by all heads).
+ *
+ * q        device, [B][n_q][Hq][d] dtype, already rotated (the attention
+ *          layer's RoPE is applied by the caller, see qsa_rope_apply).
+ * k, v     device, [B][kv_stride][Hkv][d] dtype, rows by position; k rotated.
+ * sel/nsel device, as written by qsa_index_topk_prefill.  Ids must satisfy
+ *          0 <= b < nb(t); out-of-range ids are skipped and flagged.
+ * out      device, [B][n_q][Hq][d] dtype.   lse device, [B][n_q][Hq] float or NULL.
+ * Shapes: d == 128; Hq % Hkv == 0; Hq / Hkv == 8 for QSA_BF16 (the GQA
+ *         ratio of the kernels' tiles), any ratio for QSA_FP32;
+ *         kv_stride >= q0 + n_q.
+ * workspace: none needed (pass NULL, 0).
+ */
+QSA_API int qsa_sparse_attn_prefill(const void *q, const void *k, const void *v, const int32_t *sel,
+                            const int32_t *nsel, int32_t B, int64_t n_q, int64_t q0, int64_t kv_stride,
+                            int32_t Hq, int32_t Hkv, int32_t d, int32_t top_k, float scale, void *out,
+                            float *lse, void *workspace, size_t ws_bytes, int32_t dtype, void *stream);
+
+/* ========================================================================= */
+/* a5-a6 (decode). Sparse attention for one new token per sequence            */
+/* ========================================================================= */
+/*
+ * As qsa_sparse_attn_prefill for the query at position t = seq_len[i] - 1.
+ * The caller has written the new token's rotated k and its v at row t of
+ * the caches.  The work of each sequence is split across CTAs and combined
+ * (split-KV); the partial results live in the workspace.
+ *
+ * q        device, [B][Hq][d] dtype (rotated).
+ * k, v     device, [B][kv_stride][Hkv][d] dtype.
+ * sel/nsel device, [B][top_k] / [B] from qsa_index_topk_decode.
+ * out      device, [B][Hq][d] dtype.   lse device, [B][Hq] float or NULL.
+ * workspace at least qsa_sparse_attn_decode_workspace() bytes.
+ */
+QSA_API size_t qsa_sparse_attn_decode_workspace(int32_t B, int32_t Hq, int32_t d, int32_t top_k, int32_t dtype);
+QSA_API int qsa_sparse_attn_decode(const void *q, const void *k, const void *v, const int32_t *seq_len,
+                           const int32_t *sel, const int32_t *nsel, int32_t B, int64_t kv_stride,
+                           int32_t Hq, int32_t Hkv, int32_t d, int32_t top_k, float scale, void *out,
+                           float *lse, void *workspace, size_t ws_bytes, int32_t dtype, void *stream);
+
+/* ========================================================================= */
+/* Helper: the attention layer's RoPE                                         */
+/* ========================================================================= */
+/*
+ * Rotates x[i][r][h][0..d) in place at position pos0 + r (fp64 angles,
+ * result rounded to dtype), for i < B, r < n, h < H.  This is the rotation
+ * the pages keep in the full-attention layers ("Token mixing": the
+ * full-attention layers keep rotary position embeddings); callers use it to
+ * produce the rotated q/k the sparse attention consumes.
+ * x: device, [B][n][H][d] dtype, d even, rotary_dim <= d.
+ */
+QSA_API int qsa_rope_apply(void *x, int32_t B, int64_t n, int32_t H, int32_t d, int64_t pos0, qsa_rope_t rope,
+                   int32_t dtype, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QSA_H */

@@ -1,0 +1,236 @@
+"""Stage-by-stage GPU parity against the CPU oracle on sizes the oracle
+finishes in seconds (several tiles plus a ragged tail), plus edge cases.
+
+Each stage is fed the same inputs as the oracle's stage: the GPU attention
+runs on the oracle's selection, so a tie decided differently upstream can
+neither hide nor fake an attention error."""
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from qsa_testlib import TOL, check_prefill_workload, np32, rope_of
+
+pytestmark = pytest.mark.gpu
+
+import oracle  # noqa: E402
+
+
+@pytest.fixture(scope="module")
+def qsa():
+    import block_sparse_attention_11_b200 as m
+    assert torch.cuda.is_available()
+    return m
+
+
+DEV = "cuda"
+
+
+def W(T, top_k=64, Hq=16, Hkv=2, dtype="bf16", seed=11, **kw):
+    return workloads.Workload(f"t{T}", "prefill", kw.pop("B", 1), T, top_k, Hq, Hkv, 128, dtype, seed, **kw)
+
+
+# ----------------------------------------------------------------------------- pooling
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+@pytest.mark.parametrize("n_tok,pos0,R,ps,flags", [(4099, 0, 128, 1.0, 0), (1000, 4 * 12345, 128, 1.0, 0),
+                                                  (4096, 1 << 20, 128, 4.0, 0), (515, 0, 64, 1.0, 0),
+                                                  (512, 8, 128, 1.0, 2)])
+def test_pool_prefill_bit_exact(qsa, dtype, n_tok, pos0, R, ps, flags):
+    g = torch.Generator(device=DEV).manual_seed(n_tok + pos0)
+    dt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    k_raw = torch.randn(2, n_tok, 128, generator=g, device=DEV).to(dt)
+    cap = pos0 // 4 + n_tok // 4 + 3
+    k_pool = torch.full((2, cap, 128), 7.0, dtype=dt, device=DEV)
+    rope = qsa.Rope(pos_scale=ps, rotary_dim=R)
+    qsa.qsa_pool_keys_prefill(k_raw, k_pool, pos0=pos0, rope=rope, flags=flags)
+    qsa.qsa_check_status()
+    for b in range(2):
+        ref = oracle.pool_keys(np32(k_raw[b]), pos0=pos0, pos_scale=ps, rotary_dim=R, rmsnorm=bool(flags & 2),
+                               store_bf16=dtype == "bf16")
+        got = np32(k_pool[b])
+        assert np.array_equal(got[pos0 // 4: pos0 // 4 + n_tok // 4], ref)
+        assert np.all(got[: pos0 // 4] == 7.0) and np.all(got[pos0 // 4 + n_tok // 4:] == 7.0)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_pool_decode_ring_matches_oracle(qsa, dtype):
+    B, steps = 5, 23
+    dt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    g = torch.Generator(device=DEV).manual_seed(3)
+    start = torch.tensor([0, 1, 2, 3, 101], dtype=torch.int32)
+    keys = torch.randn(B, steps, 128, generator=g, device=DEV).to(dt)
+    ring = torch.zeros(B, 4, 128, dtype=dt, device=DEV)
+    cap = (int(start.max()) + steps) // 4 + 1
+    k_pool = torch.zeros(B, cap, 128, dtype=dt, device=DEV)
+    o_ring = np.zeros((B, 4, 128), np.float32)
+    o_pool = np.zeros((B, cap, 128), np.float32)
+    rope = qsa.Rope(pos_scale=4.0)
+    for s in range(steps):
+        seq_len = (start + s + 1).to(DEV)
+        qsa.qsa_pool_keys_decode(keys[:, s].contiguous(), ring, k_pool, seq_len, rope=rope)
+        kn = np32(keys[:, s])
+        for b in range(B):
+            oracle.pool_decode(kn[b], o_ring[b], o_pool[b], int(start[b]) + s + 1, pos_scale=4.0,
+                               store_bf16=dtype == "bf16")
+    qsa.qsa_check_status()
+    assert np.array_equal(np32(ring), o_ring)
+    assert np.array_equal(np32(k_pool), o_pool)
+
+
+def test_rope_apply_matches_oracle(qsa):
+    g = torch.Generator(device=DEV).manual_seed(5)
+    x = torch.randn(2, 300, 3, 128, generator=g, device=DEV).to(torch.bfloat16)
+    ref_in = np32(x)
+    qsa.qsa_rope_apply(x, pos0=77, rope=qsa.Rope(rotary_dim=64))
+    got = np32(x)
+    for b in range(2):
+        for h in range(3):
+            rot = oracle.rope_rows(ref_in[b, :, h], np.arange(77, 377), rotary_dim=64)
+            exp = np.vectorize(oracle.round_bf16)(rot)
+            assert np.array_equal(got[b, :, h], exp.astype(np.float32))
+
+
+# ----------------------------------------------------------------------------- prefill indexer + attention
+
+@pytest.mark.parametrize("T,top_k,flags,weights,dtype", [
+    (4099, 64, 0, False, "bf16"),      # hi/lo tensor-core path, ragged tail, many tiles
+    (4099, 512, 0, False, "bf16"),     # top-512: nb < k for the first 2048 rows
+    (2315, 64, 1, False, "bf16"),      # ReLU: per-head tensor-core path
+    (2315, 64, 0, True, "bf16"),       # head weights: per-head path
+    (1024, 64, 0, False, "fp32"),      # fp32 SIMT path (tiny workload shape)
+    (1031, 64, 1, True, "fp32"),
+    (7, 4, 0, False, "bf16"),          # fewer than one tile, rows with 0 and 1 blocks
+    (1, 4, 0, False, "bf16"),          # single token: attends to itself
+])
+def test_prefill_pipeline(qsa, T, top_k, flags, weights, dtype):
+    w = W(T, top_k=top_k, dtype=dtype, Hq=8 if dtype == "fp32" else 16, Hkv=1 if dtype == "fp32" else 2)
+    x = workloads.make_prefill(w, device=DEV)
+    head_w = None
+    if weights:
+        head_w = torch.rand(1, T, 4, generator=torch.Generator(device=DEV).manual_seed(9), device=DEV) * 2
+    rows = list(range(T))
+    r = check_prefill_workload(x, w, rows, top_k=top_k, flags=flags, head_w=head_w)
+    assert r["nbad"] <= max(2, T // 200), f"too many near-tie rows: {r['nbad']}"
+
+
+def test_prefill_batched_and_chunked(qsa):
+    """B = 2 sequences; and chunked prefill (pooling and queries in chunks
+    against the growing cache) gives the same selections as one shot."""
+    w = W(3000, top_k=128, B=2, seed=21)
+    x = workloads.make_prefill(w, device=DEV)
+    g = check_prefill_workload(x, w, list(range(0, 3000, 7)), b=1)["g"]
+    rope = rope_of(w)
+    k_pool = torch.zeros(2, 750, 128, dtype=torch.bfloat16, device=DEV)
+    sel = torch.empty(2, 3000, 128, dtype=torch.int32, device=DEV)
+    nsel = torch.empty(2, 3000, dtype=torch.int32, device=DEV)
+    out = torch.empty_like(x["q"])
+    for c0, c1 in [(0, 1024), (1024, 2048), (2048, 3000)]:
+        qsa.qsa_pool_keys_prefill(x["k_idx"][:, c0:c1].contiguous(), k_pool, pos0=c0, rope=rope)
+        s = torch.empty(2, c1 - c0, 128, dtype=torch.int32, device=DEV)
+        n = torch.empty(2, c1 - c0, dtype=torch.int32, device=DEV)
+        qsa.qsa_index_topk_prefill(x["q_idx"][:, c0:c1].contiguous(), k_pool, s, n, q0=c0, top_k=128, rope=rope)
+        o = torch.empty(2, c1 - c0, 16, 128, dtype=torch.bfloat16, device=DEV)
+        qsa.qsa_sparse_attn_prefill(x["q"][:, c0:c1].contiguous(), x["k"], x["v"], s, n, o, q0=c0)
+        sel[:, c0:c1] = s
+        nsel[:, c0:c1] = n
+        out[:, c0:c1] = o
+    qsa.qsa_check_status()
+    assert torch.equal(k_pool, g["k_pool"])
+    assert torch.equal(sel, g["sel"]) and torch.equal(nsel, g["nsel"])
+    assert torch.equal(out, g["out"])
+
+
+def test_attention_stage_isolated_on_oracle_selection(qsa):
+    """GPU attention fed the oracle's selection, compared with the oracle's attention."""
+    for dtype, Hq, Hkv in [("bf16", 16, 2), ("bf16", 8, 1), ("bf16", 32, 4), ("fp32", 8, 1), ("fp32", 12, 4)]:
+        w = W(2500, top_k=96, Hq=Hq, Hkv=Hkv, dtype=dtype, seed=33)
+        x = workloads.make_prefill(w, device=DEV)
+        rows = list(range(2500))
+        kp = oracle.pool_keys(np32(x["k_idx"][0]), store_bf16=dtype == "bf16")
+        ref = oracle.prefill_rows(rows, q_idx=np32(x["q_idx"][0]), k_pool=kp, top_k=96,
+                                  store_bf16=dtype == "bf16", q=np32(x["q"][0]), k=np32(x["k"][0]),
+                                  v=np32(x["v"][0]), Hq=Hq, Hkv=Hkv, d=128)
+        sel = torch.from_numpy(ref["sel"][None]).to(DEV)
+        nsel = torch.from_numpy(ref["nsel"][None]).to(DEV)
+        out = torch.empty_like(x["q"])
+        lse = torch.empty(1, 2500, Hq, dtype=torch.float32, device=DEV)
+        qsa.qsa_sparse_attn_prefill(x["q"], x["k"], x["v"], sel, nsel, out, lse=lse)
+        qsa.qsa_check_status()
+        err = np.abs(np32(out[0]) - ref["out"]).max()
+        assert err <= TOL[dtype], (dtype, Hq, Hkv, err)
+        assert np.abs(lse[0].cpu().numpy() - ref["lse"]).max() <= (1e-3 if dtype == "bf16" else 1e-4)
+
+
+def test_attention_flags_out_of_range_ids(qsa):
+    """A selection id outside [0, nb(t)) is skipped and reported through the
+    status word (no trap)."""
+    w = W(64, top_k=4, seed=5)
+    x = workloads.make_prefill(w, device=DEV)
+    sel = torch.full((1, 64, 4), -1, dtype=torch.int32, device=DEV)
+    nsel = torch.zeros(1, 64, dtype=torch.int32, device=DEV)
+    sel[0, 40, 0] = 10            # nb(40) = 10: id 10 is not visible
+    nsel[0, 40] = 1
+    out = torch.empty_like(x["q"])
+    qsa.qsa_sparse_attn_prefill(x["q"], x["k"], x["v"], sel, nsel, out)
+    with pytest.raises(qsa.QSAError):
+        qsa.qsa_check_status()
+    qsa.qsa_check_status()        # cleared
+
+
+# ----------------------------------------------------------------------------- decode
+
+@pytest.mark.parametrize("dtype,flags,weights,L,B", [("bf16", 0, False, 20000, 6), ("bf16", 1, True, 9001, 3),
+                                                     ("fp32", 0, False, 5000, 4), ("bf16", 0, False, 2, 5)])
+def test_decode_pipeline(qsa, dtype, flags, weights, L, B):
+    w = workloads.Workload("dec", "decode", B, L, 256, 16, 2, 128, dtype, 77, pos_scale=2.0)
+    x = workloads.make_decode(w, device=DEV, ragged=True)
+    dt = x["k"].dtype
+    rope = rope_of(w)
+    lens = x["lens"]
+    cap = max(lens) // 4 + 2
+    # pooled cache of the prefix (prefill pooling), ring holding the unfinished block
+    k_pool = torch.zeros(B, cap, 128, dtype=dt, device=DEV)
+    ring = torch.zeros(B, 4, 128, dtype=dt, device=DEV)
+    for b in range(B):
+        kp = torch.zeros(1, cap, 128, dtype=dt, device=DEV)
+        qsa.qsa_pool_keys_prefill(x["k_idx"][b:b + 1, :lens[b]].contiguous(), kp, rope=rope)
+        k_pool[b] = kp[0]
+        nb0 = lens[b] // 4
+        r = lens[b] - 4 * nb0
+        if r:
+            ring[b, :r] = x["k_idx"][b, 4 * nb0: lens[b]]
+    head_w = torch.rand(B, 4, device=DEV) * 2 if weights else None
+    qsa.qsa_pool_keys_decode(x["k_idx_new"], ring, k_pool, x["seq_len"], rope=rope, flags=flags & 2)
+    sel = torch.full((B, w.top_k), -7, dtype=torch.int32, device=DEV)
+    nsel = torch.full((B,), -7, dtype=torch.int32, device=DEV)
+    qsa.qsa_index_topk_decode(x["q_idx"], k_pool, x["seq_len"], sel, nsel, top_k=w.top_k, head_w=head_w,
+                              rope=rope, flags=flags)
+    out = torch.empty_like(x["q"])
+    lse = torch.empty(B, 16, dtype=torch.float32, device=DEV)
+    qsa.qsa_sparse_attn_decode(x["q"], x["k"], x["v"], x["seq_len"], sel, nsel, out, lse=lse)
+    qsa.qsa_check_status()
+    # oracle, sequence by sequence
+    for b in range(B):
+        s = lens[b] + 1
+        kr = np32(x["k_idx"][b, :lens[b]])
+        kp = np.zeros((cap, 128), np.float32)
+        kp[: lens[b] // 4] = oracle.pool_keys(kr, pos_scale=2.0, store_bf16=dtype == "bf16")
+        rg = np.zeros((4, 128), np.float32)
+        nb0 = lens[b] // 4
+        rg[: lens[b] - 4 * nb0] = kr[4 * nb0:]
+        oracle.pool_decode(np32(x["k_idx_new"][b]), rg, kp, s, pos_scale=2.0, store_bf16=dtype == "bf16")
+        assert np.array_equal(np32(k_pool[b]), kp), f"pooled cache differs (seq {b})"
+        ref = oracle.decode(np32(x["q_idx"][b:b + 1]), kp[None], [s],
+                            head_w=None if head_w is None else head_w[b:b + 1].cpu().numpy(),
+                            q=np32(x["q"][b:b + 1]), k=np32(x["k"][b:b + 1]), v=np32(x["v"][b:b + 1]),
+                            relu=bool(flags & 1), store_bf16=dtype == "bf16", top_k=w.top_k, pos_scale=2.0)
+        g_sel = sel[b].cpu().numpy()
+        assert int(nsel[b]) == ref["nsel"][0]
+        gap = (ref["kth"][0] - ref["next"][0]) / max(abs(ref["kth"][0]), 1e-30)
+        if not np.array_equal(g_sel, ref["sel"][0]):
+            assert gap < 1e-4, f"seq {b}: selection differs with gap {gap}"
+            continue
+        err = np.abs(np32(out[b]) - ref["out"][0]).max()
+        assert err <= TOL[dtype], (b, err)
+        assert np.abs(lse[b].cpu().numpy() - ref["lse"][0]).max() <= (1e-3 if dtype == "bf16" else 1e-4)

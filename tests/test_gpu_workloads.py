@@ -1,0 +1,138 @@
+"""Full-size parity of the five workloads the method is measured on, in the
+launch configuration the benchmark times, against the CPU oracle on sampled
+rows (prefill) or every sequence (decode)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from qsa_testlib import TOL, check_prefill_workload, np32, rope_of
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module")
+def qsa():
+    import block_sparse_attention_11_b200 as m
+    return m
+
+
+def _free():
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+
+def test_tiny_prefill_fp32_all_rows(qsa):
+    w = workloads.WORKLOADS["tiny_prefill_t1k_fp32"]
+    x = workloads.make_prefill(w, device=DEV)
+    r = check_prefill_workload(x, w, list(range(w.T)))
+    assert r["nbad"] <= 2
+    assert r["err"] <= TOL["fp32"]
+
+
+def test_prefill_32k_needles(qsa):
+    w = workloads.WORKLOADS["prefill_t32k_needles"]
+    x = workloads.make_prefill(w, device=DEV)
+    rows = workloads.sample_rows(w.T, x["needles"], n_uniform=1024)
+    r = check_prefill_workload(x, w, rows)
+    # every needle block is selected by each of its aligned queries
+    g_sel = r["g"]["sel"][0].cpu().numpy()
+    g_nsel = r["g"]["nsel"][0].cpu().numpy()
+    assert len(x["needles"]) == w.needles
+    for b, ts in x["needles"]:
+        for t in ts:
+            assert b in set(g_sel[t, :g_nsel[t]].tolist()), f"needle block {b} missed by query {t}"
+    assert r["nbad"] <= len(rows) // 50
+    del x, r
+    _free()
+
+
+def test_prefill_dense_reduction_t2048(qsa):
+    """T = 2048 with top-512: every visible block is selected, so the sparse
+    path must equal textbook causal attention."""
+    w = workloads.Workload("dense2048", "prefill", 1, 2048, 512, 16, 2, 128, "bf16", 99)
+    x = workloads.make_prefill(w, device=DEV)
+    from qsa_testlib import gpu_prefill
+    g = gpu_prefill(x, w)
+    rows = np.arange(0, 2048, 3)
+    ref = oracle.dense_rows(rows, np32(x["q"][0]), np32(x["k"][0]), np32(x["v"][0]), 16, 2, 128)
+    err = np.abs(np32(g["out"][0])[rows] - ref).max()
+    assert err <= TOL["bf16"], err
+    nb = (np.arange(2048) + 1) // 4
+    assert np.array_equal(g["nsel"][0].cpu().numpy(), np.minimum(nb, 512))
+
+
+def test_prefill_128k_heavy_tail(qsa):
+    w = workloads.WORKLOADS["prefill_t128k_heavytail"]
+    x = workloads.make_prefill(w, device=DEV)
+    rows = workloads.sample_rows(w.T, n_uniform=1024)
+    r = check_prefill_workload(x, w, rows)
+    assert r["nbad"] <= len(rows) // 50
+    del x, r
+    _free()
+
+
+def _decode_check(qsa, w, B=None, L=None, ragged=False):
+    x = workloads.make_decode(w, device=DEV, B=B, L=L, ragged=ragged)
+    B = x["q"].shape[0]
+    lens = x["lens"]
+    rope = rope_of(w)
+    dt = x["k"].dtype
+    cap = max(lens) // 4 + 1
+    k_pool = torch.zeros(B, cap, 128, dtype=dt, device=DEV)
+    ring = torch.zeros(B, 4, 128, dtype=dt, device=DEV)
+    for b in range(B):
+        kp = torch.zeros(1, cap, 128, dtype=dt, device=DEV)
+        qsa.qsa_pool_keys_prefill(x["k_idx"][b:b + 1, :lens[b]].contiguous(), kp, rope=rope)
+        k_pool[b] = kp[0]
+        nb0 = lens[b] // 4
+        if lens[b] > 4 * nb0:
+            ring[b, :lens[b] - 4 * nb0] = x["k_idx"][b, 4 * nb0: lens[b]]
+    qsa.qsa_pool_keys_decode(x["k_idx_new"], ring, k_pool, x["seq_len"], rope=rope)
+    sel = torch.empty(B, w.top_k, dtype=torch.int32, device=DEV)
+    nsel = torch.empty(B, dtype=torch.int32, device=DEV)
+    qsa.qsa_index_topk_decode(x["q_idx"], k_pool, x["seq_len"], sel, nsel, top_k=w.top_k, rope=rope)
+    out = torch.empty_like(x["q"])
+    qsa.qsa_sparse_attn_decode(x["q"], x["k"], x["v"], x["seq_len"], sel, nsel, out)
+    qsa.qsa_check_status()
+    nbad = 0
+    for b in range(B):
+        s = lens[b] + 1
+        kr = np32(x["k_idx"][b, :lens[b]])
+        kp = np.zeros((cap, 128), np.float32)
+        kp[: lens[b] // 4] = oracle.pool_keys(kr, base=w.rope_base, pos_scale=w.pos_scale)
+        rg = np.zeros((4, 128), np.float32)
+        nb0 = lens[b] // 4
+        rg[: lens[b] - 4 * nb0] = kr[4 * nb0:]
+        oracle.pool_decode(np32(x["k_idx_new"][b]), rg, kp, s, base=w.rope_base, pos_scale=w.pos_scale)
+        assert np.array_equal(np32(k_pool[b]), kp), f"pooled keys differ (seq {b})"
+        ref = oracle.decode(np32(x["q_idx"][b:b + 1]), kp[None], [s], q=np32(x["q"][b:b + 1]),
+                            k=np32(x["k"][b:b + 1]), v=np32(x["v"][b:b + 1]), top_k=w.top_k,
+                            base=w.rope_base, pos_scale=w.pos_scale)
+        assert int(nsel[b]) == ref["nsel"][0]
+        g_sel = sel[b].cpu().numpy()
+        if not np.array_equal(g_sel, ref["sel"][0]):
+            gap = (ref["kth"][0] - ref["next"][0]) / max(abs(ref["kth"][0]), 1e-30)
+            assert gap < 1e-4, f"seq {b}: selection differs with gap {gap}"
+            nbad += 1
+            continue
+        err = np.abs(np32(out[b]) - ref["out"][0]).max()
+        assert err <= TOL["bf16"], (b, err)
+    assert nbad <= max(1, B // 16)
+    del x
+    _free()
+
+
+def test_decode_128k_b64(qsa):
+    _decode_check(qsa, workloads.WORKLOADS["decode_b64_l128k"])
+
+
+def test_decode_128k_ragged_tails(qsa):
+    _decode_check(qsa, workloads.WORKLOADS["decode_b64_l128k"], B=8, ragged=True)
+
+
+def test_decode_1m_b8_scaled_positions(qsa):
+    _decode_check(qsa, workloads.WORKLOADS["decode_b8_l1m_scale4"])

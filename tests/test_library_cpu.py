@@ -1,0 +1,87 @@
+"""Host-side checks of the C-ABI library that need no GPU: it builds, loads,
+exports every entry point include/qsa.h declares, and rejects invalid
+arguments before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qsa.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"^QSA_API\s+[\w\s\*]+?\b(qsa_\w+)\s*\(", src, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def qsa():
+    import __graft_entry__
+    __graft_entry__._load_build_module().build()
+    import block_sparse_attention_11_b200 as m
+    return m
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ["qsa_pool_keys_prefill", "qsa_pool_keys_decode", "qsa_index_topk_prefill", "qsa_index_topk_decode",
+              "qsa_sparse_attn_prefill", "qsa_sparse_attn_decode", "qsa_check_status", "qsa_rope_apply"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(qsa):
+    lib = ctypes.CDLL(qsa.LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, f"not exported: {missing}"
+
+
+def test_strerror_and_version(qsa):
+    assert qsa.qsa_strerror(0) == "ok"
+    assert "invalid" in qsa.qsa_strerror(1)
+    assert qsa.qsa_strerror(99) == "unknown status"
+    assert qsa.qsa_version() >= 100
+
+
+def test_invalid_arguments_are_rejected_before_launch(qsa):
+    lib = qsa.lib
+    rope = qsa.Rope().c()
+    # null pointers
+    assert lib.qsa_pool_keys_prefill(None, None, 1, 16, 0, 16, 4, rope, 0, 0, None) == qsa.QSA_ERR_INVALID_ARG
+    assert lib.qsa_pool_keys_prefill(None, None, 1, 3, 0, 3, 0, rope, 0, 0, None) == qsa.QSA_OK   # nothing to pool
+    # pos0 not a multiple of 4 (checked before any pointer is touched)
+    fake = ctypes.c_void_p(4096)
+    assert lib.qsa_pool_keys_prefill(fake, fake, 1, 16, 2, 16, 8, rope, 0, 0, None) == qsa.QSA_ERR_INVALID_ARG
+    # pooled cache too small
+    assert lib.qsa_pool_keys_prefill(fake, fake, 1, 16, 0, 16, 3, rope, 0, 0, None) == qsa.QSA_ERR_INVALID_ARG
+    # unknown flag bits
+    assert lib.qsa_pool_keys_prefill(fake, fake, 1, 16, 0, 16, 4, rope, 8, 0, None) == qsa.QSA_ERR_INVALID_ARG
+    # unsupported dtype
+    assert lib.qsa_pool_keys_prefill(fake, fake, 1, 16, 0, 16, 4, rope, 0, 7, None) == qsa.QSA_ERR_UNSUPPORTED
+    # rope: unsupported style, bad rotary_dim
+    bad_style = qsa.Rope(style=1).c()
+    assert lib.qsa_pool_keys_prefill(fake, fake, 1, 16, 0, 16, 4, bad_style, 0, 0, None) == qsa.QSA_ERR_UNSUPPORTED
+    bad_dim = qsa.Rope(rotary_dim=20).c()
+    assert lib.qsa_pool_keys_prefill(fake, fake, 1, 16, 0, 16, 4, bad_dim, 0, 0, None) == qsa.QSA_ERR_INVALID_ARG
+    # top_k out of range
+    assert lib.qsa_index_topk_prefill(fake, fake, None, 1, 16, 0, 4, 0, fake, fake, fake, 1 << 20, rope, 0, 0,
+                                      None) == qsa.QSA_ERR_INVALID_ARG
+    # attention: bf16 needs GQA ratio 8, d = 128
+    assert lib.qsa_sparse_attn_prefill(fake, fake, fake, fake, fake, 1, 4, 0, 4, 16, 4, 128, 8, 0.1, fake, None,
+                                       None, 0, 0, None) == qsa.QSA_ERR_UNSUPPORTED
+    assert lib.qsa_sparse_attn_prefill(fake, fake, fake, fake, fake, 1, 4, 0, 4, 16, 2, 64, 8, 0.1, fake, None,
+                                       None, 0, 0, None) == qsa.QSA_ERR_UNSUPPORTED
+    # kv cache shorter than the queries
+    assert lib.qsa_sparse_attn_prefill(fake, fake, fake, fake, fake, 1, 8, 0, 4, 16, 2, 128, 8, 0.1, fake, None,
+                                       None, 0, 0, None) == qsa.QSA_ERR_INVALID_ARG
+    # misaligned pointer
+    odd = ctypes.c_void_p(4098)
+    assert lib.qsa_pool_keys_prefill(odd, fake, 1, 16, 0, 16, 4, rope, 0, 0, None) == qsa.QSA_ERR_INVALID_ARG
+
+
+def test_binding_rejects_host_tensors(qsa):
+    import torch
+    x = torch.zeros(1, 8, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        qsa.qsa_pool_keys_prefill(x, torch.zeros(1, 2, 128, dtype=torch.bfloat16))

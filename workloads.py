@@ -179,7 +179,7 @@ def make_decode(w: Workload, device="cuda", L: int | None = None, B: int | None 
     B = B or w.B
     g = _gen(device, w.seed)
     dt = torch_dtype(w)
-    lens = [L - (i % 4 if ragged else 0) for i in range(B)]
+    lens = [max(0, L - (i % 4 if ragged else 0)) for i in range(B)]
     Lmax = max(lens)
     k_idx = _randn((B, Lmax, IDX_DIM), g, device, dt)
     q_idx = _randn((B, IDX_HEADS, IDX_DIM), g, device, dt)
