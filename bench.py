@@ -410,6 +410,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=None, help="override B (smaller profiling case)")
+    ap.add_argument("--tokens", type=int, default=None, help="override T / cache length (smaller profiling case)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -419,6 +421,11 @@ def main():
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     w = workloads.WORKLOADS[args.workload]
+    if args.batch or args.tokens:
+        import dataclasses
+        w = dataclasses.replace(w, B=args.batch or w.B, T=args.tokens or w.T, name=w.name + "_profile_case")
+        workloads.WORKLOADS[w.name] = w
+        args.workload = w.name
 
     if args.impl == "reference":
         if rank == 0:
