@@ -19,8 +19,10 @@
 //     M and the 8 q heads of one kv head as N (no padding waste for GQA 8),
 //     an fp32 online softmax per head column, P^T re-laid out in registers
 //     with movmatrix, and O^T += V^T P;
-//   * two warps per kv head split each stage's 32 keys (tokens {0,1} and
-//     {2,3} of the 8 blocks) and merge their softmax states at the end.
+//   * two warps per kv head take alternate stages (both 16-key tiles of a
+//     stage each) and merge their softmax states at the end of an item;
+//   * the producer stages each item's block ids in shared memory once, so
+//     no global read sits on the per-stage issue path.
 // A persistent grid walks the work items; the pipeline runs across item
 // boundaries.  Decode splits each sequence's key list over several items
 // (split-KV) and a small kernel combines the partial results.
@@ -37,15 +39,36 @@ namespace {
 constexpr int AT_BPS = 8;               // blocks per stage
 constexpr float kLog2e = 1.4426950408889634f;
 
+// Tuning knobs (compile time).  Defaults measured best on B200 for the
+// 32K-token prefill: 2 resident CTAs per SM, 2 stages in flight per CTA,
+// 4 producer warps per CTA.
+#ifndef QSA_ATTN_CTAS
+#define QSA_ATTN_CTAS 2           // resident CTAs per SM
+#endif
+#ifndef QSA_ATTN_PW
+#define QSA_ATTN_PW 4             // producer warps per CTA (each owns every PW-th slot of a stage)
+#endif
+#ifndef QSA_ATTN_NS
+#define QSA_ATTN_NS 2             // stages in flight per CTA
+#endif
+
 template <int HKV> struct AttnCfg {
-    static constexpr int kConsumers = 2 * HKV;
-    static constexpr int kThreads = (kConsumers + 1) * 32;
+    static constexpr int kWph = 2;   // consumer warps per kv head: even / odd stages
+    static constexpr int kConsumers = kWph * HKV;
+    static constexpr int kPw = QSA_ATTN_PW;
+    static constexpr int kThreads = (kConsumers + kPw) * 32;
     static constexpr int kSpan = kBlock * HKV * 128 * 2;      // bytes of one block, all kv heads
     static constexpr int kSlot = kSpan + 16;                   // padded slot
     static constexpr int kStage = 2 * AT_BPS * kSlot;          // K slots then V slots
     static constexpr int kHq = 8 * HKV;
     static constexpr int kQBytes = kHq * 128 * 2;
-    static constexpr int kNS = HKV >= 4 ? 2 : 4;               // stages in flight (smem bound)
+    static constexpr int kNS = QSA_ATTN_NS;
+    // Consumer warp hf takes the stages whose global index is = hf (mod 2); with
+    // an even number of slots it always uses the same slots, in order, so no
+    // mbarrier is ever waited on more than one phase ahead (try_wait.parity
+    // only tells the current phase from the previous one).
+    static_assert(kNS >= 2 && kNS % 2 == 0, "stages in flight must be even");
+    static_assert(AT_BPS % QSA_ATTN_PW == 0, "producer warps must divide the blocks per stage");
 };
 
 struct AttnParams {
@@ -122,15 +145,18 @@ struct __align__(128) AttnSmem {
     using Cfg = AttnCfg<HKV>;
     uint8_t stage[Cfg::kNS][AttnCfg<HKV>::kStage];
     alignas(16) uint8_t qbuf[2][AttnCfg<HKV>::kQBytes];
-    float xbuf[HKV][32][36];
+    float xbuf[HKV][AttnCfg<HKV>::kWph - 1][32][36];
     alignas(16) __nv_bfloat16 obuf[HKV][8][128];
-    uint32_t info[Cfg::kNS];
+    int32_t sel_s[2048];                 // the current item's block ids (each producer fills its own slots)
+    uint32_t st_info[Cfg::kPw][264];     // per stage of the item: token counts of the producer's slots
+    uint32_t st_bytes[Cfg::kPw][264];    // per stage of the item: bytes the producer copies per tensor
+    uint32_t info[Cfg::kNS][Cfg::kPw];
     uint64_t full[Cfg::kNS], empty[Cfg::kNS], qfull[2], qempty[2];
     uint64_t xready[HKV], xdone[HKV];   // pair merge handshake per kv head
 };
 
 template <int HKV>
-__global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, 1) attn_bf16_kernel(AttnParams p) {
+__global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, QSA_ATTN_CTAS) attn_bf16_kernel(AttnParams p) {
     using Cfg = AttnCfg<HKV>;
     extern __shared__ uint8_t asm_raw[];
     AttnSmem<HKV> &sm = *reinterpret_cast<AttnSmem<HKV> *>((reinterpret_cast<uintptr_t>(asm_raw) + 127) & ~uintptr_t(127));
@@ -140,65 +166,87 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, 1) attn_bf16_kernel(At
     for (int i = threadIdx.x; i < (int)(sizeof(sm.stage) / 16); i += blockDim.x)
         reinterpret_cast<uint4 *>(&sm.stage[0][0])[i] = make_uint4(0, 0, 0, 0);
     if (threadIdx.x == 0) {
-        for (int s = 0; s < Cfg::kNS; ++s) { mbar_init(&sm.full[s], 1); mbar_init(&sm.empty[s], Cfg::kConsumers); }
+        for (int s = 0; s < Cfg::kNS; ++s) { mbar_init(&sm.full[s], Cfg::kPw); mbar_init(&sm.empty[s], HKV); }
         for (int s = 0; s < 2; ++s) { mbar_init(&sm.qfull[s], 1); mbar_init(&sm.qempty[s], Cfg::kConsumers); }
-        for (int s = 0; s < HKV; ++s) { mbar_init(&sm.xready[s], 1); mbar_init(&sm.xdone[s], 1); }
+        for (int s = 0; s < HKV; ++s) { mbar_init(&sm.xready[s], Cfg::kWph - 1); mbar_init(&sm.xdone[s], 1); }
         fence_mbar_init();
     }
     fence_proxy_async_smem();
     __syncthreads();
 
-    if (warp == Cfg::kConsumers) {
-        // ------------------------------------------------------------ producer
+    if (warp >= Cfg::kConsumers) {
+        // ------------------------------------------------------------ producers
+        // Producer pw owns slots j = pw, pw + PW, ... of every stage.  Per item it
+        // copies the block ids to shared memory and precomputes, per stage, the
+        // token counts and byte totals of its slots, so the per-stage issue path
+        // is: wait for the slot, one expect_tx, one bulk copy per block and tensor.
+        constexpr int kSlotsPerPw = AT_BPS / Cfg::kPw;
+        const int pw = warp - Cfg::kConsumers;
+        int32_t *ids = sm.sel_s;
         int64_t it_count = 0;   // stage counter across items
         int64_t ic = 0;         // item counter
         bool ok = true;
         for (int64_t i = blockIdx.x; i < p.items && ok; i += gridDim.x, ++ic) {
             const Item it = get_item<HKV>(p, i);
+            const int id_end = min(it.lend, it.nsel);
+            // list entries of this producer's slots: e - lbeg = 8 * st + PW * jj + pw
+            for (int r = lane; r * Cfg::kPw < id_end - it.lbeg; r += 32) {
+                const int rel = (r / kSlotsPerPw) * AT_BPS + (r % kSlotsPerPw) * Cfg::kPw + pw;
+                if (rel < id_end - it.lbeg) ids[rel] = it.sel[it.lbeg + rel];
+            }
+            __syncwarp();
+            const int nst = (it.lend - it.lbeg + AT_BPS - 1) / AT_BPS;
+            for (int st = lane; st < nst; st += 32) {
+                uint32_t info = 0, bytes = 0;
+#pragma unroll
+                for (int jj = 0; jj < kSlotsPerPw; ++jj) {
+                    const int j = Cfg::kPw * jj + pw;
+                    const int e = it.lbeg + AT_BPS * st + j;
+                    int tokens = 0;
+                    if (e < it.lend) {
+                        if (e < it.nsel) {
+                            const int b = ids[e - it.lbeg];
+                            if (b >= 0 && b < it.nb) tokens = kBlock;
+                            else flag(p.status, QSA_DEV_BAD_INDEX);
+                        } else {
+                            tokens = it.tail;
+                        }
+                    }
+                    info |= (uint32_t)tokens << (3 * j);
+                    bytes += (uint32_t)tokens * HKV * 256u;
+                }
+                sm.st_info[pw][st] = info;
+                sm.st_bytes[pw][st] = bytes;
+            }
             const int qs = (int)(ic & 1);
-            if (ic >= 2) ok = mbar_wait(&sm.qempty[qs], (int)(((ic >> 1) + 1) & 1), p.status);
+            if (pw == 0 && ic >= 2) ok = mbar_wait(&sm.qempty[qs], (int)(((ic >> 1) + 1) & 1), p.status);
+            __syncwarp();
             if (!ok) break;
-            if (lane == 0) {
+            if (pw == 0 && lane == 0) {
                 mbar_arrive_expect_tx(&sm.qfull[qs], Cfg::kQBytes);
                 bulk_g2s(sm.qbuf[qs], it.qrow, Cfg::kQBytes, &sm.qfull[qs]);
             }
             const int64_t kv0 = (int64_t)it.seq * p.kv_stride;
-            for (int pos = it.lbeg; pos < it.lend && ok; pos += AT_BPS, ++it_count) {
+            for (int st = 0; st < nst && ok; ++st, ++it_count) {
                 const int s = (int)(it_count % Cfg::kNS);
                 if (it_count >= Cfg::kNS) ok = mbar_wait(&sm.empty[s], (int)(((it_count / Cfg::kNS) + 1) & 1), p.status);
                 if (!ok) break;
-                // lane j < 8 handles list entry pos + j
-                int tokens = 0;
-                int64_t blk = 0;
-                const int e = pos + lane;
-                if (lane < AT_BPS && e < it.lend) {
-                    if (e < it.nsel) {
-                        blk = it.sel[e];
-                        if (blk >= 0 && blk < it.nb) tokens = kBlock;
-                        else flag(p.status, QSA_DEV_BAD_INDEX);
-                    } else {
-                        blk = it.nb;            // the incomplete tail block
-                        tokens = it.tail;
-                    }
-                }
-                uint32_t bytes = (uint32_t)tokens * HKV * 256u;
-                uint32_t info = (uint32_t)tokens << (3 * (lane & 7));
-                if (lane >= AT_BPS) info = 0;
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    bytes += __shfl_xor_sync(0xffffffffu, bytes, o);
-                    info |= __shfl_xor_sync(0xffffffffu, info, o);
-                }
                 if (lane == 0) {
-                    sm.info[s] = info;
-                    mbar_arrive_expect_tx(&sm.full[s], 2 * bytes);
+                    sm.info[s][pw] = sm.st_info[pw][st];
+                    mbar_arrive_expect_tx(&sm.full[s], 2 * sm.st_bytes[pw][st]);
                 }
                 __syncwarp();
-                if (tokens > 0) {
-                    const int64_t off = (kv0 + blk * kBlock) * HKV * 128;
-                    const uint32_t nbytes = (uint32_t)tokens * HKV * 256u;
-                    bulk_g2s(sm.stage[s] + lane * Cfg::kSlot, p.k + off, nbytes, &sm.full[s]);
-                    bulk_g2s(sm.stage[s] + (AT_BPS + lane) * Cfg::kSlot, p.v + off, nbytes, &sm.full[s]);
+                if (lane < kSlotsPerPw) {
+                    const int j = Cfg::kPw * lane + pw;
+                    const int e = it.lbeg + AT_BPS * st + j;
+                    const int tokens = (int)((sm.st_info[pw][st] >> (3 * j)) & 7u);
+                    if (tokens > 0) {
+                        const int64_t blk = (e < it.nsel) ? (int64_t)ids[e - it.lbeg] : it.nb;
+                        const int64_t off = (kv0 + blk * kBlock) * HKV * 128;
+                        const uint32_t nbytes = (uint32_t)tokens * HKV * 256u;
+                        bulk_g2s(sm.stage[s] + j * Cfg::kSlot, p.k + off, nbytes, &sm.full[s]);
+                        bulk_g2s(sm.stage[s] + (AT_BPS + j) * Cfg::kSlot, p.v + off, nbytes, &sm.full[s]);
+                    }
                 }
             }
         }
@@ -206,21 +254,26 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, 1) attn_bf16_kernel(At
         if (lane == 0) {
             for (int64_t c = (it_count > Cfg::kNS ? it_count - Cfg::kNS : 0); c < it_count; ++c)
                 mbar_wait(&sm.full[c % Cfg::kNS], (int)((c / Cfg::kNS) & 1), p.status);
-            for (int64_t c = (ic > 2 ? ic - 2 : 0); c < ic; ++c) mbar_wait(&sm.qfull[c & 1], (int)((c >> 1) & 1), p.status);
+            if (pw == 0)
+                for (int64_t c = (ic > 2 ? ic - 2 : 0); c < ic; ++c)
+                    mbar_wait(&sm.qfull[c & 1], (int)((c >> 1) & 1), p.status);
         }
         return;
     }
 
     // ---------------------------------------------------------------- consumers
-    const int g = warp >> 1;        // kv head
-    const int hf = warp & 1;        // token pair {2hf, 2hf+1}
+    // warp (g, hf): kv head g; takes the stages whose global index is = hf
+    // (mod 2) and processes both 16-key tiles of each (tile t = tokens {2t, 2t+1} of the
+    // stage's 8 blocks).
+    const int g = warp / Cfg::kWph;
+    const int hf = warp % Cfg::kWph;
     const int gr = lane >> 2, tq = lane & 3;
     const uint32_t stage0 = smem_u32(&sm.stage[0][0]);
-    // ldmatrix row addresses (byte offsets inside a stage)
     const int mi = lane >> 3, rr = lane & 7;
-    const uint32_t k_lane_off = (uint32_t)(rr * Cfg::kSlot + (2 * hf + (mi & 1)) * HKV * 256 + g * 256 + (mi >> 1) * 16);
-    const uint32_t v_lane_off = (uint32_t)(AT_BPS * Cfg::kSlot + rr * Cfg::kSlot + (2 * hf + (mi >> 1)) * HKV * 256 +
+    const uint32_t k_lane_off = (uint32_t)(rr * Cfg::kSlot + (mi & 1) * HKV * 256 + g * 256 + (mi >> 1) * 16);
+    const uint32_t v_lane_off = (uint32_t)(AT_BPS * Cfg::kSlot + rr * Cfg::kSlot + (mi >> 1) * HKV * 256 +
                                            g * 256 + (mi & 1) * 16);
+    constexpr uint32_t kTileOff = 2 * HKV * 256;     // tokens {2,3} vs {0,1}
     int64_t it_count = 0, ic = 0;
     bool ok = true;
     for (int64_t i = blockIdx.x; i < p.items && ok; i += gridDim.x, ++ic) {
@@ -246,30 +299,43 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, 1) attn_bf16_kernel(At
         for (int a = 0; a < 8; ++a) o[a][0] = o[a][1] = o[a][2] = o[a][3] = 0.f;
 
         for (int pos = it.lbeg; pos < it.lend; pos += AT_BPS, ++it_count) {
+            if ((int)(it_count & 1) != hf) continue;
             const int s = (int)(it_count % Cfg::kNS);
             ok = mbar_wait(&sm.full[s], (int)((it_count / Cfg::kNS) & 1), p.status);
             if (!ok) break;
-            const uint32_t info = sm.info[s];
+            uint32_t info = 0;
+#pragma unroll
+            for (int q2 = 0; q2 < Cfg::kPw; ++q2) info |= sm.info[s][q2];
             const uint32_t sbase = stage0 + (uint32_t)s * Cfg::kStage;
-            // S^T (16 keys x 8 heads)
-            float sacc[4] = {0.f, 0.f, 0.f, 0.f}, sacc2[4] = {0.f, 0.f, 0.f, 0.f};
+            // S^T for both tiles (16 keys x 8 heads each), two accumulators per tile
+            float sa[2][4], sb[2][4];
+#pragma unroll
+            for (int t = 0; t < 2; ++t)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) sa[t][c] = sb[t][c] = 0.f;
 #pragma unroll
             for (int kk = 0; kk < 8; kk += 2) {
-                uint32_t a0, a1, a2, a3, c0, c1, c2, c3;
-                ldsm_x4(sbase + k_lane_off + kk * 32, a0, a1, a2, a3);
-                ldsm_x4(sbase + k_lane_off + (kk + 1) * 32, c0, c1, c2, c3);
-                mma16816(sacc, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
-                mma16816(sacc2, c0, c1, c2, c3, qf[kk + 1][0], qf[kk + 1][1]);
-            }
 #pragma unroll
-            for (int c = 0; c < 4; ++c) sacc[c] += sacc2[c];
+                for (int t = 0; t < 2; ++t) {
+                    uint32_t a0, a1, a2, a3, c0, c1, c2, c3;
+                    ldsm_x4(sbase + k_lane_off + t * kTileOff + kk * 32, a0, a1, a2, a3);
+                    ldsm_x4(sbase + k_lane_off + t * kTileOff + (kk + 1) * 32, c0, c1, c2, c3);
+                    mma16816(sa[t], a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
+                    mma16816(sb[t], c0, c1, c2, c3, qf[kk + 1][0], qf[kk + 1][1]);
+                }
+            }
             const int ntok = (int)((info >> (3 * gr)) & 7u);
-            const bool v0 = ntok > 2 * hf, v1 = ntok > 2 * hf + 1;
-            float x0 = v0 ? sacc[0] * p.scale_log2 : -INFINITY;   // key (slot gr, tok 2hf),   head 2tq
-            float x1 = v0 ? sacc[1] * p.scale_log2 : -INFINITY;   //                           head 2tq+1
-            float x2 = v1 ? sacc[2] * p.scale_log2 : -INFINITY;   // key (slot gr, tok 2hf+1), head 2tq
-            float x3 = v1 ? sacc[3] * p.scale_log2 : -INFINITY;
-            float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+            float x[2][4];
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                const bool v0 = ntok > 2 * t, v1 = ntok > 2 * t + 1;
+                x[t][0] = v0 ? (sa[t][0] + sb[t][0]) * p.scale_log2 : -INFINITY;   // (slot gr, tok 2t),   head 2tq
+                x[t][1] = v0 ? (sa[t][1] + sb[t][1]) * p.scale_log2 : -INFINITY;   //                      head 2tq+1
+                x[t][2] = v1 ? (sa[t][2] + sb[t][2]) * p.scale_log2 : -INFINITY;   // (slot gr, tok 2t+1), head 2tq
+                x[t][3] = v1 ? (sa[t][3] + sb[t][3]) * p.scale_log2 : -INFINITY;
+            }
+            float mx0 = fmaxf(fmaxf(x[0][0], x[0][2]), fmaxf(x[1][0], x[1][2]));
+            float mx1 = fmaxf(fmaxf(x[0][1], x[0][3]), fmaxf(x[1][1], x[1][3]));
 #pragma unroll
             for (int o2 = 4; o2 < 32; o2 <<= 1) {
                 mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o2));
@@ -280,20 +346,31 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, 1) attn_bf16_kernel(At
             const float al0 = exp2f(mrow[0] - mu0), al1 = exp2f(mrow[1] - mu1);
             mrow[0] = mn0;
             mrow[1] = mn1;
-            const float p0 = exp2f(x0 - mu0), p1 = exp2f(x1 - mu1), p2 = exp2f(x2 - mu0), p3 = exp2f(x3 - mu1);
-            lrow[0] = lrow[0] * al0 + p0 + p2;
-            lrow[1] = lrow[1] * al1 + p1 + p3;
-            const uint32_t b0 = movm_t(pack_bf16(p0, p1));
-            const uint32_t b1 = movm_t(pack_bf16(p2, p3));
+            uint32_t pb[2][2];
+            float ls0 = 0.f, ls1 = 0.f;
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                const float p0 = exp2f(x[t][0] - mu0), p1 = exp2f(x[t][1] - mu1);
+                const float p2 = exp2f(x[t][2] - mu0), p3 = exp2f(x[t][3] - mu1);
+                ls0 += p0 + p2;
+                ls1 += p1 + p3;
+                pb[t][0] = movm_t(pack_bf16(p0, p1));
+                pb[t][1] = movm_t(pack_bf16(p2, p3));
+            }
+            lrow[0] = lrow[0] * al0 + ls0;
+            lrow[1] = lrow[1] * al1 + ls1;
 #pragma unroll
             for (int mt = 0; mt < 8; ++mt) {
                 o[mt][0] *= al0;
                 o[mt][1] *= al1;
                 o[mt][2] *= al0;
                 o[mt][3] *= al1;
-                uint32_t a0, a1, a2, a3;
-                ldsm_x4_t(sbase + v_lane_off + mt * 32, a0, a1, a2, a3);
-                mma16816(o[mt], a0, a1, a2, a3, b0, b1);
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    uint32_t a0, a1, a2, a3;
+                    ldsm_x4_t(sbase + v_lane_off + t * kTileOff + mt * 32, a0, a1, a2, a3);
+                    mma16816(o[mt], a0, a1, a2, a3, pb[t][0], pb[t][1]);
+                }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.empty[s]);
@@ -305,11 +382,11 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, 1) attn_bf16_kernel(At
             lrow[0] += __shfl_xor_sync(0xffffffffu, lrow[0], o2);
             lrow[1] += __shfl_xor_sync(0xffffffffu, lrow[1], o2);
         }
-        // merge the two warps of this kv head
-        float *xb = sm.xbuf[g][lane];
-        if (hf == 1) {
+        // merge the warps of this kv head: warps hf >= 1 publish, warp 0 folds
+        if (hf != 0) {
             if (ic > 0) ok = mbar_wait(&sm.xdone[g], (int)((ic - 1) & 1), p.status);
             if (!ok) break;
+            float *xb = sm.xbuf[g][hf - 1][lane];
             xb[0] = mrow[0]; xb[1] = mrow[1]; xb[2] = lrow[0]; xb[3] = lrow[1];
 #pragma unroll
             for (int mt = 0; mt < 8; ++mt)
@@ -320,24 +397,35 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, 1) attn_bf16_kernel(At
         } else {
             ok = mbar_wait(&sm.xready[g], (int)(ic & 1), p.status);
             if (!ok) break;
-            float f0[2], f1[2], l[2], m[2];
+            {
+                // fold the other warp's state: symmetric in the two operands
+                // (explicitly rounded, no contraction), so the result does not
+                // depend on which warp took the even or the odd stages
+                const float *xb = sm.xbuf[g][0][lane];
+                float f0[2], f1[2];
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                const float mo = xb[c], lo = xb[2 + c];
-                m[c] = fmaxf(mrow[c], mo);
-                const float mu = (m[c] == -INFINITY) ? 0.f : m[c];
-                f0[c] = exp2f(mrow[c] - mu);
-                f1[c] = exp2f(mo - mu);
-                l[c] = lrow[c] * f0[c] + lo * f1[c];
+                for (int c = 0; c < 2; ++c) {
+                    const float mo = xb[c], lo = xb[2 + c];
+                    const float mn = fmaxf(mrow[c], mo);
+                    const float mu = (mn == -INFINITY) ? 0.f : mn;
+                    f0[c] = exp2f(mrow[c] - mu);
+                    f1[c] = exp2f(mo - mu);
+                    lrow[c] = __fadd_rn(__fmul_rn(lrow[c], f0[c]), __fmul_rn(lo, f1[c]));
+                    mrow[c] = mn;
+                }
+#pragma unroll
+                for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        o[mt][c] = __fadd_rn(__fmul_rn(o[mt][c], f0[c & 1]), __fmul_rn(xb[4 + 4 * mt + c], f1[c & 1]));
             }
+            const float l[2] = {lrow[0], lrow[1]}, m[2] = {mrow[0], mrow[1]};
             const float inv0 = l[0] > 0.f ? 1.f / l[0] : 0.f, inv1 = l[1] > 0.f ? 1.f / l[1] : 0.f;
             if (!p.decode) {
 #pragma unroll
                 for (int mt = 0; mt < 8; ++mt) {
-                    const float r0 = (o[mt][0] * f0[0] + xb[4 + 4 * mt + 0] * f1[0]) * inv0;
-                    const float r1 = (o[mt][1] * f0[1] + xb[4 + 4 * mt + 1] * f1[1]) * inv1;
-                    const float r2 = (o[mt][2] * f0[0] + xb[4 + 4 * mt + 2] * f1[0]) * inv0;
-                    const float r3 = (o[mt][3] * f0[1] + xb[4 + 4 * mt + 3] * f1[1]) * inv1;
+                    const float r0 = o[mt][0] * inv0, r1 = o[mt][1] * inv1;
+                    const float r2 = o[mt][2] * inv0, r3 = o[mt][3] * inv1;
                     sm.obuf[g][2 * tq][16 * mt + gr] = __float2bfloat16_rn(r0);
                     sm.obuf[g][2 * tq + 1][16 * mt + gr] = __float2bfloat16_rn(r1);
                     sm.obuf[g][2 * tq][16 * mt + gr + 8] = __float2bfloat16_rn(r2);
@@ -362,10 +450,10 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, 1) attn_bf16_kernel(At
                 float *po = p.part_o + (pi * Cfg::kHq + 8 * g) * 128;
 #pragma unroll
                 for (int mt = 0; mt < 8; ++mt) {
-                    po[(2 * tq) * 128 + 16 * mt + gr] = (o[mt][0] * f0[0] + xb[4 + 4 * mt + 0] * f1[0]) * inv0;
-                    po[(2 * tq + 1) * 128 + 16 * mt + gr] = (o[mt][1] * f0[1] + xb[4 + 4 * mt + 1] * f1[1]) * inv1;
-                    po[(2 * tq) * 128 + 16 * mt + gr + 8] = (o[mt][2] * f0[0] + xb[4 + 4 * mt + 2] * f1[0]) * inv0;
-                    po[(2 * tq + 1) * 128 + 16 * mt + gr + 8] = (o[mt][3] * f0[1] + xb[4 + 4 * mt + 3] * f1[1]) * inv1;
+                    po[(2 * tq) * 128 + 16 * mt + gr] = o[mt][0] * inv0;
+                    po[(2 * tq + 1) * 128 + 16 * mt + gr] = o[mt][1] * inv1;
+                    po[(2 * tq) * 128 + 16 * mt + gr + 8] = o[mt][2] * inv0;
+                    po[(2 * tq + 1) * 128 + 16 * mt + gr + 8] = o[mt][3] * inv1;
                 }
                 if (gr == 0) {
 #pragma unroll
@@ -379,22 +467,38 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, 1) attn_bf16_kernel(At
     }
 }
 
-// Decode combine: one CTA of 128 threads per (sequence, q head).
-__global__ void attn_combine_kernel(const float *__restrict__ part_o, const float *__restrict__ part_lse, int splits,
-                                    int Hq, __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
+// Decode combine: one CTA of 128 threads per (sequence, q head).  The split
+// lse values are read in parallel, then every dim sums its weighted partials.
+__global__ void __launch_bounds__(128) attn_combine_kernel(const float *__restrict__ part_o,
+                                                           const float *__restrict__ part_lse, int splits, int Hq,
+                                                           __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
+    __shared__ float wsm[1024];
+    __shared__ float red[4];
     const int seq = blockIdx.x / Hq, h = blockIdx.x % Hq, e = threadIdx.x;
     float mx = -INFINITY;
-    for (int s = 0; s < splits; ++s) mx = fmaxf(mx, part_lse[((int64_t)seq * splits + s) * Hq + h]);
-    float acc = 0.f, den = 0.f;
-    if (mx != -INFINITY) {
-        for (int s = 0; s < splits; ++s) {
-            const float ls = part_lse[((int64_t)seq * splits + s) * Hq + h];
-            if (ls == -INFINITY) continue;
-            const float w = exp2f(ls - mx);
-            den += w;
-            acc += w * part_o[(((int64_t)seq * splits + s) * Hq + h) * 128 + e];
-        }
+    for (int s = e; s < splits; s += 128) {
+        const float v = part_lse[((int64_t)seq * splits + s) * Hq + h];
+        wsm[s] = v;
+        mx = fmaxf(mx, v);
     }
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if ((e & 31) == 0) red[e >> 5] = mx;
+    __syncthreads();
+    mx = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    __syncthreads();
+    float den = 0.f;
+    for (int s = e; s < splits; s += 128) {
+        const float w = (mx == -INFINITY || wsm[s] == -INFINITY) ? 0.f : exp2f(wsm[s] - mx);
+        wsm[s] = w;
+        den += w;
+    }
+    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    if ((e & 31) == 0) red[e >> 5] = den;
+    __syncthreads();
+    den = red[0] + red[1] + red[2] + red[3];
+    float acc = 0.f;
+    const float *po = part_o + ((int64_t)seq * splits * Hq + h) * 128 + e;
+    for (int s = 0; s < splits; ++s) acc += wsm[s] * po[(int64_t)s * Hq * 128];
     out[((int64_t)seq * Hq + h) * 128 + e] = __float2bfloat16_rn(den > 0.f ? acc / den : 0.f);
     if (lse && e == 0) lse[(int64_t)seq * Hq + h] = den > 0.f ? (mx + log2f(den)) / kLog2e : -INFINITY;
 }
@@ -512,7 +616,7 @@ cudaError_t run_bf16(const AttnArgs &a, void *ws, unsigned *status, cudaStream_t
     const size_t smem = sizeof(AttnSmem<HKV>) + 128;
     cudaError_t e = cudaFuncSetAttribute(attn_bf16_kernel<HKV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    const int64_t grid = std::min<int64_t>(p.items, (int64_t)sms);
+    const int64_t grid = std::min<int64_t>(p.items, (int64_t)sms * QSA_ATTN_CTAS);
     attn_bf16_kernel<HKV><<<(unsigned)grid, Cfg::kThreads, smem, s>>>(p);
     e = cudaGetLastError();
     if (e != cudaSuccess || !a.decode) return e;

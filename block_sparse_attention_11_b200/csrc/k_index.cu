@@ -50,6 +50,7 @@ struct GemmSmem {
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
     uint32_t tmem_base;
+    alignas(16) float epi[4][32][36];   // per epilogue warp: 32 rows x 32 scores, transposed for stores
 };
 
 struct GemmParams {
@@ -162,7 +163,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         const bool row_live = qrow < r_end;
         float w = 1.0f;
         if (p.per_head && p.head_w && row_live) w = p.head_w[(seq * p.n_q + qrow) * kIdxHeads + head];
-        float *dst = p.scores + ((int64_t)seq * p.row_count + (qrow - p.row_begin)) * p.ld;
         for (int j = 0; j < ntiles; ++j) {
             const int ab = j & 1;
             if (!mbar_wait(&sm.acc_full[ab], (j >> 1) & 1, p.status)) break;
@@ -186,12 +186,26 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                         v[i] = x;
                     }
                 }
-                const bool writer = row_live && (!p.per_head || head == 0);
-                if (writer) {
-                    float4 *o = reinterpret_cast<float4 *>(dst + (int64_t)j * GN + c * 32);
+                // stage the 32 x 32 block in smem and store it row-contiguously
+                float(*tile)[36] = sm.epi[quarter];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) o[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                for (int i = 0; i < 8; ++i)
+                    *reinterpret_cast<float4 *>(&tile[lane][4 * i]) = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2],
+                                                                                 v[4 * i + 3]);
+                __syncwarp();
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int rr = 4 * i + (lane >> 3);
+                    const int lr = quarter * 32 + rr;
+                    const int64_t q = p.per_head ? r0 + lr / kIdxHeads : r0 + lr;
+                    const bool writer = q < r_end && (!p.per_head || (lr % kIdxHeads) == 0);
+                    if (writer) {
+                        float *d = p.scores + ((int64_t)seq * p.row_count + (q - p.row_begin)) * p.ld + (int64_t)j * GN +
+                                   c * 32 + 4 * (lane & 7);
+                        *reinterpret_cast<float4 *>(d) = *reinterpret_cast<const float4 *>(&tile[rr][4 * (lane & 7)]);
+                    }
                 }
+                __syncwarp();
             }
             tc_fence_before();
             __syncwarp();
@@ -246,7 +260,27 @@ __global__ void __launch_bounds__(512) select_rows_kernel(const float *__restric
     const int64_t t = q0 + row;
     const int n = (int)((t + 1) / kBlock);
     const float *src = scores + ((int64_t)seq * row_count + rloc) * ld;
-    for (int i = threadIdx.x; i < n; i += blockDim.x) keys[i] = score_key(src[i]);
+    // 16-byte loads, four in flight per thread (rows are 16-byte aligned: ld % 128 == 0)
+    const int n4 = (n + 3) >> 2;
+    const float4 *src4 = reinterpret_cast<const float4 *>(src);
+    for (int base = threadIdx.x; base < n4; base += 4 * blockDim.x) {
+        float4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i4 = base + u * blockDim.x;
+            if (i4 < n4) v[u] = src4[i4];
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i4 = base + u * blockDim.x;
+            if (i4 < n4) {
+                const float f[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    if (4 * i4 + c < n) keys[4 * i4 + c] = score_key(f[c]);
+            }
+        }
+    }
     __syncthreads();
     int32_t *out = sel + ((int64_t)seq * n_q + row) * top_k;
     const int cnt = cta_topk(keys, n, top_k, sm, [&](int pos, int i) { out[pos] = i; });

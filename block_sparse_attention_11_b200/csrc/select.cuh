@@ -1,75 +1,139 @@
 // select.cuh -- CTA-wide exact top-k over keys held in shared memory.
 //
 // The ranking is "higher score first, equal scores to the lower block id".
-// Scores are mapped to order-preserving uint32 keys (score_key), so the k-th
-// largest key K* is found with an MSB-first radix select (four 8-bit
-// digits), and the selection is
-//     { i : key_i > K* }  U  { the first (k - #{key > K*}) positions with key == K* },
-// emitted in ascending position order by an ordered stream compaction (warp
-// ballots + a CTA prefix).  Because positions are scanned in increasing
-// order, the output is sorted ascending, which is the layout the sparse
-// attention consumes.
+// Scores are mapped to order-preserving uint32 keys (score_key).  The k-th
+// largest key K* is found by an MSB-first radix select:
+//   1. an 11-bit histogram of the top digit (warp-aggregated atomics: equal
+//      digits within a warp are merged with match_any, since scores pile up in
+//      a few exponent bins);
+//   2. the keys of the bin holding K* are gathered into a small candidate
+//      list and the remaining 21 bits are resolved on that list only (two
+//      more digits); if the bin is too large for the list, the two digits are
+//      resolved on the full key array instead;
+// and the selection
+//     { i : key_i > K* }  U  { the first (k - #{key > K*}) positions with key == K* }
+// is emitted in ascending position order by a two-phase ordered compaction:
+// each warp owns a contiguous range, counts its "greater" and "equal" keys,
+// and after one exclusive prefix over warps writes its survivors with ballot
+// prefix sums.  Ascending output is the layout the sparse attention consumes.
 #pragma once
 
 #include "common.cuh"
 
 namespace qsa {
 
-// Shared scratch of one select (lives in static smem of the calling kernel).
+constexpr int kSelCandCap = 1024;
+
 struct SelectSmem {
-    uint32_t hist[256];
-    uint32_t warp_a[32];
-    uint32_t warp_b[32];
-    uint32_t kstar;
-    int32_t take_eq;
-    int32_t run_out;
-    int32_t run_eq;
+    uint32_t hist[2048];
+    uint32_t cand[kSelCandCap];
+    uint32_t warp_gt[32];
+    uint32_t warp_eq[32];
+    uint32_t kstar;      // K*
+    int32_t take_eq;     // how many keys equal to K* are taken (in position order)
+    int32_t ncand;
+    int32_t digit;
+    int32_t k_rem;
+    int32_t total;
 };
 
-// Finds K* and the number of keys equal to K* that are taken (k < n).
-// Requires every thread of the CTA.  `nt` = blockDim.x (multiple of 32).
+// All threads scan hist[0..nbins) from the top and record the digit whose
+// bin holds the k_rem-th largest key and the rank left inside that bin.
+// Thread t owns bins [per*t, per*t + per); a suffix scan over threads (warp
+// shuffles, then over warps) gives every thread the count above its range.
+// Ends with a barrier; sm.digit / sm.k_rem are then valid for all threads.
+__device__ __forceinline__ void sel_find_digit(SelectSmem &sm, int nbins, int k_rem) {
+    const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, warp = tid >> 5, nwarps = nt >> 5;
+    const int per = nbins / nt;   // nbins and nt are powers of two, nbins >= nt
+    uint32_t mine = 0;
+    for (int b = 0; b < per; ++b) mine += sm.hist[per * tid + b];
+    uint32_t incl = mine;   // inclusive suffix within the warp (towards higher lanes)
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_down_sync(0xffffffffu, incl, o);
+        if (lane + o < 32) incl += v;
+    }
+    if (lane == 0) sm.warp_eq[warp] = incl;   // warp total
+    __syncthreads();
+    uint32_t cum = incl - mine;
+    for (int w = warp + 1; w < nwarps; ++w) cum += sm.warp_eq[w];
+    if (cum < (uint32_t)k_rem && cum + mine >= (uint32_t)k_rem) {
+        for (int b = per - 1; b >= 0; --b) {
+            const uint32_t h = sm.hist[per * tid + b];
+            if (cum + h >= (uint32_t)k_rem) {
+                sm.digit = per * tid + b;
+                sm.k_rem = k_rem - (int)cum;
+                break;
+            }
+            cum += h;
+        }
+    }
+    __syncthreads();
+}
+
+// Histogram of digit (key >> shift) & mask over keys matching (key & pmask) == prefix.
+__device__ __forceinline__ void sel_histogram(const uint32_t *keys, int n, int shift, uint32_t mask, uint32_t pmask,
+                                              uint32_t prefix, SelectSmem &sm, bool aggregate) {
+    const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31;
+    const int n_round = (n + 31) & ~31;
+    for (int i = tid; i < n_round; i += nt) {
+        const bool live = i < n;
+        const uint32_t key = live ? keys[i] : 0u;
+        const bool match = live && (key & pmask) == prefix;
+        const uint32_t bin = match ? (key >> shift) & mask : 0xFFFFFFFFu;
+        if (aggregate) {
+            const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+            if (match && lane == __ffs(peers) - 1) atomicAdd(&sm.hist[bin], (uint32_t)__popc(peers));
+        } else if (match) {
+            atomicAdd(&sm.hist[bin], 1u);
+        }
+    }
+}
+
+// Finds K* and the number of keys equal to K* that are taken (requires k < n).
 __device__ __forceinline__ void radix_kth(const uint32_t *keys, int n, int k, SelectSmem &sm) {
     const int tid = threadIdx.x, nt = blockDim.x;
-    uint32_t prefix = 0, mask = 0;
-    int k_rem = k;
-    for (int pass = 0; pass < 4; ++pass) {
-        const int shift = 24 - 8 * pass;
-        for (int i = tid; i < 256; i += nt) sm.hist[i] = 0;
-        __syncthreads();
-        for (int i = tid; i < n; i += nt) {
-            const uint32_t key = keys[i];
-            if ((key & mask) == prefix) atomicAdd(&sm.hist[(key >> shift) & 255u], 1u);
+    // ---- top 11 bits
+    for (int i = tid; i < 2048; i += nt) sm.hist[i] = 0;
+    if (tid == 0) sm.ncand = 0;
+    __syncthreads();
+    sel_histogram(keys, n, 21, 2047u, 0u, 0u, sm, true);
+    __syncthreads();
+    sel_find_digit(sm, 2048, k);
+    uint32_t prefix = (uint32_t)sm.digit << 21;
+    uint32_t pmask = 0xFFE00000u;
+    int k_rem = sm.k_rem;
+    // ---- gather the keys of that bin
+    const int n_round = (n + 31) & ~31;
+    for (int i = tid; i < n_round; i += nt) {
+        const bool hit = i < n && (keys[i] & pmask) == prefix;
+        const uint32_t bal = __ballot_sync(0xffffffffu, hit);
+        int base = 0;
+        if ((tid & 31) == 0 && bal) base = atomicAdd(&sm.ncand, __popc(bal));
+        base = __shfl_sync(0xffffffffu, base, 0);
+        if (hit) {
+            const int slot = base + __popc(bal & ((1u << (tid & 31)) - 1u));
+            if (slot < kSelCandCap) sm.cand[slot] = keys[i];
         }
+    }
+    __syncthreads();
+    const int nc = sm.ncand;
+    const bool small = nc <= kSelCandCap;
+    const uint32_t *src = small ? sm.cand : keys;
+    const int ns = small ? nc : n;
+    // ---- bits 20..10, then 9..0
+    const int shifts[2] = {10, 0};
+    const uint32_t masks[2] = {2047u, 1023u};
+    for (int pass = 0; pass < 2; ++pass) {
+        const int nb = pass == 0 ? 2048 : 1024;
+        for (int i = tid; i < nb; i += nt) sm.hist[i] = 0;
         __syncthreads();
-        if (tid < 32) {
-            const int lane = tid;
-            uint32_t mine = 0;
-#pragma unroll
-            for (int b = 0; b < 8; ++b) mine += sm.hist[8 * lane + b];
-            // exclusive suffix sum over lanes: counts in bins above this lane's range
-            uint32_t incl = mine;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                uint32_t v = __shfl_down_sync(0xffffffffu, incl, o);
-                if (lane + o < 32) incl += v;
-            }
-            uint32_t above = incl - mine;
-            int found = -1;
-            uint32_t cum = above;
-            for (int b = 7; b >= 0; --b) {
-                const uint32_t h = sm.hist[8 * lane + b];
-                if (cum < (uint32_t)k_rem && cum + h >= (uint32_t)k_rem) { found = 8 * lane + b; break; }
-                cum += h;
-            }
-            if (found >= 0) {
-                sm.kstar = (uint32_t)found;
-                sm.take_eq = k_rem - (int)cum;
-            }
-        }
+        sel_histogram(src, ns, shifts[pass], masks[pass], pmask, prefix, sm, !small);
         __syncthreads();
-        prefix |= sm.kstar << shift;
-        mask |= 255u << shift;
-        k_rem = sm.take_eq;
+        sel_find_digit(sm, nb, k_rem);
+        prefix |= (uint32_t)sm.digit << shifts[pass];
+        pmask |= masks[pass] << shifts[pass];
+        k_rem = sm.k_rem;
         __syncthreads();
     }
     if (tid == 0) {
@@ -80,47 +144,55 @@ __device__ __forceinline__ void radix_kth(const uint32_t *keys, int n, int k, Se
 }
 
 // Ordered compaction of the selection described by (sm.kstar, sm.take_eq):
-// calls emit(out_pos, i) for every selected position i in increasing order of
-// i.  With all_valid (n <= k) every position is selected.  Returns the count.
+// calls emit(out_pos, i) for every selected position i, in increasing i.
+// With all_valid (n <= k) every position is selected.  Returns the count.
 template <typename Emit>
 __device__ __forceinline__ int ordered_select(const uint32_t *keys, int n, bool all_valid, SelectSmem &sm,
                                               Emit &&emit) {
     const int tid = threadIdx.x, nt = blockDim.x;
     const int lane = tid & 31, warp = tid >> 5, nwarps = nt >> 5;
+    if (all_valid) {
+        for (int i = tid; i < n; i += nt) emit(i, i);
+        return n;
+    }
     const uint32_t lt = (1u << lane) - 1u;
     const uint32_t kstar = sm.kstar;
     const int take_eq = sm.take_eq;
-    if (tid == 0) { sm.run_out = 0; sm.run_eq = 0; }
-    __syncthreads();
-    for (int base = 0; base < n; base += nt) {
-        const int i = base + tid;
-        const bool valid = i < n;
-        const uint32_t key = valid ? keys[i] : 0u;
-        const bool gt = valid && (all_valid || key > kstar);
-        const bool eq = valid && !all_valid && key == kstar;
-        const uint32_t be = __ballot_sync(0xffffffffu, eq);
-        if (lane == 0) sm.warp_a[warp] = __popc(be);
-        __syncthreads();
-        int eq_before = sm.run_eq;
-        for (int w = 0; w < warp; ++w) eq_before += sm.warp_a[w];
-        const int eq_rank = eq_before + __popc(be & lt);
-        const bool sel = gt || (eq && eq_rank < take_eq);
-        const uint32_t bs = __ballot_sync(0xffffffffu, sel);
-        if (lane == 0) sm.warp_b[warp] = __popc(bs);
-        __syncthreads();
-        int out_before = sm.run_out;
-        for (int w = 0; w < warp; ++w) out_before += sm.warp_b[w];
-        if (sel) emit(out_before + __popc(bs & lt), i);
-        __syncthreads();
-        if (tid == 0) {
-            int te = 0, ts = 0;
-            for (int w = 0; w < nwarps; ++w) { te += sm.warp_a[w]; ts += sm.warp_b[w]; }
-            sm.run_eq += te;
-            sm.run_out += ts;
-        }
-        __syncthreads();
+    const int per = (((n + nwarps - 1) / nwarps) + 31) & ~31;
+    const int r0 = min(n, warp * per), r1 = min(n, r0 + per);
+    uint32_t cgt = 0, ceq = 0;
+    for (int b = r0; b < r1; b += 32) {
+        const int i = b + lane;
+        const uint32_t key = i < r1 ? keys[i] : 0u;
+        cgt += __popc(__ballot_sync(0xffffffffu, i < r1 && key > kstar));
+        ceq += __popc(__ballot_sync(0xffffffffu, i < r1 && key == kstar));
     }
-    return sm.run_out;
+    if (lane == 0) { sm.warp_gt[warp] = cgt; sm.warp_eq[warp] = ceq; }
+    __syncthreads();
+    // exclusive prefix over warps: outputs and equal keys before this warp's range
+    int eq_before = 0, out_run = 0, total = 0, eq_run = 0;
+    for (int w = 0; w < nwarps; ++w) {
+        const int e = (int)sm.warp_eq[w];
+        const int s = (int)sm.warp_gt[w] + max(0, min(e, take_eq - eq_before));
+        if (w < warp) out_run += s;
+        if (w == warp) eq_run = eq_before;
+        total += s;
+        eq_before += e;
+    }
+    for (int b = r0; b < r1; b += 32) {
+        const int i = b + lane;
+        const uint32_t key = i < r1 ? keys[i] : 0u;
+        const bool gt = i < r1 && key > kstar;
+        const bool eq = i < r1 && key == kstar;
+        const uint32_t be = __ballot_sync(0xffffffffu, eq);
+        const bool sel = gt || (eq && eq_run + __popc(be & lt) < take_eq);
+        const uint32_t bs = __ballot_sync(0xffffffffu, sel);
+        if (sel) emit(out_run + __popc(bs & lt), i);
+        eq_run += __popc(be);
+        out_run += __popc(bs);
+    }
+    __syncthreads();
+    return total;
 }
 
 // Full select: top-k of keys[0..n) -> emit(pos, i) in ascending i; returns the count.

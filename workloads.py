@@ -85,14 +85,15 @@ def _heavy_scale(n, g, device):
     return torch.clamp(u.pow(-1.0 / 1.5), max=64.0)
 
 
-def _inverse_rotation(u: torch.Tensor, pos: float, base: float, pos_scale: float) -> torch.Tensor:
-    """Return x with rotate-half rotation R(pos) x == u (fp64).  Pairs
-    (i, i + 64) turn by (pos / pos_scale) * base^(-2i/128); the inverse turns
-    by the negative angle."""
+def _inverse_rotation(u: torch.Tensor, pos: torch.Tensor, base: float, pos_scale: float) -> torch.Tensor:
+    """Return x with rotate-half rotation R(pos) x == u (fp64), batched:
+    u [..., 128], pos broadcastable to u[..., 0].  Pairs (i, i + 64) turn by
+    (pos / pos_scale) * base^(-2i/128); the inverse turns by the negative
+    angle."""
     half = IDX_DIM // 2
     i = torch.arange(half, dtype=torch.float64, device=u.device)
-    ang = (pos / pos_scale) * torch.pow(torch.tensor(base, dtype=torch.float64, device=u.device),
-                                        -(2.0 * i) / IDX_DIM)
+    inv_freq = torch.pow(torch.tensor(base, dtype=torch.float64, device=u.device), -(2.0 * i) / IDX_DIM)
+    ang = (pos.to(torch.float64) / pos_scale).unsqueeze(-1) * inv_freq
     c, s = torch.cos(-ang), torch.sin(-ang)
     a, b = u[..., :half], u[..., half:]
     return torch.cat([a * c - b * s, b * c + a * s], dim=-1)
@@ -129,37 +130,46 @@ def _plant_needles(w, T, g, device, q_idx, k_idx, q, k, alpha=8.0, beta=8.0, per
                    min_query=2048):
     """Plant `w.needles` blocks whose indexer keys (after the method's pooling
     and rotation) point along a unit direction u_j, and add beta * u_j (in
-    the rotated frame) to the indexer queries of 16 later positions per
+    the rotated frame) to the indexer queries of up to 16 later positions per
     needle, drawn from [max(min_query, 4b+4), T).  The attention keys of the
-    block and the queries at those positions get the same direction, so the
-    attention mass follows the needle too.  Needles need T > min_query + 4."""
-    nblk = T // BLOCK
-    B = w.B
-    hi = min(nblk, (T - 4) // BLOCK)
-    perm = torch.randperm(hi, generator=g, device=device)[: w.needles]
-    out = []
-    for j in range(w.needles):
-        b = int(perm[j])
-        u = _randn((IDX_DIM,), g, device).double()
-        u = u / u.norm()
-        ua = _randn((w.d,), g, device).double()
-        ua = ua / ua.norm()
-        lo = max(min_query, BLOCK * b + BLOCK)
-        if lo >= T:
-            continue
-        ts = torch.randint(lo, T, (per_needle,), generator=g, device=device).tolist()
-        for bi in range(B):
-            for i in range(BLOCK):
-                tok = BLOCK * b + i
-                k_idx[bi, tok] = (alpha * _inverse_rotation(u, BLOCK * b, w.rope_base, w.pos_scale)
-                                  + 0.1 * _randn((IDX_DIM,), g, device).double()).float()
-                k[bi, tok] = (alpha * ua + 0.1 * _randn((w.Hkv, w.d), g, device).double()).float()
-            for t in ts:
-                add = beta * _inverse_rotation(u, t, w.rope_base, w.pos_scale)
-                q_idx[bi, t] += add.float().view(1, IDX_DIM)
-                q[bi, t] += (beta * ua).float().view(1, w.d)
-        out.append((b, sorted(set(ts))))
-    return out
+    block and the queries at those positions get a shared direction too, so
+    the attention mass follows the needle.  Needles need T > min_query + 4.
+    Vectorised: a handful of kernel launches whatever the needle count."""
+    n = w.needles
+    hi = (T - 4) // BLOCK
+    blocks = torch.randperm(hi, generator=g, device=device)[:n]
+    lo = torch.clamp(BLOCK * blocks + BLOCK, min=min_query)
+    keep = lo < T
+    blocks, lo = blocks[keep], lo[keep]
+    n = int(blocks.numel())
+    u = _randn((n, IDX_DIM), g, device).double()
+    u = u / u.norm(dim=-1, keepdim=True)
+    ua = _randn((n, w.d), g, device).double()
+    ua = ua / ua.norm(dim=-1, keepdim=True)
+    span = (T - lo).to(torch.float64)
+    ts = lo.unsqueeze(1) + torch.floor(torch.rand((n, per_needle), generator=g, device=device,
+                                                  dtype=torch.float64) * span.unsqueeze(1)).long()
+    noise_k = 0.1 * _randn((n, BLOCK, IDX_DIM), g, device).double()
+    noise_a = 0.1 * _randn((n, BLOCK, w.Hkv, w.d), g, device).double()
+    tok = (BLOCK * blocks).unsqueeze(1) + torch.arange(BLOCK, device=device)          # [n][4]
+    kvec = alpha * _inverse_rotation(u, (BLOCK * blocks).to(torch.float64), w.rope_base, w.pos_scale)
+    kvec = kvec.unsqueeze(1) + noise_k                                                  # [n][4][128]
+    avec = alpha * ua[:, None, None, :] + noise_a                                        # [n][4][Hkv][d]
+    # unique (needle, query position) pairs
+    pair = torch.unique(torch.stack([torch.arange(n, device=device).unsqueeze(1).expand(n, per_needle), ts],
+                                    dim=-1).view(-1, 2), dim=0)
+    j, t = pair[:, 0], pair[:, 1]
+    qadd = beta * _inverse_rotation(u[j], t.to(torch.float64), w.rope_base, w.pos_scale)   # [m][128]
+    for bi in range(w.B):
+        k_idx[bi].index_copy_(0, tok.reshape(-1), kvec.reshape(-1, IDX_DIM).float())
+        k[bi].index_copy_(0, tok.reshape(-1), avec.reshape(-1, w.Hkv, w.d).float())
+        q_idx[bi].index_add_(0, t, qadd.float().unsqueeze(1).expand(-1, IDX_HEADS, IDX_DIM).contiguous())
+        q[bi].index_add_(0, t, (beta * ua[j]).float().unsqueeze(1).expand(-1, w.Hq, w.d).contiguous())
+    bl = blocks.tolist()
+    tl = [[] for _ in range(n)]
+    for jj, tt in zip(j.tolist(), t.tolist()):
+        tl[jj].append(tt)
+    return [(bl[i], sorted(tl[i])) for i in range(n)]
 
 
 def make_decode(w: Workload, device="cuda", L: int | None = None, B: int | None = None,
