@@ -247,45 +247,27 @@ __global__ void __launch_bounds__(128) score_simt_kernel(const float *__restrict
     p.scores[((int64_t)seq * p.row_count + blockIdx.y) * p.ld + b] = acc;
 }
 
-// Per-row top-k over materialised scores: one CTA per (row, sequence).
-__global__ void __launch_bounds__(512) select_rows_kernel(const float *__restrict__ scores, int64_t row_begin,
-                                                          int64_t n_q, int64_t q0, int64_t ld, int top_k,
-                                                          int32_t *__restrict__ sel, int32_t *__restrict__ nsel,
-                                                          int64_t row_count) {
-    extern __shared__ uint32_t keys[];
-    __shared__ SelectSmem sm;
+// Per-row top-k over materialised scores: one warp per (row, sequence), 16
+// rows per CTA, no CTA barriers (see warp_topk_row).
+constexpr int SEL_WARPS = 16;
+
+__global__ void __launch_bounds__(SEL_WARPS * 32, 2)
+    select_rows_kernel(const float *__restrict__ scores, int64_t row_begin, int64_t n_q, int64_t q0, int64_t ld,
+                       int top_k, int32_t *__restrict__ sel, int32_t *__restrict__ nsel, int64_t row_count) {
+    extern __shared__ uint8_t ssm_raw[];
+    WarpSelSmem *wsm = reinterpret_cast<WarpSelSmem *>(ssm_raw);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int seq = blockIdx.y;
-    const int64_t rloc = blockIdx.x;
+    const int64_t rloc = (int64_t)blockIdx.x * SEL_WARPS + warp;
+    if (rloc >= row_count) return;
     const int64_t row = row_begin + rloc;
     const int64_t t = q0 + row;
     const int n = (int)((t + 1) / kBlock);
     const float *src = scores + ((int64_t)seq * row_count + rloc) * ld;
-    // 16-byte loads, four in flight per thread (rows are 16-byte aligned: ld % 128 == 0)
-    const int n4 = (n + 3) >> 2;
-    const float4 *src4 = reinterpret_cast<const float4 *>(src);
-    for (int base = threadIdx.x; base < n4; base += 4 * blockDim.x) {
-        float4 v[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int i4 = base + u * blockDim.x;
-            if (i4 < n4) v[u] = src4[i4];
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int i4 = base + u * blockDim.x;
-            if (i4 < n4) {
-                const float f[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    if (4 * i4 + c < n) keys[4 * i4 + c] = score_key(f[c]);
-            }
-        }
-    }
-    __syncthreads();
     int32_t *out = sel + ((int64_t)seq * n_q + row) * top_k;
-    const int cnt = cta_topk(keys, n, top_k, sm, [&](int pos, int i) { out[pos] = i; });
-    for (int i = cnt + threadIdx.x; i < top_k; i += blockDim.x) out[i] = -1;
-    if (threadIdx.x == 0) nsel[(int64_t)seq * n_q + row] = cnt;
+    const int cnt = warp_topk_row(src, n, top_k, wsm[warp], [&](int pos, int i) { out[pos] = i; });
+    for (int i = cnt + lane; i < top_k; i += 32) out[i] = -1;
+    if (lane == 0) nsel[(int64_t)seq * n_q + row] = cnt;
 }
 
 // Driver-API tensor-map encoder obtained through the runtime (no -lcuda).
@@ -357,13 +339,11 @@ cudaError_t launch_select_rows(const float *scores, int B, int64_t row_begin, in
                                cudaStream_t s) {
     (void)status;
     if (row_count <= 0) return cudaSuccess;
-    const size_t smem = (size_t)ld * sizeof(uint32_t);
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(select_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-    }
-    dim3 grid((unsigned)row_count, (unsigned)B);
-    select_rows_kernel<<<grid, 512, smem, s>>>(scores, row_begin, n_q, q0, ld, top_k, sel, nsel, row_count);
+    const size_t smem = SEL_WARPS * sizeof(WarpSelSmem);
+    cudaError_t e = cudaFuncSetAttribute(select_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)((row_count + SEL_WARPS - 1) / SEL_WARPS), (unsigned)B);
+    select_rows_kernel<<<grid, SEL_WARPS * 32, smem, s>>>(scores, row_begin, n_q, q0, ld, top_k, sel, nsel, row_count);
     return cudaGetLastError();
 }
 

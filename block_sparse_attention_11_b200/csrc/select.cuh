@@ -204,3 +204,204 @@ __device__ __forceinline__ int cta_topk(const uint32_t *keys, int n, int k, Sele
 }
 
 }  // namespace qsa
+
+namespace qsa {
+
+// ---------------------------------------------------------------------------
+// Warp-per-row top-k over scores held in global memory (L2-resident rows).
+//
+// Same ranking and output as cta_topk, for one row per warp and no CTA
+// barriers, so many rows are in flight per SM:
+//   pass 1  11-bit histogram of the top digit (two 16-bit counters per word,
+//           warp-aggregated shared-memory atomics);
+//   pass 2  the keys of the bin holding K* are gathered into a per-warp list
+//           and the remaining 21 bits are resolved on it (if the bin overflows
+//           the list, they are resolved on the row instead);
+//   pass 3  ordered emission: lane l holds elements 4l..4l+3 of each 128-wide
+//           chunk; warp prefix sums give output positions and equal-key ranks.
+// ---------------------------------------------------------------------------
+constexpr int kWarpSelBuf = 512;
+
+struct WarpSelSmem {
+    uint32_t hist[1024];          // 2048 16-bit counters
+    uint32_t buf[kWarpSelBuf];    // keys of the threshold bin
+};
+
+__device__ __forceinline__ uint32_t wsel_count(const WarpSelSmem &w, int bin) {
+    return (w.hist[bin >> 1] >> (16 * (bin & 1))) & 0xFFFFu;
+}
+
+// Find the digit holding the k_rem-th largest among nbins (<= 2048) counters;
+// returns digit and updates k_rem.  Lane l owns bins [l*per, l*per + per).
+__device__ __forceinline__ int wsel_find(const WarpSelSmem &w, int nbins, int &k_rem) {
+    const int lane = threadIdx.x & 31;
+    const int per = nbins / 32;
+    uint32_t mine = 0;
+    for (int b = 0; b < per; ++b) mine += wsel_count(w, per * lane + b);
+    uint32_t incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_down_sync(0xffffffffu, incl, o);
+        if (lane + o < 32) incl += v;
+    }
+    uint32_t cum = incl - mine;
+    int digit = -1, rem = 0;
+    if (cum < (uint32_t)k_rem && cum + mine >= (uint32_t)k_rem) {
+        for (int b = per - 1; b >= 0; --b) {
+            const uint32_t h = wsel_count(w, per * lane + b);
+            if (cum + h >= (uint32_t)k_rem) { digit = per * lane + b; rem = k_rem - (int)cum; break; }
+            cum += h;
+        }
+    }
+    const uint32_t who = __ballot_sync(0xffffffffu, digit >= 0);
+    const int src = __ffs(who) - 1;
+    digit = __shfl_sync(0xffffffffu, digit, src);
+    k_rem = __shfl_sync(0xffffffffu, rem, src);
+    return digit;
+}
+
+__device__ __forceinline__ void wsel_clear(WarpSelSmem &w, int nbins) {
+    const int lane = threadIdx.x & 31;
+    for (int i = lane; i < nbins / 2; i += 32) w.hist[i] = 0;
+    __syncwarp();
+}
+
+__device__ __forceinline__ void wsel_add(WarpSelSmem &w, bool live, uint32_t bin) {
+    const uint32_t b = live ? bin : 0xFFFFFFFFu;
+    const uint32_t peers = __match_any_sync(0xffffffffu, b);
+    if (live && (threadIdx.x & 31) == __ffs(peers) - 1)
+        atomicAdd(&w.hist[bin >> 1], (uint32_t)__popc(peers) << (16 * (bin & 1)));
+}
+
+// Loads element chunk [base + 4*lane, +4) of the row as keys (invalid -> live=false).
+__device__ __forceinline__ void wsel_load4(const float *row, int n, int base, uint32_t (&key)[4], bool (&live)[4]) {
+    const int lane = threadIdx.x & 31;
+    const int i = base + 4 * lane;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (i < n) v = *reinterpret_cast<const float4 *>(row + i);   // row stride keeps 16-byte alignment
+    const float f[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        live[c] = i + c < n;
+        key[c] = score_key(f[c]);
+    }
+}
+
+// Top-k of one row; emit(pos, i) in ascending i.  Returns the count.  Whole warp.
+template <typename Emit>
+__device__ __forceinline__ int warp_topk_row(const float *row, int n, int k, WarpSelSmem &w, Emit &&emit) {
+    const int lane = threadIdx.x & 31;
+    const uint32_t lt = (1u << lane) - 1u;
+    if (n <= k) {
+        for (int i = lane; i < n; i += 32) emit(i, i);
+        return n;
+    }
+    // ---- pass 1: top 11 bits
+    wsel_clear(w, 2048);
+    for (int base = 0; base < n; base += 128) {
+        uint32_t key[4];
+        bool live[4];
+        wsel_load4(row, n, base, key, live);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) wsel_add(w, live[c], key[c] >> 21);
+    }
+    __syncwarp();
+    int k_rem = k;
+    const uint32_t d1 = (uint32_t)wsel_find(w, 2048, k_rem);
+    uint32_t prefix = d1 << 21, pmask = 0xFFE00000u;
+    // ---- pass 2: gather the bin's keys
+    int cnt = 0;
+    for (int base = 0; base < n; base += 128) {
+        uint32_t key[4];
+        bool live[4];
+        wsel_load4(row, n, base, key, live);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const bool hit = live[c] && (key[c] & pmask) == prefix;
+            const uint32_t bal = __ballot_sync(0xffffffffu, hit);
+            if (hit) {
+                const int slot = cnt + __popc(bal & lt);
+                if (slot < kWarpSelBuf) w.buf[slot] = key[c];
+            }
+            cnt += __popc(bal);
+        }
+    }
+    __syncwarp();
+    const bool small = cnt <= kWarpSelBuf;
+    const int shifts[2] = {10, 0};
+    const uint32_t masks[2] = {2047u, 1023u};
+    for (int pass = 0; pass < 2; ++pass) {
+        const int nb = pass == 0 ? 2048 : 1024;
+        wsel_clear(w, nb);
+        if (small) {
+            for (int i = lane; i < ((cnt + 31) & ~31); i += 32) {
+                const bool live = i < cnt && (w.buf[i] & pmask) == prefix;
+                const uint32_t key = i < cnt ? w.buf[i] : 0u;
+                wsel_add(w, live, (key >> shifts[pass]) & masks[pass]);
+            }
+        } else {
+            for (int base = 0; base < n; base += 128) {
+                uint32_t key[4];
+                bool live[4];
+                wsel_load4(row, n, base, key, live);
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    wsel_add(w, live[c] && (key[c] & pmask) == prefix, (key[c] >> shifts[pass]) & masks[pass]);
+            }
+        }
+        __syncwarp();
+        const uint32_t d = (uint32_t)wsel_find(w, nb, k_rem);
+        prefix |= d << shifts[pass];
+        pmask |= masks[pass] << shifts[pass];
+        __syncwarp();
+    }
+    const uint32_t kstar = prefix;
+    const int take_eq = k_rem;
+    // ---- pass 3: ordered emission
+    int out_run = 0, eq_run = 0;
+    for (int base = 0; base < n; base += 128) {
+        uint32_t key[4];
+        bool live[4];
+        wsel_load4(row, n, base, key, live);
+        int ngt = 0, neq = 0;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            ngt += live[c] && key[c] > kstar;
+            neq += live[c] && key[c] == kstar;
+        }
+        // exclusive prefix of equal keys over lanes (lane order = element order)
+        int eq_incl = neq;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, eq_incl, o);
+            if (lane >= o) eq_incl += v;
+        }
+        int eq_before = eq_run + eq_incl - neq;
+        int nsel = 0;
+        bool sel[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const bool gt = live[c] && key[c] > kstar;
+            const bool eq = live[c] && key[c] == kstar;
+            sel[c] = gt || (eq && eq_before < take_eq);
+            eq_before += eq;
+            nsel += sel[c];
+        }
+        int sel_incl = nsel;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, sel_incl, o);
+            if (lane >= o) sel_incl += v;
+        }
+        int pos = out_run + sel_incl - nsel;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+            if (sel[c]) emit(pos++, base + 4 * lane + c);
+        out_run += __shfl_sync(0xffffffffu, sel_incl, 31);
+        eq_run += __shfl_sync(0xffffffffu, eq_incl, 31);
+    }
+    (void)lt;
+    return out_run;
+}
+
+}  // namespace qsa
