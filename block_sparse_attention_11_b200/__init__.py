@@ -25,6 +25,7 @@ __all__ = [
     "qsa_index_topk_prefill", "qsa_index_topk_prefill_workspace",
     "qsa_index_topk_decode", "qsa_index_topk_decode_workspace",
     "qsa_sparse_attn_prefill", "qsa_sparse_attn_decode", "qsa_sparse_attn_decode_workspace",
+    "qsa_sparse_attn_decode_noalloc",
     "qsa_rope_apply", "qsa_check_status", "qsa_strerror", "qsa_version",
     "QSA_SCORE_RELU", "QSA_POOL_RMSNORM", "QSA_BF16", "QSA_FP32",
 ]
@@ -93,6 +94,8 @@ _sig("qsa_sparse_attn_decode_workspace", _sz, _i32, _i32, _i32, _i32, _i32)
 _sig("qsa_sparse_attn_decode", ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32, _i32,
      _f32, _vp, _vp, _vp, _sz, _i32, _vp)
 _sig("qsa_rope_apply", ctypes.c_int, _vp, _i32, _i64, _i32, _i32, _i64, _Rope, _i32, _vp)
+_sig("qsa_sparse_attn_decode_noalloc", ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32,
+     _i32, _f32, _vp, _vp, _i32, _vp)
 
 
 def qsa_strerror(status: int) -> str:
@@ -242,6 +245,25 @@ def qsa_sparse_attn_decode(q, k, v, seq_len, sel, nsel, out, top_k=None, scale=N
                                     _ptr(out, q.dtype, "out"), _ptr(lse, torch.float32, "lse"), wp, wb, dt,
                                     _stream(q, stream))
     _check(st, "qsa_sparse_attn_decode")
+
+
+def qsa_sparse_attn_decode_noalloc(q, k, v, seq_len, sel, nsel, out, top_k=None, scale=None, lse=None, stream=None):
+    """As qsa_sparse_attn_decode, for callers that cannot allocate device memory
+    at the call: the library keeps the split partials in its own fixed scratch
+    (QSA_NOALLOC_SCRATCH_BYTES per GPU).  Calls that overlap on the GPU share
+    that scratch and race; the first call on a device should precede any
+    stream capture."""
+    dt = _dtype_code(q)
+    B, Hq, d = q.shape
+    Hkv = k.shape[2]
+    top_k = sel.shape[-1] if top_k is None else top_k
+    scale = (1.0 / d ** 0.5) if scale is None else scale
+    st = lib.qsa_sparse_attn_decode_noalloc(_ptr(q, None, "q"), _ptr(k, q.dtype, "k"), _ptr(v, q.dtype, "v"),
+                                            _ptr(seq_len, torch.int32, "seq_len"), _ptr(sel, torch.int32, "sel"),
+                                            _ptr(nsel, torch.int32, "nsel"), B, k.shape[1], Hq, Hkv, d, top_k, scale,
+                                            _ptr(out, q.dtype, "out"), _ptr(lse, torch.float32, "lse"), dt,
+                                            _stream(q, stream))
+    _check(st, "qsa_sparse_attn_decode_noalloc")
 
 
 def qsa_rope_apply(x, pos0=0, rope=Rope(), stream=None):

@@ -266,6 +266,34 @@ QSA_API int qsa_sparse_attn_decode(const void *q, const void *k, const void *v, 
                            float *lse, void *workspace, size_t ws_bytes, int32_t dtype, void *stream);
 
 /* ========================================================================= */
+/* Decode sparse attention without a workspace (allocation-free callers)      */
+/* ========================================================================= */
+/*
+ * Not a step of the method: the source pages have no counterpart.  This is a
+ * convenience for callers that cannot allocate device memory where they call
+ * QSA (an engine that gives all free memory to its KV pool and forbids
+ * allocation in the decode loop, a host thread that must not block on
+ * cudaMalloc/cudaFree, a fixed pre-planned memory budget).
+ *
+ * Same arguments, results and errors as qsa_sparse_attn_decode, minus the
+ * workspace: the split-KV partial results live in a scratch area compiled
+ * into the library, QSA_NOALLOC_SCRATCH_BYTES of device memory on every GPU
+ * that loads the library, held until the process exits.  Calls needing more
+ * (roughly B * splits * Hq * 516 bytes, splits ~ 2 * SMs / B) return
+ * QSA_ERR_WORKSPACE.  Allocates nothing.  The first call on a device looks up
+ * the scratch's device address (cudaGetSymbolAddress) with that device
+ * current; make that first call before any stream capture.  Every call on a
+ * device shares the one scratch area: calls whose work can overlap on the GPU
+ * (different streams without ordering) race and must be serialised by the
+ * caller.  Nothing needs clearing between calls.
+ */
+#define QSA_NOALLOC_SCRATCH_BYTES (4u << 20)
+QSA_API int qsa_sparse_attn_decode_noalloc(const void *q, const void *k, const void *v, const int32_t *seq_len,
+                                           const int32_t *sel, const int32_t *nsel, int32_t B, int64_t kv_stride,
+                                           int32_t Hq, int32_t Hkv, int32_t d, int32_t top_k, float scale, void *out,
+                                           float *lse, int32_t dtype, void *stream);
+
+/* ========================================================================= */
 /* Helper: the attention layer's RoPE                                         */
 /* ========================================================================= */
 /*
