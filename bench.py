@@ -5,7 +5,7 @@
 A step is one pass of the whole hot path over one batch of synthetic input:
   prefill workloads: compressed-key pooling + indexer (query rotation, block
     scores, per-row top-k) + sparse attention over the selected K/V;
-  decode workloads: ring pooling + decode indexer (scan + merge) + split-KV
+  decode workloads: ring pooling + decode indexer (scan + select) + split-KV
     sparse attention + combine.
 The default workload is the 32K-token prefill with planted needles (B=1,
 T=32768, top-512, 16 q / 2 kv heads, bf16).  One JSON line is printed by
@@ -221,7 +221,7 @@ class DecodeRunner:
         return self.out
 
     def launches_per_step(self):
-        return 5   # ring pool, decode scorer, merge, attention, combine
+        return 6   # ring pool, decode scorer, candidate select, ordered emission, attention, combine
 
     def units(self):
         return self.w.B

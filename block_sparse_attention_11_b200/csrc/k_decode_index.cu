@@ -3,15 +3,15 @@
 //
 // Page "Qwen3.8-Flash-Next: Day-0 Support in SGLang", section "IndexShare MTP":
 // the decode scorer reads all ceil(L/4) compressed blocks and, beyond a few
-// thousand tokens, sets the cost of the layer.  So this is an HBM-streaming
+// thousand tokens, sets the cost of the layer.  So the scan is an HBM-streaming
 // kernel: each CTA owns a contiguous chunk of one sequence's compressed keys,
-// pulls it through shared memory with 16 KB bulk TMA copies (4 in flight),
-// computes the scores with warp-level fp32 dot products, keeps them in shared
-// memory, and selects the chunk's local top-k there.  A second kernel merges
-// the chunks of each sequence.  Any block of the global top-k is in its
-// chunk's local top-k under the same (score desc, id asc) order, so the merge
-// is exact; chunks are consecutive id ranges and local lists are ascending,
-// so concatenating them keeps ascending id order for the tie rule.
+// pulls it through shared memory with TMA (bulk copies in fp32 mode, 128-byte
+// swizzled tensor tiles in bf16 mode where the scores come from warp MMAs),
+// writes one 4-byte order-preserving score key per block to the workspace and
+// adds the chunk's histogram of the keys' top 11 bits into a per-sequence
+// histogram.  The selection then runs over the keys (still in L2) on many CTAs
+// per sequence: a candidate pass that needs only the keys of the histogram bin
+// holding the k-th largest key, and an ordered emission pass.
 #include <algorithm>
 
 #include "internal.h"
@@ -24,20 +24,22 @@ namespace {
 constexpr int DI_THREADS = 256;
 constexpr int DI_NS = 4;
 constexpr int DI_STAGE_BYTES = 16384;
-constexpr int64_t DI_MAX_CHUNK = 16384;     // scores of one chunk live in smem (64 KB)
-constexpr int DI_MERGE_CAP = 24576;         // candidates one merge CTA holds (key + id = 192 KB)
-constexpr int DI_MERGE_THREADS = 1024;
 
 struct DecodeParams {
     const int32_t *seq_len;
     const float *head_w;
-    int64_t pool_stride, max_blocks, chunk;
+    int64_t pool_stride, max_blocks, chunk, kstride;
     int chunks, top_k, relu;
-    uint32_t *cand_key;
-    int32_t *cand_idx;
-    int32_t *cand_cnt;
+    uint32_t *keys;      // [B][kstride] score keys
+    uint32_t *hist;      // [B][2048] histogram of the keys' top 11 bits
     unsigned *status;
 };
+
+// Adds a CTA's local histogram (smem, 2048 bins) into the sequence's global one.
+__device__ __forceinline__ void flush_hist(const uint32_t *lh, uint32_t *gh) {
+    for (int b = threadIdx.x; b < 2048; b += blockDim.x)
+        if (lh[b]) atomicAdd(&gh[b], lh[b]);
+}
 
 template <typename T>
 __global__ void __launch_bounds__(DI_THREADS, 2)
@@ -49,11 +51,10 @@ __global__ void __launch_bounds__(DI_THREADS, 2)
     constexpr int SROWS = DI_STAGE_BYTES / ROW_BYTES;
     extern __shared__ __align__(128) uint8_t dsm[];
     uint8_t *stage = dsm;                                                   // DI_NS * 16 KB
-    uint32_t *keys = reinterpret_cast<uint32_t *>(dsm + DI_NS * DI_STAGE_BYTES);
     __shared__ uint64_t full[DI_NS];
     __shared__ float qh[kIdxHeads][kIdxDim];
     __shared__ float qsum[kIdxDim];
-    __shared__ SelectSmem sm;
+    __shared__ uint32_t lh[2048];
 
     const int seq = blockIdx.y, c = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -66,13 +67,11 @@ __global__ void __launch_bounds__(DI_THREADS, 2)
     const int64_t c0 = (int64_t)c * p.chunk;
     const int64_t c1 = min(c0 + p.chunk, nb);
     const int n = (int)(c1 > c0 ? c1 - c0 : 0);
-    const int64_t cbase = ((int64_t)seq * p.chunks + c) * p.top_k;
-    if (n == 0) {
-        if (tid == 0) p.cand_cnt[(int64_t)seq * p.chunks + c] = 0;
-        return;
-    }
+    if (n == 0) return;
+    uint32_t *gkeys = p.keys + (int64_t)seq * p.kstride + c0;
     const int nstages = (n + SROWS - 1) / SROWS;
     const T *kbase = k_pool + ((int64_t)seq * p.pool_stride + c0) * kIdxDim;
+    for (int b = tid; b < 2048; b += blockDim.x) lh[b] = 0;
     if (tid == 0) {
         for (int s = 0; s < DI_NS; ++s) mbar_init(&full[s], 1);
         fence_mbar_init();
@@ -167,7 +166,11 @@ __global__ void __launch_bounds__(DI_THREADS, 2)
 #pragma unroll
                 for (int h = 0; h < kIdxHeads; ++h) score += w[h] * (p.relu ? fmaxf(acc[h], 0.f) : acc[h]);
             }
-            if (live && sub == 0) keys[st * SROWS + r] = score_key(score);
+            if (live && sub == 0) {
+                const uint32_t key = score_key(score);
+                gkeys[st * SROWS + r] = key;
+                atomicAdd(&lh[key >> 21], 1u);
+            }
         }
         __syncthreads();
         if (tid == 0 && st + DI_NS < nstages) {
@@ -179,13 +182,7 @@ __global__ void __launch_bounds__(DI_THREADS, 2)
         }
     }
     __syncthreads();
-    uint32_t *ck = p.cand_key + cbase;
-    int32_t *ci = p.cand_idx + cbase;
-    const int cnt = cta_topk(keys, n, p.top_k, sm, [&](int pos, int i) {
-        ck[pos] = keys[i];
-        ci[pos] = (int32_t)(c0 + i);
-    });
-    if (tid == 0) p.cand_cnt[(int64_t)seq * p.chunks + c] = cnt;
+    flush_hist(lh, p.hist + (int64_t)seq * 2048);
 }
 
 // bf16 scorer on the tensor cores.  A 128-key stage arrives by two tensor
@@ -202,7 +199,7 @@ struct DecodeMmaSmem {
     alignas(16) __nv_bfloat16 qcol[8][kIdxDim];   // B operand source: 8 columns x 128 dims
     float w[kIdxHeads];
     uint64_t full[DM_NS], empty[DM_NS];
-    SelectSmem sel;
+    uint32_t lh[2048];                             // local histogram of the keys' top 11 bits
 };
 
 __global__ void __launch_bounds__(DI_THREADS, 2)
@@ -211,7 +208,6 @@ __global__ void __launch_bounds__(DI_THREADS, 2)
     extern __shared__ uint8_t dsm_raw[];
     DecodeMmaSmem &sm = *reinterpret_cast<DecodeMmaSmem *>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) &
                                                            ~uintptr_t(1023));
-    uint32_t *keys = reinterpret_cast<uint32_t *>(reinterpret_cast<uint8_t *>(&sm) + sizeof(DecodeMmaSmem));
     const int seq = blockIdx.y, c = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t s_len = p.seq_len[seq];
@@ -223,11 +219,9 @@ __global__ void __launch_bounds__(DI_THREADS, 2)
     const int64_t c0 = (int64_t)c * p.chunk;
     const int64_t c1 = min(c0 + p.chunk, nb);
     const int n = (int)(c1 > c0 ? c1 - c0 : 0);
-    const int64_t cbase = ((int64_t)seq * p.chunks + c) * p.top_k;
-    if (n == 0) {
-        if (tid == 0) p.cand_cnt[(int64_t)seq * p.chunks + c] = 0;
-        return;
-    }
+    if (n == 0) return;
+    uint32_t *gkeys = p.keys + (int64_t)seq * p.kstride + c0;
+    for (int b = tid; b < 2048; b += blockDim.x) sm.lh[b] = 0;
     const int nstages = (n + DM_ROWS - 1) / DM_ROWS;
     const int y0 = (int)(seq * p.pool_stride + c0);
     if (tid == 0) {
@@ -337,8 +331,16 @@ __global__ void __launch_bounds__(DI_THREADS, 2)
         }
         const int r0 = st * DM_ROWS + 16 * warp + gr;
         if (tq == 0) {
-            if (r0 < n) keys[r0] = score_key(s0);
-            if (r0 + 8 < n) keys[r0 + 8] = score_key(s1);
+            if (r0 < n) {
+                const uint32_t key = score_key(s0);
+                gkeys[r0] = key;
+                atomicAdd(&sm.lh[key >> 21], 1u);
+            }
+            if (r0 + 8 < n) {
+                const uint32_t key = score_key(s1);
+                gkeys[r0 + 8] = key;
+                atomicAdd(&sm.lh[key >> 21], 1u);
+            }
         }
         if (tid == 0 && st + DM_NS < nstages) {
             ok = mbar_wait(&sm.empty[slot], (st / DM_NS) & 1, p.status);
@@ -352,49 +354,7 @@ __global__ void __launch_bounds__(DI_THREADS, 2)
     }
     ok = __syncthreads_and(ok);
     if (!ok) return;
-    uint32_t *ck = p.cand_key + cbase;
-    int32_t *ci = p.cand_idx + cbase;
-    const int cnt = cta_topk(keys, n, p.top_k, sm.sel, [&](int pos, int i) {
-        ck[pos] = keys[i];
-        ci[pos] = (int32_t)(c0 + i);
-    });
-    if (tid == 0) p.cand_cnt[(int64_t)seq * p.chunks + c] = cnt;
-}
-
-__global__ void __launch_bounds__(DI_MERGE_THREADS) decode_merge_kernel(DecodePlan plan, int top_k,
-                                                                         const uint32_t *__restrict__ cand_key,
-                                                                         const int32_t *__restrict__ cand_idx,
-                                                                         const int32_t *__restrict__ cand_cnt,
-                                                                         int32_t *__restrict__ sel,
-                                                                         int32_t *__restrict__ nsel) {
-    extern __shared__ __align__(16) uint32_t msm[];
-    __shared__ int off[65];
-    __shared__ SelectSmem sm;
-    const int seq = blockIdx.x, tid = threadIdx.x;
-    const int C = plan.chunks;
-    const int cap = C * top_k;
-    uint32_t *keys = msm;
-    int32_t *ids = reinterpret_cast<int32_t *>(msm + cap);
-    if (tid == 0) {
-        int a = 0;
-        for (int c = 0; c < C; ++c) { off[c] = a; a += cand_cnt[(int64_t)seq * C + c]; }
-        off[C] = a;
-    }
-    __syncthreads();
-    const int total = off[C];
-    const int64_t base = (int64_t)seq * C * top_k;
-    for (int f = tid; f < cap; f += blockDim.x) {
-        const int c = f / top_k, i = f % top_k;
-        if (off[c] + i < off[c + 1]) {
-            keys[off[c] + i] = cand_key[base + f];
-            ids[off[c] + i] = cand_idx[base + f];
-        }
-    }
-    __syncthreads();
-    int32_t *out = sel + (int64_t)seq * top_k;
-    const int cnt = cta_topk(keys, total, top_k, sm, [&](int pos, int i) { out[pos] = ids[i]; });
-    for (int i = cnt + tid; i < top_k; i += blockDim.x) out[i] = -1;
-    if (tid == 0) nsel[seq] = cnt;
+    flush_hist(sm.lh, p.hist + (int64_t)seq * 2048);
 }
 
 using EncodeTiledFn = decltype(&cuTensorMapEncodeTiled);
@@ -419,6 +379,291 @@ bool make_kpool_map(CUtensorMap *map, const void *base, uint64_t rows) {
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// ---------------------------------------------------------------------------
+// Selection from the score keys, spread over many CTAs per sequence.
+//
+// Every CTA owns a chunk of a sequence's keys (whole tiles of DS_TILE keys,
+// 16 contiguous keys per thread, read with four 16-byte loads issued
+// together).  With the top-11-bit histogram from the scorer, the bin d1 that
+// holds the k-th largest key is known before any key is read:
+//   candidate pass  each CTA counts its keys above bin d1 and appends the keys
+//                   of bin d1, with their block ids, to a per-sequence list;
+//                   the last CTA of the sequence to finish (ticket counter)
+//                   resolves the remaining 21 bits of K* on that list, and
+//                   from the list and the per-chunk counts computes each
+//                   chunk's output offset and the number of keys equal to K*
+//                   that precede it;
+//   emission pass   each CTA writes its selected block ids in ascending order
+//                   at its chunk's offset (prefix sums over threads).
+// ---------------------------------------------------------------------------
+constexpr int DS_THREADS = 512;
+constexpr int DS_PER_THREAD = 16;
+constexpr int DS_TILE = DS_THREADS * DS_PER_THREAD;   // keys per CTA tile
+constexpr int DS_MAX_CHUNKS = 2048;                   // chunks per sequence at most
+constexpr int DS_CAND_SMEM = 4096;                    // candidates staged in shared memory
+
+struct SelMeta {           // per sequence; zeroed before the scorer runs
+    uint32_t ncand;        // candidates appended (keys of bin d1)
+    uint32_t done;         // CTAs of the candidate pass that finished
+    uint32_t kstar;        // K*
+    int32_t take_eq;       // keys equal to K* taken, in block order
+};
+
+struct SelectArgs {
+    const int32_t *seq_len;
+    int64_t pool_stride, max_blocks, kstride, chunk;   // chunk: keys per CTA, a multiple of DS_TILE
+    int gmax, top_k;
+    const uint32_t *keys;   // [B][kstride]
+    const uint32_t *hist;   // [B][2048]
+    SelMeta *meta;          // [B]
+    uint2 *cand;            // [B][kstride] (key, block id)
+    uint32_t *cnt_gt;       // [B][gmax] keys above bin d1 per chunk
+    int2 *plan;             // [B][gmax] (output offset, keys == K* before the chunk)
+    int32_t *sel, *nsel;
+};
+
+struct DsSmem {
+    SelectSmem s;
+    uint32_t ck[DS_CAND_SMEM];
+    uint32_t ci[DS_CAND_SMEM];
+    uint32_t gtc[DS_MAX_CHUNKS];
+    uint32_t eqc[DS_MAX_CHUNKS];
+    uint32_t wsum[DS_THREADS / 32];
+    uint32_t wsum2[DS_THREADS / 32];
+    int last;
+};
+
+__device__ __forceinline__ int64_t visible_blocks(const SelectArgs &a, int seq) {
+    const int64_t s_len = a.seq_len[seq];
+    const int64_t nb = s_len / kBlock;
+    return (s_len < 1 || nb > a.pool_stride || nb > a.max_blocks) ? 0 : nb;   // flagged by the scorer
+}
+
+// Loads keys [i0, i0 + 16) of a row (i0 a multiple of 16; the row holds
+// kstride keys, a multiple of 4); returns how many of them are < n.
+__device__ __forceinline__ int load16(const uint32_t *row, int64_t i0, int64_t n, int64_t kstride, uint32_t k[16]) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int64_t i = i0 + 4 * j;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (i < n && i < kstride) v = __ldcg(reinterpret_cast<const uint4 *>(row + i));
+        k[4 * j] = v.x; k[4 * j + 1] = v.y; k[4 * j + 2] = v.z; k[4 * j + 3] = v.w;
+    }
+    const int64_t m = n - i0;
+    return m <= 0 ? 0 : (m >= 16 ? 16 : (int)m);
+}
+
+// Exclusive prefix over the CTA; total in `total`.  Two barriers.
+__device__ __forceinline__ uint32_t cta_scan(uint32_t v, uint32_t *wsum, uint32_t &total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    uint32_t x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) wsum[warp] = x;
+    __syncthreads();
+    uint32_t off = 0, tot = 0;
+    for (int w = 0; w < nw; ++w) {
+        const uint32_t t = wsum[w];
+        if (w < warp) off += t;
+        tot += t;
+    }
+    __syncthreads();
+    total = tot;
+    return off + x - v;
+}
+
+__global__ void __launch_bounds__(DS_THREADS)
+    decode_cand_kernel(SelectArgs a) {
+    extern __shared__ __align__(16) uint8_t ds_raw[];
+    DsSmem &sm = *reinterpret_cast<DsSmem *>(ds_raw);
+    const int seq = blockIdx.y, g = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
+    const int64_t nb = visible_blocks(a, seq);
+    if (nb <= a.top_k) return;                       // everything is selected
+    const int gseq = (int)((nb + a.chunk - 1) / a.chunk);
+    if (g >= gseq) return;
+    const uint32_t *row = a.keys + (int64_t)seq * a.kstride;
+    uint2 *cand = a.cand + (int64_t)seq * a.kstride;
+    SelMeta &meta = a.meta[seq];
+    // bin of the k-th largest key from the scorer's histogram
+    for (int b = tid; b < 2048; b += DS_THREADS) sm.s.hist[b] = __ldcg(a.hist + (int64_t)seq * 2048 + b);
+    if (tid == 0) { sm.s.digit = 0; sm.s.k_rem = 1; }
+    __syncthreads();
+    sel_find_digit(sm.s, 2048, a.top_k);
+    const uint32_t d1 = (uint32_t)sm.s.digit;
+    const int k_rem1 = sm.s.k_rem;
+
+    const int64_t c0 = (int64_t)g * a.chunk, c1 = min(c0 + a.chunk, nb);
+    uint32_t n_gt = 0;
+    for (int64_t t0 = c0; t0 < c1; t0 += DS_TILE) {
+        uint32_t k[16];
+        const int64_t i0 = t0 + (int64_t)DS_PER_THREAD * tid;
+        const int m = load16(row, i0, c1, a.kstride, k);
+        uint32_t ce = 0;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const uint32_t dg = k[j] >> 21;
+            if (j < m) { n_gt += dg > d1; ce += dg == d1; }
+        }
+        // warp-level append of the bin-d1 keys
+        uint32_t x = ce;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        uint32_t base = 0;
+        if (lane == 31 && x) base = atomicAdd(&meta.ncand, x);
+        base = __shfl_sync(0xffffffffu, base, 31) + x - ce;
+        if (ce) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                if (j < m && (k[j] >> 21) == d1) {
+                    if (base < (uint64_t)a.kstride) cand[base] = make_uint2(k[j], (uint32_t)(i0 + j));
+                    ++base;
+                }
+            }
+        }
+    }
+    uint32_t tot;
+    cta_scan(n_gt, sm.wsum, tot);
+    if (tid == 0) a.cnt_gt[(int64_t)seq * a.gmax + g] = tot;
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) sm.last = atomicAdd(&meta.done, 1u) == (uint32_t)(gseq - 1);
+    __syncthreads();
+    if (!sm.last) return;
+    __threadfence();
+
+    // ---- last CTA of this sequence: K* from the candidates, then the chunk plan
+    const int nc = (int)min((int64_t)__ldcg(&meta.ncand), nb);
+    const bool small = nc <= DS_CAND_SMEM;
+    if (small)
+        for (int i = tid; i < nc; i += DS_THREADS) {
+            const uint2 c = __ldcg(cand + i);
+            sm.ck[i] = c.x;
+            sm.ci[i] = c.y;
+        }
+    uint32_t prefix = d1 << 21, pmask = 0xFFE00000u;
+    int k_rem = k_rem1;
+#pragma unroll 1
+    for (int pass = 0; pass < 2; ++pass) {
+        const int shift = pass == 0 ? 10 : 0, nbins = pass == 0 ? 2048 : 1024;
+        const uint32_t mask = (uint32_t)nbins - 1u;
+        for (int b = tid; b < nbins; b += DS_THREADS) sm.s.hist[b] = 0;
+        __syncthreads();
+        for (int i = tid; i < nc; i += DS_THREADS) {
+            const uint32_t key = small ? sm.ck[i] : __ldcg(&cand[i].x);
+            if ((key & pmask) == prefix) atomicAdd(&sm.s.hist[(key >> shift) & mask], 1u);
+        }
+        __syncthreads();
+        sel_find_digit(sm.s, nbins, k_rem);
+        prefix |= (uint32_t)sm.s.digit << shift;
+        pmask |= mask << shift;
+        k_rem = sm.s.k_rem;
+        __syncthreads();
+    }
+    const uint32_t kstar = prefix;
+    const int take_eq = k_rem;
+    for (int i = tid; i < gseq; i += DS_THREADS) { sm.gtc[i] = 0; sm.eqc[i] = 0; }
+    __syncthreads();
+    for (int i = tid; i < nc; i += DS_THREADS) {
+        uint32_t key, id;
+        if (small) { key = sm.ck[i]; id = sm.ci[i]; }
+        else { const uint2 c = __ldcg(cand + i); key = c.x; id = c.y; }
+        const int gc = (int)min((int64_t)id / a.chunk, (int64_t)gseq - 1);
+        if (key > kstar) atomicAdd(&sm.gtc[gc], 1u);
+        else if (key == kstar) atomicAdd(&sm.eqc[gc], 1u);
+    }
+    __syncthreads();
+    // chunk plan: thread t owns chunks [per*t, per*t + per)
+    const int per = (gseq + DS_THREADS - 1) / DS_THREADS;
+    const int g0 = min(per * tid, gseq), g1 = min(g0 + per, gseq);
+    uint32_t eq_mine = 0;
+    for (int c = g0; c < g1; ++c) eq_mine += sm.eqc[c];
+    uint32_t eq_tot;
+    uint32_t eq_run = cta_scan(eq_mine, sm.wsum, eq_tot);
+    uint32_t s_mine = 0;
+    {
+        uint32_t e = eq_run;
+        for (int c = g0; c < g1; ++c) {
+            const uint32_t gt = __ldcg(a.cnt_gt + (int64_t)seq * a.gmax + c) + sm.gtc[c];
+            const int avail = max(0, take_eq - (int)e);
+            s_mine += gt + min((uint32_t)avail, sm.eqc[c]);
+            e += sm.eqc[c];
+        }
+    }
+    uint32_t s_tot;
+    uint32_t out_run = cta_scan(s_mine, sm.wsum2, s_tot);
+    for (int c = g0; c < g1; ++c) {
+        const uint32_t gt = __ldcg(a.cnt_gt + (int64_t)seq * a.gmax + c) + sm.gtc[c];
+        a.plan[(int64_t)seq * a.gmax + c] = make_int2((int)out_run, (int)eq_run);
+        const int avail = max(0, take_eq - (int)eq_run);
+        out_run += gt + min((uint32_t)avail, sm.eqc[c]);
+        eq_run += sm.eqc[c];
+    }
+    if (tid == 0) {
+        meta.kstar = kstar;
+        meta.take_eq = take_eq;
+    }
+}
+
+__global__ void __launch_bounds__(DS_THREADS)
+    decode_emit_kernel(SelectArgs a) {
+    __shared__ uint32_t wsum[DS_THREADS / 32];
+    const int seq = blockIdx.y, g = blockIdx.x, tid = threadIdx.x;
+    const int64_t nb = visible_blocks(a, seq);
+    const int top_k = a.top_k;
+    int32_t *out = a.sel + (int64_t)seq * top_k;
+    const int cnt = (int)min(nb, (int64_t)top_k);
+    if (g == 0) {
+        if (tid == 0) a.nsel[seq] = cnt;
+        for (int i = cnt + tid; i < top_k; i += DS_THREADS) out[i] = -1;
+    }
+    const int64_t c0 = (int64_t)g * a.chunk, c1 = min(c0 + a.chunk, nb);
+    if (c0 >= c1) return;
+    if (nb <= top_k) {                               // every visible block, in order
+        for (int64_t i = c0 + tid; i < c1; i += DS_THREADS) out[i] = (int32_t)i;
+        return;
+    }
+    const uint32_t *row = a.keys + (int64_t)seq * a.kstride;
+    const uint32_t kstar = a.meta[seq].kstar;
+    const int take_eq = a.meta[seq].take_eq;
+    const int2 pl = a.plan[(int64_t)seq * a.gmax + g];
+    int64_t o_run = pl.x, e_run = pl.y;              // output slots and keys == K* before this tile
+    for (int64_t t0 = c0; t0 < c1; t0 += DS_TILE) {
+        uint32_t k[16];
+        const int64_t i0 = t0 + (int64_t)DS_PER_THREAD * tid;
+        const int m = load16(row, i0, c1, a.kstride, k);
+        uint32_t gt = 0, eq = 0;
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            if (j < m) { gt += k[j] > kstar; eq += k[j] == kstar; }
+        uint32_t tot;
+        const uint32_t ex = cta_scan(gt | (eq << 16), wsum, tot);
+        const int64_t avail = max((int64_t)0, (int64_t)take_eq - e_run);
+        const int64_t eq_before = ex >> 16;
+        int64_t pos = o_run + (ex & 0xFFFFu) + min(avail, eq_before);
+        int64_t r = e_run + eq_before;
+        if (gt | eq) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                if (j >= m) continue;
+                bool take = k[j] > kstar;
+                if (k[j] == kstar) take = r++ < take_eq;
+                if (take) {
+                    if (pos >= 0 && pos < top_k) out[pos] = (int32_t)(i0 + j);
+                    ++pos;
+                }
+            }
+        }
+        o_run += (tot & 0xFFFFu) + min(avail, (int64_t)(tot >> 16));
+        e_run += tot >> 16;
+    }
+}
+
 }  // namespace
 
 DecodePlan decode_index_plan(int B, int64_t max_blocks, bool bf16) {
@@ -426,25 +671,75 @@ DecodePlan decode_index_plan(int B, int64_t max_blocks, bool bf16) {
     const DeviceInfo *di = device_info();
     const int sms = di ? di->sm_count : 148;
     DecodePlan pl;
-    int64_t C = std::max<int64_t>(1, (2 * sms) / std::max(B, 1));
-    C = std::min<int64_t>(C, std::max<int64_t>(1, (max_blocks + 255) / 256));
+    // about two CTAs per SM over all sequences, chunks of at least 512 blocks
+    int64_t C = std::max<int64_t>(1, (2 * sms + B - 1) / std::max(B, 1));
+    C = std::min<int64_t>(C, std::max<int64_t>(1, (max_blocks + 511) / 512));
     int64_t chunk = (max_blocks + C - 1) / C;
     chunk = std::max<int64_t>(128, (chunk + 127) / 128 * 128);
-    if (chunk > DI_MAX_CHUNK) chunk = DI_MAX_CHUNK;
     C = std::max<int64_t>(1, (max_blocks + chunk - 1) / chunk);
     pl.chunks = (int)C;
     pl.chunk = chunk;
     return pl;
 }
 
+namespace {
+int64_t key_stride(int64_t max_blocks) { return std::max<int64_t>(4, (max_blocks + 3) / 4 * 4); }
+size_t r256(size_t x) { return (x + 255) / 256 * 256; }
+
+struct SelectLayout {
+    int64_t chunk;
+    int gmax;
+};
+
+SelectLayout select_layout(int64_t max_blocks) {
+    const int64_t tiles = std::max<int64_t>(1, (max_blocks + DS_TILE - 1) / DS_TILE);
+    const int64_t tiles_per_chunk = (tiles + DS_MAX_CHUNKS - 1) / DS_MAX_CHUNKS;
+    SelectLayout l;
+    l.chunk = tiles_per_chunk * DS_TILE;
+    l.gmax = (int)((tiles + tiles_per_chunk - 1) / tiles_per_chunk);
+    return l;
+}
+
+// Workspace: keys [B][kstride] u32 | cand [B][kstride] uint2 | hist [B][2048] u32 + meta [B] |
+//            cnt_gt [B][gmax] u32 | plan [B][gmax] int2
+struct DecodeWs {
+    uint32_t *keys;
+    uint2 *cand;
+    uint32_t *hist;
+    SelMeta *meta;
+    uint32_t *cnt_gt;
+    int2 *plan;
+    size_t zero_bytes;   // hist + meta, cleared before every call
+    size_t total;
+};
+
+DecodeWs decode_ws(void *base, int B, int64_t max_blocks) {
+    const int64_t ks = key_stride(max_blocks);
+    const SelectLayout l = select_layout(max_blocks);
+    uint8_t *w = static_cast<uint8_t *>(base);
+    DecodeWs d;
+    size_t off = 0;
+    d.keys = reinterpret_cast<uint32_t *>(w + off);
+    off += r256((size_t)B * ks * 4);
+    d.cand = reinterpret_cast<uint2 *>(w + off);
+    off += r256((size_t)B * ks * 8);
+    d.hist = reinterpret_cast<uint32_t *>(w + off);
+    d.meta = reinterpret_cast<SelMeta *>(w + off + (size_t)B * 2048 * 4);
+    d.zero_bytes = (size_t)B * 2048 * 4 + (size_t)B * sizeof(SelMeta);
+    off += r256(d.zero_bytes);
+    d.cnt_gt = reinterpret_cast<uint32_t *>(w + off);
+    off += r256((size_t)B * l.gmax * 4);
+    d.plan = reinterpret_cast<int2 *>(w + off);
+    off += r256((size_t)B * l.gmax * 8);
+    d.total = off;
+    return d;
+}
+}  // namespace
+
 size_t decode_index_ws_bytes(int B, int64_t max_blocks, int top_k, bool bf16) {
-    const DecodePlan pl = decode_index_plan(B, max_blocks, bf16);
-    const size_t n = (size_t)B * pl.chunks * top_k;
-    size_t bytes = n * sizeof(uint32_t);
-    bytes = (bytes + 255) / 256 * 256;
-    bytes += (n * sizeof(int32_t) + 255) / 256 * 256;
-    bytes += ((size_t)B * pl.chunks * sizeof(int32_t) + 255) / 256 * 256;
-    return bytes;
+    (void)top_k;
+    (void)bf16;
+    return decode_ws(nullptr, B, max_blocks).total;
 }
 
 cudaError_t launch_decode_index(const void *q_idx, const void *k_pool, const float *head_w,
@@ -452,27 +747,22 @@ cudaError_t launch_decode_index(const void *q_idx, const void *k_pool, const flo
                                 int top_k, int32_t *sel, int32_t *nsel, void *ws, Rope rope, bool relu,
                                 bool bf16, unsigned *status, cudaStream_t s) {
     const DecodePlan pl = decode_index_plan(B, max_blocks, bf16);
-    if ((int64_t)pl.chunks * top_k > DI_MERGE_CAP || pl.chunks > 64) return cudaErrorInvalidConfiguration;
-    const size_t n = (size_t)B * pl.chunks * top_k;
-    uint8_t *w = static_cast<uint8_t *>(ws);
-    uint32_t *ck = reinterpret_cast<uint32_t *>(w);
-    w += (n * sizeof(uint32_t) + 255) / 256 * 256;
-    int32_t *ci = reinterpret_cast<int32_t *>(w);
-    w += (n * sizeof(int32_t) + 255) / 256 * 256;
-    int32_t *cc = reinterpret_cast<int32_t *>(w);
-    DecodeParams p{seq_len, head_w, pool_stride, max_blocks, pl.chunk, pl.chunks, top_k, relu ? 1 : 0, ck, ci, cc,
-                   status};
+    const int64_t kstride = key_stride(max_blocks);
+    const DecodeWs d = decode_ws(ws, B, max_blocks);
+    cudaError_t e = cudaMemsetAsync(d.hist, 0, d.zero_bytes, s);
+    if (e != cudaSuccess) return e;
+    DecodeParams p{seq_len, head_w, pool_stride, max_blocks, pl.chunk, kstride, pl.chunks, top_k, relu ? 1 : 0,
+                   d.keys, d.hist, status};
     dim3 grid((unsigned)pl.chunks, (unsigned)B);
-    cudaError_t e;
     if (bf16) {
         CUtensorMap kmap;
         if (!make_kpool_map(&kmap, k_pool, (uint64_t)B * pool_stride)) return cudaErrorInvalidValue;
-        const size_t smem = sizeof(DecodeMmaSmem) + 1024 + (size_t)pl.chunk * sizeof(uint32_t);
+        const size_t smem = sizeof(DecodeMmaSmem) + 1024;
         e = cudaFuncSetAttribute(decode_score_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         decode_score_mma_kernel<<<grid, DI_THREADS, smem, s>>>(kmap, (const __nv_bfloat16 *)q_idx, rope, p);
     } else {
-        const size_t smem = DI_NS * DI_STAGE_BYTES + (size_t)pl.chunk * sizeof(uint32_t);
+        const size_t smem = DI_NS * DI_STAGE_BYTES;
         e = cudaFuncSetAttribute(decode_score_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         decode_score_kernel<float><<<grid, DI_THREADS, smem, s>>>((const float *)q_idx, (const float *)k_pool, rope,
@@ -480,10 +770,16 @@ cudaError_t launch_decode_index(const void *q_idx, const void *k_pool, const flo
     }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const size_t msmem = (size_t)pl.chunks * top_k * 8;
-    e = cudaFuncSetAttribute(decode_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
+    const SelectLayout l = select_layout(max_blocks);
+    SelectArgs sa{seq_len, pool_stride, max_blocks, kstride, l.chunk, l.gmax, top_k, d.keys, d.hist, d.meta,
+                  d.cand, d.cnt_gt, d.plan, sel, nsel};
+    const dim3 sgrid((unsigned)l.gmax, (unsigned)B);
+    e = cudaFuncSetAttribute(decode_cand_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(DsSmem));
     if (e != cudaSuccess) return e;
-    decode_merge_kernel<<<B, DI_MERGE_THREADS, msmem, s>>>(pl, top_k, ck, ci, cc, sel, nsel);
+    decode_cand_kernel<<<sgrid, DS_THREADS, sizeof(DsSmem), s>>>(sa);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    decode_emit_kernel<<<sgrid, DS_THREADS, 0, s>>>(sa);
     return cudaGetLastError();
 }
 

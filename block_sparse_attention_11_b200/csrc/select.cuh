@@ -213,7 +213,7 @@ namespace qsa {
 // Same ranking and output as cta_topk, for one row per warp and no CTA
 // barriers, so many rows are in flight per SM:
 //   pass 1  11-bit histogram of the top digit (two 16-bit counters per word,
-//           warp-aggregated shared-memory atomics);
+//           shared-memory atomics);
 //   pass 2  the keys of the bin holding K* are gathered into a per-warp list
 //           and the remaining 21 bits are resolved on it (if the bin overflows
 //           the list, they are resolved on the row instead);
@@ -266,11 +266,10 @@ __device__ __forceinline__ void wsel_clear(WarpSelSmem &w, int nbins) {
     __syncwarp();
 }
 
+// Plain shared-memory atomics: cheaper here than aggregating equal digits
+// with match_any (measured on B200: 1.06 vs 1.43 ms for the 32K-token indexer).
 __device__ __forceinline__ void wsel_add(WarpSelSmem &w, bool live, uint32_t bin) {
-    const uint32_t b = live ? bin : 0xFFFFFFFFu;
-    const uint32_t peers = __match_any_sync(0xffffffffu, b);
-    if (live && (threadIdx.x & 31) == __ffs(peers) - 1)
-        atomicAdd(&w.hist[bin >> 1], (uint32_t)__popc(peers) << (16 * (bin & 1)));
+    if (live) atomicAdd(&w.hist[bin >> 1], 1u << (16 * (bin & 1)));
 }
 
 // Loads element chunk [base + 4*lane, +4) of the row as keys (invalid -> live=false).

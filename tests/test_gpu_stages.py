@@ -181,7 +181,8 @@ def test_attention_flags_out_of_range_ids(qsa):
 # ----------------------------------------------------------------------------- decode
 
 @pytest.mark.parametrize("dtype,flags,weights,L,B", [("bf16", 0, False, 20000, 6), ("bf16", 1, True, 9001, 3),
-                                                     ("fp32", 0, False, 5000, 4), ("bf16", 0, False, 2, 5)])
+                                                     ("fp32", 0, False, 5000, 4), ("bf16", 0, False, 2, 5),
+                                                     ("bf16", 0, False, 70001, 3), ("fp32", 1, True, 40000, 2)])
 def test_decode_pipeline(qsa, dtype, flags, weights, L, B):
     w = workloads.Workload("dec", "decode", B, L, 256, 16, 2, 128, dtype, 77, pos_scale=2.0)
     x = workloads.make_decode(w, device=DEV, ragged=True)
@@ -234,3 +235,28 @@ def test_decode_pipeline(qsa, dtype, flags, weights, L, B):
         err = np.abs(np32(out[b]) - ref["out"][0]).max()
         assert err <= TOL[dtype], (b, err)
         assert np.abs(lse[b].cpu().numpy() - ref["lse"][0]).max() <= (1e-3 if dtype == "bf16" else 1e-4)
+
+
+@pytest.mark.parametrize("dtype,flags", [("bf16", 0), ("bf16", 1), ("fp32", 0)])
+def test_decode_select_all_ties(qsa, dtype, flags):
+    """All compressed keys zero: every score is 0, so the top-k is the k lowest
+    block ids; with 10000+ blocks the tie bin spans several select chunks."""
+    B, top_k = 3, 512
+    lens = [40000, 65537, 2049]
+    dt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    cap = max(lens) // 4 + 1
+    k_pool = torch.zeros(B, cap, 128, dtype=dt, device=DEV)
+    g = torch.Generator().manual_seed(5)
+    q_idx = torch.randn(B, 4, 128, generator=g).to(dt).to(DEV)
+    seq_len = torch.tensor(lens, dtype=torch.int32, device=DEV)
+    sel = torch.full((B, top_k), -7, dtype=torch.int32, device=DEV)
+    nsel = torch.full((B,), -7, dtype=torch.int32, device=DEV)
+    qsa.qsa_index_topk_decode(q_idx, k_pool, seq_len, sel, nsel, top_k=top_k, flags=flags)
+    qsa.qsa_check_status()
+    for b, L in enumerate(lens):
+        nb = L // 4
+        n = min(nb, top_k)
+        assert int(nsel[b]) == n
+        exp = np.full(top_k, -1, np.int32)
+        exp[:n] = np.arange(n)
+        assert np.array_equal(sel[b].cpu().numpy(), exp), b
