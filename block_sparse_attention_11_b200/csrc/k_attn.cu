@@ -19,8 +19,11 @@
 //     M and the 8 q heads of one kv head as N (no padding waste for GQA 8),
 //     an fp32 online softmax per head column, P^T re-laid out in registers
 //     with movmatrix, and O^T += V^T P;
-//   * two warps per kv head take alternate stages (both 16-key tiles of a
-//     stage each) and merge their softmax states at the end of an item;
+//   * four warps per kv head share the stages: two take alternate stages,
+//     and each of those pairs splits a stage's two 16-key tiles, so every
+//     warp runs its own short softmax chain per stage; the four softmax
+//     states are merged at the end of an item (with 4 kv heads, two warps per
+//     head take both tiles of alternate stages);
 //   * the producer stages each item's block ids in shared memory once, so
 //     no global read sits on the per-stage issue path.
 // A persistent grid walks the work items; the pipeline runs across item
@@ -38,6 +41,8 @@ namespace {
 
 constexpr int AT_BPS = 8;               // blocks per stage
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescale = 8.f;         // lazy-rescale threshold (log2 units)
+constexpr uint32_t kFullStage = 0x924924u;   // 8 slots x 3 bits, each holding 4 tokens
 
 // Tuning knobs (compile time).  Defaults measured best on B200 for the
 // 32K-token prefill: 2 resident CTAs per SM, 2 stages in flight per CTA,
@@ -52,9 +57,18 @@ constexpr float kLog2e = 1.4426950408889634f;
 #define QSA_ATTN_NS 2             // stages in flight per CTA
 #endif
 
+#ifndef QSA_ATTN_TILES
+#define QSA_ATTN_TILES 2          // 16-key tiles of a stage per consumer warp (1 or 2); 2 with 4 kv heads
+#endif
+
 template <int HKV> struct AttnCfg {
-    static constexpr int kWph = 2;   // consumer warps per kv head: even / odd stages
+    // Consumer warp (g, sub): kv head g; sub = u * 2 + hf takes the stages whose
+    // global index is = hf (mod 2), and tiles [u * kTiles, (u + 1) * kTiles) of each.
+    static constexpr int kTiles = HKV == 4 ? 2 : QSA_ATTN_TILES;
+    static constexpr int kU = 2 / kTiles;          // warps sharing one stage of one kv head
+    static constexpr int kWph = 2 * kU;            // consumer warps per kv head
     static constexpr int kConsumers = kWph * HKV;
+    static constexpr int kMinCtas = HKV == 4 ? 1 : QSA_ATTN_CTAS;   // launch-bounds residency target
     static constexpr int kPw = QSA_ATTN_PW;
     static constexpr int kThreads = (kConsumers + kPw) * 32;
     static constexpr int kSpan = kBlock * HKV * 128 * 2;      // bytes of one block, all kv heads
@@ -69,6 +83,7 @@ template <int HKV> struct AttnCfg {
     // only tells the current phase from the previous one).
     static_assert(kNS >= 2 && kNS % 2 == 0, "stages in flight must be even");
     static_assert(AT_BPS % QSA_ATTN_PW == 0, "producer warps must divide the blocks per stage");
+    static_assert(kTiles == 1 || kTiles == 2, "a stage holds two 16-key tiles");
 };
 
 struct AttnParams {
@@ -82,6 +97,7 @@ struct AttnParams {
     int splits;            // decode: items per sequence
     int split_blocks;      // decode: list entries per split (multiple of AT_BPS)
     int64_t items;
+    int sel_cap, nst_cap;  // shared-memory block-id list and per-stage table sizes (from top_k)
     __nv_bfloat16 *out;
     float *lse;
     float *part_o;         // decode: [B][splits][Hq][128]
@@ -147,16 +163,22 @@ struct __align__(128) AttnSmem {
     alignas(16) uint8_t qbuf[2][AttnCfg<HKV>::kQBytes];
     float xbuf[HKV][AttnCfg<HKV>::kWph - 1][32][36];
     alignas(16) __nv_bfloat16 obuf[HKV][8][128];
-    int32_t sel_s[2048];                 // the current item's block ids (each producer fills its own slots)
-    uint32_t st_info[Cfg::kPw][264];     // per stage of the item: token counts of the producer's slots
-    uint32_t st_bytes[Cfg::kPw][264];    // per stage of the item: bytes the producer copies per tensor
-    uint32_t info[Cfg::kNS][Cfg::kPw];
+    alignas(16) uint32_t info[Cfg::kNS][Cfg::kPw];
     uint64_t full[Cfg::kNS], empty[Cfg::kNS], qfull[2], qempty[2];
-    uint64_t xready[HKV], xdone[HKV];   // pair merge handshake per kv head
+    uint64_t xready[HKV], xdone[HKV];   // merge handshake per kv head
+    // followed in dynamic shared memory by
+    //   int32_t  sel_s[sel_cap]             the current item's block ids (each producer fills its own slots)
+    //   uint32_t st_info[kPw][nst_cap]      per stage of the item: token counts of the producer's slots
+    //   uint32_t st_bytes[kPw][nst_cap]     per stage of the item: bytes the producer copies per tensor
 };
 
 template <int HKV>
-__global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, QSA_ATTN_CTAS) attn_bf16_kernel(AttnParams p) {
+size_t attn_smem_bytes(int sel_cap, int nst_cap) {
+    return sizeof(AttnSmem<HKV>) + (size_t)sel_cap * 4 + 2 * (size_t)AttnCfg<HKV>::kPw * nst_cap * 4 + 128;
+}
+
+template <int HKV>
+__global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, AttnCfg<HKV>::kMinCtas) attn_bf16_kernel(AttnParams p) {
     using Cfg = AttnCfg<HKV>;
     extern __shared__ uint8_t asm_raw[];
     AttnSmem<HKV> &sm = *reinterpret_cast<AttnSmem<HKV> *>((reinterpret_cast<uintptr_t>(asm_raw) + 127) & ~uintptr_t(127));
@@ -166,7 +188,7 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, QSA_ATTN_CTAS) attn_bf
     for (int i = threadIdx.x; i < (int)(sizeof(sm.stage) / 16); i += blockDim.x)
         reinterpret_cast<uint4 *>(&sm.stage[0][0])[i] = make_uint4(0, 0, 0, 0);
     if (threadIdx.x == 0) {
-        for (int s = 0; s < Cfg::kNS; ++s) { mbar_init(&sm.full[s], Cfg::kPw); mbar_init(&sm.empty[s], HKV); }
+        for (int s = 0; s < Cfg::kNS; ++s) { mbar_init(&sm.full[s], Cfg::kPw); mbar_init(&sm.empty[s], HKV * Cfg::kU); }
         for (int s = 0; s < 2; ++s) { mbar_init(&sm.qfull[s], 1); mbar_init(&sm.qempty[s], Cfg::kConsumers); }
         for (int s = 0; s < HKV; ++s) { mbar_init(&sm.xready[s], Cfg::kWph - 1); mbar_init(&sm.xdone[s], 1); }
         fence_mbar_init();
@@ -182,7 +204,9 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, QSA_ATTN_CTAS) attn_bf
         // is: wait for the slot, one expect_tx, one bulk copy per block and tensor.
         constexpr int kSlotsPerPw = AT_BPS / Cfg::kPw;
         const int pw = warp - Cfg::kConsumers;
-        int32_t *ids = sm.sel_s;
+        int32_t *ids = reinterpret_cast<int32_t *>(&sm + 1);
+        uint32_t *st_info = reinterpret_cast<uint32_t *>(ids + p.sel_cap) + pw * p.nst_cap;
+        uint32_t *st_bytes = reinterpret_cast<uint32_t *>(ids + p.sel_cap) + (Cfg::kPw + pw) * p.nst_cap;
         int64_t it_count = 0;   // stage counter across items
         int64_t ic = 0;         // item counter
         bool ok = true;
@@ -215,8 +239,8 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, QSA_ATTN_CTAS) attn_bf
                     info |= (uint32_t)tokens << (3 * j);
                     bytes += (uint32_t)tokens * HKV * 256u;
                 }
-                sm.st_info[pw][st] = info;
-                sm.st_bytes[pw][st] = bytes;
+                st_info[st] = info;
+                st_bytes[st] = bytes;
             }
             const int qs = (int)(ic & 1);
             if (pw == 0 && ic >= 2) ok = mbar_wait(&sm.qempty[qs], (int)(((ic >> 1) + 1) & 1), p.status);
@@ -232,14 +256,14 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, QSA_ATTN_CTAS) attn_bf
                 if (it_count >= Cfg::kNS) ok = mbar_wait(&sm.empty[s], (int)(((it_count / Cfg::kNS) + 1) & 1), p.status);
                 if (!ok) break;
                 if (lane == 0) {
-                    sm.info[s][pw] = sm.st_info[pw][st];
-                    mbar_arrive_expect_tx(&sm.full[s], 2 * sm.st_bytes[pw][st]);
+                    sm.info[s][pw] = st_info[st];
+                    mbar_arrive_expect_tx(&sm.full[s], 2 * st_bytes[st]);
                 }
                 __syncwarp();
                 if (lane < kSlotsPerPw) {
                     const int j = Cfg::kPw * lane + pw;
                     const int e = it.lbeg + AT_BPS * st + j;
-                    const int tokens = (int)((sm.st_info[pw][st] >> (3 * j)) & 7u);
+                    const int tokens = (int)((st_info[st] >> (3 * j)) & 7u);
                     if (tokens > 0) {
                         const int64_t blk = (e < it.nsel) ? (int64_t)ids[e - it.lbeg] : it.nb;
                         const int64_t off = (kv0 + blk * kBlock) * HKV * 128;
@@ -262,11 +286,16 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, QSA_ATTN_CTAS) attn_bf
     }
 
     // ---------------------------------------------------------------- consumers
-    // warp (g, hf): kv head g; takes the stages whose global index is = hf
-    // (mod 2) and processes both 16-key tiles of each (tile t = tokens {2t, 2t+1} of the
-    // stage's 8 blocks).
+    // warp (g, sub), sub = u * 2 + hf: kv head g; takes the stages whose global
+    // index is = hf (mod 2) and the 16-key tiles [u * kTiles, (u + 1) * kTiles)
+    // of each (tile t = tokens {2t, 2t+1} of the stage's 8 blocks).  Each warp
+    // keeps its own online-softmax state; the states of a kv head's warps are
+    // merged at the end of an item.
+    constexpr int kT = Cfg::kTiles;
     const int g = warp / Cfg::kWph;
-    const int hf = warp % Cfg::kWph;
+    const int sub = warp % Cfg::kWph;
+    const int hf = sub & 1;
+    const int t0 = (sub >> 1) * kT;
     const int gr = lane >> 2, tq = lane & 3;
     const uint32_t stage0 = smem_u32(&sm.stage[0][0]);
     const int mi = lane >> 3, rr = lane & 7;
@@ -304,71 +333,91 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, QSA_ATTN_CTAS) attn_bf
             ok = mbar_wait(&sm.full[s], (int)((it_count / Cfg::kNS) & 1), p.status);
             if (!ok) break;
             uint32_t info = 0;
+            if constexpr (Cfg::kPw == 4) {
+                const uint4 w4 = *reinterpret_cast<const uint4 *>(&sm.info[s][0]);
+                info = (w4.x | w4.y) | (w4.z | w4.w);
+            } else {
 #pragma unroll
-            for (int q2 = 0; q2 < Cfg::kPw; ++q2) info |= sm.info[s][q2];
+                for (int q2 = 0; q2 < Cfg::kPw; ++q2) info |= sm.info[s][q2];
+            }
             const uint32_t sbase = stage0 + (uint32_t)s * Cfg::kStage;
-            // S^T for both tiles (16 keys x 8 heads each), two accumulators per tile
-            float sa[2][4], sb[2][4];
+            // S^T for this warp's tiles (16 keys x 8 heads each), unscaled
+            float sc[kT][4];
 #pragma unroll
-            for (int t = 0; t < 2; ++t)
+            for (int t = 0; t < kT; ++t)
 #pragma unroll
-                for (int c = 0; c < 4; ++c) sa[t][c] = sb[t][c] = 0.f;
+                for (int c = 0; c < 4; ++c) sc[t][c] = 0.f;
 #pragma unroll
-            for (int kk = 0; kk < 8; kk += 2) {
+            for (int kk = 0; kk < 8; ++kk) {
 #pragma unroll
-                for (int t = 0; t < 2; ++t) {
-                    uint32_t a0, a1, a2, a3, c0, c1, c2, c3;
-                    ldsm_x4(sbase + k_lane_off + t * kTileOff + kk * 32, a0, a1, a2, a3);
-                    ldsm_x4(sbase + k_lane_off + t * kTileOff + (kk + 1) * 32, c0, c1, c2, c3);
-                    mma16816(sa[t], a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
-                    mma16816(sb[t], c0, c1, c2, c3, qf[kk + 1][0], qf[kk + 1][1]);
+                for (int t = 0; t < kT; ++t) {
+                    uint32_t a0, a1, a2, a3;
+                    ldsm_x4(sbase + k_lane_off + (uint32_t)(t0 + t) * kTileOff + kk * 32, a0, a1, a2, a3);
+                    mma16816(sc[t], a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
                 }
             }
-            const int ntok = (int)((info >> (3 * gr)) & 7u);
-            float x[2][4];
+            // (slot gr, token 2t): heads 2tq, 2tq+1 in sc[t][0..1]; token 2t+1 in sc[t][2..3]
+            if (info != kFullStage) {           // a short or missing block: mask its absent tokens
+                const int ntok = (int)((info >> (3 * gr)) & 7u);
 #pragma unroll
-            for (int t = 0; t < 2; ++t) {
-                const bool v0 = ntok > 2 * t, v1 = ntok > 2 * t + 1;
-                x[t][0] = v0 ? (sa[t][0] + sb[t][0]) * p.scale_log2 : -INFINITY;   // (slot gr, tok 2t),   head 2tq
-                x[t][1] = v0 ? (sa[t][1] + sb[t][1]) * p.scale_log2 : -INFINITY;   //                      head 2tq+1
-                x[t][2] = v1 ? (sa[t][2] + sb[t][2]) * p.scale_log2 : -INFINITY;   // (slot gr, tok 2t+1), head 2tq
-                x[t][3] = v1 ? (sa[t][3] + sb[t][3]) * p.scale_log2 : -INFINITY;
+                for (int t = 0; t < kT; ++t) {
+                    if (ntok <= 2 * (t0 + t)) sc[t][0] = sc[t][1] = -INFINITY;
+                    if (ntok <= 2 * (t0 + t) + 1) sc[t][2] = sc[t][3] = -INFINITY;
+                }
             }
-            float mx0 = fmaxf(fmaxf(x[0][0], x[0][2]), fmaxf(x[1][0], x[1][2]));
-            float mx1 = fmaxf(fmaxf(x[0][1], x[0][3]), fmaxf(x[1][1], x[1][3]));
+            float lm0 = fmaxf(sc[0][0], sc[0][2]), lm1 = fmaxf(sc[0][1], sc[0][3]);
 #pragma unroll
-            for (int o2 = 4; o2 < 32; o2 <<= 1) {
-                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o2));
-                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o2));
+            for (int t = 1; t < kT; ++t) {
+                lm0 = fmaxf(lm0, fmaxf(sc[t][0], sc[t][2]));
+                lm1 = fmaxf(lm1, fmaxf(sc[t][1], sc[t][3]));
             }
-            const float mn0 = fmaxf(mrow[0], mx0), mn1 = fmaxf(mrow[1], mx1);
-            const float mu0 = (mn0 == -INFINITY) ? 0.f : mn0, mu1 = (mn1 == -INFINITY) ? 0.f : mn1;
-            const float al0 = exp2f(mrow[0] - mu0), al1 = exp2f(mrow[1] - mu1);
-            mrow[0] = mn0;
-            mrow[1] = mn1;
-            uint32_t pb[2][2];
-            float ls0 = 0.f, ls1 = 0.f;
+            lm0 *= p.scale_log2;
+            lm1 *= p.scale_log2;
+            // Lazy rescaling: the reference max of a head column moves only when a
+            // score exceeds it by more than kRescale (log2 units), so unscaled
+            // probabilities stay below 2^kRescale; otherwise no max reduction and
+            // no rescale of the accumulators.
+            if (__any_sync(0xffffffffu, lm0 > mrow[0] + kRescale || lm1 > mrow[1] + kRescale)) {
 #pragma unroll
-            for (int t = 0; t < 2; ++t) {
-                const float p0 = exp2f(x[t][0] - mu0), p1 = exp2f(x[t][1] - mu1);
-                const float p2 = exp2f(x[t][2] - mu0), p3 = exp2f(x[t][3] - mu1);
-                ls0 += p0 + p2;
-                ls1 += p1 + p3;
+                for (int o2 = 4; o2 < 32; o2 <<= 1) {
+                    lm0 = fmaxf(lm0, __shfl_xor_sync(0xffffffffu, lm0, o2));
+                    lm1 = fmaxf(lm1, __shfl_xor_sync(0xffffffffu, lm1, o2));
+                }
+                const float mn0 = fmaxf(mrow[0], lm0), mn1 = fmaxf(mrow[1], lm1);
+                const float al0 = exp2f(mrow[0] - ((mn0 == -INFINITY) ? 0.f : mn0));
+                const float al1 = exp2f(mrow[1] - ((mn1 == -INFINITY) ? 0.f : mn1));
+                mrow[0] = mn0;
+                mrow[1] = mn1;
+                lrow[0] *= al0;
+                lrow[1] *= al1;
+#pragma unroll
+                for (int mt = 0; mt < 8; ++mt) {
+                    o[mt][0] *= al0;
+                    o[mt][1] *= al1;
+                    o[mt][2] *= al0;
+                    o[mt][3] *= al1;
+                }
+            }
+            const float nmu0 = (mrow[0] == -INFINITY) ? 0.f : -mrow[0];
+            const float nmu1 = (mrow[1] == -INFINITY) ? 0.f : -mrow[1];
+            uint32_t pb[kT][2];
+#pragma unroll
+            for (int t = 0; t < kT; ++t) {
+                const float p0 = exp2f(fmaf(sc[t][0], p.scale_log2, nmu0));
+                const float p1 = exp2f(fmaf(sc[t][1], p.scale_log2, nmu1));
+                const float p2 = exp2f(fmaf(sc[t][2], p.scale_log2, nmu0));
+                const float p3 = exp2f(fmaf(sc[t][3], p.scale_log2, nmu1));
+                lrow[0] += p0 + p2;
+                lrow[1] += p1 + p3;
                 pb[t][0] = movm_t(pack_bf16(p0, p1));
                 pb[t][1] = movm_t(pack_bf16(p2, p3));
             }
-            lrow[0] = lrow[0] * al0 + ls0;
-            lrow[1] = lrow[1] * al1 + ls1;
 #pragma unroll
             for (int mt = 0; mt < 8; ++mt) {
-                o[mt][0] *= al0;
-                o[mt][1] *= al1;
-                o[mt][2] *= al0;
-                o[mt][3] *= al1;
 #pragma unroll
-                for (int t = 0; t < 2; ++t) {
+                for (int t = 0; t < kT; ++t) {
                     uint32_t a0, a1, a2, a3;
-                    ldsm_x4_t(sbase + v_lane_off + t * kTileOff + mt * 32, a0, a1, a2, a3);
+                    ldsm_x4_t(sbase + v_lane_off + (uint32_t)(t0 + t) * kTileOff + mt * 32, a0, a1, a2, a3);
                     mma16816(o[mt], a0, a1, a2, a3, pb[t][0], pb[t][1]);
                 }
             }
@@ -382,11 +431,11 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, QSA_ATTN_CTAS) attn_bf
             lrow[0] += __shfl_xor_sync(0xffffffffu, lrow[0], o2);
             lrow[1] += __shfl_xor_sync(0xffffffffu, lrow[1], o2);
         }
-        // merge the warps of this kv head: warps hf >= 1 publish, warp 0 folds
-        if (hf != 0) {
+        // merge the warps of this kv head: warps sub >= 1 publish, warp 0 folds
+        if (sub != 0) {
             if (ic > 0) ok = mbar_wait(&sm.xdone[g], (int)((ic - 1) & 1), p.status);
             if (!ok) break;
-            float *xb = sm.xbuf[g][hf - 1][lane];
+            float *xb = sm.xbuf[g][sub - 1][lane];
             xb[0] = mrow[0]; xb[1] = mrow[1]; xb[2] = lrow[0]; xb[3] = lrow[1];
 #pragma unroll
             for (int mt = 0; mt < 8; ++mt)
@@ -397,10 +446,13 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, QSA_ATTN_CTAS) attn_bf
         } else {
             ok = mbar_wait(&sm.xready[g], (int)(ic & 1), p.status);
             if (!ok) break;
+            // Every fold is symmetric in its two operands (explicitly rounded, no
+            // contraction), so the result does not depend on which warp of a
+            // tile group took the even or the odd stages:
+            //   A = fold(own, sub 1)               tiles of group 0
+            //   B = fold(sub 2, sub 3)             tiles of group 1 (two groups only)
+            //   result = fold(A, B)
             {
-                // fold the other warp's state: symmetric in the two operands
-                // (explicitly rounded, no contraction), so the result does not
-                // depend on which warp took the even or the odd stages
                 const float *xb = sm.xbuf[g][0][lane];
                 float f0[2], f1[2];
 #pragma unroll
@@ -418,6 +470,32 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, QSA_ATTN_CTAS) attn_bf
 #pragma unroll
                     for (int c = 0; c < 4; ++c)
                         o[mt][c] = __fadd_rn(__fmul_rn(o[mt][c], f0[c & 1]), __fmul_rn(xb[4 + 4 * mt + c], f1[c & 1]));
+            }
+            if constexpr (Cfg::kU == 2) {
+                const float *x2 = sm.xbuf[g][1][lane], *x3 = sm.xbuf[g][2][lane];
+                float f2[2], f3[2], fa[2], fb[2];
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    const float mbv = fmaxf(x2[c], x3[c]);
+                    const float mub = (mbv == -INFINITY) ? 0.f : mbv;
+                    f2[c] = exp2f(x2[c] - mub);
+                    f3[c] = exp2f(x3[c] - mub);
+                    const float lb = __fadd_rn(__fmul_rn(x2[2 + c], f2[c]), __fmul_rn(x3[2 + c], f3[c]));
+                    const float mn = fmaxf(mrow[c], mbv);
+                    const float mu = (mn == -INFINITY) ? 0.f : mn;
+                    fa[c] = exp2f(mrow[c] - mu);
+                    fb[c] = exp2f(mbv - mu);
+                    lrow[c] = __fadd_rn(__fmul_rn(lrow[c], fa[c]), __fmul_rn(lb, fb[c]));
+                    mrow[c] = mn;
+                }
+#pragma unroll
+                for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const float ob = __fadd_rn(__fmul_rn(x2[4 + 4 * mt + c], f2[c & 1]),
+                                                   __fmul_rn(x3[4 + 4 * mt + c], f3[c & 1]));
+                        o[mt][c] = __fadd_rn(__fmul_rn(o[mt][c], fa[c & 1]), __fmul_rn(ob, fb[c & 1]));
+                    }
             }
             const float l[2] = {lrow[0], lrow[1]}, m[2] = {mrow[0], mrow[1]};
             const float inv0 = l[0] > 0.f ? 1.f / l[0] : 0.f, inv1 = l[1] > 0.f ? 1.f / l[1] : 0.f;
@@ -613,10 +691,17 @@ cudaError_t run_bf16(const AttnArgs &a, void *ws, unsigned *status, cudaStream_t
         p.items = (int64_t)a.B * a.n_q;
     }
     if (p.items <= 0) return cudaSuccess;
-    const size_t smem = sizeof(AttnSmem<HKV>) + 128;
+    // an item's list holds at most top_k ids plus the tail block
+    p.sel_cap = (a.top_k + 3) & ~3;
+    p.nst_cap = (a.top_k + 1 + AT_BPS - 1) / AT_BPS;
+    const size_t smem = attn_smem_bytes<HKV>(p.sel_cap, p.nst_cap);
+    if (di && smem > di->smem_optin) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(attn_bf16_kernel<HKV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    const int64_t grid = std::min<int64_t>(p.items, (int64_t)sms * QSA_ATTN_CTAS);
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, attn_bf16_kernel<HKV>, Cfg::kThreads, smem);
+    if (e != cudaSuccess) return e;
+    const int64_t grid = std::min<int64_t>(p.items, (int64_t)sms * std::max(1, per_sm));
     attn_bf16_kernel<HKV><<<(unsigned)grid, Cfg::kThreads, smem, s>>>(p);
     e = cudaGetLastError();
     if (e != cudaSuccess || !a.decode) return e;
