@@ -128,6 +128,7 @@ class PrefillRunner:
         # the step's inputs (~200 MB at T=32K) do not all stay in L2, but the
         # flush keeps every timed step cold
         self.flush_between_steps = True
+        self.use_graph = False        # three launches of milliseconds each: nothing to gain
 
     def step(self, x=None, events=None):
         qsa, w = self.qsa, self.w
@@ -201,6 +202,8 @@ class DecodeRunner:
         # a decode step streams the whole compressed-key cache and gathers from
         # K/V caches of several GB: inputs far larger than L2, no flush needed
         self.flush_between_steps = False
+        # six launches of tens of microseconds: the step is replayed as a CUDA graph
+        self.use_graph = True
 
     def step(self, x=None, events=None):
         qsa, w = self.qsa, self.w
@@ -262,6 +265,21 @@ def run_ours(args, rank, world):
     qsa.qsa_check_status()
 
     nst = 3
+    graph = None
+    if runner.use_graph:
+        # capture one step (all library calls, preallocated workspaces) and replay it
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(side):
+            runner.step()
+        torch.cuda.current_stream(dev).wait_stream(side)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            runner.step()
+        for _ in range(args.warmup):
+            graph.replay()
+        torch.cuda.synchronize()
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)] for _ in range(args.steps)]
     sampler = ClockSampler(dev.index if "CUDA_VISIBLE_DEVICES" not in os.environ else 0)
     if world > 1:
@@ -272,14 +290,29 @@ def run_ours(args, rank, world):
     for i in range(args.steps):
         if runner.flush_between_steps:
             flush_l2(flush)             # untimed: inputs start cold in L2
-        runner.step(events=events[i])
+        if graph is not None:
+            events[i][0].record()
+            graph.replay()
+            events[i][nst].record()
+        else:
+            runner.step(events=events[i])
     torch.cuda.synchronize()
     clocks = sampler.stop()
     if world > 1:
         torch.distributed.barrier()
     qsa.qsa_check_status()
     step_ms = [events[i][0].elapsed_time(events[i][nst]) for i in range(args.steps)]
-    stage_ms = [[events[i][s].elapsed_time(events[i][s + 1]) for i in range(args.steps)] for s in range(nst)]
+    if graph is not None:
+        # stage split from eager steps (per-stage events cannot sit inside the graph)
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)] for _ in range(args.steps)]
+        for i in range(args.steps):
+            runner.step(events=ev[i])
+        torch.cuda.synchronize()
+        eager_ms = sum(ev[i][0].elapsed_time(ev[i][nst]) for i in range(args.steps)) / args.steps
+        stage_ms = [[ev[i][s].elapsed_time(ev[i][s + 1]) for i in range(args.steps)] for s in range(nst)]
+    else:
+        eager_ms = None
+        stage_ms = [[events[i][s].elapsed_time(events[i][s + 1]) for i in range(args.steps)] for s in range(nst)]
     total_ms = sum(step_ms)
     # max over ranks
     t = torch.tensor([total_ms], device=dev)
@@ -295,19 +328,41 @@ def run_ours(args, rank, world):
     d2h = out_host.numel() * out_host.element_size()
     e2e_steps = max(3, min(args.steps, 10))
     dev_x = dict(runner.x)
-    for it in range(e2e_steps + 2):
-        if it == 2:
-            torch.cuda.synchronize()
-            e0 = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
-            e0.record()
+
+    def e2e_step():
         for k, v in host.items():
             dev_x[k] = v.to(dev, non_blocking=True)
         out = runner.step(x=dev_x)
         out_host.copy_(out, non_blocking=True)
-    e1.record()
-    torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+
+    def timed(fn):
+        for it in range(e2e_steps + 2):
+            if it == 2:
+                torch.cuda.synchronize()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record()
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / e2e_steps
+
+    e2e_eager_ms = timed(e2e_step)
+    e2e_ms = e2e_eager_ms
+    if graph is not None:
+        # the same public calls and copies (pinned host buffers), captured once and replayed
+        for k, v in host.items():
+            dev_x[k] = torch.empty_like(v, device=dev)
+        g2 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g2):
+            for k, v in host.items():
+                dev_x[k].copy_(v, non_blocking=True)
+            out = runner.step(x=dev_x)
+            out_host.copy_(out, non_blocking=True)
+        e2e_ms = timed(g2.replay)
+        del g2
+    used_graph = graph is not None
+    del graph
 
     pk, pk_kind = peaks()
     alg = runner.algorithmic()
@@ -316,6 +371,8 @@ def run_ours(args, rank, world):
                gpu_launches=runner.launches_per_step() * args.steps)
     stage_avg = {n: sum(v) / len(v) for n, v in zip(runner.stage_names(), stage_ms)}
     res["stage_ms"] = {k: round(v, 4) for k, v in stage_avg.items()}
+    if eager_ms is not None:
+        res["stage_ms"]["eager_step"] = round(eager_ms, 4)
     if w.kind == "prefill":
         tokens = runner.units() * world
         res.update(metric="QSA prefill tokens/s", unit="tokens/s", higher_is_better=True,
@@ -341,14 +398,15 @@ def run_ours(args, rank, world):
     else:
         res.update(metric="QSA decode us/step", unit="us/step", higher_is_better=False,
                    value=ms_per_step * 1e3)
-        res["e2e"] = dict(value=e2e_ms * 1e3, unit="us/step", h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h)
+        res["e2e"] = dict(value=e2e_ms * 1e3, unit="us/step", h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h,
+                          graph=used_graph, eager_value=e2e_eager_ms * 1e3)
         achieved = alg["step_bytes"] / (ms_per_step / 1e3) / 1e9
         res["roofline"] = dict(kernel="decode step (scorer dominant)", bound="hbm", achieved=achieved,
                                peak=pk["hbm_gbs"], unit="GB/s", frac=achieved / pk["hbm_gbs"], traffic=None,
                                peak_kind=pk_kind)
         res["config"] = dict(workload=w.name, B=w.B, L=w.T, top_k=w.top_k, Hq=w.Hq, Hkv=w.Hkv, d=w.d,
                              pos_scale=w.pos_scale, l2="inputs larger than L2 (compressed-key cache and K/V caches)",
-                             parallelism=f"replicas x{world}")
+                             parallelism=f"replicas x{world}", cuda_graph=True)
     return res
 
 

@@ -77,6 +77,15 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// ---------------------------------------------------------- dependent launch
+// Kernels that follow another kernel of the library on a stream are launched
+// with programmatic stream serialization: their CTAs may be scheduled while the
+// previous grid drains, and each waits in pdl_wait() -- before touching any
+// global memory -- until that grid has completed and its writes are visible.
+// Outside such a launch both instructions are no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {

@@ -195,6 +195,8 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, AttnCfg<HKV>::kMinCtas
     }
     fence_proxy_async_smem();
     __syncthreads();
+    pdl_wait();      // the selection comes from the previous kernel
+    pdl_trigger();
 
     if (warp >= Cfg::kConsumers) {
         // ------------------------------------------------------------ producers
@@ -552,6 +554,7 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const float *__restri
                                                            __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
     __shared__ float wsm[1024];
     __shared__ float red[4];
+    pdl_wait();
     const int seq = blockIdx.x / Hq, h = blockIdx.x % Hq, e = threadIdx.x;
     float mx = -INFINITY;
     for (int s = e; s < splits; s += 128) {
@@ -651,6 +654,31 @@ __global__ void __launch_bounds__(256) attn_f32_kernel(const float *__restrict__
     if (lse && lane == 0) lse[qi * Hq + h] = l > 0.f ? m + logf(l) : -INFINITY;
 }
 
+// Decode split-KV plan: each sequence's list of top_k + 1 entries (ceil((top_k+1)/8)
+// stages) is cut into `splits` items of S stages; the persistent grid of `cap`
+// CTAs takes ceil(items / cap) rounds.  S minimises rounds x (S + 1) (one stage
+// of start-up per item), ties going to fewer splits.
+struct SplitPlan {
+    int splits, split_blocks;
+};
+
+SplitPlan decode_split_plan(int B, int top_k, int64_t cap) {
+    const int nst = (top_k + 1 + AT_BPS - 1) / AT_BPS;
+    SplitPlan best{1, nst * AT_BPS};
+    int64_t best_cost = -1;
+    for (int S = nst; S >= 1; --S) {
+        const int splits = (nst + S - 1) / S;
+        if (S > 1 && (nst + S - 2) / (S - 1) == splits) continue;   // same splits with a smaller S
+        const int64_t rounds = ((int64_t)B * splits + cap - 1) / cap;
+        const int64_t cost = rounds * (S + 1);
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best = SplitPlan{splits, S * AT_BPS};
+        }
+    }
+    return best;
+}
+
 template <int HKV>
 cudaError_t run_bf16(const AttnArgs &a, void *ws, unsigned *status, cudaStream_t s) {
     using Cfg = AttnCfg<HKV>;
@@ -674,13 +702,10 @@ cudaError_t run_bf16(const AttnArgs &a, void *ws, unsigned *status, cudaStream_t
     p.lse = a.lse;
     p.status = status;
     if (a.decode) {
-        const int list_max = a.top_k + 1;
-        int splits = max(1, (2 * sms + a.B - 1) / a.B);
-        int sb = (list_max + splits - 1) / splits;
-        sb = max(AT_BPS, (sb + AT_BPS - 1) / AT_BPS * AT_BPS);
-        splits = (list_max + sb - 1) / sb;
+        const SplitPlan sp = decode_split_plan(a.B, a.top_k, (int64_t)sms * Cfg::kMinCtas);
+        const int splits = sp.splits;
         p.splits = splits;
-        p.split_blocks = sb;
+        p.split_blocks = sp.split_blocks;
         p.items = (int64_t)a.B * splits;
         float *w = static_cast<float *>(ws);
         p.part_o = w;
@@ -702,25 +727,20 @@ cudaError_t run_bf16(const AttnArgs &a, void *ws, unsigned *status, cudaStream_t
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, attn_bf16_kernel<HKV>, Cfg::kThreads, smem);
     if (e != cudaSuccess) return e;
     const int64_t grid = std::min<int64_t>(p.items, (int64_t)sms * std::max(1, per_sm));
-    attn_bf16_kernel<HKV><<<(unsigned)grid, Cfg::kThreads, smem, s>>>(p);
-    e = cudaGetLastError();
+    e = launch_pdl(attn_bf16_kernel<HKV>, dim3((unsigned)grid), dim3(Cfg::kThreads), smem, s, p);
     if (e != cudaSuccess || !a.decode) return e;
-    attn_combine_kernel<<<(unsigned)(a.B * Cfg::kHq), 128, 0, s>>>(p.part_o, p.part_lse, p.splits, Cfg::kHq,
-                                                                   (__nv_bfloat16 *)a.out, a.lse);
-    return cudaGetLastError();
+    return launch_pdl(attn_combine_kernel, dim3((unsigned)(a.B * Cfg::kHq)), dim3(128), 0, s,
+                      (const float *)p.part_o, (const float *)p.part_lse, p.splits, (int)Cfg::kHq,
+                      (__nv_bfloat16 *)a.out, a.lse);
 }
 
 }  // namespace
 
 size_t attn_decode_ws_bytes(int B, int Hq, int d, int top_k) {
-    // upper bound over the split plans of run_bf16: splits <= top_k + 1
+    // the larger of the split plans run_bf16 can pick (1 or 2 resident CTAs per SM)
     const DeviceInfo *di = device_info();
     const int sms = di ? di->sm_count : 148;
-    const int list_max = top_k + 1;
-    int splits = std::max(1, (2 * sms + B - 1) / B);
-    int sb = (list_max + splits - 1) / splits;
-    sb = std::max(AT_BPS, (sb + AT_BPS - 1) / AT_BPS * AT_BPS);
-    splits = (list_max + sb - 1) / sb;
+    const int splits = std::max(decode_split_plan(B, top_k, sms).splits, decode_split_plan(B, top_k, 2 * sms).splits);
     size_t n = (size_t)B * splits * Hq;
     return (n * d * sizeof(float) + n * sizeof(float) + 255) / 256 * 256;
 }

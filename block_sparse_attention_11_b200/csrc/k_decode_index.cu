@@ -56,6 +56,7 @@ __global__ void __launch_bounds__(DI_THREADS, 2)
     __shared__ float qsum[kIdxDim];
     __shared__ uint32_t lh[2048];
 
+    pdl_trigger();
     const int seq = blockIdx.y, c = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t s_len = p.seq_len[seq];
@@ -208,6 +209,7 @@ __global__ void __launch_bounds__(DI_THREADS, 2)
     extern __shared__ uint8_t dsm_raw[];
     DecodeMmaSmem &sm = *reinterpret_cast<DecodeMmaSmem *>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) &
                                                            ~uintptr_t(1023));
+    pdl_trigger();
     const int seq = blockIdx.y, c = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t s_len = p.seq_len[seq];
@@ -479,6 +481,8 @@ __global__ void __launch_bounds__(DS_THREADS)
     decode_cand_kernel(SelectArgs a) {
     extern __shared__ __align__(16) uint8_t ds_raw[];
     DsSmem &sm = *reinterpret_cast<DsSmem *>(ds_raw);
+    pdl_wait();
+    pdl_trigger();
     const int seq = blockIdx.y, g = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
     const int64_t nb = visible_blocks(a, seq);
     if (nb <= a.top_k) return;                       // everything is selected
@@ -613,6 +617,8 @@ __global__ void __launch_bounds__(DS_THREADS)
 __global__ void __launch_bounds__(DS_THREADS)
     decode_emit_kernel(SelectArgs a) {
     __shared__ uint32_t wsum[DS_THREADS / 32];
+    pdl_wait();
+    pdl_trigger();
     const int seq = blockIdx.y, g = blockIdx.x, tid = threadIdx.x;
     const int64_t nb = visible_blocks(a, seq);
     const int top_k = a.top_k;
@@ -776,11 +782,9 @@ cudaError_t launch_decode_index(const void *q_idx, const void *k_pool, const flo
     const dim3 sgrid((unsigned)l.gmax, (unsigned)B);
     e = cudaFuncSetAttribute(decode_cand_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(DsSmem));
     if (e != cudaSuccess) return e;
-    decode_cand_kernel<<<sgrid, DS_THREADS, sizeof(DsSmem), s>>>(sa);
-    e = cudaGetLastError();
+    e = launch_pdl(decode_cand_kernel, sgrid, dim3(DS_THREADS), sizeof(DsSmem), s, sa);
     if (e != cudaSuccess) return e;
-    decode_emit_kernel<<<sgrid, DS_THREADS, 0, s>>>(sa);
-    return cudaGetLastError();
+    return launch_pdl(decode_emit_kernel, sgrid, dim3(DS_THREADS), 0, s, sa);
 }
 
 }  // namespace qsa

@@ -260,3 +260,50 @@ def test_decode_select_all_ties(qsa, dtype, flags):
         exp = np.full(top_k, -1, np.int32)
         exp[:n] = np.arange(n)
         assert np.array_equal(sel[b].cpu().numpy(), exp), b
+
+
+def test_decode_step_graph_replay_matches_eager(qsa):
+    """A decode step (ring pooling, indexer, attention with caller workspaces)
+    captured in a CUDA graph and replayed gives the eager results bit for bit."""
+    w = workloads.Workload("dec_graph", "decode", 6, 30001, 512, 16, 2, 128, "bf16", 91)
+    x = workloads.make_decode(w, device=DEV, ragged=True)
+    rope = rope_of(w)
+    B = w.B
+    cap = max(x["lens"]) // 4 + 2
+    k_pool = torch.zeros(B, cap, 128, dtype=torch.bfloat16, device=DEV)
+    for b in range(B):
+        kp = torch.zeros(1, cap, 128, dtype=torch.bfloat16, device=DEV)
+        qsa.qsa_pool_keys_prefill(x["k_idx"][b:b + 1, :x["lens"][b]].contiguous(), kp, rope=rope)
+        k_pool[b] = kp[0]
+    ring0 = torch.zeros(B, 4, 128, dtype=torch.bfloat16, device=DEV)
+    max_blocks = cap
+    ws_i = torch.empty(qsa.qsa_index_topk_decode_workspace(B, max_blocks, w.top_k), dtype=torch.uint8, device=DEV)
+    ws_a = torch.empty(qsa.qsa_sparse_attn_decode_workspace(B, w.Hq, w.d, w.top_k), dtype=torch.uint8, device=DEV)
+
+    def step(ring, pool, sel, nsel, out):
+        qsa.qsa_pool_keys_decode(x["k_idx_new"], ring, pool, x["seq_len"], rope=rope)
+        qsa.qsa_index_topk_decode(x["q_idx"], pool, x["seq_len"], sel, nsel, max_blocks=max_blocks, top_k=w.top_k,
+                                  rope=rope, workspace=ws_i)
+        qsa.qsa_sparse_attn_decode(x["q"], x["k"], x["v"], x["seq_len"], sel, nsel, out, workspace=ws_a)
+
+    def buffers():
+        return (ring0.clone(), k_pool.clone(), torch.empty(B, w.top_k, dtype=torch.int32, device=DEV),
+                torch.empty(B, dtype=torch.int32, device=DEV), torch.empty_like(x["q"]))
+
+    eager = buffers()
+    step(*eager)
+    graphed = buffers()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step(*buffers())                        # warm-up outside the capture
+    torch.cuda.current_stream().wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step(*graphed)
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    qsa.qsa_check_status()
+    for a, b in zip(eager, graphed):
+        assert torch.equal(a, b)
