@@ -9,9 +9,10 @@
 // swizzled tensor tiles in bf16 mode where the scores come from warp MMAs),
 // writes one 4-byte order-preserving score key per block to the workspace and
 // adds the chunk's histogram of the keys' top 11 bits into a per-sequence
-// histogram.  The selection then runs over the keys (still in L2) on many CTAs
-// per sequence: a candidate pass that needs only the keys of the histogram bin
-// holding the k-th largest key, and an ordered emission pass.
+// histogram.  The selection then runs over the keys (still in L2) in one pass,
+// one thread-block cluster per sequence: only the keys of the histogram bin
+// holding the k-th largest key need their remaining bits resolved, and one
+// CTA of the cluster assembles the ascending output.
 #include <algorithm>
 
 #include "internal.h"
@@ -192,7 +193,7 @@ __global__ void __launch_bounds__(DI_THREADS, 2)
 // m16n8k16 MMAs: A = keys (16 keys x 16 dims), B = the query as 8 columns
 // (hi and lo planes of the FP32 head sum, or the 4 heads), FP32 accumulate.
 constexpr int DM_ROWS = 128;                       // keys per stage
-constexpr int DM_NS = 2;                           // stages in flight per CTA (2 CTAs per SM)
+constexpr int DM_NS = 3;                           // stages in flight per CTA (2 CTAs per SM)
 constexpr int DM_STAGE_BYTES = DM_ROWS * 256;      // two 64-dim k-atoms of 128 rows x 128 B
 
 struct DecodeMmaSmem {
@@ -382,57 +383,55 @@ bool make_kpool_map(CUtensorMap *map, const void *base, uint64_t rows) {
 }
 
 // ---------------------------------------------------------------------------
-// Selection from the score keys, spread over many CTAs per sequence.
+// Selection from the score keys: one kernel, one thread-block cluster of up to
+// 16 CTAs per sequence.
 //
 // Every CTA owns a chunk of a sequence's keys (whole tiles of DS_TILE keys,
 // 16 contiguous keys per thread, read with four 16-byte loads issued
 // together).  With the top-11-bit histogram from the scorer, the bin d1 that
-// holds the k-th largest key is known before any key is read:
-//   candidate pass  each CTA counts its keys above bin d1 and appends the keys
-//                   of bin d1, with their block ids, to a per-sequence list;
-//                   the last CTA of the sequence to finish (ticket counter)
-//                   resolves the remaining 21 bits of K* on that list, and
-//                   from the list and the per-chunk counts computes each
-//                   chunk's output offset and the number of keys equal to K*
-//                   that precede it;
-//   emission pass   each CTA writes its selected block ids in ascending order
-//                   at its chunk's offset (prefix sums over threads).
+// holds the k-th largest key is known before any key is read.  Each CTA
+// writes to its own shared memory, in block order, the ids of its keys above
+// bin d1 (all of them are selected; fewer than k in the whole sequence) and
+// the (key, id) pairs of its keys in bin d1 (the candidates; past the
+// shared-memory capacity they go to a global overflow area).  After a cluster
+// barrier, CTA 0 gathers the lists through distributed shared memory, resolves
+// the remaining 21 bits of K* on the candidates, keeps the candidates above K*
+// and the first ones equal to K* (ties to the lower block id), and merges that
+// list with the above-bin ids into the ascending output.
 // ---------------------------------------------------------------------------
 constexpr int DS_THREADS = 512;
 constexpr int DS_PER_THREAD = 16;
 constexpr int DS_TILE = DS_THREADS * DS_PER_THREAD;   // keys per CTA tile
-constexpr int DS_MAX_CHUNKS = 2048;                   // chunks per sequence at most
-constexpr int DS_CAND_SMEM = 4096;                    // candidates staged in shared memory
-
-struct SelMeta {           // per sequence; zeroed before the scorer runs
-    uint32_t ncand;        // candidates appended (keys of bin d1)
-    uint32_t done;         // CTAs of the candidate pass that finished
-    uint32_t kstar;        // K*
-    int32_t take_eq;       // keys equal to K* taken, in block order
-};
+constexpr int DS_CLUSTER = 16;                        // CTAs (chunks) per sequence at most (non-portable above 8)
+constexpr int DS_LCAND = 2048;                        // candidates a CTA keeps in shared memory
+constexpr int DS_CAND_SMEM = 4096;                    // candidates CTA 0 stages in shared memory
+constexpr int DS_MAX_K = 2048;                        // largest top_k
 
 struct SelectArgs {
     const int32_t *seq_len;
     int64_t pool_stride, max_blocks, kstride, chunk;   // chunk: keys per CTA, a multiple of DS_TILE
-    int gmax, top_k;
-    const uint32_t *keys;   // [B][kstride]
-    const uint32_t *hist;   // [B][2048]
-    SelMeta *meta;          // [B]
-    uint2 *cand;            // [B][kstride] (key, block id)
-    uint32_t *cnt_gt;       // [B][gmax] keys above bin d1 per chunk
-    int2 *plan;             // [B][gmax] (output offset, keys == K* before the chunk)
+    int gmax, top_k;                                    // gmax: CTAs per cluster (<= DS_CLUSTER)
+    const uint32_t *keys;   // [B][kstride] score keys
+    const uint32_t *hist;   // [B][2048] histogram of the keys' top 11 bits
+    uint2 *cand;            // [B][kstride]: chunk g's candidates past DS_LCAND, at g * chunk + position
     int32_t *sel, *nsel;
 };
 
 struct DsSmem {
-    SelectSmem s;
-    uint32_t ck[DS_CAND_SMEM];
-    uint32_t ci[DS_CAND_SMEM];
-    uint32_t gtc[DS_MAX_CHUNKS];
-    uint32_t eqc[DS_MAX_CHUNKS];
+    SelectSmem s;                       // histogram, warp partials, digit search results
+    // this CTA's lists (read by CTA 0 through distributed shared memory)
+    int32_t my_above[DS_MAX_K];
+    uint32_t my_ck[DS_LCAND];
+    uint32_t my_ci[DS_LCAND];
+    uint32_t my_na, my_nc;
+    // CTA 0
+    uint32_t ck[DS_CAND_SMEM];          // candidate keys (block order)
+    uint32_t ci[DS_CAND_SMEM];          // candidate block ids
+    int32_t alist[DS_MAX_K];            // ids above bin d1 (ascending)
+    int32_t slist[DS_MAX_K];            // selected candidate ids (ascending)
+    uint32_t aoff[DS_CLUSTER + 1];      // prefix of the above counts per chunk
+    uint32_t coff[DS_CLUSTER + 1];      // prefix of the candidate counts per chunk
     uint32_t wsum[DS_THREADS / 32];
-    uint32_t wsum2[DS_THREADS / 32];
-    int last;
 };
 
 __device__ __forceinline__ int64_t visible_blocks(const SelectArgs &a, int seq) {
@@ -466,208 +465,220 @@ __device__ __forceinline__ uint32_t cta_scan(uint32_t v, uint32_t *wsum, uint32_
     }
     if (lane == 31) wsum[warp] = x;
     __syncthreads();
-    uint32_t off = 0, tot = 0;
-    for (int w = 0; w < nw; ++w) {
-        const uint32_t t = wsum[w];
-        if (w < warp) off += t;
-        tot += t;
-    }
+    const uint32_t wv = lane < nw ? wsum[lane] : 0u;     // lane l: warp l's total (nw <= 32)
+    const uint32_t off = __reduce_add_sync(0xffffffffu, lane < warp ? wv : 0u);
+    total = __reduce_add_sync(0xffffffffu, wv);
     __syncthreads();
-    total = tot;
     return off + x - v;
 }
 
+// Largest g < n with off[g] <= j (off ascending): the chunk that holds entry j.
+__device__ __forceinline__ int chunk_of(const uint32_t *off, int n, uint32_t j) {
+    int g = 0;
+    for (int c = 1; c < n; ++c) g = off[c] <= j ? c : g;
+    return g;
+}
+
+// Entries of the ascending list l[0..n) that are smaller than v.
+__device__ __forceinline__ int count_below(const int32_t *l, int n, int32_t v) {
+    int lo = 0, hi = n;
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (l[mid] < v) lo = mid + 1;
+        else hi = mid;
+    }
+    return lo;
+}
+
 __global__ void __launch_bounds__(DS_THREADS)
-    decode_cand_kernel(SelectArgs a) {
+    decode_select_kernel(SelectArgs a) {
     extern __shared__ __align__(16) uint8_t ds_raw[];
     DsSmem &sm = *reinterpret_cast<DsSmem *>(ds_raw);
     pdl_wait();
     pdl_trigger();
-    const int seq = blockIdx.y, g = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
-    const int64_t nb = visible_blocks(a, seq);
-    if (nb <= a.top_k) return;                       // everything is selected
-    const int gseq = (int)((nb + a.chunk - 1) / a.chunk);
-    if (g >= gseq) return;
-    const uint32_t *row = a.keys + (int64_t)seq * a.kstride;
-    uint2 *cand = a.cand + (int64_t)seq * a.kstride;
-    SelMeta &meta = a.meta[seq];
-    // bin of the k-th largest key from the scorer's histogram
-    for (int b = tid; b < 2048; b += DS_THREADS) sm.s.hist[b] = __ldcg(a.hist + (int64_t)seq * 2048 + b);
-    if (tid == 0) { sm.s.digit = 0; sm.s.k_rem = 1; }
-    __syncthreads();
-    sel_find_digit(sm.s, 2048, a.top_k);
-    const uint32_t d1 = (uint32_t)sm.s.digit;
-    const int k_rem1 = sm.s.k_rem;
-
-    const int64_t c0 = (int64_t)g * a.chunk, c1 = min(c0 + a.chunk, nb);
-    uint32_t n_gt = 0;
-    for (int64_t t0 = c0; t0 < c1; t0 += DS_TILE) {
-        uint32_t k[16];
-        const int64_t i0 = t0 + (int64_t)DS_PER_THREAD * tid;
-        const int m = load16(row, i0, c1, a.kstride, k);
-        uint32_t ce = 0;
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            const uint32_t dg = k[j] >> 21;
-            if (j < m) { n_gt += dg > d1; ce += dg == d1; }
-        }
-        // warp-level append of the bin-d1 keys
-        uint32_t x = ce;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-            if (lane >= o) x += y;
-        }
-        uint32_t base = 0;
-        if (lane == 31 && x) base = atomicAdd(&meta.ncand, x);
-        base = __shfl_sync(0xffffffffu, base, 31) + x - ce;
-        if (ce) {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                if (j < m && (k[j] >> 21) == d1) {
-                    if (base < (uint64_t)a.kstride) cand[base] = make_uint2(k[j], (uint32_t)(i0 + j));
-                    ++base;
-                }
-            }
-        }
-    }
-    uint32_t tot;
-    cta_scan(n_gt, sm.wsum, tot);
-    if (tid == 0) a.cnt_gt[(int64_t)seq * a.gmax + g] = tot;
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) sm.last = atomicAdd(&meta.done, 1u) == (uint32_t)(gseq - 1);
-    __syncthreads();
-    if (!sm.last) return;
-    __threadfence();
-
-    // ---- last CTA of this sequence: K* from the candidates, then the chunk plan
-    const int nc = (int)min((int64_t)__ldcg(&meta.ncand), nb);
-    const bool small = nc <= DS_CAND_SMEM;
-    if (small)
-        for (int i = tid; i < nc; i += DS_THREADS) {
-            const uint2 c = __ldcg(cand + i);
-            sm.ck[i] = c.x;
-            sm.ci[i] = c.y;
-        }
-    uint32_t prefix = d1 << 21, pmask = 0xFFE00000u;
-    int k_rem = k_rem1;
-#pragma unroll 1
-    for (int pass = 0; pass < 2; ++pass) {
-        const int shift = pass == 0 ? 10 : 0, nbins = pass == 0 ? 2048 : 1024;
-        const uint32_t mask = (uint32_t)nbins - 1u;
-        for (int b = tid; b < nbins; b += DS_THREADS) sm.s.hist[b] = 0;
-        __syncthreads();
-        for (int i = tid; i < nc; i += DS_THREADS) {
-            const uint32_t key = small ? sm.ck[i] : __ldcg(&cand[i].x);
-            if ((key & pmask) == prefix) atomicAdd(&sm.s.hist[(key >> shift) & mask], 1u);
-        }
-        __syncthreads();
-        sel_find_digit(sm.s, nbins, k_rem);
-        prefix |= (uint32_t)sm.s.digit << shift;
-        pmask |= mask << shift;
-        k_rem = sm.s.k_rem;
-        __syncthreads();
-    }
-    const uint32_t kstar = prefix;
-    const int take_eq = k_rem;
-    for (int i = tid; i < gseq; i += DS_THREADS) { sm.gtc[i] = 0; sm.eqc[i] = 0; }
-    __syncthreads();
-    for (int i = tid; i < nc; i += DS_THREADS) {
-        uint32_t key, id;
-        if (small) { key = sm.ck[i]; id = sm.ci[i]; }
-        else { const uint2 c = __ldcg(cand + i); key = c.x; id = c.y; }
-        const int gc = (int)min((int64_t)id / a.chunk, (int64_t)gseq - 1);
-        if (key > kstar) atomicAdd(&sm.gtc[gc], 1u);
-        else if (key == kstar) atomicAdd(&sm.eqc[gc], 1u);
-    }
-    __syncthreads();
-    // chunk plan: thread t owns chunks [per*t, per*t + per)
-    const int per = (gseq + DS_THREADS - 1) / DS_THREADS;
-    const int g0 = min(per * tid, gseq), g1 = min(g0 + per, gseq);
-    uint32_t eq_mine = 0;
-    for (int c = g0; c < g1; ++c) eq_mine += sm.eqc[c];
-    uint32_t eq_tot;
-    uint32_t eq_run = cta_scan(eq_mine, sm.wsum, eq_tot);
-    uint32_t s_mine = 0;
-    {
-        uint32_t e = eq_run;
-        for (int c = g0; c < g1; ++c) {
-            const uint32_t gt = __ldcg(a.cnt_gt + (int64_t)seq * a.gmax + c) + sm.gtc[c];
-            const int avail = max(0, take_eq - (int)e);
-            s_mine += gt + min((uint32_t)avail, sm.eqc[c]);
-            e += sm.eqc[c];
-        }
-    }
-    uint32_t s_tot;
-    uint32_t out_run = cta_scan(s_mine, sm.wsum2, s_tot);
-    for (int c = g0; c < g1; ++c) {
-        const uint32_t gt = __ldcg(a.cnt_gt + (int64_t)seq * a.gmax + c) + sm.gtc[c];
-        a.plan[(int64_t)seq * a.gmax + c] = make_int2((int)out_run, (int)eq_run);
-        const int avail = max(0, take_eq - (int)eq_run);
-        out_run += gt + min((uint32_t)avail, sm.eqc[c]);
-        eq_run += sm.eqc[c];
-    }
-    if (tid == 0) {
-        meta.kstar = kstar;
-        meta.take_eq = take_eq;
-    }
-}
-
-__global__ void __launch_bounds__(DS_THREADS)
-    decode_emit_kernel(SelectArgs a) {
-    __shared__ uint32_t wsum[DS_THREADS / 32];
-    pdl_wait();
-    pdl_trigger();
-    const int seq = blockIdx.y, g = blockIdx.x, tid = threadIdx.x;
+    const int seq = blockIdx.y, tid = threadIdx.x;
+    const uint32_t rank = cluster_rank();             // = blockIdx.x: a cluster spans the x extent
     const int64_t nb = visible_blocks(a, seq);
     const int top_k = a.top_k;
     int32_t *out = a.sel + (int64_t)seq * top_k;
-    const int cnt = (int)min(nb, (int64_t)top_k);
-    if (g == 0) {
-        if (tid == 0) a.nsel[seq] = cnt;
-        for (int i = cnt + tid; i < top_k; i += DS_THREADS) out[i] = -1;
-    }
-    const int64_t c0 = (int64_t)g * a.chunk, c1 = min(c0 + a.chunk, nb);
-    if (c0 >= c1) return;
-    if (nb <= top_k) {                               // every visible block, in order
+    const int64_t c0 = (int64_t)rank * a.chunk, c1 = min(c0 + a.chunk, nb);
+    if (nb <= top_k) {                               // every visible block, in order (whole cluster)
         for (int64_t i = c0 + tid; i < c1; i += DS_THREADS) out[i] = (int32_t)i;
+        if (rank == 0) {
+            for (int i = (int)nb + tid; i < top_k; i += DS_THREADS) out[i] = -1;
+            if (tid == 0) a.nsel[seq] = (int)nb;
+        }
         return;
     }
+    const int gseq = (int)((nb + a.chunk - 1) / a.chunk);   // CTAs with keys (<= cluster size)
     const uint32_t *row = a.keys + (int64_t)seq * a.kstride;
-    const uint32_t kstar = a.meta[seq].kstar;
-    const int take_eq = a.meta[seq].take_eq;
-    const int2 pl = a.plan[(int64_t)seq * a.gmax + g];
-    int64_t o_run = pl.x, e_run = pl.y;              // output slots and keys == K* before this tile
+    uint2 *cand_seq = a.cand + (int64_t)seq * a.kstride;
+    // first tile's keys in flight before the histogram is read
+    uint32_t k[16];
+    int m = load16(row, c0 + (int64_t)DS_PER_THREAD * tid, c1, a.kstride, k);
+    // bin of the k-th largest key from the scorer's histogram
+    static_assert(DS_THREADS * 4 == 2048, "one 16-byte histogram load per thread");
+    reinterpret_cast<uint4 *>(sm.s.hist)[tid] = __ldcg(reinterpret_cast<const uint4 *>(a.hist + (int64_t)seq * 2048) + tid);
+    if (tid == 0) { sm.s.digit = 0; sm.s.k_rem = 1; }
+    __syncthreads();
+    sel_find_digit(sm.s, 2048, top_k);
+    const uint32_t d1 = (uint32_t)sm.s.digit;
+    const int k_rem1 = sm.s.k_rem;
+
+    uint32_t na_run = 0, nc_run = 0;
     for (int64_t t0 = c0; t0 < c1; t0 += DS_TILE) {
-        uint32_t k[16];
         const int64_t i0 = t0 + (int64_t)DS_PER_THREAD * tid;
-        const int m = load16(row, i0, c1, a.kstride, k);
-        uint32_t gt = 0, eq = 0;
+        if (t0 != c0) m = load16(row, i0, c1, a.kstride, k);
+        uint32_t na = 0, nc = 0;
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-            if (j < m) { gt += k[j] > kstar; eq += k[j] == kstar; }
+        for (int j = 0; j < 16; ++j) {
+            const uint32_t dg = k[j] >> 21;
+            if (j < m) { na += dg > d1; nc += dg == d1; }
+        }
         uint32_t tot;
-        const uint32_t ex = cta_scan(gt | (eq << 16), wsum, tot);
-        const int64_t avail = max((int64_t)0, (int64_t)take_eq - e_run);
-        const int64_t eq_before = ex >> 16;
-        int64_t pos = o_run + (ex & 0xFFFFu) + min(avail, eq_before);
-        int64_t r = e_run + eq_before;
-        if (gt | eq) {
+        const uint32_t ex = cta_scan(na | (nc << 16), sm.wsum, tot);
+        uint32_t pa = na_run + (ex & 0xFFFFu), pc = nc_run + (ex >> 16);
+        if (na | nc) {
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
                 if (j >= m) continue;
-                bool take = k[j] > kstar;
-                if (k[j] == kstar) take = r++ < take_eq;
-                if (take) {
-                    if (pos >= 0 && pos < top_k) out[pos] = (int32_t)(i0 + j);
-                    ++pos;
+                const uint32_t dg = k[j] >> 21;
+                if (dg > d1) {
+                    if (pa < (uint32_t)DS_MAX_K) sm.my_above[pa] = (int32_t)(i0 + j);
+                    ++pa;
+                } else if (dg == d1) {
+                    if (pc < (uint32_t)DS_LCAND) { sm.my_ck[pc] = k[j]; sm.my_ci[pc] = (uint32_t)(i0 + j); }
+                    else cand_seq[c0 + pc] = make_uint2(k[j], (uint32_t)(i0 + j));   // pc < c1 - c0
+                    ++pc;
                 }
             }
         }
-        o_run += (tot & 0xFFFFu) + min(avail, (int64_t)(tot >> 16));
-        e_run += tot >> 16;
+        na_run += tot & 0xFFFFu;
+        nc_run += tot >> 16;
     }
+    if (tid == 0) {
+        sm.my_na = min(na_run, (uint32_t)min(top_k - 1, DS_MAX_K));
+        sm.my_nc = nc_run;
+    }
+    cluster_sync();                                  // every CTA's lists are complete
+    if (rank == 0) {
+        // per-chunk offsets of the above ids and of the candidates
+        if (tid == 0) {
+            uint32_t ea = 0, ec = 0;
+            for (int c = 0; c < gseq; ++c) {
+                sm.aoff[c] = ea;
+                sm.coff[c] = ec;
+                ea += ld_dsmem(dsmem_addr(&sm.my_na, c));
+                ec += ld_dsmem(dsmem_addr(&sm.my_nc, c));
+            }
+            sm.aoff[gseq] = ea;
+            sm.coff[gseq] = ec;
+        }
+        __syncthreads();
+        const int na_all = (int)min(sm.aoff[gseq], (uint32_t)(top_k - 1));
+        const int nc_all = (int)min((int64_t)sm.coff[gseq], nb);
+        const bool small = nc_all <= DS_CAND_SMEM;
+        for (int j = tid; j < na_all; j += DS_THREADS) {
+            const int c = chunk_of(sm.aoff, gseq, (uint32_t)j);
+            sm.alist[j] = (int32_t)ld_dsmem(dsmem_addr(&sm.my_above[j - sm.aoff[c]], c));
+        }
+        auto fetch = [&](int j) -> uint2 {           // candidate j of the sequence, block order
+            const int c = chunk_of(sm.coff, gseq, (uint32_t)j);
+            const uint32_t jj = (uint32_t)j - sm.coff[c];
+            if (jj < (uint32_t)DS_LCAND)
+                return make_uint2(ld_dsmem(dsmem_addr(&sm.my_ck[jj], c)), ld_dsmem(dsmem_addr(&sm.my_ci[jj], c)));
+            return __ldcg(cand_seq + (int64_t)c * a.chunk + jj);
+        };
+        if (small)
+            for (int j = tid; j < nc_all; j += DS_THREADS) {
+                const uint2 v = fetch(j);
+                sm.ck[j] = v.x;
+                sm.ci[j] = v.y;
+            }
+        __syncthreads();
+        auto cand_at = [&](int j) -> uint2 { return small ? make_uint2(sm.ck[j], sm.ci[j]) : fetch(j); };
+        // remaining 21 bits of K*: bits 20..10, then 9..0
+        uint32_t prefix = d1 << 21, pmask = 0xFFE00000u;
+        int k_rem = k_rem1;
+#pragma unroll 1
+        for (int pass = 0; pass < 2; ++pass) {
+            const int shift = pass == 0 ? 10 : 0, nbins = pass == 0 ? 2048 : 1024;
+            const uint32_t mask = (uint32_t)nbins - 1u;
+            for (int b = tid; b < nbins; b += DS_THREADS) sm.s.hist[b] = 0;
+            __syncthreads();
+            for (int j = tid; j < nc_all; j += DS_THREADS) {
+                const uint32_t key = cand_at(j).x;
+                if ((key & pmask) == prefix) atomicAdd(&sm.s.hist[(key >> shift) & mask], 1u);
+            }
+            __syncthreads();
+            sel_find_digit(sm.s, nbins, k_rem);
+            prefix |= (uint32_t)sm.s.digit << shift;
+            pmask |= mask << shift;
+            k_rem = sm.s.k_rem;
+            __syncthreads();
+        }
+        const uint32_t kstar = prefix;
+        const int take_eq = k_rem;
+        // selected candidates in block order: keys above K*, and the first take_eq equal to K*
+        int ns = 0;     // CTA-uniform running count
+        uint32_t eq_run = 0;
+        for (int base = 0; base < nc_all; base += DS_THREADS * 8) {
+            const int j0 = base + 8 * tid;
+            uint32_t ke[8], id[8];
+            uint32_t eq = 0;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                ke[q] = 0u;
+                id[q] = 0u;
+                if (j0 + q < nc_all) {
+                    const uint2 v = cand_at(j0 + q);
+                    ke[q] = v.x;
+                    id[q] = v.y;
+                    eq += v.x == kstar;
+                }
+            }
+            uint32_t eq_tot;
+            uint32_t r = eq_run + cta_scan(eq, sm.wsum, eq_tot);
+            uint32_t nsel_mine = 0;
+            bool take[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                take[q] = false;
+                if (j0 + q < nc_all) {
+                    if (ke[q] > kstar) take[q] = true;
+                    else if (ke[q] == kstar) take[q] = r++ < (uint32_t)take_eq;
+                }
+                nsel_mine += take[q];
+            }
+            uint32_t s_tot;
+            uint32_t pos = (uint32_t)ns + cta_scan(nsel_mine, sm.wsum, s_tot);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                if (take[q]) {
+                    if (pos < (uint32_t)DS_MAX_K) sm.slist[pos] = (int32_t)id[q];
+                    ++pos;
+                }
+            ns += (int)s_tot;
+            eq_run += eq_tot;
+        }
+        ns = min(ns, top_k - na_all);
+        __syncthreads();
+        // merge the two ascending lists into the output
+        for (int j = tid; j < na_all; j += DS_THREADS) {
+            const int32_t v = sm.alist[j];
+            const int pos = j + count_below(sm.slist, ns, v);
+            if (pos < top_k) out[pos] = v;
+        }
+        for (int j = tid; j < ns; j += DS_THREADS) {
+            const int32_t v = sm.slist[j];
+            const int pos = j + count_below(sm.alist, na_all, v);
+            if (pos < top_k) out[pos] = v;
+        }
+        const int cnt = na_all + ns;
+        for (int i = cnt + tid; i < top_k; i += DS_THREADS) out[i] = -1;
+        if (tid == 0) a.nsel[seq] = cnt;
+    }
+    cluster_sync();                                  // CTA 0 has finished reading the others' lists
 }
 
 }  // namespace
@@ -677,8 +688,10 @@ DecodePlan decode_index_plan(int B, int64_t max_blocks, bool bf16) {
     const DeviceInfo *di = device_info();
     const int sms = di ? di->sm_count : 148;
     DecodePlan pl;
-    // about two CTAs per SM over all sequences, chunks of at least 512 blocks
-    int64_t C = std::max<int64_t>(1, (2 * sms + B - 1) / std::max(B, 1));
+    // at most two CTAs per SM over all sequences (one wave: a second, partial
+    // wave would stream its chunks with a fraction of the SMs), chunks of at
+    // least 512 blocks
+    int64_t C = std::max<int64_t>(1, (2 * sms) / std::max(B, 1));
     C = std::min<int64_t>(C, std::max<int64_t>(1, (max_blocks + 511) / 512));
     int64_t chunk = (max_blocks + C - 1) / C;
     chunk = std::max<int64_t>(128, (chunk + 127) / 128 * 128);
@@ -697,31 +710,59 @@ struct SelectLayout {
     int gmax;
 };
 
+// Whether clusters of 16 CTAs of the select kernel can be resident (checked once).
+bool cluster16_ok();
+
+// Chunks of whole tiles, at most DS_CLUSTER per sequence (8 where 16 cannot run).
 SelectLayout select_layout(int64_t max_blocks) {
     const int64_t tiles = std::max<int64_t>(1, (max_blocks + DS_TILE - 1) / DS_TILE);
-    const int64_t tiles_per_chunk = (tiles + DS_MAX_CHUNKS - 1) / DS_MAX_CHUNKS;
+    const int64_t cmax = (tiles > 8 && cluster16_ok()) ? DS_CLUSTER : 8;
+    const int64_t tiles_per_chunk = (tiles + cmax - 1) / cmax;
     SelectLayout l;
     l.chunk = tiles_per_chunk * DS_TILE;
     l.gmax = (int)((tiles + tiles_per_chunk - 1) / tiles_per_chunk);
     return l;
 }
 
-// Workspace: keys [B][kstride] u32 | cand [B][kstride] uint2 | hist [B][2048] u32 + meta [B] |
-//            cnt_gt [B][gmax] u32 | plan [B][gmax] int2
+bool cluster16_ok() {
+    static int ok = -1;
+    if (ok < 0) {
+        ok = 0;
+        if (cudaFuncSetAttribute(decode_select_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+                cudaSuccess &&
+            cudaFuncSetAttribute(decode_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)sizeof(DsSmem)) == cudaSuccess) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(DS_CLUSTER, 1, 1);
+            cfg.blockDim = dim3(DS_THREADS, 1, 1);
+            cfg.dynamicSmemBytes = sizeof(DsSmem);
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = DS_CLUSTER;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, decode_select_kernel, &cfg) == cudaSuccess && n > 0) ok = 1;
+        }
+        cudaGetLastError();   // a refused query leaves no sticky error
+    }
+    return ok == 1;
+}
+
+// Workspace: keys [B][kstride] u32 | cand overflow [B][kstride] uint2 | hist [B][2048] u32
 struct DecodeWs {
     uint32_t *keys;
     uint2 *cand;
     uint32_t *hist;
-    SelMeta *meta;
-    uint32_t *cnt_gt;
-    int2 *plan;
-    size_t zero_bytes;   // hist + meta, cleared before every call
+    size_t zero_bytes;   // hist, cleared before every call
     size_t total;
 };
 
-DecodeWs decode_ws(void *base, int B, int64_t max_blocks) {
+DecodeWs decode_ws(void *base, int B, int64_t max_blocks, int top_k) {
+    (void)top_k;
     const int64_t ks = key_stride(max_blocks);
-    const SelectLayout l = select_layout(max_blocks);
     uint8_t *w = static_cast<uint8_t *>(base);
     DecodeWs d;
     size_t off = 0;
@@ -730,22 +771,16 @@ DecodeWs decode_ws(void *base, int B, int64_t max_blocks) {
     d.cand = reinterpret_cast<uint2 *>(w + off);
     off += r256((size_t)B * ks * 8);
     d.hist = reinterpret_cast<uint32_t *>(w + off);
-    d.meta = reinterpret_cast<SelMeta *>(w + off + (size_t)B * 2048 * 4);
-    d.zero_bytes = (size_t)B * 2048 * 4 + (size_t)B * sizeof(SelMeta);
+    d.zero_bytes = (size_t)B * 2048 * 4;
     off += r256(d.zero_bytes);
-    d.cnt_gt = reinterpret_cast<uint32_t *>(w + off);
-    off += r256((size_t)B * l.gmax * 4);
-    d.plan = reinterpret_cast<int2 *>(w + off);
-    off += r256((size_t)B * l.gmax * 8);
     d.total = off;
     return d;
 }
 }  // namespace
 
 size_t decode_index_ws_bytes(int B, int64_t max_blocks, int top_k, bool bf16) {
-    (void)top_k;
     (void)bf16;
-    return decode_ws(nullptr, B, max_blocks).total;
+    return decode_ws(nullptr, B, max_blocks, top_k).total;
 }
 
 cudaError_t launch_decode_index(const void *q_idx, const void *k_pool, const float *head_w,
@@ -754,7 +789,7 @@ cudaError_t launch_decode_index(const void *q_idx, const void *k_pool, const flo
                                 bool bf16, unsigned *status, cudaStream_t s) {
     const DecodePlan pl = decode_index_plan(B, max_blocks, bf16);
     const int64_t kstride = key_stride(max_blocks);
-    const DecodeWs d = decode_ws(ws, B, max_blocks);
+    const DecodeWs d = decode_ws(ws, B, max_blocks, top_k);
     cudaError_t e = cudaMemsetAsync(d.hist, 0, d.zero_bytes, s);
     if (e != cudaSuccess) return e;
     DecodeParams p{seq_len, head_w, pool_stride, max_blocks, pl.chunk, kstride, pl.chunks, top_k, relu ? 1 : 0,
@@ -777,14 +812,16 @@ cudaError_t launch_decode_index(const void *q_idx, const void *k_pool, const flo
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const SelectLayout l = select_layout(max_blocks);
-    SelectArgs sa{seq_len, pool_stride, max_blocks, kstride, l.chunk, l.gmax, top_k, d.keys, d.hist, d.meta,
-                  d.cand, d.cnt_gt, d.plan, sel, nsel};
+    SelectArgs sa{seq_len, pool_stride, max_blocks, kstride, l.chunk, l.gmax, top_k, d.keys, d.hist, d.cand, sel,
+                  nsel};
     const dim3 sgrid((unsigned)l.gmax, (unsigned)B);
-    e = cudaFuncSetAttribute(decode_cand_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(DsSmem));
+    e = cudaFuncSetAttribute(decode_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(DsSmem));
     if (e != cudaSuccess) return e;
-    e = launch_pdl(decode_cand_kernel, sgrid, dim3(DS_THREADS), sizeof(DsSmem), s, sa);
-    if (e != cudaSuccess) return e;
-    return launch_pdl(decode_emit_kernel, sgrid, dim3(DS_THREADS), 0, s, sa);
+    if (l.gmax > 8) {
+        e = cudaFuncSetAttribute(decode_select_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+    }
+    return launch_pdl_cluster(decode_select_kernel, sgrid, dim3(DS_THREADS), sizeof(DsSmem), (unsigned)l.gmax, s, sa);
 }
 
 }  // namespace qsa

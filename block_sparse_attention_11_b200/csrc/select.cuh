@@ -55,8 +55,9 @@ __device__ __forceinline__ void sel_find_digit(SelectSmem &sm, int nbins, int k_
     }
     if (lane == 0) sm.warp_eq[warp] = incl;   // warp total
     __syncthreads();
-    uint32_t cum = incl - mine;
-    for (int w = warp + 1; w < nwarps; ++w) cum += sm.warp_eq[w];
+    // count in the warps above this one: lane l holds warp l's total (nwarps <= 32)
+    const uint32_t wv = lane < nwarps ? sm.warp_eq[lane] : 0u;
+    uint32_t cum = incl - mine + __reduce_add_sync(0xffffffffu, lane > warp ? wv : 0u);
     if (cum < (uint32_t)k_rem && cum + mine >= (uint32_t)k_rem) {
         for (int b = per - 1; b >= 0; --b) {
             const uint32_t h = sm.hist[per * tid + b];
