@@ -529,27 +529,36 @@ __global__ void __launch_bounds__(DS_THREADS)
     for (int64_t t0 = c0; t0 < c1; t0 += DS_TILE) {
         const int64_t i0 = t0 + (int64_t)DS_PER_THREAD * tid;
         if (t0 != c0) m = load16(row, i0, c1, a.kstride, k);
-        uint32_t na = 0, nc = 0;
+        // bit j: key j lies above bin d1 (amask) or in it (cmask); few keys do
+        uint32_t amask = 0, cmask = 0;
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
             const uint32_t dg = k[j] >> 21;
-            if (j < m) { na += dg > d1; nc += dg == d1; }
+            amask |= (uint32_t)(dg > d1) << j;
+            cmask |= (uint32_t)(dg == d1) << j;
         }
+        const uint32_t valid = m >= 16 ? 0xFFFFu : ((1u << m) - 1u);
+        amask &= valid;
+        cmask &= valid;
         uint32_t tot;
-        const uint32_t ex = cta_scan(na | (nc << 16), sm.wsum, tot);
+        const uint32_t ex = cta_scan(__popc(amask) | (__popc(cmask) << 16), sm.wsum, tot);
         uint32_t pa = na_run + (ex & 0xFFFFu), pc = nc_run + (ex >> 16);
-        if (na | nc) {
+        const uint32_t any = amask | cmask;
+        if (any) {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                if (j >= m) continue;
-                const uint32_t dg = k[j] >> 21;
-                if (dg > d1) {
-                    if (pa < (uint32_t)DS_MAX_K) sm.my_above[pa] = (int32_t)(i0 + j);
-                    ++pa;
-                } else if (dg == d1) {
-                    if (pc < (uint32_t)DS_LCAND) { sm.my_ck[pc] = k[j]; sm.my_ci[pc] = (uint32_t)(i0 + j); }
-                    else cand_seq[c0 + pc] = make_uint2(k[j], (uint32_t)(i0 + j));   // pc < c1 - c0
-                    ++pc;
+            for (int q = 0; q < 4; ++q) {
+                if (((any >> (4 * q)) & 0xFu) == 0) continue;
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    const int j = 4 * q + jj;
+                    if ((amask >> j) & 1u) {
+                        if (pa < (uint32_t)DS_MAX_K) sm.my_above[pa] = (int32_t)(i0 + j);
+                        ++pa;
+                    } else if ((cmask >> j) & 1u) {
+                        if (pc < (uint32_t)DS_LCAND) { sm.my_ck[pc] = k[j]; sm.my_ci[pc] = (uint32_t)(i0 + j); }
+                        else cand_seq[c0 + pc] = make_uint2(k[j], (uint32_t)(i0 + j));   // pc < c1 - c0
+                        ++pc;
+                    }
                 }
             }
         }
@@ -619,45 +628,32 @@ __global__ void __launch_bounds__(DS_THREADS)
         }
         const uint32_t kstar = prefix;
         const int take_eq = k_rem;
-        // selected candidates in block order: keys above K*, and the first take_eq equal to K*
+        // selected candidates in block order: keys above K*, and the first take_eq equal to K*.
+        // Thread t takes a contiguous run of cpt candidates per round of DS_THREADS * cpt.
         int ns = 0;     // CTA-uniform running count
         uint32_t eq_run = 0;
-        for (int base = 0; base < nc_all; base += DS_THREADS * 8) {
-            const int j0 = base + 8 * tid;
-            uint32_t ke[8], id[8];
+        const int cpt = min(8, max(1, (nc_all + DS_THREADS - 1) / DS_THREADS));
+        for (int base = 0; base < nc_all; base += DS_THREADS * cpt) {
+            const int j0 = base + cpt * tid, j1 = min(j0 + cpt, nc_all);
             uint32_t eq = 0;
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                ke[q] = 0u;
-                id[q] = 0u;
-                if (j0 + q < nc_all) {
-                    const uint2 v = cand_at(j0 + q);
-                    ke[q] = v.x;
-                    id[q] = v.y;
-                    eq += v.x == kstar;
-                }
-            }
+            for (int j = j0; j < j1; ++j) eq += cand_at(j).x == kstar;
             uint32_t eq_tot;
-            uint32_t r = eq_run + cta_scan(eq, sm.wsum, eq_tot);
-            uint32_t nsel_mine = 0;
-            bool take[8];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                take[q] = false;
-                if (j0 + q < nc_all) {
-                    if (ke[q] > kstar) take[q] = true;
-                    else if (ke[q] == kstar) take[q] = r++ < (uint32_t)take_eq;
-                }
-                nsel_mine += take[q];
+            const uint32_t r0 = eq_run + cta_scan(eq, sm.wsum, eq_tot);   // rank of my first key == K*
+            uint32_t r = r0, nsel_mine = 0;
+            for (int j = j0; j < j1; ++j) {
+                const uint32_t key = cand_at(j).x;
+                nsel_mine += key > kstar || (key == kstar && r++ < (uint32_t)take_eq);
             }
             uint32_t s_tot;
             uint32_t pos = (uint32_t)ns + cta_scan(nsel_mine, sm.wsum, s_tot);
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-                if (take[q]) {
-                    if (pos < (uint32_t)DS_MAX_K) sm.slist[pos] = (int32_t)id[q];
+            r = r0;
+            for (int j = j0; j < j1; ++j) {
+                const uint2 v = cand_at(j);
+                if (v.x > kstar || (v.x == kstar && r++ < (uint32_t)take_eq)) {
+                    if (pos < (uint32_t)DS_MAX_K) sm.slist[pos] = (int32_t)v.y;
                     ++pos;
                 }
+            }
             ns += (int)s_tot;
             eq_run += eq_tot;
         }
