@@ -41,6 +41,47 @@ FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1
 L2_BYTES = 126 * 1024 * 1024
 
 
+PROFILES = os.path.join(ROOT, "profiles")
+CSRC = os.path.join(ROOT, "block_sparse_attention_11_b200", "csrc")
+# ncu summary holding the DRAM traffic of each roofline kernel, and the sources it was built from
+TRAFFIC_PROFILE = {
+    "prefill": ("attn_bf16_prefill_t32k.md", ["k_attn.cu", "common.cuh", "internal.h"]),
+    "decode": ("decode_indexer_b64_l128k.md", ["k_decode_index.cu", "select.cuh", "common.cuh", "internal.h"]),
+}
+
+
+def source_digest(files):
+    import hashlib
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(CSRC, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def profiled_traffic(kind, workload):
+    """DRAM bytes per launch from the committed ncu summary, or None when the
+    summary is missing, covers another workload, or the kernel sources changed
+    since it was captured."""
+    name, files = TRAFFIC_PROFILE[kind]
+    try:
+        with open(os.path.join(PROFILES, name)) as f:
+            txt = f.read()
+    except OSError:
+        return None
+    fields = {}
+    for line in txt.splitlines():
+        if line.startswith("- ") and ": " in line:
+            k, v = line[2:].split(": ", 1)
+            fields[k.strip().strip("`")] = v.strip().strip("`")
+    try:
+        if fields.get("workload") != workload or fields.get("source_sha256") != source_digest(files):
+            return None
+        return float(fields["traffic_bytes_per_launch"])
+    except (KeyError, ValueError, OSError):
+        return None
+
+
 def peaks():
     try:
         with open(PEAKS_PATH) as f:
@@ -224,7 +265,7 @@ class DecodeRunner:
         return self.out
 
     def launches_per_step(self):
-        return 6   # ring pool, decode scorer, candidate select, ordered emission, attention, combine
+        return 5   # ring pool, decode scorer, select, attention, combine
 
     def units(self):
         return self.w.B
@@ -250,6 +291,20 @@ class DecodeRunner:
 
 def flush_l2(buf):
     buf.add_(1.0)
+
+
+def max_over_ranks(value, world, device):
+    """The largest value over all ranks (the slowest rank's time); plain value at N=1."""
+    if world <= 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank, world, ms_per_step):
+    """Whole-job units per second: every rank processes its own replica of the workload."""
+    return units_per_rank * world / (ms_per_step / 1e3)
 
 
 def run_ours(args, rank, world):
@@ -313,12 +368,7 @@ def run_ours(args, rank, world):
     else:
         eager_ms = None
         stage_ms = [[events[i][s].elapsed_time(events[i][s + 1]) for i in range(args.steps)] for s in range(nst)]
-    total_ms = sum(step_ms)
-    # max over ranks
-    t = torch.tensor([total_ms], device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), world, dev)
     ms_per_step = total_ms / args.steps
 
     # end to end through the public API: pinned host inputs -> device -> QSA -> host result
@@ -374,15 +424,15 @@ def run_ours(args, rank, world):
     if eager_ms is not None:
         res["stage_ms"]["eager_step"] = round(eager_ms, 4)
     if w.kind == "prefill":
-        tokens = runner.units() * world
         res.update(metric="QSA prefill tokens/s", unit="tokens/s", higher_is_better=True,
-                   value=tokens / (ms_per_step / 1e3))
-        res["e2e"] = dict(value=tokens / (e2e_ms / 1e3), unit="tokens/s", h2d_bytes_per_step=h2d,
+                   value=job_throughput(runner.units(), world, ms_per_step))
+        res["e2e"] = dict(value=job_throughput(runner.units(), world, e2e_ms), unit="tokens/s", h2d_bytes_per_step=h2d,
                           d2h_bytes_per_step=d2h)
         attn_ms = stage_avg["sparse_attn"]
         achieved = alg["attn_bytes"] / (attn_ms / 1e3) / 1e9
         res["roofline"] = dict(kernel="sparse_attn_prefill", bound="hbm", achieved=achieved, peak=pk["hbm_gbs"],
-                               unit="GB/s", frac=achieved / pk["hbm_gbs"], traffic=None, peak_kind=pk_kind,
+                               unit="GB/s", frac=achieved / pk["hbm_gbs"],
+                               traffic=profiled_traffic("prefill", w.name), peak_kind=pk_kind,
                                note="algorithmic bytes = K/V rows gathered per query (4*nsel+tail positions x "
                                     "Hkv x d x 2 B x 2) + q read + out write; the unique K/V fits in L2, so "
                                     "gathers are served from L2 and frac can exceed 1")
@@ -400,10 +450,19 @@ def run_ours(args, rank, world):
                    value=ms_per_step * 1e3)
         res["e2e"] = dict(value=e2e_ms * 1e3, unit="us/step", h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h,
                           graph=used_graph, eager_value=e2e_eager_ms * 1e3)
-        achieved = alg["step_bytes"] / (ms_per_step / 1e3) / 1e9
-        res["roofline"] = dict(kernel="decode step (scorer dominant)", bound="hbm", achieved=achieved,
-                               peak=pk["hbm_gbs"], unit="GB/s", frac=achieved / pk["hbm_gbs"], traffic=None,
-                               peak_kind=pk_kind)
+        idx_ms = stage_avg["index_topk"]
+        achieved = alg["idx_bytes"] / (idx_ms / 1e3) / 1e9
+        res["roofline"] = dict(kernel="decode indexer (scorer + select)", bound="hbm", achieved=achieved,
+                               peak=pk["hbm_gbs"], unit="GB/s", frac=achieved / pk["hbm_gbs"],
+                               traffic=profiled_traffic("decode", w.name), peak_kind=pk_kind,
+                               note="algorithmic bytes = every compressed key of every sequence (ceil(L/4) x 128 x "
+                                    "2 B) + indexer query; time = the index stage of eager steps (histogram "
+                                    "clear, scorer, select); traffic = both kernels' DRAM bytes per call")
+        step_ach = alg["step_bytes"] / (ms_per_step / 1e3) / 1e9
+        res["step_roofline"] = dict(bound="hbm", achieved=step_ach, peak=pk["hbm_gbs"], unit="GB/s",
+                                    frac=step_ach / pk["hbm_gbs"], peak_kind=pk_kind,
+                                    note="whole decode step (graph replay): compressed keys + gathered K/V + q/o "
+                                         "bytes over the step time")
         res["config"] = dict(workload=w.name, B=w.B, L=w.T, top_k=w.top_k, Hq=w.Hq, Hkv=w.Hkv, d=w.d,
                              pos_scale=w.pos_scale, l2="inputs larger than L2 (compressed-key cache and K/V caches)",
                              parallelism=f"replicas x{world}", cuda_graph=True)
@@ -480,7 +539,9 @@ def main():
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
-    if world > 1:
+    if args.impl == "reference" and rank != 0:
+        return                      # the CPU oracle arm runs on rank 0 only
+    if world > 1 and args.impl != "reference":
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     w = workloads.WORKLOADS[args.workload]
@@ -500,8 +561,6 @@ def main():
                         cpu_baseline=dict(value=value, unit=unit, cores=threads, kind="oracle", sample=sample),
                         e2e=dict(value=value, unit=unit, h2d_bytes_per_step=0, d2h_bytes_per_step=0))
             print(json.dumps(line), flush=True)
-        if world > 1:
-            torch.distributed.destroy_process_group()
         return
 
     res = run_ours(args, rank, world)
@@ -513,7 +572,8 @@ def main():
         torch.distributed.destroy_process_group()
     if rank == 0:
         order = ["metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
-                 "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "tensor_roofline", "e2e",
+                 "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "tensor_roofline", "step_roofline",
+                 "e2e",
                  "cpu_baseline", "gpu_launches", "clocks", "stage_ms"]
         line = {k: res[k] for k in order if k in res}
         print(json.dumps(line), flush=True)
