@@ -196,48 +196,44 @@ constexpr int DM_ROWS = 128;                       // keys per stage
 constexpr int DM_NS = 3;                           // stages in flight per CTA (2 CTAs per SM)
 constexpr int DM_STAGE_BYTES = DM_ROWS * 256;      // two 64-dim k-atoms of 128 rows x 128 B
 
-struct DecodeMmaSmem {
-    alignas(1024) uint8_t stage[DM_NS][DM_STAGE_BYTES];
-    alignas(16) __nv_bfloat16 qcol[8][kIdxDim];   // B operand source: 8 columns x 128 dims
-    float w[kIdxHeads];
-    uint64_t full[DM_NS], empty[DM_NS];
-    uint32_t lh[2048];                             // local histogram of the keys' top 11 bits
-};
+using EncodeTiledFn = decltype(&cuTensorMapEncodeTiled);
 
-__global__ void __launch_bounds__(DI_THREADS, 2)
-    decode_score_mma_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16 *__restrict__ q_idx,
-                            Rope rope, DecodeParams p) {
-    extern __shared__ uint8_t dsm_raw[];
-    DecodeMmaSmem &sm = *reinterpret_cast<DecodeMmaSmem *>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) &
-                                                           ~uintptr_t(1023));
-    pdl_trigger();
-    const int seq = blockIdx.y, c = blockIdx.x;
+// 2-D bf16 map over the compressed keys [rows][128]: 64 x 128 boxes, 128-byte swizzle.
+bool make_kpool_map(CUtensorMap *map, const void *base, uint64_t rows) {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return false;
+        fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    cuuint64_t dims[2] = {128, rows};
+    cuuint64_t strides[1] = {128 * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)DM_ROWS};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Streams the n compressed keys of rows y0.. through NS stages, scores them
+// against the rotated query and hands each (row, key) to sink; every key's
+// top 11 bits are counted in sm.lh.  Returns false after a timed-out wait,
+// once the copies still in flight have landed (or their waits ran out too).
+template <int NS, typename Smem, typename Sink>
+__device__ __forceinline__ bool stream_scores(Smem &sm, const CUtensorMap *kmap,
+                                              const __nv_bfloat16 *__restrict__ q_idx, const Rope &rope,
+                                              const DecodeParams &p, int seq, int64_t s_len, int n, int y0,
+                                              Sink &&sink) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int64_t s_len = p.seq_len[seq];
-    int64_t nb = s_len / kBlock;
-    if (s_len < 1 || nb > p.pool_stride || nb > p.max_blocks) {
-        if (tid == 0 && c == 0) flag(p.status, QSA_DEV_BAD_LENGTH);
-        nb = 0;
-    }
-    const int64_t c0 = (int64_t)c * p.chunk;
-    const int64_t c1 = min(c0 + p.chunk, nb);
-    const int n = (int)(c1 > c0 ? c1 - c0 : 0);
-    if (n == 0) return;
-    uint32_t *gkeys = p.keys + (int64_t)seq * p.kstride + c0;
-    for (int b = tid; b < 2048; b += blockDim.x) sm.lh[b] = 0;
     const int nstages = (n + DM_ROWS - 1) / DM_ROWS;
-    const int y0 = (int)(seq * p.pool_stride + c0);
     if (tid == 0) {
-        for (int s = 0; s < DM_NS; ++s) { mbar_init(&sm.full[s], 1); mbar_init(&sm.empty[s], DI_THREADS / 32); }
-        fence_mbar_init();
-        prefetch_tmap(&kmap);
-    }
-    __syncthreads();
-    if (tid == 0) {
-        for (int st = 0; st < min(DM_NS, nstages); ++st) {
+        for (int st = 0; st < min(NS, nstages); ++st) {
             mbar_arrive_expect_tx(&sm.full[st], DM_STAGE_BYTES);
-            tma_load_2d(sm.stage[st], &kmap, 0, y0 + st * DM_ROWS, &sm.full[st]);
-            tma_load_2d(sm.stage[st] + DM_STAGE_BYTES / 2, &kmap, 64, y0 + st * DM_ROWS, &sm.full[st]);
+            tma_load_2d(sm.stage[st], kmap, 0, y0 + st * DM_ROWS, &sm.full[st]);
+            tma_load_2d(sm.stage[st] + DM_STAGE_BYTES / 2, kmap, 64, y0 + st * DM_ROWS, &sm.full[st]);
         }
     }
     const bool per_head = p.relu || p.head_w;
@@ -295,9 +291,11 @@ __global__ void __launch_bounds__(DI_THREADS, 2)
     const uint32_t row_off = (uint32_t)trow * 128u;
     const uint32_t sw = (uint32_t)(trow & 7);
     bool ok = true;
-    for (int st = 0; st < nstages; ++st) {
-        const int slot = st % DM_NS;
-        ok = mbar_wait(&sm.full[slot], (st / DM_NS) & 1, p.status);
+    int issued = min(NS, nstages);   // stages whose copies were issued (thread 0's count)
+    int st = 0;
+    for (; st < nstages; ++st) {
+        const int slot = st % NS;
+        ok = mbar_wait(&sm.full[slot], (st / NS) & 1, p.status);
         if (!ok) break;
         const uint32_t base = smem_u32(sm.stage[slot]);
         float acc[4] = {0.f, 0.f, 0.f, 0.f}, acc2[4] = {0.f, 0.f, 0.f, 0.f};
@@ -336,72 +334,100 @@ __global__ void __launch_bounds__(DI_THREADS, 2)
         if (tq == 0) {
             if (r0 < n) {
                 const uint32_t key = score_key(s0);
-                gkeys[r0] = key;
+                sink(r0, key);
                 atomicAdd(&sm.lh[key >> 21], 1u);
             }
             if (r0 + 8 < n) {
                 const uint32_t key = score_key(s1);
-                gkeys[r0 + 8] = key;
+                sink(r0 + 8, key);
                 atomicAdd(&sm.lh[key >> 21], 1u);
             }
         }
-        if (tid == 0 && st + DM_NS < nstages) {
-            ok = mbar_wait(&sm.empty[slot], (st / DM_NS) & 1, p.status);
+        if (tid == 0 && st + NS < nstages) {
+            ok = mbar_wait(&sm.empty[slot], (st / NS) & 1, p.status);
             if (ok) {
-                const int st2 = st + DM_NS;
+                const int st2 = st + NS;
                 mbar_arrive_expect_tx(&sm.full[slot], DM_STAGE_BYTES);
-                tma_load_2d(sm.stage[slot], &kmap, 0, y0 + st2 * DM_ROWS, &sm.full[slot]);
-                tma_load_2d(sm.stage[slot] + DM_STAGE_BYTES / 2, &kmap, 64, y0 + st2 * DM_ROWS, &sm.full[slot]);
+                tma_load_2d(sm.stage[slot], kmap, 0, y0 + st2 * DM_ROWS, &sm.full[slot]);
+                tma_load_2d(sm.stage[slot] + DM_STAGE_BYTES / 2, kmap, 64, y0 + st2 * DM_ROWS, &sm.full[slot]);
+                issued = st2 + 1;
             }
         }
     }
     ok = __syncthreads_and(ok);
+    if (!ok && tid == 0) {
+        // let the copies still in flight land before the shared memory is reused
+        for (int s2 = st; s2 < issued; ++s2) mbar_wait(&sm.full[s2 % NS], (s2 / NS) & 1, p.status);
+    }
+    return ok;
+}
+
+struct DecodeMmaSmem {
+    alignas(1024) uint8_t stage[DM_NS][DM_STAGE_BYTES];
+    alignas(16) __nv_bfloat16 qcol[8][kIdxDim];   // B operand source: 8 columns x 128 dims
+    float w[kIdxHeads];
+    uint64_t full[DM_NS], empty[DM_NS];
+    uint32_t lh[2048];                             // local histogram of the keys' top 11 bits
+};
+
+// Scorer of the two-kernel path: keys to the workspace, histogram added into
+// the sequence's global histogram.
+__global__ void __launch_bounds__(DI_THREADS, 2)
+    decode_score_mma_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16 *__restrict__ q_idx,
+                            Rope rope, DecodeParams p) {
+    extern __shared__ uint8_t dsm_raw[];
+    DecodeMmaSmem &sm = *reinterpret_cast<DecodeMmaSmem *>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) &
+                                                           ~uintptr_t(1023));
+    pdl_trigger();
+    const int seq = blockIdx.y, c = blockIdx.x;
+    const int tid = threadIdx.x;
+    const int64_t s_len = p.seq_len[seq];
+    int64_t nb = s_len / kBlock;
+    if (s_len < 1 || nb > p.pool_stride || nb > p.max_blocks) {
+        if (tid == 0 && c == 0) flag(p.status, QSA_DEV_BAD_LENGTH);
+        nb = 0;
+    }
+    const int64_t c0 = (int64_t)c * p.chunk;
+    const int64_t c1 = min(c0 + p.chunk, nb);
+    const int n = (int)(c1 > c0 ? c1 - c0 : 0);
+    if (n == 0) return;
+    uint32_t *gkeys = p.keys + (int64_t)seq * p.kstride + c0;
+    for (int b = tid; b < 2048; b += blockDim.x) sm.lh[b] = 0;
+    if (tid == 0) {
+        for (int s = 0; s < DM_NS; ++s) { mbar_init(&sm.full[s], 1); mbar_init(&sm.empty[s], DI_THREADS / 32); }
+        fence_mbar_init();
+        prefetch_tmap(&kmap);
+    }
+    __syncthreads();
+    const bool ok = stream_scores<DM_NS>(sm, &kmap, q_idx, rope, p, seq, s_len, n, (int)(seq * p.pool_stride + c0),
+                                         [&](int r, uint32_t key) { gkeys[r] = key; });
     if (!ok) return;
     flush_hist(sm.lh, p.hist + (int64_t)seq * 2048);
 }
 
-using EncodeTiledFn = decltype(&cuTensorMapEncodeTiled);
-
-// 2-D bf16 map over the compressed keys [rows][128]: 64 x 128 boxes, 128-byte swizzle.
-bool make_kpool_map(CUtensorMap *map, const void *base, uint64_t rows) {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
-            q != cudaDriverEntryPointSuccess)
-            return false;
-        fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    }
-    cuuint64_t dims[2] = {128, rows};
-    cuuint64_t strides[1] = {128 * 2};
-    cuuint32_t box[2] = {64, (cuuint32_t)DM_ROWS};
-    cuuint32_t estr[2] = {1, 1};
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // ---------------------------------------------------------------------------
-// Selection from the score keys: one kernel, one thread-block cluster of up to
-// 16 CTAs per sequence.
+// Selection from the score keys, one thread-block cluster per sequence.
 //
-// Every CTA owns a chunk of a sequence's keys (whole tiles of DS_TILE keys,
-// 16 contiguous keys per thread, read with four 16-byte loads issued
-// together).  With the top-11-bit histogram from the scorer, the bin d1 that
-// holds the k-th largest key is known before any key is read.  Each CTA
-// writes to its own shared memory, in block order, the ids of its keys above
-// bin d1 (all of them are selected; fewer than k in the whole sequence) and
-// the (key, id) pairs of its keys in bin d1 (the candidates; past the
-// shared-memory capacity they go to a global overflow area).  After a cluster
-// barrier, CTA 0 gathers the lists through distributed shared memory, resolves
-// the remaining 21 bits of K* on the candidates, keeps the candidates above K*
-// and the first ones equal to K* (ties to the lower block id), and merges that
-// list with the above-bin ids into the ascending output.
+// Every CTA owns a chunk of a sequence's keys (whole tiles of NT * 16 keys, 16
+// contiguous keys per thread).  With the histogram of the keys' top 11 bits,
+// the bin d1 that holds the k-th largest key is known before any key is read.
+// Each CTA writes to its own shared memory, in block order, the ids of its
+// keys above bin d1 (all of them are selected; fewer than k in the whole
+// sequence) and the (key, id) pairs of its keys in bin d1 (the candidates;
+// past the shared-memory capacity they go to a global overflow area).  After
+// a cluster barrier, CTA 0 gathers the lists through distributed shared
+// memory, resolves the remaining 21 bits of K* on the candidates, keeps the
+// candidates above K* and the first ones equal to K* (ties to the lower block
+// id), and merges that list with the above-bin ids into the ascending output.
+//
+// Two kernels use it: decode_select_kernel reads the keys and the histogram
+// that decode_score_*_kernel wrote to the workspace; decode_index_fused_kernel
+// scores, keeps its chunk's keys in shared memory and merges the CTAs'
+// histograms through distributed shared memory, with no workspace round trip.
 // ---------------------------------------------------------------------------
 constexpr int DS_THREADS = 512;
 constexpr int DS_PER_THREAD = 16;
-constexpr int DS_TILE = DS_THREADS * DS_PER_THREAD;   // keys per CTA tile
+constexpr int DS_TILE = DS_THREADS * DS_PER_THREAD;   // keys per CTA tile of decode_select_kernel
 constexpr int DS_CLUSTER = 16;                        // CTAs (chunks) per sequence at most (non-portable above 8)
 constexpr int DS_LCAND = 2048;                        // candidates a CTA keeps in shared memory
 constexpr int DS_CAND_SMEM = 4096;                    // candidates CTA 0 stages in shared memory
@@ -409,10 +435,10 @@ constexpr int DS_MAX_K = 2048;                        // largest top_k
 
 struct SelectArgs {
     const int32_t *seq_len;
-    int64_t pool_stride, max_blocks, kstride, chunk;   // chunk: keys per CTA, a multiple of DS_TILE
+    int64_t pool_stride, max_blocks, kstride, chunk;   // chunk: keys per CTA (whole tiles for the select kernel)
     int gmax, top_k;                                    // gmax: CTAs per cluster (<= DS_CLUSTER)
-    const uint32_t *keys;   // [B][kstride] score keys
-    const uint32_t *hist;   // [B][2048] histogram of the keys' top 11 bits
+    const uint32_t *keys;   // [B][kstride] score keys (select kernel)
+    const uint32_t *hist;   // [B][2048] histogram of the keys' top 11 bits (select kernel)
     uint2 *cand;            // [B][kstride]: chunk g's candidates past DS_LCAND, at g * chunk + position
     int32_t *sel, *nsel;
 };
@@ -431,13 +457,14 @@ struct DsSmem {
     int32_t slist[DS_MAX_K];            // selected candidate ids (ascending)
     uint32_t aoff[DS_CLUSTER + 1];      // prefix of the above counts per chunk
     uint32_t coff[DS_CLUSTER + 1];      // prefix of the candidate counts per chunk
-    uint32_t wsum[DS_THREADS / 32];
+    uint32_t wsum[32];
 };
 
-__device__ __forceinline__ int64_t visible_blocks(const SelectArgs &a, int seq) {
-    const int64_t s_len = a.seq_len[seq];
+__device__ __forceinline__ int64_t visible_blocks(const int32_t *seq_len, int64_t pool_stride, int64_t max_blocks,
+                                                  int seq) {
+    const int64_t s_len = seq_len[seq];
     const int64_t nb = s_len / kBlock;
-    return (s_len < 1 || nb > a.pool_stride || nb > a.max_blocks) ? 0 : nb;   // flagged by the scorer
+    return (s_len < 1 || nb > pool_stride || nb > max_blocks) ? 0 : nb;   // flagged by the scorer
 }
 
 // Loads keys [i0, i0 + 16) of a row (i0 a multiple of 16; the row holds
@@ -490,45 +517,17 @@ __device__ __forceinline__ int count_below(const int32_t *l, int n, int32_t v) {
     return lo;
 }
 
-__global__ void __launch_bounds__(DS_THREADS)
-    decode_select_kernel(SelectArgs a) {
-    extern __shared__ __align__(16) uint8_t ds_raw[];
-    DsSmem &sm = *reinterpret_cast<DsSmem *>(ds_raw);
-    pdl_wait();
-    pdl_trigger();
-    const int seq = blockIdx.y, tid = threadIdx.x;
-    const uint32_t rank = cluster_rank();             // = blockIdx.x: a cluster spans the x extent
-    const int64_t nb = visible_blocks(a, seq);
-    const int top_k = a.top_k;
-    int32_t *out = a.sel + (int64_t)seq * top_k;
-    const int64_t c0 = (int64_t)rank * a.chunk, c1 = min(c0 + a.chunk, nb);
-    if (nb <= top_k) {                               // every visible block, in order (whole cluster)
-        for (int64_t i = c0 + tid; i < c1; i += DS_THREADS) out[i] = (int32_t)i;
-        if (rank == 0) {
-            for (int i = (int)nb + tid; i < top_k; i += DS_THREADS) out[i] = -1;
-            if (tid == 0) a.nsel[seq] = (int)nb;
-        }
-        return;
-    }
-    const int gseq = (int)((nb + a.chunk - 1) / a.chunk);   // CTAs with keys (<= cluster size)
-    const uint32_t *row = a.keys + (int64_t)seq * a.kstride;
-    uint2 *cand_seq = a.cand + (int64_t)seq * a.kstride;
-    // first tile's keys in flight before the histogram is read
-    uint32_t k[16];
-    int m = load16(row, c0 + (int64_t)DS_PER_THREAD * tid, c1, a.kstride, k);
-    // bin of the k-th largest key from the scorer's histogram
-    static_assert(DS_THREADS * 4 == 2048, "one 16-byte histogram load per thread");
-    reinterpret_cast<uint4 *>(sm.s.hist)[tid] = __ldcg(reinterpret_cast<const uint4 *>(a.hist + (int64_t)seq * 2048) + tid);
-    if (tid == 0) { sm.s.digit = 0; sm.s.k_rem = 1; }
-    __syncthreads();
-    sel_find_digit(sm.s, 2048, top_k);
-    const uint32_t d1 = (uint32_t)sm.s.digit;
-    const int k_rem1 = sm.s.k_rem;
-
+// This CTA's lists from its keys [c0, c1): tiles of NT * 16 keys, thread t
+// holding keys [16t, 16t + 16) of a tile.  k/m hold the first tile's keys
+// (already loaded by the caller); load(i0, k) loads the next ones.
+template <int NT, typename Load>
+__device__ __forceinline__ void build_lists(DsSmem &sm, Load &&load, int64_t c0, int64_t c1, uint32_t d1, int top_k,
+                                            uint2 *cand_seq, uint32_t (&k)[16], int m) {
+    const int tid = threadIdx.x;
     uint32_t na_run = 0, nc_run = 0;
-    for (int64_t t0 = c0; t0 < c1; t0 += DS_TILE) {
+    for (int64_t t0 = c0; t0 < c1; t0 += (int64_t)NT * DS_PER_THREAD) {
         const int64_t i0 = t0 + (int64_t)DS_PER_THREAD * tid;
-        if (t0 != c0) m = load16(row, i0, c1, a.kstride, k);
+        if (t0 != c0) m = load(i0, k);
         // bit j: key j lies above bin d1 (amask) or in it (cmask); few keys do
         uint32_t amask = 0, cmask = 0;
 #pragma unroll
@@ -569,111 +568,272 @@ __global__ void __launch_bounds__(DS_THREADS)
         sm.my_na = min(na_run, (uint32_t)min(top_k - 1, DS_MAX_K));
         sm.my_nc = nc_run;
     }
-    cluster_sync();                                  // every CTA's lists are complete
-    if (rank == 0) {
-        // per-chunk offsets of the above ids and of the candidates
-        if (tid == 0) {
-            uint32_t ea = 0, ec = 0;
-            for (int c = 0; c < gseq; ++c) {
-                sm.aoff[c] = ea;
-                sm.coff[c] = ec;
-                ea += ld_dsmem(dsmem_addr(&sm.my_na, c));
-                ec += ld_dsmem(dsmem_addr(&sm.my_nc, c));
-            }
-            sm.aoff[gseq] = ea;
-            sm.coff[gseq] = ec;
+}
+
+// CTA 0 of the cluster, after the lists of the gseq CTAs with keys are complete.
+template <int NT>
+__device__ __forceinline__ void select_leader(DsSmem &sm, int gseq, uint32_t d1, int k_rem1, int64_t nb,
+                                              int64_t chunk, const uint2 *cand_seq, int top_k, int32_t *out,
+                                              int32_t *nsel_out) {
+    const int tid = threadIdx.x;
+    // per-chunk offsets of the above ids and of the candidates
+    if (tid == 0) {
+        uint32_t ea = 0, ec = 0;
+        for (int c = 0; c < gseq; ++c) {
+            sm.aoff[c] = ea;
+            sm.coff[c] = ec;
+            ea += ld_dsmem(dsmem_addr(&sm.my_na, c));
+            ec += ld_dsmem(dsmem_addr(&sm.my_nc, c));
         }
-        __syncthreads();
-        const int na_all = (int)min(sm.aoff[gseq], (uint32_t)(top_k - 1));
-        const int nc_all = (int)min((int64_t)sm.coff[gseq], nb);
-        const bool small = nc_all <= DS_CAND_SMEM;
-        for (int j = tid; j < na_all; j += DS_THREADS) {
-            const int c = chunk_of(sm.aoff, gseq, (uint32_t)j);
-            sm.alist[j] = (int32_t)ld_dsmem(dsmem_addr(&sm.my_above[j - sm.aoff[c]], c));
-        }
-        auto fetch = [&](int j) -> uint2 {           // candidate j of the sequence, block order
-            const int c = chunk_of(sm.coff, gseq, (uint32_t)j);
-            const uint32_t jj = (uint32_t)j - sm.coff[c];
-            if (jj < (uint32_t)DS_LCAND)
-                return make_uint2(ld_dsmem(dsmem_addr(&sm.my_ck[jj], c)), ld_dsmem(dsmem_addr(&sm.my_ci[jj], c)));
-            return __ldcg(cand_seq + (int64_t)c * a.chunk + jj);
-        };
-        if (small)
-            for (int j = tid; j < nc_all; j += DS_THREADS) {
-                const uint2 v = fetch(j);
-                sm.ck[j] = v.x;
-                sm.ci[j] = v.y;
-            }
-        __syncthreads();
-        auto cand_at = [&](int j) -> uint2 { return small ? make_uint2(sm.ck[j], sm.ci[j]) : fetch(j); };
-        // remaining 21 bits of K*: bits 20..10, then 9..0
-        uint32_t prefix = d1 << 21, pmask = 0xFFE00000u;
-        int k_rem = k_rem1;
-#pragma unroll 1
-        for (int pass = 0; pass < 2; ++pass) {
-            const int shift = pass == 0 ? 10 : 0, nbins = pass == 0 ? 2048 : 1024;
-            const uint32_t mask = (uint32_t)nbins - 1u;
-            for (int b = tid; b < nbins; b += DS_THREADS) sm.s.hist[b] = 0;
-            __syncthreads();
-            for (int j = tid; j < nc_all; j += DS_THREADS) {
-                const uint32_t key = cand_at(j).x;
-                if ((key & pmask) == prefix) atomicAdd(&sm.s.hist[(key >> shift) & mask], 1u);
-            }
-            __syncthreads();
-            sel_find_digit(sm.s, nbins, k_rem);
-            prefix |= (uint32_t)sm.s.digit << shift;
-            pmask |= mask << shift;
-            k_rem = sm.s.k_rem;
-            __syncthreads();
-        }
-        const uint32_t kstar = prefix;
-        const int take_eq = k_rem;
-        // selected candidates in block order: keys above K*, and the first take_eq equal to K*.
-        // Thread t takes a contiguous run of cpt candidates per round of DS_THREADS * cpt.
-        int ns = 0;     // CTA-uniform running count
-        uint32_t eq_run = 0;
-        const int cpt = min(8, max(1, (nc_all + DS_THREADS - 1) / DS_THREADS));
-        for (int base = 0; base < nc_all; base += DS_THREADS * cpt) {
-            const int j0 = base + cpt * tid, j1 = min(j0 + cpt, nc_all);
-            uint32_t eq = 0;
-            for (int j = j0; j < j1; ++j) eq += cand_at(j).x == kstar;
-            uint32_t eq_tot;
-            const uint32_t r0 = eq_run + cta_scan(eq, sm.wsum, eq_tot);   // rank of my first key == K*
-            uint32_t r = r0, nsel_mine = 0;
-            for (int j = j0; j < j1; ++j) {
-                const uint32_t key = cand_at(j).x;
-                nsel_mine += key > kstar || (key == kstar && r++ < (uint32_t)take_eq);
-            }
-            uint32_t s_tot;
-            uint32_t pos = (uint32_t)ns + cta_scan(nsel_mine, sm.wsum, s_tot);
-            r = r0;
-            for (int j = j0; j < j1; ++j) {
-                const uint2 v = cand_at(j);
-                if (v.x > kstar || (v.x == kstar && r++ < (uint32_t)take_eq)) {
-                    if (pos < (uint32_t)DS_MAX_K) sm.slist[pos] = (int32_t)v.y;
-                    ++pos;
-                }
-            }
-            ns += (int)s_tot;
-            eq_run += eq_tot;
-        }
-        ns = min(ns, top_k - na_all);
-        __syncthreads();
-        // merge the two ascending lists into the output
-        for (int j = tid; j < na_all; j += DS_THREADS) {
-            const int32_t v = sm.alist[j];
-            const int pos = j + count_below(sm.slist, ns, v);
-            if (pos < top_k) out[pos] = v;
-        }
-        for (int j = tid; j < ns; j += DS_THREADS) {
-            const int32_t v = sm.slist[j];
-            const int pos = j + count_below(sm.alist, na_all, v);
-            if (pos < top_k) out[pos] = v;
-        }
-        const int cnt = na_all + ns;
-        for (int i = cnt + tid; i < top_k; i += DS_THREADS) out[i] = -1;
-        if (tid == 0) a.nsel[seq] = cnt;
+        sm.aoff[gseq] = ea;
+        sm.coff[gseq] = ec;
     }
+    __syncthreads();
+    const int na_all = (int)min(sm.aoff[gseq], (uint32_t)(top_k - 1));
+    const int nc_all = (int)min((int64_t)sm.coff[gseq], nb);
+    const bool small = nc_all <= DS_CAND_SMEM;
+    for (int j = tid; j < na_all; j += NT) {
+        const int c = chunk_of(sm.aoff, gseq, (uint32_t)j);
+        sm.alist[j] = (int32_t)ld_dsmem(dsmem_addr(&sm.my_above[j - sm.aoff[c]], c));
+    }
+    auto fetch = [&](int j) -> uint2 {           // candidate j of the sequence, block order
+        const int c = chunk_of(sm.coff, gseq, (uint32_t)j);
+        const uint32_t jj = (uint32_t)j - sm.coff[c];
+        if (jj < (uint32_t)DS_LCAND)
+            return make_uint2(ld_dsmem(dsmem_addr(&sm.my_ck[jj], c)), ld_dsmem(dsmem_addr(&sm.my_ci[jj], c)));
+        return __ldcg(cand_seq + (int64_t)c * chunk + jj);
+    };
+    if (small)
+        for (int j = tid; j < nc_all; j += NT) {
+            const uint2 v = fetch(j);
+            sm.ck[j] = v.x;
+            sm.ci[j] = v.y;
+        }
+    __syncthreads();
+    auto cand_at = [&](int j) -> uint2 { return small ? make_uint2(sm.ck[j], sm.ci[j]) : fetch(j); };
+    // remaining 21 bits of K*: bits 20..10, then 9..0
+    uint32_t prefix = d1 << 21, pmask = 0xFFE00000u;
+    int k_rem = k_rem1;
+#pragma unroll 1
+    for (int pass = 0; pass < 2; ++pass) {
+        const int shift = pass == 0 ? 10 : 0, nbins = pass == 0 ? 2048 : 1024;
+        const uint32_t mask = (uint32_t)nbins - 1u;
+        for (int b = tid; b < nbins; b += NT) sm.s.hist[b] = 0;
+        __syncthreads();
+        for (int j = tid; j < nc_all; j += NT) {
+            const uint32_t key = cand_at(j).x;
+            if ((key & pmask) == prefix) atomicAdd(&sm.s.hist[(key >> shift) & mask], 1u);
+        }
+        __syncthreads();
+        sel_find_digit(sm.s, nbins, k_rem);
+        prefix |= (uint32_t)sm.s.digit << shift;
+        pmask |= mask << shift;
+        k_rem = sm.s.k_rem;
+        __syncthreads();
+    }
+    const uint32_t kstar = prefix;
+    const int take_eq = k_rem;
+    // selected candidates in block order: keys above K*, and the first take_eq equal to K*.
+    // Thread t takes a contiguous run of cpt candidates per round of NT * cpt.
+    int ns = 0;     // CTA-uniform running count
+    uint32_t eq_run = 0;
+    const int cpt = min(8, max(1, (nc_all + NT - 1) / NT));
+    for (int base = 0; base < nc_all; base += NT * cpt) {
+        const int j0 = base + cpt * tid, j1 = min(j0 + cpt, nc_all);
+        uint32_t eq = 0;
+        for (int j = j0; j < j1; ++j) eq += cand_at(j).x == kstar;
+        uint32_t eq_tot;
+        const uint32_t r0 = eq_run + cta_scan(eq, sm.wsum, eq_tot);   // rank of my first key == K*
+        uint32_t r = r0, nsel_mine = 0;
+        for (int j = j0; j < j1; ++j) {
+            const uint32_t key = cand_at(j).x;
+            nsel_mine += key > kstar || (key == kstar && r++ < (uint32_t)take_eq);
+        }
+        uint32_t s_tot;
+        uint32_t pos = (uint32_t)ns + cta_scan(nsel_mine, sm.wsum, s_tot);
+        r = r0;
+        for (int j = j0; j < j1; ++j) {
+            const uint2 v = cand_at(j);
+            if (v.x > kstar || (v.x == kstar && r++ < (uint32_t)take_eq)) {
+                if (pos < (uint32_t)DS_MAX_K) sm.slist[pos] = (int32_t)v.y;
+                ++pos;
+            }
+        }
+        ns += (int)s_tot;
+        eq_run += eq_tot;
+    }
+    ns = min(ns, top_k - na_all);
+    __syncthreads();
+    // merge the two ascending lists into the output
+    for (int j = tid; j < na_all; j += NT) {
+        const int32_t v = sm.alist[j];
+        const int pos = j + count_below(sm.slist, ns, v);
+        if (pos < top_k) out[pos] = v;
+    }
+    for (int j = tid; j < ns; j += NT) {
+        const int32_t v = sm.slist[j];
+        const int pos = j + count_below(sm.alist, na_all, v);
+        if (pos < top_k) out[pos] = v;
+    }
+    const int cnt = na_all + ns;
+    for (int i = cnt + tid; i < top_k; i += NT) out[i] = -1;
+    if (tid == 0) *nsel_out = cnt;
+}
+
+// Every visible block selected (nb <= top_k): ids in order, padded with -1.
+template <int NT>
+__device__ __forceinline__ void select_all(int64_t c0, int64_t c1, int64_t nb, int top_k, uint32_t rank,
+                                           int32_t *out, int32_t *nsel_out) {
+    for (int64_t i = c0 + threadIdx.x; i < c1; i += NT) out[i] = (int32_t)i;
+    if (rank == 0) {
+        for (int i = (int)nb + threadIdx.x; i < top_k; i += NT) out[i] = -1;
+        if (threadIdx.x == 0) *nsel_out = (int)nb;
+    }
+}
+
+__global__ void __launch_bounds__(DS_THREADS)
+    decode_select_kernel(SelectArgs a) {
+    extern __shared__ __align__(16) uint8_t ds_raw[];
+    DsSmem &sm = *reinterpret_cast<DsSmem *>(ds_raw);
+    pdl_wait();
+    pdl_trigger();
+    const int seq = blockIdx.y, tid = threadIdx.x;
+    const uint32_t rank = cluster_rank();             // = blockIdx.x: a cluster spans the x extent
+    const int64_t nb = visible_blocks(a.seq_len, a.pool_stride, a.max_blocks, seq);
+    const int top_k = a.top_k;
+    int32_t *out = a.sel + (int64_t)seq * top_k;
+    const int64_t c0 = (int64_t)rank * a.chunk, c1 = min(c0 + a.chunk, nb);
+    if (nb <= top_k) {                               // the whole cluster takes this branch
+        select_all<DS_THREADS>(c0, c1, nb, top_k, rank, out, a.nsel + seq);
+        return;
+    }
+    const int gseq = (int)((nb + a.chunk - 1) / a.chunk);   // CTAs with keys (<= cluster size)
+    const uint32_t *row = a.keys + (int64_t)seq * a.kstride;
+    uint2 *cand_seq = a.cand + (int64_t)seq * a.kstride;
+    // first tile's keys in flight before the histogram is read
+    uint32_t k[16];
+    const int m = load16(row, c0 + (int64_t)DS_PER_THREAD * tid, c1, a.kstride, k);
+    // bin of the k-th largest key from the scorer's histogram
+    static_assert(DS_THREADS * 4 == 2048, "one 16-byte histogram load per thread");
+    reinterpret_cast<uint4 *>(sm.s.hist)[tid] = __ldcg(reinterpret_cast<const uint4 *>(a.hist + (int64_t)seq * 2048) + tid);
+    if (tid == 0) { sm.s.digit = 0; sm.s.k_rem = 1; }
+    __syncthreads();
+    sel_find_digit(sm.s, 2048, top_k);
+    const uint32_t d1 = (uint32_t)sm.s.digit;
+    const int k_rem1 = sm.s.k_rem;
+    build_lists<DS_THREADS>(
+        sm, [&](int64_t i0, uint32_t (&kk)[16]) { return load16(row, i0, c1, a.kstride, kk); }, c0, c1, d1, top_k,
+        cand_seq, k, m);
+    cluster_sync();                                  // every CTA's lists are complete
+    if (rank == 0) select_leader<DS_THREADS>(sm, gseq, d1, k_rem1, nb, a.chunk, cand_seq, top_k, out, a.nsel + seq);
+    cluster_sync();                                  // CTA 0 has finished reading the others' lists
+}
+
+// ---------------------------------------------------------------------------
+// Fused decode indexer (bf16): scorer and selection in one cluster kernel.
+// One cluster of up to 16 CTAs per sequence, one CTA per SM; each CTA streams
+// its chunk of compressed keys (4 stages in flight) and keeps the chunk's score
+// keys in shared memory.  The CTAs' histograms are summed through distributed
+// shared memory (CTA r sums a slice of bins over the cluster and writes the
+// sums into every CTA), then the selection above runs on the resident keys.
+// ---------------------------------------------------------------------------
+constexpr int DF_NS = 4;              // stages in flight per CTA
+constexpr int DF_KEYS = 16384;        // keys a CTA keeps in shared memory
+constexpr int DF_THREADS = DI_THREADS;
+
+struct FusedSmem {
+    union {
+        uint8_t stage[DF_NS][DM_STAGE_BYTES];   // while streaming
+        DsSmem ds;                              // selection, once every stage has been consumed
+    } u;
+    uint32_t skeys[DF_KEYS];
+    uint32_t lh[2048];
+    alignas(16) __nv_bfloat16 qcol[8][kIdxDim];
+    float w[kIdxHeads];
+    uint64_t full[DF_NS], empty[DF_NS];
+};
+static_assert(sizeof(DsSmem) <= (size_t)DF_NS * DM_STAGE_BYTES, "selection state fits the stage buffers");
+
+// The streaming interface of FusedSmem (stage, qcol, w, full, empty, lh).
+struct FusedStream {
+    uint8_t (&stage)[DF_NS][DM_STAGE_BYTES];
+    __nv_bfloat16 (&qcol)[8][kIdxDim];
+    float (&w)[kIdxHeads];
+    uint64_t (&full)[DF_NS];
+    uint64_t (&empty)[DF_NS];
+    uint32_t (&lh)[2048];
+};
+
+__global__ void __launch_bounds__(DF_THREADS, 1)
+    decode_index_fused_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16 *__restrict__ q_idx,
+                              Rope rope, DecodeParams p, SelectArgs a) {
+    extern __shared__ uint8_t dsm_raw[];
+    FusedSmem &sm = *reinterpret_cast<FusedSmem *>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
+    pdl_wait();      // the compressed keys come from the previous kernel (ring pooling)
+    pdl_trigger();
+    const int seq = blockIdx.y, tid = threadIdx.x;
+    const uint32_t rank = cluster_rank();             // = blockIdx.x: a cluster spans the x extent
+    const int ncta = (int)a.gmax;
+    const int64_t s_len = p.seq_len[seq];
+    const int64_t nb = visible_blocks(a.seq_len, a.pool_stride, a.max_blocks, seq);
+    if ((s_len < 1 || s_len / kBlock > p.pool_stride || s_len / kBlock > p.max_blocks) && tid == 0 && rank == 0)
+        flag(p.status, QSA_DEV_BAD_LENGTH);
+    const int top_k = a.top_k;
+    int32_t *out = a.sel + (int64_t)seq * top_k;
+    const int64_t c0 = (int64_t)rank * a.chunk, c1 = min(c0 + a.chunk, nb);
+    if (nb <= top_k) {                               // the whole cluster takes this branch; no scores needed
+        select_all<DF_THREADS>(c0, c1, nb, top_k, rank, out, a.nsel + seq);
+        return;
+    }
+    const int gseq = (int)((nb + a.chunk - 1) / a.chunk);
+    const int n = (int)(c1 > c0 ? c1 - c0 : 0);      // <= DF_KEYS by the launch plan
+    uint2 *cand_seq = a.cand + (int64_t)seq * a.kstride;
+    for (int b = tid; b < 2048; b += DF_THREADS) sm.lh[b] = 0;
+    if (tid == 0) {
+        for (int s = 0; s < DF_NS; ++s) { mbar_init(&sm.full[s], 1); mbar_init(&sm.empty[s], DF_THREADS / 32); }
+        fence_mbar_init();
+        prefetch_tmap(&kmap);
+    }
+    __syncthreads();
+    bool ok = true;
+    if (n > 0) {
+        FusedStream fs{sm.u.stage, sm.qcol, sm.w, sm.full, sm.empty, sm.lh};
+        ok = stream_scores<DF_NS>(fs, &kmap, q_idx, rope, p, seq, s_len, n, (int)(seq * p.pool_stride + c0),
+                                  [&](int r, uint32_t key) { sm.skeys[r] = key; });
+    }
+    (void)ok;   // a timed-out wait is in the status word; the cluster still runs every barrier
+    __syncthreads();
+    cluster_sync();                                  // every CTA's histogram is complete; stages are free
+    // sequence histogram: CTA r sums bins [r * per, (r + 1) * per) over the cluster
+    const int per = (2048 + ncta - 1) / ncta;
+    for (int b = (int)rank * per + tid; b < min(2048, ((int)rank + 1) * per); b += DF_THREADS) {
+        uint32_t sum = 0;
+        for (int c = 0; c < ncta; ++c) sum += ld_dsmem(dsmem_addr(&sm.lh[b], (uint32_t)c));
+        for (int c = 0; c < ncta; ++c) st_dsmem(dsmem_addr(&sm.u.ds.s.hist[b], (uint32_t)c), sum);
+    }
+    DsSmem &ds = sm.u.ds;
+    if (tid == 0) { ds.s.digit = 0; ds.s.k_rem = 1; }
+    cluster_sync();                                  // every CTA holds the sequence histogram
+    sel_find_digit(ds.s, 2048, top_k);
+    const uint32_t d1 = (uint32_t)ds.s.digit;
+    const int k_rem1 = ds.s.k_rem;
+    auto load_sm = [&](int64_t i0, uint32_t (&kk)[16]) -> int {
+        const int64_t m0 = c1 - i0;
+        const int m = m0 <= 0 ? 0 : (m0 >= 16 ? 16 : (int)m0);
+        const uint4 *src = reinterpret_cast<const uint4 *>(&sm.skeys[i0 - c0]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (4 * j < m) v = src[j];
+            kk[4 * j] = v.x; kk[4 * j + 1] = v.y; kk[4 * j + 2] = v.z; kk[4 * j + 3] = v.w;
+        }
+        return m;
+    };
+    uint32_t k[16];
+    const int m = load_sm(c0 + (int64_t)DS_PER_THREAD * tid, k);
+    build_lists<DF_THREADS>(ds, load_sm, c0, c1, d1, top_k, cand_seq, k, m);
+    cluster_sync();                                  // every CTA's lists are complete
+    if (rank == 0) select_leader<DF_THREADS>(ds, gseq, d1, k_rem1, nb, a.chunk, cand_seq, top_k, out, a.nsel + seq);
     cluster_sync();                                  // CTA 0 has finished reading the others' lists
 }
 
@@ -747,6 +907,69 @@ bool cluster16_ok() {
     return ok == 1;
 }
 
+// Fused path: C CTAs per sequence (one cluster), chunks of at most DF_KEYS
+// keys, used when B x C CTAs (one per SM) cover at least half the SMs and all
+// B clusters can be resident together.
+struct FusedPlan {
+    bool use;
+    int C;
+    int64_t chunk;
+};
+
+// Clusters of C fused CTAs that can be resident at once (queried once per C).
+int fused_active_clusters(int C) {
+    static int ok[DS_CLUSTER + 1];
+    static bool init = false;
+    if (!init) {
+        for (int i = 0; i <= DS_CLUSTER; ++i) ok[i] = -1;
+        init = true;
+    }
+    if (C < 1 || C > DS_CLUSTER) return 0;
+    if (ok[C] < 0) {
+        ok[C] = 0;
+        const size_t smem = sizeof(FusedSmem) + 1024;
+        if (cudaFuncSetAttribute(decode_index_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) ==
+                cudaSuccess &&
+            (C <= 8 || cudaFuncSetAttribute(decode_index_fused_kernel,
+                                            cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess)) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3((unsigned)C, 1, 1);
+            cfg.blockDim = dim3(DF_THREADS, 1, 1);
+            cfg.dynamicSmemBytes = smem;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = (unsigned)C;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, decode_index_fused_kernel, &cfg) == cudaSuccess && n > 0) ok[C] = n;
+        }
+        cudaGetLastError();   // a refused query leaves no sticky error
+    }
+    return ok[C];
+}
+
+FusedPlan fused_plan(int B, int64_t max_blocks, bool bf16) {
+    FusedPlan f{false, 1, DF_KEYS};
+    const DeviceInfo *di = device_info();
+    const int64_t sms = di ? di->sm_count : 148;
+    if (!bf16 || B < 1 || max_blocks < 1) return f;
+    const int64_t cmin = (max_blocks + DF_KEYS - 1) / DF_KEYS;
+    if (cmin > DS_CLUSTER) return f;
+    int64_t C = std::max<int64_t>(cmin, std::min<int64_t>(DS_CLUSTER, sms / B));
+    int64_t chunk = (max_blocks + C - 1) / C;
+    chunk = (chunk + DM_ROWS - 1) / DM_ROWS * DM_ROWS;          // <= DF_KEYS: C >= cmin
+    C = (max_blocks + chunk - 1) / chunk;
+    f.C = (int)C;
+    f.chunk = chunk;
+    // one wave of clusters: a sequence whose cluster waited for a free GPC
+    // would stream after the others with a fraction of the bandwidth
+    f.use = (int64_t)B * C >= sms / 2 && fused_active_clusters((int)C) >= B;
+    return f;
+}
+
 // Workspace: keys [B][kstride] u32 | cand overflow [B][kstride] uint2 | hist [B][2048] u32
 struct DecodeWs {
     uint32_t *keys;
@@ -783,9 +1006,28 @@ cudaError_t launch_decode_index(const void *q_idx, const void *k_pool, const flo
                                 const int32_t *seq_len, int B, int64_t pool_stride, int64_t max_blocks,
                                 int top_k, int32_t *sel, int32_t *nsel, void *ws, Rope rope, bool relu,
                                 bool bf16, unsigned *status, cudaStream_t s) {
-    const DecodePlan pl = decode_index_plan(B, max_blocks, bf16);
     const int64_t kstride = key_stride(max_blocks);
     const DecodeWs d = decode_ws(ws, B, max_blocks, top_k);
+    const FusedPlan fp = fused_plan(B, max_blocks, bf16);
+    if (fp.use) {
+        CUtensorMap kmap;
+        if (!make_kpool_map(&kmap, k_pool, (uint64_t)B * pool_stride)) return cudaErrorInvalidValue;
+        DecodeParams p{seq_len, head_w, pool_stride, max_blocks, fp.chunk, kstride, fp.C, top_k, relu ? 1 : 0,
+                       d.keys, d.hist, status};
+        SelectArgs sa{seq_len, pool_stride, max_blocks, kstride, fp.chunk, fp.C, top_k, d.keys, d.hist, d.cand,
+                      sel, nsel};
+        const size_t smem = sizeof(FusedSmem) + 1024;
+        cudaError_t e =
+            cudaFuncSetAttribute(decode_index_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        if (fp.C > 8) {
+            e = cudaFuncSetAttribute(decode_index_fused_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+            if (e != cudaSuccess) return e;
+        }
+        return launch_pdl_cluster(decode_index_fused_kernel, dim3((unsigned)fp.C, (unsigned)B), dim3(DF_THREADS), smem,
+                                  (unsigned)fp.C, s, kmap, (const __nv_bfloat16 *)q_idx, rope, p, sa);
+    }
+    const DecodePlan pl = decode_index_plan(B, max_blocks, bf16);
     cudaError_t e = cudaMemsetAsync(d.hist, 0, d.zero_bytes, s);
     if (e != cudaSuccess) return e;
     DecodeParams p{seq_len, head_w, pool_stride, max_blocks, pl.chunk, kstride, pl.chunks, top_k, relu ? 1 : 0,

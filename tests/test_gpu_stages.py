@@ -237,12 +237,15 @@ def test_decode_pipeline(qsa, dtype, flags, weights, L, B):
         assert np.abs(lse[b].cpu().numpy() - ref["lse"][0]).max() <= (1e-3 if dtype == "bf16" else 1e-4)
 
 
-@pytest.mark.parametrize("dtype,flags", [("bf16", 0), ("bf16", 1), ("fp32", 0)])
-def test_decode_select_all_ties(qsa, dtype, flags):
+@pytest.mark.parametrize("dtype,flags,lens", [("bf16", 0, [40000, 65537, 2049]), ("bf16", 1, [40000, 65537, 2049]),
+                                              ("fp32", 0, [40000, 65537, 2049]),
+                                              ("bf16", 0, [65537, 40000, 2049, 17, 65000, 60001, 1, 64000, 65536,
+                                                          30000])])
+def test_decode_select_all_ties(qsa, dtype, flags, lens):
     """All compressed keys zero: every score is 0, so the top-k is the k lowest
-    block ids; with 10000+ blocks the tie bin spans several select chunks."""
-    B, top_k = 3, 512
-    lens = [40000, 65537, 2049]
+    block ids; with 10000+ blocks the tie bin spans several select chunks (and,
+    with 10 sequences, the single-kernel cluster path with candidate overflow)."""
+    B, top_k = len(lens), 512
     dt = torch.bfloat16 if dtype == "bf16" else torch.float32
     cap = max(lens) // 4 + 1
     k_pool = torch.zeros(B, cap, 128, dtype=dt, device=DEV)
