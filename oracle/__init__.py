@@ -190,17 +190,21 @@ def dense_rows(rows, q, k, v, Hq, Hkv, d, scale=None, q0=0, nthreads=None):
 
 def decode(q_idx, k_pool, seq_len, *, head_w=None, q=None, k=None, v=None, relu=False,
            store_bf16=True, top_k=512, Hq=16, Hkv=2, d=128, scale=None, base=10000.0,
-           pos_scale=1.0, rotary_dim=128, nthreads=None):
+           pos_scale=1.0, rotary_dim=128, nthreads=None, cap_len=None):
     """One decode step for B sequences (after pooling).
 
     q_idx [B][4][128]; k_pool [B][stride][128]; seq_len [B]; q [B][Hq][d];
     k, v [B][kv_stride][Hkv][d].  Returns sel, nsel, kth, next, out, lse.
+    cap_len [B] (IndexShare draft step): the selection is that of row
+    cap_len - 1 (q_idx is that row's indexer query); the attention at row
+    seq_len - 1 reads those blocks plus positions 4*floor(cap_len/4) .. seq_len - 1.
     """
     q_idx_a = _f32(q_idx)
     k_pool_a = _f32(k_pool)
     B = q_idx_a.shape[0]
     pool_stride = k_pool_a.shape[1]
     seq = np.ascontiguousarray(seq_len, dtype=np.int32)
+    cap = np.ascontiguousarray(cap_len, dtype=np.int32) if cap_len is not None else None
     if scale is None:
         scale = 1.0 / np.sqrt(d)
     head_w_a = _f32(head_w) if head_w is not None else None
@@ -215,7 +219,7 @@ def decode(q_idx, k_pool, seq_len, *, head_w=None, q=None, k=None, v=None, relu=
     out = np.zeros((B, Hq, d)) if q is not None else None
     lse = np.zeros((B, Hq)) if q is not None else None
     _L().oracle_decode(_p(q_idx_a), _p(k_pool_a), ctypes.c_int64(pool_stride), _p(head_w_a),
-                       _p(q_a), _p(k_a), _p(v_a), ctypes.c_int64(kv_stride), _p(seq),
+                       _p(q_a), _p(k_a), _p(v_a), ctypes.c_int64(kv_stride), _p(seq), _p(cap),
                        ctypes.c_int64(B), ctypes.c_int(int(relu)), ctypes.c_int(int(store_bf16)),
                        ctypes.c_int(top_k), ctypes.c_int(Hq), ctypes.c_int(Hkv), ctypes.c_int(d),
                        ctypes.c_double(scale), ctypes.c_double(base), ctypes.c_double(pos_scale),

@@ -20,6 +20,10 @@
  *   [ARCH] flozi.net architecture guide, "How a token moves through the
  *          model", item 2 "QSA's two stages" (RoPE after key pooling;
  *          512 complete blocks plus any incomplete tail block).
+ *   [MTP]  "Qwen3.8-Flash-Next: Day-0 Support in SGLang", section "IndexShare
+ *          MTP: Reusing the QSA Selection Across Draft Steps" (the selection
+ *          of the last accepted row is frozen for the draft loop; each draft
+ *          step reads it plus the positions drafted since).
  *
  * Readings where the pages are silent (each one is listed in the design
  * notes of the repository):
@@ -33,6 +37,10 @@
  *     4b + 3 <= t; the tail is positions 4*floor((t+1)/4) .. t;
  *   - ties in top-k go to the lower block index; fewer than k visible blocks
  *     means all of them;
+ *   - IndexShare draft step at position t with the selection frozen at the
+ *     capture row t_c <= t: the blocks selected for t_c plus every position
+ *     from t_c's first incomplete-block position 4*floor((t_c+1)/4) through t
+ *     (t_c's own tail and the positions drafted since, a contiguous range);
  *   - attention logits scaled by the caller's `scale` (1/sqrt(d) by default);
  *     q head h reads kv head floor(h * Hkv / Hq); one selection per query is
  *     shared by every head (the score has no head index).
@@ -280,22 +288,24 @@ int oracle_topk(const double *s, int64_t n, int k, int32_t *sel, double *kth, do
 static int64_t visible_blocks(int64_t t) { return (t + 1) / BLK; }
 
 /* Attention of one query at position t over the positions
- *   P(t) = {4b .. 4b+3 : b in sel[0..nsel)}  U  {4*nb(t) .. t},
- * q [Hq][d] (already rotated), k/v cache rows indexed by position
+ *   P(t) = {4b .. 4b+3 : b in sel[0..nsel)}  U  {tail_from .. t},
+ * where tail_from = 4*nb(t) for a query that selected its own blocks ([SGL]),
+ * or 4*nb(t_c) for an IndexShare draft step using the selection of row t_c
+ * ([MTP]).  q [Hq][d] (already rotated), k/v cache rows indexed by position
  * [pos][Hkv][d].  out [Hq][d] fp64; lse [Hq] natural-log log-sum-exp of the
  * scaled logits (may be NULL). */
-static void attend(const float *q, const float *kc, const float *vc, int64_t t,
+static void attend(const float *q, const float *kc, const float *vc, int64_t t, int64_t tail_from,
                    const int32_t *sel, int nsel, int Hq, int Hkv, int d, double scale,
                    double *out, double *lse)
 {
-    int64_t nb = visible_blocks(t);
-    int64_t ntail = t + 1 - BLK * nb;
+    int64_t ntail = t + 1 - tail_from;
+    if (ntail < 0) ntail = 0;
     int64_t npos = (int64_t)nsel * BLK + ntail;
     int64_t *pos = (int64_t *)malloc(sizeof(int64_t) * (size_t)(npos > 0 ? npos : 1));
     int64_t m = 0;
     for (int i = 0; i < nsel; ++i)
         for (int j = 0; j < BLK; ++j) pos[m++] = (int64_t)sel[i] * BLK + j;
-    for (int64_t j = 0; j < ntail; ++j) pos[m++] = BLK * nb + j;
+    for (int64_t j = 0; j < ntail; ++j) pos[m++] = tail_from + j;
 
     double *logit = (double *)malloc(sizeof(double) * (size_t)(npos > 0 ? npos : 1));
     for (int h = 0; h < Hq; ++h) {
@@ -426,7 +436,7 @@ static void run_row(const job_t *J, int64_t r)
         free(s);
     }
     if (J->out && J->q)
-        attend(J->q + i * J->Hq * J->d, J->k, J->v, t, sel, nsel, J->Hq, J->Hkv, J->d, J->scale,
+        attend(J->q + i * J->Hq * J->d, J->k, J->v, t, BLK * visible_blocks(t), sel, nsel, J->Hq, J->Hkv, J->d, J->scale,
                J->out + r * J->Hq * J->d, J->lse ? J->lse + r * J->Hq : NULL);
     free(sel_own);
 }
@@ -508,6 +518,7 @@ typedef struct {
     const float *k, *v;      /* [B][kv_stride][Hkv][d] caches incl. the new token */
     int64_t kv_stride;
     const int32_t *seq_len;  /* [B], tokens including the new one */
+    const int32_t *cap_len;  /* [B] or NULL: IndexShare, the selection is that of row cap_len - 1 */
     int relu, store_bf16, top_k, Hq, Hkv, d;
     double scale;
     orope_t rope;
@@ -520,9 +531,12 @@ typedef struct {
 static void decode_one(const djob_t *J, int64_t bi)
 {
     int64_t t = (int64_t)J->seq_len[bi] - 1;
-    int64_t nb = visible_blocks(t);
+    /* row whose selection is used: the new token itself, or the IndexShare
+     * capture row ([MTP]); q_idx is that row's indexer query */
+    int64_t t_sel = J->cap_len ? (int64_t)J->cap_len[bi] - 1 : t;
+    int64_t nb = visible_blocks(t_sel);
     double q_hat[IDX_HEADS * IDX_DIM];
-    rotate_query(J->q_idx + bi * IDX_HEADS * IDX_DIM, (double)t, &J->rope, J->store_bf16, q_hat);
+    rotate_query(J->q_idx + bi * IDX_HEADS * IDX_DIM, (double)t_sel, &J->rope, J->store_bf16, q_hat);
     double *s = (double *)malloc(sizeof(double) * (size_t)(nb > 0 ? nb : 1));
     index_scores(q_hat, J->k_pool + bi * J->pool_stride * IDX_DIM, nb,
                  J->head_w ? J->head_w + bi * IDX_HEADS : NULL, J->relu, s);
@@ -535,7 +549,7 @@ static void decode_one(const djob_t *J, int64_t bi)
     if (J->next) J->next[bi] = nxt;
     if (J->out && J->q) {
         int64_t kvoff = bi * J->kv_stride * J->Hkv * J->d;
-        attend(J->q + bi * J->Hq * J->d, J->k + kvoff, J->v + kvoff, t, sel, nsel,
+        attend(J->q + bi * J->Hq * J->d, J->k + kvoff, J->v + kvoff, t, BLK * nb, sel, nsel,
                J->Hq, J->Hkv, J->d, J->scale, J->out + bi * J->Hq * J->d,
                J->lse ? J->lse + bi * J->Hq : NULL);
     }
@@ -550,10 +564,14 @@ static void *dworker(void *arg)
 
 /* One QSA decode step for B sequences: score all floor(seq_len/4) compressed
  * blocks, select the top-k, attend over them plus the tail (the new token's
- * incomplete block).  The caller has already run oracle_pool_decode. */
+ * incomplete block).  The caller has already run oracle_pool_decode.
+ * With cap_len (IndexShare draft step, [MTP]): the selection is the one of row
+ * cap_len - 1 (q_idx is that row's indexer query, scored over the blocks it
+ * sees), and the attention at row seq_len - 1 reads those blocks plus every
+ * position from 4*floor(cap_len/4) through seq_len - 1. */
 void oracle_decode(const float *q_idx, const float *k_pool, int64_t pool_stride, const float *head_w,
                    const float *q, const float *k, const float *v, int64_t kv_stride,
-                   const int32_t *seq_len, int64_t B, int relu, int store_bf16, int top_k,
+                   const int32_t *seq_len, const int32_t *cap_len, int64_t B, int relu, int store_bf16, int top_k,
                    int Hq, int Hkv, int d, double scale, double base, double pos_scale, int rotary_dim,
                    int32_t *sel, int32_t *nsel, double *kth, double *next,
                    double *out, double *lse, int nthreads)
@@ -561,7 +579,7 @@ void oracle_decode(const float *q_idx, const float *k_pool, int64_t pool_stride,
     djob_t J;
     memset(&J, 0, sizeof J);
     J.q_idx = q_idx; J.k_pool = k_pool; J.pool_stride = pool_stride; J.head_w = head_w;
-    J.q = q; J.k = k; J.v = v; J.kv_stride = kv_stride; J.seq_len = seq_len;
+    J.q = q; J.k = k; J.v = v; J.kv_stride = kv_stride; J.seq_len = seq_len; J.cap_len = cap_len;
     J.relu = relu; J.store_bf16 = store_bf16; J.top_k = top_k; J.Hq = Hq; J.Hkv = Hkv; J.d = d;
     J.scale = scale; J.rope.base = base; J.rope.pos_scale = pos_scale; J.rope.rotary_dim = rotary_dim;
     J.sel = sel; J.nsel = nsel; J.kth = kth; J.next = next; J.out = out; J.lse = lse; J.B = B;

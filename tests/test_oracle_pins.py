@@ -394,3 +394,84 @@ def test_needle_recall_small():
     res = oracle.prefill_rows(rows, q_idx=q_idx, k_pool=kbar, top_k=w.top_k)
     for r, b in enumerate(blocks):
         assert b in set(res["sel"][r, :res["nsel"][r]].tolist())
+
+
+# ----------------------------------------------------------------------------- IndexShare draft steps
+
+def _pooled_cache(k_raw, n_tok, cap):
+    """Compressed keys of the first n_tok raw keys (complete blocks only)."""
+    kp = np.zeros((cap, 128), np.float32)
+    nb = n_tok // 4
+    if nb:
+        kp[:nb] = oracle.pool_keys(k_raw[:4 * nb])
+    return kp
+
+
+@pytest.mark.parametrize("t_c,drafts", [(4 * 300 + 2, [0, 1, 2, 5, 9]), (4 * 300 + 3, [0, 1, 4, 8]),
+                                         (4 * 300, [0, 3, 6])])
+def test_indexshare_draft_equals_dense_when_every_block_fits(t_c, drafts):
+    # With k >= nb(t_c) the frozen selection is every block visible to the
+    # capture row, and the draft step adds t_c's incomplete block and every
+    # drafted position: positions 0..t, i.e. full causal attention at t.
+    T = t_c + max(drafts) + 1
+    Hq, Hkv, d, k = 8, 2, 128, 512
+    assert k >= (t_c + 1) // 4
+    rng = np.random.default_rng(t_c)
+    k_raw = bf16(rng.standard_normal((T, 128)))
+    q_idx = bf16(rng.standard_normal((T, 4, 128)))
+    q = bf16(rng.standard_normal((T, Hq, d)))
+    kk = bf16(rng.standard_normal((T, Hkv, d)))
+    v = bf16(rng.standard_normal((T, Hkv, d)))
+    ref = _sdpa_causal(q, kk, v, Hq, Hkv)
+    kp = _pooled_cache(k_raw, t_c + 1, T // 4 + 1)
+    for j in drafts:
+        t = t_c + j
+        res = oracle.decode(q_idx[t_c][None], kp[None], [t + 1], cap_len=[t_c + 1], q=q[t][None], k=kk[None],
+                            v=v[None], top_k=k, Hq=Hq, Hkv=Hkv, d=d)
+        assert res["nsel"][0] == (t_c + 1) // 4
+        np.testing.assert_allclose(res["out"][0], ref[t], rtol=0, atol=1e-12)
+
+
+def test_indexshare_capture_row_is_a_plain_decode_step():
+    # At t == t_c the draft step reads the capture row's own selection and tail.
+    T, k, Hq, Hkv, d = 4 * 200 + 1, 32, 4, 1, 128
+    rng = np.random.default_rng(5)
+    k_raw = bf16(rng.standard_normal((T, 128)))
+    q_idx = bf16(rng.standard_normal((T, 4, 128)))
+    q = bf16(rng.standard_normal((T, Hq, d)))
+    kk = bf16(rng.standard_normal((T, Hkv, d)))
+    v = bf16(rng.standard_normal((T, Hkv, d)))
+    t = T - 1
+    kp = _pooled_cache(k_raw, T, T // 4 + 1)
+    plain = oracle.decode(q_idx[t][None], kp[None], [T], q=q[t][None], k=kk[None], v=v[None], top_k=k, Hq=Hq,
+                          Hkv=Hkv, d=d)
+    shared = oracle.decode(q_idx[t][None], kp[None], [T], cap_len=[T], q=q[t][None], k=kk[None], v=v[None],
+                           top_k=k, Hq=Hq, Hkv=Hkv, d=d)
+    np.testing.assert_array_equal(plain["sel"], shared["sel"])
+    np.testing.assert_array_equal(plain["out"], shared["out"])
+
+
+def test_indexshare_keeps_the_frozen_selection_and_sees_drafted_positions():
+    # The draft step at t = t_c + 3 must (1) attend over the blocks selected for
+    # t_c, not re-select, and (2) see the drafted positions t_c + 1 .. t: a key
+    # planted only at a drafted position, aligned with the query, carries its
+    # value to the output.
+    T, k, Hq, Hkv, d = 4 * 400 + 2, 16, 1, 1, 128
+    rng = np.random.default_rng(9)
+    k_raw = bf16(rng.standard_normal((T + 8, 128)))
+    q_idx = bf16(rng.standard_normal((T + 8, 4, 128)))
+    q = bf16(rng.standard_normal((T + 8, Hq, d)) * 0.1)
+    kk = bf16(rng.standard_normal((T + 8, Hkv, d)) * 0.1)
+    v = np.zeros((T + 8, Hkv, d), np.float32)
+    t_c, t = T - 1, T + 2
+    u = np.zeros(d, np.float32)
+    u[7] = 1.0
+    q[t, 0] = 30.0 * u
+    kk[t_c + 2, 0] = 30.0 * u          # drafted position
+    v[t_c + 2, 0, 3] = 1.0
+    kp = _pooled_cache(k_raw, T, (T + 8) // 4 + 1)
+    res = oracle.decode(q_idx[t_c][None], kp[None], [t + 1], cap_len=[t_c + 1], q=q[t][None], k=kk[None],
+                        v=v[None], top_k=k, Hq=Hq, Hkv=Hkv, d=d)
+    cap = oracle.decode(q_idx[t_c][None], kp[None], [t_c + 1], top_k=k)
+    np.testing.assert_array_equal(res["sel"], cap["sel"])          # frozen, not re-selected
+    assert res["out"][0, 0, 3] > 0.99                                # the drafted key wins
