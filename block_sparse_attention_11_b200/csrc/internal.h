@@ -119,8 +119,11 @@ struct AttnArgs {
     void *out;
     float *lse;
     bool decode;
+    const int32_t *cap_len = nullptr;   // decode, IndexShare draft step: [B] capture rows + 1
+    int max_draft = 0;                  // IndexShare: largest seq_len - cap_len
 };
-size_t attn_decode_ws_bytes(int B, int Hq, int d, int top_k);
+int attn_tail_blocks(bool indexshare, int max_draft);
+size_t attn_decode_ws_bytes(int B, int Hq, int d, int top_k, int tail_blocks = 1);
 cudaError_t launch_attn_bf16(const AttnArgs &a, void *ws, unsigned *status, cudaStream_t s);
 cudaError_t launch_attn_f32(const AttnArgs &a, unsigned *status, cudaStream_t s);
 

@@ -102,11 +102,16 @@ struct AttnParams {
     float *lse;
     float *part_o;         // decode: [B][splits][Hq][128]
     float *part_lse;       // decode: [B][splits][Hq] (log2 domain)
+    const int32_t *cap_len;  // decode, IndexShare: [B] capture rows + 1 (null: plain decode)
+    int max_draft;           // IndexShare: largest seq_len - cap_len
     unsigned *status;
 };
 
 // The key list of one work item: positions lbeg..lend of
-// [sel[0..nsel), tail block (if tail > 0)].
+// [sel[0..nsel), tail blocks].  The tail is positions 4*nb .. t: the query's
+// own incomplete block (0-3 tokens), or, for an IndexShare draft step, the
+// capture row's incomplete block and every position drafted since (nb is then
+// the capture row's visible block count), as ceil(tail / 4) blocks.
 struct Item {
     int seq;
     int64_t row;       // prefill: query row; decode: split index
@@ -142,10 +147,18 @@ __device__ __forceinline__ Item get_item(const AttnParams &p, int64_t i) {
         if (it.t >= p.kv_stride) flag(p.status, QSA_DEV_BAD_LENGTH);
         it.t = -1;   // nothing visible: the item attends to no position
     }
-    it.nb = (it.t + 1) / kBlock;
+    int64_t t_sel = it.t;   // the row whose selection the item reads
+    if (p.decode && p.cap_len && it.t >= 0) {
+        t_sel = (int64_t)p.cap_len[it.seq] - 1;
+        if (t_sel < 0 || t_sel > it.t || it.t - t_sel > p.max_draft) {
+            flag(p.status, QSA_DEV_BAD_LENGTH);
+            t_sel = it.t;   // read as a plain decode step
+        }
+    }
+    it.nb = (t_sel + 1) / kBlock;
     it.tail = (int)(it.t + 1 - kBlock * it.nb);
     it.nsel = max(0, min(it.nsel, p.top_k));
-    const int len = it.nsel + (it.tail > 0 ? 1 : 0);
+    const int len = it.nsel + (it.tail + kBlock - 1) / kBlock;
     if (!p.decode) {
         it.lbeg = 0;
         it.lend = len;
@@ -235,7 +248,7 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, AttnCfg<HKV>::kMinCtas
                             if (b >= 0 && b < it.nb) tokens = kBlock;
                             else flag(p.status, QSA_DEV_BAD_INDEX);
                         } else {
-                            tokens = it.tail;
+                            tokens = min(kBlock, it.tail - kBlock * (e - it.nsel));
                         }
                     }
                     info |= (uint32_t)tokens << (3 * j);
@@ -267,7 +280,7 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, AttnCfg<HKV>::kMinCtas
                     const int e = it.lbeg + AT_BPS * st + j;
                     const int tokens = (int)((st_info[st] >> (3 * j)) & 7u);
                     if (tokens > 0) {
-                        const int64_t blk = (e < it.nsel) ? (int64_t)ids[e - it.lbeg] : it.nb;
+                        const int64_t blk = (e < it.nsel) ? (int64_t)ids[e - it.lbeg] : it.nb + (e - it.nsel);
                         const int64_t off = (kv0 + blk * kBlock) * HKV * 128;
                         const uint32_t nbytes = (uint32_t)tokens * HKV * 256u;
                         bulk_g2s(sm.stage[s] + j * Cfg::kSlot, p.k + off, nbytes, &sm.full[s]);
@@ -591,7 +604,8 @@ __global__ void __launch_bounds__(256) attn_f32_kernel(const float *__restrict__
                                                         const int32_t *__restrict__ seq_len, int B, int64_t n_q,
                                                         int64_t q0, int64_t kv_stride, int Hq, int Hkv, int top_k,
                                                         float scale, float *__restrict__ out, float *__restrict__ lse,
-                                                        int decode, unsigned *status) {
+                                                        int decode, const int32_t *__restrict__ cap_len, int max_draft,
+                                                        unsigned *status) {
     const int64_t wid = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     const int64_t items = decode ? (int64_t)B : (int64_t)B * n_q;
@@ -607,14 +621,22 @@ __global__ void __launch_bounds__(256) attn_f32_kernel(const float *__restrict__
         if (lane == 0) flag(status, QSA_DEV_BAD_LENGTH);
         t = -1;   // nothing visible
     }
-    const int64_t nb = (t + 1) / kBlock;
-    const int tail = (int)(t + 1 - kBlock * nb);
+    int64_t t_sel = t;   // the row whose selection is read (IndexShare: the capture row)
+    if (decode && cap_len && t >= 0) {
+        t_sel = (int64_t)cap_len[seq] - 1;
+        if (t_sel < 0 || t_sel > t || t - t_sel > max_draft) {
+            if (lane == 0) flag(status, QSA_DEV_BAD_LENGTH);
+            t_sel = t;
+        }
+    }
+    const int64_t nb = (t_sel + 1) / kBlock;
+    const int tail = (int)(t + 1 - kBlock * nb);     // positions 4*nb .. t
     const int32_t *sl = sel + qi * top_k;
     const int nsel = max(0, min(nsel_p[qi], top_k));
     const float4 qv = reinterpret_cast<const float4 *>(q + (qi * Hq + h) * 128)[lane];
     float m = -INFINITY, l = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    const int len = nsel + (tail > 0 ? 1 : 0);
+    const int len = nsel + (tail + kBlock - 1) / kBlock;
     for (int e = 0; e < len; ++e) {
         int64_t b;
         int ntok;
@@ -626,8 +648,8 @@ __global__ void __launch_bounds__(256) attn_f32_kernel(const float *__restrict__
                 continue;
             }
         } else {
-            b = nb;
-            ntok = tail;
+            b = nb + (e - nsel);
+            ntok = min(kBlock, tail - kBlock * (e - nsel));
         }
         for (int j = 0; j < ntok; ++j) {
             const int64_t row = ((int64_t)seq * kv_stride + b * kBlock + j) * Hkv + g;
@@ -654,16 +676,16 @@ __global__ void __launch_bounds__(256) attn_f32_kernel(const float *__restrict__
     if (lse && lane == 0) lse[qi * Hq + h] = l > 0.f ? m + logf(l) : -INFINITY;
 }
 
-// Decode split-KV plan: each sequence's list of top_k + 1 entries (ceil((top_k+1)/8)
-// stages) is cut into `splits` items of S stages; the persistent grid of `cap`
+// Decode split-KV plan: each sequence's list of at most list_max entries (top_k
+// blocks + tail blocks; ceil(list_max/8) stages) is cut into `splits` items of S stages; the persistent grid of `cap`
 // CTAs takes ceil(items / cap) rounds.  S minimises rounds x (S + 1) (one stage
 // of start-up per item), ties going to fewer splits.
 struct SplitPlan {
     int splits, split_blocks;
 };
 
-SplitPlan decode_split_plan(int B, int top_k, int64_t cap) {
-    const int nst = (top_k + 1 + AT_BPS - 1) / AT_BPS;
+SplitPlan decode_split_plan(int B, int list_max, int64_t cap) {
+    const int nst = (list_max + AT_BPS - 1) / AT_BPS;
     SplitPlan best{1, nst * AT_BPS};
     int64_t best_cost = -1;
     for (int S = nst; S >= 1; --S) {
@@ -678,6 +700,16 @@ SplitPlan decode_split_plan(int B, int top_k, int64_t cap) {
     }
     return best;
 }
+
+}  // namespace
+
+// Tail blocks of one item's list: the query's own incomplete block, or for an
+// IndexShare draft step the capture row's (0-3 tokens) plus max_draft positions.
+int attn_tail_blocks(bool indexshare, int max_draft) {
+    return indexshare ? (3 + max_draft + kBlock - 1) / kBlock : 1;
+}
+
+namespace {
 
 template <int HKV>
 cudaError_t run_bf16(const AttnArgs &a, void *ws, unsigned *status, cudaStream_t s) {
@@ -701,8 +733,12 @@ cudaError_t run_bf16(const AttnArgs &a, void *ws, unsigned *status, cudaStream_t
     p.out = (__nv_bfloat16 *)a.out;
     p.lse = a.lse;
     p.status = status;
+    p.cap_len = a.decode ? a.cap_len : nullptr;
+    p.max_draft = a.max_draft;
+    // entries of one item's list: top_k blocks + the tail blocks
+    const int list_max = a.top_k + attn_tail_blocks(a.decode && a.cap_len, a.max_draft);
     if (a.decode) {
-        const SplitPlan sp = decode_split_plan(a.B, a.top_k, (int64_t)sms * Cfg::kMinCtas);
+        const SplitPlan sp = decode_split_plan(a.B, list_max, (int64_t)sms * Cfg::kMinCtas);
         const int splits = sp.splits;
         p.splits = splits;
         p.split_blocks = sp.split_blocks;
@@ -718,7 +754,7 @@ cudaError_t run_bf16(const AttnArgs &a, void *ws, unsigned *status, cudaStream_t
     if (p.items <= 0) return cudaSuccess;
     // an item's list holds at most top_k ids plus the tail block
     p.sel_cap = (a.top_k + 3) & ~3;
-    p.nst_cap = (a.top_k + 1 + AT_BPS - 1) / AT_BPS;
+    p.nst_cap = (list_max + AT_BPS - 1) / AT_BPS;
     const size_t smem = attn_smem_bytes<HKV>(p.sel_cap, p.nst_cap);
     if (di && smem > di->smem_optin) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(attn_bf16_kernel<HKV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -736,11 +772,13 @@ cudaError_t run_bf16(const AttnArgs &a, void *ws, unsigned *status, cudaStream_t
 
 }  // namespace
 
-size_t attn_decode_ws_bytes(int B, int Hq, int d, int top_k) {
+size_t attn_decode_ws_bytes(int B, int Hq, int d, int top_k, int tail_blocks) {
     // the larger of the split plans run_bf16 can pick (1 or 2 resident CTAs per SM)
     const DeviceInfo *di = device_info();
     const int sms = di ? di->sm_count : 148;
-    const int splits = std::max(decode_split_plan(B, top_k, sms).splits, decode_split_plan(B, top_k, 2 * sms).splits);
+    const int list_max = top_k + tail_blocks;
+    const int splits =
+        std::max(decode_split_plan(B, list_max, sms).splits, decode_split_plan(B, list_max, 2 * sms).splits);
     size_t n = (size_t)B * splits * Hq;
     return (n * d * sizeof(float) + n * sizeof(float) + 255) / 256 * 256;
 }
@@ -760,7 +798,8 @@ cudaError_t launch_attn_f32(const AttnArgs &a, unsigned *status, cudaStream_t s)
     if (warps <= 0) return cudaSuccess;
     attn_f32_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, s>>>(
         (const float *)a.q, (const float *)a.k, (const float *)a.v, a.sel, a.nsel, a.seq_len, a.B, a.n_q, a.q0,
-        a.kv_stride, a.Hq, a.Hkv, a.top_k, a.scale, (float *)a.out, a.lse, a.decode ? 1 : 0, status);
+        a.kv_stride, a.Hq, a.Hkv, a.top_k, a.scale, (float *)a.out, a.lse, a.decode ? 1 : 0,
+        a.decode ? a.cap_len : nullptr, a.max_draft, status);
     return cudaGetLastError();
 }
 

@@ -323,6 +323,35 @@ int qsa_sparse_attn_decode(const void *q, const void *k, const void *v, const in
     return cuda_status(launch_attn_f32(a, di->status, s));
 }
 
+size_t qsa_sparse_attn_decode_shared_workspace(int32_t B, int32_t Hq, int32_t d, int32_t top_k, int32_t max_draft,
+                                               int32_t dtype) {
+    if (B < 1 || Hq < 1 || d < 1 || top_k < 1 || max_draft < 0 || max_draft > 64) return 0;
+    if (dtype != QSA_BF16) return 0;
+    return attn_decode_ws_bytes(B, Hq, d, top_k, attn_tail_blocks(true, max_draft));
+}
+
+int qsa_sparse_attn_decode_shared(const void *q, const void *k, const void *v, const int32_t *seq_len,
+                                  const int32_t *cap_len, const int32_t *sel, const int32_t *nsel, int32_t B,
+                                  int64_t kv_stride, int32_t Hq, int32_t Hkv, int32_t d, int32_t top_k,
+                                  int32_t max_draft, float scale, void *out, float *lse, void *workspace,
+                                  size_t ws_bytes, int32_t dtype, void *stream) {
+    int st = attn_common_checks(q, k, v, sel, nsel, B, Hq, Hkv, d, top_k, scale, out, dtype);
+    if (st != QSA_OK) return st;
+    if (!seq_len || !cap_len || kv_stride < 1 || max_draft < 0 || max_draft > 64) return QSA_ERR_INVALID_ARG;
+    const DeviceInfo *di = nullptr;
+    if ((st = check_device(&di)) != QSA_OK) return st;
+    AttnArgs a{q, k, v, sel, nsel, seq_len, B, 1, 0, kv_stride, Hq, Hkv, d, top_k, scale, out, lse, true};
+    a.cap_len = cap_len;
+    a.max_draft = max_draft;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dtype == QSA_BF16) {
+        const size_t need = attn_decode_ws_bytes(B, Hq, d, top_k, attn_tail_blocks(true, max_draft));
+        if (!workspace || ws_bytes < need) return QSA_ERR_WORKSPACE;
+        return cuda_status(launch_attn_bf16(a, workspace, di->status, s));
+    }
+    return cuda_status(launch_attn_f32(a, di->status, s));
+}
+
 int qsa_rope_apply(void *x, int32_t B, int64_t n, int32_t H, int32_t d, int64_t pos0, qsa_rope_t rope, int32_t dtype,
                    void *stream) {
     if (!x || B < 1 || n < 0 || H < 1 || d < 2 || (d % 2) != 0 || pos0 < 0) return QSA_ERR_INVALID_ARG;

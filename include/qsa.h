@@ -266,6 +266,33 @@ QSA_API int qsa_sparse_attn_decode(const void *q, const void *k, const void *v, 
                            float *lse, void *workspace, size_t ws_bytes, int32_t dtype, void *stream);
 
 /* ========================================================================= */
+/* IndexShare draft step: decode attention over a frozen selection            */
+/* ========================================================================= */
+/*
+ * Page "Qwen3.8-Flash-Next: Day-0 Support in SGLang", section "IndexShare MTP:
+ * Reusing the QSA Selection Across Draft Steps": the selection computed for
+ * the last accepted row is held for the whole draft loop; each draft decode
+ * step skips the indexer and reads that selection plus the positions drafted
+ * since.  The query of sequence i is at t = seq_len[i] - 1; the capture row is
+ * t_c = cap_len[i] - 1 (0 <= t_c <= t <= t_c + max_draft).  It attends over
+ *   the blocks in sel/nsel (written by qsa_index_topk_decode for the capture
+ *   row, i.e. with seq_len = cap_len; ids b < floor(cap_len / 4)), and
+ *   every position from 4 * floor(cap_len / 4) through t (the capture row's
+ *   incomplete block and the drafted positions, the new token included).
+ * Other arguments as qsa_sparse_attn_decode.  A sequence outside the stated
+ * range of cap_len is read as a plain decode step and flagged in the status
+ * word (QSA_DEV_BAD_LENGTH).  max_draft in [0, 64].
+ * workspace at least qsa_sparse_attn_decode_shared_workspace() bytes.
+ */
+QSA_API size_t qsa_sparse_attn_decode_shared_workspace(int32_t B, int32_t Hq, int32_t d, int32_t top_k,
+                                                       int32_t max_draft, int32_t dtype);
+QSA_API int qsa_sparse_attn_decode_shared(const void *q, const void *k, const void *v, const int32_t *seq_len,
+                                          const int32_t *cap_len, const int32_t *sel, const int32_t *nsel,
+                                          int32_t B, int64_t kv_stride, int32_t Hq, int32_t Hkv, int32_t d,
+                                          int32_t top_k, int32_t max_draft, float scale, void *out, float *lse,
+                                          void *workspace, size_t ws_bytes, int32_t dtype, void *stream);
+
+/* ========================================================================= */
 /* Decode sparse attention without a workspace (allocation-free callers)      */
 /* ========================================================================= */
 /*

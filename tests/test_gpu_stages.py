@@ -310,3 +310,71 @@ def test_decode_step_graph_replay_matches_eager(qsa):
     qsa.qsa_check_status()
     for a, b in zip(eager, graphed):
         assert torch.equal(a, b)
+
+
+# ----------------------------------------------------------------------------- IndexShare draft steps
+
+@pytest.mark.parametrize("dtype,Hq,Hkv,B,L,top_k,max_draft", [("bf16", 16, 2, 6, 9000, 256, 8),
+                                                               ("bf16", 8, 1, 3, 2500, 64, 13),
+                                                               ("fp32", 8, 1, 3, 3000, 64, 5),
+                                                               ("bf16", 32, 4, 2, 1800, 512, 3)])
+def test_indexshare_draft_step_on_oracle_selection(qsa, dtype, Hq, Hkv, B, L, top_k, max_draft):
+    """Draft steps after a capture row: the GPU attention, fed the selection the
+    oracle made for the capture row, matches the oracle's draft step for every
+    number of drafted positions 0..max_draft (ragged over sequences)."""
+    d = 128
+    dt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    g = torch.Generator().manual_seed(L + B)
+    kv_len = L + max_draft + 8
+    k = torch.randn(B, kv_len, Hkv, d, generator=g).to(dt)
+    v = torch.randn(B, kv_len, Hkv, d, generator=g).to(dt)
+    q = torch.randn(B, Hq, d, generator=g).to(dt)
+    k_raw = torch.randn(B, kv_len, 128, generator=g).to(dt)
+    q_idx = torch.randn(B, 4, 128, generator=g).to(dt)
+    # capture rows t_c = cap_len - 1 with every residue mod 4 (and a short one)
+    cap = [L - (i % 4) for i in range(B)]
+    cap[-1] = 3 if B > 2 else cap[-1]
+    pool_cap = kv_len // 4 + 1
+    kp = np.zeros((B, pool_cap, 128), np.float32)
+    for b in range(B):
+        nb = cap[b] // 4
+        if nb:
+            kp[b, :nb] = oracle.pool_keys(np32(k_raw[b, :4 * nb]), store_bf16=dtype == "bf16")
+    ref_sel = oracle.decode(np32(q_idx), kp, cap, top_k=top_k, store_bf16=dtype == "bf16")
+    sel = torch.from_numpy(ref_sel["sel"]).to(DEV)
+    nsel = torch.from_numpy(ref_sel["nsel"]).to(DEV)
+    kd, vd, qd = k.to(DEV), v.to(DEV), q.to(DEV)
+    for step in range(max_draft + 1):
+        drafted = [(step + b) % (max_draft + 1) for b in range(B)]
+        seq = [cap[b] + drafted[b] for b in range(B)]
+        out = torch.empty_like(qd)
+        lse = torch.empty(B, Hq, dtype=torch.float32, device=DEV)
+        qsa.qsa_sparse_attn_decode_shared(qd, kd, vd, torch.tensor(seq, dtype=torch.int32, device=DEV),
+                                          torch.tensor(cap, dtype=torch.int32, device=DEV), sel, nsel, out,
+                                          max_draft, top_k=top_k, lse=lse)
+        qsa.qsa_check_status()
+        ref = oracle.decode(np32(q_idx), kp, seq, cap_len=cap, q=np32(q), k=np32(k), v=np32(v), top_k=top_k,
+                            Hq=Hq, Hkv=Hkv, d=d, store_bf16=dtype == "bf16")
+        np.testing.assert_array_equal(ref["sel"], ref_sel["sel"])
+        err = np.abs(np32(out) - ref["out"]).max()
+        assert err <= TOL[dtype], (step, err)
+        assert np.abs(lse.cpu().numpy() - ref["lse"]).max() <= (1e-3 if dtype == "bf16" else 1e-4)
+
+
+def test_indexshare_flags_out_of_range_capture(qsa):
+    """seq_len < cap_len, or more drafted positions than max_draft, is read as
+    a plain decode step and reported through the status word (no trap)."""
+    B, Hq, Hkv, d, L = 2, 16, 2, 128, 600
+    g = torch.Generator().manual_seed(3)
+    k = torch.randn(B, L + 40, Hkv, d, generator=g).to(torch.bfloat16).to(DEV)
+    v = torch.randn(B, L + 40, Hkv, d, generator=g).to(torch.bfloat16).to(DEV)
+    q = torch.randn(B, Hq, d, generator=g).to(torch.bfloat16).to(DEV)
+    sel = torch.full((B, 64), -1, dtype=torch.int32, device=DEV)
+    nsel = torch.zeros(B, dtype=torch.int32, device=DEV)
+    out = torch.empty_like(q)
+    for seq, cap in [([L, L], [L + 1, L]), ([L + 9, L], [L, L])]:   # behind the capture; 9 > max_draft 4
+        qsa.qsa_sparse_attn_decode_shared(q, k, v, torch.tensor(seq, dtype=torch.int32, device=DEV),
+                                          torch.tensor(cap, dtype=torch.int32, device=DEV), sel, nsel, out, 4)
+        with pytest.raises(qsa.QSAError):
+            qsa.qsa_check_status()
+        qsa.qsa_check_status()        # cleared

@@ -75,6 +75,13 @@ def test_invalid_arguments_are_rejected_before_launch(qsa):
     # kv cache shorter than the queries
     assert lib.qsa_sparse_attn_prefill(fake, fake, fake, fake, fake, 1, 8, 0, 4, 16, 2, 128, 8, 0.1, fake, None,
                                        None, 0, 0, None) == qsa.QSA_ERR_INVALID_ARG
+    # IndexShare draft step: capture lengths required, max_draft in [0, 64]
+    assert lib.qsa_sparse_attn_decode_shared(fake, fake, fake, fake, None, fake, fake, 1, 64, 16, 2, 128, 8, 4, 0.1,
+                                             fake, None, fake, 1 << 20, 0, None) == qsa.QSA_ERR_INVALID_ARG
+    assert lib.qsa_sparse_attn_decode_shared(fake, fake, fake, fake, fake, fake, fake, 1, 64, 16, 2, 128, 8, 65,
+                                             0.1, fake, None, fake, 1 << 20, 0, None) == qsa.QSA_ERR_INVALID_ARG
+    assert lib.qsa_sparse_attn_decode_shared_workspace(4, 16, 128, 512, -1, 0) == 0
+    assert lib.qsa_sparse_attn_decode_shared_workspace(4, 16, 128, 512, 8, 1) == 0     # fp32 needs none
     # misaligned pointer
     odd = ctypes.c_void_p(4098)
     assert lib.qsa_pool_keys_prefill(odd, fake, 1, 16, 0, 16, 4, rope, 0, 0, None) == qsa.QSA_ERR_INVALID_ARG
