@@ -287,6 +287,78 @@ class DecodeRunner:
         return {k: self.x[k].cpu().pin_memory() for k in keys}
 
 
+class DraftRunner:
+    """IndexShare draft step: the selection of the capture row (the cache's
+    new token) is made once, untimed; each timed step is the draft token's
+    attention over that frozen selection plus the positions drafted since."""
+
+    def __init__(self, w, dev):
+        import block_sparse_attention_11_b200 as qsa
+        self.qsa = qsa
+        self.w = w
+        self.dev = dev
+        x = workloads.make_decode(w, device=dev)
+        self.x = x
+        dt = workloads.torch_dtype(w)
+        B, L = w.B, w.T
+        self.drafted = int(w.extra["drafted"])
+        self.max_draft = int(w.extra["max_draft"])
+        rope = qsa.Rope(base=w.rope_base, pos_scale=w.pos_scale, rotary_dim=128)
+        cap = L // 4 + 1
+        k_pool = torch.zeros(B, cap, 128, dtype=dt, device=dev)
+        qsa.qsa_pool_keys_prefill(x["k_idx"], k_pool, rope=rope)
+        ring = torch.zeros(B, 4, 128, dtype=dt, device=dev)
+        qsa.qsa_pool_keys_decode(x["k_idx_new"], ring, k_pool, x["seq_len"], rope=rope)
+        self.sel = torch.empty(B, w.top_k, dtype=torch.int32, device=dev)
+        self.nsel = torch.empty(B, dtype=torch.int32, device=dev)
+        qsa.qsa_index_topk_decode(x["q_idx"], k_pool, x["seq_len"], self.sel, self.nsel, max_blocks=(L + 1) // 4,
+                                  top_k=w.top_k, rope=rope)      # the capture row's selection (setup)
+        torch.cuda.synchronize()
+        del x["k_idx"], k_pool
+        torch.cuda.empty_cache()
+        x["cap_len"] = x["seq_len"].clone()
+        x["seq_len"] = x["seq_len"] + self.drafted
+        self.out = torch.empty_like(x["q"])
+        self.ws_a = torch.empty(qsa.qsa_sparse_attn_decode_shared_workspace(B, w.Hq, w.d, w.top_k, self.max_draft),
+                                dtype=torch.uint8, device=dev)
+        self.flush_between_steps = False      # K/V caches of several GB
+        self.use_graph = True
+
+    def step(self, x=None, events=None):
+        qsa, w = self.qsa, self.w
+        x = x or self.x
+        if events is not None:
+            events[0].record()
+            events[1].record()
+            events[2].record()
+        qsa.qsa_sparse_attn_decode_shared(x["q"], x["k"], x["v"], x["seq_len"], x["cap_len"], self.sel, self.nsel,
+                                          self.out, self.max_draft, workspace=self.ws_a)
+        if events is not None:
+            events[3].record()
+        return self.out
+
+    def launches_per_step(self):
+        return 2   # attention, combine
+
+    def units(self):
+        return self.w.B
+
+    def stage_names(self):
+        return ["pool_ring_skipped", "index_skipped_frozen_selection", "sparse_attn"]
+
+    def algorithmic(self):
+        w = self.w
+        t_c = w.T                                   # capture row (the cache's new token)
+        nb = (t_c + 1) // 4
+        npos = min(nb, w.top_k) * 4 + (t_c + self.drafted + 1 - 4 * nb)
+        kv_bytes = npos * w.Hkv * w.d * 2 * 2 + 2 * w.Hq * w.d * 2
+        return dict(attn_bytes=kv_bytes * w.B, step_bytes=kv_bytes * w.B, positions=npos)
+
+    def host_inputs(self):
+        keys = ["q", "seq_len", "cap_len"]
+        return {k: self.x[k].cpu().pin_memory() for k in keys}
+
+
 # ----------------------------------------------------------------------------- measurement
 
 def flush_l2(buf):
@@ -311,7 +383,7 @@ def run_ours(args, rank, world):
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
     w = workloads.WORKLOADS[args.workload]
-    runner = (PrefillRunner if w.kind == "prefill" else DecodeRunner)(w, dev)
+    runner = {"prefill": PrefillRunner, "decode": DecodeRunner, "draft": DraftRunner}[w.kind](w, dev)
     flush = torch.zeros(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
     qsa = runner.qsa
     for _ in range(args.warmup):
@@ -445,6 +517,21 @@ def run_ours(args, rank, world):
         res["config"] = dict(workload=w.name, B=w.B, T=w.T, top_k=w.top_k, Hq=w.Hq, Hkv=w.Hkv, d=w.d,
                              needles=w.needles, l2="flushed between timed steps (256 MB write)",
                              parallelism=f"replicas x{world}")
+    elif w.kind == "draft":
+        res.update(metric="QSA IndexShare draft step us/step", unit="us/step", higher_is_better=False,
+                   value=ms_per_step * 1e3)
+        res["e2e"] = dict(value=e2e_ms * 1e3, unit="us/step", h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h,
+                          graph=used_graph, eager_value=e2e_eager_ms * 1e3)
+        achieved = alg["attn_bytes"] / (ms_per_step / 1e3) / 1e9
+        res["roofline"] = dict(kernel="sparse_attn_decode (frozen selection)", bound="hbm", achieved=achieved,
+                               peak=pk["hbm_gbs"], unit="GB/s", frac=achieved / pk["hbm_gbs"], traffic=None,
+                               peak_kind=pk_kind,
+                               note=f"algorithmic bytes = {alg['positions']} gathered positions per sequence x Hkv x "
+                                    f"d x 2 B x 2 + q/out; time = the graph-replayed step (attention + combine)")
+        res["config"] = dict(workload=w.name, B=w.B, L=w.T, top_k=w.top_k, Hq=w.Hq, Hkv=w.Hkv, d=w.d,
+                             drafted=w.extra["drafted"],
+                             l2="inputs larger than L2 (K/V caches)", parallelism=f"replicas x{world}",
+                             cuda_graph=True)
     else:
         res.update(metric="QSA decode us/step", unit="us/step", higher_is_better=False,
                    value=ms_per_step * 1e3)
@@ -509,18 +596,31 @@ def run_oracle_sample(w, budget_s=15.0, seed=0):
     kr = x["k_idx"][0].float().numpy()
     kp = oracle.pool_keys(kr, base=w.rope_base, pos_scale=w.pos_scale, store_bf16=True)
     q, k, v = x["q"].float().numpy(), x["k"].float().numpy(), x["v"].float().numpy()
+    seq_len = x["seq_len"].numpy()
+    cap_len = None
+    if w.kind == "draft":                # the drafted positions follow the capture row
+        cap_len = seq_len.copy()
+        seq_len = seq_len + int(w.extra["drafted"])
     t0 = time.perf_counter()
     reps = 0
     while True:
-        oracle.decode(x["q_idx"].float().numpy(), kp[None], x["seq_len"].numpy(), q=q, k=k, v=v, top_k=w.top_k,
-                      base=w.rope_base, pos_scale=w.pos_scale, Hq=w.Hq, Hkv=w.Hkv, d=w.d, nthreads=nthreads)
+        oracle.decode(x["q_idx"].float().numpy(), kp[None], seq_len, cap_len=cap_len, q=q, k=k, v=v,
+                      top_k=w.top_k, base=w.rope_base, pos_scale=w.pos_scale, Hq=w.Hq, Hkv=w.Hkv, d=w.d,
+                      nthreads=nthreads)
         reps += 1
         if time.perf_counter() - t0 > min(budget_s, 5.0):
             break
     per_seq = (time.perf_counter() - t0) / reps
-    value = per_seq * w.B * 1e6          # a decode step of all B sequences, us
+    value = per_seq * w.B * 1e6          # a step of all B sequences, us
     sample = f"{reps} decode steps of one {w.T}-token sequence, scaled to B={w.B}"
+    if w.kind == "draft":
+        sample += " (the oracle selects for the capture row on every step: it takes no frozen selection)"
     return value, sample, nthreads, "us/step"
+
+
+def metric_name(w):
+    return {"prefill": "QSA prefill tokens/s", "decode": "QSA decode us/step",
+            "draft": "QSA IndexShare draft step us/step"}[w.kind]
 
 
 def main():
@@ -554,8 +654,8 @@ def main():
     if args.impl == "reference":
         if rank == 0:
             value, sample, threads, unit = run_oracle_sample(w, budget_s=args.cpu_budget)
-            line = dict(impl="reference", metric="QSA prefill tokens/s" if w.kind == "prefill" else
-                        "QSA decode us/step", value=value, unit=unit, higher_is_better=w.kind == "prefill",
+            line = dict(impl="reference", metric=metric_name(w), value=value, unit=unit,
+                        higher_is_better=w.kind == "prefill",
                         n_gpus=args.gpus, steps=args.steps, warmup=args.warmup, dtype=w.dtype, data="synthetic",
                         config=dict(workload=w.name), vs_baseline=None,
                         cpu_baseline=dict(value=value, unit=unit, cores=threads, kind="oracle", sample=sample),

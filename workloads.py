@@ -33,7 +33,7 @@ BLOCK = 4
 @dataclass(frozen=True)
 class Workload:
     name: str
-    kind: str                 # "prefill" or "decode"
+    kind: str                 # "prefill", "decode", or "draft" (IndexShare draft step after a decode capture)
     B: int
     T: int                    # prefill tokens, or decode cache length before the new token
     top_k: int
@@ -60,6 +60,9 @@ WORKLOADS = {
                                         128, "bf16", 1004, heavy_tail=True),
     "decode_b8_l1m_scale4": Workload("decode_b8_l1m_scale4", "decode", 8, 1048576, 512, 16, 2, 128,
                                      "bf16", 1005, pos_scale=4.0),
+    # IndexShare draft step: 3 positions drafted since the capture row (at most 4)
+    "draft_b64_l128k": Workload("draft_b64_l128k", "draft", 64, 131072, 512, 16, 2, 128, "bf16", 1006,
+                                extra={"drafted": 3, "max_draft": 4}),
 }
 
 
@@ -182,21 +185,23 @@ def make_decode(w: Workload, device="cuda", L: int | None = None, B: int | None 
                  q_idx [B][4][128], k_idx_new [B][128] raw indexer key of the
                  new token, q [B][Hq][d], k, v [B][Lmax+1][Hkv][d] caches that
                  already hold the new token at position L_i, seq_len [B]
-                 int32 = L_i + 1).
+                 int32 = L_i + 1).  Draft workloads ("drafted" in extra) get
+    extra[drafted] more cache rows: the positions drafted after the new token.
     """
-    assert w.kind == "decode"
+    assert w.kind in ("decode", "draft")
     L = L or w.T
     B = B or w.B
     g = _gen(device, w.seed)
     dt = torch_dtype(w)
     lens = [max(0, L - (i % 4 if ragged else 0)) for i in range(B)]
     Lmax = max(lens)
+    extra = int(w.extra.get("drafted", 0))   # draft workloads: cache rows for the drafted positions
     k_idx = _randn((B, Lmax, IDX_DIM), g, device, dt)
     q_idx = _randn((B, IDX_HEADS, IDX_DIM), g, device, dt)
     k_idx_new = _randn((B, IDX_DIM), g, device, dt)
     q = _randn((B, w.Hq, w.d), g, device, dt)
-    k = _randn((B, Lmax + 1, w.Hkv, w.d), g, device, dt)
-    v = _randn((B, Lmax + 1, w.Hkv, w.d), g, device, dt)
+    k = _randn((B, Lmax + 1 + extra, w.Hkv, w.d), g, device, dt)
+    v = _randn((B, Lmax + 1 + extra, w.Hkv, w.d), g, device, dt)
     seq_len = torch.tensor([x + 1 for x in lens], dtype=torch.int32, device=device)
     return dict(k_idx=k_idx, q_idx=q_idx, k_idx_new=k_idx_new, q=q, k=k, v=v, seq_len=seq_len,
                 lens=lens)
