@@ -359,6 +359,55 @@ class DraftRunner:
         return {k: self.x[k].cpu().pin_memory() for k in keys}
 
 
+class DenseRunner:
+    """Full causal decode attention over every cached position (the baseline
+    QSA replaces), on the same caches as the QSA decode workloads."""
+
+    def __init__(self, w, dev):
+        import block_sparse_attention_11_b200 as qsa
+        self.qsa = qsa
+        self.w = w
+        self.dev = dev
+        x = workloads.make_decode(w, device=dev)
+        del x["k_idx"]
+        torch.cuda.empty_cache()
+        self.x = x
+        self.out = torch.empty_like(x["q"])
+        self.ws = torch.empty(qsa.qsa_dense_attn_decode_workspace(w.B, w.Hq, w.d, x["k"].shape[1]),
+                              dtype=torch.uint8, device=dev)
+        self.flush_between_steps = False      # K/V caches of several GB
+        self.use_graph = True
+
+    def step(self, x=None, events=None):
+        x = x or self.x
+        if events is not None:
+            events[0].record()
+            events[1].record()
+            events[2].record()
+        self.qsa.qsa_dense_attn_decode(x["q"], x["k"], x["v"], x["seq_len"], self.out, workspace=self.ws)
+        if events is not None:
+            events[3].record()
+        return self.out
+
+    def launches_per_step(self):
+        return 2   # attention, combine
+
+    def units(self):
+        return self.w.B
+
+    def stage_names(self):
+        return ["no_pool", "no_index", "dense_attn"]
+
+    def algorithmic(self):
+        w = self.w
+        npos = w.T + 1
+        kv_bytes = npos * w.Hkv * w.d * 2 * 2 + 2 * w.Hq * w.d * 2
+        return dict(attn_bytes=kv_bytes * w.B, step_bytes=kv_bytes * w.B, positions=npos)
+
+    def host_inputs(self):
+        return {k: self.x[k].cpu().pin_memory() for k in ["q", "seq_len"]}
+
+
 # ----------------------------------------------------------------------------- measurement
 
 def flush_l2(buf):
@@ -383,7 +432,8 @@ def run_ours(args, rank, world):
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
     w = workloads.WORKLOADS[args.workload]
-    runner = {"prefill": PrefillRunner, "decode": DecodeRunner, "draft": DraftRunner}[w.kind](w, dev)
+    runner = {"prefill": PrefillRunner, "decode": DecodeRunner, "draft": DraftRunner,
+              "dense": DenseRunner}[w.kind](w, dev)
     flush = torch.zeros(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
     qsa = runner.qsa
     for _ in range(args.warmup):
@@ -517,19 +567,19 @@ def run_ours(args, rank, world):
         res["config"] = dict(workload=w.name, B=w.B, T=w.T, top_k=w.top_k, Hq=w.Hq, Hkv=w.Hkv, d=w.d,
                              needles=w.needles, l2="flushed between timed steps (256 MB write)",
                              parallelism=f"replicas x{world}")
-    elif w.kind == "draft":
-        res.update(metric="QSA IndexShare draft step us/step", unit="us/step", higher_is_better=False,
-                   value=ms_per_step * 1e3)
+    elif w.kind in ("draft", "dense"):
+        res.update(metric=metric_name(w), unit="us/step", higher_is_better=False, value=ms_per_step * 1e3)
         res["e2e"] = dict(value=e2e_ms * 1e3, unit="us/step", h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h,
                           graph=used_graph, eager_value=e2e_eager_ms * 1e3)
         achieved = alg["attn_bytes"] / (ms_per_step / 1e3) / 1e9
-        res["roofline"] = dict(kernel="sparse_attn_decode (frozen selection)", bound="hbm", achieved=achieved,
+        res["roofline"] = dict(kernel="sparse_attn_decode (frozen selection)" if w.kind == "draft"
+                               else "dense causal decode attention", bound="hbm", achieved=achieved,
                                peak=pk["hbm_gbs"], unit="GB/s", frac=achieved / pk["hbm_gbs"], traffic=None,
                                peak_kind=pk_kind,
                                note=f"algorithmic bytes = {alg['positions']} gathered positions per sequence x Hkv x "
                                     f"d x 2 B x 2 + q/out; time = the graph-replayed step (attention + combine)")
         res["config"] = dict(workload=w.name, B=w.B, L=w.T, top_k=w.top_k, Hq=w.Hq, Hkv=w.Hkv, d=w.d,
-                             drafted=w.extra["drafted"],
+                             drafted=w.extra.get("drafted", 0),
                              l2="inputs larger than L2 (K/V caches)", parallelism=f"replicas x{world}",
                              cuda_graph=True)
     else:
@@ -591,6 +641,19 @@ def run_oracle_sample(w, budget_s=15.0, seed=0):
         sample = (f"{done} uniformly drawn query rows of the {w.T}-token workload (full indexer scan, top-k, "
                   f"attention per row) + pooling of all keys; extrapolated per row to all rows")
         return value, sample, nthreads, "tokens/s"
+    if w.kind == "dense":   # textbook causal attention of one sequence's new token
+        x = workloads.make_decode(w, device="cpu", B=1)
+        q, k, v = x["q"].float().numpy(), x["k"][0].float().numpy(), x["v"][0].float().numpy()
+        t = int(x["seq_len"][0]) - 1
+        t0 = time.perf_counter()
+        reps = 0
+        while True:
+            oracle.dense_rows([0], q=q, k=k, v=v, Hq=w.Hq, Hkv=w.Hkv, d=w.d, q0=t, nthreads=nthreads)
+            reps += 1
+            if time.perf_counter() - t0 > min(budget_s, 5.0):
+                break
+        value = (time.perf_counter() - t0) / reps * w.B * 1e6
+        return value, f"{reps} steps of one {w.T}-token sequence, scaled to B={w.B}", nthreads, "us/step"
     # decode: a subset of sequences at full length
     x = workloads.make_decode(w, device="cpu", B=1)
     kr = x["k_idx"][0].float().numpy()
@@ -620,7 +683,7 @@ def run_oracle_sample(w, budget_s=15.0, seed=0):
 
 def metric_name(w):
     return {"prefill": "QSA prefill tokens/s", "decode": "QSA decode us/step",
-            "draft": "QSA IndexShare draft step us/step"}[w.kind]
+            "draft": "QSA IndexShare draft step us/step", "dense": "full causal decode attention us/step"}[w.kind]
 
 
 def main():

@@ -26,6 +26,7 @@ __all__ = [
     "qsa_index_topk_decode", "qsa_index_topk_decode_workspace",
     "qsa_sparse_attn_prefill", "qsa_sparse_attn_decode", "qsa_sparse_attn_decode_workspace",
     "qsa_sparse_attn_decode_noalloc", "qsa_sparse_attn_decode_shared", "qsa_sparse_attn_decode_shared_workspace",
+    "qsa_dense_attn_decode", "qsa_dense_attn_decode_workspace",
     "qsa_rope_apply", "qsa_check_status", "qsa_strerror", "qsa_version",
     "QSA_SCORE_RELU", "QSA_POOL_RMSNORM", "QSA_BF16", "QSA_FP32",
 ]
@@ -96,6 +97,9 @@ _sig("qsa_sparse_attn_decode", ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _i32,
 _sig("qsa_sparse_attn_decode_shared_workspace", _sz, _i32, _i32, _i32, _i32, _i32, _i32)
 _sig("qsa_sparse_attn_decode_shared", ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32,
      _i32, _i32, _f32, _vp, _vp, _vp, _sz, _i32, _vp)
+_sig("qsa_dense_attn_decode_workspace", _sz, _i32, _i32, _i32, _i64, _i32)
+_sig("qsa_dense_attn_decode", ctypes.c_int, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32, _f32, _vp, _vp, _vp, _sz,
+     _i32, _vp)
 _sig("qsa_rope_apply", ctypes.c_int, _vp, _i32, _i64, _i32, _i32, _i64, _Rope, _i32, _vp)
 _sig("qsa_sparse_attn_decode_noalloc", ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32,
      _i32, _f32, _vp, _vp, _i32, _vp)
@@ -273,6 +277,26 @@ def qsa_sparse_attn_decode_shared(q, k, v, seq_len, cap_len, sel, nsel, out, max
                                            max_draft, scale, _ptr(out, q.dtype, "out"),
                                            _ptr(lse, torch.float32, "lse"), wp, wb, dt, _stream(q, stream))
     _check(st, "qsa_sparse_attn_decode_shared")
+
+
+def qsa_dense_attn_decode_workspace(B, Hq, d, kv_stride, dtype=QSA_BF16) -> int:
+    return lib.qsa_dense_attn_decode_workspace(B, Hq, d, kv_stride, dtype)
+
+
+def qsa_dense_attn_decode(q, k, v, seq_len, out, scale=None, lse=None, workspace=None, stream=None):
+    """Full causal attention of the token at seq_len - 1 over positions 0..seq_len - 1
+    (the baseline QSA replaces).  q [B][Hq][d]; k, v [B][L][Hkv][d]."""
+    dt = _dtype_code(q)
+    B, Hq, d = q.shape
+    Hkv = k.shape[2]
+    scale = (1.0 / d ** 0.5) if scale is None else scale
+    need = qsa_dense_attn_decode_workspace(B, Hq, d, k.shape[1], dt)
+    wp, wb = _ws(need, q.device, workspace)
+    st = lib.qsa_dense_attn_decode(_ptr(q, None, "q"), _ptr(k, q.dtype, "k"), _ptr(v, q.dtype, "v"),
+                                   _ptr(seq_len, torch.int32, "seq_len"), B, k.shape[1], Hq, Hkv, d, scale,
+                                   _ptr(out, q.dtype, "out"), _ptr(lse, torch.float32, "lse"), wp, wb, dt,
+                                   _stream(q, stream))
+    _check(st, "qsa_dense_attn_decode")
 
 
 def qsa_sparse_attn_decode_noalloc(q, k, v, seq_len, sel, nsel, out, top_k=None, scale=None, lse=None, stream=None):

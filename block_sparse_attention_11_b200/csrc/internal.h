@@ -121,9 +121,11 @@ struct AttnArgs {
     bool decode;
     const int32_t *cap_len = nullptr;   // decode, IndexShare draft step: [B] capture rows + 1
     int max_draft = 0;                  // IndexShare: largest seq_len - cap_len
+    bool dense = false;                 // decode: dense causal attention over every position (no selection)
 };
 int attn_tail_blocks(bool indexshare, int max_draft);
 size_t attn_decode_ws_bytes(int B, int Hq, int d, int top_k, int tail_blocks = 1);
+size_t attn_dense_decode_ws_bytes(int B, int Hq, int d, int64_t kv_stride);
 cudaError_t launch_attn_bf16(const AttnArgs &a, void *ws, unsigned *status, cudaStream_t s);
 cudaError_t launch_attn_f32(const AttnArgs &a, unsigned *status, cudaStream_t s);
 

@@ -104,6 +104,7 @@ struct AttnParams {
     float *part_lse;       // decode: [B][splits][Hq] (log2 domain)
     const int32_t *cap_len;  // decode, IndexShare: [B] capture rows + 1 (null: plain decode)
     int max_draft;           // IndexShare: largest seq_len - cap_len
+    int dense;               // decode: every visible block in order (dense causal attention, no selection)
     unsigned *status;
 };
 
@@ -139,8 +140,8 @@ __device__ __forceinline__ Item get_item(const AttnParams &p, int64_t i) {
         it.seq = (int)(i / p.splits);
         it.row = i % p.splits;
         it.t = (int64_t)p.seq_len[it.seq] - 1;
-        it.sel = p.sel + (int64_t)it.seq * p.top_k;
-        it.nsel = p.nsel[it.seq];
+        it.sel = p.dense ? nullptr : p.sel + (int64_t)it.seq * p.top_k;
+        it.nsel = p.dense ? 0 : p.nsel[it.seq];
         it.qrow = p.q + (int64_t)it.seq * AttnCfg<HKV>::kHq * 128;
     }
     if (it.t < 0 || it.t >= p.kv_stride) {
@@ -157,7 +158,7 @@ __device__ __forceinline__ Item get_item(const AttnParams &p, int64_t i) {
     }
     it.nb = (t_sel + 1) / kBlock;
     it.tail = (int)(it.t + 1 - kBlock * it.nb);
-    it.nsel = max(0, min(it.nsel, p.top_k));
+    it.nsel = p.dense ? (int)it.nb : max(0, min(it.nsel, p.top_k));
     const int len = it.nsel + (it.tail + kBlock - 1) / kBlock;
     if (!p.decode) {
         it.lbeg = 0;
@@ -229,13 +230,14 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, AttnCfg<HKV>::kMinCtas
             const Item it = get_item<HKV>(p, i);
             const int id_end = min(it.lend, it.nsel);
             // list entries of this producer's slots: e - lbeg = 8 * st + PW * jj + pw
-            for (int r = lane; r * Cfg::kPw < id_end - it.lbeg; r += 32) {
+            // (dense: the ids are the entries themselves, nothing to stage)
+            for (int r = lane; !p.dense && r * Cfg::kPw < id_end - it.lbeg; r += 32) {
                 const int rel = (r / kSlotsPerPw) * AT_BPS + (r % kSlotsPerPw) * Cfg::kPw + pw;
                 if (rel < id_end - it.lbeg) ids[rel] = it.sel[it.lbeg + rel];
             }
             __syncwarp();
             const int nst = (it.lend - it.lbeg + AT_BPS - 1) / AT_BPS;
-            for (int st = lane; st < nst; st += 32) {
+            for (int st = lane; !p.dense && st < nst; st += 32) {
                 uint32_t info = 0, bytes = 0;
 #pragma unroll
                 for (int jj = 0; jj < kSlotsPerPw; ++jj) {
@@ -268,19 +270,37 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, AttnCfg<HKV>::kMinCtas
             const int64_t kv0 = (int64_t)it.seq * p.kv_stride;
             for (int st = 0; st < nst && ok; ++st, ++it_count) {
                 const int s = (int)(it_count % Cfg::kNS);
+                uint32_t sinfo, sbytes;
+                if (!p.dense) {
+                    sinfo = st_info[st];
+                    sbytes = st_bytes[st];
+                } else {   // every visible block, then the tail: counts straight from the entry index
+                    sinfo = 0;
+                    sbytes = 0;
+#pragma unroll
+                    for (int jj = 0; jj < kSlotsPerPw; ++jj) {
+                        const int j = Cfg::kPw * jj + pw;
+                        const int e = it.lbeg + AT_BPS * st + j;
+                        const int tokens = e >= it.lend ? 0
+                                           : (e < it.nsel ? kBlock : min(kBlock, it.tail - kBlock * (e - it.nsel)));
+                        sinfo |= (uint32_t)tokens << (3 * j);
+                        sbytes += (uint32_t)tokens * HKV * 256u;
+                    }
+                }
                 if (it_count >= Cfg::kNS) ok = mbar_wait(&sm.empty[s], (int)(((it_count / Cfg::kNS) + 1) & 1), p.status);
                 if (!ok) break;
                 if (lane == 0) {
-                    sm.info[s][pw] = st_info[st];
-                    mbar_arrive_expect_tx(&sm.full[s], 2 * st_bytes[st]);
+                    sm.info[s][pw] = sinfo;
+                    mbar_arrive_expect_tx(&sm.full[s], 2 * sbytes);
                 }
                 __syncwarp();
                 if (lane < kSlotsPerPw) {
                     const int j = Cfg::kPw * lane + pw;
                     const int e = it.lbeg + AT_BPS * st + j;
-                    const int tokens = (int)((st_info[st] >> (3 * j)) & 7u);
+                    const int tokens = (int)((sinfo >> (3 * j)) & 7u);
                     if (tokens > 0) {
-                        const int64_t blk = (e < it.nsel) ? (int64_t)ids[e - it.lbeg] : it.nb + (e - it.nsel);
+                        const int64_t blk = (e < it.nsel) ? (p.dense ? (int64_t)e : (int64_t)ids[e - it.lbeg])
+                                                          : it.nb + (e - it.nsel);
                         const int64_t off = (kv0 + blk * kBlock) * HKV * 128;
                         const uint32_t nbytes = (uint32_t)tokens * HKV * 256u;
                         bulk_g2s(sm.stage[s] + j * Cfg::kSlot, p.k + off, nbytes, &sm.full[s]);
@@ -605,7 +625,7 @@ __global__ void __launch_bounds__(256) attn_f32_kernel(const float *__restrict__
                                                         int64_t q0, int64_t kv_stride, int Hq, int Hkv, int top_k,
                                                         float scale, float *__restrict__ out, float *__restrict__ lse,
                                                         int decode, const int32_t *__restrict__ cap_len, int max_draft,
-                                                        unsigned *status) {
+                                                        int dense, unsigned *status) {
     const int64_t wid = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     const int64_t items = decode ? (int64_t)B : (int64_t)B * n_q;
@@ -631,8 +651,8 @@ __global__ void __launch_bounds__(256) attn_f32_kernel(const float *__restrict__
     }
     const int64_t nb = (t_sel + 1) / kBlock;
     const int tail = (int)(t + 1 - kBlock * nb);     // positions 4*nb .. t
-    const int32_t *sl = sel + qi * top_k;
-    const int nsel = max(0, min(nsel_p[qi], top_k));
+    const int32_t *sl = dense ? nullptr : sel + qi * top_k;
+    const int nsel = dense ? (int)nb : max(0, min(nsel_p[qi], top_k));
     const float4 qv = reinterpret_cast<const float4 *>(q + (qi * Hq + h) * 128)[lane];
     float m = -INFINITY, l = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -641,7 +661,7 @@ __global__ void __launch_bounds__(256) attn_f32_kernel(const float *__restrict__
         int64_t b;
         int ntok;
         if (e < nsel) {
-            b = sl[e];
+            b = dense ? e : sl[e];
             ntok = kBlock;
             if (b < 0 || b >= nb) {
                 if (lane == 0) flag(status, QSA_DEV_BAD_INDEX);
@@ -735,8 +755,10 @@ cudaError_t run_bf16(const AttnArgs &a, void *ws, unsigned *status, cudaStream_t
     p.status = status;
     p.cap_len = a.decode ? a.cap_len : nullptr;
     p.max_draft = a.max_draft;
-    // entries of one item's list: top_k blocks + the tail blocks
-    const int list_max = a.top_k + attn_tail_blocks(a.decode && a.cap_len, a.max_draft);
+    p.dense = a.decode && a.dense ? 1 : 0;
+    // entries of one item's list: top_k blocks + the tail blocks (dense: every block of the cache)
+    const int list_max = p.dense ? (int)(a.kv_stride / kBlock + 1)
+                                 : a.top_k + attn_tail_blocks(a.decode && a.cap_len, a.max_draft);
     if (a.decode) {
         const SplitPlan sp = decode_split_plan(a.B, list_max, (int64_t)sms * Cfg::kMinCtas);
         const int splits = sp.splits;
@@ -753,8 +775,8 @@ cudaError_t run_bf16(const AttnArgs &a, void *ws, unsigned *status, cudaStream_t
     }
     if (p.items <= 0) return cudaSuccess;
     // an item's list holds at most top_k ids plus the tail block
-    p.sel_cap = (a.top_k + 3) & ~3;
-    p.nst_cap = (list_max + AT_BPS - 1) / AT_BPS;
+    p.sel_cap = p.dense ? 4 : (a.top_k + 3) & ~3;                  // dense: no id list, no stage tables
+    p.nst_cap = p.dense ? 1 : (list_max + AT_BPS - 1) / AT_BPS;
     const size_t smem = attn_smem_bytes<HKV>(p.sel_cap, p.nst_cap);
     if (di && smem > di->smem_optin) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(attn_bf16_kernel<HKV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -783,6 +805,16 @@ size_t attn_decode_ws_bytes(int B, int Hq, int d, int top_k, int tail_blocks) {
     return (n * d * sizeof(float) + n * sizeof(float) + 255) / 256 * 256;
 }
 
+size_t attn_dense_decode_ws_bytes(int B, int Hq, int d, int64_t kv_stride) {
+    const DeviceInfo *di = device_info();
+    const int sms = di ? di->sm_count : 148;
+    const int list_max = (int)(kv_stride / kBlock + 1);
+    const int splits =
+        std::max(decode_split_plan(B, list_max, sms).splits, decode_split_plan(B, list_max, 2 * sms).splits);
+    size_t n = (size_t)B * splits * Hq;
+    return (n * d * sizeof(float) + n * sizeof(float) + 255) / 256 * 256;
+}
+
 cudaError_t launch_attn_bf16(const AttnArgs &a, void *ws, unsigned *status, cudaStream_t s) {
     switch (a.Hkv) {
     case 1: return run_bf16<1>(a, ws, status, s);
@@ -799,7 +831,7 @@ cudaError_t launch_attn_f32(const AttnArgs &a, unsigned *status, cudaStream_t s)
     attn_f32_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, s>>>(
         (const float *)a.q, (const float *)a.k, (const float *)a.v, a.sel, a.nsel, a.seq_len, a.B, a.n_q, a.q0,
         a.kv_stride, a.Hq, a.Hkv, a.top_k, a.scale, (float *)a.out, a.lse, a.decode ? 1 : 0,
-        a.decode ? a.cap_len : nullptr, a.max_draft, status);
+        a.decode ? a.cap_len : nullptr, a.max_draft, a.decode && a.dense ? 1 : 0, status);
     return cudaGetLastError();
 }
 

@@ -352,6 +352,33 @@ int qsa_sparse_attn_decode_shared(const void *q, const void *k, const void *v, c
     return cuda_status(launch_attn_f32(a, di->status, s));
 }
 
+size_t qsa_dense_attn_decode_workspace(int32_t B, int32_t Hq, int32_t d, int64_t kv_stride, int32_t dtype) {
+    if (B < 1 || Hq < 1 || d < 1 || kv_stride < 1 || kv_stride > ((int64_t)1 << 30)) return 0;
+    if (dtype != QSA_BF16) return 0;
+    return attn_dense_decode_ws_bytes(B, Hq, d, kv_stride);
+}
+
+int qsa_dense_attn_decode(const void *q, const void *k, const void *v, const int32_t *seq_len, int32_t B,
+                          int64_t kv_stride, int32_t Hq, int32_t Hkv, int32_t d, float scale, void *out, float *lse,
+                          void *workspace, size_t ws_bytes, int32_t dtype, void *stream) {
+    // the shape rules of the sparse kernels, with a dummy (unused) selection
+    const int32_t dummy = 0;
+    int st = attn_common_checks(q, k, v, &dummy, &dummy, B, Hq, Hkv, d, 1, scale, out, dtype);
+    if (st != QSA_OK) return st;
+    if (!seq_len || kv_stride < 1 || kv_stride > ((int64_t)1 << 30)) return QSA_ERR_INVALID_ARG;
+    const DeviceInfo *di = nullptr;
+    if ((st = check_device(&di)) != QSA_OK) return st;
+    AttnArgs a{q, k, v, nullptr, nullptr, seq_len, B, 1, 0, kv_stride, Hq, Hkv, d, 1, scale, out, lse, true};
+    a.dense = true;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dtype == QSA_BF16) {
+        const size_t need = attn_dense_decode_ws_bytes(B, Hq, d, kv_stride);
+        if (!workspace || ws_bytes < need) return QSA_ERR_WORKSPACE;
+        return cuda_status(launch_attn_bf16(a, workspace, di->status, s));
+    }
+    return cuda_status(launch_attn_f32(a, di->status, s));
+}
+
 int qsa_rope_apply(void *x, int32_t B, int64_t n, int32_t H, int32_t d, int64_t pos0, qsa_rope_t rope, int32_t dtype,
                    void *stream) {
     if (!x || B < 1 || n < 0 || H < 1 || d < 2 || (d % 2) != 0 || pos0 < 0) return QSA_ERR_INVALID_ARG;

@@ -293,6 +293,24 @@ QSA_API int qsa_sparse_attn_decode_shared(const void *q, const void *k, const vo
                                           void *workspace, size_t ws_bytes, int32_t dtype, void *stream);
 
 /* ========================================================================= */
+/* Dense causal decode attention (the full-attention baseline)                */
+/* ========================================================================= */
+/*
+ * Not a step of QSA: the full attention QSA replaces.  Pages "Qwen3.8-Flash-
+ * Next, Layer by Layer" (section "Token mixing") and the aicontrolled journal
+ * (section "Where the measurement ends") compare the QSA attention module with
+ * full attention at 1M tokens; this is the full attention, on the same
+ * kernels, so that ratio can be measured on one GPU.  The query of sequence i
+ * at t = seq_len[i] - 1 attends over every position 0..t.  Arguments as
+ * qsa_sparse_attn_decode without a selection; 1 <= seq_len[i] <= kv_stride.
+ * workspace at least qsa_dense_attn_decode_workspace() bytes.
+ */
+QSA_API size_t qsa_dense_attn_decode_workspace(int32_t B, int32_t Hq, int32_t d, int64_t kv_stride, int32_t dtype);
+QSA_API int qsa_dense_attn_decode(const void *q, const void *k, const void *v, const int32_t *seq_len, int32_t B,
+                                  int64_t kv_stride, int32_t Hq, int32_t Hkv, int32_t d, float scale, void *out,
+                                  float *lse, void *workspace, size_t ws_bytes, int32_t dtype, void *stream);
+
+/* ========================================================================= */
 /* Decode sparse attention without a workspace (allocation-free callers)      */
 /* ========================================================================= */
 /*

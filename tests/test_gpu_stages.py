@@ -378,3 +378,27 @@ def test_indexshare_flags_out_of_range_capture(qsa):
         with pytest.raises(qsa.QSAError):
             qsa.qsa_check_status()
         qsa.qsa_check_status()        # cleared
+
+
+# ----------------------------------------------------------------------------- dense decode baseline
+
+@pytest.mark.parametrize("dtype,Hq,Hkv,B,L", [("bf16", 16, 2, 4, 20001), ("bf16", 8, 1, 3, 3), ("fp32", 8, 1, 3, 7000),
+                                             ("bf16", 32, 4, 2, 9000)])
+def test_dense_decode_matches_textbook_attention(qsa, dtype, Hq, Hkv, B, L):
+    """Full causal decode attention (the baseline QSA replaces) against the
+    oracle's textbook causal attention, ragged lengths."""
+    d = 128
+    dt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    g = torch.Generator().manual_seed(L)
+    k = torch.randn(B, L + 4, Hkv, d, generator=g).to(dt)
+    v = torch.randn(B, L + 4, Hkv, d, generator=g).to(dt)
+    q = torch.randn(B, Hq, d, generator=g).to(dt)
+    lens = [max(1, L - i) for i in range(B)]
+    out = torch.empty(B, Hq, d, dtype=dt, device=DEV)
+    qsa.qsa_dense_attn_decode(q.to(DEV), k.to(DEV), v.to(DEV), torch.tensor(lens, dtype=torch.int32, device=DEV), out)
+    qsa.qsa_check_status()
+    for b in range(B):
+        t = lens[b] - 1
+        ref = oracle.dense_rows([0], q=np32(q[b])[None], k=np32(k[b]), v=np32(v[b]), Hq=Hq, Hkv=Hkv, d=d, q0=t)
+        err = np.abs(np32(out[b]) - ref[0]).max()
+        assert err <= TOL[dtype], (b, err)

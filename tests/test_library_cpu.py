@@ -82,6 +82,11 @@ def test_invalid_arguments_are_rejected_before_launch(qsa):
                                              0.1, fake, None, fake, 1 << 20, 0, None) == qsa.QSA_ERR_INVALID_ARG
     assert lib.qsa_sparse_attn_decode_shared_workspace(4, 16, 128, 512, -1, 0) == 0
     assert lib.qsa_sparse_attn_decode_shared_workspace(4, 16, 128, 512, 8, 1) == 0     # fp32 needs none
+    # dense decode baseline: a cache length is required
+    assert lib.qsa_dense_attn_decode(fake, fake, fake, fake, 1, 0, 16, 2, 128, 0.1, fake, None, fake, 1 << 20, 0,
+                                     None) == qsa.QSA_ERR_INVALID_ARG
+    assert lib.qsa_dense_attn_decode(fake, fake, fake, None, 1, 64, 16, 2, 128, 0.1, fake, None, fake, 1 << 20, 0,
+                                     None) == qsa.QSA_ERR_INVALID_ARG
     # misaligned pointer
     odd = ctypes.c_void_p(4098)
     assert lib.qsa_pool_keys_prefill(odd, fake, 1, 16, 0, 16, 4, rope, 0, 0, None) == qsa.QSA_ERR_INVALID_ARG

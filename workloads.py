@@ -33,7 +33,8 @@ BLOCK = 4
 @dataclass(frozen=True)
 class Workload:
     name: str
-    kind: str                 # "prefill", "decode", or "draft" (IndexShare draft step after a decode capture)
+    kind: str                 # "prefill", "decode", "draft" (IndexShare draft step after a decode capture)
+                              # or "dense" (full causal decode attention, the baseline QSA replaces)
     B: int
     T: int                    # prefill tokens, or decode cache length before the new token
     top_k: int
@@ -60,6 +61,10 @@ WORKLOADS = {
                                         128, "bf16", 1004, heavy_tail=True),
     "decode_b8_l1m_scale4": Workload("decode_b8_l1m_scale4", "decode", 8, 1048576, 512, 16, 2, 128,
                                      "bf16", 1005, pos_scale=4.0),
+    # full causal decode attention on the same caches as the QSA decode workloads
+    "dense_b64_l128k": Workload("dense_b64_l128k", "dense", 64, 131072, 512, 16, 2, 128, "bf16", 1003),
+    "dense_b8_l1m_scale4": Workload("dense_b8_l1m_scale4", "dense", 8, 1048576, 512, 16, 2, 128, "bf16", 1005,
+                                    pos_scale=4.0),
     # IndexShare draft step: 3 positions drafted since the capture row (at most 4)
     "draft_b64_l128k": Workload("draft_b64_l128k", "draft", 64, 131072, 512, 16, 2, 128, "bf16", 1006,
                                 extra={"drafted": 3, "max_draft": 4}),
@@ -188,7 +193,7 @@ def make_decode(w: Workload, device="cuda", L: int | None = None, B: int | None 
                  int32 = L_i + 1).  Draft workloads ("drafted" in extra) get
     extra[drafted] more cache rows: the positions drafted after the new token.
     """
-    assert w.kind in ("decode", "draft")
+    assert w.kind in ("decode", "draft", "dense")
     L = L or w.T
     B = B or w.B
     g = _gen(device, w.seed)
