@@ -51,6 +51,8 @@ def _L():
         _lib = ctypes.CDLL(build())
         _lib.oracle_round_bf16.restype = ctypes.c_double
         _lib.oracle_round_bf16.argtypes = [ctypes.c_double]
+        _lib.oracle_round_e4m3.restype = ctypes.c_double
+        _lib.oracle_round_e4m3.argtypes = [ctypes.c_double]
         _lib.oracle_topk.restype = ctypes.c_int
     return _lib
 
@@ -86,22 +88,33 @@ def rope_rows(x, pos, base=10000.0, pos_scale=1.0, rotary_dim=128):
     return out
 
 
+def _store_code(store_bf16, store_fp8):
+    return 2 if store_fp8 else int(bool(store_bf16))
+
+
+def round_e4m3(x):
+    """Elementwise round-to-nearest-even to FP8 E4M3 (saturating at +-448), from float64."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    f = _L().oracle_round_e4m3
+    return np.vectorize(lambda v: f(ctypes.c_double(v)))(x)
+
+
 def pool_keys(k_raw, pos0=0, base=10000.0, pos_scale=1.0, rotary_dim=128,
-              rmsnorm=False, store_bf16=True):
+              rmsnorm=False, store_bf16=True, store_fp8=False):
     """Compressed keys [n/4][128] from raw indexer keys [n][128] (first token
-    at position pos0, a multiple of 4)."""
+    at position pos0, a multiple of 4); stored as BF16, FP32 or FP8 E4M3 values."""
     k_raw = _f32(k_raw)
     n = k_raw.shape[0]
     out = np.empty((n // BLOCK, IDX_DIM), np.float32)
     _L().oracle_pool_keys(_p(k_raw), ctypes.c_int64(n), ctypes.c_int64(pos0),
                           ctypes.c_double(base), ctypes.c_double(pos_scale),
                           ctypes.c_int(rotary_dim), ctypes.c_int(int(rmsnorm)),
-                          ctypes.c_int(int(store_bf16)), _p(out))
+                          ctypes.c_int(_store_code(store_bf16, store_fp8)), _p(out))
     return out
 
 
 def pool_decode(k_new, ring, k_pool, seq_len, base=10000.0, pos_scale=1.0,
-                rotary_dim=128, rmsnorm=False, store_bf16=True):
+                rotary_dim=128, rmsnorm=False, store_bf16=True, store_fp8=False):
     """One decode pooling step for one sequence; updates ring [4][128] and
     k_pool [cap][128] (float32 arrays) in place."""
     assert ring.dtype == np.float32 and ring.flags.c_contiguous
@@ -110,7 +123,7 @@ def pool_decode(k_new, ring, k_pool, seq_len, base=10000.0, pos_scale=1.0,
     _L().oracle_pool_decode(_p(k_new), _p(ring), _p(k_pool), ctypes.c_int64(int(seq_len)),
                             ctypes.c_double(base), ctypes.c_double(pos_scale),
                             ctypes.c_int(rotary_dim), ctypes.c_int(int(rmsnorm)),
-                            ctypes.c_int(int(store_bf16)))
+                            ctypes.c_int(_store_code(store_bf16, store_fp8)))
 
 
 def topk(scores, k):

@@ -86,8 +86,29 @@ double oracle_round_bf16(double x)
     return y;
 }
 
+/* Round a double to the nearest FP8 E4M3 value (ties to even), directly from
+ * the double, saturating to +-448.  E4M3 (the FP8 format of the pages' FP8
+ * indexer-key cache, "--attention-config.indexer_kv_dtype fp8"): 1 sign bit,
+ * 4 exponent bits with bias 7, 3 mantissa bits; normal values 2^-6 .. 448,
+ * subnormals k * 2^-9; no infinities. */
+double oracle_round_e4m3(double x)
+{
+    if (x == 0.0 || isnan(x)) return x;
+    if (isinf(x)) return copysign(448.0, x);
+    int e;
+    frexp(x, &e);               /* x = m * 2^e, 0.5 <= |m| < 1 */
+    int ex = e - 1;             /* x = 1.f * 2^ex */
+    if (ex < -6) ex = -6;       /* subnormal range: fixed quantum 2^-9 */
+    double quantum = ldexp(1.0, ex - 3);
+    double y = nearbyint(x / quantum) * quantum;   /* ties to even */
+    if (fabs(y) > 448.0) y = copysign(448.0, x);
+    return y;
+}
+
+/* store: 0 = FP32, 1 = BF16, 2 = FP8 E4M3 */
 static double round_store(double x, int store_bf16)
 {
+    if (store_bf16 == 2) return oracle_round_e4m3(x);
     return store_bf16 ? oracle_round_bf16(x) : (double)(float)x;
 }
 
@@ -209,7 +230,7 @@ static void rotate_query(const float *q_raw, double t, const orope_t *r, int sto
         double x[IDX_DIM];
         for (int i = 0; i < IDX_DIM; ++i) x[i] = q_raw[h * IDX_DIM + i];
         rope_rotate(x, t, r);
-        for (int i = 0; i < IDX_DIM; ++i) q_hat[h * IDX_DIM + i] = round_store(x[i], store_bf16);
+        for (int i = 0; i < IDX_DIM; ++i) q_hat[h * IDX_DIM + i] = round_store(x[i], store_bf16 ? 1 : 0);
     }
 }
 

@@ -475,3 +475,65 @@ def test_indexshare_keeps_the_frozen_selection_and_sees_drafted_positions():
     cap = oracle.decode(q_idx[t_c][None], kp[None], [t_c + 1], top_k=k)
     np.testing.assert_array_equal(res["sel"], cap["sel"])          # frozen, not re-selected
     assert res["out"][0, 0, 3] > 0.99                                # the drafted key wins
+
+
+# ----------------------------------------------------------------------------- FP8 E4M3 storage
+
+def _e4m3_codes():
+    """Every finite E4M3 value, from the bit layout (1 sign, 4 exponent bits with
+    bias 7, 3 mantissa bits; exponent 15 with mantissa 7 is NaN)."""
+    vals = []
+    for e in range(16):
+        for m in range(8):
+            if e == 15 and m == 7:
+                continue
+            v = (m / 8.0) * 2.0 ** -6 if e == 0 else (1 + m / 8.0) * 2.0 ** (e - 7)
+            vals.append(v)
+    pos = sorted(set(vals))
+    return np.array(sorted(set([-v for v in pos] + pos)))
+
+
+def test_e4m3_code_points_round_trip_and_max():
+    codes = _e4m3_codes()
+    assert codes.max() == 448.0 and len(codes) == 253      # 126 positive, 126 negative, zero
+    np.testing.assert_array_equal(oracle.round_e4m3(codes), codes)
+
+
+def test_e4m3_ties_to_even_and_nearest():
+    pos = _e4m3_codes()
+    pos = pos[pos >= 0]
+    lo, hi = pos[:-1], pos[1:]
+    mid = (lo + hi) / 2
+    # the code of a value is even iff its mantissa's last bit is 0; consecutive
+    # codes alternate, starting with 0 (even)
+    even_lo = (np.arange(len(lo)) % 2) == 0
+    exp_tie = np.where(even_lo, lo, hi)
+    np.testing.assert_array_equal(oracle.round_e4m3(mid), exp_tie)
+    np.testing.assert_array_equal(oracle.round_e4m3(-mid), -exp_tie)
+    eps = (hi - lo) * 1e-3
+    np.testing.assert_array_equal(oracle.round_e4m3(mid - eps), lo)
+    np.testing.assert_array_equal(oracle.round_e4m3(mid + eps), hi)
+
+
+def test_e4m3_saturates_and_matches_torch_in_range():
+    np.testing.assert_array_equal(oracle.round_e4m3([448.0, 460.0, 464.0, 500.0, 1e9, np.inf, -np.inf]),
+                                  [448.0, 448.0, 448.0, 448.0, 448.0, 448.0, -448.0])
+    rng = np.random.default_rng(2)
+    x = (rng.standard_normal(20000) * np.exp(rng.uniform(-8, 5, 20000))).astype(np.float32)
+    x = x[np.abs(x) < 440]
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).float().numpy()
+    np.testing.assert_array_equal(oracle.round_e4m3(x.astype(np.float64)), ref)
+
+
+def test_pooled_keys_in_fp8_are_the_rounded_bf16_free_values():
+    # FP8 storage rounds the same fp64 rotated mean that BF16 storage rounds:
+    # pooled FP32 keys (no storage rounding) rounded to E4M3 equal the FP8 path.
+    rng = np.random.default_rng(4)
+    k_raw = bf16(rng.standard_normal((4 * 300, 128)))
+    exact = oracle.pool_keys(k_raw, store_bf16=False)       # fp32 store of the fp64 value
+    fp8 = oracle.pool_keys(k_raw, store_fp8=True)
+    codes = set(_e4m3_codes().tolist())
+    assert set(np.unique(fp8).tolist()) <= codes
+    # fp32 storage is within half an fp32 ulp of the fp64 value, so re-rounding
+    # it to E4M3 differs only where it straddles an E4M3 midpoint: never here
+    np.testing.assert_array_equal(oracle.round_e4m3(exact.astype(np.float64)), fp8)
