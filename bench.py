@@ -44,9 +44,10 @@ L2_BYTES = 126 * 1024 * 1024
 PROFILES = os.path.join(ROOT, "profiles")
 CSRC = os.path.join(ROOT, "block_sparse_attention_11_b200", "csrc")
 # ncu summary holding the DRAM traffic of each roofline kernel, and the sources it was built from
+_DECODE_SRC = ["k_decode_index.cu", "select.cuh", "common.cuh", "internal.h"]
 TRAFFIC_PROFILE = {
-    "prefill": ("attn_bf16_prefill_t32k.md", ["k_attn.cu", "common.cuh", "internal.h"]),
-    "decode": ("decode_indexer_b64_l128k.md", ["k_decode_index.cu", "select.cuh", "common.cuh", "internal.h"]),
+    "prefill": [("attn_bf16_prefill_t32k.md", ["k_attn.cu", "common.cuh", "internal.h"])],
+    "decode": [("decode_indexer_b64_l128k.md", _DECODE_SRC), ("decode_indexer_b64_l128k_fp8keys.md", _DECODE_SRC)],
 }
 
 
@@ -63,23 +64,26 @@ def profiled_traffic(kind, workload):
     """DRAM bytes per launch from the committed ncu summary, or None when the
     summary is missing, covers another workload, or the kernel sources changed
     since it was captured."""
-    name, files = TRAFFIC_PROFILE[kind]
-    try:
-        with open(os.path.join(PROFILES, name)) as f:
-            txt = f.read()
-    except OSError:
-        return None
-    fields = {}
-    for line in txt.splitlines():
-        if line.startswith("- ") and ": " in line:
-            k, v = line[2:].split(": ", 1)
-            fields[k.strip().strip("`")] = v.strip().strip("`")
-    try:
-        if fields.get("workload") != workload or fields.get("source_sha256") != source_digest(files):
+    for name, files in TRAFFIC_PROFILE[kind]:
+        try:
+            with open(os.path.join(PROFILES, name)) as f:
+                txt = f.read()
+        except OSError:
+            continue
+        fields = {}
+        for line in txt.splitlines():
+            if line.startswith("- ") and ": " in line:
+                k, v = line[2:].split(": ", 1)
+                fields[k.strip().strip("`")] = v.strip().strip("`")
+        if fields.get("workload") != workload:
+            continue
+        try:
+            if fields.get("source_sha256") != source_digest(files):
+                return None
+            return float(fields["traffic_bytes_per_launch"])
+        except (KeyError, ValueError, OSError):
             return None
-        return float(fields["traffic_bytes_per_launch"])
-    except (KeyError, ValueError, OSError):
-        return None
+    return None
 
 
 def peaks():
@@ -227,8 +231,12 @@ class DecodeRunner:
         B, L = w.B, w.T
         self.rope = qsa.Rope(base=w.rope_base, pos_scale=w.pos_scale, rotary_dim=128)
         self.cap = L // 4 + 1
-        self.k_pool = torch.zeros(B, self.cap, 128, dtype=dt, device=dev)
-        qsa.qsa_pool_keys_prefill(x["k_idx"], self.k_pool, rope=self.rope)      # the cache's compressed keys
+        # compressed keys in the computation type, or FP8 E4M3 ("keys": "fp8")
+        self.fp8 = w.extra.get("keys") == "fp8"
+        self.kflags = qsa.QSA_KEYS_FP8 if self.fp8 else 0
+        self.k_pool = torch.zeros(B, self.cap, 128, dtype=torch.float8_e4m3fn if self.fp8 else dt, device=dev)
+        qsa.qsa_pool_keys_prefill(x["k_idx"], self.k_pool, rope=self.rope,      # the cache's compressed keys
+                                  flags=self.kflags)
         self.ring = torch.zeros(B, 4, 128, dtype=dt, device=dev)
         del x["k_idx"]
         torch.cuda.empty_cache()
@@ -236,8 +244,8 @@ class DecodeRunner:
         self.nsel = torch.empty(B, dtype=torch.int32, device=dev)
         self.out = torch.empty_like(x["q"])
         self.max_blocks = (L + 1) // 4
-        self.ws_i = torch.empty(qsa.qsa_index_topk_decode_workspace(B, self.max_blocks, w.top_k), dtype=torch.uint8,
-                                device=dev)
+        self.ws_i = torch.empty(qsa.qsa_index_topk_decode_workspace(B, self.max_blocks, w.top_k, self.kflags),
+                                dtype=torch.uint8, device=dev)
         self.ws_a = torch.empty(qsa.qsa_sparse_attn_decode_workspace(B, w.Hq, w.d, w.top_k), dtype=torch.uint8,
                                 device=dev)
         # a decode step streams the whole compressed-key cache and gathers from
@@ -251,11 +259,13 @@ class DecodeRunner:
         x = x or self.x
         if events is not None:
             events[0].record()
-        qsa.qsa_pool_keys_decode(x["k_idx_new"], self.ring, self.k_pool, x["seq_len"], rope=self.rope)
+        qsa.qsa_pool_keys_decode(x["k_idx_new"], self.ring, self.k_pool, x["seq_len"], rope=self.rope,
+                                 flags=self.kflags)
         if events is not None:
             events[1].record()
         qsa.qsa_index_topk_decode(x["q_idx"], self.k_pool, x["seq_len"], self.sel, self.nsel,
-                                  max_blocks=self.max_blocks, top_k=w.top_k, rope=self.rope, workspace=self.ws_i)
+                                  max_blocks=self.max_blocks, top_k=w.top_k, rope=self.rope, flags=self.kflags,
+                                  workspace=self.ws_i)
         if events is not None:
             events[2].record()
         qsa.qsa_sparse_attn_decode(x["q"], x["k"], x["v"], x["seq_len"], self.sel, self.nsel, self.out,
@@ -278,7 +288,8 @@ class DecodeRunner:
         nb = (w.T + 1) // 4
         tail = (w.T + 1) - 4 * nb
         npos = min(nb, w.top_k) * 4 + tail
-        idx_bytes = nb * 128 * 2 + 4 * 128 * 2                        # compressed keys + indexer query
+        kbytes = 1 if w.extra.get("keys") == "fp8" else 2
+        idx_bytes = nb * 128 * kbytes + 4 * 128 * 2                   # compressed keys + indexer query
         kv_bytes = npos * w.Hkv * w.d * 2 * 2 + 2 * w.Hq * w.d * 2     # gathered K/V + q + out
         return dict(idx_bytes=idx_bytes * w.B, attn_bytes=kv_bytes * w.B, step_bytes=(idx_bytes + kv_bytes) * w.B)
 
@@ -657,7 +668,8 @@ def run_oracle_sample(w, budget_s=15.0, seed=0):
     # decode: a subset of sequences at full length
     x = workloads.make_decode(w, device="cpu", B=1)
     kr = x["k_idx"][0].float().numpy()
-    kp = oracle.pool_keys(kr, base=w.rope_base, pos_scale=w.pos_scale, store_bf16=True)
+    kp = oracle.pool_keys(kr, base=w.rope_base, pos_scale=w.pos_scale, store_bf16=True,
+                          store_fp8=w.extra.get("keys") == "fp8")
     q, k, v = x["q"].float().numpy(), x["k"].float().numpy(), x["v"].float().numpy()
     seq_len = x["seq_len"].numpy()
     cap_len = None

@@ -35,7 +35,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libqsa.so")
 
 QSA_OK, QSA_ERR_INVALID_ARG, QSA_ERR_UNSUPPORTED, QSA_ERR_CUDA, QSA_ERR_DEVICE, QSA_ERR_WORKSPACE = range(6)
 QSA_BF16, QSA_FP32 = 0, 1
-QSA_SCORE_RELU, QSA_POOL_RMSNORM = 1, 2
+QSA_SCORE_RELU, QSA_POOL_RMSNORM, QSA_KEYS_FP8 = 1, 2, 4
 
 
 class QSAError(RuntimeError):
@@ -137,6 +137,16 @@ def _ptr(t, dtype=None, name="tensor"):
     return t.data_ptr()
 
 
+def _kpool_ptr(k_pool, dtype, flags):
+    """Compressed-key cache pointer: `dtype` (the computation type), or one
+    byte per value (float8_e4m3fn or uint8) under QSA_KEYS_FP8."""
+    if flags & QSA_KEYS_FP8:
+        if not isinstance(k_pool, torch.Tensor) or k_pool.dtype not in (torch.float8_e4m3fn, torch.uint8):
+            raise TypeError("k_pool must be float8_e4m3fn (or uint8) with QSA_KEYS_FP8")
+        return _ptr(k_pool, None, "k_pool")
+    return _ptr(k_pool, dtype, "k_pool")
+
+
 def _stream(t: torch.Tensor, stream=None):
     if stream is None:
         stream = torch.cuda.current_stream(t.device)
@@ -166,7 +176,7 @@ def qsa_pool_keys_prefill(k_raw, k_pool, pos0=0, rope=Rope(), flags=0, n_tok=Non
     B, S, D = k_raw.shape
     assert D == 128 and k_pool.dim() == 3 and k_pool.shape[0] == B and k_pool.shape[2] == 128
     n_tok = S if n_tok is None else n_tok
-    st = lib.qsa_pool_keys_prefill(_ptr(k_raw, None, "k_raw"), _ptr(k_pool, k_raw.dtype, "k_pool"), B, n_tok, pos0, S,
+    st = lib.qsa_pool_keys_prefill(_ptr(k_raw, None, "k_raw"), _kpool_ptr(k_pool, k_raw.dtype, flags), B, n_tok, pos0, S,
                                    k_pool.shape[1], rope.c(), flags, dt, _stream(k_raw, stream))
     _check(st, "qsa_pool_keys_prefill")
 
@@ -175,7 +185,7 @@ def qsa_pool_keys_decode(k_new, ring, k_pool, seq_len, rope=Rope(), flags=0, str
     dt = _dtype_code(k_new)
     B = k_new.shape[0]
     st = lib.qsa_pool_keys_decode(_ptr(k_new, None, "k_new"), _ptr(ring, k_new.dtype, "ring"),
-                                  _ptr(k_pool, k_new.dtype, "k_pool"), _ptr(seq_len, torch.int32, "seq_len"), B,
+                                  _kpool_ptr(k_pool, k_new.dtype, flags), _ptr(seq_len, torch.int32, "seq_len"), B,
                                   k_pool.shape[1], rope.c(), flags, dt, _stream(k_new, stream))
     _check(st, "qsa_pool_keys_decode")
 
@@ -210,7 +220,7 @@ def qsa_index_topk_decode(q_idx, k_pool, seq_len, sel, nsel, max_blocks=None, to
     max_blocks = k_pool.shape[1] if max_blocks is None else max_blocks
     need = qsa_index_topk_decode_workspace(B, max_blocks, top_k, flags, dt)
     wp, wb = _ws(need, q_idx.device, workspace)
-    st = lib.qsa_index_topk_decode(_ptr(q_idx, None, "q_idx"), _ptr(k_pool, q_idx.dtype, "k_pool"),
+    st = lib.qsa_index_topk_decode(_ptr(q_idx, None, "q_idx"), _kpool_ptr(k_pool, q_idx.dtype, flags),
                                    _ptr(head_w, torch.float32, "head_w"), _ptr(seq_len, torch.int32, "seq_len"), B,
                                    k_pool.shape[1], max_blocks, top_k, _ptr(sel, torch.int32, "sel"),
                                    _ptr(nsel, torch.int32, "nsel"), wp, wb, rope.c(), flags, dt,

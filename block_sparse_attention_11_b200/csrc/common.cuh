@@ -52,6 +52,42 @@ __device__ __forceinline__ __nv_bfloat16 d2bf(double x) {
     return __float2bfloat16_rn(f);
 }
 
+// double -> FP8 E4M3 (round to nearest even, saturating at +-448), packed two
+// per 16 bits (first value in the low byte): round to odd into float (no
+// double rounding), then the float -> e4m3x2 conversion.
+__device__ __forceinline__ float d2f_odd(double x) {
+    float f = __double2float_rz(x);
+    if ((double)f != x && !isinf(f)) f = __uint_as_float(__float_as_uint(f) | 1u);
+    return f;
+}
+__device__ __forceinline__ uint16_t d2e4m3x2(double first, double second) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(d2f_odd(second)), "f"(d2f_odd(first)));
+    return r;
+}
+// Four FP8 E4M3 values (value i in byte i) -> two f16x2 words, exactly
+// (E4M3 is a subset of FP16): lo = values 0, 1 and hi = values 2, 3, the
+// first of each pair in the low half.
+__device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t w, uint32_t &lo, uint32_t &hi) {
+    asm("{\n\t.reg .b16 a, b;\n\t"
+        "mov.b32 {a, b}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, a;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(w));
+}
+// FP32 <-> FP16 bits, round to nearest even (FP16 to FP32 is exact).
+__device__ __forceinline__ uint16_t f2h_bits(float x) {
+    uint16_t r;
+    asm("cvt.rn.f16.f32 %0, %1;" : "=h"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ float h_bits2f(uint16_t h) {
+    float r;
+    asm("cvt.f32.f16 %0, %1;" : "=f"(r) : "h"(h));
+    return r;
+}
+
 template <typename T> __device__ __forceinline__ T from_double(double x);
 template <> __device__ __forceinline__ __nv_bfloat16 from_double<__nv_bfloat16>(double x) { return d2bf(x); }
 template <> __device__ __forceinline__ float from_double<float>(double x) { return (float)x; }
@@ -296,6 +332,15 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
                                          uint32_t b0, uint32_t b1) {
     asm volatile(
         "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// D (16x8 f32) += A (16x16 f16, row) * B (16x8 f16, col)
+__device__ __forceinline__ void mma16816_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                             uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
         "{%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));

@@ -60,11 +60,12 @@ struct DeviceInfo {
 const DeviceInfo *device_info();
 
 // ---- pooling / rotation (k_rope.cu)
+// fp8: the compressed keys are stored as FP8 E4M3 (bf16 raw keys only).
 cudaError_t launch_pool_prefill(const void *k_raw, void *k_pool, int B, int64_t nblk, int64_t pos0,
                                 int64_t raw_stride, int64_t pool_stride, Rope rope, bool rmsnorm, bool bf16,
-                                cudaStream_t s);
+                                bool fp8, cudaStream_t s);
 cudaError_t launch_pool_decode(const void *k_new, void *ring, void *k_pool, const int32_t *seq_len, int B,
-                               int64_t pool_stride, Rope rope, bool rmsnorm, bool bf16, unsigned *status,
+                               int64_t pool_stride, Rope rope, bool rmsnorm, bool bf16, bool fp8, unsigned *status,
                                cudaStream_t s);
 cudaError_t launch_rope_apply(void *x, int B, int64_t n, int H, int d, int64_t pos0, Rope rope, bool bf16,
                               cudaStream_t s);
@@ -105,7 +106,7 @@ size_t decode_index_ws_bytes(int B, int64_t max_blocks, int top_k, bool bf16);
 cudaError_t launch_decode_index(const void *q_idx, const void *k_pool, const float *head_w,
                                 const int32_t *seq_len, int B, int64_t pool_stride, int64_t max_blocks,
                                 int top_k, int32_t *sel, int32_t *nsel, void *ws, Rope rope, bool relu,
-                                bool bf16, unsigned *status, cudaStream_t s);
+                                bool bf16, bool fp8, unsigned *status, cudaStream_t s);
 
 // ---- sparse attention (k_attn.cu)
 struct AttnArgs {

@@ -194,12 +194,18 @@ __global__ void __launch_bounds__(DI_THREADS, 2)
 // (hi and lo planes of the FP32 head sum, or the 4 heads), FP32 accumulate.
 constexpr int DM_ROWS = 128;                       // keys per stage
 constexpr int DM_NS = 3;                           // stages in flight per CTA (2 CTAs per SM)
+constexpr int DM_NS_FP8 = 6;                       // FP8 stages are half the bytes
 constexpr int DM_STAGE_BYTES = DM_ROWS * 256;      // two 64-dim k-atoms of 128 rows x 128 B
+// FP8 E4M3 compressed keys: a stage is one 128-byte-swizzled box of 128 rows x
+// 128 B, the A operand of m16n8k32 E4M3 MMAs as it lands.
+constexpr int DM_STAGE_BYTES_FP8 = DM_ROWS * 128;
+template <bool FP8> __host__ __device__ constexpr int stage_bytes() { return FP8 ? DM_STAGE_BYTES_FP8 : DM_STAGE_BYTES; }
 
 using EncodeTiledFn = decltype(&cuTensorMapEncodeTiled);
 
-// 2-D bf16 map over the compressed keys [rows][128]: 64 x 128 boxes, 128-byte swizzle.
-bool make_kpool_map(CUtensorMap *map, const void *base, uint64_t rows) {
+// 2-D map over the compressed keys [rows][128]: bf16 in 64 x 128 boxes, or
+// FP8 E4M3 (as bytes) in 128 x 128 boxes; 128-byte swizzle.
+bool make_kpool_map(CUtensorMap *map, const void *base, uint64_t rows, bool fp8 = false) {
     static EncodeTiledFn fn = nullptr;
     if (!fn) {
         void *ptr = nullptr;
@@ -210,37 +216,52 @@ bool make_kpool_map(CUtensorMap *map, const void *base, uint64_t rows) {
         fn = reinterpret_cast<EncodeTiledFn>(ptr);
     }
     cuuint64_t dims[2] = {128, rows};
-    cuuint64_t strides[1] = {128 * 2};
-    cuuint32_t box[2] = {64, (cuuint32_t)DM_ROWS};
+    cuuint64_t strides[1] = {fp8 ? 128u : 128u * 2};
+    cuuint32_t box[2] = {fp8 ? 128u : 64u, (cuuint32_t)DM_ROWS};
     cuuint32_t estr[2] = {1, 1};
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+    return fn(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base),
+              dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // Streams the n compressed keys of rows y0.. through NS stages, scores them
 // against the rotated query and hands each (row, key) to sink; every key's
-// top 11 bits are counted in sm.lh.  Returns false after a timed-out wait,
-// once the copies still in flight have landed (or their waits ran out too).
-template <int NS, typename Smem, typename Sink>
+// top 11 bits are counted in sm.lh.  NT threads form NT / 256 groups of 8
+// warps; group g consumes (and refills) the stages st = g mod NT / 256, each
+// warp scoring 16 rows of a 128-row stage.  Returns false after a timed-out
+// wait, once the copies still in flight have landed (or their waits ran out).
+template <int NS, bool FP8, int NT, typename Smem, typename Sink>
 __device__ __forceinline__ bool stream_scores(Smem &sm, const CUtensorMap *kmap,
                                               const __nv_bfloat16 *__restrict__ q_idx, const Rope &rope,
                                               const DecodeParams &p, int seq, int64_t s_len, int n, int y0,
                                               Sink &&sink) {
+    constexpr int G = NT / 256;
+    static_assert(NT % 256 == 0 && NS % G == 0, "whole groups; each slot stays with one group");
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int grp = warp >> 3, gw = warp & 7;            // stage group, warp within the group
+    const bool leader = (tid & 255) == 0;
     const int nstages = (n + DM_ROWS - 1) / DM_ROWS;
-    if (tid == 0) {
-        for (int st = 0; st < min(NS, nstages); ++st) {
-            mbar_arrive_expect_tx(&sm.full[st], DM_STAGE_BYTES);
-            tma_load_2d(sm.stage[st], kmap, 0, y0 + st * DM_ROWS, &sm.full[st]);
-            tma_load_2d(sm.stage[st] + DM_STAGE_BYTES / 2, kmap, 64, y0 + st * DM_ROWS, &sm.full[st]);
-        }
-    }
+    constexpr int SB = stage_bytes<FP8>();
+    auto issue = [&](int slot, int st2) {
+        mbar_arrive_expect_tx(&sm.full[slot], SB);
+        tma_load_2d(sm.stage[slot], kmap, 0, y0 + st2 * DM_ROWS, &sm.full[slot]);
+        if constexpr (!FP8) tma_load_2d(sm.stage[slot] + SB / 2, kmap, 64, y0 + st2 * DM_ROWS, &sm.full[slot]);
+    };
+    if (tid == 0)
+        for (int st = 0; st < min(NS, nstages); ++st) issue(st, st);
     const bool per_head = p.relu || p.head_w;
-    // rotated query heads of the new token (position s_len - 1), rounded to bf16;
-    // columns: hi/lo of the FP32 head sum, or the 4 heads
+    // Rotated query heads of the new token (position s_len - 1), rounded to
+    // bf16, as the B operand's columns.  BF16 keys: hi/lo bf16 planes of the
+    // FP32 head sum, or the 4 heads.  FP8 keys (scored as FP16, which holds
+    // every E4M3 value): the same values times 2^qexp, which puts the largest
+    // magnitude in [2^14, 2^15), as FP16 -- three pieces that add up to the
+    // scaled head sum, or one per head (exact for any bf16 value above 2^-31 of
+    // the largest); the scores are scaled back by 2^-qexp.
+    const int e = tid;
+    float rv[kIdxHeads], hs = 0.0f;
     if (tid < kIdxDim) {
-        const int e = tid, R = rope.rotary_dim, half = R >> 1;
+        const int R = rope.rotary_dim, half = R >> 1;
         const __nv_bfloat16 *src = q_idx + (int64_t)seq * kIdxHeads * kIdxDim;
         double cs = 1.0, sn = 0.0;
         int pr = e;
@@ -250,7 +271,7 @@ __device__ __forceinline__ bool stream_scores(Smem &sm, const CUtensorMap *kmap,
                                          rope_inv_freq(rope, e < half ? e : e - half));
             sincos(ang, &sn, &cs);
         }
-        float hs = 0.0f;
+#pragma unroll
         for (int h = 0; h < kIdxHeads; ++h) {
             const double xe = __bfloat162float(src[h * kIdxDim + e]);
             double o = xe;
@@ -259,60 +280,120 @@ __device__ __forceinline__ bool stream_scores(Smem &sm, const CUtensorMap *kmap,
                 o = (e < half) ? __dsub_rn(__dmul_rn(xe, cs), __dmul_rn(xp, sn))
                                : __dadd_rn(__dmul_rn(xe, cs), __dmul_rn(xp, sn));
             }
-            const __nv_bfloat16 r = d2bf(o);
-            if (per_head) sm.qcol[h][e] = r;
-            hs = (h == 0) ? __bfloat162float(r) : __fadd_rn(hs, __bfloat162float(r));
+            rv[h] = __bfloat162float(d2bf(o));
+            hs = (h == 0) ? rv[0] : __fadd_rn(hs, rv[h]);
         }
-        const __nv_bfloat16 zero = __float2bfloat16_rn(0.f);
-        if (!per_head) {
-            const __nv_bfloat16 hi = __float2bfloat16_rn(hs);
-            sm.qcol[0][e] = hi;
-            sm.qcol[1][e] = __float2bfloat16_rn(__fsub_rn(hs, __bfloat162float(hi)));
-            for (int col = 2; col < 8; ++col) sm.qcol[col][e] = zero;
+        if constexpr (!FP8) {
+            const __nv_bfloat16 zero = __float2bfloat16_rn(0.f);
+            if (!per_head) {
+                const __nv_bfloat16 hi = __float2bfloat16_rn(hs);
+                sm.qcol[0][e] = hi;
+                sm.qcol[1][e] = __float2bfloat16_rn(__fsub_rn(hs, __bfloat162float(hi)));
+                for (int col = 2; col < 8; ++col) sm.qcol[col][e] = zero;
+            } else {
+                for (int h = 0; h < kIdxHeads; ++h) sm.qcol[h][e] = __float2bfloat16_rn(rv[h]);
+                for (int col = 4; col < 8; ++col) sm.qcol[col][e] = zero;
+            }
         } else {
-            for (int col = 4; col < 8; ++col) sm.qcol[col][e] = zero;
+            float m = per_head ? fmaxf(fmaxf(fabsf(rv[0]), fabsf(rv[1])), fmaxf(fabsf(rv[2]), fabsf(rv[3])))
+                               : fabsf(hs);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            if (lane == 0) sm.qred[warp] = m;
         }
     }
     if (tid < kIdxHeads) sm.w[tid] = p.head_w ? p.head_w[(int64_t)seq * kIdxHeads + tid] : 1.f;
+    float qinv = 1.0f;   // FP8: 2^-qexp
+    if constexpr (FP8) {
+        __syncthreads();
+        const float m = fmaxf(fmaxf(sm.qred[0], sm.qred[1]), fmaxf(sm.qred[2], sm.qred[3]));
+        int qexp = 0;
+        if (m > 0.0f && m <= 3.0e38f) {
+            int ex;
+            frexpf(m, &ex);                       // m in [2^(ex-1), 2^ex)
+            qexp = min(max(15 - ex, -100), 100);
+        }
+        qinv = ldexpf(1.0f, -qexp);
+        if (tid < kIdxDim) {
+            const float sc = ldexpf(1.0f, qexp);
+            uint16_t(*q16)[kIdxDim] = reinterpret_cast<uint16_t(*)[kIdxDim]>(&sm.qcol[0][0]);
+            if (!per_head) {
+                float x = __fmul_rn(hs, sc);
+#pragma unroll
+                for (int j = 0; j < 3; ++j) {
+                    const uint16_t b = f2h_bits(x);
+                    q16[j][e] = b;
+                    x = __fsub_rn(x, h_bits2f(b));
+                }
+                for (int col = 3; col < 8; ++col) q16[col][e] = 0;
+            } else {
+#pragma unroll
+                for (int h = 0; h < kIdxHeads; ++h) q16[h][e] = f2h_bits(__fmul_rn(rv[h], sc));
+                for (int col = 4; col < 8; ++col) q16[col][e] = 0;
+            }
+        }
+    }
     __syncthreads();
     const int gr = lane >> 2, tq = lane & 3;
+    // B fragments.  BF16: k-step kk covers dims 16kk .. 16kk + 15.  FP8: the
+    // E4M3 A fragment of a 32-dim block j (4 bytes of dims 32j + 4tq + {0..3}
+    // per register, as ldmatrix gives them) widens into two FP16 k16 steps
+    // whose k order is a permutation of the block's dims: step 2j takes dims
+    // 32j + 4tq + {0..3}, step 2j + 1 dims 32j + 16 + 4tq + {0..3}; the query
+    // fragments follow the same order.
     uint32_t qf[8][2];
     {
         const uint32_t *qw = reinterpret_cast<const uint32_t *>(&sm.qcol[gr][0]);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-            qf[kk][0] = qw[(16 * kk + 2 * tq) >> 1];
-            qf[kk][1] = qw[(16 * kk + 8 + 2 * tq) >> 1];
+            const int d0 = FP8 ? 32 * (kk >> 1) + 16 * (kk & 1) + 4 * tq : 16 * kk + 2 * tq;
+            const int d1 = FP8 ? d0 + 2 : d0 + 8;
+            qf[kk][0] = qw[d0 >> 1];
+            qf[kk][1] = qw[d1 >> 1];
         }
     }
     const float w0 = sm.w[2 * (tq & 1)], w1 = sm.w[2 * (tq & 1) + 1];
     const int mi = lane >> 3, rr = lane & 7;
-    const int trow = 16 * warp + rr + 8 * (mi & 1);      // row of this lane's ldmatrix address in the stage
+    const int trow = 16 * gw + rr + 8 * (mi & 1);        // row of this lane's ldmatrix address in the stage
     const uint32_t row_off = (uint32_t)trow * 128u;
     const uint32_t sw = (uint32_t)(trow & 7);
+    constexpr uint32_t kAtom = DM_STAGE_BYTES / 2;
     bool ok = true;
-    int issued = min(NS, nstages);   // stages whose copies were issued (thread 0's count)
-    int st = 0;
-    for (; st < nstages; ++st) {
+    int issued = min(NS, nstages);   // the group's stages below this were issued (leader's count)
+    int st = grp;
+    for (; st < nstages; st += G) {
         const int slot = st % NS;
         ok = mbar_wait(&sm.full[slot], (st / NS) & 1, p.status);
         if (!ok) break;
         const uint32_t base = smem_u32(sm.stage[slot]);
         float acc[4] = {0.f, 0.f, 0.f, 0.f}, acc2[4] = {0.f, 0.f, 0.f, 0.f};
+        if constexpr (FP8) {
 #pragma unroll
-        for (int kk = 0; kk < 8; kk += 2) {
-            uint32_t a[4], b[4];
-            {
-                const uint32_t chunk = (uint32_t)(2 * (kk & 3) + (mi >> 1));
-                ldsm_x4(base + (kk >> 2) * (DM_STAGE_BYTES / 2) + row_off + ((chunk ^ sw) << 4), a[0], a[1], a[2], a[3]);
+            for (int j = 0; j < 4; ++j) {
+                uint32_t r[4], lo[4], hi[4];
+                const uint32_t chunk = (uint32_t)(2 * j + (mi >> 1));
+                ldsm_x4(base + row_off + ((chunk ^ sw) << 4), r[0], r[1], r[2], r[3]);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) e4m3x4_to_f16x4(r[i], lo[i], hi[i]);
+                mma16816_f16(acc, lo[0], lo[1], hi[0], hi[1], qf[2 * j][0], qf[2 * j][1]);
+                mma16816_f16(acc2, lo[2], lo[3], hi[2], hi[3], qf[2 * j + 1][0], qf[2 * j + 1][1]);
             }
-            {
-                const uint32_t chunk = (uint32_t)(2 * ((kk + 1) & 3) + (mi >> 1));
-                ldsm_x4(base + ((kk + 1) >> 2) * (DM_STAGE_BYTES / 2) + row_off + ((chunk ^ sw) << 4), b[0], b[1], b[2],
-                        b[3]);
+        } else {
+#pragma unroll
+            for (int kk = 0; kk < 8; kk += 2) {
+                uint32_t a[4], b[4];
+                {
+                    const uint32_t chunk = (uint32_t)(2 * (kk & 3) + (mi >> 1));
+                    ldsm_x4(base + (kk >> 2) * kAtom + row_off + ((chunk ^ sw) << 4), a[0], a[1], a[2], a[3]);
+                }
+                {
+                    const uint32_t chunk = (uint32_t)(2 * ((kk + 1) & 3) + (mi >> 1));
+                    ldsm_x4(base + ((kk + 1) >> 2) * kAtom + row_off + ((chunk ^ sw) << 4), b[0], b[1], b[2],
+                            b[3]);
+                }
+                mma16816(acc, a[0], a[1], a[2], a[3], qf[kk][0], qf[kk][1]);
+                mma16816(acc2, b[0], b[1], b[2], b[3], qf[kk + 1][0], qf[kk + 1][1]);
             }
-            mma16816(acc, a[0], a[1], a[2], a[3], qf[kk][0], qf[kk][1]);
-            mma16816(acc2, b[0], b[1], b[2], b[3], qf[kk + 1][0], qf[kk + 1][1]);
         }
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[i] += acc2[i];
@@ -322,6 +403,10 @@ __device__ __forceinline__ bool stream_scores(Smem &sm, const CUtensorMap *kmap,
         if (!per_head) {
             s0 = acc[0] + acc[1];
             s1 = acc[2] + acc[3];
+            if constexpr (FP8) {   // the third piece is column 2, in lane tq = 1
+                s0 += __shfl_xor_sync(0xffffffffu, s0, 1);
+                s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
+            }
         } else {
             float a0 = acc[0], a1 = acc[1], a2 = acc[2], a3 = acc[3];
             if (p.relu) { a0 = fmaxf(a0, 0.f); a1 = fmaxf(a1, 0.f); a2 = fmaxf(a2, 0.f); a3 = fmaxf(a3, 0.f); }
@@ -330,7 +415,11 @@ __device__ __forceinline__ bool stream_scores(Smem &sm, const CUtensorMap *kmap,
             s0 += __shfl_xor_sync(0xffffffffu, s0, 1);
             s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
         }
-        const int r0 = st * DM_ROWS + 16 * warp + gr;
+        if constexpr (FP8) {
+            s0 = __fmul_rn(s0, qinv);
+            s1 = __fmul_rn(s1, qinv);
+        }
+        const int r0 = st * DM_ROWS + 16 * gw + gr;
         if (tq == 0) {
             if (r0 < n) {
                 const uint32_t key = score_key(s0);
@@ -343,41 +432,42 @@ __device__ __forceinline__ bool stream_scores(Smem &sm, const CUtensorMap *kmap,
                 atomicAdd(&sm.lh[key >> 21], 1u);
             }
         }
-        if (tid == 0 && st + NS < nstages) {
+        if (leader && st + NS < nstages) {
             ok = mbar_wait(&sm.empty[slot], (st / NS) & 1, p.status);
             if (ok) {
-                const int st2 = st + NS;
-                mbar_arrive_expect_tx(&sm.full[slot], DM_STAGE_BYTES);
-                tma_load_2d(sm.stage[slot], kmap, 0, y0 + st2 * DM_ROWS, &sm.full[slot]);
-                tma_load_2d(sm.stage[slot] + DM_STAGE_BYTES / 2, kmap, 64, y0 + st2 * DM_ROWS, &sm.full[slot]);
-                issued = st2 + 1;
+                issue(slot, st + NS);
+                issued = st + NS + 1;
             }
         }
     }
     ok = __syncthreads_and(ok);
-    if (!ok && tid == 0) {
+    if (!ok && leader) {
         // let the copies still in flight land before the shared memory is reused
-        for (int s2 = st; s2 < issued; ++s2) mbar_wait(&sm.full[s2 % NS], (s2 / NS) & 1, p.status);
+        for (int s2 = st; s2 < issued; s2 += G) mbar_wait(&sm.full[s2 % NS], (s2 / NS) & 1, p.status);
     }
     return ok;
 }
 
+template <bool FP8>
 struct DecodeMmaSmem {
-    alignas(1024) uint8_t stage[DM_NS][DM_STAGE_BYTES];
-    alignas(16) __nv_bfloat16 qcol[8][kIdxDim];   // B operand source: 8 columns x 128 dims
+    static constexpr int NS = FP8 ? DM_NS_FP8 : DM_NS;
+    alignas(1024) uint8_t stage[NS][stage_bytes<FP8>()];
+    alignas(16) __nv_bfloat16 qcol[8][kIdxDim];   // B operand source: 8 columns x 128 dims (FP8: as FP16)
     float w[kIdxHeads];
-    uint64_t full[DM_NS], empty[DM_NS];
+    float qred[4];                                 // FP8: per-warp largest query magnitude
+    uint64_t full[NS], empty[NS];
     uint32_t lh[2048];                             // local histogram of the keys' top 11 bits
 };
 
 // Scorer of the two-kernel path: keys to the workspace, histogram added into
 // the sequence's global histogram.
+template <bool FP8>
 __global__ void __launch_bounds__(DI_THREADS, 2)
     decode_score_mma_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16 *__restrict__ q_idx,
                             Rope rope, DecodeParams p) {
     extern __shared__ uint8_t dsm_raw[];
-    DecodeMmaSmem &sm = *reinterpret_cast<DecodeMmaSmem *>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) &
-                                                           ~uintptr_t(1023));
+    DecodeMmaSmem<FP8> &sm = *reinterpret_cast<DecodeMmaSmem<FP8> *>(
+        (reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
     pdl_trigger();
     const int seq = blockIdx.y, c = blockIdx.x;
     const int tid = threadIdx.x;
@@ -394,12 +484,16 @@ __global__ void __launch_bounds__(DI_THREADS, 2)
     uint32_t *gkeys = p.keys + (int64_t)seq * p.kstride + c0;
     for (int b = tid; b < 2048; b += blockDim.x) sm.lh[b] = 0;
     if (tid == 0) {
-        for (int s = 0; s < DM_NS; ++s) { mbar_init(&sm.full[s], 1); mbar_init(&sm.empty[s], DI_THREADS / 32); }
+        for (int s = 0; s < DecodeMmaSmem<FP8>::NS; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], 8);   // the warps of the stage's group
+        }
         fence_mbar_init();
         prefetch_tmap(&kmap);
     }
     __syncthreads();
-    const bool ok = stream_scores<DM_NS>(sm, &kmap, q_idx, rope, p, seq, s_len, n, (int)(seq * p.pool_stride + c0),
+    const bool ok = stream_scores<DecodeMmaSmem<FP8>::NS, FP8, DI_THREADS>(sm, &kmap, q_idx, rope, p, seq, s_len, n,
+                                              (int)(seq * p.pool_stride + c0),
                                          [&](int r, uint32_t key) { gkeys[r] = key; });
     if (!ok) return;
     flush_hist(sm.lh, p.hist + (int64_t)seq * 2048);
@@ -732,43 +826,52 @@ __global__ void __launch_bounds__(DS_THREADS)
 // ---------------------------------------------------------------------------
 // Fused decode indexer (bf16): scorer and selection in one cluster kernel.
 // One cluster of up to 16 CTAs per sequence, one CTA per SM; each CTA streams
-// its chunk of compressed keys (4 stages in flight) and keeps the chunk's score
+// its chunk of compressed keys (4 stages in flight, two groups of 8 warps
+// taking alternate stages) and keeps the chunk's score
 // keys in shared memory.  The CTAs' histograms are summed through distributed
 // shared memory (CTA r sums a slice of bins over the cluster and writes the
 // sums into every CTA), then the selection above runs on the resident keys.
 // ---------------------------------------------------------------------------
 constexpr int DF_NS = 4;              // stages in flight per CTA
+constexpr int DF_NS_FP8 = 8;          // FP8 stages are half the bytes
+template <bool FP8> __host__ __device__ constexpr int fused_stages() { return FP8 ? DF_NS_FP8 : DF_NS; }
 constexpr int DF_KEYS = 16384;        // keys a CTA keeps in shared memory
-constexpr int DF_THREADS = DI_THREADS;
+constexpr int DF_THREADS = 512;      // two stage groups of 8 warps
 
+template <bool FP8>
 struct FusedSmem {
     union {
-        uint8_t stage[DF_NS][DM_STAGE_BYTES];   // while streaming
+        struct {
+            uint8_t stage[fused_stages<FP8>()][stage_bytes<FP8>()];     // while streaming
+        } st;
         DsSmem ds;                              // selection, once every stage has been consumed
     } u;
     uint32_t skeys[DF_KEYS];
     uint32_t lh[2048];
     alignas(16) __nv_bfloat16 qcol[8][kIdxDim];
     float w[kIdxHeads];
-    uint64_t full[DF_NS], empty[DF_NS];
+    float qred[4];
+    uint64_t full[fused_stages<FP8>()], empty[fused_stages<FP8>()];
 };
-static_assert(sizeof(DsSmem) <= (size_t)DF_NS * DM_STAGE_BYTES, "selection state fits the stage buffers");
-
-// The streaming interface of FusedSmem (stage, qcol, w, full, empty, lh).
+// The streaming interface of FusedSmem (stage, qcol, w, qred, full, empty, lh).
+template <bool FP8>
 struct FusedStream {
-    uint8_t (&stage)[DF_NS][DM_STAGE_BYTES];
+    uint8_t (&stage)[fused_stages<FP8>()][stage_bytes<FP8>()];
     __nv_bfloat16 (&qcol)[8][kIdxDim];
     float (&w)[kIdxHeads];
-    uint64_t (&full)[DF_NS];
-    uint64_t (&empty)[DF_NS];
+    float (&qred)[4];
+    uint64_t (&full)[fused_stages<FP8>()];
+    uint64_t (&empty)[fused_stages<FP8>()];
     uint32_t (&lh)[2048];
 };
 
+template <bool FP8>
 __global__ void __launch_bounds__(DF_THREADS, 1)
     decode_index_fused_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16 *__restrict__ q_idx,
                               Rope rope, DecodeParams p, SelectArgs a) {
     extern __shared__ uint8_t dsm_raw[];
-    FusedSmem &sm = *reinterpret_cast<FusedSmem *>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
+    FusedSmem<FP8> &sm = *reinterpret_cast<FusedSmem<FP8> *>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) &
+                                                             ~uintptr_t(1023));
     pdl_wait();      // the compressed keys come from the previous kernel (ring pooling)
     pdl_trigger();
     const int seq = blockIdx.y, tid = threadIdx.x;
@@ -790,15 +893,18 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
     uint2 *cand_seq = a.cand + (int64_t)seq * a.kstride;
     for (int b = tid; b < 2048; b += DF_THREADS) sm.lh[b] = 0;
     if (tid == 0) {
-        for (int s = 0; s < DF_NS; ++s) { mbar_init(&sm.full[s], 1); mbar_init(&sm.empty[s], DF_THREADS / 32); }
+        for (int s = 0; s < fused_stages<FP8>(); ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], 8);   // the warps of the stage's group
+        }
         fence_mbar_init();
         prefetch_tmap(&kmap);
     }
     __syncthreads();
     bool ok = true;
     if (n > 0) {
-        FusedStream fs{sm.u.stage, sm.qcol, sm.w, sm.full, sm.empty, sm.lh};
-        ok = stream_scores<DF_NS>(fs, &kmap, q_idx, rope, p, seq, s_len, n, (int)(seq * p.pool_stride + c0),
+        FusedStream<FP8> fs{sm.u.st.stage, sm.qcol, sm.w, sm.qred, sm.full, sm.empty, sm.lh};
+        ok = stream_scores<fused_stages<FP8>(), FP8, DF_THREADS>(fs, &kmap, q_idx, rope, p, seq, s_len, n, (int)(seq * p.pool_stride + c0),
                                   [&](int r, uint32_t key) { sm.skeys[r] = key; });
     }
     (void)ok;   // a timed-out wait is in the status word; the cluster still runs every barrier
@@ -917,6 +1023,7 @@ struct FusedPlan {
 };
 
 // Clusters of C fused CTAs that can be resident at once (queried once per C).
+template <bool FP8>
 int fused_active_clusters(int C) {
     static int ok[DS_CLUSTER + 1];
     static bool init = false;
@@ -927,10 +1034,10 @@ int fused_active_clusters(int C) {
     if (C < 1 || C > DS_CLUSTER) return 0;
     if (ok[C] < 0) {
         ok[C] = 0;
-        const size_t smem = sizeof(FusedSmem) + 1024;
-        if (cudaFuncSetAttribute(decode_index_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) ==
-                cudaSuccess &&
-            (C <= 8 || cudaFuncSetAttribute(decode_index_fused_kernel,
+        const size_t smem = sizeof(FusedSmem<FP8>) + 1024;
+        if (cudaFuncSetAttribute(decode_index_fused_kernel<FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem) == cudaSuccess &&
+            (C <= 8 || cudaFuncSetAttribute(decode_index_fused_kernel<FP8>,
                                             cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess)) {
             cudaLaunchConfig_t cfg = {};
             cfg.gridDim = dim3((unsigned)C, 1, 1);
@@ -944,14 +1051,15 @@ int fused_active_clusters(int C) {
             cfg.attrs = attr;
             cfg.numAttrs = 1;
             int n = 0;
-            if (cudaOccupancyMaxActiveClusters(&n, decode_index_fused_kernel, &cfg) == cudaSuccess && n > 0) ok[C] = n;
+            if (cudaOccupancyMaxActiveClusters(&n, decode_index_fused_kernel<FP8>, &cfg) == cudaSuccess && n > 0)
+                ok[C] = n;
         }
         cudaGetLastError();   // a refused query leaves no sticky error
     }
     return ok[C];
 }
 
-FusedPlan fused_plan(int B, int64_t max_blocks, bool bf16) {
+FusedPlan fused_plan(int B, int64_t max_blocks, bool bf16, bool fp8) {
     FusedPlan f{false, 1, DF_KEYS};
     const DeviceInfo *di = device_info();
     const int64_t sms = di ? di->sm_count : 148;
@@ -966,7 +1074,8 @@ FusedPlan fused_plan(int B, int64_t max_blocks, bool bf16) {
     f.chunk = chunk;
     // one wave of clusters: a sequence whose cluster waited for a free GPC
     // would stream after the others with a fraction of the bandwidth
-    f.use = (int64_t)B * C >= sms / 2 && fused_active_clusters((int)C) >= B;
+    f.use = (int64_t)B * C >= sms / 2 &&
+            (fp8 ? fused_active_clusters<true>((int)C) : fused_active_clusters<false>((int)C)) >= B;
     return f;
 }
 
@@ -1005,27 +1114,28 @@ size_t decode_index_ws_bytes(int B, int64_t max_blocks, int top_k, bool bf16) {
 cudaError_t launch_decode_index(const void *q_idx, const void *k_pool, const float *head_w,
                                 const int32_t *seq_len, int B, int64_t pool_stride, int64_t max_blocks,
                                 int top_k, int32_t *sel, int32_t *nsel, void *ws, Rope rope, bool relu,
-                                bool bf16, unsigned *status, cudaStream_t s) {
+                                bool bf16, bool fp8, unsigned *status, cudaStream_t s) {
+    if (fp8 && !bf16) return cudaErrorInvalidValue;
     const int64_t kstride = key_stride(max_blocks);
     const DecodeWs d = decode_ws(ws, B, max_blocks, top_k);
-    const FusedPlan fp = fused_plan(B, max_blocks, bf16);
+    const FusedPlan fp = fused_plan(B, max_blocks, bf16, fp8);
     if (fp.use) {
         CUtensorMap kmap;
-        if (!make_kpool_map(&kmap, k_pool, (uint64_t)B * pool_stride)) return cudaErrorInvalidValue;
+        if (!make_kpool_map(&kmap, k_pool, (uint64_t)B * pool_stride, fp8)) return cudaErrorInvalidValue;
         DecodeParams p{seq_len, head_w, pool_stride, max_blocks, fp.chunk, kstride, fp.C, top_k, relu ? 1 : 0,
                        d.keys, d.hist, status};
         SelectArgs sa{seq_len, pool_stride, max_blocks, kstride, fp.chunk, fp.C, top_k, d.keys, d.hist, d.cand,
                       sel, nsel};
-        const size_t smem = sizeof(FusedSmem) + 1024;
-        cudaError_t e =
-            cudaFuncSetAttribute(decode_index_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        auto kern = fp8 ? decode_index_fused_kernel<true> : decode_index_fused_kernel<false>;
+        const size_t smem = (fp8 ? sizeof(FusedSmem<true>) : sizeof(FusedSmem<false>)) + 1024;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         if (fp.C > 8) {
-            e = cudaFuncSetAttribute(decode_index_fused_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
             if (e != cudaSuccess) return e;
         }
-        return launch_pdl_cluster(decode_index_fused_kernel, dim3((unsigned)fp.C, (unsigned)B), dim3(DF_THREADS), smem,
-                                  (unsigned)fp.C, s, kmap, (const __nv_bfloat16 *)q_idx, rope, p, sa);
+        return launch_pdl_cluster(kern, dim3((unsigned)fp.C, (unsigned)B), dim3(DF_THREADS), smem, (unsigned)fp.C, s,
+                                  kmap, (const __nv_bfloat16 *)q_idx, rope, p, sa);
     }
     const DecodePlan pl = decode_index_plan(B, max_blocks, bf16);
     cudaError_t e = cudaMemsetAsync(d.hist, 0, d.zero_bytes, s);
@@ -1035,11 +1145,12 @@ cudaError_t launch_decode_index(const void *q_idx, const void *k_pool, const flo
     dim3 grid((unsigned)pl.chunks, (unsigned)B);
     if (bf16) {
         CUtensorMap kmap;
-        if (!make_kpool_map(&kmap, k_pool, (uint64_t)B * pool_stride)) return cudaErrorInvalidValue;
-        const size_t smem = sizeof(DecodeMmaSmem) + 1024;
-        e = cudaFuncSetAttribute(decode_score_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (!make_kpool_map(&kmap, k_pool, (uint64_t)B * pool_stride, fp8)) return cudaErrorInvalidValue;
+        auto kern = fp8 ? decode_score_mma_kernel<true> : decode_score_mma_kernel<false>;
+        const size_t smem = (fp8 ? sizeof(DecodeMmaSmem<true>) : sizeof(DecodeMmaSmem<false>)) + 1024;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        decode_score_mma_kernel<<<grid, DI_THREADS, smem, s>>>(kmap, (const __nv_bfloat16 *)q_idx, rope, p);
+        kern<<<grid, DI_THREADS, smem, s>>>(kmap, (const __nv_bfloat16 *)q_idx, rope, p);
     } else {
         const size_t smem = DI_NS * DI_STAGE_BYTES;
         e = cudaFuncSetAttribute(decode_score_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -71,8 +71,18 @@ template <> struct Vec16<float> {
 
 // One compressed key per 8 threads; 32 keys per 256-thread CTA.  Thread j of
 // a key handles dims [16j, 16j + 16).
-template <typename T>
-__global__ void __launch_bounds__(256) pool_prefill_kernel(const T *__restrict__ k_raw, T *__restrict__ k_pool,
+// 16 rotated values -> 16 FP8 E4M3 bytes.
+__device__ __forceinline__ void store16_e4m3(uint8_t *dst, const double (&v)[16]) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        w[i] = (uint32_t)d2e4m3x2(v[4 * i], v[4 * i + 1]) | ((uint32_t)d2e4m3x2(v[4 * i + 2], v[4 * i + 3]) << 16);
+    *reinterpret_cast<uint4 *>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// FP8: the compressed keys are stored as FP8 E4M3 (raw keys stay T).
+template <typename T, bool FP8 = false>
+__global__ void __launch_bounds__(256) pool_prefill_kernel(const T *__restrict__ k_raw, void *__restrict__ k_pool_v,
                                                            int64_t nblk, int64_t pos0, int64_t raw_stride,
                                                            int64_t pool_stride, Rope rope, int rmsnorm) {
     __shared__ float mean_s[32][kIdxDim];
@@ -129,16 +139,22 @@ __global__ void __launch_bounds__(256) pool_prefill_kernel(const T *__restrict__
             out[i] = xe;
         }
     }
-    T *dst = k_pool + ((int64_t)seq * pool_stride + pos0 / kBlock + blk) * kIdxDim + 16 * j;
-    Vec16<T>::store(dst, out);
+    const int64_t row = (int64_t)seq * pool_stride + pos0 / kBlock + blk;
+    if constexpr (FP8) {
+        store16_e4m3(static_cast<uint8_t *>(k_pool_v) + row * kIdxDim + 16 * j, out);
+    } else {
+        T *dst = static_cast<T *>(k_pool_v) + row * kIdxDim + 16 * j;
+        Vec16<T>::store(dst, out);
+    }
 }
 
 // Decode: one CTA of 128 threads per sequence, thread e owns dim e.
-template <typename T>
+template <typename T, bool FP8 = false>
 __global__ void __launch_bounds__(128) pool_decode_kernel(const T *__restrict__ k_new, T *__restrict__ ring,
-                                                          T *__restrict__ k_pool, const int32_t *__restrict__ seq_len,
-                                                          int64_t pool_stride, Rope rope, int rmsnorm,
-                                                          unsigned *status) {
+                                                          void *__restrict__ k_pool_v,
+                                                          const int32_t *__restrict__ seq_len, int64_t pool_stride,
+                                                          Rope rope, int rmsnorm, unsigned *status) {
+    __shared__ double out_s[kIdxDim];
     __shared__ float mean_s[kIdxDim];
     __shared__ double red[4];
     const int seq = blockIdx.x;
@@ -185,7 +201,16 @@ __global__ void __launch_bounds__(128) pool_decode_kernel(const T *__restrict__ 
         rope_cs(rope, (double)(s - kBlock), e < half ? e : e - half, c, sn);
         out = rope_dim(xe, xp, e, half, c, sn);
     }
-    k_pool[((int64_t)seq * pool_stride + b) * kIdxDim + e] = from_double<T>(out);
+    const int64_t row = (int64_t)seq * pool_stride + b;
+    if constexpr (FP8) {   // pairs of dims -> one 16-bit store
+        out_s[e] = out;
+        __syncthreads();
+        if ((e & 1) == 0)
+            reinterpret_cast<uint16_t *>(static_cast<uint8_t *>(k_pool_v) + row * kIdxDim)[e >> 1] =
+                d2e4m3x2(out_s[e], out_s[e + 1]);
+    } else {
+        static_cast<T *>(k_pool_v)[row * kIdxDim + e] = from_double<T>(out);
+    }
 }
 
 // Attention-layer RoPE: one CTA per (sequence, row), thread i < R/2 turns
@@ -255,28 +280,32 @@ __global__ void __launch_bounds__(128) rotate_index_q_kernel(const T *__restrict
 
 cudaError_t launch_pool_prefill(const void *k_raw, void *k_pool, int B, int64_t nblk, int64_t pos0,
                                 int64_t raw_stride, int64_t pool_stride, Rope rope, bool rmsnorm, bool bf16,
-                                cudaStream_t s) {
+                                bool fp8, cudaStream_t s) {
     if (nblk <= 0) return cudaSuccess;
     dim3 grid((unsigned)((nblk + 31) / 32), (unsigned)B);
-    if (bf16)
-        pool_prefill_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
-            (const __nv_bfloat16 *)k_raw, (__nv_bfloat16 *)k_pool, nblk, pos0, raw_stride, pool_stride, rope,
-            rmsnorm);
+    if (bf16 && fp8)
+        pool_prefill_kernel<__nv_bfloat16, true><<<grid, 256, 0, s>>>(
+            (const __nv_bfloat16 *)k_raw, k_pool, nblk, pos0, raw_stride, pool_stride, rope, rmsnorm);
+    else if (bf16)
+        pool_prefill_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>((const __nv_bfloat16 *)k_raw, k_pool, nblk, pos0,
+                                                                raw_stride, pool_stride, rope, rmsnorm);
     else
-        pool_prefill_kernel<float><<<grid, 256, 0, s>>>((const float *)k_raw, (float *)k_pool, nblk, pos0,
-                                                        raw_stride, pool_stride, rope, rmsnorm);
+        pool_prefill_kernel<float><<<grid, 256, 0, s>>>((const float *)k_raw, k_pool, nblk, pos0, raw_stride,
+                                                        pool_stride, rope, rmsnorm);
     return cudaGetLastError();
 }
 
 cudaError_t launch_pool_decode(const void *k_new, void *ring, void *k_pool, const int32_t *seq_len, int B,
-                               int64_t pool_stride, Rope rope, bool rmsnorm, bool bf16, unsigned *status,
+                               int64_t pool_stride, Rope rope, bool rmsnorm, bool bf16, bool fp8, unsigned *status,
                                cudaStream_t s) {
-    if (bf16)
+    if (bf16 && fp8)
+        pool_decode_kernel<__nv_bfloat16, true><<<B, 128, 0, s>>>(
+            (const __nv_bfloat16 *)k_new, (__nv_bfloat16 *)ring, k_pool, seq_len, pool_stride, rope, rmsnorm, status);
+    else if (bf16)
         pool_decode_kernel<__nv_bfloat16><<<B, 128, 0, s>>>((const __nv_bfloat16 *)k_new, (__nv_bfloat16 *)ring,
-                                                            (__nv_bfloat16 *)k_pool, seq_len, pool_stride, rope,
-                                                            rmsnorm, status);
+                                                            k_pool, seq_len, pool_stride, rope, rmsnorm, status);
     else
-        pool_decode_kernel<float><<<B, 128, 0, s>>>((const float *)k_new, (float *)ring, (float *)k_pool, seq_len,
+        pool_decode_kernel<float><<<B, 128, 0, s>>>((const float *)k_new, (float *)ring, k_pool, seq_len,
                                                     pool_stride, rope, rmsnorm, status);
     return cudaGetLastError();
 }

@@ -77,7 +77,7 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? QSA_OK : QSA_ERR_CUDA; }
 
-constexpr uint32_t kAllFlags = QSA_SCORE_RELU | QSA_POOL_RMSNORM;
+constexpr uint32_t kAllFlags = QSA_SCORE_RELU | QSA_POOL_RMSNORM | QSA_KEYS_FP8;
 
 size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 
@@ -147,6 +147,7 @@ int qsa_pool_keys_prefill(const void *k_raw, void *k_pool, int32_t B, int64_t n_
     if (!k_raw || !k_pool) return QSA_ERR_INVALID_ARG;
     if (flags & ~kAllFlags) return QSA_ERR_INVALID_ARG;
     if (dtype != QSA_BF16 && dtype != QSA_FP32) return QSA_ERR_UNSUPPORTED;
+    if ((flags & QSA_KEYS_FP8) && dtype != QSA_BF16) return QSA_ERR_UNSUPPORTED;
     const int64_t nblk = n_tok / kBlock;
     if (pool_stride < pos0 / kBlock + nblk) return QSA_ERR_INVALID_ARG;
     if (!aligned16(k_raw) || !aligned16(k_pool)) return QSA_ERR_INVALID_ARG;
@@ -156,7 +157,7 @@ int qsa_pool_keys_prefill(const void *k_raw, void *k_pool, int32_t B, int64_t n_
     if ((st = check_device(&di)) != QSA_OK) return st;
     return cuda_status(launch_pool_prefill(k_raw, k_pool, B, nblk, pos0, raw_stride, pool_stride, to_rope(rope),
                                            (flags & QSA_POOL_RMSNORM) != 0, dtype == QSA_BF16,
-                                           static_cast<cudaStream_t>(stream)));
+                                           (flags & QSA_KEYS_FP8) != 0, static_cast<cudaStream_t>(stream)));
 }
 
 int qsa_pool_keys_decode(const void *k_new, void *ring, void *k_pool, const int32_t *seq_len, int32_t B,
@@ -164,13 +165,14 @@ int qsa_pool_keys_decode(const void *k_new, void *ring, void *k_pool, const int3
     if (!k_new || !ring || !k_pool || !seq_len || B < 1 || pool_stride < 1) return QSA_ERR_INVALID_ARG;
     if (flags & ~kAllFlags) return QSA_ERR_INVALID_ARG;
     if (dtype != QSA_BF16 && dtype != QSA_FP32) return QSA_ERR_UNSUPPORTED;
+    if ((flags & QSA_KEYS_FP8) && dtype != QSA_BF16) return QSA_ERR_UNSUPPORTED;
     int st = check_rope(rope);
     if (st != QSA_OK) return st;
     const DeviceInfo *di = nullptr;
     if ((st = check_device(&di)) != QSA_OK) return st;
     return cuda_status(launch_pool_decode(k_new, ring, k_pool, seq_len, B, pool_stride, to_rope(rope),
-                                          (flags & QSA_POOL_RMSNORM) != 0, dtype == QSA_BF16, di->status,
-                                          static_cast<cudaStream_t>(stream)));
+                                          (flags & QSA_POOL_RMSNORM) != 0, dtype == QSA_BF16,
+                                          (flags & QSA_KEYS_FP8) != 0, di->status, static_cast<cudaStream_t>(stream)));
 }
 
 size_t qsa_index_topk_prefill_workspace(int32_t B, int64_t n_q, int64_t q0, int32_t top_k, uint32_t flags,
@@ -191,6 +193,7 @@ int qsa_index_topk_prefill(const void *q_idx, const void *k_pool, const float *h
     if (top_k < 1 || top_k > 2048) return QSA_ERR_INVALID_ARG;
     if (flags & ~kAllFlags) return QSA_ERR_INVALID_ARG;
     if (dtype != QSA_BF16 && dtype != QSA_FP32) return QSA_ERR_UNSUPPORTED;
+    if (flags & QSA_KEYS_FP8) return QSA_ERR_UNSUPPORTED;   // the prefill GEMM reads BF16 compressed keys
     if (n_q == 0) return QSA_OK;
     const int64_t nb_max = (q0 + n_q) / kBlock;
     if (pool_stride < std::max<int64_t>(nb_max, 1)) return QSA_ERR_INVALID_ARG;
@@ -248,6 +251,7 @@ int qsa_index_topk_decode(const void *q_idx, const void *k_pool, const float *he
     if (top_k < 1 || top_k > 2048) return QSA_ERR_INVALID_ARG;
     if (flags & ~kAllFlags) return QSA_ERR_INVALID_ARG;
     if (dtype != QSA_BF16 && dtype != QSA_FP32) return QSA_ERR_UNSUPPORTED;
+    if ((flags & QSA_KEYS_FP8) && dtype != QSA_BF16) return QSA_ERR_UNSUPPORTED;
     if (!aligned16(q_idx) || !aligned16(k_pool)) return QSA_ERR_INVALID_ARG;
     int st = check_rope(rope);
     if (st != QSA_OK) return st;
@@ -259,7 +263,7 @@ int qsa_index_topk_decode(const void *q_idx, const void *k_pool, const float *he
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return QSA_ERR_INVALID_ARG;
     cudaError_t e = launch_decode_index(q_idx, k_pool, head_w, seq_len, B, pool_stride, mb, top_k, sel, nsel,
                                         workspace, to_rope(rope), (flags & QSA_SCORE_RELU) != 0, dtype == QSA_BF16,
-                                        di->status, static_cast<cudaStream_t>(stream));
+                                        (flags & QSA_KEYS_FP8) != 0, di->status, static_cast<cudaStream_t>(stream));
     if (e == cudaErrorInvalidConfiguration) return QSA_ERR_UNSUPPORTED;
     return cuda_status(e);
 }

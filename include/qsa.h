@@ -76,6 +76,15 @@ extern "C" {
  * eps 1e-6); the same section says the mean is "normalized" without naming
  * the norm.  Off by default. */
 #define QSA_POOL_RMSNORM 2u
+/* Compressed keys stored as FP8 E4M3 (1 byte per value, round to nearest
+ * even from the exact rotated value, saturating at +-448): the FP8
+ * indexer-key cache of the page "Qwen3.8-Flash-Next, Layer by Layer"
+ * (section "Serving it", the recipe's indexer_kv_dtype fp8).  Accepted by
+ * qsa_pool_keys_prefill / qsa_pool_keys_decode (they write FP8 compressed
+ * keys) and qsa_index_topk_decode (it reads them); dtype must be QSA_BF16
+ * (raw keys, ring and indexer queries stay BF16).  qsa_index_topk_prefill
+ * returns QSA_ERR_UNSUPPORTED with it. */
+#define QSA_KEYS_FP8 4u
 
 /* RoPE parameters.  Rotate-half convention (style 0): for i < rotary_dim/2
  * the pair (x_i, x_{i + rotary_dim/2}) turns by the angle

@@ -78,6 +78,49 @@ def test_pool_decode_ring_matches_oracle(qsa, dtype):
     assert np.array_equal(np32(k_pool), o_pool)
 
 
+@pytest.mark.parametrize("n_tok,pos0,amp,flags", [(4099, 0, 1.0, 0), (1000, 4 * 12345, 300.0, 0),
+                                                  (515, 8, 1.0, 2), (2048, 1 << 20, 0.01, 0)])
+def test_pool_prefill_fp8_bit_exact(qsa, n_tok, pos0, amp, flags):
+    """FP8 E4M3 compressed keys: bit-exact against the oracle's rounding of
+    the exact rotated mean, including saturation (amp 300: rotated values
+    beyond 448) and subnormals (amp 0.01)."""
+    g = torch.Generator(device=DEV).manual_seed(n_tok + pos0 + 1)
+    k_raw = (torch.randn(2, n_tok, 128, generator=g, device=DEV) * amp).to(torch.bfloat16)
+    cap = pos0 // 4 + n_tok // 4 + 3
+    k_pool = torch.full((2, cap, 128), 7.0, device=DEV).to(torch.float8_e4m3fn)
+    rope = qsa.Rope(pos_scale=2.0)
+    qsa.qsa_pool_keys_prefill(k_raw, k_pool, pos0=pos0, rope=rope, flags=flags | qsa.QSA_KEYS_FP8)
+    qsa.qsa_check_status()
+    for b in range(2):
+        ref = oracle.pool_keys(np32(k_raw[b]), pos0=pos0, pos_scale=2.0, rmsnorm=bool(flags & 2), store_fp8=True)
+        got = np32(k_pool[b])
+        assert np.array_equal(got[pos0 // 4: pos0 // 4 + n_tok // 4], ref)
+        assert np.all(got[: pos0 // 4] == 7.0) and np.all(got[pos0 // 4 + n_tok // 4:] == 7.0)
+    if amp > 100:
+        assert np.abs(np32(k_pool)).max() == 448.0
+
+
+def test_pool_decode_ring_fp8_matches_oracle(qsa):
+    B, steps = 5, 23
+    g = torch.Generator(device=DEV).manual_seed(4)
+    start = torch.tensor([0, 1, 2, 3, 101], dtype=torch.int32)
+    keys = (torch.randn(B, steps, 128, generator=g, device=DEV) * 60).to(torch.bfloat16)
+    ring = torch.zeros(B, 4, 128, dtype=torch.bfloat16, device=DEV)
+    cap = (int(start.max()) + steps) // 4 + 1
+    k_pool = torch.zeros(B, cap, 128, device=DEV).to(torch.float8_e4m3fn)
+    o_ring = np.zeros((B, 4, 128), np.float32)
+    o_pool = np.zeros((B, cap, 128), np.float32)
+    for s in range(steps):
+        seq_len = (start + s + 1).to(DEV)
+        qsa.qsa_pool_keys_decode(keys[:, s].contiguous(), ring, k_pool, seq_len, flags=qsa.QSA_KEYS_FP8)
+        kn = np32(keys[:, s])
+        for b in range(B):
+            oracle.pool_decode(kn[b], o_ring[b], o_pool[b], int(start[b]) + s + 1, store_fp8=True)
+    qsa.qsa_check_status()
+    assert np.array_equal(np32(ring), o_ring)
+    assert np.array_equal(np32(k_pool), o_pool)
+
+
 def test_rope_apply_matches_oracle(qsa):
     g = torch.Generator(device=DEV).manual_seed(5)
     x = torch.randn(2, 300, 3, 128, generator=g, device=DEV).to(torch.bfloat16)
@@ -182,27 +225,32 @@ def test_attention_flags_out_of_range_ids(qsa):
 
 @pytest.mark.parametrize("dtype,flags,weights,L,B", [("bf16", 0, False, 20000, 6), ("bf16", 1, True, 9001, 3),
                                                      ("fp32", 0, False, 5000, 4), ("bf16", 0, False, 2, 5),
-                                                     ("bf16", 0, False, 70001, 3), ("fp32", 1, True, 40000, 2)])
+                                                     ("bf16", 0, False, 70001, 3), ("fp32", 1, True, 40000, 2),
+                                                     # FP8 E4M3 compressed keys: fused indexer (B 6) and
+                                                     # two-kernel path (B 3), tiny sequences
+                                                     ("bf16", 4, False, 20000, 6), ("bf16", 5, True, 70001, 3),
+                                                     ("bf16", 4, False, 2, 5), ("bf16", 6, False, 9001, 12)])
 def test_decode_pipeline(qsa, dtype, flags, weights, L, B):
     w = workloads.Workload("dec", "decode", B, L, 256, 16, 2, 128, dtype, 77, pos_scale=2.0)
     x = workloads.make_decode(w, device=DEV, ragged=True)
-    dt = x["k"].dtype
+    fp8 = bool(flags & qsa.QSA_KEYS_FP8)
+    dt = torch.float8_e4m3fn if fp8 else x["k"].dtype
     rope = rope_of(w)
     lens = x["lens"]
     cap = max(lens) // 4 + 2
     # pooled cache of the prefix (prefill pooling), ring holding the unfinished block
     k_pool = torch.zeros(B, cap, 128, dtype=dt, device=DEV)
-    ring = torch.zeros(B, 4, 128, dtype=dt, device=DEV)
+    ring = torch.zeros(B, 4, 128, dtype=x["k"].dtype, device=DEV)
     for b in range(B):
         kp = torch.zeros(1, cap, 128, dtype=dt, device=DEV)
-        qsa.qsa_pool_keys_prefill(x["k_idx"][b:b + 1, :lens[b]].contiguous(), kp, rope=rope)
+        qsa.qsa_pool_keys_prefill(x["k_idx"][b:b + 1, :lens[b]].contiguous(), kp, rope=rope, flags=flags & 6)
         k_pool[b] = kp[0]
         nb0 = lens[b] // 4
         r = lens[b] - 4 * nb0
         if r:
             ring[b, :r] = x["k_idx"][b, 4 * nb0: lens[b]]
     head_w = torch.rand(B, 4, device=DEV) * 2 if weights else None
-    qsa.qsa_pool_keys_decode(x["k_idx_new"], ring, k_pool, x["seq_len"], rope=rope, flags=flags & 2)
+    qsa.qsa_pool_keys_decode(x["k_idx_new"], ring, k_pool, x["seq_len"], rope=rope, flags=flags & 6)
     sel = torch.full((B, w.top_k), -7, dtype=torch.int32, device=DEV)
     nsel = torch.full((B,), -7, dtype=torch.int32, device=DEV)
     qsa.qsa_index_topk_decode(x["q_idx"], k_pool, x["seq_len"], sel, nsel, top_k=w.top_k, head_w=head_w,
@@ -216,11 +264,13 @@ def test_decode_pipeline(qsa, dtype, flags, weights, L, B):
         s = lens[b] + 1
         kr = np32(x["k_idx"][b, :lens[b]])
         kp = np.zeros((cap, 128), np.float32)
-        kp[: lens[b] // 4] = oracle.pool_keys(kr, pos_scale=2.0, store_bf16=dtype == "bf16")
+        kp[: lens[b] // 4] = oracle.pool_keys(kr, pos_scale=2.0, rmsnorm=bool(flags & 2),
+                                              store_bf16=dtype == "bf16", store_fp8=fp8)
         rg = np.zeros((4, 128), np.float32)
         nb0 = lens[b] // 4
         rg[: lens[b] - 4 * nb0] = kr[4 * nb0:]
-        oracle.pool_decode(np32(x["k_idx_new"][b]), rg, kp, s, pos_scale=2.0, store_bf16=dtype == "bf16")
+        oracle.pool_decode(np32(x["k_idx_new"][b]), rg, kp, s, pos_scale=2.0, rmsnorm=bool(flags & 2),
+                           store_bf16=dtype == "bf16", store_fp8=fp8)
         assert np.array_equal(np32(k_pool[b]), kp), f"pooled cache differs (seq {b})"
         ref = oracle.decode(np32(x["q_idx"][b:b + 1]), kp[None], [s],
                             head_w=None if head_w is None else head_w[b:b + 1].cpu().numpy(),
@@ -235,6 +285,38 @@ def test_decode_pipeline(qsa, dtype, flags, weights, L, B):
         err = np.abs(np32(out[b]) - ref["out"][0]).max()
         assert err <= TOL[dtype], (b, err)
         assert np.abs(lse[b].cpu().numpy() - ref["lse"][0]).max() <= (1e-3 if dtype == "bf16" else 1e-4)
+
+
+@pytest.mark.parametrize("B", [1, 40])
+def test_decode_fp8_keys_every_code_scored_exactly(qsa, B):
+    """Every finite FP8 E4M3 code but -0 (subnormals included) is one block's
+    key, in dim 127, which the rotation (rotary_dim 64) leaves alone; the
+    query is the unit vector there, so each score is exactly the key's value.
+    The top-k for k around the subnormals must then match the oracle's: a
+    widening that lost a subnormal would tie it with zero and pick lower
+    block ids.  B = 40 runs the fused indexer, B = 1 the two-kernel path."""
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0x80, 0xFF)], np.uint8)
+    nb = len(codes)
+    cap = nb + 1
+    rng = np.random.default_rng(17)
+    k_pool = torch.zeros(B, cap, 128, dtype=torch.uint8)
+    for b in range(B):
+        k_pool[b, :nb, 127] = torch.from_numpy(codes[rng.permutation(nb)])
+    k_pool = k_pool.view(torch.float8_e4m3fn).to(DEV)
+    q_idx = torch.zeros(B, 4, 128, dtype=torch.bfloat16, device=DEV)
+    q_idx[:, 0, 127] = 1.0
+    seq_len = torch.full((B,), 4 * nb + 1, dtype=torch.int32, device=DEV)
+    rope = qsa.Rope(rotary_dim=64)
+    kp = np32(k_pool)
+    for top_k in [1, 100, 119, 120, 123, 126, 127, 128, 130, 252]:
+        sel = torch.full((B, top_k), -7, dtype=torch.int32, device=DEV)
+        nsel = torch.full((B,), -7, dtype=torch.int32, device=DEV)
+        qsa.qsa_index_topk_decode(q_idx, k_pool, seq_len, sel, nsel, top_k=top_k, rope=rope,
+                                  flags=qsa.QSA_KEYS_FP8)
+        qsa.qsa_check_status()
+        ref = oracle.decode(np32(q_idx), kp, seq_len.cpu().numpy(), top_k=top_k, rotary_dim=64)
+        assert np.array_equal(nsel.cpu().numpy(), ref["nsel"])
+        assert np.array_equal(sel.cpu().numpy(), ref["sel"]), top_k
 
 
 @pytest.mark.parametrize("dtype,flags,lens", [("bf16", 0, [40000, 65537, 2049]), ("bf16", 1, [40000, 65537, 2049]),

@@ -81,20 +81,23 @@ def _decode_check(qsa, w, B=None, L=None, ragged=False):
     lens = x["lens"]
     rope = rope_of(w)
     dt = x["k"].dtype
+    fp8 = w.extra.get("keys") == "fp8"          # compressed keys stored as FP8 E4M3
+    kflags = qsa.QSA_KEYS_FP8 if fp8 else 0
+    kdt = torch.float8_e4m3fn if fp8 else dt
     cap = max(lens) // 4 + 1
-    k_pool = torch.zeros(B, cap, 128, dtype=dt, device=DEV)
+    k_pool = torch.zeros(B, cap, 128, dtype=kdt, device=DEV)
     ring = torch.zeros(B, 4, 128, dtype=dt, device=DEV)
     for b in range(B):
-        kp = torch.zeros(1, cap, 128, dtype=dt, device=DEV)
-        qsa.qsa_pool_keys_prefill(x["k_idx"][b:b + 1, :lens[b]].contiguous(), kp, rope=rope)
+        kp = torch.zeros(1, cap, 128, dtype=kdt, device=DEV)
+        qsa.qsa_pool_keys_prefill(x["k_idx"][b:b + 1, :lens[b]].contiguous(), kp, rope=rope, flags=kflags)
         k_pool[b] = kp[0]
         nb0 = lens[b] // 4
         if lens[b] > 4 * nb0:
             ring[b, :lens[b] - 4 * nb0] = x["k_idx"][b, 4 * nb0: lens[b]]
-    qsa.qsa_pool_keys_decode(x["k_idx_new"], ring, k_pool, x["seq_len"], rope=rope)
+    qsa.qsa_pool_keys_decode(x["k_idx_new"], ring, k_pool, x["seq_len"], rope=rope, flags=kflags)
     sel = torch.empty(B, w.top_k, dtype=torch.int32, device=DEV)
     nsel = torch.empty(B, dtype=torch.int32, device=DEV)
-    qsa.qsa_index_topk_decode(x["q_idx"], k_pool, x["seq_len"], sel, nsel, top_k=w.top_k, rope=rope)
+    qsa.qsa_index_topk_decode(x["q_idx"], k_pool, x["seq_len"], sel, nsel, top_k=w.top_k, rope=rope, flags=kflags)
     out = torch.empty_like(x["q"])
     qsa.qsa_sparse_attn_decode(x["q"], x["k"], x["v"], x["seq_len"], sel, nsel, out)
     qsa.qsa_check_status()
@@ -103,11 +106,12 @@ def _decode_check(qsa, w, B=None, L=None, ragged=False):
         s = lens[b] + 1
         kr = np32(x["k_idx"][b, :lens[b]])
         kp = np.zeros((cap, 128), np.float32)
-        kp[: lens[b] // 4] = oracle.pool_keys(kr, base=w.rope_base, pos_scale=w.pos_scale)
+        kp[: lens[b] // 4] = oracle.pool_keys(kr, base=w.rope_base, pos_scale=w.pos_scale, store_fp8=fp8)
         rg = np.zeros((4, 128), np.float32)
         nb0 = lens[b] // 4
         rg[: lens[b] - 4 * nb0] = kr[4 * nb0:]
-        oracle.pool_decode(np32(x["k_idx_new"][b]), rg, kp, s, base=w.rope_base, pos_scale=w.pos_scale)
+        oracle.pool_decode(np32(x["k_idx_new"][b]), rg, kp, s, base=w.rope_base, pos_scale=w.pos_scale,
+                           store_fp8=fp8)
         assert np.array_equal(np32(k_pool[b]), kp), f"pooled keys differ (seq {b})"
         ref = oracle.decode(np32(x["q_idx"][b:b + 1]), kp[None], [s], q=np32(x["q"][b:b + 1]),
                             k=np32(x["k"][b:b + 1]), v=np32(x["v"][b:b + 1]), top_k=w.top_k,
@@ -136,3 +140,11 @@ def test_decode_128k_ragged_tails(qsa):
 
 def test_decode_1m_b8_scaled_positions(qsa):
     _decode_check(qsa, workloads.WORKLOADS["decode_b8_l1m_scale4"])
+
+
+def test_decode_128k_b64_fp8_keys(qsa):
+    _decode_check(qsa, workloads.WORKLOADS["decode_b64_l128k_fp8keys"])
+
+
+def test_decode_1m_b8_fp8_keys(qsa):
+    _decode_check(qsa, workloads.WORKLOADS["decode_b8_l1m_scale4_fp8keys"])

@@ -87,6 +87,14 @@ def test_invalid_arguments_are_rejected_before_launch(qsa):
                                      None) == qsa.QSA_ERR_INVALID_ARG
     assert lib.qsa_dense_attn_decode(fake, fake, fake, None, 1, 64, 16, 2, 128, 0.1, fake, None, fake, 1 << 20, 0,
                                      None) == qsa.QSA_ERR_INVALID_ARG
+    # FP8 compressed keys: BF16 only; the prefill indexer reads BF16 keys
+    fp8 = qsa.QSA_KEYS_FP8
+    assert lib.qsa_pool_keys_prefill(fake, fake, 1, 16, 0, 16, 4, rope, fp8, 1, None) == qsa.QSA_ERR_UNSUPPORTED
+    assert lib.qsa_pool_keys_decode(fake, fake, fake, fake, 1, 4, rope, fp8, 1, None) == qsa.QSA_ERR_UNSUPPORTED
+    assert lib.qsa_index_topk_prefill(fake, fake, None, 1, 16, 0, 4, 4, fake, fake, fake, 1 << 20, rope, fp8, 0,
+                                      None) == qsa.QSA_ERR_UNSUPPORTED
+    assert lib.qsa_index_topk_decode(fake, fake, None, fake, 1, 4, 4, 4, fake, fake, fake, 1 << 20, rope, fp8, 1,
+                                     None) == qsa.QSA_ERR_UNSUPPORTED
     # misaligned pointer
     odd = ctypes.c_void_p(4098)
     assert lib.qsa_pool_keys_prefill(odd, fake, 1, 16, 0, 16, 4, rope, 0, 0, None) == qsa.QSA_ERR_INVALID_ARG

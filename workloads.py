@@ -61,6 +61,11 @@ WORKLOADS = {
                                         128, "bf16", 1004, heavy_tail=True),
     "decode_b8_l1m_scale4": Workload("decode_b8_l1m_scale4", "decode", 8, 1048576, 512, 16, 2, 128,
                                      "bf16", 1005, pos_scale=4.0),
+    # the decode workloads with the compressed keys stored as FP8 E4M3 (same data and seeds)
+    "decode_b64_l128k_fp8keys": Workload("decode_b64_l128k_fp8keys", "decode", 64, 131072, 512, 16, 2, 128,
+                                         "bf16", 1003, extra={"keys": "fp8"}),
+    "decode_b8_l1m_scale4_fp8keys": Workload("decode_b8_l1m_scale4_fp8keys", "decode", 8, 1048576, 512, 16, 2,
+                                             128, "bf16", 1005, pos_scale=4.0, extra={"keys": "fp8"}),
     # full causal decode attention on the same caches as the QSA decode workloads
     "dense_b64_l128k": Workload("dense_b64_l128k", "dense", 64, 131072, 512, 16, 2, 128, "bf16", 1003),
     "dense_b8_l1m_scale4": Workload("dense_b8_l1m_scale4", "dense", 8, 1048576, 512, 16, 2, 128, "bf16", 1005,
