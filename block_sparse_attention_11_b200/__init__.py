@@ -158,11 +158,13 @@ def _check(status: int, where: str):
         raise QSAError(status, where)
 
 
-def _ws(nbytes: int, device, workspace):
+def _ws(nbytes: int, device, workspace, zero=False):
+    """Workspace pointer and size; allocated here when none is given (zero-filled
+    for an entry point whose workspace must start zero)."""
     if nbytes == 0:
         return None, 0
     if workspace is None:
-        workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        workspace = (torch.zeros if zero else torch.empty)(nbytes, dtype=torch.uint8, device=device)
     if workspace.numel() * workspace.element_size() < nbytes:
         raise ValueError(f"workspace too small: need {nbytes} bytes")
     return workspace.data_ptr(), workspace.numel() * workspace.element_size()
@@ -219,7 +221,7 @@ def qsa_index_topk_decode(q_idx, k_pool, seq_len, sel, nsel, max_blocks=None, to
     B = q_idx.shape[0]
     max_blocks = k_pool.shape[1] if max_blocks is None else max_blocks
     need = qsa_index_topk_decode_workspace(B, max_blocks, top_k, flags, dt)
-    wp, wb = _ws(need, q_idx.device, workspace)
+    wp, wb = _ws(need, q_idx.device, workspace, zero=True)   # zero-filled once; calls leave it zero
     st = lib.qsa_index_topk_decode(_ptr(q_idx, None, "q_idx"), _kpool_ptr(k_pool, q_idx.dtype, flags),
                                    _ptr(head_w, torch.float32, "head_w"), _ptr(seq_len, torch.int32, "seq_len"), B,
                                    k_pool.shape[1], max_blocks, top_k, _ptr(sel, torch.int32, "sel"),

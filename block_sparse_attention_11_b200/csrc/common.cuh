@@ -17,6 +17,7 @@
 #define QSA_DEV_BAD_LENGTH 2u   // a sequence length beyond the caller's capacity
 #define QSA_DEV_TIMEOUT 4u      // an mbarrier wait ran out of polls
 #define QSA_DEV_SELECT 8u       // internal inconsistency in a top-k select
+#define QSA_DEV_WORKSPACE 16u   // a decode-indexer workspace whose histogram was not zero at the call
 
 namespace qsa {
 

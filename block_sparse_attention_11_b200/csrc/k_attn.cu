@@ -580,41 +580,60 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, AttnCfg<HKV>::kMinCtas
     }
 }
 
-// Decode combine: one CTA of 128 threads per (sequence, q head).  The split
-// lse values are read in parallel, then every dim sums its weighted partials.
+// Decode combine: one CTA of 128 threads per (sequence, q head): out =
+// sum_s w_s o_s / sum_s w_s with w_s = 2^(lse_s - max lse).  Warp j sums the
+// splits s = j mod 4 (lane l: dims 4l .. 4l + 3), so four independent chains
+// of loads are in flight; warps 1-3 hand their sums to warp 0.
 __global__ void __launch_bounds__(128) attn_combine_kernel(const float *__restrict__ part_o,
                                                            const float *__restrict__ part_lse, int splits, int Hq,
                                                            __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
-    __shared__ float wsm[1024];
-    __shared__ float red[4];
+    __shared__ float4 red_o[3][32];
+    __shared__ float red_m[4], red_d[4];
     pdl_wait();
-    const int seq = blockIdx.x / Hq, h = blockIdx.x % Hq, e = threadIdx.x;
+    const int seq = blockIdx.x / Hq, h = blockIdx.x % Hq, tid = threadIdx.x, lane = tid & 31, sg = tid >> 5;
+    const float *pl = part_lse + (int64_t)seq * splits * Hq + h;   // split s at pl[s * Hq]
     float mx = -INFINITY;
-    for (int s = e; s < splits; s += 128) {
-        const float v = part_lse[((int64_t)seq * splits + s) * Hq + h];
-        wsm[s] = v;
-        mx = fmaxf(mx, v);
-    }
+    for (int s = tid; s < splits; s += 128) mx = fmaxf(mx, pl[(int64_t)s * Hq]);
+#pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    if ((e & 31) == 0) red[e >> 5] = mx;
+    if (lane == 0) red_m[sg] = mx;
     __syncthreads();
-    mx = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-    __syncthreads();
+    mx = fmaxf(fmaxf(red_m[0], red_m[1]), fmaxf(red_m[2], red_m[3]));
+    const float *po = part_o + ((int64_t)seq * splits * Hq + h) * 128 + 4 * lane;
     float den = 0.f;
-    for (int s = e; s < splits; s += 128) {
-        const float w = (mx == -INFINITY || wsm[s] == -INFINITY) ? 0.f : exp2f(wsm[s] - mx);
-        wsm[s] = w;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int s = sg; s < splits; s += 4) {
+        const float v = pl[(int64_t)s * Hq];
+        const float4 x = *reinterpret_cast<const float4 *>(po + (int64_t)s * Hq * 128);
+        const float w = (mx == -INFINITY || v == -INFINITY) ? 0.f : exp2f(v - mx);
         den += w;
+        acc.x += w * x.x;
+        acc.y += w * x.y;
+        acc.z += w * x.z;
+        acc.w += w * x.w;
     }
-    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-    if ((e & 31) == 0) red[e >> 5] = den;
+    if (sg > 0) {
+        red_o[sg - 1][lane] = acc;
+        if (lane == 0) red_d[sg] = den;
+    }
     __syncthreads();
-    den = red[0] + red[1] + red[2] + red[3];
-    float acc = 0.f;
-    const float *po = part_o + ((int64_t)seq * splits * Hq + h) * 128 + e;
-    for (int s = 0; s < splits; ++s) acc += wsm[s] * po[(int64_t)s * Hq * 128];
-    out[((int64_t)seq * Hq + h) * 128 + e] = __float2bfloat16_rn(den > 0.f ? acc / den : 0.f);
-    if (lse && e == 0) lse[(int64_t)seq * Hq + h] = den > 0.f ? (mx + log2f(den)) / kLog2e : -INFINITY;
+    if (sg != 0) return;
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+        const float4 o = red_o[j][lane];
+        acc.x += o.x;
+        acc.y += o.y;
+        acc.z += o.z;
+        acc.w += o.w;
+        den += red_d[j + 1];
+    }
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+    uint2 v;
+    v.x = pack_bf16(acc.x * inv, acc.y * inv);
+    v.y = pack_bf16(acc.z * inv, acc.w * inv);
+    *reinterpret_cast<uint2 *>(out + ((int64_t)seq * Hq + h) * 128 + 4 * lane) = v;
+    if (lse && lane == 0) lse[(int64_t)seq * Hq + h] = den > 0.f ? (mx + log2f(den)) / kLog2e : -INFINITY;
 }
 
 // fp32 SIMT attention: one warp per (item, q head); lane owns 4 dims.

@@ -57,6 +57,7 @@ __global__ void __launch_bounds__(DI_THREADS, 2)
     __shared__ float qsum[kIdxDim];
     __shared__ uint32_t lh[2048];
 
+    pdl_wait();      // the compressed keys come from the previous kernel (ring pooling)
     pdl_trigger();
     const int seq = blockIdx.y, c = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -468,6 +469,7 @@ __global__ void __launch_bounds__(DI_THREADS, 2)
     extern __shared__ uint8_t dsm_raw[];
     DecodeMmaSmem<FP8> &sm = *reinterpret_cast<DecodeMmaSmem<FP8> *>(
         (reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
+    pdl_wait();      // the compressed keys come from the previous kernel (ring pooling)
     pdl_trigger();
     const int seq = blockIdx.y, c = blockIdx.x;
     const int tid = threadIdx.x;
@@ -532,9 +534,10 @@ struct SelectArgs {
     int64_t pool_stride, max_blocks, kstride, chunk;   // chunk: keys per CTA (whole tiles for the select kernel)
     int gmax, top_k;                                    // gmax: CTAs per cluster (<= DS_CLUSTER)
     const uint32_t *keys;   // [B][kstride] score keys (select kernel)
-    const uint32_t *hist;   // [B][2048] histogram of the keys' top 11 bits (select kernel)
+    uint32_t *hist;         // [B][2048] histogram of the keys' top 11 bits (select kernel; cleared after use)
     uint2 *cand;            // [B][kstride]: chunk g's candidates past DS_LCAND, at g * chunk + position
     int32_t *sel, *nsel;
+    unsigned *status;
 };
 
 struct DsSmem {
@@ -549,6 +552,7 @@ struct DsSmem {
     uint32_t ci[DS_CAND_SMEM];          // candidate block ids
     int32_t alist[DS_MAX_K];            // ids above bin d1 (ascending)
     int32_t slist[DS_MAX_K];            // selected candidate ids (ascending)
+    uint32_t htotal;                    // select kernel: sum of the scorer's histogram
     uint32_t aoff[DS_CLUSTER + 1];      // prefix of the above counts per chunk
     uint32_t coff[DS_CLUSTER + 1];      // prefix of the candidate counts per chunk
     uint32_t wsum[32];
@@ -670,17 +674,23 @@ __device__ __forceinline__ void select_leader(DsSmem &sm, int gseq, uint32_t d1,
                                               int64_t chunk, const uint2 *cand_seq, int top_k, int32_t *out,
                                               int32_t *nsel_out) {
     const int tid = threadIdx.x;
-    // per-chunk offsets of the above ids and of the candidates
-    if (tid == 0) {
-        uint32_t ea = 0, ec = 0;
-        for (int c = 0; c < gseq; ++c) {
-            sm.aoff[c] = ea;
-            sm.coff[c] = ec;
-            ea += ld_dsmem(dsmem_addr(&sm.my_na, c));
-            ec += ld_dsmem(dsmem_addr(&sm.my_nc, c));
+    // per-chunk offsets of the above ids and of the candidates: lane c reads
+    // CTA c's counts (all at once), an exclusive warp scan gives the offsets
+    if (tid < 32) {
+        const int lane = tid;
+        uint32_t na = 0, nc = 0;
+        if (lane < gseq) {
+            na = ld_dsmem(dsmem_addr(&sm.my_na, lane));
+            nc = ld_dsmem(dsmem_addr(&sm.my_nc, lane));
         }
-        sm.aoff[gseq] = ea;
-        sm.coff[gseq] = ec;
+        uint32_t ia = na, ic = nc;   // inclusive scans
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t va = __shfl_up_sync(0xffffffffu, ia, o), vc = __shfl_up_sync(0xffffffffu, ic, o);
+            if (lane >= o) { ia += va; ic += vc; }
+        }
+        if (lane < gseq) { sm.aoff[lane] = ia - na; sm.coff[lane] = ic - nc; }
+        if (lane == gseq - 1) { sm.aoff[gseq] = ia; sm.coff[gseq] = ic; }
     }
     __syncthreads();
     const int na_all = (int)min(sm.aoff[gseq], (uint32_t)(top_k - 1));
@@ -797,8 +807,10 @@ __global__ void __launch_bounds__(DS_THREADS)
     const int top_k = a.top_k;
     int32_t *out = a.sel + (int64_t)seq * top_k;
     const int64_t c0 = (int64_t)rank * a.chunk, c1 = min(c0 + a.chunk, nb);
+    uint32_t *ghist = a.hist + (int64_t)seq * 2048;  // the scorer's counts; zero again when this kernel ends
     if (nb <= top_k) {                               // the whole cluster takes this branch
         select_all<DS_THREADS>(c0, c1, nb, top_k, rank, out, a.nsel + seq);
+        if (rank == 0) reinterpret_cast<uint4 *>(ghist)[tid] = make_uint4(0u, 0u, 0u, 0u);
         return;
     }
     const int gseq = (int)((nb + a.chunk - 1) / a.chunk);   // CTAs with keys (<= cluster size)
@@ -809,17 +821,28 @@ __global__ void __launch_bounds__(DS_THREADS)
     const int m = load16(row, c0 + (int64_t)DS_PER_THREAD * tid, c1, a.kstride, k);
     // bin of the k-th largest key from the scorer's histogram
     static_assert(DS_THREADS * 4 == 2048, "one 16-byte histogram load per thread");
-    reinterpret_cast<uint4 *>(sm.s.hist)[tid] = __ldcg(reinterpret_cast<const uint4 *>(a.hist + (int64_t)seq * 2048) + tid);
-    if (tid == 0) { sm.s.digit = 0; sm.s.k_rem = 1; }
+    const uint4 hv = __ldcg(reinterpret_cast<const uint4 *>(ghist) + tid);
+    reinterpret_cast<uint4 *>(sm.s.hist)[tid] = hv;
+    if (tid == 0) { sm.s.digit = 0; sm.s.k_rem = 1; sm.htotal = 0; }
     __syncthreads();
+    if (rank == 0) {   // the counts must add up to the keys scored: else the workspace was not zero
+        uint32_t part = hv.x + hv.y + hv.z + hv.w;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+        if ((tid & 31) == 0) atomicAdd(&sm.htotal, part);
+    }
     sel_find_digit(sm.s, 2048, top_k);
     const uint32_t d1 = (uint32_t)sm.s.digit;
     const int k_rem1 = sm.s.k_rem;
     build_lists<DS_THREADS>(
         sm, [&](int64_t i0, uint32_t (&kk)[16]) { return load16(row, i0, c1, a.kstride, kk); }, c0, c1, d1, top_k,
         cand_seq, k, m);
-    cluster_sync();                                  // every CTA's lists are complete
-    if (rank == 0) select_leader<DS_THREADS>(sm, gseq, d1, k_rem1, nb, a.chunk, cand_seq, top_k, out, a.nsel + seq);
+    cluster_sync();                                  // every CTA's lists are complete (and has read ghist)
+    if (rank == 0) {
+        reinterpret_cast<uint4 *>(ghist)[tid] = make_uint4(0u, 0u, 0u, 0u);
+        if (tid == 0 && sm.htotal != (uint32_t)nb) flag(a.status, QSA_DEV_WORKSPACE);
+        select_leader<DS_THREADS>(sm, gseq, d1, k_rem1, nb, a.chunk, cand_seq, top_k, out, a.nsel + seq);
+    }
     cluster_sync();                                  // CTA 0 has finished reading the others' lists
 }
 
@@ -1084,7 +1107,7 @@ struct DecodeWs {
     uint32_t *keys;
     uint2 *cand;
     uint32_t *hist;
-    size_t zero_bytes;   // hist, cleared before every call
+    size_t hist_bytes;   // zero between calls: the select kernel clears what the scorer added
     size_t total;
 };
 
@@ -1099,8 +1122,8 @@ DecodeWs decode_ws(void *base, int B, int64_t max_blocks, int top_k) {
     d.cand = reinterpret_cast<uint2 *>(w + off);
     off += r256((size_t)B * ks * 8);
     d.hist = reinterpret_cast<uint32_t *>(w + off);
-    d.zero_bytes = (size_t)B * 2048 * 4;
-    off += r256(d.zero_bytes);
+    d.hist_bytes = (size_t)B * 2048 * 4;
+    off += r256(d.hist_bytes);
     d.total = off;
     return d;
 }
@@ -1125,7 +1148,7 @@ cudaError_t launch_decode_index(const void *q_idx, const void *k_pool, const flo
         DecodeParams p{seq_len, head_w, pool_stride, max_blocks, fp.chunk, kstride, fp.C, top_k, relu ? 1 : 0,
                        d.keys, d.hist, status};
         SelectArgs sa{seq_len, pool_stride, max_blocks, kstride, fp.chunk, fp.C, top_k, d.keys, d.hist, d.cand,
-                      sel, nsel};
+                      sel, nsel, status};
         auto kern = fp8 ? decode_index_fused_kernel<true> : decode_index_fused_kernel<false>;
         const size_t smem = (fp8 ? sizeof(FusedSmem<true>) : sizeof(FusedSmem<false>)) + 1024;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -1138,8 +1161,7 @@ cudaError_t launch_decode_index(const void *q_idx, const void *k_pool, const flo
                                   kmap, (const __nv_bfloat16 *)q_idx, rope, p, sa);
     }
     const DecodePlan pl = decode_index_plan(B, max_blocks, bf16);
-    cudaError_t e = cudaMemsetAsync(d.hist, 0, d.zero_bytes, s);
-    if (e != cudaSuccess) return e;
+    cudaError_t e;
     DecodeParams p{seq_len, head_w, pool_stride, max_blocks, pl.chunk, kstride, pl.chunks, top_k, relu ? 1 : 0,
                    d.keys, d.hist, status};
     dim3 grid((unsigned)pl.chunks, (unsigned)B);
@@ -1150,19 +1172,21 @@ cudaError_t launch_decode_index(const void *q_idx, const void *k_pool, const flo
         const size_t smem = (fp8 ? sizeof(DecodeMmaSmem<true>) : sizeof(DecodeMmaSmem<false>)) + 1024;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        kern<<<grid, DI_THREADS, smem, s>>>(kmap, (const __nv_bfloat16 *)q_idx, rope, p);
+        e = launch_pdl(kern, grid, dim3(DI_THREADS), smem, s, kmap, (const __nv_bfloat16 *)q_idx, rope, p);
+        if (e != cudaSuccess) return e;
     } else {
         const size_t smem = DI_NS * DI_STAGE_BYTES;
         e = cudaFuncSetAttribute(decode_score_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        decode_score_kernel<float><<<grid, DI_THREADS, smem, s>>>((const float *)q_idx, (const float *)k_pool, rope,
-                                                                  p);
+        e = launch_pdl(decode_score_kernel<float>, grid, dim3(DI_THREADS), smem, s, (const float *)q_idx,
+                       (const float *)k_pool, rope, p);
+        if (e != cudaSuccess) return e;
     }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const SelectLayout l = select_layout(max_blocks);
     SelectArgs sa{seq_len, pool_stride, max_blocks, kstride, l.chunk, l.gmax, top_k, d.keys, d.hist, d.cand, sel,
-                  nsel};
+                  nsel, status};
     const dim3 sgrid((unsigned)l.gmax, (unsigned)B);
     e = cudaFuncSetAttribute(decode_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(DsSmem));
     if (e != cudaSuccess) return e;

@@ -157,6 +157,8 @@ __global__ void __launch_bounds__(128) pool_decode_kernel(const T *__restrict__ 
     __shared__ double out_s[kIdxDim];
     __shared__ float mean_s[kIdxDim];
     __shared__ double red[4];
+    pdl_wait();      // k_new and seq_len may come from the previous kernel
+    pdl_trigger();   // the indexer may launch; it waits for this grid before reading k_pool
     const int seq = blockIdx.x;
     const int e = threadIdx.x;
     const int64_t s = seq_len[seq];
@@ -298,16 +300,17 @@ cudaError_t launch_pool_prefill(const void *k_raw, void *k_pool, int B, int64_t 
 cudaError_t launch_pool_decode(const void *k_new, void *ring, void *k_pool, const int32_t *seq_len, int B,
                                int64_t pool_stride, Rope rope, bool rmsnorm, bool bf16, bool fp8, unsigned *status,
                                cudaStream_t s) {
+    const int rn = rmsnorm ? 1 : 0;
     if (bf16 && fp8)
-        pool_decode_kernel<__nv_bfloat16, true><<<B, 128, 0, s>>>(
-            (const __nv_bfloat16 *)k_new, (__nv_bfloat16 *)ring, k_pool, seq_len, pool_stride, rope, rmsnorm, status);
-    else if (bf16)
-        pool_decode_kernel<__nv_bfloat16><<<B, 128, 0, s>>>((const __nv_bfloat16 *)k_new, (__nv_bfloat16 *)ring,
-                                                            k_pool, seq_len, pool_stride, rope, rmsnorm, status);
-    else
-        pool_decode_kernel<float><<<B, 128, 0, s>>>((const float *)k_new, (float *)ring, k_pool, seq_len,
-                                                    pool_stride, rope, rmsnorm, status);
-    return cudaGetLastError();
+        return launch_pdl(pool_decode_kernel<__nv_bfloat16, true>, dim3(B), dim3(128), 0, s,
+                          (const __nv_bfloat16 *)k_new, (__nv_bfloat16 *)ring, k_pool, seq_len, pool_stride, rope,
+                          rn, status);
+    if (bf16)
+        return launch_pdl(pool_decode_kernel<__nv_bfloat16, false>, dim3(B), dim3(128), 0, s,
+                          (const __nv_bfloat16 *)k_new, (__nv_bfloat16 *)ring, k_pool, seq_len, pool_stride, rope,
+                          rn, status);
+    return launch_pdl(pool_decode_kernel<float, false>, dim3(B), dim3(128), 0, s, (const float *)k_new, (float *)ring,
+                      k_pool, seq_len, pool_stride, rope, rn, status);
 }
 
 cudaError_t launch_rope_apply(void *x, int B, int64_t n, int H, int d, int64_t pos0, Rope rope, bool bf16,

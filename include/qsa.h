@@ -106,8 +106,11 @@ QSA_API int qsa_version(void);
 
 /* Reads and clears the device status word of the current device after
  * synchronising `stream`.  Returns QSA_OK, or QSA_ERR_DEVICE when a kernel
- * flagged an out-of-range index or a wait timeout since the last call.  If
- * detail != NULL it receives the raw status bits (host pointer). */
+ * flagged an error since the last call.  If detail != NULL it receives the
+ * raw status bits (host pointer): 1 a selected block id out of range, 2 a
+ * sequence length beyond the caller's capacity, 4 a bounded wait that ran
+ * out, 8 an internal inconsistency of a top-k select, 16 a decode-indexer
+ * workspace that was not zero-filled before its first use. */
 QSA_API int qsa_check_status(void *stream, uint32_t *detail);
 
 /* ========================================================================= */
@@ -213,7 +216,12 @@ QSA_API int qsa_index_topk_prefill(const void *q_idx, const void *k_pool, const 
  *           a sequence beyond it or beyond pool_stride is flagged and gets
  *           nsel = 0).
  * sel       device, [B][top_k] int32;  nsel device, [B] int32.
- * workspace at least qsa_index_topk_decode_workspace() bytes.
+ * workspace at least qsa_index_topk_decode_workspace() bytes, zero-filled
+ *           once after it is allocated (cudaMemset): it holds per-sequence
+ *           score histograms that a call accumulates and clears again, so a
+ *           workspace stays zero between calls and serves any number of them
+ *           in stream order.  A call that finds a histogram not zero at its
+ *           start flags status bit 16 (its selection is then unreliable).
  */
 QSA_API size_t qsa_index_topk_decode_workspace(int32_t B, int64_t max_blocks, int32_t top_k, uint32_t flags,
                                        int32_t dtype);

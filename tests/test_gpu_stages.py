@@ -347,6 +347,40 @@ def test_decode_select_all_ties(qsa, dtype, flags, lens):
         assert np.array_equal(sel[b].cpu().numpy(), exp), b
 
 
+def test_decode_index_workspace_stays_zero_and_dirty_one_is_flagged(qsa):
+    """The two-kernel decode indexer leaves its workspace zero after a call,
+    so one zero-filled workspace serves any number of calls; a workspace whose
+    histogram was not zero is flagged (status bit 16)."""
+    w = workloads.Workload("dec_ws", "decode", 2, 20001, 256, 16, 2, 128, "bf16", 93)
+    x = workloads.make_decode(w, device=DEV)
+    rope = rope_of(w)
+    cap = w.T // 4 + 1
+    k_pool = torch.zeros(2, cap, 128, dtype=torch.bfloat16, device=DEV)
+    qsa.qsa_pool_keys_prefill(x["k_idx"], k_pool, rope=rope)
+    need = qsa.qsa_index_topk_decode_workspace(2, cap, w.top_k)
+    ws = torch.zeros(need, dtype=torch.uint8, device=DEV)
+    sel = torch.empty(2, w.top_k, dtype=torch.int32, device=DEV)
+    nsel = torch.empty(2, dtype=torch.int32, device=DEV)
+    run = lambda: qsa.qsa_index_topk_decode(x["q_idx"], k_pool, x["seq_len"], sel, nsel, max_blocks=cap,
+                                            top_k=w.top_k, rope=rope, workspace=ws)
+    run()
+    qsa.qsa_check_status()
+    first = sel.clone()
+    hist_bytes = (2 * 2048 * 4 + 255) // 256 * 256        # the workspace ends with [B][2048] u32 counts
+    assert int(ws[need - hist_bytes:].count_nonzero()) == 0
+    run()
+    qsa.qsa_check_status()
+    assert torch.equal(sel, first)
+    ws[need - hist_bytes] = 1                              # one stray count in sequence 0's lowest bin
+    run()
+    with pytest.raises(qsa.QSAError):
+        qsa.qsa_check_status()
+    assert torch.equal(sel, first)                         # a count in the lowest bin moves nothing
+    assert int(ws[need - hist_bytes:].count_nonzero()) == 0
+    run()
+    qsa.qsa_check_status()
+
+
 def test_decode_step_graph_replay_matches_eager(qsa):
     """A decode step (ring pooling, indexer, attention with caller workspaces)
     captured in a CUDA graph and replayed gives the eager results bit for bit."""
@@ -362,7 +396,7 @@ def test_decode_step_graph_replay_matches_eager(qsa):
         k_pool[b] = kp[0]
     ring0 = torch.zeros(B, 4, 128, dtype=torch.bfloat16, device=DEV)
     max_blocks = cap
-    ws_i = torch.empty(qsa.qsa_index_topk_decode_workspace(B, max_blocks, w.top_k), dtype=torch.uint8, device=DEV)
+    ws_i = torch.zeros(qsa.qsa_index_topk_decode_workspace(B, max_blocks, w.top_k), dtype=torch.uint8, device=DEV)
     ws_a = torch.empty(qsa.qsa_sparse_attn_decode_workspace(B, w.Hq, w.d, w.top_k), dtype=torch.uint8, device=DEV)
 
     def step(ring, pool, sel, nsel, out):
