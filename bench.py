@@ -234,9 +234,29 @@ class DecodeRunner:
         # compressed keys in the computation type, or FP8 E4M3 ("keys": "fp8")
         self.fp8 = w.extra.get("keys") == "fp8"
         self.kflags = qsa.QSA_KEYS_FP8 if self.fp8 else 0
-        self.k_pool = torch.zeros(B, self.cap, 128, dtype=torch.float8_e4m3fn if self.fp8 else dt, device=dev)
-        qsa.qsa_pool_keys_prefill(x["k_idx"], self.k_pool, rope=self.rope,      # the cache's compressed keys
-                                  flags=self.kflags)
+        kdt = torch.float8_e4m3fn if self.fp8 else dt
+        # paged caches ("page_tokens"): every sequence's pages scattered over a
+        # shuffled pool, one page-table row per sequence
+        self.pt = int(w.extra.get("page_tokens", 0))
+        if self.pt:
+            per_seq = (L + self.pt) // self.pt                 # positions 0 .. L
+            num_pages = B * per_seq
+            perm = torch.randperm(num_pages, generator=torch.Generator().manual_seed(w.seed))
+            self.table = perm.view(B, per_seq).to(torch.int32).to(dev)
+            pos = torch.arange(L + 1, device=dev)
+            slots = (self.table[:, pos // self.pt].long() * self.pt + pos % self.pt)   # [B][L + 1]
+            for name in ("k", "v"):
+                pg = torch.empty(num_pages * self.pt, w.Hkv, w.d, dtype=dt, device=dev)
+                pg[slots.reshape(-1)] = x[name][:, :L + 1].reshape(-1, w.Hkv, w.d)
+                x[name] = pg
+            torch.cuda.empty_cache()
+            self.k_pool = torch.zeros(num_pages * self.pt // 4, 128, dtype=kdt, device=dev)
+            qsa.qsa_pool_keys_prefill_paged(x["k_idx"], self.k_pool, self.table, self.pt, rope=self.rope,
+                                            flags=self.kflags)
+        else:
+            self.k_pool = torch.zeros(B, self.cap, 128, dtype=kdt, device=dev)
+            qsa.qsa_pool_keys_prefill(x["k_idx"], self.k_pool, rope=self.rope,      # the cache's compressed keys
+                                      flags=self.kflags)
         self.ring = torch.zeros(B, 4, 128, dtype=dt, device=dev)
         del x["k_idx"]
         torch.cuda.empty_cache()
@@ -259,23 +279,37 @@ class DecodeRunner:
         x = x or self.x
         if events is not None:
             events[0].record()
-        qsa.qsa_pool_keys_decode(x["k_idx_new"], self.ring, self.k_pool, x["seq_len"], rope=self.rope,
-                                 flags=self.kflags)
+        if self.pt:
+            qsa.qsa_pool_keys_decode_paged(x["k_idx_new"], self.ring, self.k_pool, self.table, self.pt,
+                                           x["seq_len"], rope=self.rope, flags=self.kflags)
+        else:
+            qsa.qsa_pool_keys_decode(x["k_idx_new"], self.ring, self.k_pool, x["seq_len"], rope=self.rope,
+                                     flags=self.kflags)
         if events is not None:
             events[1].record()
-        qsa.qsa_index_topk_decode(x["q_idx"], self.k_pool, x["seq_len"], self.sel, self.nsel,
-                                  max_blocks=self.max_blocks, top_k=w.top_k, rope=self.rope, flags=self.kflags,
-                                  workspace=self.ws_i)
+        if self.pt:
+            qsa.qsa_index_topk_decode_paged(x["q_idx"], self.k_pool, self.table, self.pt, x["seq_len"], self.sel,
+                                            self.nsel, max_blocks=self.max_blocks, top_k=w.top_k, rope=self.rope,
+                                            flags=self.kflags, workspace=self.ws_i)
+        else:
+            qsa.qsa_index_topk_decode(x["q_idx"], self.k_pool, x["seq_len"], self.sel, self.nsel,
+                                      max_blocks=self.max_blocks, top_k=w.top_k, rope=self.rope, flags=self.kflags,
+                                      workspace=self.ws_i)
         if events is not None:
             events[2].record()
-        qsa.qsa_sparse_attn_decode(x["q"], x["k"], x["v"], x["seq_len"], self.sel, self.nsel, self.out,
-                                   workspace=self.ws_a)
+        if self.pt:
+            qsa.qsa_sparse_attn_decode_paged(x["q"], x["k"], x["v"], self.table, self.pt, x["seq_len"], self.sel,
+                                             self.nsel, self.out, workspace=self.ws_a)
+        else:
+            qsa.qsa_sparse_attn_decode(x["q"], x["k"], x["v"], x["seq_len"], self.sel, self.nsel, self.out,
+                                       workspace=self.ws_a)
         if events is not None:
             events[3].record()
         return self.out
 
     def launches_per_step(self):
-        return 5   # ring pool, decode scorer, select, attention, combine
+        # ring pool, the indexer (one fused kernel, or scorer + select), attention, combine
+        return 3 + self.qsa.qsa_index_topk_decode_kernels(self.w.B, self.max_blocks, self.kflags)
 
     def units(self):
         return self.w.B

@@ -23,12 +23,14 @@ __all__ = [
     "QSAError", "Rope", "lib", "LIB_PATH",
     "qsa_pool_keys_prefill", "qsa_pool_keys_decode",
     "qsa_index_topk_prefill", "qsa_index_topk_prefill_workspace",
-    "qsa_index_topk_decode", "qsa_index_topk_decode_workspace",
+    "qsa_index_topk_decode", "qsa_index_topk_decode_workspace", "qsa_index_topk_decode_kernels",
     "qsa_sparse_attn_prefill", "qsa_sparse_attn_decode", "qsa_sparse_attn_decode_workspace",
     "qsa_sparse_attn_decode_noalloc", "qsa_sparse_attn_decode_shared", "qsa_sparse_attn_decode_shared_workspace",
     "qsa_dense_attn_decode", "qsa_dense_attn_decode_workspace",
+    "qsa_pool_keys_prefill_paged", "qsa_pool_keys_decode_paged", "qsa_index_topk_decode_paged",
+    "qsa_sparse_attn_decode_paged",
     "qsa_rope_apply", "qsa_check_status", "qsa_strerror", "qsa_version",
-    "QSA_SCORE_RELU", "QSA_POOL_RMSNORM", "QSA_BF16", "QSA_FP32",
+    "QSA_SCORE_RELU", "QSA_POOL_RMSNORM", "QSA_KEYS_FP8", "QSA_BF16", "QSA_FP32",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libqsa.so")
@@ -42,6 +44,11 @@ class QSAError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
         super().__init__(f"{where}: {qsa_strerror(status)} (status {status})")
+
+
+class _Paging(ctypes.Structure):
+    _fields_ = [("page_table", ctypes.c_void_p), ("max_pages", ctypes.c_int64), ("num_pages", ctypes.c_int64),
+                ("page_tokens", ctypes.c_int32)]
 
 
 class _Rope(ctypes.Structure):
@@ -87,6 +94,7 @@ _sig("qsa_index_topk_prefill_workspace", _sz, _i32, _i64, _i64, _i32, _u32, _i32
 _sig("qsa_index_topk_prefill", ctypes.c_int, _vp, _vp, _vp, _i32, _i64, _i64, _i64, _i32, _vp, _vp, _vp, _sz,
      _Rope, _u32, _i32, _vp)
 _sig("qsa_index_topk_decode_workspace", _sz, _i32, _i64, _i32, _u32, _i32)
+_sig("qsa_index_topk_decode_kernels", ctypes.c_int, _i32, _i64, _u32, _i32)
 _sig("qsa_index_topk_decode", ctypes.c_int, _vp, _vp, _vp, _vp, _i32, _i64, _i64, _i32, _vp, _vp, _vp, _sz,
      _Rope, _u32, _i32, _vp)
 _sig("qsa_sparse_attn_prefill", ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i64, _i64, _i32, _i32, _i32,
@@ -101,6 +109,12 @@ _sig("qsa_dense_attn_decode_workspace", _sz, _i32, _i32, _i32, _i64, _i32)
 _sig("qsa_dense_attn_decode", ctypes.c_int, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32, _f32, _vp, _vp, _vp, _sz,
      _i32, _vp)
 _sig("qsa_rope_apply", ctypes.c_int, _vp, _i32, _i64, _i32, _i32, _i64, _Rope, _i32, _vp)
+_sig("qsa_pool_keys_prefill_paged", ctypes.c_int, _vp, _vp, _Paging, _i32, _i64, _i64, _i64, _Rope, _u32, _i32, _vp)
+_sig("qsa_pool_keys_decode_paged", ctypes.c_int, _vp, _vp, _vp, _Paging, _vp, _i32, _Rope, _u32, _i32, _vp)
+_sig("qsa_index_topk_decode_paged", ctypes.c_int, _vp, _vp, _Paging, _vp, _vp, _i32, _i64, _i32, _vp, _vp, _vp, _sz,
+     _Rope, _u32, _i32, _vp)
+_sig("qsa_sparse_attn_decode_paged", ctypes.c_int, _vp, _vp, _vp, _Paging, _vp, _vp, _vp, _i32, _i32, _i32, _i32,
+     _i32, _f32, _vp, _vp, _vp, _sz, _i32, _vp)
 _sig("qsa_sparse_attn_decode_noalloc", ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32,
      _i32, _f32, _vp, _vp, _i32, _vp)
 
@@ -208,6 +222,11 @@ def qsa_index_topk_prefill(q_idx, k_pool, sel, nsel, q0=0, top_k=512, head_w=Non
                                     _ptr(sel, torch.int32, "sel"), _ptr(nsel, torch.int32, "nsel"), wp, wb,
                                     rope.c(), flags, dt, _stream(q_idx, stream))
     _check(st, "qsa_index_topk_prefill")
+
+
+def qsa_index_topk_decode_kernels(B, max_blocks, flags=0, dtype=QSA_BF16) -> int:
+    """Kernels one qsa_index_topk_decode call launches (1 fused, 2 scorer + select)."""
+    return lib.qsa_index_topk_decode_kernels(B, max_blocks, flags, dtype)
 
 
 def qsa_index_topk_decode_workspace(B, max_blocks, top_k, flags=0, dtype=QSA_BF16) -> int:
@@ -328,6 +347,74 @@ def qsa_sparse_attn_decode_noalloc(q, k, v, seq_len, sel, nsel, out, top_k=None,
                                             _ptr(out, q.dtype, "out"), _ptr(lse, torch.float32, "lse"), dt,
                                             _stream(q, stream))
     _check(st, "qsa_sparse_attn_decode_noalloc")
+
+
+def _paging(page_table, num_pages, page_tokens):
+    """Paging descriptor: page_table [B][max_pages] int32 on the device."""
+    return _Paging(_ptr(page_table, torch.int32, "page_table"), page_table.shape[1], int(num_pages), int(page_tokens))
+
+
+def qsa_pool_keys_prefill_paged(k_raw, k_pool, page_table, page_tokens, pos0=0, rope=Rope(), flags=0, n_tok=None,
+                                stream=None):
+    """k_raw [B][S][128] -> rows slot(b, 4j) / 4 of the paged compressed-key cache
+    k_pool [num_pages * page_tokens / 4][128] for blocks j of positions pos0 .. pos0 + n_tok."""
+    dt = _dtype_code(k_raw)
+    B, S, D = k_raw.shape
+    assert D == 128 and k_pool.dim() == 2 and k_pool.shape[1] == 128
+    n_tok = S if n_tok is None else n_tok
+    pg = _paging(page_table, k_pool.shape[0] * 4 // page_tokens, page_tokens)
+    st = lib.qsa_pool_keys_prefill_paged(_ptr(k_raw, None, "k_raw"), _kpool_ptr(k_pool, k_raw.dtype, flags), pg, B,
+                                         n_tok, pos0, S, rope.c(), flags, dt, _stream(k_raw, stream))
+    _check(st, "qsa_pool_keys_prefill_paged")
+
+
+def qsa_pool_keys_decode_paged(k_new, ring, k_pool, page_table, page_tokens, seq_len, rope=Rope(), flags=0,
+                               stream=None):
+    dt = _dtype_code(k_new)
+    B = k_new.shape[0]
+    pg = _paging(page_table, k_pool.shape[0] * 4 // page_tokens, page_tokens)
+    st = lib.qsa_pool_keys_decode_paged(_ptr(k_new, None, "k_new"), _ptr(ring, k_new.dtype, "ring"),
+                                        _kpool_ptr(k_pool, k_new.dtype, flags), pg,
+                                        _ptr(seq_len, torch.int32, "seq_len"), B, rope.c(), flags, dt,
+                                        _stream(k_new, stream))
+    _check(st, "qsa_pool_keys_decode_paged")
+
+
+def qsa_index_topk_decode_paged(q_idx, k_pool, page_table, page_tokens, seq_len, sel, nsel, max_blocks=None,
+                                top_k=512, head_w=None, rope=Rope(), flags=0, workspace=None, stream=None):
+    """As qsa_index_topk_decode over the paged compressed-key cache k_pool
+    [num_pages * page_tokens / 4][128]."""
+    dt = _dtype_code(q_idx)
+    B = q_idx.shape[0]
+    max_blocks = page_table.shape[1] * page_tokens // 4 if max_blocks is None else max_blocks
+    need = qsa_index_topk_decode_workspace(B, max_blocks, top_k, flags, dt)
+    wp, wb = _ws(need, q_idx.device, workspace, zero=True)
+    pg = _paging(page_table, k_pool.shape[0] * 4 // page_tokens, page_tokens)
+    st = lib.qsa_index_topk_decode_paged(_ptr(q_idx, None, "q_idx"), _kpool_ptr(k_pool, q_idx.dtype, flags), pg,
+                                         _ptr(head_w, torch.float32, "head_w"), _ptr(seq_len, torch.int32, "seq_len"),
+                                         B, max_blocks, top_k, _ptr(sel, torch.int32, "sel"),
+                                         _ptr(nsel, torch.int32, "nsel"), wp, wb, rope.c(), flags, dt,
+                                         _stream(q_idx, stream))
+    _check(st, "qsa_index_topk_decode_paged")
+
+
+def qsa_sparse_attn_decode_paged(q, k, v, page_table, page_tokens, seq_len, sel, nsel, out, top_k=None, scale=None,
+                                 lse=None, workspace=None, stream=None):
+    """As qsa_sparse_attn_decode over paged K/V caches k, v [num_pages * page_tokens][Hkv][d]."""
+    dt = _dtype_code(q)
+    B, Hq, d = q.shape
+    Hkv = k.shape[1]
+    top_k = sel.shape[-1] if top_k is None else top_k
+    scale = (1.0 / d ** 0.5) if scale is None else scale
+    need = qsa_sparse_attn_decode_workspace(B, Hq, d, top_k, dt)
+    wp, wb = _ws(need, q.device, workspace)
+    pg = _paging(page_table, k.shape[0] // page_tokens, page_tokens)
+    st = lib.qsa_sparse_attn_decode_paged(_ptr(q, None, "q"), _ptr(k, q.dtype, "k"), _ptr(v, q.dtype, "v"), pg,
+                                          _ptr(seq_len, torch.int32, "seq_len"), _ptr(sel, torch.int32, "sel"),
+                                          _ptr(nsel, torch.int32, "nsel"), B, Hq, Hkv, d, top_k, scale,
+                                          _ptr(out, q.dtype, "out"), _ptr(lse, torch.float32, "lse"), wp, wb, dt,
+                                          _stream(q, stream))
+    _check(st, "qsa_sparse_attn_decode_paged")
 
 
 def qsa_rope_apply(x, pos0=0, rope=Rope(), stream=None):

@@ -39,6 +39,30 @@ __device__ __forceinline__ void flag(unsigned *status, unsigned bits) {
     if (status) atomicOr(status, bits);
 }
 
+// ---------------------------------------------------------------- paged caches
+// A paged cache holds token slots in pages of page_tokens slots; position pos
+// of sequence seq lives at slot table[seq][pos / page_tokens] * page_tokens +
+// pos % page_tokens.  The compressed-key cache is paged with the same table:
+// block b of a sequence is row slot(4b) / 4 (page_tokens is a multiple of 4,
+// so a block never straddles a page).  table == nullptr: contiguous caches.
+struct Paging {
+    const int32_t *table = nullptr;   // [B][max_pages] page ids
+    int64_t max_pages = 0;            // table row length
+    int64_t num_pages = 0;            // pages in the cache (valid ids are 0 .. num_pages - 1)
+    int page_tokens = 0;              // slots per page, a power of two
+    int page_shift = 0;               // log2(page_tokens)
+};
+
+// Slot of position pos of sequence seq, or -1 when its page id is outside
+// the cache (or its page index outside the table row).
+__device__ __forceinline__ int64_t paged_slot(const Paging &pg, int seq, int64_t pos) {
+    const int64_t pi = pos >> pg.page_shift;
+    if (pos < 0 || pi >= pg.max_pages) return -1;
+    const int32_t page = __ldg(pg.table + (int64_t)seq * pg.max_pages + pi);
+    if (page < 0 || page >= pg.num_pages) return -1;
+    return ((int64_t)page << pg.page_shift) + (pos & (pg.page_tokens - 1));
+}
+
 // ---------------------------------------------------------------- rounding
 
 // double -> bfloat16, round to nearest even, without double rounding:

@@ -61,12 +61,13 @@ const DeviceInfo *device_info();
 
 // ---- pooling / rotation (k_rope.cu)
 // fp8: the compressed keys are stored as FP8 E4M3 (bf16 raw keys only).
+// pg.table != nullptr: the compressed-key cache is paged (pool_stride unused).
 cudaError_t launch_pool_prefill(const void *k_raw, void *k_pool, int B, int64_t nblk, int64_t pos0,
                                 int64_t raw_stride, int64_t pool_stride, Rope rope, bool rmsnorm, bool bf16,
-                                bool fp8, cudaStream_t s);
+                                bool fp8, const Paging &pg, unsigned *status, cudaStream_t s);
 cudaError_t launch_pool_decode(const void *k_new, void *ring, void *k_pool, const int32_t *seq_len, int B,
-                               int64_t pool_stride, Rope rope, bool rmsnorm, bool bf16, bool fp8, unsigned *status,
-                               cudaStream_t s);
+                               int64_t pool_stride, Rope rope, bool rmsnorm, bool bf16, bool fp8, const Paging &pg,
+                               unsigned *status, cudaStream_t s);
 cudaError_t launch_rope_apply(void *x, int B, int64_t n, int H, int d, int64_t pos0, Rope rope, bool bf16,
                               cudaStream_t s);
 // Indexer queries for prefill: mode 0 -> hi/lo bf16 planes of the head sum
@@ -103,10 +104,12 @@ struct DecodePlan {
 };
 DecodePlan decode_index_plan(int B, int64_t max_blocks, bool bf16);
 size_t decode_index_ws_bytes(int B, int64_t max_blocks, int top_k, bool bf16);
+// Kernels one decode-index call launches: 1 (fused scorer-select) or 2 (scorer, select).
+int decode_index_kernel_count(int B, int64_t max_blocks, bool bf16, bool fp8);
 cudaError_t launch_decode_index(const void *q_idx, const void *k_pool, const float *head_w,
                                 const int32_t *seq_len, int B, int64_t pool_stride, int64_t max_blocks,
                                 int top_k, int32_t *sel, int32_t *nsel, void *ws, Rope rope, bool relu,
-                                bool bf16, bool fp8, unsigned *status, cudaStream_t s);
+                                bool bf16, bool fp8, const Paging &pg, unsigned *status, cudaStream_t s);
 
 // ---- sparse attention (k_attn.cu)
 struct AttnArgs {
@@ -123,6 +126,7 @@ struct AttnArgs {
     const int32_t *cap_len = nullptr;   // decode, IndexShare draft step: [B] capture rows + 1
     int max_draft = 0;                  // IndexShare: largest seq_len - cap_len
     bool dense = false;                 // decode: dense causal attention over every position (no selection)
+    Paging pg;                          // pg.table: paged K/V caches (bf16 kernels), kv_stride = its capacity
 };
 int attn_tail_blocks(bool indexshare, int max_draft);
 size_t attn_decode_ws_bytes(int B, int Hq, int d, int top_k, int tail_blocks = 1);

@@ -106,6 +106,7 @@ struct AttnParams {
     int max_draft;           // IndexShare: largest seq_len - cap_len
     int dense;               // decode: every visible block in order (dense causal attention, no selection)
     unsigned *status;
+    Paging pg;               // pg.table: K/V are paged caches [slots][Hkv][128] (kv_stride = table capacity)
 };
 
 // The key list of one work item: positions lbeg..lend of
@@ -191,7 +192,9 @@ size_t attn_smem_bytes(int sel_cap, int nst_cap) {
     return sizeof(AttnSmem<HKV>) + (size_t)sel_cap * 4 + 2 * (size_t)AttnCfg<HKV>::kPw * nst_cap * 4 + 128;
 }
 
-template <int HKV>
+// PAGED: K/V are paged caches addressed through p.pg (a separate instantiation,
+// so the contiguous kernels carry none of the page-table code).
+template <int HKV, bool PAGED>
 __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, AttnCfg<HKV>::kMinCtas) attn_bf16_kernel(AttnParams p) {
     using Cfg = AttnCfg<HKV>;
     extern __shared__ uint8_t asm_raw[];
@@ -245,12 +248,18 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, AttnCfg<HKV>::kMinCtas
                     const int e = it.lbeg + AT_BPS * st + j;
                     int tokens = 0;
                     if (e < it.lend) {
+                        int64_t blk = it.nb + (e - it.nsel);
                         if (e < it.nsel) {
                             const int b = ids[e - it.lbeg];
+                            blk = b;
                             if (b >= 0 && b < it.nb) tokens = kBlock;
                             else flag(p.status, QSA_DEV_BAD_INDEX);
                         } else {
                             tokens = min(kBlock, it.tail - kBlock * (e - it.nsel));
+                        }
+                        if (PAGED && tokens > 0 && paged_slot(p.pg, it.seq, blk * kBlock) < 0) {
+                            tokens = 0;   // a page outside the cache: skipped, flagged
+                            flag(p.status, QSA_DEV_BAD_INDEX);
                         }
                     }
                     info |= (uint32_t)tokens << (3 * j);
@@ -281,8 +290,12 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, AttnCfg<HKV>::kMinCtas
                     for (int jj = 0; jj < kSlotsPerPw; ++jj) {
                         const int j = Cfg::kPw * jj + pw;
                         const int e = it.lbeg + AT_BPS * st + j;
-                        const int tokens = e >= it.lend ? 0
-                                           : (e < it.nsel ? kBlock : min(kBlock, it.tail - kBlock * (e - it.nsel)));
+                        int tokens = e >= it.lend ? 0
+                                     : (e < it.nsel ? kBlock : min(kBlock, it.tail - kBlock * (e - it.nsel)));
+                        if (PAGED && tokens > 0 && paged_slot(p.pg, it.seq, (int64_t)e * kBlock) < 0) {
+                            tokens = 0;   // a page outside the cache: skipped, flagged
+                            flag(p.status, QSA_DEV_BAD_INDEX);
+                        }
                         sinfo |= (uint32_t)tokens << (3 * j);
                         sbytes += (uint32_t)tokens * HKV * 256u;
                     }
@@ -301,7 +314,8 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, AttnCfg<HKV>::kMinCtas
                     if (tokens > 0) {
                         const int64_t blk = (e < it.nsel) ? (p.dense ? (int64_t)e : (int64_t)ids[e - it.lbeg])
                                                           : it.nb + (e - it.nsel);
-                        const int64_t off = (kv0 + blk * kBlock) * HKV * 128;
+                        const int64_t tok = PAGED ? paged_slot(p.pg, it.seq, blk * kBlock) : kv0 + blk * kBlock;
+                        const int64_t off = tok * HKV * 128;
                         const uint32_t nbytes = (uint32_t)tokens * HKV * 256u;
                         bulk_g2s(sm.stage[s] + j * Cfg::kSlot, p.k + off, nbytes, &sm.full[s]);
                         bulk_g2s(sm.stage[s] + (AT_BPS + j) * Cfg::kSlot, p.v + off, nbytes, &sm.full[s]);
@@ -775,6 +789,7 @@ cudaError_t run_bf16(const AttnArgs &a, void *ws, unsigned *status, cudaStream_t
     p.cap_len = a.decode ? a.cap_len : nullptr;
     p.max_draft = a.max_draft;
     p.dense = a.decode && a.dense ? 1 : 0;
+    p.pg = a.pg;
     // entries of one item's list: top_k blocks + the tail blocks (dense: every block of the cache)
     const int list_max = p.dense ? (int)(a.kv_stride / kBlock + 1)
                                  : a.top_k + attn_tail_blocks(a.decode && a.cap_len, a.max_draft);
@@ -798,13 +813,14 @@ cudaError_t run_bf16(const AttnArgs &a, void *ws, unsigned *status, cudaStream_t
     p.nst_cap = p.dense ? 1 : (list_max + AT_BPS - 1) / AT_BPS;
     const size_t smem = attn_smem_bytes<HKV>(p.sel_cap, p.nst_cap);
     if (di && smem > di->smem_optin) return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(attn_bf16_kernel<HKV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto kern = p.pg.table ? attn_bf16_kernel<HKV, true> : attn_bf16_kernel<HKV, false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, attn_bf16_kernel<HKV>, Cfg::kThreads, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, Cfg::kThreads, smem);
     if (e != cudaSuccess) return e;
     const int64_t grid = std::min<int64_t>(p.items, (int64_t)sms * std::max(1, per_sm));
-    e = launch_pdl(attn_bf16_kernel<HKV>, dim3((unsigned)grid), dim3(Cfg::kThreads), smem, s, p);
+    e = launch_pdl(kern, dim3((unsigned)grid), dim3(Cfg::kThreads), smem, s, p);
     if (e != cudaSuccess || !a.decode) return e;
     return launch_pdl(attn_combine_kernel, dim3((unsigned)(a.B * Cfg::kHq)), dim3(128), 0, s,
                       (const float *)p.part_o, (const float *)p.part_lse, p.splits, (int)Cfg::kHq,

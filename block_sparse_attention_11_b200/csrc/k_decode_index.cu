@@ -29,12 +29,45 @@ constexpr int DI_STAGE_BYTES = 16384;
 struct DecodeParams {
     const int32_t *seq_len;
     const float *head_w;
-    int64_t pool_stride, max_blocks, chunk, kstride;
+    int64_t pool_stride, max_blocks, chunk, kstride;   // paged: pool_stride = max_pages * page_tokens / 4
     int chunks, top_k, relu;
     uint32_t *keys;      // [B][kstride] score keys
     uint32_t *hist;      // [B][2048] histogram of the keys' top 11 bits
     unsigned *status;
+    Paging pg;           // pg.table: the compressed keys are paged (rows slot / 4)
 };
+
+// Bulk copy of rows [lr0, lr0 + rows) of sequence seq's compressed keys
+// (row_bytes each) into dst, completing on bar: one copy when contiguous, one
+// per page run when paged.  Returns the bytes issued (rows of a page outside
+// the cache are skipped and flagged), to be posted with expect_tx first: call
+// once with issue = false to count, then with issue = true.
+__device__ __forceinline__ uint32_t copy_key_rows(const DecodeParams &p, const uint8_t *k_pool, int seq,
+                                                  int64_t lr0, int rows, int row_bytes, uint8_t *dst, uint64_t *bar,
+                                                  bool issue) {
+    if (!p.pg.table) {
+        if (issue)
+            bulk_g2s(dst, k_pool + ((int64_t)seq * p.pool_stride + lr0) * row_bytes, (uint32_t)(rows * row_bytes),
+                     bar);
+        return (uint32_t)(rows * row_bytes);
+    }
+    const int page_rows = p.pg.page_tokens / kBlock;
+    uint32_t bytes = 0;
+    for (int r = 0; r < rows;) {
+        const int64_t lr = lr0 + r;
+        const int run = min(rows - r, page_rows - (int)(lr & (page_rows - 1)));
+        const int64_t slot = paged_slot(p.pg, seq, lr * kBlock);
+        if (slot >= 0) {
+            if (issue) bulk_g2s(dst + (int64_t)r * row_bytes, k_pool + (slot / kBlock) * row_bytes,
+                                (uint32_t)(run * row_bytes), bar);
+            bytes += (uint32_t)(run * row_bytes);
+        } else if (!issue) {
+            flag(p.status, QSA_DEV_BAD_INDEX);
+        }
+        r += run;
+    }
+    return bytes;
+}
 
 // Adds a CTA's local histogram (smem, 2048 bins) into the sequence's global one.
 __device__ __forceinline__ void flush_hist(const uint32_t *lh, uint32_t *gh) {
@@ -73,7 +106,7 @@ __global__ void __launch_bounds__(DI_THREADS, 2)
     if (n == 0) return;
     uint32_t *gkeys = p.keys + (int64_t)seq * p.kstride + c0;
     const int nstages = (n + SROWS - 1) / SROWS;
-    const T *kbase = k_pool + ((int64_t)seq * p.pool_stride + c0) * kIdxDim;
+    const uint8_t *kbytes = reinterpret_cast<const uint8_t *>(k_pool);
     for (int b = tid; b < 2048; b += blockDim.x) lh[b] = 0;
     if (tid == 0) {
         for (int s = 0; s < DI_NS; ++s) mbar_init(&full[s], 1);
@@ -83,8 +116,10 @@ __global__ void __launch_bounds__(DI_THREADS, 2)
     if (tid == 0) {
         for (int st = 0; st < min(DI_NS, nstages); ++st) {
             const int rows = min(SROWS, n - st * SROWS);
-            mbar_arrive_expect_tx(&full[st], rows * ROW_BYTES);
-            bulk_g2s(stage + st * DI_STAGE_BYTES, kbase + (int64_t)st * SROWS * kIdxDim, rows * ROW_BYTES, &full[st]);
+            const int64_t lr = c0 + (int64_t)st * SROWS;
+            uint8_t *dst = stage + st * DI_STAGE_BYTES;
+            mbar_arrive_expect_tx(&full[st], copy_key_rows(p, kbytes, seq, lr, rows, ROW_BYTES, dst, &full[st], false));
+            copy_key_rows(p, kbytes, seq, lr, rows, ROW_BYTES, dst, &full[st], true);
         }
     }
     // rotated query heads of the new token (position s_len - 1), rounded to T
@@ -179,9 +214,11 @@ __global__ void __launch_bounds__(DI_THREADS, 2)
         if (tid == 0 && st + DI_NS < nstages) {
             const int st2 = st + DI_NS;
             const int rows2 = min(SROWS, n - st2 * SROWS);
-            mbar_arrive_expect_tx(&full[slot], rows2 * ROW_BYTES);
-            bulk_g2s(stage + slot * DI_STAGE_BYTES, kbase + (int64_t)st2 * SROWS * kIdxDim, rows2 * ROW_BYTES,
-                     &full[slot]);
+            const int64_t lr = c0 + (int64_t)st2 * SROWS;
+            uint8_t *dst = stage + slot * DI_STAGE_BYTES;
+            mbar_arrive_expect_tx(&full[slot],
+                                  copy_key_rows(p, kbytes, seq, lr, rows2, ROW_BYTES, dst, &full[slot], false));
+            copy_key_rows(p, kbytes, seq, lr, rows2, ROW_BYTES, dst, &full[slot], true);
         }
     }
     __syncthreads();
@@ -200,13 +237,14 @@ constexpr int DM_STAGE_BYTES = DM_ROWS * 256;      // two 64-dim k-atoms of 128 
 // FP8 E4M3 compressed keys: a stage is one 128-byte-swizzled box of 128 rows x
 // 128 B, the A operand of m16n8k32 E4M3 MMAs as it lands.
 constexpr int DM_STAGE_BYTES_FP8 = DM_ROWS * 128;
+constexpr int DM_PG_IDS = 1024;                    // paged: page ids a scorer CTA keeps (bounds its chunk)
 template <bool FP8> __host__ __device__ constexpr int stage_bytes() { return FP8 ? DM_STAGE_BYTES_FP8 : DM_STAGE_BYTES; }
 
 using EncodeTiledFn = decltype(&cuTensorMapEncodeTiled);
 
 // 2-D map over the compressed keys [rows][128]: bf16 in 64 x 128 boxes, or
 // FP8 E4M3 (as bytes) in 128 x 128 boxes; 128-byte swizzle.
-bool make_kpool_map(CUtensorMap *map, const void *base, uint64_t rows, bool fp8 = false) {
+bool make_kpool_map(CUtensorMap *map, const void *base, uint64_t rows, bool fp8 = false, int box_rows = DM_ROWS) {
     static EncodeTiledFn fn = nullptr;
     if (!fn) {
         void *ptr = nullptr;
@@ -218,7 +256,7 @@ bool make_kpool_map(CUtensorMap *map, const void *base, uint64_t rows, bool fp8 
     }
     cuuint64_t dims[2] = {128, rows};
     cuuint64_t strides[1] = {fp8 ? 128u : 128u * 2};
-    cuuint32_t box[2] = {fp8 ? 128u : 64u, (cuuint32_t)DM_ROWS};
+    cuuint32_t box[2] = {fp8 ? 128u : 64u, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
     return fn(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base),
               dims, strides, box, estr,
@@ -232,11 +270,11 @@ bool make_kpool_map(CUtensorMap *map, const void *base, uint64_t rows, bool fp8 
 // warps; group g consumes (and refills) the stages st = g mod NT / 256, each
 // warp scoring 16 rows of a 128-row stage.  Returns false after a timed-out
 // wait, once the copies still in flight have landed (or their waits ran out).
-template <int NS, bool FP8, int NT, typename Smem, typename Sink>
+template <int NS, bool FP8, int NT, bool PAGED, typename Smem, typename Sink>
 __device__ __forceinline__ bool stream_scores(Smem &sm, const CUtensorMap *kmap,
                                               const __nv_bfloat16 *__restrict__ q_idx, const Rope &rope,
                                               const DecodeParams &p, int seq, int64_t s_len, int n, int y0,
-                                              Sink &&sink) {
+                                              int64_t c0, Sink &&sink) {
     constexpr int G = NT / 256;
     static_assert(NT % 256 == 0 && NS % G == 0, "whole groups; each slot stays with one group");
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -244,13 +282,60 @@ __device__ __forceinline__ bool stream_scores(Smem &sm, const CUtensorMap *kmap,
     const bool leader = (tid & 255) == 0;
     const int nstages = (n + DM_ROWS - 1) / DM_ROWS;
     constexpr int SB = stage_bytes<FP8>();
-    auto issue = [&](int slot, int st2) {
+    const int pr = PAGED ? p.pg.page_tokens / kBlock : 1;   // rows per page (a power of two)
+    const int pshift = PAGED ? p.pg.page_shift - 2 : 0;      // log2(pr)
+    const int64_t pg_first = PAGED ? c0 >> pshift : 0;       // the chunk's first page index
+    auto issue = [&](int slot, int st2) {   // contiguous: rows y0 + 128 st2 .. as one box (per 64-dim atom)
         mbar_arrive_expect_tx(&sm.full[slot], SB);
         tma_load_2d(sm.stage[slot], kmap, 0, y0 + st2 * DM_ROWS, &sm.full[slot]);
         if constexpr (!FP8) tma_load_2d(sm.stage[slot] + SB / 2, kmap, 64, y0 + st2 * DM_ROWS, &sm.full[slot]);
     };
-    if (tid == 0)
+    // Paged stages are issued by a whole warp: lane ch copies box ch of the
+    // stage (cr rows: a page, or 128 rows of one) from its page, so the up to
+    // 16 boxes of a stage of small pages go out in parallel; boxes past the
+    // chunk's keys are skipped.
+    auto issue_paged = [&](int slot, int st2) {
+        const int cr = min(DM_ROWS, pr);
+        const int ch = lane;
+        bool live = ch * cr < DM_ROWS && st2 * DM_ROWS + ch * cr < n;
+        int y = 0;
+        if (live) {
+            const int64_t lr = c0 + (int64_t)st2 * DM_ROWS + ch * cr;
+            const int32_t id = sm.pg_ids[(lr >> pshift) - pg_first];
+            if (id < 0) {
+                flag(p.status, QSA_DEV_BAD_INDEX);
+                live = false;
+            }
+            y = (int)(((int64_t)id << pshift) + (lr & (pr - 1)));
+        }
+        const uint32_t bytes = __reduce_add_sync(0xffffffffu, live ? (uint32_t)cr * (SB / DM_ROWS) : 0u);
+        if (lane == 0) mbar_arrive_expect_tx(&sm.full[slot], bytes);
+        __syncwarp();
+        if (live) {
+            tma_load_2d(sm.stage[slot] + ch * cr * 128, kmap, 0, y, &sm.full[slot]);
+            if constexpr (!FP8) tma_load_2d(sm.stage[slot] + SB / 2 + ch * cr * 128, kmap, 64, y, &sm.full[slot]);
+        }
+    };
+    if constexpr (PAGED) {
+        // the page ids of the chunk's rows, once, into shared memory (-1: outside the cache)
+        const int cnt = (int)(((c0 + n + pr - 1) >> pshift) - pg_first);   // <= the window by the launch plan
+        for (int i = tid; i < cnt; i += NT) {
+            const int64_t pi = pg_first + i;
+            int32_t id = -1;
+            if (pi < p.pg.max_pages) {
+                id = p.pg.table[(int64_t)seq * p.pg.max_pages + pi];
+                if (id < 0 || id >= p.pg.num_pages) id = -1;
+            }
+            sm.pg_ids[i] = id;
+        }
+        __syncthreads();
+    }
+    if constexpr (PAGED) {
+        if (tid < 32)
+            for (int st = 0; st < min(NS, nstages); ++st) issue_paged(st, st);
+    } else if (tid == 0) {
         for (int st = 0; st < min(NS, nstages); ++st) issue(st, st);
+    }
     const bool per_head = p.relu || p.head_w;
     // Rotated query heads of the new token (position s_len - 1), rounded to
     // bf16, as the B operand's columns.  BF16 keys: hi/lo bf16 planes of the
@@ -433,7 +518,16 @@ __device__ __forceinline__ bool stream_scores(Smem &sm, const CUtensorMap *kmap,
                 atomicAdd(&sm.lh[key >> 21], 1u);
             }
         }
-        if (leader && st + NS < nstages) {
+        if constexpr (PAGED) {
+            if (gw == 0 && st + NS < nstages) {   // the group's first warp refills the slot
+                bool okw = true;
+                if (lane == 0) okw = ok = mbar_wait(&sm.empty[slot], (st / NS) & 1, p.status);
+                if (__shfl_sync(0xffffffffu, okw, 0)) {
+                    issue_paged(slot, st + NS);
+                    issued = st + NS + 1;
+                }
+            }
+        } else if (leader && st + NS < nstages) {
             ok = mbar_wait(&sm.empty[slot], (st / NS) & 1, p.status);
             if (ok) {
                 issue(slot, st + NS);
@@ -458,11 +552,12 @@ struct DecodeMmaSmem {
     float qred[4];                                 // FP8: per-warp largest query magnitude
     uint64_t full[NS], empty[NS];
     uint32_t lh[2048];                             // local histogram of the keys' top 11 bits
+    int32_t pg_ids[DM_PG_IDS];                     // paged: page ids of the chunk's rows
 };
 
 // Scorer of the two-kernel path: keys to the workspace, histogram added into
-// the sequence's global histogram.
-template <bool FP8>
+// the sequence's global histogram.  PAGED: paged compressed keys (p.pg).
+template <bool FP8, bool PAGED>
 __global__ void __launch_bounds__(DI_THREADS, 2)
     decode_score_mma_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16 *__restrict__ q_idx,
                             Rope rope, DecodeParams p) {
@@ -494,8 +589,8 @@ __global__ void __launch_bounds__(DI_THREADS, 2)
         prefetch_tmap(&kmap);
     }
     __syncthreads();
-    const bool ok = stream_scores<DecodeMmaSmem<FP8>::NS, FP8, DI_THREADS>(sm, &kmap, q_idx, rope, p, seq, s_len, n,
-                                              (int)(seq * p.pool_stride + c0),
+    const bool ok = stream_scores<DecodeMmaSmem<FP8>::NS, FP8, DI_THREADS, PAGED>(sm, &kmap, q_idx, rope, p, seq, s_len, n,
+                                              (int)(seq * p.pool_stride + c0), c0,
                                          [&](int r, uint32_t key) { gkeys[r] = key; });
     if (!ok) return;
     flush_hist(sm.lh, p.hist + (int64_t)seq * 2048);
@@ -875,6 +970,7 @@ struct FusedSmem {
     float w[kIdxHeads];
     float qred[4];
     uint64_t full[fused_stages<FP8>()], empty[fused_stages<FP8>()];
+    int32_t pg_ids[DF_KEYS / 8];                // paged: page ids of the chunk's rows (pages of >= 8 rows)
 };
 // The streaming interface of FusedSmem (stage, qcol, w, qred, full, empty, lh).
 template <bool FP8>
@@ -886,9 +982,10 @@ struct FusedStream {
     uint64_t (&full)[fused_stages<FP8>()];
     uint64_t (&empty)[fused_stages<FP8>()];
     uint32_t (&lh)[2048];
+    int32_t (&pg_ids)[DF_KEYS / 8];
 };
 
-template <bool FP8>
+template <bool FP8, bool PAGED>
 __global__ void __launch_bounds__(DF_THREADS, 1)
     decode_index_fused_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16 *__restrict__ q_idx,
                               Rope rope, DecodeParams p, SelectArgs a) {
@@ -926,8 +1023,9 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
     __syncthreads();
     bool ok = true;
     if (n > 0) {
-        FusedStream<FP8> fs{sm.u.st.stage, sm.qcol, sm.w, sm.qred, sm.full, sm.empty, sm.lh};
-        ok = stream_scores<fused_stages<FP8>(), FP8, DF_THREADS>(fs, &kmap, q_idx, rope, p, seq, s_len, n, (int)(seq * p.pool_stride + c0),
+        FusedStream<FP8> fs{sm.u.st.stage, sm.qcol, sm.w, sm.qred, sm.full, sm.empty, sm.lh, sm.pg_ids};
+        ok = stream_scores<fused_stages<FP8>(), FP8, DF_THREADS, PAGED>(fs, &kmap, q_idx, rope, p, seq, s_len, n,
+                                                                 (int)(seq * p.pool_stride + c0), c0,
                                   [&](int r, uint32_t key) { sm.skeys[r] = key; });
     }
     (void)ok;   // a timed-out wait is in the status word; the cluster still runs every barrier
@@ -1058,9 +1156,9 @@ int fused_active_clusters(int C) {
     if (ok[C] < 0) {
         ok[C] = 0;
         const size_t smem = sizeof(FusedSmem<FP8>) + 1024;
-        if (cudaFuncSetAttribute(decode_index_fused_kernel<FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(decode_index_fused_kernel<FP8, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)smem) == cudaSuccess &&
-            (C <= 8 || cudaFuncSetAttribute(decode_index_fused_kernel<FP8>,
+            (C <= 8 || cudaFuncSetAttribute(decode_index_fused_kernel<FP8, false>,
                                             cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess)) {
             cudaLaunchConfig_t cfg = {};
             cfg.gridDim = dim3((unsigned)C, 1, 1);
@@ -1074,7 +1172,7 @@ int fused_active_clusters(int C) {
             cfg.attrs = attr;
             cfg.numAttrs = 1;
             int n = 0;
-            if (cudaOccupancyMaxActiveClusters(&n, decode_index_fused_kernel<FP8>, &cfg) == cudaSuccess && n > 0)
+            if (cudaOccupancyMaxActiveClusters(&n, decode_index_fused_kernel<FP8, false>, &cfg) == cudaSuccess && n > 0)
                 ok[C] = n;
         }
         cudaGetLastError();   // a refused query leaves no sticky error
@@ -1129,6 +1227,10 @@ DecodeWs decode_ws(void *base, int B, int64_t max_blocks, int top_k) {
 }
 }  // namespace
 
+int decode_index_kernel_count(int B, int64_t max_blocks, bool bf16, bool fp8) {
+    return fused_plan(B, std::max<int64_t>(max_blocks, 1), bf16, fp8).use ? 1 : 2;
+}
+
 size_t decode_index_ws_bytes(int B, int64_t max_blocks, int top_k, bool bf16) {
     (void)bf16;
     return decode_ws(nullptr, B, max_blocks, top_k).total;
@@ -1137,19 +1239,24 @@ size_t decode_index_ws_bytes(int B, int64_t max_blocks, int top_k, bool bf16) {
 cudaError_t launch_decode_index(const void *q_idx, const void *k_pool, const float *head_w,
                                 const int32_t *seq_len, int B, int64_t pool_stride, int64_t max_blocks,
                                 int top_k, int32_t *sel, int32_t *nsel, void *ws, Rope rope, bool relu,
-                                bool bf16, bool fp8, unsigned *status, cudaStream_t s) {
+                                bool bf16, bool fp8, const Paging &pg, unsigned *status, cudaStream_t s) {
     if (fp8 && !bf16) return cudaErrorInvalidValue;
     const int64_t kstride = key_stride(max_blocks);
     const DecodeWs d = decode_ws(ws, B, max_blocks, top_k);
     const FusedPlan fp = fused_plan(B, max_blocks, bf16, fp8);
+    // the compressed keys as one 2-D tensor: B * pool_stride rows, or the paged
+    // cache's num_pages * page_tokens / 4 rows read in boxes of one page (<= 128 rows)
+    const uint64_t map_rows = pg.table ? (uint64_t)pg.num_pages * (pg.page_tokens / kBlock) : (uint64_t)B * pool_stride;
+    const int box_rows = pg.table ? std::min(DM_ROWS, pg.page_tokens / kBlock) : DM_ROWS;
     if (fp.use) {
         CUtensorMap kmap;
-        if (!make_kpool_map(&kmap, k_pool, (uint64_t)B * pool_stride, fp8)) return cudaErrorInvalidValue;
+        if (!make_kpool_map(&kmap, k_pool, map_rows, fp8, box_rows)) return cudaErrorInvalidValue;
         DecodeParams p{seq_len, head_w, pool_stride, max_blocks, fp.chunk, kstride, fp.C, top_k, relu ? 1 : 0,
-                       d.keys, d.hist, status};
+                       d.keys, d.hist, status, pg};
         SelectArgs sa{seq_len, pool_stride, max_blocks, kstride, fp.chunk, fp.C, top_k, d.keys, d.hist, d.cand,
                       sel, nsel, status};
-        auto kern = fp8 ? decode_index_fused_kernel<true> : decode_index_fused_kernel<false>;
+        auto kern = fp8 ? (pg.table ? decode_index_fused_kernel<true, true> : decode_index_fused_kernel<true, false>)
+                        : (pg.table ? decode_index_fused_kernel<false, true> : decode_index_fused_kernel<false, false>);
         const size_t smem = (fp8 ? sizeof(FusedSmem<true>) : sizeof(FusedSmem<false>)) + 1024;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
@@ -1160,15 +1267,24 @@ cudaError_t launch_decode_index(const void *q_idx, const void *k_pool, const flo
         return launch_pdl_cluster(kern, dim3((unsigned)fp.C, (unsigned)B), dim3(DF_THREADS), smem, (unsigned)fp.C, s,
                                   kmap, (const __nv_bfloat16 *)q_idx, rope, p, sa);
     }
-    const DecodePlan pl = decode_index_plan(B, max_blocks, bf16);
+    DecodePlan pl = decode_index_plan(B, max_blocks, bf16);
+    if (pg.table) {   // a scorer CTA keeps the page ids of its chunk: at most DM_PG_IDS pages
+        const int64_t pr = pg.page_tokens / kBlock;
+        const int64_t cap = std::max<int64_t>(DM_ROWS, (DM_PG_IDS - 2) * pr / DM_ROWS * DM_ROWS);
+        if (pl.chunk > cap) {
+            pl.chunk = cap;
+            pl.chunks = (int)((max_blocks + cap - 1) / cap);
+        }
+    }
     cudaError_t e;
     DecodeParams p{seq_len, head_w, pool_stride, max_blocks, pl.chunk, kstride, pl.chunks, top_k, relu ? 1 : 0,
-                   d.keys, d.hist, status};
+                   d.keys, d.hist, status, pg};
     dim3 grid((unsigned)pl.chunks, (unsigned)B);
     if (bf16) {
         CUtensorMap kmap;
-        if (!make_kpool_map(&kmap, k_pool, (uint64_t)B * pool_stride, fp8)) return cudaErrorInvalidValue;
-        auto kern = fp8 ? decode_score_mma_kernel<true> : decode_score_mma_kernel<false>;
+        if (!make_kpool_map(&kmap, k_pool, map_rows, fp8, box_rows)) return cudaErrorInvalidValue;
+        auto kern = fp8 ? (pg.table ? decode_score_mma_kernel<true, true> : decode_score_mma_kernel<true, false>)
+                        : (pg.table ? decode_score_mma_kernel<false, true> : decode_score_mma_kernel<false, false>);
         const size_t smem = (fp8 ? sizeof(DecodeMmaSmem<true>) : sizeof(DecodeMmaSmem<false>)) + 1024;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;

@@ -84,7 +84,8 @@ __device__ __forceinline__ void store16_e4m3(uint8_t *dst, const double (&v)[16]
 template <typename T, bool FP8 = false>
 __global__ void __launch_bounds__(256) pool_prefill_kernel(const T *__restrict__ k_raw, void *__restrict__ k_pool_v,
                                                            int64_t nblk, int64_t pos0, int64_t raw_stride,
-                                                           int64_t pool_stride, Rope rope, int rmsnorm) {
+                                                           int64_t pool_stride, Rope rope, int rmsnorm, Paging pg,
+                                                           unsigned *status) {
     __shared__ float mean_s[32][kIdxDim];
     const int seq = blockIdx.y;
     const int kl = threadIdx.x >> 3;    // key within CTA
@@ -139,7 +140,15 @@ __global__ void __launch_bounds__(256) pool_prefill_kernel(const T *__restrict__
             out[i] = xe;
         }
     }
-    const int64_t row = (int64_t)seq * pool_stride + pos0 / kBlock + blk;
+    int64_t row = (int64_t)seq * pool_stride + pos0 / kBlock + blk;
+    if (pg.table) {   // paged: the row of the block's first token slot
+        const int64_t slot = paged_slot(pg, seq, pos0 + blk * kBlock);
+        if (slot < 0) {
+            if (j == 0) flag(status, QSA_DEV_BAD_INDEX);
+            return;
+        }
+        row = slot / kBlock;
+    }
     if constexpr (FP8) {
         store16_e4m3(static_cast<uint8_t *>(k_pool_v) + row * kIdxDim + 16 * j, out);
     } else {
@@ -153,7 +162,7 @@ template <typename T, bool FP8 = false>
 __global__ void __launch_bounds__(128) pool_decode_kernel(const T *__restrict__ k_new, T *__restrict__ ring,
                                                           void *__restrict__ k_pool_v,
                                                           const int32_t *__restrict__ seq_len, int64_t pool_stride,
-                                                          Rope rope, int rmsnorm, unsigned *status) {
+                                                          Rope rope, int rmsnorm, Paging pg, unsigned *status) {
     __shared__ double out_s[kIdxDim];
     __shared__ float mean_s[kIdxDim];
     __shared__ double red[4];
@@ -172,7 +181,15 @@ __global__ void __launch_bounds__(128) pool_decode_kernel(const T *__restrict__ 
     rg[(p % kBlock) * kIdxDim + e] = knew;
     if (s % kBlock != 0) return;
     const int64_t b = s / kBlock - 1;
-    if (b >= pool_stride) {
+    int64_t row = (int64_t)seq * pool_stride + b;
+    if (pg.table) {   // paged: the row of the block's first token slot
+        const int64_t slot = paged_slot(pg, seq, b * kBlock);
+        if (slot < 0) {
+            if (e == 0) flag(status, QSA_DEV_BAD_INDEX);
+            return;
+        }
+        row = slot / kBlock;
+    } else if (b >= pool_stride) {
         if (e == 0) flag(status, QSA_DEV_BAD_LENGTH);
         return;
     }
@@ -203,7 +220,6 @@ __global__ void __launch_bounds__(128) pool_decode_kernel(const T *__restrict__ 
         rope_cs(rope, (double)(s - kBlock), e < half ? e : e - half, c, sn);
         out = rope_dim(xe, xp, e, half, c, sn);
     }
-    const int64_t row = (int64_t)seq * pool_stride + b;
     if constexpr (FP8) {   // pairs of dims -> one 16-bit store
         out_s[e] = out;
         __syncthreads();
@@ -282,35 +298,36 @@ __global__ void __launch_bounds__(128) rotate_index_q_kernel(const T *__restrict
 
 cudaError_t launch_pool_prefill(const void *k_raw, void *k_pool, int B, int64_t nblk, int64_t pos0,
                                 int64_t raw_stride, int64_t pool_stride, Rope rope, bool rmsnorm, bool bf16,
-                                bool fp8, cudaStream_t s) {
+                                bool fp8, const Paging &pg, unsigned *status, cudaStream_t s) {
     if (nblk <= 0) return cudaSuccess;
     dim3 grid((unsigned)((nblk + 31) / 32), (unsigned)B);
+    const int rn = rmsnorm ? 1 : 0;
     if (bf16 && fp8)
         pool_prefill_kernel<__nv_bfloat16, true><<<grid, 256, 0, s>>>(
-            (const __nv_bfloat16 *)k_raw, k_pool, nblk, pos0, raw_stride, pool_stride, rope, rmsnorm);
+            (const __nv_bfloat16 *)k_raw, k_pool, nblk, pos0, raw_stride, pool_stride, rope, rn, pg, status);
     else if (bf16)
         pool_prefill_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>((const __nv_bfloat16 *)k_raw, k_pool, nblk, pos0,
-                                                                raw_stride, pool_stride, rope, rmsnorm);
+                                                                raw_stride, pool_stride, rope, rn, pg, status);
     else
         pool_prefill_kernel<float><<<grid, 256, 0, s>>>((const float *)k_raw, k_pool, nblk, pos0, raw_stride,
-                                                        pool_stride, rope, rmsnorm);
+                                                        pool_stride, rope, rn, pg, status);
     return cudaGetLastError();
 }
 
 cudaError_t launch_pool_decode(const void *k_new, void *ring, void *k_pool, const int32_t *seq_len, int B,
-                               int64_t pool_stride, Rope rope, bool rmsnorm, bool bf16, bool fp8, unsigned *status,
-                               cudaStream_t s) {
+                               int64_t pool_stride, Rope rope, bool rmsnorm, bool bf16, bool fp8, const Paging &pg,
+                               unsigned *status, cudaStream_t s) {
     const int rn = rmsnorm ? 1 : 0;
     if (bf16 && fp8)
         return launch_pdl(pool_decode_kernel<__nv_bfloat16, true>, dim3(B), dim3(128), 0, s,
                           (const __nv_bfloat16 *)k_new, (__nv_bfloat16 *)ring, k_pool, seq_len, pool_stride, rope,
-                          rn, status);
+                          rn, pg, status);
     if (bf16)
         return launch_pdl(pool_decode_kernel<__nv_bfloat16, false>, dim3(B), dim3(128), 0, s,
                           (const __nv_bfloat16 *)k_new, (__nv_bfloat16 *)ring, k_pool, seq_len, pool_stride, rope,
-                          rn, status);
+                          rn, pg, status);
     return launch_pdl(pool_decode_kernel<float, false>, dim3(B), dim3(128), 0, s, (const float *)k_new, (float *)ring,
-                      k_pool, seq_len, pool_stride, rope, rn, status);
+                      k_pool, seq_len, pool_stride, rope, rn, pg, status);
 }
 
 cudaError_t launch_rope_apply(void *x, int B, int64_t n, int H, int d, int64_t pos0, Rope rope, bool bf16,

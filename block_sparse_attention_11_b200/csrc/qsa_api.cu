@@ -157,7 +157,8 @@ int qsa_pool_keys_prefill(const void *k_raw, void *k_pool, int32_t B, int64_t n_
     if ((st = check_device(&di)) != QSA_OK) return st;
     return cuda_status(launch_pool_prefill(k_raw, k_pool, B, nblk, pos0, raw_stride, pool_stride, to_rope(rope),
                                            (flags & QSA_POOL_RMSNORM) != 0, dtype == QSA_BF16,
-                                           (flags & QSA_KEYS_FP8) != 0, static_cast<cudaStream_t>(stream)));
+                                           (flags & QSA_KEYS_FP8) != 0, Paging{}, di->status,
+                                           static_cast<cudaStream_t>(stream)));
 }
 
 int qsa_pool_keys_decode(const void *k_new, void *ring, void *k_pool, const int32_t *seq_len, int32_t B,
@@ -172,7 +173,8 @@ int qsa_pool_keys_decode(const void *k_new, void *ring, void *k_pool, const int3
     if ((st = check_device(&di)) != QSA_OK) return st;
     return cuda_status(launch_pool_decode(k_new, ring, k_pool, seq_len, B, pool_stride, to_rope(rope),
                                           (flags & QSA_POOL_RMSNORM) != 0, dtype == QSA_BF16,
-                                          (flags & QSA_KEYS_FP8) != 0, di->status, static_cast<cudaStream_t>(stream)));
+                                          (flags & QSA_KEYS_FP8) != 0, Paging{}, di->status,
+                                          static_cast<cudaStream_t>(stream)));
 }
 
 size_t qsa_index_topk_prefill_workspace(int32_t B, int64_t n_q, int64_t q0, int32_t top_k, uint32_t flags,
@@ -242,6 +244,13 @@ size_t qsa_index_topk_decode_workspace(int32_t B, int64_t max_blocks, int32_t to
     return decode_index_ws_bytes(B, std::max<int64_t>(max_blocks, 1), top_k, dtype == QSA_BF16);
 }
 
+int qsa_index_topk_decode_kernels(int32_t B, int64_t max_blocks, uint32_t flags, int32_t dtype) {
+    if (B < 1 || max_blocks < 0 || (flags & ~kAllFlags) || (dtype != QSA_BF16 && dtype != QSA_FP32)) return 0;
+    const DeviceInfo *di = nullptr;
+    if (check_device(&di) != QSA_OK) return 0;
+    return decode_index_kernel_count(B, max_blocks, dtype == QSA_BF16, (flags & QSA_KEYS_FP8) != 0);
+}
+
 int qsa_index_topk_decode(const void *q_idx, const void *k_pool, const float *head_w, const int32_t *seq_len,
                           int32_t B, int64_t pool_stride, int64_t max_blocks, int32_t top_k, int32_t *sel,
                           int32_t *nsel, void *workspace, size_t ws_bytes, qsa_rope_t rope, uint32_t flags,
@@ -263,7 +272,8 @@ int qsa_index_topk_decode(const void *q_idx, const void *k_pool, const float *he
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return QSA_ERR_INVALID_ARG;
     cudaError_t e = launch_decode_index(q_idx, k_pool, head_w, seq_len, B, pool_stride, mb, top_k, sel, nsel,
                                         workspace, to_rope(rope), (flags & QSA_SCORE_RELU) != 0, dtype == QSA_BF16,
-                                        (flags & QSA_KEYS_FP8) != 0, di->status, static_cast<cudaStream_t>(stream));
+                                        (flags & QSA_KEYS_FP8) != 0, Paging{}, di->status,
+                                        static_cast<cudaStream_t>(stream));
     if (e == cudaErrorInvalidConfiguration) return QSA_ERR_UNSUPPORTED;
     return cuda_status(e);
 }
@@ -394,6 +404,112 @@ int qsa_rope_apply(void *x, int32_t B, int64_t n, int32_t H, int32_t d, int64_t 
     if ((st = check_device(&di)) != QSA_OK) return st;
     return cuda_status(launch_rope_apply(x, B, n, H, d, pos0, to_rope(rope), dtype == QSA_BF16,
                                          static_cast<cudaStream_t>(stream)));
+}
+
+// ---------------------------------------------------------------- paged caches
+
+namespace {
+// Validates a paging descriptor for capacity `need_tokens` (positions 0 ..
+// need_tokens - 1 of a sequence must fit the table row).
+int check_paging(const qsa_paging_t &pg, int64_t need_tokens, Paging *out) {
+    if (!pg.page_table || pg.max_pages < 1 || pg.num_pages < 1) return QSA_ERR_INVALID_ARG;
+    const int pt = pg.page_tokens;
+    if (pt < 32 || (pt & (pt - 1)) != 0) return QSA_ERR_INVALID_ARG;   // a power of two >= 32
+    if (pg.num_pages > ((int64_t)1 << 31) / pt) return QSA_ERR_INVALID_ARG;
+    if (need_tokens > pg.max_pages * (int64_t)pt) return QSA_ERR_INVALID_ARG;
+    out->table = pg.page_table;
+    out->max_pages = pg.max_pages;
+    out->num_pages = pg.num_pages;
+    out->page_tokens = pt;
+    out->page_shift = 0;
+    while ((1 << out->page_shift) < pt) ++out->page_shift;
+    return QSA_OK;
+}
+}  // namespace
+
+int qsa_pool_keys_prefill_paged(const void *k_raw, void *k_pool, qsa_paging_t paging, int32_t B, int64_t n_tok,
+                                int64_t pos0, int64_t raw_stride, qsa_rope_t rope, uint32_t flags, int32_t dtype,
+                                void *stream) {
+    if (B < 1 || n_tok < 0 || pos0 < 0 || (pos0 % kBlock) != 0 || raw_stride < n_tok) return QSA_ERR_INVALID_ARG;
+    Paging pg;
+    int st = check_paging(paging, pos0 + n_tok, &pg);
+    if (st != QSA_OK) return st;
+    if (n_tok < kBlock) return QSA_OK;
+    if (!k_raw || !k_pool) return QSA_ERR_INVALID_ARG;
+    if (flags & ~kAllFlags) return QSA_ERR_INVALID_ARG;
+    if (dtype != QSA_BF16) return QSA_ERR_UNSUPPORTED;
+    if (!aligned16(k_raw) || !aligned16(k_pool)) return QSA_ERR_INVALID_ARG;
+    if ((st = check_rope(rope)) != QSA_OK) return st;
+    const DeviceInfo *di = nullptr;
+    if ((st = check_device(&di)) != QSA_OK) return st;
+    return cuda_status(launch_pool_prefill(k_raw, k_pool, B, n_tok / kBlock, pos0, raw_stride, 0, to_rope(rope),
+                                           (flags & QSA_POOL_RMSNORM) != 0, true, (flags & QSA_KEYS_FP8) != 0, pg,
+                                           di->status, static_cast<cudaStream_t>(stream)));
+}
+
+int qsa_pool_keys_decode_paged(const void *k_new, void *ring, void *k_pool, qsa_paging_t paging,
+                               const int32_t *seq_len, int32_t B, qsa_rope_t rope, uint32_t flags, int32_t dtype,
+                               void *stream) {
+    if (!k_new || !ring || !k_pool || !seq_len || B < 1) return QSA_ERR_INVALID_ARG;
+    Paging pg;
+    int st = check_paging(paging, 0, &pg);
+    if (st != QSA_OK) return st;
+    if (flags & ~kAllFlags) return QSA_ERR_INVALID_ARG;
+    if (dtype != QSA_BF16) return QSA_ERR_UNSUPPORTED;
+    if ((st = check_rope(rope)) != QSA_OK) return st;
+    const DeviceInfo *di = nullptr;
+    if ((st = check_device(&di)) != QSA_OK) return st;
+    return cuda_status(launch_pool_decode(k_new, ring, k_pool, seq_len, B, 0, to_rope(rope),
+                                          (flags & QSA_POOL_RMSNORM) != 0, true, (flags & QSA_KEYS_FP8) != 0, pg,
+                                          di->status, static_cast<cudaStream_t>(stream)));
+}
+
+int qsa_index_topk_decode_paged(const void *q_idx, const void *k_pool, qsa_paging_t paging, const float *head_w,
+                                const int32_t *seq_len, int32_t B, int64_t max_blocks, int32_t top_k, int32_t *sel,
+                                int32_t *nsel, void *workspace, size_t ws_bytes, qsa_rope_t rope, uint32_t flags,
+                                int32_t dtype, void *stream) {
+    if (!q_idx || !k_pool || !seq_len || !sel || !nsel || B < 1 || max_blocks < 0) return QSA_ERR_INVALID_ARG;
+    Paging pg;
+    int st = check_paging(paging, max_blocks * kBlock, &pg);
+    if (st != QSA_OK) return st;
+    if (top_k < 1 || top_k > 2048) return QSA_ERR_INVALID_ARG;
+    if (flags & ~kAllFlags) return QSA_ERR_INVALID_ARG;
+    if (dtype != QSA_BF16) return QSA_ERR_UNSUPPORTED;
+    if (!aligned16(q_idx) || !aligned16(k_pool)) return QSA_ERR_INVALID_ARG;
+    if ((st = check_rope(rope)) != QSA_OK) return st;
+    const DeviceInfo *di = nullptr;
+    if ((st = check_device(&di)) != QSA_OK) return st;
+    const int64_t mb = std::max<int64_t>(max_blocks, 1);
+    const size_t need = decode_index_ws_bytes(B, mb, top_k, true);
+    if (!workspace || ws_bytes < need) return QSA_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return QSA_ERR_INVALID_ARG;
+    const int64_t capacity_rows = pg.max_pages * (pg.page_tokens / kBlock);
+    cudaError_t e = launch_decode_index(q_idx, k_pool, head_w, seq_len, B, capacity_rows, mb, top_k, sel, nsel,
+                                        workspace, to_rope(rope), (flags & QSA_SCORE_RELU) != 0, true,
+                                        (flags & QSA_KEYS_FP8) != 0, pg, di->status,
+                                        static_cast<cudaStream_t>(stream));
+    if (e == cudaErrorInvalidConfiguration) return QSA_ERR_UNSUPPORTED;
+    return cuda_status(e);
+}
+
+int qsa_sparse_attn_decode_paged(const void *q, const void *k, const void *v, qsa_paging_t paging,
+                                 const int32_t *seq_len, const int32_t *sel, const int32_t *nsel, int32_t B,
+                                 int32_t Hq, int32_t Hkv, int32_t d, int32_t top_k, float scale, void *out,
+                                 float *lse, void *workspace, size_t ws_bytes, int32_t dtype, void *stream) {
+    int st = attn_common_checks(q, k, v, sel, nsel, B, Hq, Hkv, d, top_k, scale, out, dtype);
+    if (st != QSA_OK) return st;
+    if (!seq_len) return QSA_ERR_INVALID_ARG;
+    Paging pg;
+    if ((st = check_paging(paging, 0, &pg)) != QSA_OK) return st;
+    if (dtype != QSA_BF16) return QSA_ERR_UNSUPPORTED;
+    const DeviceInfo *di = nullptr;
+    if ((st = check_device(&di)) != QSA_OK) return st;
+    const int64_t capacity = pg.max_pages * (int64_t)pg.page_tokens;
+    AttnArgs a{q, k, v, sel, nsel, seq_len, B, 1, 0, capacity, Hq, Hkv, d, top_k, scale, out, lse, true};
+    a.pg = pg;
+    const size_t need = attn_decode_ws_bytes(B, Hq, d, top_k);
+    if (!workspace || ws_bytes < need) return QSA_ERR_WORKSPACE;
+    return cuda_status(launch_attn_bf16(a, workspace, di->status, static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

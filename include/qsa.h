@@ -223,6 +223,11 @@ QSA_API int qsa_index_topk_prefill(const void *q_idx, const void *k_pool, const 
  *           in stream order.  A call that finds a histogram not zero at its
  *           start flags status bit 16 (its selection is then unreliable).
  */
+/* Kernels a qsa_index_topk_decode call with these sizes launches on the
+ * current device: 1 (scorer and select fused, one thread-block cluster per
+ * sequence, when the clusters fit the GPU at once) or 2 (scorer, then
+ * select); 0 for invalid arguments or an unsupported device. */
+QSA_API int qsa_index_topk_decode_kernels(int32_t B, int64_t max_blocks, uint32_t flags, int32_t dtype);
 QSA_API size_t qsa_index_topk_decode_workspace(int32_t B, int64_t max_blocks, int32_t top_k, uint32_t flags,
                                        int32_t dtype);
 QSA_API int qsa_index_topk_decode(const void *q_idx, const void *k_pool, const float *head_w,
@@ -354,6 +359,58 @@ QSA_API int qsa_sparse_attn_decode_noalloc(const void *q, const void *k, const v
                                            const int32_t *sel, const int32_t *nsel, int32_t B, int64_t kv_stride,
                                            int32_t Hq, int32_t Hkv, int32_t d, int32_t top_k, float scale, void *out,
                                            float *lse, int32_t dtype, void *stream);
+
+/* ========================================================================= */
+/* Paged caches (decode)                                                      */
+/* ========================================================================= */
+/*
+ * Page "Qwen3.8-Flash-Next: Day-0 Support in SGLang", section "Qwen Sparse
+ * Attention: Retrieve Coarsely, Attend Precisely": serving keeps the
+ * original K/V in the engine's paged pool, and a paged scorer reads the
+ * compressed keys there.  The K/V cache is a pool of fixed-size pages
+ * and addresses the compressed-key cache at full_slot / 4, so the 4 tokens of
+ * a block share one page and their compressed key is one row of a paged
+ * compressed-key cache.  A page table maps each sequence's positions to
+ * slots:
+ *   slot(b, i) = page_table[b][i / page_tokens] * page_tokens + i % page_tokens
+ * The K/V caches are [num_pages * page_tokens][Hkv][d]; the compressed-key
+ * cache is [num_pages * page_tokens / 4][128] and block j of sequence b is
+ * its row slot(b, 4j) / 4.  page_tokens is a power of two >= 32; positions
+ * 0 .. max_pages * page_tokens - 1 of a sequence are addressable.  A page id
+ * outside [0, num_pages) met by a kernel is flagged (status bit 1) and its
+ * rows are skipped.  BF16 only (QSA_ERR_UNSUPPORTED otherwise); results are
+ * those of the contiguous entry points on the same logical caches.
+ */
+typedef struct {
+    const int32_t *page_table;   /* device, [B][max_pages] int32 page ids */
+    int64_t max_pages;           /* entries per table row */
+    int64_t num_pages;           /* pages in the caches */
+    int32_t page_tokens;         /* token slots per page */
+} qsa_paging_t;
+
+/* qsa_pool_keys_prefill into a paged compressed-key cache (k_pool as above). */
+QSA_API int qsa_pool_keys_prefill_paged(const void *k_raw, void *k_pool, qsa_paging_t paging, int32_t B,
+                                        int64_t n_tok, int64_t pos0, int64_t raw_stride, qsa_rope_t rope,
+                                        uint32_t flags, int32_t dtype, void *stream);
+/* qsa_pool_keys_decode into a paged compressed-key cache (the ring stays
+ * [B][4][128] per sequence). */
+QSA_API int qsa_pool_keys_decode_paged(const void *k_new, void *ring, void *k_pool, qsa_paging_t paging,
+                                       const int32_t *seq_len, int32_t B, qsa_rope_t rope, uint32_t flags,
+                                       int32_t dtype, void *stream);
+/* qsa_index_topk_decode over a paged compressed-key cache; max_blocks as
+ * there (<= max_pages * page_tokens / 4); workspace sized and kept as for
+ * qsa_index_topk_decode (qsa_index_topk_decode_workspace). */
+QSA_API int qsa_index_topk_decode_paged(const void *q_idx, const void *k_pool, qsa_paging_t paging,
+                                        const float *head_w, const int32_t *seq_len, int32_t B, int64_t max_blocks,
+                                        int32_t top_k, int32_t *sel, int32_t *nsel, void *workspace,
+                                        size_t ws_bytes, qsa_rope_t rope, uint32_t flags, int32_t dtype,
+                                        void *stream);
+/* qsa_sparse_attn_decode over paged K/V caches; workspace as
+ * qsa_sparse_attn_decode_workspace(). */
+QSA_API int qsa_sparse_attn_decode_paged(const void *q, const void *k, const void *v, qsa_paging_t paging,
+                                         const int32_t *seq_len, const int32_t *sel, const int32_t *nsel, int32_t B,
+                                         int32_t Hq, int32_t Hkv, int32_t d, int32_t top_k, float scale, void *out,
+                                         float *lse, void *workspace, size_t ws_bytes, int32_t dtype, void *stream);
 
 /* ========================================================================= */
 /* Helper: the attention layer's RoPE                                         */

@@ -347,6 +347,108 @@ def test_decode_select_all_ties(qsa, dtype, flags, lens):
         assert np.array_equal(sel[b].cpu().numpy(), exp), b
 
 
+def _paged_layout(lens, page_tokens, extra_pages, seed):
+    """A page table that scatters each sequence's pages over a shuffled pool;
+    table entries past a sequence's pages are -1 (never read)."""
+    rng = np.random.default_rng(seed)
+    need = [(L + page_tokens) // page_tokens for L in lens]          # positions 0 .. L (the new token)
+    max_pages = max(need) + 1
+    num_pages = sum(need) + extra_pages
+    perm = rng.permutation(num_pages)
+    table = np.full((len(lens), max_pages), -1, np.int32)
+    k = 0
+    for b, n in enumerate(need):
+        table[b, :n] = perm[k:k + n]
+        k += n
+    return table, num_pages
+
+
+@pytest.mark.parametrize("B,L,page_tokens,keys", [(6, 20000, 64, "bf16"), (3, 70001, 256, "bf16"),
+                                                  (12, 9001, 32, "fp8"), (5, 2, 64, "bf16"),
+                                                  (4, 5000, 1024, "bf16")])
+def test_decode_paged_matches_contiguous(qsa, B, L, page_tokens, keys):
+    """Paged caches (a shuffled page pool, one table row per sequence) give the
+    contiguous results bit for bit: pooled rows, selections, attention output."""
+    w = workloads.Workload("dec_paged", "decode", B, L, 256, 16, 2, 128, "bf16", 78, pos_scale=2.0)
+    x = workloads.make_decode(w, device=DEV, ragged=True)
+    rope = rope_of(w)
+    lens = x["lens"]
+    fp8 = keys == "fp8"
+    kf = qsa.QSA_KEYS_FP8 if fp8 else 0
+    kdt = torch.float8_e4m3fn if fp8 else torch.bfloat16
+    table_np, num_pages = _paged_layout(lens, page_tokens, 3, B + L)
+    table = torch.from_numpy(table_np).to(DEV)
+    pt = page_tokens
+    # contiguous reference pipeline
+    cap = max(lens) // 4 + 2
+    k_pool = torch.zeros(B, cap, 128, dtype=kdt, device=DEV)
+    ring = torch.zeros(B, 4, 128, dtype=torch.bfloat16, device=DEV)
+    for b in range(B):
+        kp = torch.zeros(1, cap, 128, dtype=kdt, device=DEV)
+        qsa.qsa_pool_keys_prefill(x["k_idx"][b:b + 1, :lens[b]].contiguous(), kp, rope=rope, flags=kf)
+        k_pool[b] = kp[0]
+        nb0 = lens[b] // 4
+        if lens[b] > 4 * nb0:
+            ring[b, :lens[b] - 4 * nb0] = x["k_idx"][b, 4 * nb0: lens[b]]
+    ring_p = ring.clone()
+    qsa.qsa_pool_keys_decode(x["k_idx_new"], ring, k_pool, x["seq_len"], rope=rope, flags=kf)
+    sel = torch.empty(B, w.top_k, dtype=torch.int32, device=DEV)
+    nsel = torch.empty(B, dtype=torch.int32, device=DEV)
+    qsa.qsa_index_topk_decode(x["q_idx"], k_pool, x["seq_len"], sel, nsel, top_k=w.top_k, rope=rope, flags=kf)
+    out = torch.empty_like(x["q"])
+    qsa.qsa_sparse_attn_decode(x["q"], x["k"], x["v"], x["seq_len"], sel, nsel, out)
+    # paged caches: K/V scattered to their slots, compressed keys pooled straight into pages
+    slots = [torch.from_numpy((table_np[b, np.arange(lens[b] + 1) // pt].astype(np.int64) * pt
+                               + np.arange(lens[b] + 1) % pt)).to(DEV) for b in range(B)]
+    k_pg = torch.zeros(num_pages * pt, 2, 128, dtype=torch.bfloat16, device=DEV)
+    v_pg = torch.zeros_like(k_pg)
+    for b in range(B):
+        k_pg[slots[b]] = x["k"][b, :lens[b] + 1]
+        v_pg[slots[b]] = x["v"][b, :lens[b] + 1]
+    kpool_pg = torch.zeros(num_pages * pt // 4, 128, dtype=kdt, device=DEV)
+    for b in range(B):
+        qsa.qsa_pool_keys_prefill_paged(x["k_idx"][b:b + 1, :lens[b]].contiguous(), kpool_pg, table[b:b + 1], pt,
+                                        rope=rope, flags=kf)
+    qsa.qsa_pool_keys_decode_paged(x["k_idx_new"], ring_p, kpool_pg, table, pt, x["seq_len"], rope=rope, flags=kf)
+    sel_p = torch.full((B, w.top_k), -7, dtype=torch.int32, device=DEV)
+    nsel_p = torch.full((B,), -7, dtype=torch.int32, device=DEV)
+    qsa.qsa_index_topk_decode_paged(x["q_idx"], kpool_pg, table, pt, x["seq_len"], sel_p, nsel_p, top_k=w.top_k,
+                                    rope=rope, flags=kf)
+    out_p = torch.empty_like(x["q"])
+    qsa.qsa_sparse_attn_decode_paged(x["q"], k_pg, v_pg, table, pt, x["seq_len"], sel_p, nsel_p, out_p)
+    qsa.qsa_check_status()                       # no page outside the table was touched
+    assert torch.equal(ring_p, ring)
+    for b in range(B):
+        nbk = (lens[b] + 1) // 4
+        rows = slots[b][0:4 * nbk:4] // 4
+        assert torch.equal(kpool_pg[rows].view(torch.uint8), k_pool[b, :nbk].view(torch.uint8)), b
+    assert torch.equal(nsel_p, nsel) and torch.equal(sel_p, sel)
+    assert torch.equal(out_p, out)
+
+
+def test_decode_paged_flags_a_page_outside_the_cache(qsa):
+    B, L, pt = 2, 3000, 64
+    w = workloads.Workload("dec_paged_bad", "decode", B, L, 64, 16, 2, 128, "bf16", 79)
+    x = workloads.make_decode(w, device=DEV)
+    table_np, num_pages = _paged_layout([L] * B, pt, 0, 5)
+    table_np[1, 3] = num_pages + 7               # one page id past the pool
+    table = torch.from_numpy(table_np).to(DEV)
+    kpool = torch.zeros(num_pages * pt // 4, 128, dtype=torch.bfloat16, device=DEV)
+    kv = torch.zeros(num_pages * pt, 2, 128, dtype=torch.bfloat16, device=DEV)
+    sel = torch.empty(B, w.top_k, dtype=torch.int32, device=DEV)
+    nsel = torch.empty(B, dtype=torch.int32, device=DEV)
+    qsa.qsa_index_topk_decode_paged(x["q_idx"], kpool, table, pt, x["seq_len"], sel, nsel, top_k=w.top_k,
+                                    rope=rope_of(w))
+    with pytest.raises(qsa.QSAError):
+        qsa.qsa_check_status()
+    out = torch.empty_like(x["q"])
+    sel_all = torch.arange(w.top_k, dtype=torch.int32, device=DEV).repeat(B, 1) + 40   # blocks 40.. cross page 3
+    nsel_all = torch.full((B,), w.top_k, dtype=torch.int32, device=DEV)
+    qsa.qsa_sparse_attn_decode_paged(x["q"], kv, kv, table, pt, x["seq_len"], sel_all, nsel_all, out)
+    with pytest.raises(qsa.QSAError):
+        qsa.qsa_check_status()
+
+
 def test_decode_index_workspace_stays_zero_and_dirty_one_is_flagged(qsa):
     """The two-kernel decode indexer leaves its workspace zero after a call,
     so one zero-filled workspace serves any number of calls; a workspace whose

@@ -95,6 +95,22 @@ def test_invalid_arguments_are_rejected_before_launch(qsa):
                                       None) == qsa.QSA_ERR_UNSUPPORTED
     assert lib.qsa_index_topk_decode(fake, fake, None, fake, 1, 4, 4, 4, fake, fake, fake, 1 << 20, rope, fp8, 1,
                                      None) == qsa.QSA_ERR_UNSUPPORTED
+    # paged caches: a table is required, page_tokens a power of two >= 32, BF16 only
+    pg = qsa._Paging(4096, 8, 16, 64)
+    assert lib.qsa_pool_keys_decode_paged(fake, fake, fake, qsa._Paging(None, 8, 16, 64), fake, 1, rope, 0, 0,
+                                          None) == qsa.QSA_ERR_INVALID_ARG
+    assert lib.qsa_pool_keys_decode_paged(fake, fake, fake, qsa._Paging(4096, 8, 16, 48), fake, 1, rope, 0, 0,
+                                          None) == qsa.QSA_ERR_INVALID_ARG
+    assert lib.qsa_pool_keys_decode_paged(fake, fake, fake, qsa._Paging(4096, 8, 16, 16), fake, 1, rope, 0, 0,
+                                          None) == qsa.QSA_ERR_INVALID_ARG
+    assert lib.qsa_pool_keys_decode_paged(fake, fake, fake, pg, fake, 1, rope, 0, 1, None) == qsa.QSA_ERR_UNSUPPORTED
+    # max_blocks beyond the table's capacity (8 pages x 64 tokens = 128 blocks)
+    assert lib.qsa_index_topk_decode_paged(fake, fake, pg, None, fake, 1, 129, 64, fake, fake, fake, 1 << 20, rope,
+                                           0, 0, None) == qsa.QSA_ERR_INVALID_ARG
+    assert lib.qsa_pool_keys_prefill_paged(fake, fake, pg, 1, 16, 512, 16, rope, 0, 0, None) == qsa.QSA_ERR_INVALID_ARG
+    assert lib.qsa_sparse_attn_decode_paged(fake, fake, fake, pg, fake, fake, fake, 1, 16, 2, 128, 64, 0.1, fake,
+                                            None, fake, 1 << 20, 1, None) == qsa.QSA_ERR_UNSUPPORTED
+    assert lib.qsa_index_topk_decode_kernels(0, 100, 0, 0) == 0
     # misaligned pointer
     odd = ctypes.c_void_p(4098)
     assert lib.qsa_pool_keys_prefill(odd, fake, 1, 16, 0, 16, 4, rope, 0, 0, None) == qsa.QSA_ERR_INVALID_ARG

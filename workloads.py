@@ -66,6 +66,9 @@ WORKLOADS = {
                                          "bf16", 1003, extra={"keys": "fp8"}),
     "decode_b8_l1m_scale4_fp8keys": Workload("decode_b8_l1m_scale4_fp8keys", "decode", 8, 1048576, 512, 16, 2,
                                              128, "bf16", 1005, pos_scale=4.0, extra={"keys": "fp8"}),
+    # the 128K decode workload over paged caches (64-token pages, shuffled page pool)
+    "decode_b64_l128k_paged": Workload("decode_b64_l128k_paged", "decode", 64, 131072, 512, 16, 2, 128, "bf16",
+                                       1003, extra={"page_tokens": 64}),
     # full causal decode attention on the same caches as the QSA decode workloads
     "dense_b64_l128k": Workload("dense_b64_l128k", "dense", 64, 131072, 512, 16, 2, 128, "bf16", 1003),
     "dense_b8_l1m_scale4": Workload("dense_b8_l1m_scale4", "dense", 8, 1048576, 512, 16, 2, 128, "bf16", 1005,
