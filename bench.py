@@ -163,6 +163,11 @@ class PrefillRunner:
         self.x = workloads.make_prefill(w, device=dev)
         B, T = w.B, w.T
         dt = workloads.torch_dtype(w)
+        # FP8 E4M3 K/V caches with per-tensor scales ("kv": "fp8"): the attention reads them
+        self.kv8 = w.extra.get("kv") == "fp8"
+        if self.kv8:
+            self.x["k"], self.k_scale = workloads.to_e4m3(self.x["k"])
+            self.x["v"], self.v_scale = workloads.to_e4m3(self.x["v"])
         self.rope = qsa.Rope(base=w.rope_base, pos_scale=w.pos_scale, rotary_dim=128)
         self.k_pool = torch.zeros(B, max(T // 4, 1), 128, dtype=dt, device=dev)
         self.sel = torch.empty(B, T, w.top_k, dtype=torch.int32, device=dev)
@@ -187,7 +192,11 @@ class PrefillRunner:
                                    workspace=self.ws)
         if events is not None:
             events[2].record()
-        qsa.qsa_sparse_attn_prefill(x["q"], x["k"], x["v"], self.sel, self.nsel, self.out)
+        if self.kv8:
+            qsa.qsa_sparse_attn_prefill_kv8(x["q"], x["k"], x["v"], self.k_scale, self.v_scale, self.sel, self.nsel,
+                                            self.out)
+        else:
+            qsa.qsa_sparse_attn_prefill(x["q"], x["k"], x["v"], self.sel, self.nsel, self.out)
         if events is not None:
             events[3].record()
         return self.out
@@ -208,7 +217,8 @@ class PrefillRunner:
         t = torch.arange(T, dtype=torch.float64)
         nb = torch.floor((t + 1) / 4)
         npos = torch.minimum(nb, torch.tensor(float(K))) * 4 + (t + 1 - 4 * nb)
-        gather = float(npos.sum()) * w.Hkv * w.d * 2 * 2 * w.B        # K and V bytes gathered
+        el = 1 if w.extra.get("kv") == "fp8" else 2                    # bytes per K/V element
+        gather = float(npos.sum()) * w.Hkv * w.d * el * 2 * w.B       # K and V bytes gathered
         qo = 2.0 * T * w.Hq * w.d * 2 * w.B                            # q read + out write
         attn_flops = float(npos.sum()) * 4 * w.d * w.Hq * w.B
         pairs = float(nb.sum()) * w.B
@@ -235,6 +245,12 @@ class DecodeRunner:
         self.fp8 = w.extra.get("keys") == "fp8"
         self.kflags = qsa.QSA_KEYS_FP8 if self.fp8 else 0
         kdt = torch.float8_e4m3fn if self.fp8 else dt
+        # FP8 E4M3 K/V caches with per-tensor scales ("kv": "fp8")
+        self.kv8 = w.extra.get("kv") == "fp8"
+        if self.kv8:
+            x["k"], self.k_scale = workloads.to_e4m3(x["k"])
+            x["v"], self.v_scale = workloads.to_e4m3(x["v"])
+            torch.cuda.empty_cache()
         # paged caches ("page_tokens"): every sequence's pages scattered over a
         # shuffled pool, one page-table row per sequence
         self.pt = int(w.extra.get("page_tokens", 0))
@@ -300,6 +316,9 @@ class DecodeRunner:
         if self.pt:
             qsa.qsa_sparse_attn_decode_paged(x["q"], x["k"], x["v"], self.table, self.pt, x["seq_len"], self.sel,
                                              self.nsel, self.out, workspace=self.ws_a)
+        elif self.kv8:
+            qsa.qsa_sparse_attn_decode_kv8(x["q"], x["k"], x["v"], self.k_scale, self.v_scale, x["seq_len"], self.sel,
+                                           self.nsel, self.out, workspace=self.ws_a)
         else:
             qsa.qsa_sparse_attn_decode(x["q"], x["k"], x["v"], x["seq_len"], self.sel, self.nsel, self.out,
                                        workspace=self.ws_a)
@@ -323,8 +342,9 @@ class DecodeRunner:
         tail = (w.T + 1) - 4 * nb
         npos = min(nb, w.top_k) * 4 + tail
         kbytes = 1 if w.extra.get("keys") == "fp8" else 2
+        el = 1 if w.extra.get("kv") == "fp8" else 2                    # bytes per K/V element
         idx_bytes = nb * 128 * kbytes + 4 * 128 * 2                   # compressed keys + indexer query
-        kv_bytes = npos * w.Hkv * w.d * 2 * 2 + 2 * w.Hq * w.d * 2     # gathered K/V + q + out
+        kv_bytes = npos * w.Hkv * w.d * el * 2 + 2 * w.Hq * w.d * 2    # gathered K/V + q + out
         return dict(idx_bytes=idx_bytes * w.B, attn_bytes=kv_bytes * w.B, step_bytes=(idx_bytes + kv_bytes) * w.B)
 
     def host_inputs(self):
@@ -669,6 +689,7 @@ def run_oracle_sample(w, budget_s=15.0, seed=0):
     nthreads = os.cpu_count() or 1
     if w.kind == "prefill":
         x = workloads.make_prefill(w, device="cpu")
+        dequant_kv(w, x)
         q_idx = x["q_idx"][0].float().numpy()
         k_raw = x["k_idx"][0].float().numpy()
         q, k, v = (x[n][0].float().numpy() for n in ("q", "k", "v"))
@@ -708,6 +729,7 @@ def run_oracle_sample(w, budget_s=15.0, seed=0):
         return value, f"{reps} steps of one {w.T}-token sequence, scaled to B={w.B}", nthreads, "us/step"
     # decode: a subset of sequences at full length
     x = workloads.make_decode(w, device="cpu", B=1)
+    dequant_kv(w, x)
     kr = x["k_idx"][0].float().numpy()
     kp = oracle.pool_keys(kr, base=w.rope_base, pos_scale=w.pos_scale, store_bf16=True,
                           store_fp8=w.extra.get("keys") == "fp8")
@@ -732,6 +754,14 @@ def run_oracle_sample(w, budget_s=15.0, seed=0):
     if w.kind == "draft":
         sample += " (the oracle selects for the capture row on every step: it takes no frozen selection)"
     return value, sample, nthreads, "us/step"
+
+
+def dequant_kv(w, x):
+    """FP8 K/V workloads: the oracle reads the dequantized caches."""
+    if w.extra.get("kv") == "fp8":
+        for n in ("k", "v"):
+            c, sc = workloads.to_e4m3(x[n])
+            x[n] = c.float() * sc
 
 
 def metric_name(w):

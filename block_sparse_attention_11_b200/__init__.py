@@ -28,7 +28,7 @@ __all__ = [
     "qsa_sparse_attn_decode_noalloc", "qsa_sparse_attn_decode_shared", "qsa_sparse_attn_decode_shared_workspace",
     "qsa_dense_attn_decode", "qsa_dense_attn_decode_workspace",
     "qsa_pool_keys_prefill_paged", "qsa_pool_keys_decode_paged", "qsa_index_topk_decode_paged",
-    "qsa_sparse_attn_decode_paged",
+    "qsa_sparse_attn_decode_paged", "qsa_sparse_attn_prefill_kv8", "qsa_sparse_attn_decode_kv8",
     "qsa_rope_apply", "qsa_check_status", "qsa_strerror", "qsa_version",
     "QSA_SCORE_RELU", "QSA_POOL_RMSNORM", "QSA_KEYS_FP8", "QSA_BF16", "QSA_FP32",
 ]
@@ -115,6 +115,10 @@ _sig("qsa_index_topk_decode_paged", ctypes.c_int, _vp, _vp, _Paging, _vp, _vp, _
      _Rope, _u32, _i32, _vp)
 _sig("qsa_sparse_attn_decode_paged", ctypes.c_int, _vp, _vp, _vp, _Paging, _vp, _vp, _vp, _i32, _i32, _i32, _i32,
      _i32, _f32, _vp, _vp, _vp, _sz, _i32, _vp)
+_sig("qsa_sparse_attn_prefill_kv8", ctypes.c_int, _vp, _vp, _vp, _f32, _f32, _vp, _vp, _i32, _i64, _i64, _i64, _i32,
+     _i32, _i32, _i32, _f32, _vp, _vp, _vp)
+_sig("qsa_sparse_attn_decode_kv8", ctypes.c_int, _vp, _vp, _vp, _f32, _f32, _vp, _vp, _vp, _i32, _i64, _i32, _i32,
+     _i32, _i32, _f32, _vp, _vp, _vp, _sz, _vp)
 _sig("qsa_sparse_attn_decode_noalloc", ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32,
      _i32, _f32, _vp, _vp, _i32, _vp)
 
@@ -415,6 +419,45 @@ def qsa_sparse_attn_decode_paged(q, k, v, page_table, page_tokens, seq_len, sel,
                                           _ptr(out, q.dtype, "out"), _ptr(lse, torch.float32, "lse"), wp, wb, dt,
                                           _stream(q, stream))
     _check(st, "qsa_sparse_attn_decode_paged")
+
+
+def _kv8_ptr(t, name):
+    if not isinstance(t, torch.Tensor) or t.dtype not in (torch.float8_e4m3fn, torch.uint8):
+        raise TypeError(f"{name} must be float8_e4m3fn (or uint8)")
+    return _ptr(t, None, name)
+
+
+def qsa_sparse_attn_prefill_kv8(q, k, v, k_scale, v_scale, sel, nsel, out, q0=0, top_k=None, scale=None, lse=None,
+                                stream=None):
+    """As qsa_sparse_attn_prefill with FP8 E4M3 K/V caches (K = k_scale * k, V = v_scale * v);
+    q, out bfloat16 [B][n_q][Hq][d]; k, v [B][L][Hkv][d] float8_e4m3fn."""
+    B, n_q, Hq, d = q.shape
+    Hkv = k.shape[2]
+    top_k = sel.shape[-1] if top_k is None else top_k
+    scale = (1.0 / d ** 0.5) if scale is None else scale
+    st = lib.qsa_sparse_attn_prefill_kv8(_ptr(q, torch.bfloat16, "q"), _kv8_ptr(k, "k"), _kv8_ptr(v, "v"),
+                                         float(k_scale), float(v_scale), _ptr(sel, torch.int32, "sel"),
+                                         _ptr(nsel, torch.int32, "nsel"), B, n_q, q0, k.shape[1], Hq, Hkv, d, top_k,
+                                         scale, _ptr(out, torch.bfloat16, "out"), _ptr(lse, torch.float32, "lse"),
+                                         _stream(q, stream))
+    _check(st, "qsa_sparse_attn_prefill_kv8")
+
+
+def qsa_sparse_attn_decode_kv8(q, k, v, k_scale, v_scale, seq_len, sel, nsel, out, top_k=None, scale=None, lse=None,
+                               workspace=None, stream=None):
+    """As qsa_sparse_attn_decode with FP8 E4M3 K/V caches (K = k_scale * k, V = v_scale * v)."""
+    B, Hq, d = q.shape
+    Hkv = k.shape[2]
+    top_k = sel.shape[-1] if top_k is None else top_k
+    scale = (1.0 / d ** 0.5) if scale is None else scale
+    need = qsa_sparse_attn_decode_workspace(B, Hq, d, top_k, QSA_BF16)
+    wp, wb = _ws(need, q.device, workspace)
+    st = lib.qsa_sparse_attn_decode_kv8(_ptr(q, torch.bfloat16, "q"), _kv8_ptr(k, "k"), _kv8_ptr(v, "v"),
+                                        float(k_scale), float(v_scale), _ptr(seq_len, torch.int32, "seq_len"),
+                                        _ptr(sel, torch.int32, "sel"), _ptr(nsel, torch.int32, "nsel"), B,
+                                        k.shape[1], Hq, Hkv, d, top_k, scale, _ptr(out, torch.bfloat16, "out"),
+                                        _ptr(lse, torch.float32, "lse"), wp, wb, _stream(q, stream))
+    _check(st, "qsa_sparse_attn_decode_kv8")
 
 
 def qsa_rope_apply(x, pos0=0, rope=Rope(), stream=None):

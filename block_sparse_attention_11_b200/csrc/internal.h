@@ -127,6 +127,8 @@ struct AttnArgs {
     int max_draft = 0;                  // IndexShare: largest seq_len - cap_len
     bool dense = false;                 // decode: dense causal attention over every position (no selection)
     Paging pg;                          // pg.table: paged K/V caches (bf16 kernels), kv_stride = its capacity
+    bool kv8 = false;                   // K/V caches of FP8 E4M3 (bf16 q/out): K = k_scale * k8, V = v_scale * v8
+    float k_scale = 1.f, v_scale = 1.f;
 };
 int attn_tail_blocks(bool indexshare, int max_draft);
 size_t attn_decode_ws_bytes(int B, int Hq, int d, int top_k, int tail_blocks = 1);

@@ -61,7 +61,8 @@ constexpr uint32_t kFullStage = 0x924924u;   // 8 slots x 3 bits, each holding 4
 #define QSA_ATTN_TILES 2          // 16-key tiles of a stage per consumer warp (1 or 2); 2 with 4 kv heads
 #endif
 
-template <int HKV> struct AttnCfg {
+// KV8: K/V caches of FP8 E4M3 values (times per-tensor scales), 1 byte per element.
+template <int HKV, bool KV8 = false> struct AttnCfg {
     // Consumer warp (g, sub): kv head g; sub = u * 2 + hf takes the stages whose
     // global index is = hf (mod 2), and tiles [u * kTiles, (u + 1) * kTiles) of each.
     static constexpr int kTiles = HKV == 4 ? 2 : QSA_ATTN_TILES;
@@ -71,7 +72,9 @@ template <int HKV> struct AttnCfg {
     static constexpr int kMinCtas = HKV == 4 ? 1 : QSA_ATTN_CTAS;   // launch-bounds residency target
     static constexpr int kPw = QSA_ATTN_PW;
     static constexpr int kThreads = (kConsumers + kPw) * 32;
-    static constexpr int kSpan = kBlock * HKV * 128 * 2;      // bytes of one block, all kv heads
+    static constexpr int kEl = KV8 ? 1 : 2;                    // bytes per K/V element
+    static constexpr int kTokBytes = HKV * 128 * kEl;          // one token, all kv heads
+    static constexpr int kSpan = kBlock * kTokBytes;           // bytes of one block, all kv heads
     static constexpr int kSlot = kSpan + 16;                   // padded slot
     static constexpr int kStage = 2 * AT_BPS * kSlot;          // K slots then V slots
     static constexpr int kHq = 8 * HKV;
@@ -106,6 +109,7 @@ struct AttnParams {
     int max_draft;           // IndexShare: largest seq_len - cap_len
     int dense;               // decode: every visible block in order (dense causal attention, no selection)
     unsigned *status;
+    float k_scale, v_scale;  // KV8: K = k_scale * stored E4M3 value, V = v_scale * stored value
     Paging pg;               // pg.table: K/V are paged caches [slots][Hkv][128] (kv_stride = table capacity)
 };
 
@@ -171,12 +175,12 @@ __device__ __forceinline__ Item get_item(const AttnParams &p, int64_t i) {
     return it;
 }
 
-template <int HKV>
+template <int HKV, bool KV8>
 struct __align__(128) AttnSmem {
-    using Cfg = AttnCfg<HKV>;
-    uint8_t stage[Cfg::kNS][AttnCfg<HKV>::kStage];
-    alignas(16) uint8_t qbuf[2][AttnCfg<HKV>::kQBytes];
-    float xbuf[HKV][AttnCfg<HKV>::kWph - 1][32][36];
+    using Cfg = AttnCfg<HKV, KV8>;
+    uint8_t stage[Cfg::kNS][Cfg::kStage];
+    alignas(16) uint8_t qbuf[2][Cfg::kQBytes];
+    float xbuf[HKV][Cfg::kWph - 1][32][36];
     alignas(16) __nv_bfloat16 obuf[HKV][8][128];
     alignas(16) uint32_t info[Cfg::kNS][Cfg::kPw];
     uint64_t full[Cfg::kNS], empty[Cfg::kNS], qfull[2], qempty[2];
@@ -187,18 +191,19 @@ struct __align__(128) AttnSmem {
     //   uint32_t st_bytes[kPw][nst_cap]     per stage of the item: bytes the producer copies per tensor
 };
 
-template <int HKV>
+template <int HKV, bool KV8>
 size_t attn_smem_bytes(int sel_cap, int nst_cap) {
-    return sizeof(AttnSmem<HKV>) + (size_t)sel_cap * 4 + 2 * (size_t)AttnCfg<HKV>::kPw * nst_cap * 4 + 128;
+    return sizeof(AttnSmem<HKV, KV8>) + (size_t)sel_cap * 4 + 2 * (size_t)AttnCfg<HKV>::kPw * nst_cap * 4 + 128;
 }
 
 // PAGED: K/V are paged caches addressed through p.pg (a separate instantiation,
 // so the contiguous kernels carry none of the page-table code).
-template <int HKV, bool PAGED>
+template <int HKV, bool PAGED, bool KV8>
 __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, AttnCfg<HKV>::kMinCtas) attn_bf16_kernel(AttnParams p) {
-    using Cfg = AttnCfg<HKV>;
+    using Cfg = AttnCfg<HKV, KV8>;
     extern __shared__ uint8_t asm_raw[];
-    AttnSmem<HKV> &sm = *reinterpret_cast<AttnSmem<HKV> *>((reinterpret_cast<uintptr_t>(asm_raw) + 127) & ~uintptr_t(127));
+    AttnSmem<HKV, KV8> &sm =
+        *reinterpret_cast<AttnSmem<HKV, KV8> *>((reinterpret_cast<uintptr_t>(asm_raw) + 127) & ~uintptr_t(127));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     // zero the slots once: masked keys must read finite values (0 * NaN = NaN)
@@ -263,7 +268,7 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, AttnCfg<HKV>::kMinCtas
                         }
                     }
                     info |= (uint32_t)tokens << (3 * j);
-                    bytes += (uint32_t)tokens * HKV * 256u;
+                    bytes += (uint32_t)tokens * Cfg::kTokBytes;
                 }
                 st_info[st] = info;
                 st_bytes[st] = bytes;
@@ -297,7 +302,7 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, AttnCfg<HKV>::kMinCtas
                             flag(p.status, QSA_DEV_BAD_INDEX);
                         }
                         sinfo |= (uint32_t)tokens << (3 * j);
-                        sbytes += (uint32_t)tokens * HKV * 256u;
+                        sbytes += (uint32_t)tokens * Cfg::kTokBytes;
                     }
                 }
                 if (it_count >= Cfg::kNS) ok = mbar_wait(&sm.empty[s], (int)(((it_count / Cfg::kNS) + 1) & 1), p.status);
@@ -315,10 +320,12 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, AttnCfg<HKV>::kMinCtas
                         const int64_t blk = (e < it.nsel) ? (p.dense ? (int64_t)e : (int64_t)ids[e - it.lbeg])
                                                           : it.nb + (e - it.nsel);
                         const int64_t tok = PAGED ? paged_slot(p.pg, it.seq, blk * kBlock) : kv0 + blk * kBlock;
-                        const int64_t off = tok * HKV * 128;
-                        const uint32_t nbytes = (uint32_t)tokens * HKV * 256u;
-                        bulk_g2s(sm.stage[s] + j * Cfg::kSlot, p.k + off, nbytes, &sm.full[s]);
-                        bulk_g2s(sm.stage[s] + (AT_BPS + j) * Cfg::kSlot, p.v + off, nbytes, &sm.full[s]);
+                        const int64_t off = tok * Cfg::kTokBytes;   // bytes
+                        const uint32_t nbytes = (uint32_t)tokens * Cfg::kTokBytes;
+                        bulk_g2s(sm.stage[s] + j * Cfg::kSlot, reinterpret_cast<const uint8_t *>(p.k) + off, nbytes,
+                                 &sm.full[s]);
+                        bulk_g2s(sm.stage[s] + (AT_BPS + j) * Cfg::kSlot, reinterpret_cast<const uint8_t *>(p.v) + off,
+                                 nbytes, &sm.full[s]);
                     }
                 }
             }
@@ -348,10 +355,20 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, AttnCfg<HKV>::kMinCtas
     const int gr = lane >> 2, tq = lane & 3;
     const uint32_t stage0 = smem_u32(&sm.stage[0][0]);
     const int mi = lane >> 3, rr = lane & 7;
-    const uint32_t k_lane_off = (uint32_t)(rr * Cfg::kSlot + (mi & 1) * HKV * 256 + g * 256 + (mi >> 1) * 16);
-    const uint32_t v_lane_off = (uint32_t)(AT_BPS * Cfg::kSlot + rr * Cfg::kSlot + (mi >> 1) * HKV * 256 +
-                                           g * 256 + (mi & 1) * 16);
-    constexpr uint32_t kTileOff = 2 * HKV * 256;     // tokens {2,3} vs {0,1}
+    // ldmatrix lane addresses: matrix mi = lane / 8 reads row rr (= block) of
+    // the stage's 8 slots.  K: token + (mi & 1), 16 bytes + (mi >> 1).  V (bf16,
+    // transposed): token + (mi >> 1), 16 bytes + (mi & 1); V (FP8): token +
+    // (mi & 1), 16 bytes + (mi >> 1), so registers 0/1 hold the two tokens of
+    // one 16-byte column and 2/3 of the next.
+    constexpr int kHead = 128 * Cfg::kEl;            // bytes of one kv head of one token
+    const uint32_t k_lane_off =
+        (uint32_t)(rr * Cfg::kSlot + (mi & 1) * Cfg::kTokBytes + g * kHead + (mi >> 1) * 16);
+    const uint32_t v_lane_off =
+        KV8 ? (uint32_t)(AT_BPS * Cfg::kSlot + rr * Cfg::kSlot + (mi & 1) * Cfg::kTokBytes + g * kHead +
+                         (mi >> 1) * 16)
+            : (uint32_t)(AT_BPS * Cfg::kSlot + rr * Cfg::kSlot + (mi >> 1) * Cfg::kTokBytes + g * kHead +
+                         (mi & 1) * 16);
+    constexpr uint32_t kTileOff = 2 * Cfg::kTokBytes;   // tokens {2,3} vs {0,1}
     int64_t it_count = 0, ic = 0;
     bool ok = true;
     for (int64_t i = blockIdx.x; i < p.items && ok; i += gridDim.x, ++ic) {
@@ -360,7 +377,8 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, AttnCfg<HKV>::kMinCtas
         ok = mbar_wait(&sm.qfull[qs], (int)((ic >> 1) & 1), p.status);
         if (!ok) break;
         uint32_t qf[8][2];
-        {
+        float sl2 = p.scale_log2;   // logit scale in log2 units
+        if constexpr (!KV8) {
             const uint32_t *qw = reinterpret_cast<const uint32_t *>(sm.qbuf[qs]);
             const int head = 8 * g + gr;
 #pragma unroll
@@ -368,6 +386,37 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, AttnCfg<HKV>::kMinCtas
                 qf[kk][0] = qw[(head * 128 + 16 * kk + 2 * tq) >> 1];
                 qf[kk][1] = qw[(head * 128 + 16 * kk + 8 + 2 * tq) >> 1];
             }
+        } else {
+            // FP8 keys are scored as FP16 (E4M3 is a subset of FP16); the query
+            // goes to FP16 times 2^e (e puts the kv head's largest |q| in
+            // [2^14, 2^15)), in the k order of the widened key fragments:
+            // k-step 2j takes dims 32j + 4tq + {0..3}, k-step 2j + 1 dims
+            // 32j + 16 + 4tq + {0..3}.
+            const __nv_bfloat16 *qh = reinterpret_cast<const __nv_bfloat16 *>(sm.qbuf[qs]) + (8 * g + gr) * 128;
+            float qv[8][4];
+            float mx = 0.f;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    qv[kk][c] = __bfloat162float(qh[32 * (kk >> 1) + 16 * (kk & 1) + 4 * tq + c]);
+                    mx = fmaxf(mx, fabsf(qv[kk][c]));
+                }
+#pragma unroll
+            for (int o2 = 16; o2 > 0; o2 >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o2));
+            int qexp = 0;
+            if (mx > 0.f && mx <= 3.0e38f) {
+                int ex;
+                frexpf(mx, &ex);
+                qexp = min(max(15 - ex, -100), 100);
+            }
+            const float sc2 = ldexpf(1.0f, qexp);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                qf[kk][0] = pack_f16(__fmul_rn(qv[kk][0], sc2), __fmul_rn(qv[kk][1], sc2));
+                qf[kk][1] = pack_f16(__fmul_rn(qv[kk][2], sc2), __fmul_rn(qv[kk][3], sc2));
+            }
+            sl2 = p.scale_log2 * p.k_scale * ldexpf(1.0f, -qexp);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.qempty[qs]);
@@ -396,13 +445,30 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, AttnCfg<HKV>::kMinCtas
             for (int t = 0; t < kT; ++t)
 #pragma unroll
                 for (int c = 0; c < 4; ++c) sc[t][c] = 0.f;
+            if constexpr (!KV8) {
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
+                for (int kk = 0; kk < 8; ++kk) {
 #pragma unroll
-                for (int t = 0; t < kT; ++t) {
-                    uint32_t a0, a1, a2, a3;
-                    ldsm_x4(sbase + k_lane_off + (uint32_t)(t0 + t) * kTileOff + kk * 32, a0, a1, a2, a3);
-                    mma16816(sc[t], a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
+                    for (int t = 0; t < kT; ++t) {
+                        uint32_t a0, a1, a2, a3;
+                        ldsm_x4(sbase + k_lane_off + (uint32_t)(t0 + t) * kTileOff + kk * 32, a0, a1, a2, a3);
+                        mma16816(sc[t], a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
+                    }
+                }
+            } else {
+                // register r: 4 E4M3 keys' dims; r0/r1 tokens 2t/2t+1 at dims
+                // 32j + 4tq.., r2/r3 the same at 32j + 16 + 4tq..
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+#pragma unroll
+                    for (int t = 0; t < kT; ++t) {
+                        uint32_t r[4], lo[4], hi[4];
+                        ldsm_x4(sbase + k_lane_off + (uint32_t)(t0 + t) * kTileOff + j * 32, r[0], r[1], r[2], r[3]);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) e4m3x4_to_f16x4(r[i], lo[i], hi[i]);
+                        mma16816_f16(sc[t], lo[0], lo[1], hi[0], hi[1], qf[2 * j][0], qf[2 * j][1]);
+                        mma16816_f16(sc[t], lo[2], lo[3], hi[2], hi[3], qf[2 * j + 1][0], qf[2 * j + 1][1]);
+                    }
                 }
             }
             // (slot gr, token 2t): heads 2tq, 2tq+1 in sc[t][0..1]; token 2t+1 in sc[t][2..3]
@@ -420,8 +486,8 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, AttnCfg<HKV>::kMinCtas
                 lm0 = fmaxf(lm0, fmaxf(sc[t][0], sc[t][2]));
                 lm1 = fmaxf(lm1, fmaxf(sc[t][1], sc[t][3]));
             }
-            lm0 *= p.scale_log2;
-            lm1 *= p.scale_log2;
+            lm0 *= sl2;
+            lm1 *= sl2;
             // Lazy rescaling: the reference max of a head column moves only when a
             // score exceeds it by more than kRescale (log2 units), so unscaled
             // probabilities stay below 2^kRescale; otherwise no max reduction and
@@ -452,22 +518,43 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, AttnCfg<HKV>::kMinCtas
             uint32_t pb[kT][2];
 #pragma unroll
             for (int t = 0; t < kT; ++t) {
-                const float p0 = exp2f(fmaf(sc[t][0], p.scale_log2, nmu0));
-                const float p1 = exp2f(fmaf(sc[t][1], p.scale_log2, nmu1));
-                const float p2 = exp2f(fmaf(sc[t][2], p.scale_log2, nmu0));
-                const float p3 = exp2f(fmaf(sc[t][3], p.scale_log2, nmu1));
+                const float p0 = exp2f(fmaf(sc[t][0], sl2, nmu0));
+                const float p1 = exp2f(fmaf(sc[t][1], sl2, nmu1));
+                const float p2 = exp2f(fmaf(sc[t][2], sl2, nmu0));
+                const float p3 = exp2f(fmaf(sc[t][3], sl2, nmu1));
                 lrow[0] += p0 + p2;
                 lrow[1] += p1 + p3;
-                pb[t][0] = movm_t(pack_bf16(p0, p1));
-                pb[t][1] = movm_t(pack_bf16(p2, p3));
+                pb[t][0] = movm_t(KV8 ? pack_f16(p0, p1) : pack_bf16(p0, p1));
+                pb[t][1] = movm_t(KV8 ? pack_f16(p2, p3) : pack_bf16(p2, p3));
             }
+            if constexpr (KV8) {
+                // transposed E4M3 V: register r holds (block 2tq, dims d, d + 1)
+                // and (block 2tq + 1, dims d, d + 1), d = 2gr of its 16-byte
+                // column; pairing bytes (0, 2) and (1, 3) gives the A rows of
+                // dims d and d + 1 (output rows gr <-> dim 16 mt + 2gr,
+                // gr + 8 <-> 16 mt + 2gr + 1)
 #pragma unroll
-            for (int mt = 0; mt < 8; ++mt) {
+                for (int c2 = 0; c2 < 4; ++c2) {
 #pragma unroll
-                for (int t = 0; t < kT; ++t) {
-                    uint32_t a0, a1, a2, a3;
-                    ldsm_x4_t(sbase + v_lane_off + (uint32_t)(t0 + t) * kTileOff + mt * 32, a0, a1, a2, a3);
-                    mma16816(o[mt], a0, a1, a2, a3, pb[t][0], pb[t][1]);
+                    for (int t = 0; t < kT; ++t) {
+                        uint32_t r[4], a[8];
+                        ldsm_x4_t(sbase + v_lane_off + (uint32_t)(t0 + t) * kTileOff + c2 * 32, r[0], r[1], r[2],
+                                  r[3]);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) e4m3x4_to_f16x4(__byte_perm(r[i], 0u, 0x3120), a[2 * i], a[2 * i + 1]);
+                        mma16816_f16(o[2 * c2], a[0], a[1], a[2], a[3], pb[t][0], pb[t][1]);
+                        mma16816_f16(o[2 * c2 + 1], a[4], a[5], a[6], a[7], pb[t][0], pb[t][1]);
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int mt = 0; mt < 8; ++mt) {
+#pragma unroll
+                    for (int t = 0; t < kT; ++t) {
+                        uint32_t a0, a1, a2, a3;
+                        ldsm_x4_t(sbase + v_lane_off + (uint32_t)(t0 + t) * kTileOff + mt * 32, a0, a1, a2, a3);
+                        mma16816(o[mt], a0, a1, a2, a3, pb[t][0], pb[t][1]);
+                    }
                 }
             }
             __syncwarp();
@@ -547,16 +634,19 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, AttnCfg<HKV>::kMinCtas
                     }
             }
             const float l[2] = {lrow[0], lrow[1]}, m[2] = {mrow[0], mrow[1]};
-            const float inv0 = l[0] > 0.f ? 1.f / l[0] : 0.f, inv1 = l[1] > 0.f ? 1.f / l[1] : 0.f;
+            const float vsc = KV8 ? p.v_scale : 1.f;
+            const float inv0 = l[0] > 0.f ? vsc / l[0] : 0.f, inv1 = l[1] > 0.f ? vsc / l[1] : 0.f;
+            // output rows gr / gr + 8 of m-tile mt are dims 16 mt + gr / + 8 (FP8 V: 16 mt + 2gr / + 1)
+            const int dr0 = KV8 ? 2 * gr : gr, dr1 = KV8 ? 2 * gr + 1 : gr + 8;
             if (!p.decode) {
 #pragma unroll
                 for (int mt = 0; mt < 8; ++mt) {
                     const float r0 = o[mt][0] * inv0, r1 = o[mt][1] * inv1;
                     const float r2 = o[mt][2] * inv0, r3 = o[mt][3] * inv1;
-                    sm.obuf[g][2 * tq][16 * mt + gr] = __float2bfloat16_rn(r0);
-                    sm.obuf[g][2 * tq + 1][16 * mt + gr] = __float2bfloat16_rn(r1);
-                    sm.obuf[g][2 * tq][16 * mt + gr + 8] = __float2bfloat16_rn(r2);
-                    sm.obuf[g][2 * tq + 1][16 * mt + gr + 8] = __float2bfloat16_rn(r3);
+                    sm.obuf[g][2 * tq][16 * mt + dr0] = __float2bfloat16_rn(r0);
+                    sm.obuf[g][2 * tq + 1][16 * mt + dr0] = __float2bfloat16_rn(r1);
+                    sm.obuf[g][2 * tq][16 * mt + dr1] = __float2bfloat16_rn(r2);
+                    sm.obuf[g][2 * tq + 1][16 * mt + dr1] = __float2bfloat16_rn(r3);
                 }
                 __syncwarp();
                 const int64_t qi = (int64_t)it.seq * p.n_q + it.row;
@@ -577,10 +667,10 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, AttnCfg<HKV>::kMinCtas
                 float *po = p.part_o + (pi * Cfg::kHq + 8 * g) * 128;
 #pragma unroll
                 for (int mt = 0; mt < 8; ++mt) {
-                    po[(2 * tq) * 128 + 16 * mt + gr] = o[mt][0] * inv0;
-                    po[(2 * tq + 1) * 128 + 16 * mt + gr] = o[mt][1] * inv1;
-                    po[(2 * tq) * 128 + 16 * mt + gr + 8] = o[mt][2] * inv0;
-                    po[(2 * tq + 1) * 128 + 16 * mt + gr + 8] = o[mt][3] * inv1;
+                    po[(2 * tq) * 128 + 16 * mt + dr0] = o[mt][0] * inv0;
+                    po[(2 * tq + 1) * 128 + 16 * mt + dr0] = o[mt][1] * inv1;
+                    po[(2 * tq) * 128 + 16 * mt + dr1] = o[mt][2] * inv0;
+                    po[(2 * tq + 1) * 128 + 16 * mt + dr1] = o[mt][3] * inv1;
                 }
                 if (gr == 0) {
 #pragma unroll
@@ -764,9 +854,9 @@ int attn_tail_blocks(bool indexshare, int max_draft) {
 
 namespace {
 
-template <int HKV>
+template <int HKV, bool KV8>
 cudaError_t run_bf16(const AttnArgs &a, void *ws, unsigned *status, cudaStream_t s) {
-    using Cfg = AttnCfg<HKV>;
+    using Cfg = AttnCfg<HKV, KV8>;
     const DeviceInfo *di = device_info();
     const int sms = di ? di->sm_count : 148;
     AttnParams p{};
@@ -790,6 +880,8 @@ cudaError_t run_bf16(const AttnArgs &a, void *ws, unsigned *status, cudaStream_t
     p.max_draft = a.max_draft;
     p.dense = a.decode && a.dense ? 1 : 0;
     p.pg = a.pg;
+    p.k_scale = a.k_scale;
+    p.v_scale = a.v_scale;
     // entries of one item's list: top_k blocks + the tail blocks (dense: every block of the cache)
     const int list_max = p.dense ? (int)(a.kv_stride / kBlock + 1)
                                  : a.top_k + attn_tail_blocks(a.decode && a.cap_len, a.max_draft);
@@ -811,9 +903,9 @@ cudaError_t run_bf16(const AttnArgs &a, void *ws, unsigned *status, cudaStream_t
     // an item's list holds at most top_k ids plus the tail block
     p.sel_cap = p.dense ? 4 : (a.top_k + 3) & ~3;                  // dense: no id list, no stage tables
     p.nst_cap = p.dense ? 1 : (list_max + AT_BPS - 1) / AT_BPS;
-    const size_t smem = attn_smem_bytes<HKV>(p.sel_cap, p.nst_cap);
+    const size_t smem = attn_smem_bytes<HKV, KV8>(p.sel_cap, p.nst_cap);
     if (di && smem > di->smem_optin) return cudaErrorInvalidValue;
-    auto kern = p.pg.table ? attn_bf16_kernel<HKV, true> : attn_bf16_kernel<HKV, false>;
+    auto kern = p.pg.table ? attn_bf16_kernel<HKV, true, KV8> : attn_bf16_kernel<HKV, false, KV8>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
@@ -852,9 +944,9 @@ size_t attn_dense_decode_ws_bytes(int B, int Hq, int d, int64_t kv_stride) {
 
 cudaError_t launch_attn_bf16(const AttnArgs &a, void *ws, unsigned *status, cudaStream_t s) {
     switch (a.Hkv) {
-    case 1: return run_bf16<1>(a, ws, status, s);
-    case 2: return run_bf16<2>(a, ws, status, s);
-    case 4: return run_bf16<4>(a, ws, status, s);
+    case 1: return a.kv8 ? run_bf16<1, true>(a, ws, status, s) : run_bf16<1, false>(a, ws, status, s);
+    case 2: return a.kv8 ? run_bf16<2, true>(a, ws, status, s) : run_bf16<2, false>(a, ws, status, s);
+    case 4: return a.kv8 ? run_bf16<4, true>(a, ws, status, s) : run_bf16<4, false>(a, ws, status, s);
     default: return cudaErrorInvalidValue;
     }
 }

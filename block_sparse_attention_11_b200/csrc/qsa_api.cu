@@ -406,6 +406,55 @@ int qsa_rope_apply(void *x, int32_t B, int64_t n, int32_t H, int32_t d, int64_t 
                                          static_cast<cudaStream_t>(stream)));
 }
 
+// ---------------------------------------------------------------- FP8 K/V caches
+
+namespace {
+int kv8_checks(const void *q, const void *k, const void *v, const int32_t *sel, const int32_t *nsel, int32_t B,
+               int32_t Hq, int32_t Hkv, int32_t d, int32_t top_k, float scale, float k_scale, float v_scale,
+               const void *out) {
+    int st = attn_common_checks(q, k, v, sel, nsel, B, Hq, Hkv, d, top_k, scale, out, QSA_BF16);
+    if (st != QSA_OK) return st;
+    if (!(k_scale > 0.f) || !std::isfinite(k_scale) || !(v_scale > 0.f) || !std::isfinite(v_scale))
+        return QSA_ERR_INVALID_ARG;
+    return QSA_OK;
+}
+}  // namespace
+
+int qsa_sparse_attn_prefill_kv8(const void *q, const void *k, const void *v, float k_scale, float v_scale,
+                                const int32_t *sel, const int32_t *nsel, int32_t B, int64_t n_q, int64_t q0,
+                                int64_t kv_stride, int32_t Hq, int32_t Hkv, int32_t d, int32_t top_k, float scale,
+                                void *out, float *lse, void *stream) {
+    int st = kv8_checks(q, k, v, sel, nsel, B, Hq, Hkv, d, top_k, scale, k_scale, v_scale, out);
+    if (st != QSA_OK) return st;
+    if (n_q < 0 || q0 < 0 || kv_stride < q0 + n_q) return QSA_ERR_INVALID_ARG;
+    if (n_q == 0) return QSA_OK;
+    const DeviceInfo *di = nullptr;
+    if ((st = check_device(&di)) != QSA_OK) return st;
+    AttnArgs a{q, k, v, sel, nsel, nullptr, B, n_q, q0, kv_stride, Hq, Hkv, d, top_k, scale, out, lse, false};
+    a.kv8 = true;
+    a.k_scale = k_scale;
+    a.v_scale = v_scale;
+    return cuda_status(launch_attn_bf16(a, nullptr, di->status, static_cast<cudaStream_t>(stream)));
+}
+
+int qsa_sparse_attn_decode_kv8(const void *q, const void *k, const void *v, float k_scale, float v_scale,
+                               const int32_t *seq_len, const int32_t *sel, const int32_t *nsel, int32_t B,
+                               int64_t kv_stride, int32_t Hq, int32_t Hkv, int32_t d, int32_t top_k, float scale,
+                               void *out, float *lse, void *workspace, size_t ws_bytes, void *stream) {
+    int st = kv8_checks(q, k, v, sel, nsel, B, Hq, Hkv, d, top_k, scale, k_scale, v_scale, out);
+    if (st != QSA_OK) return st;
+    if (!seq_len || kv_stride < 1) return QSA_ERR_INVALID_ARG;
+    const DeviceInfo *di = nullptr;
+    if ((st = check_device(&di)) != QSA_OK) return st;
+    const size_t need = attn_decode_ws_bytes(B, Hq, d, top_k);
+    if (!workspace || ws_bytes < need) return QSA_ERR_WORKSPACE;
+    AttnArgs a{q, k, v, sel, nsel, seq_len, B, 1, 0, kv_stride, Hq, Hkv, d, top_k, scale, out, lse, true};
+    a.kv8 = true;
+    a.k_scale = k_scale;
+    a.v_scale = v_scale;
+    return cuda_status(launch_attn_bf16(a, workspace, di->status, static_cast<cudaStream_t>(stream)));
+}
+
 // ---------------------------------------------------------------- paged caches
 
 namespace {

@@ -361,6 +361,33 @@ QSA_API int qsa_sparse_attn_decode_noalloc(const void *q, const void *k, const v
                                            float *lse, int32_t dtype, void *stream);
 
 /* ========================================================================= */
+/* FP8 K/V caches                                                             */
+/* ========================================================================= */
+/*
+ * Page "Qwen3.8-Flash-Next, Layer by Layer", section "Serving it": with an
+ * FP8 cache the QSA keys and values take 12 KiB per token, and the serving
+ * recipe there runs with an FP8 KV cache.  The pages give no scaling
+ * scheme; here the caches hold FP8 E4M3 bytes with one scale per tensor
+ * (K = k_scale * stored value, V = v_scale * stored value, the engines'
+ * per-tensor form), q and out stay BF16.  Scores use the exact products of
+ * the BF16 query and the dequantized keys (FP16 tensor-core MMAs, the query
+ * scaled by a power of two), probabilities are rounded to FP16 for the value
+ * MMAs.  As qsa_sparse_attn_prefill / qsa_sparse_attn_decode otherwise
+ * (Hq = 8 Hkv, Hkv in {1, 2, 4}, d = 128); k, v are [B][kv_stride][Hkv][d]
+ * bytes; k_scale, v_scale finite and > 0.  Decode workspace as
+ * qsa_sparse_attn_decode_workspace(..., QSA_BF16).
+ */
+QSA_API int qsa_sparse_attn_prefill_kv8(const void *q, const void *k, const void *v, float k_scale, float v_scale,
+                                        const int32_t *sel, const int32_t *nsel, int32_t B, int64_t n_q, int64_t q0,
+                                        int64_t kv_stride, int32_t Hq, int32_t Hkv, int32_t d, int32_t top_k,
+                                        float scale, void *out, float *lse, void *stream);
+QSA_API int qsa_sparse_attn_decode_kv8(const void *q, const void *k, const void *v, float k_scale, float v_scale,
+                                       const int32_t *seq_len, const int32_t *sel, const int32_t *nsel, int32_t B,
+                                       int64_t kv_stride, int32_t Hq, int32_t Hkv, int32_t d, int32_t top_k,
+                                       float scale, void *out, float *lse, void *workspace, size_t ws_bytes,
+                                       void *stream);
+
+/* ========================================================================= */
 /* Paged caches (decode)                                                      */
 /* ========================================================================= */
 /*

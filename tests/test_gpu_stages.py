@@ -205,6 +205,76 @@ def test_attention_stage_isolated_on_oracle_selection(qsa):
         assert np.abs(lse[0].cpu().numpy() - ref["lse"]).max() <= (1e-3 if dtype == "bf16" else 1e-4)
 
 
+def _to_e4m3(t):
+    """Per-tensor FP8 E4M3 cache of t (scale = amax / 448) and its scale."""
+    scale = float(t.float().abs().max()) / 448.0
+    return (t.float() / scale).to(torch.float8_e4m3fn), scale
+
+
+@pytest.mark.parametrize("Hq,Hkv,T,top_k", [(16, 2, 2500, 96), (8, 1, 1031, 64), (32, 4, 777, 32), (16, 2, 7, 4)])
+def test_attention_fp8_kv_prefill_on_oracle_selection(qsa, Hq, Hkv, T, top_k):
+    """FP8 E4M3 K/V caches (per-tensor scales): the GPU attention on the
+    oracle's selection equals the oracle's attention over the dequantized
+    K/V within the BF16 tolerance."""
+    w = W(T, top_k=top_k, Hq=Hq, Hkv=Hkv, seed=34 + Hq)
+    x = workloads.make_prefill(w, device=DEV)
+    k8, ks = _to_e4m3(x["k"])
+    v8, vs = _to_e4m3(x["v"] * 3.0)
+    kd = k8.float() * ks
+    vd = v8.float() * vs
+    rows = list(range(T))
+    kp = oracle.pool_keys(np32(x["k_idx"][0]))
+    ref = oracle.prefill_rows(rows, q_idx=np32(x["q_idx"][0]), k_pool=kp, top_k=top_k, q=np32(x["q"][0]),
+                              k=kd[0].cpu().numpy(), v=vd[0].cpu().numpy(), Hq=Hq, Hkv=Hkv, d=128)
+    sel = torch.from_numpy(ref["sel"][None]).to(DEV)
+    nsel = torch.from_numpy(ref["nsel"][None]).to(DEV)
+    out = torch.empty_like(x["q"])
+    lse = torch.empty(1, T, Hq, dtype=torch.float32, device=DEV)
+    qsa.qsa_sparse_attn_prefill_kv8(x["q"], k8, v8, ks, vs, sel, nsel, out, lse=lse)
+    qsa.qsa_check_status()
+    err = np.abs(np32(out[0]) - ref["out"]).max()
+    assert err <= TOL["bf16"] * 3, err          # outputs scaled by 3: the bf16 rounding of |o| <= 3 max|v|
+    assert np.abs(lse[0].cpu().numpy() - ref["lse"]).max() <= 1e-3
+
+
+@pytest.mark.parametrize("B,L", [(6, 20000), (3, 70001), (5, 2)])
+def test_attention_fp8_kv_decode(qsa, B, L):
+    """Decode attention over FP8 K/V caches against the oracle's decode step
+    on the dequantized caches (same compressed keys, so the same selection)."""
+    w = workloads.Workload("dec_kv8", "decode", B, L, 256, 16, 2, 128, "bf16", 80)
+    x = workloads.make_decode(w, device=DEV, ragged=True)
+    rope = rope_of(w)
+    lens = x["lens"]
+    k8, ks = _to_e4m3(x["k"])
+    v8, vs = _to_e4m3(x["v"])
+    cap = max(lens) // 4 + 2
+    k_pool = torch.zeros(B, cap, 128, dtype=torch.bfloat16, device=DEV)
+    sel = torch.empty(B, w.top_k, dtype=torch.int32, device=DEV)
+    nsel = torch.empty(B, dtype=torch.int32, device=DEV)
+    # compressed keys of all L + 1 keys (the new token's block included) by prefill pooling
+    for b in range(B):
+        kp = torch.zeros(1, cap, 128, dtype=torch.bfloat16, device=DEV)
+        full = torch.cat([x["k_idx"][b, :lens[b]], x["k_idx_new"][b:b + 1]], 0)[None].contiguous()
+        qsa.qsa_pool_keys_prefill(full, kp, rope=rope)
+        k_pool[b] = kp[0]
+    qsa.qsa_index_topk_decode(x["q_idx"], k_pool, x["seq_len"], sel, nsel, top_k=w.top_k, rope=rope)
+    out = torch.empty_like(x["q"])
+    lse = torch.empty(B, 16, dtype=torch.float32, device=DEV)
+    qsa.qsa_sparse_attn_decode_kv8(x["q"], k8, v8, ks, vs, x["seq_len"], sel, nsel, out, lse=lse)
+    qsa.qsa_check_status()
+    kd, vd = k8.float() * ks, v8.float() * vs
+    for b in range(B):
+        s = lens[b] + 1
+        ref = oracle.decode(np32(x["q_idx"][b:b + 1]), np32(k_pool[b])[None], [s], q=np32(x["q"][b:b + 1]),
+                            k=kd[b:b + 1].cpu().numpy(), v=vd[b:b + 1].cpu().numpy(), top_k=w.top_k)
+        if not np.array_equal(sel[b].cpu().numpy(), ref["sel"][0]):
+            gap = (ref["kth"][0] - ref["next"][0]) / max(abs(ref["kth"][0]), 1e-30)
+            assert gap < 1e-4, f"seq {b}: selection differs with gap {gap}"
+            continue
+        assert np.abs(np32(out[b]) - ref["out"][0]).max() <= TOL["bf16"], b
+        assert np.abs(lse[b].cpu().numpy() - ref["lse"][0]).max() <= 1e-3
+
+
 def test_attention_flags_out_of_range_ids(qsa):
     """A selection id outside [0, nb(t)) is skipped and reported through the
     status word (no trap)."""

@@ -66,6 +66,14 @@ WORKLOADS = {
                                          "bf16", 1003, extra={"keys": "fp8"}),
     "decode_b8_l1m_scale4_fp8keys": Workload("decode_b8_l1m_scale4_fp8keys", "decode", 8, 1048576, 512, 16, 2,
                                              128, "bf16", 1005, pos_scale=4.0, extra={"keys": "fp8"}),
+    # FP8 serving configuration: FP8 E4M3 compressed keys and FP8 E4M3 K/V caches (per-tensor scales)
+    "decode_b64_l128k_fp8": Workload("decode_b64_l128k_fp8", "decode", 64, 131072, 512, 16, 2, 128, "bf16", 1003,
+                                     extra={"keys": "fp8", "kv": "fp8"}),
+    "decode_b8_l1m_scale4_fp8": Workload("decode_b8_l1m_scale4_fp8", "decode", 8, 1048576, 512, 16, 2, 128, "bf16",
+                                         1005, pos_scale=4.0, extra={"keys": "fp8", "kv": "fp8"}),
+    # the 32K prefill workload with FP8 E4M3 K/V caches
+    "prefill_t32k_needles_kv8": Workload("prefill_t32k_needles_kv8", "prefill", 1, 32768, 512, 16, 2, 128, "bf16",
+                                         1002, needles=64, extra={"kv": "fp8"}),
     # the 128K decode workload over paged caches (64-token pages, shuffled page pool)
     "decode_b64_l128k_paged": Workload("decode_b64_l128k_paged", "decode", 64, 131072, 512, 16, 2, 128, "bf16",
                                        1003, extra={"page_tokens": 64}),
@@ -77,6 +85,13 @@ WORKLOADS = {
     "draft_b64_l128k": Workload("draft_b64_l128k", "draft", 64, 131072, 512, 16, 2, 128, "bf16", 1006,
                                 extra={"drafted": 3, "max_draft": 4}),
 }
+
+
+def to_e4m3(t: torch.Tensor):
+    """A per-tensor FP8 E4M3 cache of t: (values / scale) rounded to E4M3, and
+    scale = amax / 448, so that scale * cache approximates t."""
+    scale = float(t.float().abs().max()) / 448.0
+    return (t.float() / scale).to(torch.float8_e4m3fn), scale
 
 
 def torch_dtype(w: Workload):
