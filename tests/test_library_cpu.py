@@ -111,6 +111,13 @@ def test_invalid_arguments_are_rejected_before_launch(qsa):
     assert lib.qsa_sparse_attn_decode_paged(fake, fake, fake, pg, fake, fake, fake, 1, 16, 2, 128, 64, 0.1, fake,
                                             None, fake, 1 << 20, 1, None) == qsa.QSA_ERR_UNSUPPORTED
     assert lib.qsa_index_topk_decode_kernels(0, 100, 0, 0) == 0
+    # FP8 K/V attention: scales must be finite and positive; bf16 shapes only (GQA 8)
+    assert lib.qsa_sparse_attn_prefill_kv8(fake, fake, fake, 0.0, 1.0, fake, fake, 1, 4, 0, 4, 16, 2, 128, 8, 0.1,
+                                           fake, None, None) == qsa.QSA_ERR_INVALID_ARG
+    assert lib.qsa_sparse_attn_decode_kv8(fake, fake, fake, 1.0, float("inf"), fake, fake, fake, 1, 64, 16, 2, 128,
+                                          8, 0.1, fake, None, fake, 1 << 20, None) == qsa.QSA_ERR_INVALID_ARG
+    assert lib.qsa_sparse_attn_prefill_kv8(fake, fake, fake, 1.0, 1.0, fake, fake, 1, 4, 0, 4, 12, 4, 128, 8, 0.1,
+                                           fake, None, None) == qsa.QSA_ERR_UNSUPPORTED
     # misaligned pointer
     odd = ctypes.c_void_p(4098)
     assert lib.qsa_pool_keys_prefill(odd, fake, 1, 16, 0, 16, 4, rope, 0, 0, None) == qsa.QSA_ERR_INVALID_ARG
