@@ -287,6 +287,31 @@ __device__ __forceinline__ void wsel_load4(const float *row, int n, int base, ui
     }
 }
 
+// Four consecutive 128-element chunks [base + 128u, +128), u < 4: the four
+// 16-byte loads are issued before any key is used, so each lane keeps four
+// loads in flight (one at a time left the row passes latency-bound).
+__device__ __forceinline__ void wsel_load4x4(const float *row, int n, int base, uint32_t (&key)[4][4],
+                                             bool (&live)[4][4]) {
+    const int lane = threadIdx.x & 31;
+    float4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int i = base + 128 * u + 4 * lane;
+        v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (i < n) v[u] = *reinterpret_cast<const float4 *>(row + i);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int i = base + 128 * u + 4 * lane;
+        const float f[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            live[u][c] = i + c < n;
+            key[u][c] = score_key(f[c]);
+        }
+    }
+}
+
 // Top-k of one row; emit(pos, i) in ascending i.  Returns the count.  Whole warp.
 template <typename Emit>
 __device__ __forceinline__ int warp_topk_row(const float *row, int n, int k, WarpSelSmem &w, Emit &&emit) {
@@ -298,12 +323,14 @@ __device__ __forceinline__ int warp_topk_row(const float *row, int n, int k, War
     }
     // ---- pass 1: top 11 bits
     wsel_clear(w, 2048);
-    for (int base = 0; base < n; base += 128) {
-        uint32_t key[4];
-        bool live[4];
-        wsel_load4(row, n, base, key, live);
+    for (int base = 0; base < n; base += 512) {
+        uint32_t key[4][4];
+        bool live[4][4];
+        wsel_load4x4(row, n, base, key, live);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) wsel_add(w, live[c], key[c] >> 21);
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) wsel_add(w, live[u][c], key[u][c] >> 21);
     }
     __syncwarp();
     int k_rem = k;
@@ -311,20 +338,22 @@ __device__ __forceinline__ int warp_topk_row(const float *row, int n, int k, War
     uint32_t prefix = d1 << 21, pmask = 0xFFE00000u;
     // ---- pass 2: gather the bin's keys
     int cnt = 0;
-    for (int base = 0; base < n; base += 128) {
-        uint32_t key[4];
-        bool live[4];
-        wsel_load4(row, n, base, key, live);
+    for (int base = 0; base < n; base += 512) {
+        uint32_t key[4][4];
+        bool live[4][4];
+        wsel_load4x4(row, n, base, key, live);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const bool hit = live[c] && (key[c] & pmask) == prefix;
-            const uint32_t bal = __ballot_sync(0xffffffffu, hit);
-            if (hit) {
-                const int slot = cnt + __popc(bal & lt);
-                if (slot < kWarpSelBuf) w.buf[slot] = key[c];
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const bool hit = live[u][c] && (key[u][c] & pmask) == prefix;
+                const uint32_t bal = __ballot_sync(0xffffffffu, hit);
+                if (hit) {
+                    const int slot = cnt + __popc(bal & lt);
+                    if (slot < kWarpSelBuf) w.buf[slot] = key[u][c];
+                }
+                cnt += __popc(bal);
             }
-            cnt += __popc(bal);
-        }
     }
     __syncwarp();
     const bool small = cnt <= kWarpSelBuf;
@@ -359,46 +388,52 @@ __device__ __forceinline__ int warp_topk_row(const float *row, int n, int k, War
     const int take_eq = k_rem;
     // ---- pass 3: ordered emission
     int out_run = 0, eq_run = 0;
-    for (int base = 0; base < n; base += 128) {
-        uint32_t key[4];
-        bool live[4];
-        wsel_load4(row, n, base, key, live);
-        int ngt = 0, neq = 0;
+    for (int base4 = 0; base4 < n; base4 += 512) {
+        uint32_t key4[4][4];
+        bool live4[4][4];
+        wsel_load4x4(row, n, base4, key4, live4);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            ngt += live[c] && key[c] > kstar;
-            neq += live[c] && key[c] == kstar;
+        for (int u = 0; u < 4; ++u) {
+            const int base = base4 + 128 * u;
+            const uint32_t(&key)[4] = key4[u];
+            const bool(&live)[4] = live4[u];
+            int ngt = 0, neq = 0;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                ngt += live[c] && key[c] > kstar;
+                neq += live[c] && key[c] == kstar;
+            }
+            // exclusive prefix of equal keys over lanes (lane order = element order)
+            int eq_incl = neq;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, eq_incl, o);
+                if (lane >= o) eq_incl += v;
+            }
+            int eq_before = eq_run + eq_incl - neq;
+            int nsel = 0;
+            bool sel[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const bool gt = live[c] && key[c] > kstar;
+                const bool eq = live[c] && key[c] == kstar;
+                sel[c] = gt || (eq && eq_before < take_eq);
+                eq_before += eq;
+                nsel += sel[c];
+            }
+            int sel_incl = nsel;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, sel_incl, o);
+                if (lane >= o) sel_incl += v;
+            }
+            int pos = out_run + sel_incl - nsel;
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                if (sel[c]) emit(pos++, base + 4 * lane + c);
+            out_run += __shfl_sync(0xffffffffu, sel_incl, 31);
+            eq_run += __shfl_sync(0xffffffffu, eq_incl, 31);
         }
-        // exclusive prefix of equal keys over lanes (lane order = element order)
-        int eq_incl = neq;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, eq_incl, o);
-            if (lane >= o) eq_incl += v;
-        }
-        int eq_before = eq_run + eq_incl - neq;
-        int nsel = 0;
-        bool sel[4];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const bool gt = live[c] && key[c] > kstar;
-            const bool eq = live[c] && key[c] == kstar;
-            sel[c] = gt || (eq && eq_before < take_eq);
-            eq_before += eq;
-            nsel += sel[c];
-        }
-        int sel_incl = nsel;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, sel_incl, o);
-            if (lane >= o) sel_incl += v;
-        }
-        int pos = out_run + sel_incl - nsel;
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-            if (sel[c]) emit(pos++, base + 4 * lane + c);
-        out_run += __shfl_sync(0xffffffffu, sel_incl, 31);
-        eq_run += __shfl_sync(0xffffffffu, eq_incl, 31);
     }
     (void)lt;
     return out_run;
