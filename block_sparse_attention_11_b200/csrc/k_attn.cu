@@ -62,23 +62,30 @@ constexpr uint32_t kFullStage = 0x924924u;   // 8 slots x 3 bits, each holding 4
 #endif
 
 // KV8: K/V caches of FP8 E4M3 values (times per-tensor scales), 1 byte per element.
-template <int HKV, bool KV8 = false> struct AttnCfg {
-    // Consumer warp (g, sub): kv head g; sub = u * 2 + hf takes the stages whose
-    // global index is = hf (mod 2), and tiles [u * kTiles, (u + 1) * kTiles) of each.
-    static constexpr int kTiles = HKV == 4 ? 2 : QSA_ATTN_TILES;
-    static constexpr int kU = 2 / kTiles;          // warps sharing one stage of one kv head
-    static constexpr int kWph = 2 * kU;            // consumer warps per kv head
-    static constexpr int kConsumers = kWph * HKV;
-    static constexpr int kMinCtas = HKV == 4 ? 1 : QSA_ATTN_CTAS;   // launch-bounds residency target
+// D: head dim (128 or 256).  G: q heads per kv head (8, or 12 for the released
+// 24q/2kv shape: two 8-head MMA column tiles, the second one half padding).
+template <int HKV, bool KV8 = false, int D = 128, int G = 8> struct AttnCfg {
+    static constexpr int kD = D, kG = G;
+    static constexpr int kNT = (G + 7) / 8;        // 8-head column tiles per kv head
+    static constexpr int kMT = D / 16;             // 16-dim MMA k-steps (QK) and m-tiles (PV)
+    // Consumer warp (grp, sub): group grp = kv head g, column tile nt; sub = u * 2
+    // + hf takes the stages whose global index is = hf (mod 2), and tiles
+    // [u * kTiles, (u + 1) * kTiles) of each.
+    static constexpr int kTiles = (HKV == 4 || D > 128) ? 2 : QSA_ATTN_TILES;
+    static constexpr int kU = 2 / kTiles;          // warps sharing one stage of one group
+    static constexpr int kWph = 2 * kU;            // consumer warps per group
+    static constexpr int kGroups = HKV * kNT;
+    static constexpr int kConsumers = kWph * kGroups;
+    static constexpr int kMinCtas = (HKV == 4 || D > 128) ? 1 : QSA_ATTN_CTAS;   // launch-bounds residency target
     static constexpr int kPw = QSA_ATTN_PW;
     static constexpr int kThreads = (kConsumers + kPw) * 32;
     static constexpr int kEl = KV8 ? 1 : 2;                    // bytes per K/V element
-    static constexpr int kTokBytes = HKV * 128 * kEl;          // one token, all kv heads
+    static constexpr int kTokBytes = HKV * D * kEl;            // one token, all kv heads
     static constexpr int kSpan = kBlock * kTokBytes;           // bytes of one block, all kv heads
     static constexpr int kSlot = kSpan + 16;                   // padded slot
     static constexpr int kStage = 2 * AT_BPS * kSlot;          // K slots then V slots
-    static constexpr int kHq = 8 * HKV;
-    static constexpr int kQBytes = kHq * 128 * 2;
+    static constexpr int kHq = G * HKV;
+    static constexpr int kQBytes = kHq * D * 2;
     static constexpr int kNS = QSA_ATTN_NS;
     // Consumer warp hf takes the stages whose global index is = hf (mod 2); with
     // an even number of slots it always uses the same slots, in order, so no
@@ -103,14 +110,14 @@ struct AttnParams {
     int sel_cap, nst_cap;  // shared-memory block-id list and per-stage table sizes (from top_k)
     __nv_bfloat16 *out;
     float *lse;
-    float *part_o;         // decode: [B][splits][Hq][128]
+    float *part_o;         // decode: [B][splits][Hq][D]
     float *part_lse;       // decode: [B][splits][Hq] (log2 domain)
     const int32_t *cap_len;  // decode, IndexShare: [B] capture rows + 1 (null: plain decode)
     int max_draft;           // IndexShare: largest seq_len - cap_len
     int dense;               // decode: every visible block in order (dense causal attention, no selection)
     unsigned *status;
     float k_scale, v_scale;  // KV8: K = k_scale * stored E4M3 value, V = v_scale * stored value
-    Paging pg;               // pg.table: K/V are paged caches [slots][Hkv][128] (kv_stride = table capacity)
+    Paging pg;               // pg.table: K/V are paged caches [slots][Hkv][D] (kv_stride = table capacity)
 };
 
 // The key list of one work item: positions lbeg..lend of
@@ -130,7 +137,7 @@ struct Item {
     const __nv_bfloat16 *qrow;
 };
 
-template <int HKV>
+template <class Cfg>
 __device__ __forceinline__ Item get_item(const AttnParams &p, int64_t i) {
     Item it;
     if (!p.decode) {
@@ -140,14 +147,14 @@ __device__ __forceinline__ Item get_item(const AttnParams &p, int64_t i) {
         const int64_t qi = (int64_t)it.seq * p.n_q + it.row;
         it.sel = p.sel + qi * p.top_k;
         it.nsel = p.nsel[qi];
-        it.qrow = p.q + qi * (int64_t)AttnCfg<HKV>::kHq * 128;
+        it.qrow = p.q + qi * (int64_t)Cfg::kHq * Cfg::kD;
     } else {
         it.seq = (int)(i / p.splits);
         it.row = i % p.splits;
         it.t = (int64_t)p.seq_len[it.seq] - 1;
         it.sel = p.dense ? nullptr : p.sel + (int64_t)it.seq * p.top_k;
         it.nsel = p.dense ? 0 : p.nsel[it.seq];
-        it.qrow = p.q + (int64_t)it.seq * AttnCfg<HKV>::kHq * 128;
+        it.qrow = p.q + (int64_t)it.seq * Cfg::kHq * Cfg::kD;
     }
     if (it.t < 0 || it.t >= p.kv_stride) {
         if (it.t >= p.kv_stride) flag(p.status, QSA_DEV_BAD_LENGTH);
@@ -175,44 +182,47 @@ __device__ __forceinline__ Item get_item(const AttnParams &p, int64_t i) {
     return it;
 }
 
-template <int HKV, bool KV8>
+template <class Cfg>
 struct __align__(128) AttnSmem {
-    using Cfg = AttnCfg<HKV, KV8>;
     uint8_t stage[Cfg::kNS][Cfg::kStage];
     alignas(16) uint8_t qbuf[2][Cfg::kQBytes];
-    float xbuf[HKV][Cfg::kWph - 1][32][36];
-    alignas(16) __nv_bfloat16 obuf[HKV][8][128];
+    float xbuf[Cfg::kGroups][Cfg::kWph - 1][32][4 + 4 * Cfg::kMT];
+    alignas(16) __nv_bfloat16 obuf[Cfg::kGroups][8][Cfg::kD];
     alignas(16) uint32_t info[Cfg::kNS][Cfg::kPw];
     uint64_t full[Cfg::kNS], empty[Cfg::kNS], qfull[2], qempty[2];
-    uint64_t xready[HKV], xdone[HKV];   // merge handshake per kv head
+    uint64_t xready[Cfg::kGroups], xdone[Cfg::kGroups];   // merge handshake per group
     // followed in dynamic shared memory by
     //   int32_t  sel_s[sel_cap]             the current item's block ids (each producer fills its own slots)
     //   uint32_t st_info[kPw][nst_cap]      per stage of the item: token counts of the producer's slots
     //   uint32_t st_bytes[kPw][nst_cap]     per stage of the item: bytes the producer copies per tensor
 };
 
-template <int HKV, bool KV8>
+template <class Cfg>
 size_t attn_smem_bytes(int sel_cap, int nst_cap) {
-    return sizeof(AttnSmem<HKV, KV8>) + (size_t)sel_cap * 4 + 2 * (size_t)AttnCfg<HKV>::kPw * nst_cap * 4 + 128;
+    return sizeof(AttnSmem<Cfg>) + (size_t)sel_cap * 4 + 2 * (size_t)Cfg::kPw * nst_cap * 4 + 128;
 }
 
 // PAGED: K/V are paged caches addressed through p.pg (a separate instantiation,
 // so the contiguous kernels carry none of the page-table code).
-template <int HKV, bool PAGED, bool KV8>
-__global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, AttnCfg<HKV>::kMinCtas) attn_bf16_kernel(AttnParams p) {
-    using Cfg = AttnCfg<HKV, KV8>;
+template <int HKV, int D, int G, bool PAGED, bool KV8>
+__global__ void __launch_bounds__(AttnCfg<HKV, KV8, D, G>::kThreads, AttnCfg<HKV, KV8, D, G>::kMinCtas)
+    attn_bf16_kernel(AttnParams p) {
+    using Cfg = AttnCfg<HKV, KV8, D, G>;
     extern __shared__ uint8_t asm_raw[];
-    AttnSmem<HKV, KV8> &sm =
-        *reinterpret_cast<AttnSmem<HKV, KV8> *>((reinterpret_cast<uintptr_t>(asm_raw) + 127) & ~uintptr_t(127));
+    AttnSmem<Cfg> &sm =
+        *reinterpret_cast<AttnSmem<Cfg> *>((reinterpret_cast<uintptr_t>(asm_raw) + 127) & ~uintptr_t(127));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     // zero the slots once: masked keys must read finite values (0 * NaN = NaN)
     for (int i = threadIdx.x; i < (int)(sizeof(sm.stage) / 16); i += blockDim.x)
         reinterpret_cast<uint4 *>(&sm.stage[0][0])[i] = make_uint4(0, 0, 0, 0);
     if (threadIdx.x == 0) {
-        for (int s = 0; s < Cfg::kNS; ++s) { mbar_init(&sm.full[s], Cfg::kPw); mbar_init(&sm.empty[s], HKV * Cfg::kU); }
+        for (int s = 0; s < Cfg::kNS; ++s) {
+            mbar_init(&sm.full[s], Cfg::kPw);
+            mbar_init(&sm.empty[s], Cfg::kGroups * Cfg::kU);
+        }
         for (int s = 0; s < 2; ++s) { mbar_init(&sm.qfull[s], 1); mbar_init(&sm.qempty[s], Cfg::kConsumers); }
-        for (int s = 0; s < HKV; ++s) { mbar_init(&sm.xready[s], Cfg::kWph - 1); mbar_init(&sm.xdone[s], 1); }
+        for (int s = 0; s < Cfg::kGroups; ++s) { mbar_init(&sm.xready[s], Cfg::kWph - 1); mbar_init(&sm.xdone[s], 1); }
         fence_mbar_init();
     }
     fence_proxy_async_smem();
@@ -235,7 +245,7 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, AttnCfg<HKV>::kMinCtas
         int64_t ic = 0;         // item counter
         bool ok = true;
         for (int64_t i = blockIdx.x; i < p.items && ok; i += gridDim.x, ++ic) {
-            const Item it = get_item<HKV>(p, i);
+            const Item it = get_item<Cfg>(p, i);
             const int id_end = min(it.lend, it.nsel);
             // list entries of this producer's slots: e - lbeg = 8 * st + PW * jj + pw
             // (dense: the ids are the entries themselves, nothing to stage)
@@ -347,8 +357,9 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, AttnCfg<HKV>::kMinCtas
     // of each (tile t = tokens {2t, 2t+1} of the stage's 8 blocks).  Each warp
     // keeps its own online-softmax state; the states of a kv head's warps are
     // merged at the end of an item.
-    constexpr int kT = Cfg::kTiles;
-    const int g = warp / Cfg::kWph;
+    constexpr int kT = Cfg::kTiles, kMT = Cfg::kMT;
+    const int grp = warp / Cfg::kWph;              // group: kv head g, 8-head column tile nt
+    const int g = grp / Cfg::kNT, nt = grp % Cfg::kNT;
     const int sub = warp % Cfg::kWph;
     const int hf = sub & 1;
     const int t0 = (sub >> 1) * kT;
@@ -360,7 +371,7 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, AttnCfg<HKV>::kMinCtas
     // transposed): token + (mi >> 1), 16 bytes + (mi & 1); V (FP8): token +
     // (mi & 1), 16 bytes + (mi >> 1), so registers 0/1 hold the two tokens of
     // one 16-byte column and 2/3 of the next.
-    constexpr int kHead = 128 * Cfg::kEl;            // bytes of one kv head of one token
+    constexpr int kHead = D * Cfg::kEl;              // bytes of one kv head of one token
     const uint32_t k_lane_off =
         (uint32_t)(rr * Cfg::kSlot + (mi & 1) * Cfg::kTokBytes + g * kHead + (mi >> 1) * 16);
     const uint32_t v_lane_off =
@@ -372,19 +383,23 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, AttnCfg<HKV>::kMinCtas
     int64_t it_count = 0, ic = 0;
     bool ok = true;
     for (int64_t i = blockIdx.x; i < p.items && ok; i += gridDim.x, ++ic) {
-        const Item it = get_item<HKV>(p, i);
+        const Item it = get_item<Cfg>(p, i);
         const int qs = (int)(ic & 1);
         ok = mbar_wait(&sm.qfull[qs], (int)((ic >> 1) & 1), p.status);
         if (!ok) break;
-        uint32_t qf[8][2];
+        // this lane's q head (the B column gr of the tile); padding columns of the
+        // last tile (G not a multiple of 8) read zeros and are never written out
+        const int hloc = 8 * nt + gr;
+        const bool hvalid = hloc < G;
+        uint32_t qf[kMT][2];
         float sl2 = p.scale_log2;   // logit scale in log2 units
         if constexpr (!KV8) {
             const uint32_t *qw = reinterpret_cast<const uint32_t *>(sm.qbuf[qs]);
-            const int head = 8 * g + gr;
+            const int head = G * g + hloc;
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                qf[kk][0] = qw[(head * 128 + 16 * kk + 2 * tq) >> 1];
-                qf[kk][1] = qw[(head * 128 + 16 * kk + 8 + 2 * tq) >> 1];
+            for (int kk = 0; kk < kMT; ++kk) {
+                qf[kk][0] = hvalid ? qw[(head * D + 16 * kk + 2 * tq) >> 1] : 0u;
+                qf[kk][1] = hvalid ? qw[(head * D + 16 * kk + 8 + 2 * tq) >> 1] : 0u;
             }
         } else {
             // FP8 keys are scored as FP16 (E4M3 is a subset of FP16); the query
@@ -392,14 +407,14 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, AttnCfg<HKV>::kMinCtas
             // [2^14, 2^15)), in the k order of the widened key fragments:
             // k-step 2j takes dims 32j + 4tq + {0..3}, k-step 2j + 1 dims
             // 32j + 16 + 4tq + {0..3}.
-            const __nv_bfloat16 *qh = reinterpret_cast<const __nv_bfloat16 *>(sm.qbuf[qs]) + (8 * g + gr) * 128;
-            float qv[8][4];
+            const __nv_bfloat16 *qh = reinterpret_cast<const __nv_bfloat16 *>(sm.qbuf[qs]) + (G * g + hloc) * D;
+            float qv[kMT][4];
             float mx = 0.f;
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
+            for (int kk = 0; kk < kMT; ++kk)
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    qv[kk][c] = __bfloat162float(qh[32 * (kk >> 1) + 16 * (kk & 1) + 4 * tq + c]);
+                    qv[kk][c] = hvalid ? __bfloat162float(qh[32 * (kk >> 1) + 16 * (kk & 1) + 4 * tq + c]) : 0.f;
                     mx = fmaxf(mx, fabsf(qv[kk][c]));
                 }
 #pragma unroll
@@ -412,7 +427,7 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, AttnCfg<HKV>::kMinCtas
             }
             const float sc2 = ldexpf(1.0f, qexp);
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
+            for (int kk = 0; kk < kMT; ++kk) {
                 qf[kk][0] = pack_f16(__fmul_rn(qv[kk][0], sc2), __fmul_rn(qv[kk][1], sc2));
                 qf[kk][1] = pack_f16(__fmul_rn(qv[kk][2], sc2), __fmul_rn(qv[kk][3], sc2));
             }
@@ -421,9 +436,9 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, AttnCfg<HKV>::kMinCtas
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.qempty[qs]);
         float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
-        float o[8][4];
+        float o[kMT][4];
 #pragma unroll
-        for (int a = 0; a < 8; ++a) o[a][0] = o[a][1] = o[a][2] = o[a][3] = 0.f;
+        for (int a = 0; a < kMT; ++a) o[a][0] = o[a][1] = o[a][2] = o[a][3] = 0.f;
 
         for (int pos = it.lbeg; pos < it.lend; pos += AT_BPS, ++it_count) {
             if ((int)(it_count & 1) != hf) continue;
@@ -447,7 +462,7 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, AttnCfg<HKV>::kMinCtas
                 for (int c = 0; c < 4; ++c) sc[t][c] = 0.f;
             if constexpr (!KV8) {
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
+                for (int kk = 0; kk < kMT; ++kk) {
 #pragma unroll
                     for (int t = 0; t < kT; ++t) {
                         uint32_t a0, a1, a2, a3;
@@ -459,7 +474,7 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, AttnCfg<HKV>::kMinCtas
                 // register r: 4 E4M3 keys' dims; r0/r1 tokens 2t/2t+1 at dims
                 // 32j + 4tq.., r2/r3 the same at 32j + 16 + 4tq..
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
+                for (int j = 0; j < kMT / 2; ++j) {
 #pragma unroll
                     for (int t = 0; t < kT; ++t) {
                         uint32_t r[4], lo[4], hi[4];
@@ -506,7 +521,7 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, AttnCfg<HKV>::kMinCtas
                 lrow[0] *= al0;
                 lrow[1] *= al1;
 #pragma unroll
-                for (int mt = 0; mt < 8; ++mt) {
+                for (int mt = 0; mt < kMT; ++mt) {
                     o[mt][0] *= al0;
                     o[mt][1] *= al1;
                     o[mt][2] *= al0;
@@ -534,7 +549,7 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, AttnCfg<HKV>::kMinCtas
                 // dims d and d + 1 (output rows gr <-> dim 16 mt + 2gr,
                 // gr + 8 <-> 16 mt + 2gr + 1)
 #pragma unroll
-                for (int c2 = 0; c2 < 4; ++c2) {
+                for (int c2 = 0; c2 < kMT / 2; ++c2) {
 #pragma unroll
                     for (int t = 0; t < kT; ++t) {
                         uint32_t r[4], a[8];
@@ -548,7 +563,7 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, AttnCfg<HKV>::kMinCtas
                 }
             } else {
 #pragma unroll
-                for (int mt = 0; mt < 8; ++mt) {
+                for (int mt = 0; mt < kMT; ++mt) {
 #pragma unroll
                     for (int t = 0; t < kT; ++t) {
                         uint32_t a0, a1, a2, a3;
@@ -569,18 +584,18 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, AttnCfg<HKV>::kMinCtas
         }
         // merge the warps of this kv head: warps sub >= 1 publish, warp 0 folds
         if (sub != 0) {
-            if (ic > 0) ok = mbar_wait(&sm.xdone[g], (int)((ic - 1) & 1), p.status);
+            if (ic > 0) ok = mbar_wait(&sm.xdone[grp], (int)((ic - 1) & 1), p.status);
             if (!ok) break;
-            float *xb = sm.xbuf[g][sub - 1][lane];
+            float *xb = sm.xbuf[grp][sub - 1][lane];
             xb[0] = mrow[0]; xb[1] = mrow[1]; xb[2] = lrow[0]; xb[3] = lrow[1];
 #pragma unroll
-            for (int mt = 0; mt < 8; ++mt)
+            for (int mt = 0; mt < kMT; ++mt)
 #pragma unroll
                 for (int c = 0; c < 4; ++c) xb[4 + 4 * mt + c] = o[mt][c];
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.xready[g]);
+            if (lane == 0) mbar_arrive(&sm.xready[grp]);
         } else {
-            ok = mbar_wait(&sm.xready[g], (int)(ic & 1), p.status);
+            ok = mbar_wait(&sm.xready[grp], (int)(ic & 1), p.status);
             if (!ok) break;
             // Every fold is symmetric in its two operands (explicitly rounded, no
             // contraction), so the result does not depend on which warp of a
@@ -589,7 +604,7 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, AttnCfg<HKV>::kMinCtas
             //   B = fold(sub 2, sub 3)             tiles of group 1 (two groups only)
             //   result = fold(A, B)
             {
-                const float *xb = sm.xbuf[g][0][lane];
+                const float *xb = sm.xbuf[grp][0][lane];
                 float f0[2], f1[2];
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
@@ -602,13 +617,13 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, AttnCfg<HKV>::kMinCtas
                     mrow[c] = mn;
                 }
 #pragma unroll
-                for (int mt = 0; mt < 8; ++mt)
+                for (int mt = 0; mt < kMT; ++mt)
 #pragma unroll
                     for (int c = 0; c < 4; ++c)
                         o[mt][c] = __fadd_rn(__fmul_rn(o[mt][c], f0[c & 1]), __fmul_rn(xb[4 + 4 * mt + c], f1[c & 1]));
             }
             if constexpr (Cfg::kU == 2) {
-                const float *x2 = sm.xbuf[g][1][lane], *x3 = sm.xbuf[g][2][lane];
+                const float *x2 = sm.xbuf[grp][1][lane], *x3 = sm.xbuf[grp][2][lane];
                 float f2[2], f3[2], fa[2], fb[2];
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
@@ -625,7 +640,7 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, AttnCfg<HKV>::kMinCtas
                     mrow[c] = mn;
                 }
 #pragma unroll
-                for (int mt = 0; mt < 8; ++mt)
+                for (int mt = 0; mt < kMT; ++mt)
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
                         const float ob = __fadd_rn(__fmul_rn(x2[4 + 4 * mt + c], f2[c & 1]),
@@ -638,60 +653,66 @@ __global__ void __launch_bounds__(AttnCfg<HKV>::kThreads, AttnCfg<HKV>::kMinCtas
             const float inv0 = l[0] > 0.f ? vsc / l[0] : 0.f, inv1 = l[1] > 0.f ? vsc / l[1] : 0.f;
             // output rows gr / gr + 8 of m-tile mt are dims 16 mt + gr / + 8 (FP8 V: 16 mt + 2gr / + 1)
             const int dr0 = KV8 ? 2 * gr : gr, dr1 = KV8 ? 2 * gr + 1 : gr + 8;
+            // the tile's heads: columns 2tq, 2tq + 1 are heads h0 + 2tq (+1), valid below G
+            const int h0 = G * g + 8 * nt;
+            const int nv = min(8, G - 8 * nt);
+            const bool cv0 = 2 * tq < nv, cv1 = 2 * tq + 1 < nv;
             if (!p.decode) {
 #pragma unroll
-                for (int mt = 0; mt < 8; ++mt) {
+                for (int mt = 0; mt < kMT; ++mt) {
                     const float r0 = o[mt][0] * inv0, r1 = o[mt][1] * inv1;
                     const float r2 = o[mt][2] * inv0, r3 = o[mt][3] * inv1;
-                    sm.obuf[g][2 * tq][16 * mt + dr0] = __float2bfloat16_rn(r0);
-                    sm.obuf[g][2 * tq + 1][16 * mt + dr0] = __float2bfloat16_rn(r1);
-                    sm.obuf[g][2 * tq][16 * mt + dr1] = __float2bfloat16_rn(r2);
-                    sm.obuf[g][2 * tq + 1][16 * mt + dr1] = __float2bfloat16_rn(r3);
+                    sm.obuf[grp][2 * tq][16 * mt + dr0] = __float2bfloat16_rn(r0);
+                    sm.obuf[grp][2 * tq + 1][16 * mt + dr0] = __float2bfloat16_rn(r1);
+                    sm.obuf[grp][2 * tq][16 * mt + dr1] = __float2bfloat16_rn(r2);
+                    sm.obuf[grp][2 * tq + 1][16 * mt + dr1] = __float2bfloat16_rn(r3);
                 }
                 __syncwarp();
                 const int64_t qi = (int64_t)it.seq * p.n_q + it.row;
-                uint4 *dst = reinterpret_cast<uint4 *>(p.out + (qi * Cfg::kHq + 8 * g) * 128);
-                const uint4 *src = reinterpret_cast<const uint4 *>(&sm.obuf[g][0][0]);
-#pragma unroll
-                for (int c = 0; c < 4; ++c) dst[lane + 32 * c] = src[lane + 32 * c];
+                uint4 *dst = reinterpret_cast<uint4 *>(p.out + (qi * Cfg::kHq + h0) * D);
+                const uint4 *src = reinterpret_cast<const uint4 *>(&sm.obuf[grp][0][0]);
+                for (int c = lane; c < nv * D / 8; c += 32) dst[c] = src[c];
                 if (p.lse && gr == 0) {
 #pragma unroll
                     for (int c = 0; c < 2; ++c) {
                         const float v = (l[c] > 0.f) ? (m[c] + log2f(l[c])) / kLog2e : -INFINITY;
-                        p.lse[qi * Cfg::kHq + 8 * g + 2 * tq + c] = v;
+                        if (2 * tq + c < nv) p.lse[qi * Cfg::kHq + h0 + 2 * tq + c] = v;
                     }
                 }
                 __syncwarp();
             } else {
                 const int64_t pi = (int64_t)it.seq * p.splits + it.row;
-                float *po = p.part_o + (pi * Cfg::kHq + 8 * g) * 128;
+                float *po = p.part_o + (pi * Cfg::kHq + h0) * D;
 #pragma unroll
-                for (int mt = 0; mt < 8; ++mt) {
-                    po[(2 * tq) * 128 + 16 * mt + dr0] = o[mt][0] * inv0;
-                    po[(2 * tq + 1) * 128 + 16 * mt + dr0] = o[mt][1] * inv1;
-                    po[(2 * tq) * 128 + 16 * mt + dr1] = o[mt][2] * inv0;
-                    po[(2 * tq + 1) * 128 + 16 * mt + dr1] = o[mt][3] * inv1;
+                for (int mt = 0; mt < kMT; ++mt) {
+                    if (cv0) po[(2 * tq) * D + 16 * mt + dr0] = o[mt][0] * inv0;
+                    if (cv1) po[(2 * tq + 1) * D + 16 * mt + dr0] = o[mt][1] * inv1;
+                    if (cv0) po[(2 * tq) * D + 16 * mt + dr1] = o[mt][2] * inv0;
+                    if (cv1) po[(2 * tq + 1) * D + 16 * mt + dr1] = o[mt][3] * inv1;
                 }
                 if (gr == 0) {
 #pragma unroll
                     for (int c = 0; c < 2; ++c)
-                        p.part_lse[pi * Cfg::kHq + 8 * g + 2 * tq + c] = (l[c] > 0.f) ? m[c] + log2f(l[c]) : -INFINITY;
+                        if (2 * tq + c < nv)
+                            p.part_lse[pi * Cfg::kHq + h0 + 2 * tq + c] = (l[c] > 0.f) ? m[c] + log2f(l[c]) : -INFINITY;
                 }
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.xdone[g]);
+            if (lane == 0) mbar_arrive(&sm.xdone[grp]);
         }
     }
 }
 
 // Decode combine: one CTA of 128 threads per (sequence, q head): out =
 // sum_s w_s o_s / sum_s w_s with w_s = 2^(lse_s - max lse).  Warp j sums the
-// splits s = j mod 4 (lane l: dims 4l .. 4l + 3), so four independent chains
-// of loads are in flight; warps 1-3 hand their sums to warp 0.
+// splits s = j mod 4 (lane l: dims 4l + 128c .. +3), so four independent
+// chains of loads are in flight; warps 1-3 hand their sums to warp 0.
+template <int D>
 __global__ void __launch_bounds__(128) attn_combine_kernel(const float *__restrict__ part_o,
                                                            const float *__restrict__ part_lse, int splits, int Hq,
                                                            __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
-    __shared__ float4 red_o[3][32];
+    constexpr int NC = D / 128;
+    __shared__ float4 red_o[3][NC][32];
     __shared__ float red_m[4], red_d[4];
     pdl_wait();
     const int seq = blockIdx.x / Hq, h = blockIdx.x % Hq, tid = threadIdx.x, lane = tid & 31, sg = tid >> 5;
@@ -703,40 +724,54 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const float *__restri
     if (lane == 0) red_m[sg] = mx;
     __syncthreads();
     mx = fmaxf(fmaxf(red_m[0], red_m[1]), fmaxf(red_m[2], red_m[3]));
-    const float *po = part_o + ((int64_t)seq * splits * Hq + h) * 128 + 4 * lane;
+    const float *po = part_o + ((int64_t)seq * splits * Hq + h) * D + 4 * lane;
     float den = 0.f;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 acc[NC];
+#pragma unroll
+    for (int c = 0; c < NC; ++c) acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 4
     for (int s = sg; s < splits; s += 4) {
         const float v = pl[(int64_t)s * Hq];
-        const float4 x = *reinterpret_cast<const float4 *>(po + (int64_t)s * Hq * 128);
+        float4 x[NC];
+#pragma unroll
+        for (int c = 0; c < NC; ++c) x[c] = *reinterpret_cast<const float4 *>(po + (int64_t)s * Hq * D + 128 * c);
         const float w = (mx == -INFINITY || v == -INFINITY) ? 0.f : exp2f(v - mx);
         den += w;
-        acc.x += w * x.x;
-        acc.y += w * x.y;
-        acc.z += w * x.z;
-        acc.w += w * x.w;
+#pragma unroll
+        for (int c = 0; c < NC; ++c) {
+            acc[c].x += w * x[c].x;
+            acc[c].y += w * x[c].y;
+            acc[c].z += w * x[c].z;
+            acc[c].w += w * x[c].w;
+        }
     }
     if (sg > 0) {
-        red_o[sg - 1][lane] = acc;
+#pragma unroll
+        for (int c = 0; c < NC; ++c) red_o[sg - 1][c][lane] = acc[c];
         if (lane == 0) red_d[sg] = den;
     }
     __syncthreads();
     if (sg != 0) return;
 #pragma unroll
     for (int j = 0; j < 3; ++j) {
-        const float4 o = red_o[j][lane];
-        acc.x += o.x;
-        acc.y += o.y;
-        acc.z += o.z;
-        acc.w += o.w;
+#pragma unroll
+        for (int c = 0; c < NC; ++c) {
+            const float4 o = red_o[j][c][lane];
+            acc[c].x += o.x;
+            acc[c].y += o.y;
+            acc[c].z += o.z;
+            acc[c].w += o.w;
+        }
         den += red_d[j + 1];
     }
     const float inv = den > 0.f ? 1.f / den : 0.f;
-    uint2 v;
-    v.x = pack_bf16(acc.x * inv, acc.y * inv);
-    v.y = pack_bf16(acc.z * inv, acc.w * inv);
-    *reinterpret_cast<uint2 *>(out + ((int64_t)seq * Hq + h) * 128 + 4 * lane) = v;
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+        uint2 v;
+        v.x = pack_bf16(acc[c].x * inv, acc[c].y * inv);
+        v.y = pack_bf16(acc[c].z * inv, acc[c].w * inv);
+        *reinterpret_cast<uint2 *>(out + ((int64_t)seq * Hq + h) * D + 128 * c + 4 * lane) = v;
+    }
     if (lse && lane == 0) lse[(int64_t)seq * Hq + h] = den > 0.f ? (mx + log2f(den)) / kLog2e : -INFINITY;
 }
 
@@ -854,9 +889,9 @@ int attn_tail_blocks(bool indexshare, int max_draft) {
 
 namespace {
 
-template <int HKV, bool KV8>
+template <int HKV, bool KV8, int D, int G>
 cudaError_t run_bf16(const AttnArgs &a, void *ws, unsigned *status, cudaStream_t s) {
-    using Cfg = AttnCfg<HKV, KV8>;
+    using Cfg = AttnCfg<HKV, KV8, D, G>;
     const DeviceInfo *di = device_info();
     const int sms = di ? di->sm_count : 148;
     AttnParams p{};
@@ -893,7 +928,7 @@ cudaError_t run_bf16(const AttnArgs &a, void *ws, unsigned *status, cudaStream_t
         p.items = (int64_t)a.B * splits;
         float *w = static_cast<float *>(ws);
         p.part_o = w;
-        p.part_lse = w + (size_t)a.B * splits * Cfg::kHq * 128;
+        p.part_lse = w + (size_t)a.B * splits * Cfg::kHq * D;
     } else {
         p.splits = 1;
         p.split_blocks = 0;
@@ -903,9 +938,9 @@ cudaError_t run_bf16(const AttnArgs &a, void *ws, unsigned *status, cudaStream_t
     // an item's list holds at most top_k ids plus the tail block
     p.sel_cap = p.dense ? 4 : (a.top_k + 3) & ~3;                  // dense: no id list, no stage tables
     p.nst_cap = p.dense ? 1 : (list_max + AT_BPS - 1) / AT_BPS;
-    const size_t smem = attn_smem_bytes<HKV, KV8>(p.sel_cap, p.nst_cap);
+    const size_t smem = attn_smem_bytes<Cfg>(p.sel_cap, p.nst_cap);
     if (di && smem > di->smem_optin) return cudaErrorInvalidValue;
-    auto kern = p.pg.table ? attn_bf16_kernel<HKV, true, KV8> : attn_bf16_kernel<HKV, false, KV8>;
+    auto kern = p.pg.table ? attn_bf16_kernel<HKV, D, G, true, KV8> : attn_bf16_kernel<HKV, D, G, false, KV8>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
@@ -914,7 +949,7 @@ cudaError_t run_bf16(const AttnArgs &a, void *ws, unsigned *status, cudaStream_t
     const int64_t grid = std::min<int64_t>(p.items, (int64_t)sms * std::max(1, per_sm));
     e = launch_pdl(kern, dim3((unsigned)grid), dim3(Cfg::kThreads), smem, s, p);
     if (e != cudaSuccess || !a.decode) return e;
-    return launch_pdl(attn_combine_kernel, dim3((unsigned)(a.B * Cfg::kHq)), dim3(128), 0, s,
+    return launch_pdl(attn_combine_kernel<D>, dim3((unsigned)(a.B * Cfg::kHq)), dim3(128), 0, s,
                       (const float *)p.part_o, (const float *)p.part_lse, p.splits, (int)Cfg::kHq,
                       (__nv_bfloat16 *)a.out, a.lse);
 }
@@ -944,9 +979,12 @@ size_t attn_dense_decode_ws_bytes(int B, int Hq, int d, int64_t kv_stride) {
 
 cudaError_t launch_attn_bf16(const AttnArgs &a, void *ws, unsigned *status, cudaStream_t s) {
     switch (a.Hkv) {
-    case 1: return a.kv8 ? run_bf16<1, true>(a, ws, status, s) : run_bf16<1, false>(a, ws, status, s);
-    case 2: return a.kv8 ? run_bf16<2, true>(a, ws, status, s) : run_bf16<2, false>(a, ws, status, s);
-    case 4: return a.kv8 ? run_bf16<4, true>(a, ws, status, s) : run_bf16<4, false>(a, ws, status, s);
+    case 1: return a.kv8 ? run_bf16<1, true, 128, 8>(a, ws, status, s) : run_bf16<1, false, 128, 8>(a, ws, status, s);
+    case 2:
+        if (a.d == 256)   // the released 24q/2kv, d = 256 shape
+            return a.kv8 ? run_bf16<2, true, 256, 12>(a, ws, status, s) : run_bf16<2, false, 256, 12>(a, ws, status, s);
+        return a.kv8 ? run_bf16<2, true, 128, 8>(a, ws, status, s) : run_bf16<2, false, 128, 8>(a, ws, status, s);
+    case 4: return a.kv8 ? run_bf16<4, true, 128, 8>(a, ws, status, s) : run_bf16<4, false, 128, 8>(a, ws, status, s);
     default: return cudaErrorInvalidValue;
     }
 }

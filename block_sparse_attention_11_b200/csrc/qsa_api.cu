@@ -287,8 +287,12 @@ int attn_common_checks(const void *q, const void *k, const void *v, const int32_
     if (Hq < 1 || Hkv < 1 || (Hq % Hkv) != 0) return QSA_ERR_INVALID_ARG;
     if (!(scale > 0.f) || !std::isfinite(scale)) return QSA_ERR_INVALID_ARG;
     if (dtype != QSA_BF16 && dtype != QSA_FP32) return QSA_ERR_UNSUPPORTED;
-    if (d != 128) return QSA_ERR_UNSUPPORTED;
-    if (dtype == QSA_BF16 && (Hq != 8 * Hkv || (Hkv != 1 && Hkv != 2 && Hkv != 4))) return QSA_ERR_UNSUPPORTED;
+    // shapes: d = 128 with 8 q heads per kv head (1, 2 or 4 kv heads; fp32: any GQA),
+    // and the released 24q / 2kv, d = 256 shape (bf16)
+    const bool released = dtype == QSA_BF16 && d == 256 && Hkv == 2 && Hq == 24;
+    if (d != 128 && !released) return QSA_ERR_UNSUPPORTED;
+    if (dtype == QSA_BF16 && !released && (Hq != 8 * Hkv || (Hkv != 1 && Hkv != 2 && Hkv != 4)))
+        return QSA_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return QSA_ERR_INVALID_ARG;
     return QSA_OK;
 }

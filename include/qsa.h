@@ -25,7 +25,8 @@
  *     every floating-point tensor of the call, except head weights (always
  *     float) and the fp32 scratch.
  *   - Indexer geometry is fixed by the pages: 4 query heads, 1 key head,
- *     128 dims, blocks of 4 tokens.  Attention head dim d = 128.
+ *     128 dims, blocks of 4 tokens.  Attention head dim d = 128, or 256 for
+ *     the released 24q / 2kv shape.
  *   - Positions: token i of a sequence has RoPE position i.  Block b holds
  *     positions 4b..4b+3 and is visible to the query at position t iff
  *     4b + 3 <= t, so nb(t) = floor((t + 1) / 4) blocks are visible and the
@@ -256,9 +257,11 @@ QSA_API int qsa_index_topk_decode(const void *q_idx, const void *k_pool, const f
  * sel/nsel device, as written by qsa_index_topk_prefill.  Ids must satisfy
  *          0 <= b < nb(t); out-of-range ids are skipped and flagged.
  * out      device, [B][n_q][Hq][d] dtype.   lse device, [B][n_q][Hq] float or NULL.
- * Shapes: d == 128; Hq % Hkv == 0; Hq / Hkv == 8 for QSA_BF16 (the GQA
- *         ratio of the kernels' tiles), any ratio for QSA_FP32;
- *         kv_stride >= q0 + n_q.
+ * Shapes: d == 128 with Hq % Hkv == 0 and, for QSA_BF16, Hq / Hkv == 8 and
+ *         Hkv in {1, 2, 4} (any ratio for QSA_FP32); or, QSA_BF16 only, the
+ *         released model's shape Hq = 24, Hkv = 2, d = 256 (the architecture
+ *         guide page, section "How a token moves through the model", item 2:
+ *         24 query heads, two KV heads of dimension 256); kv_stride >= q0 + n_q.
  * workspace: none needed (pass NULL, 0).
  */
 QSA_API int qsa_sparse_attn_prefill(const void *q, const void *k, const void *v, const int32_t *sel,
@@ -373,7 +376,8 @@ QSA_API int qsa_sparse_attn_decode_noalloc(const void *q, const void *k, const v
  * the BF16 query and the dequantized keys (FP16 tensor-core MMAs, the query
  * scaled by a power of two), probabilities are rounded to FP16 for the value
  * MMAs.  As qsa_sparse_attn_prefill / qsa_sparse_attn_decode otherwise
- * (Hq = 8 Hkv, Hkv in {1, 2, 4}, d = 128); k, v are [B][kv_stride][Hkv][d]
+ * (Hq = 8 Hkv with Hkv in {1, 2, 4} and d = 128, or 24q / 2kv with d = 256);
+ * k, v are [B][kv_stride][Hkv][d]
  * bytes; k_scale, v_scale finite and > 0.  Decode workspace as
  * qsa_sparse_attn_decode_workspace(..., QSA_BF16).
  */

@@ -275,6 +275,91 @@ def test_attention_fp8_kv_decode(qsa, B, L):
         assert np.abs(lse[b].cpu().numpy() - ref["lse"][0]).max() <= 1e-3
 
 
+@pytest.mark.parametrize("T,top_k,kv8", [(2500, 96, False), (2500, 96, True), (7, 4, False), (1031, 512, False)])
+def test_attention_released_shape_prefill(qsa, T, top_k, kv8):
+    """The released 24q / 2kv, d = 256 shape (two 8-head column tiles per kv
+    head, the second half padding) on the oracle's selection, BF16 or FP8 K/V."""
+    w = workloads.Workload(f"t{T}", "prefill", 1, T, top_k, 24, 2, 256, "bf16", 35)
+    x = workloads.make_prefill(w, device=DEV)
+    k, v = x["k"], x["v"]
+    ks = vs = 1.0
+    if kv8:
+        k, ks = _to_e4m3(x["k"])
+        v, vs = _to_e4m3(x["v"])
+    kd = k.float() * ks
+    vd = v.float() * vs
+    rows = list(range(T))
+    kp = oracle.pool_keys(np32(x["k_idx"][0]))
+    ref = oracle.prefill_rows(rows, q_idx=np32(x["q_idx"][0]), k_pool=kp, top_k=top_k, q=np32(x["q"][0]),
+                              k=kd[0].cpu().numpy(), v=vd[0].cpu().numpy(), Hq=24, Hkv=2, d=256)
+    sel = torch.from_numpy(ref["sel"][None]).to(DEV)
+    nsel = torch.from_numpy(ref["nsel"][None]).to(DEV)
+    out = torch.full_like(x["q"], 7.0)
+    lse = torch.empty(1, T, 24, dtype=torch.float32, device=DEV)
+    if kv8:
+        qsa.qsa_sparse_attn_prefill_kv8(x["q"], k, v, ks, vs, sel, nsel, out, lse=lse)
+    else:
+        qsa.qsa_sparse_attn_prefill(x["q"], k, v, sel, nsel, out, lse=lse)
+    qsa.qsa_check_status()
+    err = np.abs(np32(out[0]) - ref["out"]).max()
+    assert err <= TOL["bf16"], err
+    assert np.abs(lse[0].cpu().numpy() - ref["lse"]).max() <= 1e-3
+
+
+@pytest.mark.parametrize("B,L,kv8", [(6, 20000, False), (3, 70001, True), (5, 2, False)])
+def test_attention_released_shape_decode(qsa, B, L, kv8):
+    """Decode attention with the released 24q / 2kv, d = 256 shape against the
+    oracle's decode step (selection and attention), and the dense decode
+    baseline against textbook attention."""
+    w = workloads.Workload("dec_rel", "decode", B, L, 256, 24, 2, 256, "bf16", 81)
+    x = workloads.make_decode(w, device=DEV, ragged=True)
+    rope = rope_of(w)
+    lens = x["lens"]
+    k, v = x["k"], x["v"]
+    ks = vs = 1.0
+    if kv8:
+        k, ks = _to_e4m3(x["k"])
+        v, vs = _to_e4m3(x["v"])
+    cap = max(lens) // 4 + 2
+    k_pool = torch.zeros(B, cap, 128, dtype=torch.bfloat16, device=DEV)
+    for b in range(B):
+        kp = torch.zeros(1, cap, 128, dtype=torch.bfloat16, device=DEV)
+        full = torch.cat([x["k_idx"][b, :lens[b]], x["k_idx_new"][b:b + 1]], 0)[None].contiguous()
+        qsa.qsa_pool_keys_prefill(full, kp, rope=rope)
+        k_pool[b] = kp[0]
+    sel = torch.empty(B, w.top_k, dtype=torch.int32, device=DEV)
+    nsel = torch.empty(B, dtype=torch.int32, device=DEV)
+    qsa.qsa_index_topk_decode(x["q_idx"], k_pool, x["seq_len"], sel, nsel, top_k=w.top_k, rope=rope)
+    out = torch.empty_like(x["q"])
+    lse = torch.empty(B, 24, dtype=torch.float32, device=DEV)
+    if kv8:
+        qsa.qsa_sparse_attn_decode_kv8(x["q"], k, v, ks, vs, x["seq_len"], sel, nsel, out, lse=lse)
+    else:
+        qsa.qsa_sparse_attn_decode(x["q"], k, v, x["seq_len"], sel, nsel, out, lse=lse)
+    qsa.qsa_check_status()
+    kd, vd = k.float() * ks, v.float() * vs
+    for b in range(B):
+        s = lens[b] + 1
+        ref = oracle.decode(np32(x["q_idx"][b:b + 1]), np32(k_pool[b])[None], [s], q=np32(x["q"][b:b + 1]),
+                            k=kd[b:b + 1].cpu().numpy(), v=vd[b:b + 1].cpu().numpy(), top_k=w.top_k,
+                            Hq=24, Hkv=2, d=256)
+        if not np.array_equal(sel[b].cpu().numpy(), ref["sel"][0]):
+            gap = (ref["kth"][0] - ref["next"][0]) / max(abs(ref["kth"][0]), 1e-30)
+            assert gap < 1e-4, f"seq {b}: selection differs with gap {gap}"
+            continue
+        assert np.abs(np32(out[b]) - ref["out"][0]).max() <= TOL["bf16"], b
+        assert np.abs(lse[b].cpu().numpy() - ref["lse"][0]).max() <= 1e-3
+    if not kv8:
+        outd = torch.empty_like(x["q"])
+        qsa.qsa_dense_attn_decode(x["q"], x["k"], x["v"], x["seq_len"], outd)
+        qsa.qsa_check_status()
+        for b in range(min(B, 2)):
+            t = lens[b]
+            refd = oracle.dense_rows([0], q=np32(x["q"][b])[None], k=np32(x["k"][b]), v=np32(x["v"][b]), Hq=24,
+                                     Hkv=2, d=256, q0=t)
+            assert np.abs(np32(outd[b]) - refd[0]).max() <= TOL["bf16"], b
+
+
 def test_attention_flags_out_of_range_ids(qsa):
     """A selection id outside [0, nb(t)) is skipped and reported through the
     status word (no trap)."""

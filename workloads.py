@@ -74,6 +74,12 @@ WORKLOADS = {
     # the 32K prefill workload with FP8 E4M3 K/V caches
     "prefill_t32k_needles_kv8": Workload("prefill_t32k_needles_kv8", "prefill", 1, 32768, 512, 16, 2, 128, "bf16",
                                          1002, needles=64, extra={"kv": "fp8"}),
+    # the released model's attention shape: 24 q heads, 2 kv heads of 256 dims (BF16, and the FP8 serving form)
+    "prefill_t32k_d256": Workload("prefill_t32k_d256", "prefill", 1, 32768, 512, 24, 2, 256, "bf16", 1002,
+                                  needles=64),
+    "decode_b64_l128k_d256": Workload("decode_b64_l128k_d256", "decode", 64, 131072, 512, 24, 2, 256, "bf16", 1003),
+    "decode_b64_l128k_d256_fp8": Workload("decode_b64_l128k_d256_fp8", "decode", 64, 131072, 512, 24, 2, 256, "bf16",
+                                          1003, extra={"keys": "fp8", "kv": "fp8"}),
     # the 128K decode workload over paged caches (64-token pages, shuffled page pool)
     "decode_b64_l128k_paged": Workload("decode_b64_l128k_paged", "decode", 64, 131072, 512, 16, 2, 128, "bf16",
                                        1003, extra={"page_tokens": 64}),
