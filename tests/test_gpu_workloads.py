@@ -148,3 +148,55 @@ def test_decode_128k_b64_fp8_keys(qsa):
 
 def test_decode_1m_b8_fp8_keys(qsa):
     _decode_check(qsa, workloads.WORKLOADS["decode_b8_l1m_scale4_fp8keys"])
+
+
+def _bench_decode_check(qsa, name):
+    """One decode step of the benchmark's own runner (its caches, layout and
+    calls: paged, FP8 keys, FP8 K/V, head shape as the workload says) against
+    the oracle, sequence by sequence, on the same seeded inputs."""
+    import bench
+    w = workloads.WORKLOADS[name]
+    r = bench.DecodeRunner(w, torch.device(DEV))
+    out = r.step().float().cpu().numpy()
+    sel, nsel = r.sel.cpu().numpy(), r.nsel.cpu().numpy()
+    qsa.qsa_check_status()
+    del r
+    _free()
+    x = workloads.make_decode(w, device=DEV)
+    fp8 = w.extra.get("keys") == "fp8"
+    k, v = x["k"], x["v"]
+    if w.extra.get("kv") == "fp8":
+        k8, ks = workloads.to_e4m3(x["k"])
+        v8, vs = workloads.to_e4m3(x["v"])
+        k, v = k8.float() * ks, v8.float() * vs
+        del k8, v8
+    nbad = 0
+    for b in range(w.B):
+        L = x["lens"][b]
+        kr = np32(x["k_idx"][b, :L])
+        kp = np.zeros((L // 4 + 1, 128), np.float32)
+        kp[: L // 4] = oracle.pool_keys(kr, base=w.rope_base, pos_scale=w.pos_scale, store_fp8=fp8)
+        rg = np.zeros((4, 128), np.float32)
+        rg[: L - 4 * (L // 4)] = kr[4 * (L // 4):]
+        oracle.pool_decode(np32(x["k_idx_new"][b]), rg, kp, L + 1, base=w.rope_base, pos_scale=w.pos_scale,
+                           store_fp8=fp8)
+        ref = oracle.decode(np32(x["q_idx"][b:b + 1]), kp[None], [L + 1], q=np32(x["q"][b:b + 1]),
+                            k=np32(k[b:b + 1]), v=np32(v[b:b + 1]), top_k=w.top_k, base=w.rope_base,
+                            pos_scale=w.pos_scale, Hq=w.Hq, Hkv=w.Hkv, d=w.d)
+        assert int(nsel[b]) == ref["nsel"][0]
+        if not np.array_equal(sel[b], ref["sel"][0]):
+            gap = (ref["kth"][0] - ref["next"][0]) / max(abs(ref["kth"][0]), 1e-30)
+            assert gap < 1e-4, f"seq {b}: selection differs with gap {gap}"
+            nbad += 1
+            continue
+        err = np.abs(out[b] - ref["out"][0]).max()
+        assert err <= TOL["bf16"], (b, err)
+    assert nbad <= max(1, w.B // 16)
+    del x, k, v
+    _free()
+
+
+@pytest.mark.parametrize("name", ["decode_b64_l128k_paged", "decode_b64_l128k_fp8", "decode_b64_l128k_d256",
+                                  "decode_b64_l128k_d256_fp8"])
+def test_bench_decode_runner_full_size(qsa, name):
+    _bench_decode_check(qsa, name)
