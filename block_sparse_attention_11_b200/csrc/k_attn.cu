@@ -65,7 +65,7 @@ constexpr uint32_t kFullStage = 0x924924u;   // 8 slots x 3 bits, each holding 4
 // D: head dim (128 or 256).  G: q heads per kv head (8, or 12 for the released
 // 24q/2kv shape: two 8-head MMA column tiles, the second one half padding).
 template <int HKV, bool KV8 = false, int D = 128, int G = 8> struct AttnCfg {
-    static constexpr int kD = D, kG = G;
+    static constexpr int kD = D;
     static constexpr int kNT = (G + 7) / 8;        // 8-head column tiles per kv head
     static constexpr int kMT = D / 16;             // 16-dim MMA k-steps (QK) and m-tiles (PV)
     // Consumer warp (grp, sub): group grp = kv head g, column tile nt; sub = u * 2
