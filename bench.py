@@ -590,8 +590,56 @@ def run_ours(args, rank, world):
         torch.cuda.synchronize()
         return e0.elapsed_time(e1) / e2e_steps
 
-    e2e_eager_ms = timed(e2e_step)
-    e2e_ms = e2e_eager_ms
+    e2e_serial_ms = timed(e2e_step)
+
+    def e2e_pipelined(n):
+        """n steps through the public API with the host copies of one step
+        overlapping the compute of another: step i's inputs go host -> device on
+        a copy stream into buffer set i % 2 while step i - 1 computes, and its
+        output comes back on a third stream while step i + 1 computes.  Every
+        step still copies all its inputs in and its result out."""
+        bufs = [{k: torch.empty_like(v, device=dev) for k, v in host.items()} for _ in range(2)]
+        outs = [torch.empty_like(runner.out) for _ in range(2)]
+        outs_h = [torch.empty(runner.out.shape, dtype=runner.out.dtype, pin_memory=True) for _ in range(2)]
+        s_h2d, s_d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        comp = torch.cuda.current_stream(dev)
+        ev = {n_: [torch.cuda.Event() for _ in range(2)] for n_ in ("h2d", "comp", "d2h")}
+        keep_out = runner.out
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(comp)
+        s_h2d.wait_stream(comp)
+        for i in range(n):
+            b = i & 1
+            with torch.cuda.stream(s_h2d):
+                if i >= 2:
+                    s_h2d.wait_event(ev["comp"][b])        # step i - 2 has finished reading buffer set b
+                for k, v in host.items():
+                    bufs[b][k].copy_(v, non_blocking=True)
+                ev["h2d"][b].record(s_h2d)
+            comp.wait_event(ev["h2d"][b])
+            if i >= 2:
+                comp.wait_event(ev["d2h"][b])              # step i - 2's output has been read back
+            xs = dict(runner.x)
+            xs.update(bufs[b])
+            runner.out = outs[b]
+            runner.step(x=xs)
+            ev["comp"][b].record(comp)
+            with torch.cuda.stream(s_d2h):
+                s_d2h.wait_event(ev["comp"][b])
+                outs_h[b].copy_(outs[b], non_blocking=True)
+                ev["d2h"][b].record(s_d2h)
+        comp.wait_stream(s_d2h)
+        e1.record(comp)
+        torch.cuda.synchronize()
+        runner.out = keep_out
+        return e0.elapsed_time(e1) / n
+
+    e2e_pipelined(2)                    # untimed: allocations and first launches
+    e2e_pipe_ms = e2e_pipelined(e2e_steps)
+    e2e_ms = min(e2e_serial_ms, e2e_pipe_ms)
+    e2e_mode = "pipelined" if e2e_pipe_ms <= e2e_serial_ms else "serial"
+    e2e_eager_ms = e2e_serial_ms
     if graph is not None:
         # the same public calls and copies (pinned host buffers), captured once and replayed
         for k, v in host.items():
@@ -602,8 +650,10 @@ def run_ours(args, rank, world):
                 dev_x[k].copy_(v, non_blocking=True)
             out = runner.step(x=dev_x)
             out_host.copy_(out, non_blocking=True)
-        e2e_ms = timed(g2.replay)
+        e2e_graph_ms = timed(g2.replay)
         del g2
+        if e2e_graph_ms < e2e_ms:
+            e2e_ms, e2e_mode = e2e_graph_ms, "graph"
     used_graph = graph is not None
     del graph
 
@@ -620,7 +670,8 @@ def run_ours(args, rank, world):
         res.update(metric="QSA prefill tokens/s", unit="tokens/s", higher_is_better=True,
                    value=job_throughput(runner.units(), world, ms_per_step))
         res["e2e"] = dict(value=job_throughput(runner.units(), world, e2e_ms), unit="tokens/s", h2d_bytes_per_step=h2d,
-                          d2h_bytes_per_step=d2h)
+                          d2h_bytes_per_step=d2h, mode=e2e_mode,
+                          serial_value=job_throughput(runner.units(), world, e2e_serial_ms))
         attn_ms = stage_avg["sparse_attn"]
         achieved = alg["attn_bytes"] / (attn_ms / 1e3) / 1e9
         res["roofline"] = dict(kernel="sparse_attn_prefill", bound="hbm", achieved=achieved, peak=pk["hbm_gbs"],
@@ -641,7 +692,7 @@ def run_ours(args, rank, world):
     elif w.kind in ("draft", "dense"):
         res.update(metric=metric_name(w), unit="us/step", higher_is_better=False, value=ms_per_step * 1e3)
         res["e2e"] = dict(value=e2e_ms * 1e3, unit="us/step", h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h,
-                          graph=used_graph, eager_value=e2e_eager_ms * 1e3)
+                          mode=e2e_mode, serial_value=e2e_eager_ms * 1e3)
         achieved = alg["attn_bytes"] / (ms_per_step / 1e3) / 1e9
         res["roofline"] = dict(kernel="sparse_attn_decode (frozen selection)" if w.kind == "draft"
                                else "dense causal decode attention", bound="hbm", achieved=achieved,
@@ -657,7 +708,7 @@ def run_ours(args, rank, world):
         res.update(metric="QSA decode us/step", unit="us/step", higher_is_better=False,
                    value=ms_per_step * 1e3)
         res["e2e"] = dict(value=e2e_ms * 1e3, unit="us/step", h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h,
-                          graph=used_graph, eager_value=e2e_eager_ms * 1e3)
+                          mode=e2e_mode, serial_value=e2e_eager_ms * 1e3)
         idx_ms = stage_avg["index_topk"]
         achieved = alg["idx_bytes"] / (idx_ms / 1e3) / 1e9
         res["roofline"] = dict(kernel="decode indexer (scorer + select)", bound="hbm", achieved=achieved,
