@@ -473,6 +473,52 @@ class DenseRunner:
         return {k: self.x[k].cpu().pin_memory() for k in ["q", "seq_len"]}
 
 
+class DensePrefillRunner:
+    """Full causal prefill attention over every earlier position (the dense
+    baseline the pages compare QSA's prefill with), on the QSA prefill
+    workloads' q/k/v."""
+
+    def __init__(self, w, dev):
+        import block_sparse_attention_11_b200 as qsa
+        self.qsa = qsa
+        self.w = w
+        self.dev = dev
+        x = workloads.make_prefill(w, device=dev)
+        self.x = {n: x[n] for n in ("q", "k", "v")}
+        torch.cuda.empty_cache()
+        self.out = torch.empty_like(x["q"])
+        self.flush_between_steps = True
+        self.use_graph = False
+
+    def step(self, x=None, events=None):
+        x = x or self.x
+        if events is not None:
+            events[0].record()
+            events[1].record()
+            events[2].record()
+        self.qsa.qsa_dense_attn_prefill(x["q"], x["k"], x["v"], self.out)
+        if events is not None:
+            events[3].record()
+        return self.out
+
+    def launches_per_step(self):
+        return 1
+
+    def units(self):
+        return self.w.B * self.w.T   # tokens
+
+    def stage_names(self):
+        return ["no_pool", "no_index", "dense_attn"]
+
+    def algorithmic(self):
+        w = self.w
+        pairs = w.T * (w.T + 1) / 2 * w.B                              # (query, key) pairs, causal
+        return dict(attn_flops=pairs * 4 * w.d * w.Hq)
+
+    def host_inputs(self):
+        return {k: v.cpu().pin_memory() for k, v in self.x.items()}
+
+
 # ----------------------------------------------------------------------------- measurement
 
 def flush_l2(buf):
@@ -498,7 +544,7 @@ def run_ours(args, rank, world):
     torch.cuda.set_device(dev)
     w = workloads.WORKLOADS[args.workload]
     runner = {"prefill": PrefillRunner, "decode": DecodeRunner, "draft": DraftRunner,
-              "dense": DenseRunner}[w.kind](w, dev)
+              "dense": DenseRunner, "dense_prefill": DensePrefillRunner}[w.kind](w, dev)
     flush = torch.zeros(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
     qsa = runner.qsa
     for _ in range(args.warmup):
@@ -689,6 +735,20 @@ def run_ours(args, rank, world):
         res["config"] = dict(workload=w.name, B=w.B, T=w.T, top_k=w.top_k, Hq=w.Hq, Hkv=w.Hkv, d=w.d,
                              needles=w.needles, l2="flushed between timed steps (256 MB write)",
                              parallelism=f"replicas x{world}")
+    elif w.kind == "dense_prefill":
+        res.update(metric=metric_name(w), unit="tokens/s", higher_is_better=True,
+                   value=job_throughput(runner.units(), world, ms_per_step))
+        res["e2e"] = dict(value=job_throughput(runner.units(), world, e2e_ms), unit="tokens/s", h2d_bytes_per_step=h2d,
+                          d2h_bytes_per_step=d2h, mode=e2e_mode,
+                          serial_value=job_throughput(runner.units(), world, e2e_serial_ms))
+        tf = alg["attn_flops"] / (ms_per_step / 1e3) / 1e12
+        peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+        res["roofline"] = dict(kernel="dense_prefill_kernel", bound="tensor", achieved=tf, peak=peak,
+                               unit="TFLOP/s", frac=tf / peak, traffic=None, peak_kind=pk_kind,
+                               note="4*d*Hq flop per causal (query, key) pair over the step time; sustained bf16 "
+                                    "peak (a step of tens of ms)")
+        res["config"] = dict(workload=w.name, B=w.B, T=w.T, Hq=w.Hq, Hkv=w.Hkv, d=w.d,
+                             l2="flushed between timed steps (256 MB write)", parallelism=f"replicas x{world}")
     elif w.kind in ("draft", "dense"):
         res.update(metric=metric_name(w), unit="us/step", higher_is_better=False, value=ms_per_step * 1e3)
         res["e2e"] = dict(value=e2e_ms * 1e3, unit="us/step", h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h,
@@ -765,6 +825,21 @@ def run_oracle_sample(w, budget_s=15.0, seed=0):
         sample = (f"{done} uniformly drawn query rows of the {w.T}-token workload (full indexer scan, top-k, "
                   f"attention per row) + pooling of all keys; extrapolated per row to all rows")
         return value, sample, nthreads, "tokens/s"
+    if w.kind == "dense_prefill":   # textbook causal attention of sampled rows, per row cost ~ its position
+        x = workloads.make_prefill(w, device="cpu")
+        q, k, v = (x[n][0].float().numpy() for n in ("q", "k", "v"))
+        rng = np.random.default_rng(seed)
+        done_pos, elapsed, n = 0.0, 0.0, 8
+        while elapsed < budget_s:
+            rows = rng.integers(0, w.T, n)
+            t0 = time.perf_counter()
+            oracle.dense_rows(rows, q=q, k=k, v=v, Hq=w.Hq, Hkv=w.Hkv, d=w.d, nthreads=nthreads)
+            elapsed += time.perf_counter() - t0
+            done_pos += float((rows + 1).sum())
+            n = min(1024, n * 2)
+        total = elapsed / done_pos * (w.T * (w.T + 1) / 2) * w.B       # extrapolated by causal positions
+        return (w.T * w.B / total, "uniformly drawn query rows (textbook attention over their causal prefix); "
+                "extrapolated by positions to all rows", nthreads, "tokens/s")
     if w.kind == "dense":   # textbook causal attention of one sequence's new token
         x = workloads.make_decode(w, device="cpu", B=1)
         q, k, v = x["q"].float().numpy(), x["k"][0].float().numpy(), x["v"][0].float().numpy()
@@ -817,7 +892,8 @@ def dequant_kv(w, x):
 
 def metric_name(w):
     return {"prefill": "QSA prefill tokens/s", "decode": "QSA decode us/step",
-            "draft": "QSA IndexShare draft step us/step", "dense": "full causal decode attention us/step"}[w.kind]
+            "draft": "QSA IndexShare draft step us/step", "dense": "full causal decode attention us/step",
+            "dense_prefill": "full causal prefill attention tokens/s"}[w.kind]
 
 
 def main():
@@ -852,7 +928,7 @@ def main():
         if rank == 0:
             value, sample, threads, unit = run_oracle_sample(w, budget_s=args.cpu_budget)
             line = dict(impl="reference", metric=metric_name(w), value=value, unit=unit,
-                        higher_is_better=w.kind == "prefill",
+                        higher_is_better=w.kind in ("prefill", "dense_prefill"),
                         n_gpus=args.gpus, steps=args.steps, warmup=args.warmup, dtype=w.dtype, data="synthetic",
                         config=dict(workload=w.name), vs_baseline=None,
                         cpu_baseline=dict(value=value, unit=unit, cores=threads, kind="oracle", sample=sample),

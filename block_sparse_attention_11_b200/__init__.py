@@ -26,7 +26,7 @@ __all__ = [
     "qsa_index_topk_decode", "qsa_index_topk_decode_workspace", "qsa_index_topk_decode_kernels",
     "qsa_sparse_attn_prefill", "qsa_sparse_attn_decode", "qsa_sparse_attn_decode_workspace",
     "qsa_sparse_attn_decode_noalloc", "qsa_sparse_attn_decode_shared", "qsa_sparse_attn_decode_shared_workspace",
-    "qsa_dense_attn_decode", "qsa_dense_attn_decode_workspace",
+    "qsa_dense_attn_decode", "qsa_dense_attn_decode_workspace", "qsa_dense_attn_prefill",
     "qsa_pool_keys_prefill_paged", "qsa_pool_keys_decode_paged", "qsa_index_topk_decode_paged",
     "qsa_sparse_attn_decode_paged", "qsa_sparse_attn_prefill_kv8", "qsa_sparse_attn_decode_kv8",
     "qsa_rope_apply", "qsa_check_status", "qsa_strerror", "qsa_version",
@@ -115,6 +115,8 @@ _sig("qsa_index_topk_decode_paged", ctypes.c_int, _vp, _vp, _Paging, _vp, _vp, _
      _Rope, _u32, _i32, _vp)
 _sig("qsa_sparse_attn_decode_paged", ctypes.c_int, _vp, _vp, _vp, _Paging, _vp, _vp, _vp, _i32, _i32, _i32, _i32,
      _i32, _f32, _vp, _vp, _vp, _sz, _i32, _vp)
+_sig("qsa_dense_attn_prefill", ctypes.c_int, _vp, _vp, _vp, _i32, _i64, _i64, _i64, _i32, _i32, _i32, _f32, _vp, _vp,
+     _i32, _vp)
 _sig("qsa_sparse_attn_prefill_kv8", ctypes.c_int, _vp, _vp, _vp, _f32, _f32, _vp, _vp, _i32, _i64, _i64, _i64, _i32,
      _i32, _i32, _i32, _f32, _vp, _vp, _vp)
 _sig("qsa_sparse_attn_decode_kv8", ctypes.c_int, _vp, _vp, _vp, _f32, _f32, _vp, _vp, _vp, _i32, _i64, _i32, _i32,
@@ -419,6 +421,19 @@ def qsa_sparse_attn_decode_paged(q, k, v, page_table, page_tokens, seq_len, sel,
                                           _ptr(out, q.dtype, "out"), _ptr(lse, torch.float32, "lse"), wp, wb, dt,
                                           _stream(q, stream))
     _check(st, "qsa_sparse_attn_decode_paged")
+
+
+def qsa_dense_attn_prefill(q, k, v, out, q0=0, scale=None, lse=None, stream=None):
+    """Full causal attention of query rows q0 .. q0 + n_q - 1 over every cached position up
+    to each row's own (the dense baseline).  q, out [B][n_q][Hq][d]; k, v [B][L][Hkv][d]."""
+    dt = _dtype_code(q)
+    B, n_q, Hq, d = q.shape
+    Hkv = k.shape[2]
+    scale = (1.0 / d ** 0.5) if scale is None else scale
+    st = lib.qsa_dense_attn_prefill(_ptr(q, None, "q"), _ptr(k, q.dtype, "k"), _ptr(v, q.dtype, "v"), B, n_q, q0,
+                                    k.shape[1], Hq, Hkv, d, scale, _ptr(out, q.dtype, "out"),
+                                    _ptr(lse, torch.float32, "lse"), dt, _stream(q, stream))
+    _check(st, "qsa_dense_attn_prefill")
 
 
 def _kv8_ptr(t, name):

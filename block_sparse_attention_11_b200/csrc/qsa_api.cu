@@ -8,6 +8,7 @@
 #include <mutex>
 
 #include "../../include/qsa.h"
+#include "dense.h"
 #include "internal.h"
 
 namespace qsa {
@@ -408,6 +409,26 @@ int qsa_rope_apply(void *x, int32_t B, int64_t n, int32_t H, int32_t d, int64_t 
     if ((st = check_device(&di)) != QSA_OK) return st;
     return cuda_status(launch_rope_apply(x, B, n, H, d, pos0, to_rope(rope), dtype == QSA_BF16,
                                          static_cast<cudaStream_t>(stream)));
+}
+
+// ---------------------------------------------------------------- dense causal prefill (baseline)
+
+int qsa_dense_attn_prefill(const void *q, const void *k, const void *v, int32_t B, int64_t n_q, int64_t q0,
+                           int64_t kv_stride, int32_t Hq, int32_t Hkv, int32_t d, float scale, void *out, float *lse,
+                           int32_t dtype, void *stream) {
+    if (!q || !k || !v || !out || B < 1 || n_q < 0 || q0 < 0 || kv_stride < q0 + n_q) return QSA_ERR_INVALID_ARG;
+    if (Hq < 1 || Hkv < 1 || (Hq % Hkv) != 0) return QSA_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !std::isfinite(scale)) return QSA_ERR_INVALID_ARG;
+    if (dtype != QSA_BF16 || d != 128 || Hq != 8 * Hkv || (Hkv != 1 && Hkv != 2 && Hkv != 4))
+        return QSA_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return QSA_ERR_INVALID_ARG;
+    if ((int64_t)B * kv_stride > ((int64_t)1 << 31)) return QSA_ERR_UNSUPPORTED;   // TMA row coordinates
+    if (n_q == 0) return QSA_OK;
+    const DeviceInfo *di = nullptr;
+    int st = check_device(&di);
+    if (st != QSA_OK) return st;
+    return cuda_status(launch_dense_prefill(q, k, v, B, n_q, q0, kv_stride, Hkv, scale, out, lse, di->status,
+                                            static_cast<cudaStream_t>(stream)));
 }
 
 // ---------------------------------------------------------------- FP8 K/V caches

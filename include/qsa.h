@@ -363,6 +363,19 @@ QSA_API int qsa_sparse_attn_decode_noalloc(const void *q, const void *k, const v
                                            int32_t Hq, int32_t Hkv, int32_t d, int32_t top_k, float scale, void *out,
                                            float *lse, int32_t dtype, void *stream);
 
+/*
+ * The prefill counterpart: full causal attention of query rows q0 .. q0 +
+ * n_q - 1 over every cached position up to each row's own (the baseline the
+ * pages' 7.6x prefill ratio is quoted against).  Tiled over queries and keys
+ * (each K/V tile is loaded once for 8 queries of a kv head).  QSA_BF16 with
+ * Hq = 8 Hkv, Hkv in {1, 2, 4}, d = 128.  q, out [B][n_q][Hq][d]; k, v
+ * [B][kv_stride][Hkv][d]; lse [B][n_q][Hq] float or NULL; kv_stride >= q0 +
+ * n_q and B * kv_stride <= 2^31.  No workspace.
+ */
+QSA_API int qsa_dense_attn_prefill(const void *q, const void *k, const void *v, int32_t B, int64_t n_q, int64_t q0,
+                                   int64_t kv_stride, int32_t Hq, int32_t Hkv, int32_t d, float scale, void *out,
+                                   float *lse, int32_t dtype, void *stream);
+
 /* ========================================================================= */
 /* FP8 K/V caches                                                             */
 /* ========================================================================= */

@@ -360,6 +360,27 @@ def test_attention_released_shape_decode(qsa, B, L, kv8):
             assert np.abs(np32(outd[b]) - refd[0]).max() <= TOL["bf16"], b
 
 
+@pytest.mark.parametrize("Hq,Hkv,T,q0,B", [(16, 2, 1000, 0, 1), (8, 1, 333, 0, 2), (32, 4, 200, 0, 1),
+                                          (16, 2, 700, 600, 1), (16, 2, 5, 0, 1)])
+def test_dense_prefill_matches_textbook_attention(qsa, Hq, Hkv, T, q0, B):
+    """Full causal prefill attention (the dense baseline) against textbook
+    attention over positions 0..t on every row; q0 > 0: a chunk of rows after
+    a cached prefix."""
+    g = torch.Generator(device=DEV).manual_seed(T + q0 + Hq)
+    L = q0 + T + 3
+    q = torch.randn(B, T, Hq, 128, generator=g, device=DEV).to(torch.bfloat16)
+    k = torch.randn(B, L, Hkv, 128, generator=g, device=DEV).to(torch.bfloat16)
+    v = torch.randn(B, L, Hkv, 128, generator=g, device=DEV).to(torch.bfloat16)
+    out = torch.full_like(q, 9.0)
+    lse = torch.empty(B, T, Hq, dtype=torch.float32, device=DEV)
+    qsa.qsa_dense_attn_prefill(q, k, v, out, q0=q0, lse=lse)
+    qsa.qsa_check_status()
+    rows = list(range(T))
+    for b in range(B):
+        ref = oracle.dense_rows(rows, q=np32(q[b]), k=np32(k[b]), v=np32(v[b]), Hq=Hq, Hkv=Hkv, d=128, q0=q0)
+        assert np.abs(np32(out[b]) - ref).max() <= TOL["bf16"], b
+
+
 def test_attention_flags_out_of_range_ids(qsa):
     """A selection id outside [0, nb(t)) is skipped and reported through the
     status word (no trap)."""

@@ -74,6 +74,11 @@ WORKLOADS = {
     # the 32K prefill workload with FP8 E4M3 K/V caches
     "prefill_t32k_needles_kv8": Workload("prefill_t32k_needles_kv8", "prefill", 1, 32768, 512, 16, 2, 128, "bf16",
                                          1002, needles=64, extra={"kv": "fp8"}),
+    # full causal prefill attention on the QSA prefill workloads' q/k/v (the dense baseline)
+    "dense_prefill_t32k": Workload("dense_prefill_t32k", "dense_prefill", 1, 32768, 512, 16, 2, 128, "bf16", 1002,
+                                   needles=64),
+    "dense_prefill_t128k": Workload("dense_prefill_t128k", "dense_prefill", 1, 131072, 512, 16, 2, 128, "bf16",
+                                    1004, heavy_tail=True),
     # the released model's attention shape: 24 q heads, 2 kv heads of 256 dims (BF16, and the FP8 serving form)
     "prefill_t32k_d256": Workload("prefill_t32k_d256", "prefill", 1, 32768, 512, 24, 2, 256, "bf16", 1002,
                                   needles=64),
@@ -142,7 +147,7 @@ def make_prefill(w: Workload, device="cuda", T: int | None = None):
     Returns dict(q_idx, k_idx, q, k, v, needles) with needles a list of
     (block, [query positions]) when the workload plants them.
     """
-    assert w.kind == "prefill"
+    assert w.kind in ("prefill", "dense_prefill")
     T = T or w.T
     g = _gen(device, w.seed)
     B = w.B
