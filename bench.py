@@ -170,17 +170,27 @@ class PrefillRunner:
             self.x["v"], self.v_scale = workloads.to_e4m3(self.x["v"])
         self.rope = qsa.Rope(base=w.rope_base, pos_scale=w.pos_scale, rotary_dim=128)
         self.k_pool = torch.zeros(B, max(T // 4, 1), 128, dtype=dt, device=dev)
-        self.sel = torch.empty(B, T, w.top_k, dtype=torch.int32, device=dev)
-        self.nsel = torch.empty(B, T, dtype=torch.int32, device=dev)
+        # chunked prefill ("chunk" in extra): each chunk pools its keys into the growing
+        # compressed cache, then selects and attends for its rows at offset q0 = c0
+        self.chunks = chunk_bounds(T, w.extra.get("chunk"))
+        if len(self.chunks) > 1:
+            assert B == 1, "chunked prefill slices [1][T] inputs in place"
+        rows = max(c1 - c0 for c0, c1 in self.chunks)
+        self.sel = torch.empty(B, rows, w.top_k, dtype=torch.int32, device=dev)
+        self.nsel = torch.empty(B, rows, dtype=torch.int32, device=dev)
         self.out = torch.empty_like(self.x["q"])
-        ws = qsa.qsa_index_topk_prefill_workspace(B, T, 0, w.top_k, 0, 0 if w.dtype == "bf16" else 1)
+        ws = max(qsa.qsa_index_topk_prefill_workspace(B, c1 - c0, c0, w.top_k, 0, 0 if w.dtype == "bf16" else 1)
+                 for c0, c1 in self.chunks)
         self.ws = torch.empty(ws, dtype=torch.uint8, device=dev)
         # the step's inputs (~200 MB at T=32K) do not all stay in L2, but the
         # flush keeps every timed step cold
         self.flush_between_steps = True
         self.use_graph = False        # three launches of milliseconds each: nothing to gain
+        self.long_step = T > 262144   # steps of a second or more: shorter end-to-end runs
 
     def step(self, x=None, events=None):
+        if len(self.chunks) > 1:
+            return self.step_chunked(x, events)
         qsa, w = self.qsa, self.w
         x = x or self.x
         if events is not None:
@@ -201,8 +211,49 @@ class PrefillRunner:
             events[3].record()
         return self.out
 
+    def step_chunked(self, x=None, events=None):
+        """One chunked prefill of the whole prompt; per-chunk stage events are
+        appended to `events` (after its first 4) for stage_times."""
+        qsa, w = self.qsa, self.w
+        x = x or self.x
+        if events is not None:
+            del events[4:]
+            events[0].record()
+        for c0, c1 in self.chunks:
+            n = c1 - c0
+            sel, nsel = self.sel[:, :n], self.nsel[:, :n]
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)] if events is not None else None
+            if ev:
+                ev[0].record()
+            qsa.qsa_pool_keys_prefill(x["k_idx"][:, c0:c1], self.k_pool, pos0=c0, rope=self.rope)
+            if ev:
+                ev[1].record()
+            qsa.qsa_index_topk_prefill(x["q_idx"][:, c0:c1], self.k_pool, sel, nsel, q0=c0, top_k=w.top_k,
+                                       rope=self.rope, workspace=self.ws)
+            if ev:
+                ev[2].record()
+            qsa.qsa_sparse_attn_prefill(x["q"][:, c0:c1], x["k"], x["v"], sel, nsel, self.out[:, c0:c1], q0=c0)
+            if ev:
+                ev[3].record()
+                events.extend(ev)
+        if events is not None:
+            events[1].record()
+            events[2].record()
+            events[3].record()
+        return self.out
+
+    def stage_times(self, events):
+        """Stage milliseconds of one step: summed over chunks when chunked."""
+        if len(events) <= 4:
+            return [events[s].elapsed_time(events[s + 1]) for s in range(3)]
+        t = [0.0, 0.0, 0.0]
+        for j in range(4, len(events), 4):
+            for s in range(3):
+                t[s] += events[j + s].elapsed_time(events[j + s + 1])
+        return t
+
     def launches_per_step(self):
-        return 5   # pool, query rotation, score GEMM, row select, attention
+        return 5 * len(self.chunks)   # per chunk: pool, query rotation, score GEMM, row select, attention
 
     def units(self):
         return self.w.B * self.w.T   # tokens
@@ -227,6 +278,12 @@ class PrefillRunner:
 
     def host_inputs(self):
         return {k: v.cpu().pin_memory() for k, v in self.x.items() if isinstance(v, torch.Tensor)}
+
+
+def chunk_bounds(T, chunk):
+    """[(c0, c1)] row ranges of a prefill done in chunks of `chunk` tokens (one range if None)."""
+    chunk = int(chunk or T)
+    return [(c0, min(c0 + chunk, T)) for c0 in range(0, T, chunk)]
 
 
 class DecodeRunner:
@@ -485,10 +542,15 @@ class DensePrefillRunner:
         self.dev = dev
         x = workloads.make_prefill(w, device=dev)
         self.x = {n: x[n] for n in ("q", "k", "v")}
+        del x
         torch.cuda.empty_cache()
-        self.out = torch.empty_like(x["q"])
+        self.out = torch.empty_like(self.x["q"])
+        self.chunks = chunk_bounds(w.T, w.extra.get("chunk"))
+        if len(self.chunks) > 1:
+            assert w.B == 1, "chunked prefill slices [1][T] inputs in place"
         self.flush_between_steps = True
         self.use_graph = False
+        self.long_step = w.T > 65536
 
     def step(self, x=None, events=None):
         x = x or self.x
@@ -496,13 +558,14 @@ class DensePrefillRunner:
             events[0].record()
             events[1].record()
             events[2].record()
-        self.qsa.qsa_dense_attn_prefill(x["q"], x["k"], x["v"], self.out)
+        for c0, c1 in self.chunks:   # query rows c0 .. c1 - 1 over the cache up to each row
+            self.qsa.qsa_dense_attn_prefill(x["q"][:, c0:c1], x["k"], x["v"], self.out[:, c0:c1], q0=c0)
         if events is not None:
             events[3].record()
         return self.out
 
     def launches_per_step(self):
-        return 1
+        return len(self.chunks)
 
     def units(self):
         return self.w.B * self.w.T   # tokens
@@ -606,7 +669,10 @@ def run_ours(args, rank, world):
         stage_ms = [[ev[i][s].elapsed_time(ev[i][s + 1]) for i in range(args.steps)] for s in range(nst)]
     else:
         eager_ms = None
-        stage_ms = [[events[i][s].elapsed_time(events[i][s + 1]) for i in range(args.steps)] for s in range(nst)]
+        split = getattr(runner, "stage_times", None) or (lambda ev: [ev[s].elapsed_time(ev[s + 1])
+                                                                      for s in range(nst)])
+        per_step = [split(events[i]) for i in range(args.steps)]
+        stage_ms = [[per_step[i][s] for i in range(args.steps)] for s in range(nst)]
     total_ms = max_over_ranks(sum(step_ms), world, dev)
     ms_per_step = total_ms / args.steps
 
@@ -615,7 +681,10 @@ def run_ours(args, rank, world):
     h2d = sum(v.numel() * v.element_size() for v in host.values())
     out_host = torch.empty(runner.out.shape, dtype=runner.out.dtype, pin_memory=True)
     d2h = out_host.numel() * out_host.element_size()
-    e2e_steps = max(3, min(args.steps, 10))
+    long_step = getattr(runner, "long_step", False)
+    # steps of a second or more: one warm-up and one timed end-to-end step, serial only
+    e2e_steps = 1 if long_step else max(3, min(args.steps, 10))
+    e2e_warm = 1 if long_step else 2
     dev_x = dict(runner.x)
 
     def e2e_step():
@@ -625,8 +694,8 @@ def run_ours(args, rank, world):
         out_host.copy_(out, non_blocking=True)
 
     def timed(fn):
-        for it in range(e2e_steps + 2):
-            if it == 2:
+        for it in range(e2e_steps + e2e_warm):
+            if it == e2e_warm:
                 torch.cuda.synchronize()
                 e0 = torch.cuda.Event(enable_timing=True)
                 e1 = torch.cuda.Event(enable_timing=True)
@@ -681,8 +750,11 @@ def run_ours(args, rank, world):
         runner.out = keep_out
         return e0.elapsed_time(e1) / n
 
-    e2e_pipelined(2)                    # untimed: allocations and first launches
-    e2e_pipe_ms = e2e_pipelined(e2e_steps)
+    if long_step:
+        e2e_pipe_ms = float("inf")
+    else:
+        e2e_pipelined(2)                # untimed: allocations and first launches
+        e2e_pipe_ms = e2e_pipelined(e2e_steps)
     e2e_ms = min(e2e_serial_ms, e2e_pipe_ms)
     e2e_mode = "pipelined" if e2e_pipe_ms <= e2e_serial_ms else "serial"
     e2e_eager_ms = e2e_serial_ms
@@ -733,7 +805,8 @@ def run_ours(args, rank, world):
                                       note="indexer (2*128 flop per visible (query, block) pair) + attention "
                                            "(4*d*Hq flop per selected position) over the whole step")
         res["config"] = dict(workload=w.name, B=w.B, T=w.T, top_k=w.top_k, Hq=w.Hq, Hkv=w.Hkv, d=w.d,
-                             needles=w.needles, l2="flushed between timed steps (256 MB write)",
+                             needles=w.needles, chunk=w.extra.get("chunk"),
+                             l2="flushed between timed steps (256 MB write)",
                              parallelism=f"replicas x{world}")
     elif w.kind == "dense_prefill":
         res.update(metric=metric_name(w), unit="tokens/s", higher_is_better=True,
@@ -748,7 +821,10 @@ def run_ours(args, rank, world):
                                note="4*d*Hq flop per causal (query, key) pair over the step time; sustained bf16 "
                                     "peak (a step of tens of ms)")
         res["config"] = dict(workload=w.name, B=w.B, T=w.T, Hq=w.Hq, Hkv=w.Hkv, d=w.d,
-                             l2="flushed between timed steps (256 MB write)", parallelism=f"replicas x{world}")
+                             chunk=w.extra.get("chunk"), l2="flushed between timed steps (256 MB write)",
+                             parallelism=f"replicas x{world}")
+        if not args.no_library_context:
+            res["library_context"] = library_dense_context(runner, alg["attn_flops"])
     elif w.kind in ("draft", "dense"):
         res.update(metric=metric_name(w), unit="us/step", higher_is_better=False, value=ms_per_step * 1e3)
         res["e2e"] = dict(value=e2e_ms * 1e3, unit="us/step", h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h,
@@ -787,6 +863,51 @@ def run_ours(args, rank, world):
                              pos_scale=w.pos_scale, l2="inputs larger than L2 (compressed-key cache and K/V caches)",
                              parallelism=f"replicas x{world}", cuda_graph="the K timed steps captured in one graph")
     return res
+
+
+def library_dense_context(runner, flops, reps=2):
+    """Context for the dense comparator, not a figure of this library: cuDNN's
+    fused causal attention (torch SDPA, cuDNN backend) on the same q/k/v as one
+    whole-sequence call per group of q heads (each call's q at most 2^28
+    elements), timed with CUDA events after one untimed call."""
+    import torch.nn.functional as F
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+    w = runner.w
+    q, k, v = (runner.x[n] for n in ("q", "k", "v"))
+    B, T, Hq, d = q.shape
+    G = Hq // w.Hkv
+    hq_call = max(1, min(Hq, (1 << 28) // (B * T * d)))
+    while Hq % hq_call or (hq_call % G and G % hq_call):
+        hq_call -= 1
+    out = torch.empty_like(q)
+
+    def run():
+        for h0 in range(0, Hq, hq_call):
+            kv0, kv1 = h0 // G, (h0 + hq_call - 1) // G + 1
+            o = F.scaled_dot_product_attention(q[:, :, h0:h0 + hq_call].transpose(1, 2),
+                                               k[:, :, kv0:kv1].transpose(1, 2), v[:, :, kv0:kv1].transpose(1, 2),
+                                               is_causal=True, enable_gqa=True)
+            out[:, :, h0:h0 + hq_call] = o.transpose(1, 2)
+
+    try:
+        with sdpa_kernel([SDPBackend.CUDNN_ATTENTION]):
+            run()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(reps):
+                run()
+            e1.record()
+            torch.cuda.synchronize()
+    except Exception as e:   # backend unavailable on this build / device
+        return dict(library="cuDNN fused attention via torch SDPA", unavailable=repr(e)[:160])
+    ms = e0.elapsed_time(e1) / reps
+    tail = slice(max(0, T - 2048), T)
+    diff = (out[:, tail].float() - runner.out[:, tail].float()).abs().max().item()
+    return dict(library="cuDNN fused attention via torch SDPA (context only; not this library)",
+                ms_per_step=ms, tokens_per_s=B * T / (ms / 1e3), tflops=flops / (ms / 1e3) / 1e12,
+                calls_per_step=Hq // hq_call, max_abs_diff_vs_ours_last_2048_rows=diff,
+                note="whole-sequence causal calls (the same (query, key) pairs as the chunked steps)")
 
 
 # ----------------------------------------------------------------------------- CPU oracle arm
@@ -905,6 +1026,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-library-context", action="store_true",
+                    help="full-attention workloads: skip timing cuDNN's attention beside ours")
     ap.add_argument("--batch", type=int, default=None, help="override B (smaller profiling case)")
     ap.add_argument("--tokens", type=int, default=None, help="override T / cache length (smaller profiling case)")
     args = ap.parse_args()
@@ -947,7 +1070,7 @@ def main():
         order = ["metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
                  "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "tensor_roofline", "step_roofline",
                  "e2e",
-                 "cpu_baseline", "gpu_launches", "clocks", "stage_ms"]
+                 "cpu_baseline", "gpu_launches", "clocks", "stage_ms", "library_context"]
         line = {k: res[k] for k in order if k in res}
         print(json.dumps(line), flush=True)
 

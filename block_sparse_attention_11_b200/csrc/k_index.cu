@@ -59,6 +59,8 @@ struct GemmParams {
     const float *head_w;
     float *scores;
     unsigned *status;
+    int nsplit;           // CTAs per row tile, each over `span` key tiles
+    int span;
 };
 
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
@@ -69,12 +71,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int seq = blockIdx.y;
     const int rows_per_tile = p.per_head ? GM / kIdxHeads : GM;
-    const int m = gridDim.x - 1 - blockIdx.x;                 // heaviest (latest) tiles first
+    // row tile m (heaviest, latest rows first), key tiles [j0, j0 + ntiles) of it
+    const int m = (int)(gridDim.x / p.nsplit) - 1 - (int)(blockIdx.x / p.nsplit);
+    const int j0 = (int)(blockIdx.x % p.nsplit) * p.span;
     const int64_t r0 = p.row_begin + (int64_t)m * rows_per_tile;
     const int64_t r_end = min(r0 + rows_per_tile, p.row_begin + p.row_count);
     const int64_t t_last = p.q0 + r_end - 1;
     const int64_t nb_tile = (t_last + 1) / kBlock;
-    const int ntiles = (int)((nb_tile + GN - 1) / GN);
+    const int ntiles = max(0, min((int)((nb_tile + GN - 1) / GN) - j0, p.span));
     const int kplanes = p.per_head ? 1 : 2;
 
     if (threadIdx.x == 0) {
@@ -110,7 +114,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 const int s = j % NST;
                 if (j >= NST) ok = mbar_wait(&sm.b_empty[s], ((j / NST) + 1) & 1, p.status);
                 if (!ok) break;
-                const int by = (int)(seq * p.pool_stride + (int64_t)j * GN);
+                const int by = (int)(seq * p.pool_stride + (int64_t)(j0 + j) * GN);
                 mbar_arrive_expect_tx(&sm.b_full[s], B_STAGE_BYTES);
                 tma_load_2d(sm.b[s], &map_b, 0, by, &sm.b_full[s]);
                 tma_load_2d(sm.b[s] + KATOM_BYTES_B, &map_b, 64, by, &sm.b_full[s]);
@@ -200,8 +204,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     const int64_t q = p.per_head ? r0 + lr / kIdxHeads : r0 + lr;
                     const bool writer = q < r_end && (!p.per_head || (lr % kIdxHeads) == 0);
                     if (writer) {
-                        float *d = p.scores + ((int64_t)seq * p.row_count + (q - p.row_begin)) * p.ld + (int64_t)j * GN +
-                                   c * 32 + 4 * (lane & 7);
+                        float *d = p.scores + ((int64_t)seq * p.row_count + (q - p.row_begin)) * p.ld +
+                                   (int64_t)(j0 + j) * GN + c * 32 + 4 * (lane & 7);
                         *reinterpret_cast<float4 *>(d) = *reinterpret_cast<const float4 *>(&tile[rr][4 * (lane & 7)]);
                     }
                 }
@@ -248,14 +252,16 @@ __global__ void __launch_bounds__(128) score_simt_kernel(const float *__restrict
 }
 
 // Per-row top-k over materialised scores: one warp per (row, sequence), 16
-// rows per CTA, no CTA barriers (see warp_topk_row).
+// rows per CTA, no CTA barriers (see warp_topk_row).  kWide: rows of more
+// than 65535 visible blocks (positions from 262140 on) count in 32 bits.
 constexpr int SEL_WARPS = 16;
 
+template <bool kWide>
 __global__ void __launch_bounds__(SEL_WARPS * 32, 2)
     select_rows_kernel(const float *__restrict__ scores, int64_t row_begin, int64_t n_q, int64_t q0, int64_t ld,
                        int top_k, int32_t *__restrict__ sel, int32_t *__restrict__ nsel, int64_t row_count) {
     extern __shared__ uint8_t ssm_raw[];
-    WarpSelSmem *wsm = reinterpret_cast<WarpSelSmem *>(ssm_raw);
+    WarpSelSmemT<kWide> *wsm = reinterpret_cast<WarpSelSmemT<kWide> *>(ssm_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int seq = blockIdx.y;
     const int64_t rloc = (int64_t)blockIdx.x * SEL_WARPS + warp;
@@ -268,6 +274,219 @@ __global__ void __launch_bounds__(SEL_WARPS * 32, 2)
     const int cnt = warp_topk_row(src, n, top_k, wsm[warp], [&](int pos, int i) { out[pos] = i; });
     for (int i = cnt + lane; i < top_k; i += 32) out[i] = -1;
     if (lane == 0) nsel[(int64_t)seq * n_q + row] = cnt;
+}
+
+// ---- long rows: one CTA per row, two passes over the row
+//
+// The warp kernel reads a row three times (five when the bin of the k-th key
+// overflows its list), and one warp keeps too few loads in flight for rows of
+// 10^5 scores.  Here a CTA of SR_THREADS takes one row:
+//   pass 1  11-bit histogram of the top digit of every key; a CTA scan finds
+//           the bin d1 holding the k-th largest key and k_rem, the number of
+//           picks that bin supplies;
+//   pass 2  every element of a higher bin is picked (exactly k - k_rem of
+//           them); the elements of bin d1 are listed as (~key << 32 | id);
+//   rank    the list is sorted ascending (key descending, id ascending: the
+//           ranking's tie rule) and its first k_rem ids are picked;
+//   order   the k picked ids are sorted ascending and written.
+// A bin of more than SR_TIE_CAP elements (massive ties) falls back to the
+// warp kernel's passes, run by warp 0.
+constexpr int SR_THREADS = 256;
+constexpr int SR_TIE_CAP = 4096;
+constexpr int SR_SPAN = SR_THREADS * 16;   // elements per iteration: four float4 per thread
+constexpr int SR_MIN_BLOCKS = 16384;       // longest row of a launch from which this kernel is used
+
+struct RowSelSmem {
+    uint32_t hist[2048];
+    union {
+        unsigned long long tie[SR_TIE_CAP];
+        WarpSelSmemT<true> warp;            // fallback
+    };
+    uint32_t pick[2048];                    // picked ids (top_k <= 2048)
+    uint32_t wsum[SR_THREADS / 32];
+    int n_sure, n_tie, d1, k_rem;
+};
+
+// Ascending bitonic sort of a[0, P), P a power of two; all threads of the CTA.
+template <typename T>
+__device__ __forceinline__ void cta_bitonic_sort(T *a, int P) {
+    for (int size = 2; size <= P; size <<= 1)
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            for (int i = threadIdx.x; i < P / 2; i += blockDim.x) {
+                const int lo = 2 * i - (i & (stride - 1));
+                const int hi = lo + stride;
+                const bool up = (lo & size) == 0;
+                const T x = a[lo], y = a[hi];
+                if ((x > y) == up) {
+                    a[lo] = y;
+                    a[hi] = x;
+                }
+            }
+            __syncthreads();
+        }
+}
+
+__device__ __forceinline__ int pow2_ceil(int x) {
+    int p = 1;
+    while (p < x) p <<= 1;
+    return p;
+}
+
+// Element i0 + 4 * tid + SR_THREADS * 4 * u + c of the row, u < 4, c < 4.
+template <bool kLast>
+__device__ __forceinline__ void sr_load(const float *row, int n, int base, float (&f)[4][4]) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int i = base + u * SR_THREADS * 4 + 4 * (int)threadIdx.x;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        // i < n <= ld and ld % 4 == 0: the whole float4 lies inside the row's stride
+        if (i < n) v = kLast ? __ldcs(reinterpret_cast<const float4 *>(row + i))
+                             : *reinterpret_cast<const float4 *>(row + i);
+        f[u][0] = v.x;
+        f[u][1] = v.y;
+        f[u][2] = v.z;
+        f[u][3] = v.w;
+    }
+}
+
+__global__ void __launch_bounds__(SR_THREADS)
+    select_rows_cta_kernel(const float *__restrict__ scores, int64_t row_begin, int64_t n_q, int64_t q0,
+                           int64_t ld, int top_k, int32_t *__restrict__ sel, int32_t *__restrict__ nsel,
+                           int64_t row_count) {
+    extern __shared__ __align__(16) uint8_t rsm_raw[];
+    RowSelSmem &sm = *reinterpret_cast<RowSelSmem *>(rsm_raw);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const uint32_t lt = (1u << lane) - 1u;
+    const int seq = blockIdx.y;
+    const int64_t rloc = blockIdx.x;
+    const int64_t row = row_begin + rloc;
+    const int n = (int)((q0 + row + 1) / kBlock);
+    const int k = top_k;
+    const float *src = scores + ((int64_t)seq * row_count + rloc) * ld;
+    int32_t *out = sel + ((int64_t)seq * n_q + row) * top_k;
+    int32_t *cnt_out = nsel + (int64_t)seq * n_q + row;
+    if (n <= k) {
+        for (int i = tid; i < k; i += SR_THREADS) out[i] = i < n ? i : -1;
+        if (tid == 0) *cnt_out = n;
+        return;
+    }
+    for (int i = tid; i < 2048; i += SR_THREADS) sm.hist[i] = 0;
+    if (tid == 0) sm.n_sure = sm.n_tie = 0;
+    __syncthreads();
+
+    // ---- pass 1: histogram of the top 11 bits
+    for (int base = 0; base < n; base += SR_SPAN) {
+        float f[4][4];
+        sr_load<false>(src, n, base, f);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                if (base + u * SR_THREADS * 4 + 4 * tid + c < n) atomicAdd(&sm.hist[score_key(f[u][c]) >> 21], 1u);
+    }
+    __syncthreads();
+
+    // ---- the bin holding the k-th largest key: thread t owns bins 2047-8t .. 2040-8t
+    {
+        const int top_bin = 2047 - 8 * tid;
+        uint32_t mine = 0;
+#pragma unroll
+        for (int b = 0; b < 8; ++b) mine += sm.hist[top_bin - b];
+        uint32_t incl = mine;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        if (lane == 31) sm.wsum[warp] = incl;
+        __syncthreads();
+        uint32_t cum = incl - mine;
+        for (int w = 0; w < warp; ++w) cum += sm.wsum[w];
+        if (cum < (uint32_t)k && cum + mine >= (uint32_t)k) {
+            for (int b = 0; b < 8; ++b) {
+                const uint32_t h = sm.hist[top_bin - b];
+                if (cum + h >= (uint32_t)k) {
+                    sm.d1 = top_bin - b;
+                    sm.k_rem = k - (int)cum;
+                    break;
+                }
+                cum += h;
+            }
+        }
+        __syncthreads();
+    }
+    const uint32_t d1 = (uint32_t)sm.d1;
+    const int k_rem = sm.k_rem;
+
+    // ---- pass 2: pick the higher bins, list bin d1
+    for (int base = 0; base < n; base += SR_SPAN) {
+        float f[4][4];
+        sr_load<true>(src, n, base, f);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i0 = base + u * SR_THREADS * 4 + 4 * tid;
+            uint32_t key[4];
+            bool above[4], in_bin[4];
+            bool any = false;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                key[c] = score_key(f[u][c]);
+                const bool live = i0 + c < n;
+                above[c] = live && (key[c] >> 21) > d1;
+                in_bin[c] = live && (key[c] >> 21) == d1;
+                any |= above[c] || in_bin[c];
+            }
+            if (!__any_sync(0xffffffffu, any)) continue;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const uint32_t ba = __ballot_sync(0xffffffffu, above[c]);
+                if (ba) {
+                    const int leader = __ffs(ba) - 1;
+                    int slot0 = 0;
+                    if (lane == leader) slot0 = atomicAdd(&sm.n_sure, __popc(ba));
+                    slot0 = __shfl_sync(0xffffffffu, slot0, leader);
+                    const int slot = slot0 + __popc(ba & lt);
+                    if (above[c] && slot < 2048) sm.pick[slot] = (uint32_t)(i0 + c);
+                }
+                const uint32_t bt = __ballot_sync(0xffffffffu, in_bin[c]);
+                if (bt) {
+                    const int leader = __ffs(bt) - 1;
+                    int slot0 = 0;
+                    if (lane == leader) slot0 = atomicAdd(&sm.n_tie, __popc(bt));
+                    slot0 = __shfl_sync(0xffffffffu, slot0, leader);
+                    const int slot = slot0 + __popc(bt & lt);
+                    if (in_bin[c] && slot < SR_TIE_CAP)
+                        sm.tie[slot] = ((unsigned long long)(~key[c]) << 32) | (uint32_t)(i0 + c);
+                }
+            }
+        }
+    }
+    __syncthreads();
+    const int m = sm.n_tie;
+    const int n_sure = sm.n_sure;
+    if (m > SR_TIE_CAP || n_sure != k - k_rem) {
+        // massive ties: the warp kernel's passes (the union's list is no longer needed)
+        if (warp == 0) {
+            const int cnt = warp_topk_row(src, n, k, sm.warp, [&](int pos, int i) { out[pos] = i; });
+            for (int i = cnt + lane; i < k; i += 32) out[i] = -1;
+            if (lane == 0) *cnt_out = cnt;
+        }
+        return;
+    }
+
+    // ---- rank bin d1: key descending, id ascending; its first k_rem are picked
+    const int P = pow2_ceil(max(m, 2));
+    for (int i = m + tid; i < P; i += SR_THREADS) sm.tie[i] = ~0ull;
+    __syncthreads();
+    cta_bitonic_sort(sm.tie, P);
+    for (int j = tid; j < k_rem; j += SR_THREADS) sm.pick[n_sure + j] = (uint32_t)sm.tie[j];
+    // ---- ascending ids
+    const int P2 = pow2_ceil(max(k, 2));
+    for (int i = k + tid; i < P2; i += SR_THREADS) sm.pick[i] = 0xFFFFFFFFu;
+    __syncthreads();
+    cta_bitonic_sort(sm.pick, P2);
+    for (int i = tid; i < k; i += SR_THREADS) out[i] = (int32_t)sm.pick[i];
+    if (tid == 0) *cnt_out = k;
 }
 
 // Driver-API tensor-map encoder obtained through the runtime (no -lcuda).
@@ -310,7 +529,17 @@ cudaError_t launch_score_gemm(const ScoreGemmArgs &a, const void *qa0, const voi
     if (!make_map(&ma1, a.per_head ? qa0 : qa1, a_rows, GM)) return cudaErrorInvalidValue;
     if (!make_map(&mb, k_pool, (uint64_t)a.B * a.pool_stride, GN)) return cudaErrorInvalidValue;
     GemmParams p{a.n_q, a.q0, a.row_begin, a.row_count, a.pool_stride, a.ld, a.per_head, a.relu, a.head_w,
-                 a.scores, status};
+                 a.scores, status, 1, 0};
+    // Split each row tile's key tiles over several CTAs so that the grid holds
+    // about four CTAs per SM whatever the row count (a 2048-row chunk of a
+    // 1M-token context has 16 row tiles of 2048 key tiles each).
+    const int64_t row_tiles = (a.row_count + rows_per_tile - 1) / rows_per_tile;
+    const int64_t max_tiles = ((a.q0 + a.row_begin + a.row_count) / kBlock + GN - 1) / GN;
+    const DeviceInfo *di = device_info();
+    const int64_t want = 4 * (int64_t)(di ? di->sm_count : 148);
+    const int64_t nsplit = std::max<int64_t>(1, std::min<int64_t>(max_tiles, (want + row_tiles * a.B - 1) / (row_tiles * a.B)));
+    p.nsplit = (int)nsplit;
+    p.span = (int)std::max<int64_t>(1, (max_tiles + nsplit - 1) / nsplit);
     const size_t smem = sizeof(GemmSmem) + 1024;
     static bool attr_done = false;
     if (!attr_done) {
@@ -318,7 +547,7 @@ cudaError_t launch_score_gemm(const ScoreGemmArgs &a, const void *qa0, const voi
         if (e != cudaSuccess) return e;
         attr_done = true;
     }
-    dim3 grid((unsigned)((a.row_count + rows_per_tile - 1) / rows_per_tile), (unsigned)a.B);
+    dim3 grid((unsigned)(row_tiles * nsplit), (unsigned)a.B);
     score_gemm_kernel<<<grid, GEMM_THREADS, smem, s>>>(ma0, ma1, mb, p);
     return cudaGetLastError();
 }
@@ -339,11 +568,24 @@ cudaError_t launch_select_rows(const float *scores, int B, int64_t row_begin, in
                                cudaStream_t s) {
     (void)status;
     if (row_count <= 0) return cudaSuccess;
-    const size_t smem = SEL_WARPS * sizeof(WarpSelSmem);
-    cudaError_t e = cudaFuncSetAttribute(select_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const int64_t n_max = (q0 + row_begin + row_count) / kBlock;   // the longest row's blocks
+    if (n_max >= SR_MIN_BLOCKS) {
+        const size_t smem = sizeof(RowSelSmem);
+        cudaError_t e = cudaFuncSetAttribute(select_rows_cta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+        dim3 grid((unsigned)row_count, (unsigned)B);
+        select_rows_cta_kernel<<<grid, SR_THREADS, smem, s>>>(scores, row_begin, n_q, q0, ld, top_k, sel, nsel,
+                                                              row_count);
+        return cudaGetLastError();
+    }
+    const bool wide = n_max > kWarpSelNarrowMax;
+    auto kernel = wide ? select_rows_kernel<true> : select_rows_kernel<false>;
+    const size_t smem = SEL_WARPS * (wide ? sizeof(WarpSelSmemT<true>) : sizeof(WarpSelSmemT<false>));
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)((row_count + SEL_WARPS - 1) / SEL_WARPS), (unsigned)B);
-    select_rows_kernel<<<grid, SEL_WARPS * 32, smem, s>>>(scores, row_begin, n_q, q0, ld, top_k, sel, nsel, row_count);
+    kernel<<<grid, SEL_WARPS * 32, smem, s>>>(scores, row_begin, n_q, q0, ld, top_k, sel, nsel, row_count);
     return cudaGetLastError();
 }
 

@@ -209,7 +209,6 @@ int qsa_index_topk_prefill(const void *q_idx, const void *k_pool, const float *h
     const PrefillPlan pl = prefill_plan(B, n_q, q0, flags, dtype, head_w != nullptr);
     if (!workspace || ws_bytes < pl.q_bytes + pl.score_bytes) return QSA_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return QSA_ERR_INVALID_ARG;
-    if ((size_t)pl.ld * 4 > di->smem_optin) return QSA_ERR_UNSUPPORTED;   // one row's scores in smem
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     void *q0buf = ws;

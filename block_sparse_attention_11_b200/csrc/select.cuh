@@ -213,8 +213,9 @@ namespace qsa {
 //
 // Same ranking and output as cta_topk, for one row per warp and no CTA
 // barriers, so many rows are in flight per SM:
-//   pass 1  11-bit histogram of the top digit (two 16-bit counters per word,
-//           shared-memory atomics);
+//   pass 1  11-bit histogram of the top digit (shared-memory atomics; two
+//           16-bit counters per word for rows below 65536 elements, one
+//           32-bit counter per bin for longer rows, kWide);
 //   pass 2  the keys of the bin holding K* are gathered into a per-warp list
 //           and the remaining 21 bits are resolved on it (if the bin overflows
 //           the list, they are resolved on the row instead);
@@ -223,18 +224,26 @@ namespace qsa {
 // ---------------------------------------------------------------------------
 constexpr int kWarpSelBuf = 512;
 
-struct WarpSelSmem {
-    uint32_t hist[1024];          // 2048 16-bit counters
+// A bin of the narrow form counts to 65535: rows of fewer than 65536
+// elements only; longer rows take kWide (2048 32-bit counters).
+template <bool kWide>
+struct WarpSelSmemT {
+    uint32_t hist[kWide ? 2048 : 1024];
     uint32_t buf[kWarpSelBuf];    // keys of the threshold bin
 };
+using WarpSelSmem = WarpSelSmemT<false>;
+constexpr int kWarpSelNarrowMax = 65535;   // longest row of the narrow form
 
-__device__ __forceinline__ uint32_t wsel_count(const WarpSelSmem &w, int bin) {
-    return (w.hist[bin >> 1] >> (16 * (bin & 1))) & 0xFFFFu;
+template <bool kWide>
+__device__ __forceinline__ uint32_t wsel_count(const WarpSelSmemT<kWide> &w, int bin) {
+    if constexpr (kWide) return w.hist[bin];
+    else return (w.hist[bin >> 1] >> (16 * (bin & 1))) & 0xFFFFu;
 }
 
 // Find the digit holding the k_rem-th largest among nbins (<= 2048) counters;
 // returns digit and updates k_rem.  Lane l owns bins [l*per, l*per + per).
-__device__ __forceinline__ int wsel_find(const WarpSelSmem &w, int nbins, int &k_rem) {
+template <bool kWide>
+__device__ __forceinline__ int wsel_find(const WarpSelSmemT<kWide> &w, int nbins, int &k_rem) {
     const int lane = threadIdx.x & 31;
     const int per = nbins / 32;
     uint32_t mine = 0;
@@ -261,16 +270,22 @@ __device__ __forceinline__ int wsel_find(const WarpSelSmem &w, int nbins, int &k
     return digit;
 }
 
-__device__ __forceinline__ void wsel_clear(WarpSelSmem &w, int nbins) {
+template <bool kWide>
+__device__ __forceinline__ void wsel_clear(WarpSelSmemT<kWide> &w, int nbins) {
     const int lane = threadIdx.x & 31;
-    for (int i = lane; i < nbins / 2; i += 32) w.hist[i] = 0;
+    for (int i = lane; i < (kWide ? nbins : nbins / 2); i += 32) w.hist[i] = 0;
     __syncwarp();
 }
 
 // Plain shared-memory atomics: cheaper here than aggregating equal digits
 // with match_any (measured on B200: 1.06 vs 1.43 ms for the 32K-token indexer).
-__device__ __forceinline__ void wsel_add(WarpSelSmem &w, bool live, uint32_t bin) {
-    if (live) atomicAdd(&w.hist[bin >> 1], 1u << (16 * (bin & 1)));
+template <bool kWide>
+__device__ __forceinline__ void wsel_add(WarpSelSmemT<kWide> &w, bool live, uint32_t bin) {
+    if constexpr (kWide) {
+        if (live) atomicAdd(&w.hist[bin], 1u);
+    } else {
+        if (live) atomicAdd(&w.hist[bin >> 1], 1u << (16 * (bin & 1)));
+    }
 }
 
 // Loads element chunk [base + 4*lane, +4) of the row as keys (invalid -> live=false).
@@ -312,9 +327,11 @@ __device__ __forceinline__ void wsel_load4x4(const float *row, int n, int base, 
     }
 }
 
-// Top-k of one row; emit(pos, i) in ascending i.  Returns the count.  Whole warp.
-template <typename Emit>
-__device__ __forceinline__ int warp_topk_row(const float *row, int n, int k, WarpSelSmem &w, Emit &&emit) {
+// Top-k of one row; emit(pos, i) in ascending i, pos < k.  Returns the count
+// (min(n, k)).  Whole warp.  kWide is required for n > kWarpSelNarrowMax.
+template <bool kWide, typename Emit>
+__device__ __forceinline__ int warp_topk_row(const float *row, int n, int k, WarpSelSmemT<kWide> &w,
+                                             Emit &&emit) {
     const int lane = threadIdx.x & 31;
     const uint32_t lt = (1u << lane) - 1u;
     if (n <= k) {
@@ -430,13 +447,16 @@ __device__ __forceinline__ int warp_topk_row(const float *row, int n, int k, War
             int pos = out_run + sel_incl - nsel;
 #pragma unroll
             for (int c = 0; c < 4; ++c)
-                if (sel[c]) emit(pos++, base + 4 * lane + c);
+                if (sel[c]) {
+                    if (pos < k) emit(pos, base + 4 * lane + c);   // exact counts give pos < k always
+                    ++pos;
+                }
             out_run += __shfl_sync(0xffffffffu, sel_incl, 31);
             eq_run += __shfl_sync(0xffffffffu, eq_incl, 31);
         }
     }
     (void)lt;
-    return out_run;
+    return min(out_run, k);
 }
 
 }  // namespace qsa

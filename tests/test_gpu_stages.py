@@ -381,6 +381,88 @@ def test_dense_prefill_matches_textbook_attention(qsa, Hq, Hkv, T, q0, B):
         assert np.abs(np32(out[b]) - ref).max() <= TOL["bf16"], b
 
 
+@pytest.mark.parametrize("q0", [262100, 262130, 1048000])
+def test_prefill_chunk_beyond_65535_blocks_all_ties(qsa, q0):
+    """Chunked prefill rows near and beyond position 262143, from which a row
+    scores more than 65535 blocks: the cache's indexer keys are zero except
+    300 planted blocks, so nearly every block scores exactly 0 and falls in
+    one histogram bin of the row select (ties go to the lower block id).
+    Selections (bit-exact) and attention against the oracle.  Chunk 262100
+    ends at 65533 blocks per row, chunk 262130 crosses the line, chunk
+    1048000 sits at a 1M-token context."""
+    n_q = 32
+    L = q0 + n_q
+    g = torch.Generator(device=DEV).manual_seed(q0)
+    k_idx = torch.zeros(1, L, 128, device=DEV)
+    planted = torch.randperm(L // 4, generator=g, device=DEV)[:300]
+    tok = (4 * planted[:, None] + torch.arange(4, device=DEV)).reshape(-1)
+    k_idx[0, tok] = 3 * torch.randn(tok.numel(), 128, generator=g, device=DEV)
+    k_idx = k_idx.to(torch.bfloat16)
+    q_idx = torch.randn(1, n_q, 4, 128, generator=g, device=DEV).to(torch.bfloat16)
+    q = torch.randn(1, n_q, 16, 128, generator=g, device=DEV).to(torch.bfloat16)
+    k = torch.randn(1, L, 2, 128, generator=g, device=DEV).to(torch.bfloat16)
+    v = torch.randn(1, L, 2, 128, generator=g, device=DEV).to(torch.bfloat16)
+    rope = qsa.Rope()
+    k_pool = torch.zeros(1, L // 4, 128, dtype=torch.bfloat16, device=DEV)
+    qsa.qsa_pool_keys_prefill(k_idx, k_pool, rope=rope)
+    sel = torch.full((1, n_q, 512), -7, dtype=torch.int32, device=DEV)
+    nsel = torch.full((1, n_q), -7, dtype=torch.int32, device=DEV)
+    qsa.qsa_index_topk_prefill(q_idx, k_pool, sel, nsel, q0=q0, top_k=512, rope=rope)
+    out = torch.empty_like(q)
+    qsa.qsa_sparse_attn_prefill(q, k, v, sel, nsel, out, q0=q0)
+    qsa.qsa_check_status()
+    kp = oracle.pool_keys(np32(k_idx[0]), store_bf16=True)
+    assert np.array_equal(np32(k_pool[0]), kp)
+    rows = [0, 5, 11, 18, 31]
+    ref = oracle.prefill_rows(rows, q_idx=np32(q_idx[0]), k_pool=kp, top_k=512, store_bf16=True, q=np32(q[0]),
+                              k=np32(k[0]), v=np32(v[0]), Hq=16, Hkv=2, d=128, q0=q0)
+    assert np.array_equal(nsel[0].cpu().numpy()[rows], ref["nsel"])
+    assert np.array_equal(sel[0].cpu().numpy()[rows], ref["sel"])
+    assert np.abs(np32(out[0])[rows] - ref["out"]).max() <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("keys", ["groups", "random"])
+def test_prefill_long_rows_select(qsa, keys):
+    """Rows of about 17500 blocks (the CTA-per-row select).  "groups": every
+    block's key is one of 64 vectors and the rotation is the identity
+    (pos_scale 1e15), so each row's scores take 64 values, each shared
+    exactly by ~270 blocks: the top-512 end inside a group of exact ties
+    ranked by block id (bit-exact against the oracle).  "random": the usual
+    case under the near-tie acceptance rule."""
+    n_q, q0 = 32, 69984
+    L = q0 + n_q
+    g = torch.Generator(device=DEV).manual_seed(L)
+    if keys == "groups":
+        rope = qsa.Rope(pos_scale=1e15)
+        vecs = torch.randn(64, 128, generator=g, device=DEV).to(torch.bfloat16)
+        grp = torch.randint(0, 64, (L // 4,), generator=g, device=DEV)
+        k_idx = vecs[grp].repeat_interleave(4, dim=0)[None].contiguous()
+    else:
+        rope = qsa.Rope()
+        k_idx = torch.randn(1, L, 128, generator=g, device=DEV).to(torch.bfloat16)
+    q_idx = torch.randn(1, n_q, 4, 128, generator=g, device=DEV).to(torch.bfloat16)
+    k_pool = torch.zeros(1, L // 4, 128, dtype=torch.bfloat16, device=DEV)
+    qsa.qsa_pool_keys_prefill(k_idx, k_pool, rope=rope)
+    sel = torch.full((1, n_q, 512), -7, dtype=torch.int32, device=DEV)
+    nsel = torch.full((1, n_q), -7, dtype=torch.int32, device=DEV)
+    qsa.qsa_index_topk_prefill(q_idx, k_pool, sel, nsel, q0=q0, top_k=512, rope=rope)
+    qsa.qsa_check_status()
+    kp = oracle.pool_keys(np32(k_idx[0]), pos_scale=rope.pos_scale, store_bf16=True)
+    assert np.array_equal(np32(k_pool[0]), kp)
+    rows = list(range(n_q))
+    kw = dict(q_idx=np32(q_idx[0]), k_pool=kp, top_k=512, store_bf16=True, pos_scale=rope.pos_scale, q0=q0)
+    ref = oracle.prefill_rows(rows, **kw)
+    g_sel, g_nsel = sel[0].cpu().numpy(), nsel[0].cpu().numpy()
+    if keys == "groups":
+        assert np.array_equal(g_nsel, ref["nsel"])
+        assert np.array_equal(g_sel, ref["sel"])
+    else:
+        from qsa_testlib import selection_report
+        _, _, nbad = selection_report(g_sel, g_nsel, ref,
+                                      lambda rr: oracle.prefill_rows(rr, want_scores=True, **kw)["scores"], rows)
+        assert nbad <= 2
+
+
 def test_attention_flags_out_of_range_ids(qsa):
     """A selection id outside [0, nb(t)) is skipped and reported through the
     status word (no trap)."""

@@ -79,6 +79,12 @@ WORKLOADS = {
                                    needles=64),
     "dense_prefill_t128k": Workload("dense_prefill_t128k", "dense_prefill", 1, 131072, 512, 16, 2, 128, "bf16",
                                     1004, heavy_tail=True),
+    # a 1M-token prompt prefilled in chunks of 16,000 tokens (the pages' speed comparison), QSA and full
+    # attention on the same inputs (heavy-tailed like the 128K workload)
+    "prefill_l1m_chunk16k": Workload("prefill_l1m_chunk16k", "prefill", 1, 1048576, 512, 16, 2, 128, "bf16", 1007,
+                                     heavy_tail=True, extra={"chunk": 16000}),
+    "dense_prefill_l1m_chunk16k": Workload("dense_prefill_l1m_chunk16k", "dense_prefill", 1, 1048576, 512, 16, 2,
+                                           128, "bf16", 1007, heavy_tail=True, extra={"chunk": 16000}),
     # the released model's attention shape: 24 q heads, 2 kv heads of 256 dims (BF16, and the FP8 serving form)
     "prefill_t32k_d256": Workload("prefill_t32k_d256", "prefill", 1, 32768, 512, 24, 2, 256, "bf16", 1002,
                                   needles=64),
