@@ -246,8 +246,18 @@ template <bool kWide>
 __device__ __forceinline__ int wsel_find(const WarpSelSmemT<kWide> &w, int nbins, int &k_rem) {
     const int lane = threadIdx.x & 31;
     const int per = nbins / 32;
+    // the lane's words are visited rotated by its lane index, so the 32 lanes
+    // read 32 different banks (in order, all lanes would hit one bank)
     uint32_t mine = 0;
-    for (int b = 0; b < per; ++b) mine += wsel_count(w, per * lane + b);
+    if constexpr (kWide) {
+        for (int j = 0; j < per; ++j) mine += w.hist[per * lane + ((j + lane) & (per - 1))];
+    } else {
+        const int pw = per / 2;                       // words per lane, two 16-bit counters each
+        for (int j = 0; j < pw; ++j) {
+            const uint32_t x = w.hist[pw * lane + ((j + lane) & (pw - 1))];
+            mine += (x & 0xFFFFu) + (x >> 16);
+        }
+    }
     uint32_t incl = mine;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
