@@ -424,48 +424,40 @@ __device__ __forceinline__ int warp_topk_row(const float *row, int n, int k, War
             const int base = base4 + 128 * u;
             const uint32_t(&key)[4] = key4[u];
             const bool(&live)[4] = live4[u];
-            int ngt = 0, neq = 0;
+            // element order is (lane, c): ranks come from ballots, lanes below
+            // plus this lane's earlier elements
+            bool gt[4], eq[4];
+            uint32_t be[4];
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                ngt += live[c] && key[c] > kstar;
-                neq += live[c] && key[c] == kstar;
+                gt[c] = live[c] && key[c] > kstar;
+                eq[c] = live[c] && key[c] == kstar;
+                be[c] = __ballot_sync(0xffffffffu, eq[c]);
             }
-            // exclusive prefix of equal keys over lanes (lane order = element order)
-            int eq_incl = neq;
+            int eq_before = eq_run;
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int v = __shfl_up_sync(0xffffffffu, eq_incl, o);
-                if (lane >= o) eq_incl += v;
-            }
-            int eq_before = eq_run + eq_incl - neq;
-            int nsel = 0;
+            for (int c = 0; c < 4; ++c) eq_before += __popc(be[c] & lt);
             bool sel[4];
+            uint32_t bs[4];
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                const bool gt = live[c] && key[c] > kstar;
-                const bool eq = live[c] && key[c] == kstar;
-                sel[c] = gt || (eq && eq_before < take_eq);
-                eq_before += eq;
-                nsel += sel[c];
+                sel[c] = gt[c] || (eq[c] && eq_before < take_eq);
+                eq_before += eq[c];
+                bs[c] = __ballot_sync(0xffffffffu, sel[c]);
             }
-            int sel_incl = nsel;
+            int pos = out_run;
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int v = __shfl_up_sync(0xffffffffu, sel_incl, o);
-                if (lane >= o) sel_incl += v;
-            }
-            int pos = out_run + sel_incl - nsel;
+            for (int c = 0; c < 4; ++c) pos += __popc(bs[c] & lt);
 #pragma unroll
             for (int c = 0; c < 4; ++c)
                 if (sel[c]) {
                     if (pos < k) emit(pos, base + 4 * lane + c);   // exact counts give pos < k always
                     ++pos;
                 }
-            out_run += __shfl_sync(0xffffffffu, sel_incl, 31);
-            eq_run += __shfl_sync(0xffffffffu, eq_incl, 31);
+            out_run += __popc(bs[0]) + __popc(bs[1]) + __popc(bs[2]) + __popc(bs[3]);
+            eq_run += __popc(be[0]) + __popc(be[1]) + __popc(be[2]) + __popc(be[3]);
         }
     }
-    (void)lt;
     return min(out_run, k);
 }
 
