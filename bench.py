@@ -804,6 +804,18 @@ def run_ours(args, rank, world):
                                       frac=tf / pk["bf16_tflops"], peak_kind=pk_kind,
                                       note="indexer (2*128 flop per visible (query, block) pair) + attention "
                                            "(4*d*Hq flop per selected position) over the whole step")
+        # per stage, the slower of its flops at the bf16 peak and its algorithmic bytes at the HBM
+        # peak, summed, over the measured step (the attention's gathers are served from L2 when the
+        # unique K/V fits there, so this can exceed 1)
+        hbm, tens = pk["hbm_gbs"] * 1e9, pk["bf16_tflops"] * 1e12
+        el = 2 if w.dtype == "bf16" else 4
+        pool_b = w.B * w.T * 128 * el * 1.25
+        idx_b = w.B * w.T * (4 * 128 * el + w.top_k * 4 + 4) + w.B * (w.T // 4) * 128 * el
+        t_bound = (pool_b / hbm + max(alg["idx_flops"] / tens, idx_b / hbm)
+                   + max(alg["attn_flops"] / tens, alg["attn_bytes"] / hbm))
+        res["bound_aware"] = dict(bound_ms=t_bound * 1e3, frac=t_bound * 1e3 / ms_per_step,
+                                  note="sum over pool, indexer, attention of max(flops / bf16 peak, algorithmic "
+                                       "bytes / HBM peak), over the measured step time")
         res["config"] = dict(workload=w.name, B=w.B, T=w.T, top_k=w.top_k, Hq=w.Hq, Hkv=w.Hkv, d=w.d,
                              needles=w.needles, chunk=w.extra.get("chunk"),
                              l2="flushed between timed steps (256 MB write)",
@@ -912,6 +924,9 @@ def library_dense_context(runner, flops, reps=2):
 
 # ----------------------------------------------------------------------------- CPU oracle arm
 
+ORACLE_EXTRA = {}   # figures beside the main oracle timing (the one-thread rate), per run
+
+
 def run_oracle_sample(w, budget_s=15.0, seed=0):
     """Time the CPU oracle on a bounded sample of the workload; returns
     (value in the workload's unit, sample description, threads)."""
@@ -943,6 +958,15 @@ def run_oracle_sample(w, budget_s=15.0, seed=0):
         per_row = elapsed / done
         total = t_pool + per_row * w.T * w.B
         value = w.T * w.B / total
+        # one thread on a short sample of the same rows' distribution
+        rows1 = rng.integers(0, w.T, 32)
+        t0 = time.perf_counter()
+        oracle.prefill_rows(rows1, q_idx=q_idx, k_pool=kp, top_k=w.top_k, base=w.rope_base,
+                            pos_scale=w.pos_scale, store_bf16=w.dtype == "bf16", q=q, k=k, v=v, Hq=w.Hq,
+                            Hkv=w.Hkv, d=w.d, nthreads=1)
+        per_row1 = (time.perf_counter() - t0) / len(rows1)
+        ORACLE_EXTRA["value_1thread"] = w.T * w.B / (t_pool + per_row1 * w.T * w.B)
+        ORACLE_EXTRA["sample_1thread"] = "32 uniformly drawn rows, one thread, extrapolated the same way"
         sample = (f"{done} uniformly drawn query rows of the {w.T}-token workload (full indexer scan, top-k, "
                   f"attention per row) + pooling of all keys; extrapolated per row to all rows")
         return value, sample, nthreads, "tokens/s"
@@ -1054,7 +1078,8 @@ def main():
                         higher_is_better=w.kind in ("prefill", "dense_prefill"),
                         n_gpus=args.gpus, steps=args.steps, warmup=args.warmup, dtype=w.dtype, data="synthetic",
                         config=dict(workload=w.name), vs_baseline=None,
-                        cpu_baseline=dict(value=value, unit=unit, cores=threads, kind="oracle", sample=sample),
+                        cpu_baseline=dict(value=value, unit=unit, cores=threads, kind="oracle", sample=sample,
+                                          **ORACLE_EXTRA),
                         e2e=dict(value=value, unit=unit, h2d_bytes_per_step=0, d2h_bytes_per_step=0))
             print(json.dumps(line), flush=True)
         return
@@ -1062,13 +1087,15 @@ def main():
     res = run_ours(args, rank, world)
     if rank == 0 and not args.no_cpu_baseline:
         value, sample, threads, unit = run_oracle_sample(w, budget_s=args.cpu_budget)
-        res["cpu_baseline"] = dict(value=value, unit=unit, cores=threads, kind="oracle", sample=sample)
+        res["cpu_baseline"] = dict(value=value, unit=unit, cores=threads, kind="oracle", sample=sample,
+                                   **ORACLE_EXTRA)
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
     if rank == 0:
         order = ["metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
-                 "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "tensor_roofline", "step_roofline",
+                 "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "tensor_roofline", "bound_aware",
+                 "step_roofline",
                  "e2e",
                  "cpu_baseline", "gpu_launches", "clocks", "stage_ms", "library_context"]
         line = {k: res[k] for k in order if k in res}
