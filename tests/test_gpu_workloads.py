@@ -200,3 +200,69 @@ def _bench_decode_check(qsa, name):
                                   "decode_b64_l128k_d256_fp8"])
 def test_bench_decode_runner_full_size(qsa, name):
     _bench_decode_check(qsa, name)
+
+
+def test_bench_prefill_1m_chunked_runner(qsa):
+    """The benchmark's 1M-token prompt prefilled in 16,000-token chunks by its
+    own runner (chunk offsets, growing compressed cache, score chunks and the
+    CTA-per-row select of long rows) against the oracle on sampled rows: the
+    first and last rows, both sides of chunk boundaries, of 65536 (16384
+    blocks: the select changes kernel) and of 262144 (65536 blocks), and
+    uniform rows."""
+    import bench
+    from qsa_testlib import selection_report
+    w = workloads.WORKLOADS["prefill_l1m_chunk16k"]
+    r = bench.PrefillRunner(w, torch.device(DEV))
+    assert len(r.chunks) == 66
+    r.step()
+    qsa.qsa_check_status()
+    # the runner keeps one chunk's selection: rerun the chunk of each sampled row for it
+    T = w.T
+    g = torch.Generator().manual_seed(5)
+    rows = {0, 1, 15999, 16000, 16001, 65535, 65536, 262139, 262143, 262144, 523999, 524000, T - 2, T - 1}
+    rows |= set(torch.randint(0, T, (10,), generator=g).tolist())
+    rows = sorted(rows)
+    ri = torch.tensor(rows, device=DEV)
+    out = r.out[0, ri].float().cpu().numpy()
+    sel = np.zeros((len(rows), w.top_k), np.int32)
+    nsel = np.zeros(len(rows), np.int32)
+    for c0, c1 in r.chunks:
+        mine = [i for i, t in enumerate(rows) if c0 <= t < c1]
+        if not mine:
+            continue
+        n = c1 - c0
+        s, ns = r.sel[:, :n], r.nsel[:, :n]
+        qsa.qsa_index_topk_prefill(r.x["q_idx"][:, c0:c1], r.k_pool, s, ns, q0=c0, top_k=w.top_k, rope=r.rope,
+                                   workspace=r.ws)
+        for i in mine:
+            sel[i] = s[0, rows[i] - c0].cpu().numpy()
+            nsel[i] = int(ns[0, rows[i] - c0])
+    qsa.qsa_check_status()
+    kp = oracle.pool_keys(np32(r.x["k_idx"][0]), base=w.rope_base, pos_scale=w.pos_scale)
+    assert np.array_equal(np32(r.k_pool[0]), kp)
+    q_idx = np32(r.x["q_idx"][0, ri])
+    q = np32(r.x["q"][0, ri])
+    k, v = np32(r.x["k"][0]), np32(r.x["v"][0])
+    del r
+    _free()
+    ref = {"sel": [], "nsel": [], "kth": [], "out": []}
+    for i, t in enumerate(rows):          # the oracle takes rows relative to q0: one row per call
+        o = oracle.prefill_rows([0], q_idx=q_idx[i:i + 1], k_pool=kp, top_k=w.top_k, base=w.rope_base,
+                                pos_scale=w.pos_scale, q=q[i:i + 1], k=k, v=v, Hq=w.Hq, Hkv=w.Hkv, d=w.d, q0=t)
+        for key in ref:
+            ref[key].append(o[key][0])
+    ref = {key: np.stack(val) for key, val in ref.items()}
+
+    def score_fn(idx_rows):
+        res = []
+        for rr in idx_rows:
+            i = rows.index(rr)
+            sc = oracle.prefill_rows([0], q_idx=q_idx[i:i + 1], k_pool=kp, top_k=w.top_k, base=w.rope_base,
+                                     pos_scale=w.pos_scale, q0=rr, want_scores=True)["scores"][0]
+            res.append(np.pad(sc, (0, kp.shape[0] - sc.shape[0]), constant_values=np.nan))
+        return np.stack(res)
+
+    exact, _, nbad = selection_report(sel, nsel, ref, score_fn, rows)
+    assert nbad <= 2
+    err = np.abs(out - ref["out"])[exact].max()
+    assert err <= TOL["bf16"], err
