@@ -294,7 +294,10 @@ __global__ void __launch_bounds__(SEL_WARPS * 32, 2)
 constexpr int SR_THREADS = 256;
 constexpr int SR_TIE_CAP = 4096;
 constexpr int SR_SPAN = SR_THREADS * 16;   // elements per iteration: four float4 per thread
-constexpr int SR_MIN_BLOCKS = 16384;       // longest row of a launch from which this kernel is used
+#ifndef QSA_SELECT_CTA_MIN_BLOCKS
+#define QSA_SELECT_CTA_MIN_BLOCKS 32768
+#endif
+constexpr int SR_MIN_BLOCKS = QSA_SELECT_CTA_MIN_BLOCKS;   // longest row of a launch from which this kernel is used
 
 struct RowSelSmem {
     uint32_t hist[2048];

@@ -423,13 +423,13 @@ def test_prefill_chunk_beyond_65535_blocks_all_ties(qsa, q0):
 
 @pytest.mark.parametrize("keys", ["groups", "random"])
 def test_prefill_long_rows_select(qsa, keys):
-    """Rows of about 17500 blocks (the CTA-per-row select).  "groups": every
+    """Rows of about 33000 blocks (the CTA-per-row select).  "groups": every
     block's key is one of 64 vectors and the rotation is the identity
     (pos_scale 1e15), so each row's scores take 64 values, each shared
-    exactly by ~270 blocks: the top-512 end inside a group of exact ties
+    exactly by ~515 blocks: the top-512 end inside a group of exact ties
     ranked by block id (bit-exact against the oracle).  "random": the usual
     case under the near-tie acceptance rule."""
-    n_q, q0 = 32, 69984
+    n_q, q0 = 32, 131968
     L = q0 + n_q
     g = torch.Generator(device=DEV).manual_seed(L)
     if keys == "groups":

@@ -206,7 +206,7 @@ def test_bench_prefill_1m_chunked_runner(qsa):
     """The benchmark's 1M-token prompt prefilled in 16,000-token chunks by its
     own runner (chunk offsets, growing compressed cache, score chunks and the
     CTA-per-row select of long rows) against the oracle on sampled rows: the
-    first and last rows, both sides of chunk boundaries, of 65536 (16384
+    first and last rows, both sides of chunk boundaries, of 131072 (32768
     blocks: the select changes kernel) and of 262144 (65536 blocks), and
     uniform rows."""
     import bench
@@ -219,7 +219,8 @@ def test_bench_prefill_1m_chunked_runner(qsa):
     # the runner keeps one chunk's selection: rerun the chunk of each sampled row for it
     T = w.T
     g = torch.Generator().manual_seed(5)
-    rows = {0, 1, 15999, 16000, 16001, 65535, 65536, 262139, 262143, 262144, 523999, 524000, T - 2, T - 1}
+    rows = {0, 1, 15999, 16000, 16001, 65535, 65536, 131071, 131072, 262139, 262143, 262144, 523999, 524000,
+            T - 2, T - 1}
     rows |= set(torch.randint(0, T, (10,), generator=g).tolist())
     rows = sorted(rows)
     ri = torch.tensor(rows, device=DEV)
