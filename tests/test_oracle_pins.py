@@ -324,6 +324,20 @@ def test_qsa_equals_dense_causal_when_every_block_fits(T, k, Hq, Hkv):
     np.testing.assert_allclose(dense, ref[rows], rtol=0, atol=1e-10)
 
 
+def test_dense_rows_with_a_chunk_offset_match_the_full_sequence():
+    # rows of a chunk starting at q0 attend over positions 0 .. q0 + i: they are
+    # rows q0 + i of textbook causal attention over the whole sequence
+    T, q0, Hq, Hkv, d = 300, 203, 8, 2, 128
+    rng = np.random.default_rng(77)
+    q = bf16(rng.standard_normal((T, Hq, d)))
+    kk = bf16(rng.standard_normal((T, Hkv, d)))
+    v = bf16(rng.standard_normal((T, Hkv, d)))
+    ref = _sdpa_causal(q, kk, v, Hq, Hkv)
+    rows = np.arange(T - q0)
+    dense = oracle.dense_rows(rows, q[q0:], kk, v, Hq, Hkv, d, q0=q0)
+    np.testing.assert_allclose(dense, ref[q0:], rtol=0, atol=1e-10)
+
+
 def test_attention_special_cases():
     T, Hq, Hkv, d = 64, 4, 2, 128
     rng = np.random.default_rng(21)
