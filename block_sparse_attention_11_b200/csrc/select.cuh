@@ -348,12 +348,25 @@ __device__ __forceinline__ int warp_topk_row(const float *row, int n, int k, War
         for (int i = lane; i < n; i += 32) emit(i, i);
         return n;
     }
-    // ---- pass 1: top 11 bits
+    // ---- pass 1: top 11 bits (full 512-element steps need no bounds checks)
     wsel_clear(w, 2048);
-    for (int base = 0; base < n; base += 512) {
+    const int n_full = n & ~511;
+    for (int base = 0; base < n_full; base += 512) {
+        float4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) v[u] = *reinterpret_cast<const float4 *>(row + base + 128 * u + 4 * lane);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            wsel_add(w, true, score_key(v[u].x) >> 21);
+            wsel_add(w, true, score_key(v[u].y) >> 21);
+            wsel_add(w, true, score_key(v[u].z) >> 21);
+            wsel_add(w, true, score_key(v[u].w) >> 21);
+        }
+    }
+    if (n_full < n) {
         uint32_t key[4][4];
         bool live[4][4];
-        wsel_load4x4(row, n, base, key, live);
+        wsel_load4x4(row, n, n_full, key, live);
 #pragma unroll
         for (int u = 0; u < 4; ++u)
 #pragma unroll
@@ -363,24 +376,35 @@ __device__ __forceinline__ int warp_topk_row(const float *row, int n, int k, War
     int k_rem = k;
     const uint32_t d1 = (uint32_t)wsel_find(w, 2048, k_rem);
     uint32_t prefix = d1 << 21, pmask = 0xFFE00000u;
-    // ---- pass 2: gather the bin's keys
+    // ---- pass 2: gather the bin's keys (a multiset: order does not matter);
+    // each lane's hits of a step as a 16-bit mask, one warp scan for the slots
     int cnt = 0;
     for (int base = 0; base < n; base += 512) {
         uint32_t key[4][4];
         bool live[4][4];
         wsel_load4x4(row, n, base, key, live);
+        uint32_t hm = 0;
 #pragma unroll
         for (int u = 0; u < 4; ++u)
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const bool hit = live[u][c] && (key[u][c] & pmask) == prefix;
-                const uint32_t bal = __ballot_sync(0xffffffffu, hit);
-                if (hit) {
-                    const int slot = cnt + __popc(bal & lt);
+            for (int c = 0; c < 4; ++c) hm |= (uint32_t)(live[u][c] && (key[u][c] & pmask) == prefix) << (4 * u + c);
+        const int mine = __popc(hm);
+        int incl = mine;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        int slot = cnt + incl - mine;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                if ((hm >> (4 * u + c)) & 1u) {
                     if (slot < kWarpSelBuf) w.buf[slot] = key[u][c];
+                    ++slot;
                 }
-                cnt += __popc(bal);
-            }
+        cnt += __shfl_sync(0xffffffffu, incl, 31);
     }
     __syncwarp();
     const bool small = cnt <= kWarpSelBuf;
