@@ -188,8 +188,14 @@ QSA_API int qsa_pool_keys_decode(const void *k_new, void *ring, void *k_pool, co
  * head_w   device, [B][n_q][4] float, or NULL.
  * sel      device, [B][n_q][top_k] int32.   nsel  device, [B][n_q] int32.
  * workspace device scratch of at least qsa_index_topk_prefill_workspace()
- *          bytes, 256-byte aligned; contents on entry are ignored.
+ *          bytes, 256-byte aligned; contents on entry are ignored.  The
+ *          scores of a group of rows are materialised there in fp32 (groups
+ *          of at most 2 GiB: 2048 rows at a 1M-token context), so the size
+ *          grows with q0 + n_q up to that cap.
  * top_k    1..2048.
+ * Chunked prefill: one call per chunk of rows with q0 = the chunk's first
+ * position, after that chunk's keys were pooled into k_pool; the selections
+ * equal those of one call over all rows (tested to 1,048,576 positions).
  */
 QSA_API size_t qsa_index_topk_prefill_workspace(int32_t B, int64_t n_q, int64_t q0, int32_t top_k,
                                         uint32_t flags, int32_t dtype);
