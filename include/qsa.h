@@ -74,7 +74,7 @@ extern "C" {
  * default: the default score is the plain sum over heads. */
 #define QSA_SCORE_RELU 1u
 /* Normalise the FP32 block mean before rotation (unit-weight RMS norm,
- * eps 1e-6); the same section says the mean is "normalized" without naming
+ * eps 1e-6); the same section calls the mean normalised without naming
  * the norm.  Off by default. */
 #define QSA_POOL_RMSNORM 2u
 /* Compressed keys stored as FP8 E4M3 (1 byte per value, round to nearest

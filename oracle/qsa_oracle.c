@@ -29,8 +29,8 @@
  * notes of the repository):
  *   - score rule: identity by default, ReLU of [SGL]'s equation behind a flag;
  *     optional per-head weights applied outside the nonlinearity;
- *   - "normalized": optional unit-weight RMS normalisation (eps 1e-6) of the
- *     FP32 mean, off by default;
+ *   - key normalisation (named, not defined, by the pages): optional
+ *     unit-weight RMS normalisation (eps 1e-6) of the FP32 mean, off by default;
  *   - RoPE: rotate-half pairs (i, i + R/2), inv_freq_i = base^(-2i/R),
  *     angle = (pos / pos_scale) * inv_freq_i;
  *   - visibility: block b is visible to the query at position t iff
