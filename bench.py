@@ -911,7 +911,7 @@ def library_dense_context(runner, flops, reps=2):
                 run()
             e1.record()
             torch.cuda.synchronize()
-    except Exception as e:   # backend unavailable on this build / device
+    except Exception as e:   # backend unavailable in this torch or on this device
         return dict(library="cuDNN fused attention via torch SDPA", unavailable=repr(e)[:160])
     ms = e0.elapsed_time(e1) / reps
     tail = slice(max(0, T - 2048), T)

@@ -59,7 +59,7 @@ extern "C" {
 /* ---- status codes ---- */
 #define QSA_OK 0
 #define QSA_ERR_INVALID_ARG 1   /* null pointer, bad size, bad stride, bad flag */
-#define QSA_ERR_UNSUPPORTED 2   /* shape/dtype/option this build does not implement, or not an sm_100 device */
+#define QSA_ERR_UNSUPPORTED 2   /* shape/dtype/option the library does not implement, or not an sm_100 device */
 #define QSA_ERR_CUDA 3          /* a CUDA launch or runtime call failed */
 #define QSA_ERR_DEVICE 4        /* a kernel reported a bounds violation or a wait timeout */
 #define QSA_ERR_WORKSPACE 5     /* workspace pointer null or smaller than the size query returned */
