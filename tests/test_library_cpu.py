@@ -128,3 +128,16 @@ def test_binding_rejects_host_tensors(qsa):
     x = torch.zeros(1, 8, 128, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         qsa.qsa_pool_keys_prefill(x, torch.zeros(1, 2, 128, dtype=torch.bfloat16))
+
+
+def test_prefill_index_workspace_grows_with_context_up_to_its_cap(qsa):
+    """The prefill indexer materialises scores of row groups of at most 2 GiB:
+    its workspace grows with the context, stays below the cap plus the rotated
+    queries, and a 16,000-row chunk at a 1M-token context is supported."""
+    ws = qsa.qsa_index_topk_prefill_workspace
+    sizes = [ws(1, 16000, q0, 512) for q0 in (0, 48000, 112000, 496000, 1032576)]
+    assert all(a <= b for a, b in zip(sizes, sizes[1:]))
+    q_bytes = 2 * 16000 * 128 * 2
+    assert sizes[-1] <= (1 << 31) + 4 * q_bytes + (1 << 20)
+    assert sizes[-1] >= 2048 * 262144 * 4                      # at least one 2048-row group of 1M-context scores
+    assert ws(0, 16000, 0, 512) == 0 and ws(1, 16000, -1, 512) == 0     # invalid shapes: 0
