@@ -38,6 +38,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libqsa.so")
 QSA_OK, QSA_ERR_INVALID_ARG, QSA_ERR_UNSUPPORTED, QSA_ERR_CUDA, QSA_ERR_DEVICE, QSA_ERR_WORKSPACE = range(6)
 QSA_BF16, QSA_FP32 = 0, 1
 QSA_SCORE_RELU, QSA_POOL_RMSNORM, QSA_KEYS_FP8 = 1, 2, 4
+QSA_NOALLOC_SCRATCH_BYTES = 4 << 20   # as in include/qsa.h
 
 
 class QSAError(RuntimeError):

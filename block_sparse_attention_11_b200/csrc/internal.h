@@ -54,10 +54,21 @@ struct DeviceInfo {
     int major = 0, minor = 0;
     size_t smem_optin = 0;
     unsigned *status = nullptr;   // device address of the library status word
+    void *noalloc_scratch = nullptr;   // device address of the allocation-free decode scratch
 };
 
 // Per-device info of the current device (cached).  Returns nullptr on error.
 const DeviceInfo *device_info();
+
+// Device address of the allocation-free decode scratch on the current device
+// (qsa_noalloc.cu); device_info() looks it up once per device.
+cudaError_t noalloc_scratch_address(void **out);
+
+// Argument checks shared by the sparse attention entry points (qsa_api.cu):
+// null pointers, top_k, head shapes, scale, dtype and 16-byte alignment.
+int attn_common_checks(const void *q, const void *k, const void *v, const int32_t *sel, const int32_t *nsel,
+                       int32_t B, int32_t Hq, int32_t Hkv, int32_t d, int32_t top_k, float scale, const void *out,
+                       int32_t dtype);
 
 // ---- pooling / rotation (k_rope.cu)
 // fp8: the compressed keys are stored as FP8 E4M3 (bf16 raw keys only).

@@ -38,6 +38,7 @@ const DeviceInfo *device_info() {
         void *addr = nullptr;
         if (cudaGetSymbolAddress(&addr, g_status) != cudaSuccess) return nullptr;
         d.status = static_cast<unsigned *>(addr);
+        if (noalloc_scratch_address(&d.noalloc_scratch) != cudaSuccess || !d.noalloc_scratch) return nullptr;
         g_info[dev] = d;
         g_info_ok[dev] = true;
     }
@@ -109,6 +110,26 @@ PrefillPlan prefill_plan(int B, int64_t n_q, int64_t q0, uint32_t flags, int dty
 }
 
 }  // namespace
+
+namespace qsa {
+int attn_common_checks(const void *q, const void *k, const void *v, const int32_t *sel, const int32_t *nsel,
+                       int32_t B, int32_t Hq, int32_t Hkv, int32_t d, int32_t top_k, float scale, const void *out,
+                       int32_t dtype) {
+    if (!q || !k || !v || !sel || !nsel || !out || B < 1) return QSA_ERR_INVALID_ARG;
+    if (top_k < 1 || top_k > 2048) return QSA_ERR_INVALID_ARG;
+    if (Hq < 1 || Hkv < 1 || (Hq % Hkv) != 0) return QSA_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !std::isfinite(scale)) return QSA_ERR_INVALID_ARG;
+    if (dtype != QSA_BF16 && dtype != QSA_FP32) return QSA_ERR_UNSUPPORTED;
+    // shapes: d = 128 with 8 q heads per kv head (1, 2 or 4 kv heads; fp32: any GQA),
+    // and the released 24q / 2kv, d = 256 shape (bf16)
+    const bool released = dtype == QSA_BF16 && d == 256 && Hkv == 2 && Hq == 24;
+    if (d != 128 && !released) return QSA_ERR_UNSUPPORTED;
+    if (dtype == QSA_BF16 && !released && (Hq != 8 * Hkv || (Hkv != 1 && Hkv != 2 && Hkv != 4)))
+        return QSA_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return QSA_ERR_INVALID_ARG;
+    return QSA_OK;
+}
+}  // namespace qsa
 
 extern "C" {
 
@@ -278,25 +299,6 @@ int qsa_index_topk_decode(const void *q_idx, const void *k_pool, const float *he
     return cuda_status(e);
 }
 
-namespace {
-int attn_common_checks(const void *q, const void *k, const void *v, const int32_t *sel, const int32_t *nsel,
-                       int32_t B, int32_t Hq, int32_t Hkv, int32_t d, int32_t top_k, float scale, const void *out,
-                       int32_t dtype) {
-    if (!q || !k || !v || !sel || !nsel || !out || B < 1) return QSA_ERR_INVALID_ARG;
-    if (top_k < 1 || top_k > 2048) return QSA_ERR_INVALID_ARG;
-    if (Hq < 1 || Hkv < 1 || (Hq % Hkv) != 0) return QSA_ERR_INVALID_ARG;
-    if (!(scale > 0.f) || !std::isfinite(scale)) return QSA_ERR_INVALID_ARG;
-    if (dtype != QSA_BF16 && dtype != QSA_FP32) return QSA_ERR_UNSUPPORTED;
-    // shapes: d = 128 with 8 q heads per kv head (1, 2 or 4 kv heads; fp32: any GQA),
-    // and the released 24q / 2kv, d = 256 shape (bf16)
-    const bool released = dtype == QSA_BF16 && d == 256 && Hkv == 2 && Hq == 24;
-    if (d != 128 && !released) return QSA_ERR_UNSUPPORTED;
-    if (dtype == QSA_BF16 && !released && (Hq != 8 * Hkv || (Hkv != 1 && Hkv != 2 && Hkv != 4)))
-        return QSA_ERR_UNSUPPORTED;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return QSA_ERR_INVALID_ARG;
-    return QSA_OK;
-}
-}  // namespace
 
 int qsa_sparse_attn_prefill(const void *q, const void *k, const void *v, const int32_t *sel, const int32_t *nsel,
                             int32_t B, int64_t n_q, int64_t q0, int64_t kv_stride, int32_t Hq, int32_t Hkv, int32_t d,

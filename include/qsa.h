@@ -356,9 +356,13 @@ QSA_API int qsa_dense_attn_decode(const void *q, const void *k, const void *v, c
  * into the library, QSA_NOALLOC_SCRATCH_BYTES of device memory on every GPU
  * that loads the library, held until the process exits.  Calls needing more
  * (roughly B * splits * Hq * 516 bytes, splits ~ 2 * SMs / B) return
- * QSA_ERR_WORKSPACE.  Allocates nothing.  The first call on a device looks up
- * the scratch's device address (cudaGetSymbolAddress) with that device
- * current; make that first call before any stream capture.  Every call on a
+ * QSA_ERR_WORKSPACE (for example B = 64 with Hq = 32: 4,227,072 bytes).
+ * Allocates nothing.  The scratch's device address is looked up
+ * (cudaGetSymbolAddress) by the first call of any entry point of this library
+ * on a device, with that device current, and cached; make that first call (for
+ * example qsa_check_status) before any stream capture, since a lookup inside
+ * a capture can fail with QSA_ERR_CUDA depending on the capture mode.  The
+ * fp32 path keeps no partial results and uses no scratch.  Every call on a
  * device shares the one scratch area: calls whose work can overlap on the GPU
  * (different streams without ordering) race and must be serialised by the
  * caller.  Nothing needs clearing between calls.

@@ -141,3 +141,9 @@ def test_prefill_index_workspace_grows_with_context_up_to_its_cap(qsa):
     assert sizes[-1] <= (1 << 31) + 4 * q_bytes + (1 << 20)
     assert sizes[-1] >= 2048 * 262144 * 4                      # at least one 2048-row group of 1M-context scores
     assert ws(0, 16000, 0, 512) == 0 and ws(1, 16000, -1, 512) == 0     # invalid shapes: 0
+
+
+def test_binding_constants_match_the_header(qsa):
+    src = open(HEADER).read()
+    m = re.search(r"#define QSA_NOALLOC_SCRATCH_BYTES \((\d+)u << (\d+)\)", src)
+    assert m and qsa.QSA_NOALLOC_SCRATCH_BYTES == int(m.group(1)) << int(m.group(2))
