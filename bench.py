@@ -7,9 +7,12 @@ A step is one pass of the whole hot path over one batch of synthetic input:
     scores, per-row top-k) + sparse attention over the selected K/V;
   decode workloads: ring pooling + decode indexer (scan + select) + split-KV
     sparse attention + combine.
-The default workload is the 32K-token prefill with planted needles (B=1,
-T=32768, top-512, 16 q / 2 kv heads, bf16).  One JSON line is printed by
-rank 0.  With N > 1 (torchrun) every rank runs its own replica of the
+The default run is the metric's own configurations: the line's workload is
+the 128K-token prefill with heavy-tailed keys (B=1, T=131072, top-512, 16 q /
+2 kv heads, bf16), and the same run measures the two decode workloads (8
+sequences of 1M cached tokens, 64 sequences of 128K) and reports their
+us/step under "decode".  --workload NAME measures one workload alone.  One
+JSON line is printed by rank 0.  With N > 1 (torchrun) every rank runs its own replica of the
 workload (QSA has no exchange step: replicas only), the timed region is
 bracketed by barriers and the max over ranks is reported; value is the whole
 job's throughput.
@@ -37,6 +40,9 @@ import torch  # noqa: E402
 import workloads  # noqa: E402
 
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+# the metric's configurations: 128K-token prefill (the line), and the 1M and 128K decode steps
+DEFAULT_WORKLOAD = "prefill_t128k_heavytail"
+DEFAULT_DECODE = ("decode_b8_l1m_scale4", "decode_b64_l128k")
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_BYTES = 126 * 1024 * 1024
 
@@ -84,6 +90,29 @@ def profiled_traffic(kind, workload):
         except (KeyError, ValueError, OSError):
             return None
     return None
+
+
+def measure_l2_read(dev, reps=40):
+    """L2 read bandwidth (GB/s) measured here with CUDA events: a float32
+    buffer far smaller than L2 (48 MiB of the 126 MB) is read repeatedly by a
+    sum reduction after one warm-up pass, so every read after the first is
+    served by L2; the best of three sizes' rates is reported."""
+    best = 0.0
+    for mib in (24, 48, 64):
+        x = torch.ones(mib * (1 << 20) // 4, dtype=torch.float32, device=dev)
+        acc = torch.empty((), dtype=torch.float32, device=dev)
+        for _ in range(3):
+            torch.sum(x, out=acc)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            torch.sum(x, out=acc)
+        e1.record()
+        torch.cuda.synchronize()
+        best = max(best, x.numel() * 4 * reps / (e0.elapsed_time(e1) / 1e3) / 1e9)
+        del x
+    return best
 
 
 def peaks():
@@ -370,6 +399,15 @@ class DecodeRunner:
                                       workspace=self.ws_i)
         if events is not None:
             events[2].record()
+        self.attend(x)
+        if events is not None:
+            events[3].record()
+        return self.out
+
+    def attend(self, x=None):
+        """The step's attention call alone, on the current self.sel / self.nsel."""
+        qsa = self.qsa
+        x = x or self.x
         if self.pt:
             qsa.qsa_sparse_attn_decode_paged(x["q"], x["k"], x["v"], self.table, self.pt, x["seq_len"], self.sel,
                                              self.nsel, self.out, workspace=self.ws_a)
@@ -379,8 +417,6 @@ class DecodeRunner:
         else:
             qsa.qsa_sparse_attn_decode(x["q"], x["k"], x["v"], x["seq_len"], self.sel, self.nsel, self.out,
                                        workspace=self.ws_a)
-        if events is not None:
-            events[3].record()
         return self.out
 
     def launches_per_step(self):
@@ -791,13 +827,23 @@ def run_ours(args, rank, world):
                           d2h_bytes_per_step=d2h, mode=e2e_mode,
                           serial_value=job_throughput(runner.units(), world, e2e_serial_ms))
         attn_ms = stage_avg["sparse_attn"]
-        achieved = alg["attn_bytes"] / (attn_ms / 1e3) / 1e9
-        res["roofline"] = dict(kernel="sparse_attn_prefill", bound="hbm", achieved=achieved, peak=pk["hbm_gbs"],
-                               unit="GB/s", frac=achieved / pk["hbm_gbs"],
-                               traffic=profiled_traffic("prefill", w.name), peak_kind=pk_kind,
-                               note="algorithmic bytes = K/V rows gathered per query (4*nsel+tail positions x "
-                                    "Hkv x d x 2 B x 2) + q read + out write; the unique K/V fits in L2, so "
-                                    "gathers are served from L2 and frac can exceed 1")
+        attn_tf = alg["attn_flops"] / (attn_ms / 1e3) / 1e12
+        peak_tf = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+        res["roofline"] = dict(kernel="sparse_attn_prefill", bound="tensor", achieved=attn_tf, peak=peak_tf,
+                               unit="TFLOP/s", frac=attn_tf / peak_tf,
+                               traffic=profiled_traffic("prefill", w.name), peak_kind=pk_kind + " (sustained bf16)",
+                               note="algorithmic flops = 4*d*Hq per selected position (4*nsel + tail per query) "
+                                    "over the attention stage's CUDA-event time; the bf16 sustained peak (a step "
+                                    "of tens of ms)")
+        l2 = measure_l2_read(torch.device("cuda", torch.cuda.current_device()))
+        gb = alg["attn_bytes"] / (attn_ms / 1e3) / 1e9
+        res["l2_roofline"] = dict(kernel="sparse_attn_prefill", achieved=gb, peak=l2, unit="GB/s", frac=gb / l2,
+                                  peak_kind="L2 read rate measured in this run (sum over a 24-64 MiB L2-resident "
+                                            "buffer, CUDA events)",
+                                  note="algorithmic bytes = the K/V rows each query attends to (4*nsel+tail "
+                                       "positions x Hkv x d x 2 B x 2) + q read + out write, as if every query "
+                                       "gathered its own; a kernel that shares a gathered block between the "
+                                       "queries selecting it moves fewer bytes than this")
         flops = alg["attn_flops"] + alg["idx_flops"]
         tf = flops / (ms_per_step / 1e3) / 1e12
         res["tensor_roofline"] = dict(achieved=tf, peak=pk["bf16_tflops"], unit="TFLOP/s",
@@ -1046,7 +1092,9 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="prefill_t32k_needles", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--workload", default=None, choices=sorted(workloads.WORKLOADS),
+                    help="one workload alone (default: the 128K prefill line with both decode workloads)")
+    ap.add_argument("--no-decode", action="store_true", help="default run: skip the two decode workloads")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -1056,6 +1104,9 @@ def main():
     ap.add_argument("--tokens", type=int, default=None, help="override T / cache length (smaller profiling case)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    with_decode = args.workload is None and not args.no_decode
+    if args.workload is None:
+        args.workload = DEFAULT_WORKLOAD
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -1089,15 +1140,31 @@ def main():
         value, sample, threads, unit = run_oracle_sample(w, budget_s=args.cpu_budget)
         res["cpu_baseline"] = dict(value=value, unit=unit, cores=threads, kind="oracle", sample=sample,
                                    **ORACLE_EXTRA)
+    if with_decode:
+        # the metric's decode half, in the same run: each decode workload timed as its own step
+        res["decode"] = {}
+        for name in DEFAULT_DECODE:
+            torch.cuda.empty_cache()
+            sub_args = argparse.Namespace(**vars(args))
+            sub_args.workload = name
+            sub = run_ours(sub_args, rank, world)
+            if rank == 0 and not args.no_cpu_baseline:
+                ORACLE_EXTRA.clear()
+                value, sample, threads, unit = run_oracle_sample(workloads.WORKLOADS[name],
+                                                                 budget_s=min(args.cpu_budget, 6.0))
+                sub["cpu_baseline"] = dict(value=value, unit=unit, cores=threads, kind="oracle", sample=sample)
+            keep = ["metric", "value", "unit", "ms_per_step", "higher_is_better", "config", "roofline",
+                    "step_roofline", "e2e", "cpu_baseline", "gpu_launches", "clocks", "stage_ms"]
+            res["decode"][name] = {k: sub[k] for k in keep if k in sub}
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
     if rank == 0:
         order = ["metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
-                 "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "tensor_roofline", "bound_aware",
-                 "step_roofline",
+                 "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "l2_roofline", "tensor_roofline",
+                 "bound_aware", "step_roofline",
                  "e2e",
-                 "cpu_baseline", "gpu_launches", "clocks", "stage_ms", "library_context"]
+                 "cpu_baseline", "gpu_launches", "clocks", "stage_ms", "library_context", "decode"]
         line = {k: res[k] for k in order if k in res}
         print(json.dumps(line), flush=True)
 

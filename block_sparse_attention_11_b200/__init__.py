@@ -29,7 +29,7 @@ __all__ = [
     "qsa_dense_attn_decode", "qsa_dense_attn_decode_workspace", "qsa_dense_attn_prefill",
     "qsa_pool_keys_prefill_paged", "qsa_pool_keys_decode_paged", "qsa_index_topk_decode_paged",
     "qsa_sparse_attn_decode_paged", "qsa_sparse_attn_prefill_kv8", "qsa_sparse_attn_decode_kv8",
-    "qsa_rope_apply", "qsa_check_status", "qsa_strerror", "qsa_version",
+    "qsa_rope_apply", "qsa_check_status", "qsa_selftest_wait_timeout", "qsa_strerror", "qsa_version",
     "QSA_SCORE_RELU", "QSA_POOL_RMSNORM", "QSA_KEYS_FP8", "QSA_BF16", "QSA_FP32",
 ]
 
@@ -89,6 +89,7 @@ def _sig(name, res, *args):
 _sig("qsa_strerror", ctypes.c_char_p, ctypes.c_int)
 _sig("qsa_version", ctypes.c_int)
 _sig("qsa_check_status", ctypes.c_int, _vp, ctypes.POINTER(_u32))
+_sig("qsa_selftest_wait_timeout", ctypes.c_int, ctypes.c_uint64, _vp, _vp)
 _sig("qsa_pool_keys_prefill", ctypes.c_int, _vp, _vp, _i32, _i64, _i64, _i64, _i64, _Rope, _u32, _i32, _vp)
 _sig("qsa_pool_keys_decode", ctypes.c_int, _vp, _vp, _vp, _vp, _i32, _i64, _Rope, _u32, _i32, _vp)
 _sig("qsa_index_topk_prefill_workspace", _sz, _i32, _i64, _i64, _i32, _u32, _i32)
@@ -482,6 +483,14 @@ def qsa_rope_apply(x, pos0=0, rope=Rope(), stream=None):
     B, n, H, d = x.shape
     st = lib.qsa_rope_apply(_ptr(x, None, "x"), B, n, H, d, pos0, rope.c(), dt, _stream(x, stream))
     _check(st, "qsa_rope_apply")
+
+
+def qsa_selftest_wait_timeout(limit_ns, result, stream=None):
+    """Run the bounded-wait self-test: one CTA waits on an mbarrier nothing
+    arrives on, gives up after limit_ns, frees its TMEM and returns; result
+    (a 1-element int32 device tensor) receives 0 when the wait gave up."""
+    _check(lib.qsa_selftest_wait_timeout(int(limit_ns), _ptr(result, torch.int32, "result"), _stream(result, stream)),
+           "qsa_selftest_wait_timeout")
 
 
 def qsa_check_status(stream=None, device=None):

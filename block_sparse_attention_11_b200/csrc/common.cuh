@@ -217,15 +217,17 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 
 // Bounded wait for the phase with the given parity to complete: polls, and
 // after the first 4096 polls checks the global timer every 256 polls; gives
-// up after kWaitNs, flags QSA_DEV_TIMEOUT and returns false.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsigned *status) {
+// up after limit_ns (kWaitNs unless a self-test passes a shorter limit),
+// flags QSA_DEV_TIMEOUT and returns false.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsigned *status,
+                                          uint64_t limit_ns = kWaitNs) {
     for (int i = 0; i < 4096; ++i)
         if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (;;) {
         for (int i = 0; i < 256; ++i)
             if (mbar_try_wait(bar, parity)) return true;
-        if (globaltimer_ns() - t0 > kWaitNs) break;
+        if (globaltimer_ns() - t0 > limit_ns) break;
     }
     flag(status, QSA_DEV_TIMEOUT);
     return false;

@@ -70,6 +70,11 @@ int attn_common_checks(const void *q, const void *k, const void *v, const int32_
                        int32_t B, int32_t Hq, int32_t Hkv, int32_t d, int32_t top_k, float scale, const void *out,
                        int32_t dtype);
 
+// ---- self-test of the bounded waits (k_selftest.cu): one CTA waits on an
+// mbarrier nothing arrives on, with the given limit; writes 0 to *result when
+// the wait gave up (and QSA_DEV_TIMEOUT to the status word), 1 otherwise.
+cudaError_t launch_wait_timeout_selftest(uint64_t limit_ns, unsigned *status, unsigned *result, cudaStream_t s);
+
 // ---- pooling / rotation (k_rope.cu)
 // fp8: the compressed keys are stored as FP8 E4M3 (bf16 raw keys only).
 // pg.table != nullptr: the compressed-key cache is paged (pool_stride unused).

@@ -161,6 +161,15 @@ int qsa_check_status(void *stream, uint32_t *detail) {
     return v ? QSA_ERR_DEVICE : QSA_OK;
 }
 
+int qsa_selftest_wait_timeout(uint64_t limit_ns, uint32_t *result, void *stream) {
+    if (!result || limit_ns < 1 || limit_ns > kWaitNs) return QSA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(result) & 3u) != 0) return QSA_ERR_INVALID_ARG;
+    const DeviceInfo *di = nullptr;
+    int st = check_device(&di);
+    if (st != QSA_OK) return st;
+    return cuda_status(launch_wait_timeout_selftest(limit_ns, di->status, result, static_cast<cudaStream_t>(stream)));
+}
+
 int qsa_pool_keys_prefill(const void *k_raw, void *k_pool, int32_t B, int64_t n_tok, int64_t pos0,
                           int64_t raw_stride, int64_t pool_stride, qsa_rope_t rope, uint32_t flags, int32_t dtype,
                           void *stream) {

@@ -114,6 +114,20 @@ QSA_API int qsa_version(void);
  * workspace that was not zero-filled before its first use. */
 QSA_API int qsa_check_status(void *stream, uint32_t *detail);
 
+/*
+ * Self-test of the bounded waits (not a step of the method; the pages have no
+ * counterpart).  Every pipeline of the library waits on mbarriers through one
+ * bounded wait that gives up after 2 s, records QSA_DEV_TIMEOUT (status bit 4)
+ * and lets the kernel release its tensor memory and return, so a broken
+ * pipeline ends its kernel instead of hanging the GPU.  This call runs that
+ * wait on purpose: one CTA takes TMEM columns, waits on an mbarrier that
+ * nothing arrives on with a limit of limit_ns (1 .. 2e9 ns), gives up, frees
+ * the TMEM and returns.  It writes 0 to *result (device, 4-byte aligned) when
+ * the wait gave up (1 would mean it completed), and qsa_check_status then
+ * reports QSA_ERR_DEVICE with detail bit 4.  No fault, no hang.
+ */
+QSA_API int qsa_selftest_wait_timeout(uint64_t limit_ns, uint32_t *result, void *stream);
+
 /* ========================================================================= */
 /* a1. Compressed-key pooling, prefill                                        */
 /* ========================================================================= */

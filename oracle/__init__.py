@@ -203,7 +203,7 @@ def dense_rows(rows, q, k, v, Hq, Hkv, d, scale=None, q0=0, nthreads=None):
 
 def decode(q_idx, k_pool, seq_len, *, head_w=None, q=None, k=None, v=None, relu=False,
            store_bf16=True, top_k=512, Hq=16, Hkv=2, d=128, scale=None, base=10000.0,
-           pos_scale=1.0, rotary_dim=128, nthreads=None, cap_len=None):
+           pos_scale=1.0, rotary_dim=128, nthreads=None, cap_len=None, want_scores=False):
     """One decode step for B sequences (after pooling).
 
     q_idx [B][4][128]; k_pool [B][stride][128]; seq_len [B]; q [B][Hq][d];
@@ -211,6 +211,8 @@ def decode(q_idx, k_pool, seq_len, *, head_w=None, q=None, k=None, v=None, relu=
     cap_len [B] (IndexShare draft step): the selection is that of row
     cap_len - 1 (q_idx is that row's indexer query); the attention at row
     seq_len - 1 reads those blocks plus positions 4*floor(cap_len/4) .. seq_len - 1.
+    want_scores: also return scores [B][cap], the block scores the selection
+    ranked (NaN past each sequence's visible blocks).
     """
     q_idx_a = _f32(q_idx)
     k_pool_a = _f32(k_pool)
@@ -231,14 +233,21 @@ def decode(q_idx, k_pool, seq_len, *, head_w=None, q=None, k=None, v=None, relu=
     nxt = np.full(B, np.nan)
     out = np.zeros((B, Hq, d)) if q is not None else None
     lse = np.zeros((B, Hq)) if q is not None else None
+    scores, score_cap = None, 0
+    if want_scores:
+        rows_sel = cap if cap is not None else seq
+        score_cap = max(1, int(max(int(x) for x in rows_sel)) // BLOCK) if B else 1
+        scores = np.full((B, score_cap), np.nan)
     _L().oracle_decode(_p(q_idx_a), _p(k_pool_a), ctypes.c_int64(pool_stride), _p(head_w_a),
                        _p(q_a), _p(k_a), _p(v_a), ctypes.c_int64(kv_stride), _p(seq), _p(cap),
                        ctypes.c_int64(B), ctypes.c_int(int(relu)), ctypes.c_int(int(store_bf16)),
                        ctypes.c_int(top_k), ctypes.c_int(Hq), ctypes.c_int(Hkv), ctypes.c_int(d),
                        ctypes.c_double(scale), ctypes.c_double(base), ctypes.c_double(pos_scale),
                        ctypes.c_int(rotary_dim), _p(sel), _p(nsel), _p(kth), _p(nxt), _p(out),
-                       _p(lse), ctypes.c_int(nthreads or nthreads_default()))
+                       _p(lse), _p(scores), ctypes.c_int64(score_cap), ctypes.c_int(nthreads or nthreads_default()))
     res = dict(sel=sel, nsel=nsel, kth=kth, next=nxt)
+    if want_scores:
+        res["scores"] = scores
     if q is not None:
         res.update(out=out, lse=lse)
     return res

@@ -545,6 +545,8 @@ typedef struct {
     orope_t rope;
     int32_t *sel, *nsel;
     double *kth, *next, *out, *lse;
+    double *scores;          /* [B][score_cap] or NULL: the block scores, as ranked */
+    int64_t score_cap;
     int64_t B;
     int nthreads, tid;
 } djob_t;
@@ -561,6 +563,8 @@ static void decode_one(const djob_t *J, int64_t bi)
     double *s = (double *)malloc(sizeof(double) * (size_t)(nb > 0 ? nb : 1));
     index_scores(q_hat, J->k_pool + bi * J->pool_stride * IDX_DIM, nb,
                  J->head_w ? J->head_w + bi * IDX_HEADS : NULL, J->relu, s);
+    if (J->scores)
+        for (int64_t b = 0; b < nb && b < J->score_cap; ++b) J->scores[bi * J->score_cap + b] = s[b];
     int32_t *sel = J->sel + bi * J->top_k;
     double kth, nxt;
     int nsel = oracle_topk(s, nb, J->top_k, sel, &kth, &nxt);
@@ -595,7 +599,7 @@ void oracle_decode(const float *q_idx, const float *k_pool, int64_t pool_stride,
                    const int32_t *seq_len, const int32_t *cap_len, int64_t B, int relu, int store_bf16, int top_k,
                    int Hq, int Hkv, int d, double scale, double base, double pos_scale, int rotary_dim,
                    int32_t *sel, int32_t *nsel, double *kth, double *next,
-                   double *out, double *lse, int nthreads)
+                   double *out, double *lse, double *scores, int64_t score_cap, int nthreads)
 {
     djob_t J;
     memset(&J, 0, sizeof J);
@@ -604,6 +608,7 @@ void oracle_decode(const float *q_idx, const float *k_pool, int64_t pool_stride,
     J.relu = relu; J.store_bf16 = store_bf16; J.top_k = top_k; J.Hq = Hq; J.Hkv = Hkv; J.d = d;
     J.scale = scale; J.rope.base = base; J.rope.pos_scale = pos_scale; J.rope.rotary_dim = rotary_dim;
     J.sel = sel; J.nsel = nsel; J.kth = kth; J.next = next; J.out = out; J.lse = lse; J.B = B;
+    J.scores = scores; J.score_cap = score_cap;
     int nt = nthreads < 1 ? 1 : (nthreads > 256 ? 256 : nthreads);
     pthread_t th[256];
     djob_t jobs[256];

@@ -128,3 +128,53 @@ def check_prefill_workload(x, w, rows, top_k=None, flags=0, head_w=None, b=0, ch
         lerr = float(np.abs(gl - ref["lse"][exact]).max()) if gl.size else 0.0
         assert lerr <= (1e-3 if w.dtype == "bf16" else 1e-4), f"lse error {lerr}"
     return dict(exact=exact, overlap=overlap, nbad=nbad, err=err, g=g, ref=ref)
+
+
+def decode_selection_matches(g_sel, g_nsel, ref, i=0):
+    """Compare one decode sequence's GPU selection with the oracle's (ref from
+    oracle.decode(..., want_scores=True), sequence i of it).
+
+    Returns True when the selections are equal.  Otherwise asserts the
+    acceptance rule -- every block in the symmetric difference scores within
+    GAP_REL of the oracle's k-th score, ids ascending, padding -1 -- and
+    returns False (the caller then checks the attention on the oracle's
+    selection instead)."""
+    ns = int(ref["nsel"][i])
+    assert int(g_nsel) == ns, f"selection count {int(g_nsel)} != oracle {ns}"
+    o_sel = ref["sel"][i]
+    if np.array_equal(g_sel, o_sel):
+        return True
+    scores = ref["scores"][i]
+    kth = ref["kth"][i]
+    tol = GAP_REL * max(abs(kth), 1e-30)
+    a, o = set(g_sel[:ns].tolist()), set(o_sel[:ns].tolist())
+    for blk in a ^ o:
+        assert 0 <= blk < scores.shape[0] and np.isfinite(scores[blk]), f"block {blk} out of range"
+        assert abs(scores[blk] - kth) <= tol, (
+            f"block {blk} (score {scores[blk]}) differs from the oracle selection but is not within "
+            f"{GAP_REL} of the k-th score {kth}")
+    assert np.all(np.diff(g_sel[:ns]) > 0), "selection not strictly ascending"
+    assert np.all(g_sel[ns:] == -1), "padding is not -1"
+    return False
+
+
+def stage_isolated_decode(refs, attn_fn, B, top_k, tol, lse_tol=None):
+    """For the decode sequences whose selection differed (refs: {b: oracle
+    result of that sequence}), run the GPU attention of the whole batch on
+    the oracle's selections (attn_fn(sel, nsel) -> (out, lse or None), device
+    tensors) and compare those sequences with the oracle's attention."""
+    if not refs:
+        return
+    dev = "cuda"
+    sel = torch.full((B, top_k), -1, dtype=torch.int32)
+    nsel = torch.zeros(B, dtype=torch.int32)
+    for b, r in refs.items():
+        sel[b] = torch.from_numpy(r["sel"][0])
+        nsel[b] = int(r["nsel"][0])
+    out, lse = attn_fn(sel.to(dev), nsel.to(dev))
+    qsa.qsa_check_status()
+    for b, r in refs.items():
+        err = float(np.abs(np32(out[b]) - r["out"][0]).max())
+        assert err <= tol, f"seq {b}: attention on the oracle's selection, error {err}"
+        if lse is not None and lse_tol is not None:
+            assert float(np.abs(lse[b].cpu().numpy() - r["lse"][0]).max()) <= lse_tol

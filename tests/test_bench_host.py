@@ -37,3 +37,12 @@ def test_oracle_sample_reports_one_thread_rate():
     assert bench.ORACLE_EXTRA["value_1thread"] > 0
     # all cores are not slower than one (within timing noise on a loaded host)
     assert value >= 0.5 * bench.ORACLE_EXTRA["value_1thread"]
+
+
+def test_default_run_is_the_metrics_configurations():
+    """The metric is quoted at 128K-1M context: the default line is the 128K
+    prefill, and the same run measures the 1M and 128K decode steps."""
+    w = workloads.WORKLOADS[bench.DEFAULT_WORKLOAD]
+    assert w.kind == "prefill" and w.T == 131072 and w.heavy_tail
+    dec = [workloads.WORKLOADS[n] for n in bench.DEFAULT_DECODE]
+    assert [(d.kind, d.B, d.T) for d in dec] == [("decode", 8, 1 << 20), ("decode", 64, 131072)]

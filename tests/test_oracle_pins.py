@@ -383,9 +383,12 @@ def test_decode_step_equals_prefill_row():
         for s in range(t + 1):
             oracle.pool_decode(k_raw[s], ring, kp, s + 1)
         dec = oracle.decode(q_idx[t][None], kp[None], [t + 1], q=q[t][None], k=kk[None], v=v[None],
-                            top_k=k, Hq=Hq, Hkv=Hkv, d=d)
+                            top_k=k, Hq=Hq, Hkv=Hkv, d=d, want_scores=True)
         pre = oracle.prefill_rows([t], q_idx=q_idx, k_pool=kbar, top_k=k, q=q, k=kk, v=v,
-                                  Hq=Hq, Hkv=Hkv, d=d)
+                                  Hq=Hq, Hkv=Hkv, d=d, want_scores=True)
+        nb = (t + 1) // 4
+        if nb:   # the scores the decode selection ranked are the prefill row's
+            np.testing.assert_array_equal(dec["scores"][0][:nb], pre["scores"][0][:nb])
         assert dec["nsel"][0] == pre["nsel"][0]
         np.testing.assert_array_equal(dec["sel"][0], pre["sel"][0])
         np.testing.assert_array_equal(dec["out"][0], pre["out"][0])
