@@ -208,9 +208,14 @@ class PrefillRunner:
         self.sel = torch.empty(B, rows, w.top_k, dtype=torch.int32, device=dev)
         self.nsel = torch.empty(B, rows, dtype=torch.int32, device=dev)
         self.out = torch.empty_like(self.x["q"])
-        ws = max(qsa.qsa_index_topk_prefill_workspace(B, c1 - c0, c0, w.top_k, 0, 0 if w.dtype == "bf16" else 1)
+        self.dt_code = 0 if w.dtype == "bf16" else 1
+        ws = max(qsa.qsa_index_topk_prefill_workspace(B, c1 - c0, c0, w.top_k, 0, self.dt_code)
                  for c0, c1 in self.chunks)
         self.ws = torch.empty(ws, dtype=torch.uint8, device=dev)
+        # the attention's workspace (block lists of its 16-query tiles), allocated once
+        wa = 0 if self.kv8 else max(qsa.qsa_sparse_attn_prefill_workspace(B, c1 - c0, w.top_k, w.Hq, w.Hkv, w.d,
+                                                                          self.dt_code) for c0, c1 in self.chunks)
+        self.ws_a = torch.empty(max(wa, 1), dtype=torch.uint8, device=dev)
         # the step's inputs (~200 MB at T=32K) do not all stay in L2, but the
         # flush keeps every timed step cold
         self.flush_between_steps = True
@@ -235,7 +240,7 @@ class PrefillRunner:
             qsa.qsa_sparse_attn_prefill_kv8(x["q"], x["k"], x["v"], self.k_scale, self.v_scale, self.sel, self.nsel,
                                             self.out)
         else:
-            qsa.qsa_sparse_attn_prefill(x["q"], x["k"], x["v"], self.sel, self.nsel, self.out)
+            qsa.qsa_sparse_attn_prefill(x["q"], x["k"], x["v"], self.sel, self.nsel, self.out, workspace=self.ws_a)
         if events is not None:
             events[3].record()
         return self.out
@@ -261,7 +266,8 @@ class PrefillRunner:
                                        rope=self.rope, workspace=self.ws)
             if ev:
                 ev[2].record()
-            qsa.qsa_sparse_attn_prefill(x["q"][:, c0:c1], x["k"], x["v"], sel, nsel, self.out[:, c0:c1], q0=c0)
+            qsa.qsa_sparse_attn_prefill(x["q"][:, c0:c1], x["k"], x["v"], sel, nsel, self.out[:, c0:c1], q0=c0,
+                                        workspace=self.ws_a)
             if ev:
                 ev[3].record()
                 events.extend(ev)
@@ -282,7 +288,15 @@ class PrefillRunner:
         return t
 
     def launches_per_step(self):
-        return 5 * len(self.chunks)   # per chunk: pool, query rotation, score GEMM, row select, attention
+        # per chunk: pooling, the indexer's kernels (query rotation, then scores + row select per row
+        # chunk), the attention's kernels (block lists + attention per launch of query tiles, or one)
+        qsa, w = self.qsa, self.w
+        n = 0
+        for c0, c1 in self.chunks:
+            n += 1 + qsa.qsa_index_topk_prefill_kernels(w.B, c1 - c0, c0, 0, self.dt_code)
+            n += 1 if self.kv8 else qsa.qsa_sparse_attn_prefill_kernels(w.B, c1 - c0, w.top_k, w.Hq, w.Hkv, w.d,
+                                                                        self.dt_code)
+        return n
 
     def units(self):
         return self.w.B * self.w.T   # tokens

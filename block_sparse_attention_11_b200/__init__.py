@@ -24,7 +24,8 @@ __all__ = [
     "qsa_pool_keys_prefill", "qsa_pool_keys_decode",
     "qsa_index_topk_prefill", "qsa_index_topk_prefill_workspace",
     "qsa_index_topk_decode", "qsa_index_topk_decode_workspace", "qsa_index_topk_decode_kernels",
-    "qsa_sparse_attn_prefill", "qsa_sparse_attn_decode", "qsa_sparse_attn_decode_workspace",
+    "qsa_sparse_attn_prefill", "qsa_sparse_attn_prefill_workspace", "qsa_sparse_attn_prefill_kernels",
+    "qsa_index_topk_prefill_kernels", "qsa_sparse_attn_decode", "qsa_sparse_attn_decode_workspace",
     "qsa_sparse_attn_decode_noalloc", "qsa_sparse_attn_decode_shared", "qsa_sparse_attn_decode_shared_workspace",
     "qsa_dense_attn_decode", "qsa_dense_attn_decode_workspace", "qsa_dense_attn_prefill",
     "qsa_pool_keys_prefill_paged", "qsa_pool_keys_decode_paged", "qsa_index_topk_decode_paged",
@@ -102,6 +103,9 @@ _sig("qsa_index_topk_decode", ctypes.c_int, _vp, _vp, _vp, _vp, _i32, _i64, _i64
 _sig("qsa_sparse_attn_prefill", ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i64, _i64, _i32, _i32, _i32,
      _i32, _f32, _vp, _vp, _vp, _sz, _i32, _vp)
 _sig("qsa_sparse_attn_decode_workspace", _sz, _i32, _i32, _i32, _i32, _i32)
+_sig("qsa_sparse_attn_prefill_workspace", _sz, _i32, _i64, _i32, _i32, _i32, _i32, _i32)
+_sig("qsa_sparse_attn_prefill_kernels", ctypes.c_int, _i32, _i64, _i32, _i32, _i32, _i32, _i32)
+_sig("qsa_index_topk_prefill_kernels", ctypes.c_int, _i32, _i64, _i64, _u32, _i32)
 _sig("qsa_sparse_attn_decode", ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32, _i32,
      _f32, _vp, _vp, _vp, _sz, _i32, _vp)
 _sig("qsa_sparse_attn_decode_shared_workspace", _sz, _i32, _i32, _i32, _i32, _i32, _i32)
@@ -257,17 +261,33 @@ def qsa_index_topk_decode(q_idx, k_pool, seq_len, sel, nsel, max_blocks=None, to
     _check(st, "qsa_index_topk_decode")
 
 
-def qsa_sparse_attn_prefill(q, k, v, sel, nsel, out, q0=0, top_k=None, scale=None, lse=None, stream=None):
-    """q [B][n_q][Hq][d]; k, v [B][L][Hkv][d]; sel [B][n_q][top_k]; out like q."""
+def qsa_sparse_attn_prefill_kernels(B, n_q, top_k, Hq, Hkv, d, dtype=QSA_BF16) -> int:
+    return lib.qsa_sparse_attn_prefill_kernels(B, n_q, top_k, Hq, Hkv, d, dtype)
+
+
+def qsa_index_topk_prefill_kernels(B, n_q, q0=0, flags=0, dtype=QSA_BF16) -> int:
+    return lib.qsa_index_topk_prefill_kernels(B, n_q, q0, flags, dtype)
+
+
+def qsa_sparse_attn_prefill_workspace(B, n_q, top_k, Hq, Hkv, d, dtype=QSA_BF16) -> int:
+    return lib.qsa_sparse_attn_prefill_workspace(B, n_q, top_k, Hq, Hkv, d, dtype)
+
+
+def qsa_sparse_attn_prefill(q, k, v, sel, nsel, out, q0=0, top_k=None, scale=None, lse=None, workspace=None,
+                            stream=None):
+    """q [B][n_q][Hq][d]; k, v [B][L][Hkv][d]; sel [B][n_q][top_k]; out like q.  workspace: a uint8
+    device tensor of at least qsa_sparse_attn_prefill_workspace() bytes (allocated here when None)."""
     dt = _dtype_code(q)
     B, n_q, Hq, d = q.shape
     Hkv = k.shape[2]
     top_k = sel.shape[-1] if top_k is None else top_k
     scale = (1.0 / d ** 0.5) if scale is None else scale
+    need = qsa_sparse_attn_prefill_workspace(B, max(n_q, 1), top_k, Hq, Hkv, d, dt)
+    wp, wb = _ws(need, q.device, workspace) if need else (None, 0)
     st = lib.qsa_sparse_attn_prefill(_ptr(q, None, "q"), _ptr(k, q.dtype, "k"), _ptr(v, q.dtype, "v"),
                                      _ptr(sel, torch.int32, "sel"), _ptr(nsel, torch.int32, "nsel"), B, n_q, q0,
                                      k.shape[1], Hq, Hkv, d, top_k, scale, _ptr(out, q.dtype, "out"),
-                                     _ptr(lse, torch.float32, "lse"), None, 0, dt, _stream(q, stream))
+                                     _ptr(lse, torch.float32, "lse"), wp, wb, dt, _stream(q, stream))
     _check(st, "qsa_sparse_attn_prefill")
 
 

@@ -150,6 +150,13 @@ int attn_tail_blocks(bool indexshare, int max_draft);
 size_t attn_decode_ws_bytes(int B, int Hq, int d, int top_k, int tail_blocks = 1);
 size_t attn_dense_decode_ws_bytes(int B, int Hq, int d, int64_t kv_stride);
 cudaError_t launch_attn_bf16(const AttnArgs &a, void *ws, unsigned *status, cudaStream_t s);
+// Prefill on the tensor cores over tiles of 16 queries (k_attn_tc.cu): BF16,
+// d = 128, 8 q heads per kv head, contiguous BF16 K/V.  Its workspace holds
+// the merged block lists of the query tiles.
+bool attn_union_supported(const AttnArgs &a);
+size_t attn_union_ws_bytes(int B, int64_t n_q, int top_k);
+int attn_union_launches(int B, int64_t n_q, int top_k);   // launches of query tiles per call
+cudaError_t launch_attn_union(const AttnArgs &a, void *ws, unsigned *status, cudaStream_t s);
 cudaError_t launch_attn_f32(const AttnArgs &a, unsigned *status, cudaStream_t s);
 
 }  // namespace qsa

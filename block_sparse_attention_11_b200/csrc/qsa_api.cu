@@ -268,6 +268,14 @@ int qsa_index_topk_prefill(const void *q_idx, const void *k_pool, const float *h
     return QSA_OK;
 }
 
+int qsa_index_topk_prefill_kernels(int32_t B, int64_t n_q, int64_t q0, uint32_t flags, int32_t dtype) {
+    if (B < 1 || n_q < 0 || q0 < 0 || (flags & ~kAllFlags) || (dtype != QSA_BF16 && dtype != QSA_FP32)) return 0;
+    if (n_q == 0) return 0;
+    const PrefillPlan pl = prefill_plan(B, n_q, q0, flags, dtype, false);
+    // query rotation, then per chunk of rows: scores and the row select
+    return 1 + 2 * (int)((n_q + pl.chunk - 1) / pl.chunk);
+}
+
 size_t qsa_index_topk_decode_workspace(int32_t B, int64_t max_blocks, int32_t top_k, uint32_t flags, int32_t dtype) {
     (void)flags;
     if (B < 1 || max_blocks < 0 || top_k < 1) return 0;
@@ -309,20 +317,47 @@ int qsa_index_topk_decode(const void *q_idx, const void *k_pool, const float *he
 }
 
 
+size_t qsa_sparse_attn_prefill_workspace(int32_t B, int64_t n_q, int32_t top_k, int32_t Hq, int32_t Hkv, int32_t d,
+                                         int32_t dtype) {
+    if (B < 1 || n_q < 1 || top_k < 1 || top_k > 2048 || Hq < 1 || Hkv < 1) return 0;
+    AttnArgs a{};
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.d = d;
+    if (dtype != QSA_BF16 || !attn_union_supported(a)) return 0;
+    return attn_union_ws_bytes(B, n_q, top_k);
+}
+
+int qsa_sparse_attn_prefill_kernels(int32_t B, int64_t n_q, int32_t top_k, int32_t Hq, int32_t Hkv, int32_t d,
+                                    int32_t dtype) {
+    if (B < 1 || n_q < 1 || top_k < 1 || top_k > 2048 || Hq < 1 || Hkv < 1) return 0;
+    AttnArgs a{};
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.d = d;
+    if (dtype != QSA_BF16 || !attn_union_supported(a)) return 1;
+    return 2 * attn_union_launches(B, n_q, top_k);   // per launch of query tiles: block lists, attention
+}
+
 int qsa_sparse_attn_prefill(const void *q, const void *k, const void *v, const int32_t *sel, const int32_t *nsel,
                             int32_t B, int64_t n_q, int64_t q0, int64_t kv_stride, int32_t Hq, int32_t Hkv, int32_t d,
                             int32_t top_k, float scale, void *out, float *lse, void *workspace, size_t ws_bytes,
                             int32_t dtype, void *stream) {
-    (void)workspace;
-    (void)ws_bytes;
     int st = attn_common_checks(q, k, v, sel, nsel, B, Hq, Hkv, d, top_k, scale, out, dtype);
     if (st != QSA_OK) return st;
     if (n_q < 0 || q0 < 0 || kv_stride < q0 + n_q) return QSA_ERR_INVALID_ARG;
     if (n_q == 0) return QSA_OK;
+    if ((int64_t)B * n_q > INT32_MAX || (int64_t)kv_stride > INT32_MAX) return QSA_ERR_UNSUPPORTED;   // TMA coordinates
     const DeviceInfo *di = nullptr;
     if ((st = check_device(&di)) != QSA_OK) return st;
     AttnArgs a{q, k, v, sel, nsel, nullptr, B, n_q, q0, kv_stride, Hq, Hkv, d, top_k, scale, out, lse, false};
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dtype == QSA_BF16 && attn_union_supported(a)) {
+        const size_t need = attn_union_ws_bytes(B, n_q, top_k);
+        if (!workspace || ws_bytes < need) return QSA_ERR_WORKSPACE;
+        if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return QSA_ERR_INVALID_ARG;
+        return cuda_status(launch_attn_union(a, workspace, di->status, s));
+    }
     cudaError_t e = dtype == QSA_BF16 ? launch_attn_bf16(a, nullptr, di->status, s) : launch_attn_f32(a, di->status, s);
     return cuda_status(e);
 }

@@ -211,6 +211,10 @@ QSA_API int qsa_pool_keys_decode(const void *k_new, void *ring, void *k_pool, co
  * position, after that chunk's keys were pooled into k_pool; the selections
  * equal those of one call over all rows (tested to 1,048,576 positions).
  */
+/* Kernels one qsa_index_topk_prefill call with these sizes launches: the
+ * query rotation, then a score kernel and a row select per chunk of query rows
+ * (chunks keep the score block under 2 GiB); 0 for invalid arguments. */
+QSA_API int qsa_index_topk_prefill_kernels(int32_t B, int64_t n_q, int64_t q0, uint32_t flags, int32_t dtype);
 QSA_API size_t qsa_index_topk_prefill_workspace(int32_t B, int64_t n_q, int64_t q0, int32_t top_k,
                                         uint32_t flags, int32_t dtype);
 QSA_API int qsa_index_topk_prefill(const void *q_idx, const void *k_pool, const float *head_w, int32_t B,
@@ -281,9 +285,28 @@ QSA_API int qsa_index_topk_decode(const void *q_idx, const void *k_pool, const f
  *         Hkv in {1, 2, 4} (any ratio for QSA_FP32); or, QSA_BF16 only, the
  *         released model's shape Hq = 24, Hkv = 2, d = 256 (the architecture
  *         guide page, section "How a token moves through the model", item 2:
- *         24 query heads, two KV heads of dimension 256); kv_stride >= q0 + n_q.
- * workspace: none needed (pass NULL, 0).
+ *         24 query heads, two KV heads of dimension 256); kv_stride >= q0 + n_q;
+ *         B * n_q and kv_stride below 2^31.
+ * workspace: device, 256-byte aligned, at least qsa_sparse_attn_prefill_workspace()
+ *          bytes, caller-owned and needing no initialisation; 0 bytes (pass
+ *          NULL) for the shapes that run without one.  QSA_BF16 with d = 128,
+ *          Hq = 8 Hkv runs on the tensor cores over tiles of 16 consecutive
+ *          query rows: a pre-pass merges the tile's 16 selections and tail
+ *          blocks into one ascending block list (with a per-block mask of the
+ *          queries attending to it) in the workspace, so each listed block's
+ *          K/V is gathered once per tile and kv head; masked keys contribute
+ *          exactly zero.  The workspace is capped near 512 MiB: longer
+ *          prompts run as several launches of whole query tiles.  Results of a
+ *          chunk starting at a row that is a multiple of 16 equal those of the
+ *          same rows in one call bit for bit.  Too small: QSA_ERR_WORKSPACE.
  */
+/* Kernels one qsa_sparse_attn_prefill call with these sizes launches: 1 (the
+ * gather kernels: fp32, d = 256, other GQA ratios) or 2 per launch of query
+ * tiles (block lists, attention); 0 for invalid arguments. */
+QSA_API int qsa_sparse_attn_prefill_kernels(int32_t B, int64_t n_q, int32_t top_k, int32_t Hq, int32_t Hkv, int32_t d,
+                                            int32_t dtype);
+QSA_API size_t qsa_sparse_attn_prefill_workspace(int32_t B, int64_t n_q, int32_t top_k, int32_t Hq, int32_t Hkv,
+                                                 int32_t d, int32_t dtype);
 QSA_API int qsa_sparse_attn_prefill(const void *q, const void *k, const void *v, const int32_t *sel,
                             const int32_t *nsel, int32_t B, int64_t n_q, int64_t q0, int64_t kv_stride,
                             int32_t Hq, int32_t Hkv, int32_t d, int32_t top_k, float scale, void *out,

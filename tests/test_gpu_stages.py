@@ -906,3 +906,96 @@ def test_dense_decode_matches_textbook_attention(qsa, dtype, Hq, Hkv, B, L):
         ref = oracle.dense_rows([0], q=np32(q[b])[None], k=np32(k[b]), v=np32(v[b]), Hq=Hq, Hkv=Hkv, d=d, q0=t)
         err = np.abs(np32(out[b]) - ref[0]).max()
         assert err <= TOL[dtype], (b, err)
+
+
+# ----------------------------------------------------------------------------- tensor-core prefill over query tiles
+
+def _overlapping_selection(T, top_k, seed, hot=64, short_every=5):
+    """Seeded selections whose neighbouring rows overlap (a shared hot set of
+    blocks plus row-specific ones), some rows shorter than min(top_k, nb)."""
+    rng = np.random.default_rng(seed)
+    sel = np.full((T, top_k), -1, np.int32)
+    nsel = np.zeros(T, np.int32)
+    hot_ids = rng.permutation(max(T // 4, 1))[:hot]
+    for t in range(T):
+        nb = (t + 1) // 4
+        if nb == 0:
+            continue
+        want = min(top_k, nb)
+        if t % short_every == 0:
+            want = max(1, want // 3)
+        cand = [b for b in hot_ids if b < nb][: want // 2]
+        rest = rng.permutation(nb)
+        chosen = list(dict.fromkeys(list(cand) + list(rest)))[:want]
+        chosen = np.sort(np.array(chosen, np.int32))
+        sel[t, :len(chosen)] = chosen
+        nsel[t] = len(chosen)
+    return sel, nsel
+
+
+@pytest.mark.parametrize("Hq,Hkv,T,top_k", [(16, 2, 1500, 96), (8, 1, 777, 64), (32, 4, 2049, 128),
+                                           (16, 2, 9000, 2048), (16, 2, 5, 4)])
+def test_tile_attention_on_overlapping_selections(qsa, Hq, Hkv, T, top_k):
+    """Hand-built overlapping selections (hot blocks shared by many rows, rows
+    with fewer than min(top_k, nb) blocks, a last partial 16-row tile): the
+    tensor-core prefill equals the oracle's attention over the same selections,
+    B = 2 sequences with different selections."""
+    w = W(T, top_k=top_k, Hq=Hq, Hkv=Hkv, B=2, seed=90 + Hq)
+    x = workloads.make_prefill(w, device=DEV)
+    sels, nsels = zip(*[_overlapping_selection(T, top_k, seed=7 + b) for b in range(2)])
+    sel = torch.from_numpy(np.stack(sels)).to(DEV)
+    nsel = torch.from_numpy(np.stack(nsels)).to(DEV)
+    out = torch.full_like(x["q"], 9.0)
+    lse = torch.empty(2, T, Hq, dtype=torch.float32, device=DEV)
+    qsa.qsa_sparse_attn_prefill(x["q"], x["k"], x["v"], sel, nsel, out, lse=lse)
+    qsa.qsa_check_status()
+    rows = list(range(T)) if T <= 2100 else sorted(set(range(0, T, 3)) | set(range(T - 40, T)))
+    for b in range(2):
+        ref = oracle.prefill_rows(rows, sel_in=sels[b][rows], nsel_in=nsels[b][rows], top_k=top_k,
+                                  q=np32(x["q"][b]), k=np32(x["k"][b]), v=np32(x["v"][b]), Hq=Hq, Hkv=Hkv, d=128)
+        err = np.abs(np32(out[b])[rows] - ref["out"]).max()
+        assert err <= TOL["bf16"], (b, err)
+        assert np.abs(lse[b].cpu().numpy()[rows] - ref["lse"]).max() <= 1e-3
+
+
+def test_tile_attention_chunks_off_the_tile_grid(qsa):
+    """Chunks that start off the 16-row tile grid (q0 = 1000, 1001) form other
+    tiles than one call does; every row still matches the oracle."""
+    T, top_k = 1700, 64
+    w = W(T, top_k=top_k, seed=95)
+    x = workloads.make_prefill(w, device=DEV)
+    sel_np, nsel_np = _overlapping_selection(T, top_k, seed=3)
+    sel = torch.from_numpy(sel_np[None]).to(DEV)
+    nsel = torch.from_numpy(nsel_np[None]).to(DEV)
+    out = torch.empty_like(x["q"])
+    for c0, c1 in [(0, 1000), (1000, 1001), (1001, 1700)]:
+        o = torch.empty(1, c1 - c0, 16, 128, dtype=torch.bfloat16, device=DEV)
+        qsa.qsa_sparse_attn_prefill(x["q"][:, c0:c1].contiguous(), x["k"], x["v"], sel[:, c0:c1].contiguous(),
+                                    nsel[:, c0:c1].contiguous(), o, q0=c0)
+        out[:, c0:c1] = o
+    qsa.qsa_check_status()
+    rows = list(range(T))
+    ref = oracle.prefill_rows(rows, sel_in=sel_np, nsel_in=nsel_np, top_k=top_k, q=np32(x["q"][0]),
+                              k=np32(x["k"][0]), v=np32(x["v"][0]), Hq=16, Hkv=2, d=128)
+    assert np.abs(np32(out[0]) - ref["out"]).max() <= TOL["bf16"]
+
+
+def test_tile_attention_aligned_chunks_are_bit_exact(qsa):
+    """Chunks starting on the 16-row tile grid reproduce one call bit for bit
+    (same tiles, same block lists, same order of accumulation)."""
+    T, top_k = 2000, 96
+    w = W(T, top_k=top_k, seed=96)
+    x = workloads.make_prefill(w, device=DEV)
+    sel_np, nsel_np = _overlapping_selection(T, top_k, seed=4)
+    sel = torch.from_numpy(sel_np[None]).to(DEV)
+    nsel = torch.from_numpy(nsel_np[None]).to(DEV)
+    one = torch.empty_like(x["q"])
+    qsa.qsa_sparse_attn_prefill(x["q"], x["k"], x["v"], sel, nsel, one)
+    out = torch.empty_like(x["q"])
+    for c0, c1 in [(0, 512), (512, 1536), (1536, 2000)]:
+        o = torch.empty(1, c1 - c0, 16, 128, dtype=torch.bfloat16, device=DEV)
+        qsa.qsa_sparse_attn_prefill(x["q"][:, c0:c1].contiguous(), x["k"], x["v"], sel[:, c0:c1].contiguous(),
+                                    nsel[:, c0:c1].contiguous(), o, q0=c0)
+        out[:, c0:c1] = o
+    qsa.qsa_check_status()
+    assert torch.equal(out, one)
