@@ -100,14 +100,13 @@ def measure_l2_read(dev, reps=40):
     best = 0.0
     for mib in (24, 48, 64):
         x = torch.ones(mib * (1 << 20) // 4, dtype=torch.float32, device=dev)
-        acc = torch.empty((), dtype=torch.float32, device=dev)
         for _ in range(3):
-            torch.sum(x, out=acc)
+            x.sum()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         for _ in range(reps):
-            torch.sum(x, out=acc)
+            x.sum()
         e1.record()
         torch.cuda.synchronize()
         best = max(best, x.numel() * 4 * reps / (e0.elapsed_time(e1) / 1e3) / 1e9)

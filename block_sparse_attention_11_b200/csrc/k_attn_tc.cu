@@ -58,7 +58,10 @@ constexpr uint32_t TM_Q = 384;         // Q, 64 columns (bf16 pairs)
 constexpr uint32_t TM_COLS = 512;
 constexpr int UCHUNK = 16384;          // pre-pass: block ids per pass (one 32-bit mask word each)
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kRescale = 8.f;        // lazy rescale threshold (log2 units)
+#ifndef QSA_UT_RESCALE
+#define QSA_UT_RESCALE 8.f
+#endif
+constexpr float kRescale = QSA_UT_RESCALE;   // lazy rescale threshold (log2 units)
 
 struct UtMeta {
     int32_t id[UB];                    // listed block ids of the tile (-1: padding)
@@ -73,7 +76,7 @@ struct UtSmem {
     UtMeta meta[UNS];
     uint64_t full[UNS], empty[UNS];
     uint64_t q_full, q_empty, q_ready;
-    uint64_t s_full[2], p_ready[2], pv_done, drain;
+    uint64_t s_full[2], p_ready[2], pv_done, o_full, drain;
     uint32_t tmem_base;
 };
 
@@ -234,6 +237,7 @@ __global__ void __launch_bounds__(UT_THREADS, 1)
             mbar_init(&sm.p_ready[b], 4);
         }
         mbar_init(&sm.pv_done, 1);
+        mbar_init(&sm.o_full, 1);
         mbar_init(&sm.drain, 1);
         fence_mbar_init();
     }
@@ -360,6 +364,11 @@ __global__ void __launch_bounds__(UT_THREADS, 1)
                         tc_commit(&sm.pv_done);
                     }
                 }
+                // the item's O is complete: one phase of o_full per item.  (The
+                // epilogue cannot wait on pv_done by parity: when it gets there
+                // the item's last two products may both still be in flight, two
+                // phases behind, which a parity wait cannot tell apart.)
+                if (ok) tc_commit(&sm.o_full);
                 c += ntile;
             }
             // every MMA issued has completed before the TMEM is released
@@ -441,7 +450,10 @@ __global__ void __launch_bounds__(UT_THREADS, 1)
                 const bool grow = mx > m_run + kRescale;       // also the first keys of the row
                 const bool resc = grow && m_run != -INFINITY;  // O and l already hold earlier keys
                 if (__any_sync(0xffffffffu, resc)) {
-                    // the previous P V must have landed before O is read
+                    // the previous P V must have landed before O is read.  A parity
+                    // wait is exact here: S(c) landing means every MMA issued before
+                    // QK(c) is done, P V(c - 2) included, and P V(c) needs this
+                    // warp's P(c), so pv_done is at phase c - 1 or c.
                     ok = __all_sync(0xffffffffu, mbar_wait(&sm.pv_done, (int)((c - 1) & 1), p.status));
                     if (!ok) break;
                     tc_fence_after();
@@ -487,7 +499,7 @@ __global__ void __launch_bounds__(UT_THREADS, 1)
             }
             if (!ok) break;
             // epilogue: O / l -> bf16 rows of the output; lse
-            ok = __all_sync(0xffffffffu, ntile == 0 || mbar_wait(&sm.pv_done, (int)((c - 1) & 1), p.status));
+            ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_full, (int)(ic & 1), p.status));
             if (!ok) break;
             tc_fence_after();
             const bool live = qi < it.nrows;
