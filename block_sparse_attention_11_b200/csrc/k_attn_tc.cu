@@ -1,5 +1,5 @@
 // k_attn_tc.cu -- prefill sparse attention on the tensor cores, one tile of
-// 16 consecutive queries at a time.
+// 8 consecutive queries at a time.
 //
 // Page "Qwen3.8-Flash-Next: Day-0 Support in SGLang", section "Qwen Sparse
 // Attention: Retrieve Coarsely, Attend Precisely": each query attends over the
@@ -9,27 +9,43 @@
 //
 // Neighbouring queries select overlapping blocks (heavy-tailed keys are chosen
 // by many queries; early queries see few blocks), so this kernel gathers each
-// block once for a tile of UQ = 16 queries:
-//   * a pre-pass (union_build_kernel) merges the 16 selections and tail blocks
-//     of a query tile into one ascending list of blocks, each with a 16-bit
-//     mask of the queries that attend to it;
-//   * for one kv head g, the 16 queries x 8 q heads form the M = 128 rows of
-//     two tcgen05 GEMMs per key tile of 32 listed blocks (N = 128 keys):
-//       S = Q K^T   (A = Q from tensor memory, B = K tile, 128-byte swizzle)
-//       O += P V    (A = P from tensor memory, B = V tile read MN-major)
-//     with S, P and O in tensor memory and K/V tiles landing in shared memory
-//     by TMA (one 4-token x 64-dim box per block, dim half and tensor);
-//   * 4 softmax warps own one TMEM row each ((query, head) = row / 8, row % 8):
-//     they mask the keys their query does not attend to (mask bit, and for the
-//     blocks at the diagonal key position <= query position), keep the fp32
-//     online-softmax state of their row, rescale their O row in tensor memory
-//     when the row maximum grows by more than 2^8 (lazy rescaling), and write
-//     P back over S as bf16.
-// A masked key contributes p = 0 exactly, so each query's result is its own
-// softmax over its own positions; the extra products are the price of reading
-// each block once.  Warp roles: 0 = TMA producer, 1 = MMA issuer and TMEM
-// owner, 2..5 = softmax and epilogue.  A persistent grid walks the work items
-// (sequence, query tile, kv head), latest query tiles first.
+// block once for a tile of UQ = 8 queries:
+//   * a pre-pass (union_build_kernel) merges the 8 selections and tail blocks
+//     of a query tile into one ascending list of blocks, each with a mask of
+//     the queries that attend to it;
+//   * a block of a pair of kv heads (4 tokens x 2 heads x 128 dims = 2 KB per
+//     tensor) arrives as ONE 5-D TMA box, already in the 128-byte-swizzled
+//     layout the tensor cores read: two 8-row atoms (dims 0-63, dims 64-127),
+//     row = head * 4 + token.  Measured on B200, the TMA engine's cost is per
+//     request, so whole 2 KB blocks issued by four producer warps gather about
+//     7x faster than 4-row boxes of one head from one warp;
+//   * the 8 queries x 16 q heads of the kv-head pair form the M = 128 rows of
+//     two tcgen05 GEMMs per key tile of 16 listed blocks (N = 128 keys):
+//       S = Q K^T          (A = Q, staged once per item in shared memory)
+//       O_h += P_h V_h     (A = P from tensor memory, B = V tile read MN-major)
+//     A row of S pairs each q head with the keys of both kv heads; the other
+//     head's keys are masked (p = 0), the price of one 2 KB request per block.
+//     Rows are ordered (kv head, query, q head), so each TMEM lane quarter
+//     holds the rows of one kv head;
+//   * the key tile is split in two column halves h (blocks 0-7, 8-15), each
+//     with its own accumulator O_h in tensor memory and its own running
+//     maximum: 8 softmax warps, two per TMEM lane quarter (one per half), run
+//     the online softmax of their half with no exchange per key tile, rescale
+//     their O_h only when their maximum grows by more than 2^64 (lazy
+//     rescaling: P is bf16, with fp32's exponent range, so p <= 2^64 and
+//     the fp32 sums of O and l stay far from overflow; the final division
+//     cancels the common scale),
+//     and write P over their half of S as bf16.  At the end of an item the
+//     two halves exchange (maximum, sum) through tensor memory and combine:
+//       O = (2^(m_0 - m) O_0 + 2^(m_1 - m) O_1) / (2^(m_0 - m) l_0 + 2^(m_1 - m) l_1),
+//     m = max(m_0, m_1), the usual merge of two partial softmaxes.
+// A masked key contributes p = 0 exactly (the query's mask bit, the other kv
+// head, and at the diagonal key position <= query position), so each query's
+// result is its own softmax over its own positions.  Warp roles: 0-2 = TMA
+// producers, 3 = MMA issuer and TMEM owner, 4-11 = softmax and epilogue (12
+// warps leave 168 registers a thread, so the softmax state never spills).  A
+// persistent grid walks the work items (sequence, query tile, kv-head pair),
+// latest tiles first.
 #include <algorithm>
 
 #include "internal.h"
@@ -38,28 +54,34 @@ namespace qsa {
 
 namespace {
 
-constexpr int UQ = 16;                 // queries per tile
+constexpr int UQ = 8;                  // queries per tile
 constexpr int UG = 8;                  // q heads per kv head
-constexpr int UM = UQ * UG;            // MMA rows
-constexpr int UB = 32;                 // listed blocks per key tile
-constexpr int UN = UB * kBlock;        // keys per tile
+constexpr int UH = 2 * UG;             // q heads of a kv-head pair
+constexpr int UM = UQ * UH;            // MMA rows
+constexpr int UB = 16;                 // listed blocks per key tile
+constexpr int UBLK = 2048;             // one block of a kv-head pair, one tensor: 2 atoms of 8 x 128 B
+constexpr int UN = UB * 8;             // S columns per tile: 16 blocks x 4 tokens x 2 heads
 constexpr int UD = 128;                // head dim
-constexpr int UREG = UN * 128;         // 128 rows x 128 bytes (64 bf16 dims), 128-byte swizzle
-constexpr int USTAGE = 4 * UREG;       // K dims 0-63, K dims 64-127, V dims 0-63, V dims 64-127
-constexpr int UBOX = kBlock * 128;     // one TMA box: 4 tokens x 64 dims
+constexpr int UKV = UB * UBLK;         // one tensor's tile (32 KB)
+constexpr int USTAGE = 2 * UKV;        // K tile, V tile
+constexpr int UPW = 3;                 // producer warps
+constexpr int UBPW = (UB + UPW - 1) / UPW;   // blocks per producer warp per tile (the last takes fewer)
 #ifndef QSA_UT_STAGES
 #define QSA_UT_STAGES 3
 #endif
 constexpr int UNS = QSA_UT_STAGES;     // key tiles in flight
-constexpr int UT_THREADS = 192;
+constexpr int UPRE = 4;                // key tiles whose block ids the producers hold ahead
+constexpr int UW_MMA = UPW;            // warp index of the MMA issuer
+constexpr int USW = 8;                 // softmax warps: two per TMEM lane quarter, one per column half
+constexpr int UT_THREADS = (UPW + 1 + USW) * 32;
+constexpr int UQH = UM * 128;          // Q in shared memory: one 64-dim half of 128 rows (16 KB)
 constexpr uint32_t TM_S = 0;           // S / P, two buffers of 128 columns
-constexpr uint32_t TM_O = 256;         // O, 128 columns
-constexpr uint32_t TM_Q = 384;         // Q, 64 columns (bf16 pairs)
+constexpr uint32_t TM_O = 256;         // O_0, O_1: 128 columns each
 constexpr uint32_t TM_COLS = 512;
 constexpr int UCHUNK = 16384;          // pre-pass: block ids per pass (one 32-bit mask word each)
 constexpr float kLog2e = 1.4426950408889634f;
 #ifndef QSA_UT_RESCALE
-#define QSA_UT_RESCALE 8.f
+#define QSA_UT_RESCALE 64.f
 #endif
 constexpr float kRescale = QSA_UT_RESCALE;   // lazy rescale threshold (log2 units)
 
@@ -67,15 +89,15 @@ struct UtMeta {
     int32_t id[UB];                    // listed block ids of the tile (-1: padding)
     uint32_t mw[UQ];                   // per query: bit j = the query attends to block j of the tile
     int32_t diag;                      // a block of the tile reaches past the tile's first query
-    int32_t pad[15];
+    int32_t pad[7];
 };
 
 struct UtSmem {
     alignas(1024) uint8_t kv[UNS][USTAGE];
-    alignas(1024) uint8_t qs[2 * UREG];            // Q tile staging: 128 rows x 128 dims, two swizzled halves
+    alignas(1024) uint8_t q[2 * UQH];              // Q: dims 0-63 | dims 64-127, rows of 128 B, 128-B swizzle
     UtMeta meta[UNS];
     uint64_t full[UNS], empty[UNS];
-    uint64_t q_full, q_empty, q_ready;
+    uint64_t q_ready;
     uint64_t s_full[2], p_ready[2], pv_done, o_full, drain;
     uint32_t tmem_base;
 };
@@ -83,6 +105,7 @@ struct UtSmem {
 static_assert(sizeof(UtSmem) + 1024 <= 232448, "shared memory of the attention CTA exceeds 227 KB");
 
 struct UtParams {
+    const __nv_bfloat16 *q;  // [B][n_q][Hq][128]
     int B;
     int64_t n_q, q0;
     int Hq, Hkv;
@@ -100,7 +123,7 @@ struct UtParams {
 };
 
 struct UtItem {
-    int seq, g, nrows, n_u;
+    int seq, pair, nrows, n_u;
     int64_t r0, t0;
     const uint32_t *ids;
     const uint16_t *msk;
@@ -108,11 +131,12 @@ struct UtItem {
 
 __device__ __forceinline__ UtItem ut_item(const UtParams &p, int64_t i) {
     UtItem it;
-    const int64_t per = (int64_t)p.B * p.Hkv;
+    const int npair = p.Hkv / 2;
+    const int64_t per = (int64_t)p.B * npair;
     const int64_t qt = p.n_qt - 1 - i / per;   // latest (longest) query tiles first
     const int rem = (int)(i % per);
-    it.seq = rem / p.Hkv;
-    it.g = rem % p.Hkv;
+    it.seq = rem / npair;
+    it.pair = rem % npair;
     it.r0 = p.row0 + qt * UQ;
     it.nrows = (int)(p.row_end - it.r0 < UQ ? p.row_end - it.r0 : UQ);
     it.t0 = p.q0 + it.r0;
@@ -124,7 +148,7 @@ __device__ __forceinline__ UtItem ut_item(const UtParams &p, int64_t i) {
 }
 
 // ---------------------------------------------------------------- pre-pass
-// One CTA per (query tile, sequence).  Block ids of the tile's 16 selections
+// One CTA per (query tile, sequence).  Block ids of the tile's selections
 // (validated: 0 <= b < nb(t)) and each query's tail block (when it holds 1-3
 // tokens) set bit q in a mask word per id; the non-zero words are compacted
 // in id order.  Ids are processed UCHUNK at a time.
@@ -214,8 +238,8 @@ __global__ void __launch_bounds__(256) union_build_kernel(const int32_t *__restr
 
 // ---------------------------------------------------------------- attention
 __global__ void __launch_bounds__(UT_THREADS, 1)
-    attn_union_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
-                      const __grid_constant__ CUtensorMap map_v, UtParams p) {
+    attn_union_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
+                      UtParams p) {
     extern __shared__ uint8_t ut_raw[];
     UtSmem &sm = *reinterpret_cast<UtSmem *>((reinterpret_cast<uintptr_t>(ut_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -226,22 +250,20 @@ __global__ void __launch_bounds__(UT_THREADS, 1)
         reinterpret_cast<uint4 *>(&sm.kv[0][0])[i] = make_uint4(0, 0, 0, 0);
     if (threadIdx.x == 0) {
         for (int s = 0; s < UNS; ++s) {
-            mbar_init(&sm.full[s], 32);
+            mbar_init(&sm.full[s], 32 + UPW - 1);   // warp 0's lanes (they write the meta), lane 0 of the others
             mbar_init(&sm.empty[s], 1);
         }
-        mbar_init(&sm.q_full, 1);
-        mbar_init(&sm.q_empty, 4);
-        mbar_init(&sm.q_ready, 4);
+        mbar_init(&sm.q_ready, USW);
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm.s_full[b], 1);
-            mbar_init(&sm.p_ready[b], 4);
+            mbar_init(&sm.p_ready[b], USW);
         }
         mbar_init(&sm.pv_done, 1);
         mbar_init(&sm.o_full, 1);
         mbar_init(&sm.drain, 1);
         fence_mbar_init();
     }
-    if (warp == 1) {
+    if (warp == UW_MMA) {
         tmem_alloc(&sm.tmem_base, TM_COLS);
         tmem_relinquish();
     }
@@ -253,79 +275,99 @@ __global__ void __launch_bounds__(UT_THREADS, 1)
     pdl_wait();       // the block lists come from the pre-pass
     pdl_trigger();
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            prefetch_tmap(&map_q);
+    if (warp < UPW) {
+        // ------------------------------------------------------------ TMA producers
+        // Every producer warp reads the tile's 16 entries (lanes 0-15); warp 0
+        // writes the tile's meta, warp w issues the boxes of blocks
+        // [UBPW w, UBPW w + UBPW).
+        if (warp == 0 && lane == 0) {
             prefetch_tmap(&map_k);
             prefetch_tmap(&map_v);
         }
-        int64_t c = 0, nq = 0;   // stages issued, Q tiles issued
+        int64_t c = 0;   // stages issued
+        int st = 0;      // stage of the next tile
+        uint32_t eph = 1;   // parity of the empty phase to wait for (the first round waits for nothing)
         bool ok = true;
         for (int64_t i = blockIdx.x; i < p.items && ok; i += gridDim.x) {
             const UtItem it = ut_item(p, i);
-            if (nq >= 1) ok = mbar_wait(&sm.q_empty, (int)((nq - 1) & 1), p.status);
-            ok = __all_sync(0xffffffffu, ok);
-            if (!ok) break;
-            if (lane == 0) {
-                mbar_arrive_expect_tx(&sm.q_full, 2 * UREG);
-                const int qrow = (int)((int64_t)it.seq * p.n_q + it.r0);
-                tma_load_3d(sm.qs, &map_q, 0, UG * it.g, qrow, &sm.q_full);
-                tma_load_3d(sm.qs + UREG, &map_q, 64, UG * it.g, qrow, &sm.q_full);
-            }
-            ++nq;
             const int ntile = (it.n_u + UB - 1) / UB;
-            uint32_t e_id = lane < it.n_u ? it.ids[lane] : 0xFFFFFFFFu;
-            uint32_t e_m = lane < it.n_u ? it.msk[lane] : 0u;
-            for (int u = 0; u < ntile; ++u) {
-                const int nx = (u + 1) * UB + lane;            // next tile's entries, loaded ahead
-                const uint32_t n_id = nx < it.n_u ? it.ids[nx] : 0xFFFFFFFFu;
-                const uint32_t n_m = nx < it.n_u ? it.msk[nx] : 0u;
-                const int s = (int)(c % UNS);
-                if (c >= UNS) ok = mbar_wait(&sm.empty[s], (int)(((c / UNS) + 1) & 1), p.status);
-                ok = __all_sync(0xffffffffu, ok);
-                if (!ok) break;
-                const bool live = e_id != 0xFFFFFFFFu;
-                UtMeta &mt = sm.meta[s];
-                mt.id[lane] = live ? (int32_t)e_id : -1;
-                uint32_t mine = 0;
+            const bool rl = lane < UB;
+            // the entries of the next UPRE key tiles are in flight (lanes 0-15 of each warp):
+            // one tile ahead leaves every stage waiting a full L2 round trip for its ids
+            uint32_t rid[UPRE], rmk[UPRE];
 #pragma unroll
-                for (int q = 0; q < UQ; ++q) {
-                    const uint32_t b = __ballot_sync(0xffffffffu, (e_m >> q) & 1u);
-                    if (lane == q) mine = b;
+            for (int k = 0; k < UPRE; ++k) {
+                const int x = k * UB + lane;
+                rid[k] = (rl && x < it.n_u) ? __ldg(it.ids + x) : 0xFFFFFFFFu;
+                rmk[k] = (rl && x < it.n_u) ? (uint32_t)__ldg(it.msk + x) : 0u;
+            }
+            for (int u0 = 0; u0 < ntile && ok; u0 += UPRE) {
+#pragma unroll
+                for (int k = 0; k < UPRE; ++k) {
+                    const int u = u0 + k;
+                    if (u >= ntile) break;
+                    const uint32_t e_id = rid[k], e_m = rmk[k];
+                    {
+                        const int x = (u + UPRE) * UB + lane;
+                        rid[k] = (rl && x < it.n_u) ? __ldg(it.ids + x) : 0xFFFFFFFFu;
+                        rmk[k] = (rl && x < it.n_u) ? (uint32_t)__ldg(it.msk + x) : 0u;
+                    }
+                    const int s = st;
+                    if (c >= UNS) ok = mbar_wait(&sm.empty[s], eph, p.status);
+                    ok = __all_sync(0xffffffffu, ok);
+                    if (!ok) break;
+                    const bool live = e_id != 0xFFFFFFFFu;
+                    if (warp == 0) {
+                        UtMeta &mt = sm.meta[s];
+                        if (rl) mt.id[lane] = live ? (int32_t)e_id : -1;
+                        uint32_t mine = 0;
+#pragma unroll
+                        for (int q = 0; q < UQ; ++q) {
+                            const uint32_t b = __ballot_sync(0xffffffffu, (e_m >> q) & 1u);
+                            if (lane == q) mine = b;
+                        }
+                        if (lane < UQ) mt.mw[lane] = mine;
+                        const int maxid = __reduce_max_sync(0xffffffffu, live ? (int)e_id : -1);
+                        if (lane == 0) mt.diag = ((int64_t)kBlock * maxid + kBlock - 1 > it.t0) ? 1 : 0;
+                    }
+                    const bool mine_blk = lane >= UBPW * warp && lane < UBPW * (warp + 1);
+                    const uint32_t nlive = __popc(__ballot_sync(0xffffffffu, live && mine_blk));
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_expect_tx(&sm.full[s], nlive * 2u * UBLK);
+                    else if (warp == 0) mbar_arrive(&sm.full[s]);
+                    __syncwarp();
+                    if (live && mine_blk) {
+                        uint8_t *dst = sm.kv[s] + lane * UBLK;
+                        const int tok = kBlock * (int)e_id;
+                        tma_load_5d(dst, &map_k, 0, tok, 2 * it.pair, 0, it.seq, &sm.full[s]);
+                        tma_load_5d(dst + UKV, &map_v, 0, tok, 2 * it.pair, 0, it.seq, &sm.full[s]);
+                    }
+                    ++c;
+                    if (++st == UNS) {
+                        st = 0;
+                        eph ^= 1u;
+                    }
                 }
-                if (lane < UQ) mt.mw[lane] = mine;
-                const int maxid = __reduce_max_sync(0xffffffffu, live ? (int)e_id : -1);
-                if (lane == 0) mt.diag = ((int64_t)kBlock * maxid + kBlock - 1 > it.t0) ? 1 : 0;
-                const uint32_t nlive = __popc(__ballot_sync(0xffffffffu, live));
-                __syncwarp();
-                if (lane == 0) mbar_arrive_expect_tx(&sm.full[s], nlive * 4u * UBOX);
-                else mbar_arrive(&sm.full[s]);
-                if (live) {
-                    uint8_t *st = sm.kv[s] + lane * UBOX;
-                    const int tok = kBlock * (int)e_id;
-                    tma_load_4d(st, &map_k, 0, it.g, tok, it.seq, &sm.full[s]);
-                    tma_load_4d(st + UREG, &map_k, 64, it.g, tok, it.seq, &sm.full[s]);
-                    tma_load_4d(st + 2 * UREG, &map_v, 0, it.g, tok, it.seq, &sm.full[s]);
-                    tma_load_4d(st + 3 * UREG, &map_v, 64, it.g, tok, it.seq, &sm.full[s]);
-                }
-                ++c;
-                e_id = n_id;
-                e_m = n_m;
             }
         }
         // no copy may still be landing when the CTA ends (bounded waits)
-        if (lane == 0) {
+        if (lane == 0)
             for (int64_t cc = (c > UNS ? c - UNS : 0); cc < c; ++cc)
                 mbar_wait(&sm.full[cc % UNS], (int)((cc / UNS) & 1), p.status);
-            if (nq >= 1) mbar_wait(&sm.q_full, (int)((nq - 1) & 1), p.status);
-        }
-    } else if (warp == 1) {
+    } else if (warp == UW_MMA) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t idesc_qk = idesc_bf16_f32(UM, UN);
             const uint32_t idesc_pv = idesc_bf16_f32(UM, UD) | (1u << 16);   // B = V tile, MN-major
+            // shared-memory descriptors: the start address (bits 0-13, 16-byte units) of each
+            // operand advances by adding to the descriptor of stage 0 / k-step 0
+            const uint64_t dq = sw128_desc(smem_u32(sm.q));                     // Q, 8-row groups 1024 B apart
+            const uint64_t dk0 = sw128_desc_ls(smem_u32(sm.kv[0]), 16, UBLK);  // K tile, 8-row groups 2048 B apart
+            const uint64_t dv0 = sw128_desc_ls(smem_u32(sm.kv[0]) + UKV, 1024, UBLK);   // V tile, MN-major
+            constexpr uint64_t kStageD = USTAGE >> 4;
             int64_t c = 0, ic = 0;
+            int qs = 0, ps = 0;      // stages of the next QK and the next P V
+            uint32_t qph = 0;        // phase of the next QK's stage
             bool ok = true;
             for (int64_t i = blockIdx.x; i < p.items && ok; i += gridDim.x, ++ic) {
                 const UtItem it = ut_item(p, i);
@@ -336,32 +378,43 @@ __global__ void __launch_bounds__(UT_THREADS, 1)
                 for (int u = 0; u <= ntile && ok; ++u) {
                     if (u < ntile) {   // S(u) = Q K(u)^T
                         const int64_t cu = c + u;
-                        const int s = (int)(cu % UNS);
-                        ok = mbar_wait(&sm.full[s], (int)((cu / UNS) & 1), p.status);
+                        ok = mbar_wait(&sm.full[qs], qph, p.status);
                         if (!ok) break;
                         tc_fence_after();
                         const uint32_t d = tmem + TM_S + (uint32_t)((cu & 1) * 128);
-                        const uint32_t kb = smem_u32(sm.kv[s]);
+                        const uint64_t dk = dk0 + (uint64_t)qs * kStageD;
+                        // k-step k: dims 16 k .. 16 k + 15 = 32-byte column (k & 3) of the 64-dim half k >> 2
+                        // (Q: halves 16 KB apart; K tile: block j's dims 0-63 atom at 2048 j, dims 64-127 at + 1024)
 #pragma unroll
                         for (int k = 0; k < 8; ++k)
-                            tc_mma_ts(d, tmem + TM_Q + 8 * k, sw128_desc(kb + (k >> 2) * UREG + (k & 3) * 32),
-                                      idesc_qk, k > 0 ? 1u : 0u);
+                            tc_mma_f16(d, dq + (uint64_t)(((k >> 2) * UQH + (k & 3) * 32) >> 4),
+                                       dk + (uint64_t)(((k >> 2) * 1024 + (k & 3) * 32) >> 4), idesc_qk,
+                                       k > 0 ? 1u : 0u);
                         tc_commit(&sm.s_full[cu & 1]);
+                        if (++qs == UNS) {
+                            qs = 0;
+                            qph ^= 1u;
+                        }
                     }
-                    if (u >= 1) {      // O += P(u-1) V(u-1)
+                    if (u >= 1) {      // O_h += P_h(u-1) V_h(u-1), h = 0, 1
                         const int64_t cp = c + u - 1;
                         ok = mbar_wait(&sm.p_ready[cp & 1], (int)((cp >> 1) & 1), p.status);
                         if (!ok) break;
                         tc_fence_after();
-                        const int s = (int)(cp % UNS);
-                        const uint32_t vb = smem_u32(sm.kv[s]) + 2 * UREG;
+                        const uint64_t dv = dv0 + (uint64_t)ps * kStageD;
                         const uint32_t pa = tmem + TM_S + (uint32_t)((cp & 1) * 128);
+                        // P_h: 32 columns at 64 h (keys 64 h .. 64 h + 63); V tile MN-major, 16 rows
+                        // (2 blocks) per k-step, dims 64-127 one atom (1024 B) on
 #pragma unroll
-                        for (int k = 0; k < 8; ++k)
-                            tc_mma_ts(tmem + TM_O, pa + 8 * k, sw128_desc_ls(vb + k * 2048, UREG, 1024), idesc_pv,
-                                      (u > 1 || k > 0) ? 1u : 0u);
-                        tc_commit(&sm.empty[s]);
+                        for (int h = 0; h < 2; ++h)
+#pragma unroll
+                            for (int k = 0; k < 4; ++k)
+                                tc_mma_ts(tmem + TM_O + 128 * h, pa + 64 * h + 8 * k,
+                                          dv + (uint64_t)(((4 * h + k) * 2 * UBLK) >> 4), idesc_pv,
+                                          (u > 1 || k > 0) ? 1u : 0u);
+                        tc_commit(&sm.empty[ps]);
                         tc_commit(&sm.pv_done);
+                        if (++ps == UNS) ps = 0;
                     }
                 }
                 // the item's O is complete: one phase of o_full per item.  (The
@@ -378,77 +431,106 @@ __global__ void __launch_bounds__(UT_THREADS, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------------------ softmax / epilogue
+        // TMEM lane (row) = 64 hd + 8 query + q head: quarters 0-1 hold kv head 0 of the
+        // pair, quarters 2-3 kv head 1.  Warp (quarter, hf) owns S columns [64 hf, 64 hf + 64)
+        // (blocks 8 hf .. 8 hf + 7 of the key tile), their running maximum and sum, the
+        // accumulator O_hf, and writes Q dims [64 hf, 64 hf + 64) and output dims of the same range.
+        const int sw = warp - (UW_MMA + 1);
         const int quarter = warp & 3;
-        const int row = quarter * 32 + lane;          // TMEM lane: query row / 8, head row % 8
-        const int qi = row >> 3, hl = row & 7;
+        const int hf = sw >> 2;
+        const int row = quarter * 32 + lane;
+        const int hd = quarter >> 1;                    // kv head within the pair (warp-uniform)
+        const int qi = (row >> 3) & (UQ - 1);           // query of the tile
+        const int hq = row & (UG - 1);                  // q head within the kv head's group
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+        const uint32_t o_own = lane_base + TM_O + 128 * hf;
+        const uint32_t o_oth = lane_base + TM_O + 128 * (hf ^ 1);
+        uint8_t *qrow = sm.q + hf * UQH + (row >> 3) * 1024 + (row & 7) * 128;
         const float sl2 = p.scale_log2;
         int64_t c = 0, ic = 0;
+        int ms = 0;           // stage of the tile's meta
+        uint32_t mph = 0;     // its phase
         bool ok = true;
         for (int64_t i = blockIdx.x; i < p.items && ok; i += gridDim.x, ++ic) {
             const UtItem it = ut_item(p, i);
             const int ntile = (it.n_u + UB - 1) / UB;
             const int64_t tq = it.t0 + qi;
-            // Q tile: staging shared memory -> this row's 64 TMEM columns
-            ok = __all_sync(0xffffffffu, mbar_wait(&sm.q_full, (int)(ic & 1), p.status));
-            if (!ok) break;
+            const int head = UH * it.pair + UG * hd + hq;
+            // Q: this row's dims [64 hf, 64 hf + 64) -> shared memory, 128-byte swizzle (rows
+            // past the tile's queries hold zeros).  Every QK product of the previous item is
+            // complete: its O was read after its last product.
             {
-                uint32_t qv[64];
+                const bool qlive = qi < it.nrows;
+                const uint4 *src = reinterpret_cast<const uint4 *>(
+                    p.q + (((int64_t)it.seq * p.n_q + it.r0 + (qlive ? qi : 0)) * p.Hq + head) * UD + 64 * hf);
 #pragma unroll
-                for (int c8 = 0; c8 < 16; ++c8) {
-                    const int half = c8 >> 3, ch = c8 & 7;
-                    const uint4 v = *reinterpret_cast<const uint4 *>(sm.qs + half * UREG + row * 128 +
-                                                                     ((ch ^ (row & 7)) << 4));
-                    qv[4 * c8] = v.x;
-                    qv[4 * c8 + 1] = v.y;
-                    qv[4 * c8 + 2] = v.z;
-                    qv[4 * c8 + 3] = v.w;
+                for (int ch = 0; ch < 8; ++ch) {
+                    const uint4 v = qlive ? __ldg(src + ch) : make_uint4(0, 0, 0, 0);
+                    *reinterpret_cast<uint4 *>(qrow + ((ch ^ (row & 7)) << 4)) = v;
                 }
-                tmem_st32(lane_base + TM_Q, *reinterpret_cast<const uint32_t(*)[32]>(&qv[0]));
-                tmem_st32(lane_base + TM_Q + 32, *reinterpret_cast<const uint32_t(*)[32]>(&qv[32]));
-                tc_wait_st();
             }
-            tc_fence_before();
+            fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&sm.q_ready);
-                mbar_arrive(&sm.q_empty);
-            }
+            if (lane == 0) mbar_arrive(&sm.q_ready);
             float m_run = -INFINITY, l_run = 0.f;
             for (int u = 0; u < ntile; ++u, ++c) {
-                const int s = (int)(c % UNS);
+                const int s = ms;
+                const uint32_t sph = mph;
+                if (++ms == UNS) {
+                    ms = 0;
+                    mph ^= 1u;
+                }
                 bool w_ok = mbar_wait(&sm.s_full[c & 1], (int)((c >> 1) & 1), p.status);
-                if (w_ok) w_ok = mbar_wait(&sm.full[s], (int)((c / UNS) & 1), p.status);   // the tile's meta
+                if (w_ok) w_ok = mbar_wait(&sm.full[s], sph, p.status);   // the tile's meta
                 ok = __all_sync(0xffffffffu, w_ok);
                 if (!ok) break;
                 tc_fence_after();
                 const UtMeta &mt = sm.meta[s];
-                const uint32_t mw = mt.mw[qi];
-                const uint32_t wmask = __reduce_or_sync(0xffffffffu, mw);
+                const uint32_t mw = (mt.mw[qi] >> (8 * hf)) & 0xFFu;          // this half's 8 blocks
                 const bool diag = mt.diag != 0;
-                const uint32_t sa = lane_base + TM_S + (uint32_t)((c & 1) * 128);
-                uint32_t sv[128];
-#pragma unroll
-                for (int ch = 0; ch < 4; ++ch)
-                    tmem_ld32(sa + 32 * ch, *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * ch]));
+                const uint32_t sbuf = lane_base + TM_S + (uint32_t)((c & 1) * 128);
+                // S column 64 hf + 8 j + 4 h + tk: block 8 hf + j, kv head h of the pair, token tk;
+                // xs[4 j + tk] = this row's kv head hd
+                uint32_t sv[64], xs[32];
+                tmem_ld32(sbuf + 64 * hf, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+                tmem_ld32(sbuf + 64 * hf + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
                 tc_wait_ld();
-                // logits in log2 units; keys the query does not attend to -> -inf
-                float mx = -INFINITY;
 #pragma unroll
-                for (int j = 0; j < UB; ++j) {
-                    const bool on = (mw >> j) & 1u;
-                    int64_t kpos = 0;
-                    if (diag) kpos = (int64_t)kBlock * mt.id[j];
+                for (int j = 0; j < 8; ++j)
 #pragma unroll
-                    for (int tk = 0; tk < kBlock; ++tk) {
-                        const bool valid = on && (!diag || kpos + tk <= tq);
-                        const float x = valid ? __uint_as_float(sv[kBlock * j + tk]) * sl2 : -INFINITY;
-                        sv[kBlock * j + tk] = __float_as_uint(x);
-                        mx = fmaxf(mx, x);
+                    for (int tk = 0; tk < kBlock; ++tk) xs[4 * j + tk] = hd ? sv[8 * j + 4 + tk] : sv[8 * j + tk];
+                // the keys this row attends to: bit 4 j + tk of vm (the query's mask bit; at the
+                // diagonal also key position <= query position)
+                uint32_t vm = 0;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) vm |= ((mw >> j) & 1u) ? (0xFu << (4 * j)) : 0u;
+                if (diag) {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int64_t lim = tq - (int64_t)kBlock * mt.id[8 * hf + j];   // tokens tk <= lim
+                        const uint32_t tm = lim >= kBlock - 1 ? 0xFu : (lim < 0 ? 0u : ((2u << lim) - 1u));
+                        vm &= ~(0xFu << (4 * j)) | (tm << (4 * j));
                     }
                 }
-                const bool grow = mx > m_run + kRescale;       // also the first keys of the row
-                const bool resc = grow && m_run != -INFINITY;  // O and l already hold earlier keys
+                // pass 1: the row maximum.  The maximum over all of the half's scores bounds the one
+                // over the keys this row attends to; only when it could move the running maximum
+                // by more than the threshold is the exact (masked) maximum taken.  (sl2 > 0)
+                float m4[4] = {__uint_as_float(xs[0]), __uint_as_float(xs[1]), __uint_as_float(xs[2]),
+                               __uint_as_float(xs[3])};
+#pragma unroll
+                for (int e = 4; e < 32; ++e) m4[e & 3] = fmaxf(m4[e & 3], __uint_as_float(xs[e]));
+                float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
+                bool grow = false;
+                if (__any_sync(0xffffffffu, mx > m_run + kRescale)) {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) m4[k] = -INFINITY;
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        m4[e & 3] = fmaxf(m4[e & 3], ((vm >> e) & 1u) ? __uint_as_float(xs[e]) : -INFINITY);
+                    mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
+                    grow = mx > m_run + kRescale;               // also the first keys of the row
+                }
+                const bool resc = grow && m_run != -INFINITY;  // O_hf and l already hold earlier keys
                 if (__any_sync(0xffffffffu, resc)) {
                     // the previous P V must have landed before O is read.  A parity
                     // wait is exact here: S(c) landing means every MMA issued before
@@ -457,83 +539,107 @@ __global__ void __launch_bounds__(UT_THREADS, 1)
                     ok = __all_sync(0xffffffffu, mbar_wait(&sm.pv_done, (int)((c - 1) & 1), p.status));
                     if (!ok) break;
                     tc_fence_after();
-                    const float alpha = resc ? exp2f(m_run - mx) : 1.f;
-#pragma unroll
-                    for (int ch = 0; ch < 4; ++ch) {
-                        uint32_t ov[32];
-                        tmem_ld32(lane_base + TM_O + 32 * ch, ov);
+                    const float alpha = resc ? ex2_approx(m_run - mx) : 1.f;
+#pragma unroll 1
+                    for (int ch = 0; ch < 8; ++ch) {   // rare: kept rolled, so its loads do not crowd the registers
+                        uint32_t ov[16];
+                        tmem_ld16(o_own + 16 * ch, ov);
                         tc_wait_ld();
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-                        tmem_st32(lane_base + TM_O + 32 * ch, ov);
+                        for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+                        tmem_st16(o_own + 16 * ch, ov);
                     }
                     tc_wait_st();
                     l_run *= alpha;
                 }
                 if (grow) m_run = mx;
                 const float mneg = (m_run == -INFINITY) ? 0.f : -m_run;
-                uint32_t pk[64];
-                float ls = 0.f;
+                // pass 2: p for this row's keys (2^-inf = 0 for the others), P (bf16 pairs) over this
+                // half's S columns: word 64 hf + 4 j + 2 h + tk / 2 holds tokens tk, tk + 1 of kv head
+                // h of block j; the other kv head's words are zero
+                float pv[32];
+                float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int j = 0; j < UB; ++j) {
-                    if ((wmask >> j) & 1u) {   // some query of this warp attends to block j
-                        const float p0 = exp2f(__uint_as_float(sv[4 * j]) + mneg);
-                        const float p1 = exp2f(__uint_as_float(sv[4 * j + 1]) + mneg);
-                        const float p2 = exp2f(__uint_as_float(sv[4 * j + 2]) + mneg);
-                        const float p3 = exp2f(__uint_as_float(sv[4 * j + 3]) + mneg);
-                        ls += (p0 + p1) + (p2 + p3);
-                        pk[2 * j] = pack_bf16(p0, p1);
-                        pk[2 * j + 1] = pack_bf16(p2, p3);
-                    } else {
-                        pk[2 * j] = 0u;
-                        pk[2 * j + 1] = 0u;
-                    }
+                for (int e = 0; e < 32; ++e) {
+                    pv[e] = ex2_approx(((vm >> e) & 1u) ? fmaf(__uint_as_float(xs[e]), sl2, mneg) : -INFINITY);
+                    l4[e & 3] += pv[e];
                 }
+                uint32_t pk[32];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const uint32_t w0 = pack_bf16(pv[4 * j], pv[4 * j + 1]), w1 = pack_bf16(pv[4 * j + 2], pv[4 * j + 3]);
+                    pk[4 * j] = hd ? 0u : w0;
+                    pk[4 * j + 1] = hd ? 0u : w1;
+                    pk[4 * j + 2] = hd ? w0 : 0u;
+                    pk[4 * j + 3] = hd ? w1 : 0u;
+                }
+                const float ls = (l4[0] + l4[1]) + (l4[2] + l4[3]);
+                tmem_st32(sbuf + 64 * hf, pk);
                 l_run += ls;
-                tmem_st32(sa, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
-                tmem_st32(sa + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
                 tc_wait_st();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm.p_ready[c & 1]);
             }
             if (!ok) break;
-            // epilogue: O / l -> bf16 rows of the output; lse
+            // epilogue.  o_full: every product of the item is done, so both S buffers
+            // are free until the next item's Q is staged; the halves exchange (m, l)
+            // through columns [4 hf, 4 hf + 4) of S buffer 0.
             ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_full, (int)(ic & 1), p.status));
             if (!ok) break;
             tc_fence_after();
+            {
+                const uint32_t xv[4] = {__float_as_uint(m_run), __float_as_uint(l_run), 0u, 0u};
+                tmem_st4(lane_base + TM_S + 4 * hf, xv);
+                tc_wait_st();
+            }
+            tc_fence_before();
+            named_bar_sync(1, USW * 32);
+            tc_fence_after();
+            uint32_t yv[4];
+            tmem_ld4(lane_base + TM_S + 4 * (hf ^ 1), yv);
+            tc_wait_ld();
+            const float m_oth = __uint_as_float(yv[0]), l_oth = __uint_as_float(yv[1]);
+            const float m_all = fmaxf(m_run, m_oth);
+            const bool any = ntile > 0 && m_all != -INFINITY;
+            const float a_own = any ? ex2_approx(m_run - m_all) : 0.f;
+            const float a_oth = any ? ex2_approx(m_oth - m_all) : 0.f;
+            const float l_tot = a_own * l_run + a_oth * l_oth;
+            const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
+            const float c_own = a_own * inv, c_oth = a_oth * inv;
             const bool live = qi < it.nrows;
-            const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-            __nv_bfloat16 *dst = p.out + (((int64_t)it.seq * p.n_q + it.r0 + qi) * p.Hq + UG * it.g + hl) * UD;
+            __nv_bfloat16 *dst = p.out + (((int64_t)it.seq * p.n_q + it.r0 + qi) * p.Hq + head) * UD + 64 * hf;
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch) {
-                uint32_t ov[32];
-                tmem_ld32(lane_base + TM_O + 32 * ch, ov);
+                uint32_t o0[16], o1[16];
+                tmem_ld16(o_own + 64 * hf + 16 * ch, o0);
+                tmem_ld16(o_oth + 64 * hf + 16 * ch, o1);
                 tc_wait_ld();
-                if (ntile == 0)   // no position at all: the output is zero
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) ov[e] = 0u;
                 if (live) {
+                    uint32_t w[8];
 #pragma unroll
-                    for (int v4 = 0; v4 < 4; ++v4) {
-                        uint4 w;
-                        w.x = pack_bf16(__uint_as_float(ov[8 * v4]) * inv, __uint_as_float(ov[8 * v4 + 1]) * inv);
-                        w.y = pack_bf16(__uint_as_float(ov[8 * v4 + 2]) * inv, __uint_as_float(ov[8 * v4 + 3]) * inv);
-                        w.z = pack_bf16(__uint_as_float(ov[8 * v4 + 4]) * inv, __uint_as_float(ov[8 * v4 + 5]) * inv);
-                        w.w = pack_bf16(__uint_as_float(ov[8 * v4 + 6]) * inv, __uint_as_float(ov[8 * v4 + 7]) * inv);
-                        *reinterpret_cast<uint4 *>(dst + 32 * ch + 8 * v4) = w;
+                    for (int e = 0; e < 8; ++e) {
+                        // no position at all (ntile = 0): nothing was accumulated, the output is zero
+                        const float v0 = any ? __uint_as_float(o0[2 * e]) * c_own + __uint_as_float(o1[2 * e]) * c_oth
+                                             : 0.f;
+                        const float v1 = any ? __uint_as_float(o0[2 * e + 1]) * c_own +
+                                                   __uint_as_float(o1[2 * e + 1]) * c_oth
+                                             : 0.f;
+                        w[e] = pack_bf16(v0, v1);
                     }
+                    *reinterpret_cast<uint4 *>(dst + 16 * ch) = make_uint4(w[0], w[1], w[2], w[3]);
+                    *reinterpret_cast<uint4 *>(dst + 16 * ch + 8) = make_uint4(w[4], w[5], w[6], w[7]);
                 }
             }
-            if (live && p.lse)
-                p.lse[((int64_t)it.seq * p.n_q + it.r0 + qi) * p.Hq + UG * it.g + hl] =
-                    l_run > 0.f ? (m_run + log2f(l_run)) / kLog2e : -INFINITY;
+            if (live && hf == 0 && p.lse)
+                p.lse[((int64_t)it.seq * p.n_q + it.r0 + qi) * p.Hq + head] =
+                    l_tot > 0.f ? (m_all + log2f(l_tot)) / kLog2e : -INFINITY;
             tc_fence_before();
         }
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == UW_MMA) {
         tc_fence_after();
         tmem_dealloc(tmem, TM_COLS);
     }
@@ -579,7 +685,7 @@ UnionPlan union_plan(int B, int64_t n_q, int top_k) {
 }  // namespace
 
 bool attn_union_supported(const AttnArgs &a) {
-    return !a.decode && !a.kv8 && a.d == UD && a.Hq == UG * a.Hkv && !a.pg.table;
+    return !a.decode && !a.kv8 && a.d == UD && a.Hq == UG * a.Hkv && (a.Hkv == 2 || a.Hkv == 4) && !a.pg.table;
 }
 
 size_t attn_union_ws_bytes(int B, int64_t n_q, int top_k) {
@@ -606,25 +712,16 @@ cudaError_t launch_attn_union(const AttnArgs &a, void *ws, unsigned *status, cud
 
     auto enc = get_encode_fn();
     if (!enc) return cudaErrorInvalidValue;
-    // q: [B * n_q][Hq][128], box 64 dims x 8 heads x 16 queries
-    CUtensorMap mq, mk, mv;
-    {
-        cuuint64_t dims[3] = {UD, (cuuint64_t)a.Hq, (cuuint64_t)a.B * a.n_q};
-        cuuint64_t strides[2] = {UD * 2, (cuuint64_t)a.Hq * UD * 2};
-        cuuint32_t box[3] = {64, UG, UQ};
-        cuuint32_t estr[3] = {1, 1, 1};
-        if (enc(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(a.q), dims, strides, box, estr,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return cudaErrorInvalidValue;
-    }
-    // k, v: [B][kv_stride][Hkv][128], box 64 dims x 1 head x 4 tokens x 1 sequence
+    CUtensorMap mk, mv;
+    // k, v: [B][kv_stride][Hkv][128] seen as (64 dims, token, kv head, dim half, sequence); a box of
+    // 64 dims x 4 tokens x 2 heads x 2 halves x 1 sequence lands as [half][head][token][64 dims]
     for (int t = 0; t < 2; ++t) {
-        cuuint64_t dims[4] = {UD, (cuuint64_t)a.Hkv, (cuuint64_t)a.kv_stride, (cuuint64_t)a.B};
-        cuuint64_t strides[3] = {UD * 2, (cuuint64_t)a.Hkv * UD * 2, (cuuint64_t)a.kv_stride * a.Hkv * UD * 2};
-        cuuint32_t box[4] = {64, 1, kBlock, 1};
-        cuuint32_t estr[4] = {1, 1, 1, 1};
-        if (enc(t ? &mv : &mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(t ? a.v : a.k), dims, strides,
+        const cuuint64_t row = (cuuint64_t)a.Hkv * UD * 2;
+        cuuint64_t dims[5] = {64, (cuuint64_t)a.kv_stride, (cuuint64_t)a.Hkv, 2, (cuuint64_t)a.B};
+        cuuint64_t strides[4] = {row, UD * 2, 128, (cuuint64_t)a.kv_stride * row};
+        cuuint32_t box[5] = {64, kBlock, 2, 2, 1};
+        cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+        if (enc(t ? &mv : &mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(t ? a.v : a.k), dims, strides,
                 box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
@@ -642,6 +739,7 @@ cudaError_t launch_attn_union(const AttnArgs &a, void *ws, unsigned *status, cud
                        a.sel, a.nsel, a.n_q, a.q0, a.top_k, r, r + rows, n_qt, u.cap, u_count, u_id, u_mask, status);
         if (e != cudaSuccess) return e;
         UtParams p{};
+        p.q = static_cast<const __nv_bfloat16 *>(a.q);
         p.B = a.B;
         p.n_q = a.n_q;
         p.q0 = a.q0;
@@ -658,9 +756,9 @@ cudaError_t launch_attn_union(const AttnArgs &a, void *ws, unsigned *status, cud
         p.out = static_cast<__nv_bfloat16 *>(a.out);
         p.lse = a.lse;
         p.status = status;
-        p.items = (int64_t)a.B * n_qt * a.Hkv;
+        p.items = (int64_t)a.B * n_qt * (a.Hkv / 2);
         const int64_t grid = std::min<int64_t>(p.items, sms);
-        e = launch_pdl(attn_union_kernel, dim3((unsigned)grid), dim3(UT_THREADS), smem, s, mq, mk, mv, p);
+        e = launch_pdl(attn_union_kernel, dim3((unsigned)grid), dim3(UT_THREADS), smem, s, mk, mv, p);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;

@@ -290,15 +290,16 @@ QSA_API int qsa_index_topk_decode(const void *q_idx, const void *k_pool, const f
  * workspace: device, 256-byte aligned, at least qsa_sparse_attn_prefill_workspace()
  *          bytes, caller-owned and needing no initialisation; 0 bytes (pass
  *          NULL) for the shapes that run without one.  QSA_BF16 with d = 128,
- *          Hq = 8 Hkv runs on the tensor cores over tiles of 16 consecutive
- *          query rows: a pre-pass merges the tile's 16 selections and tail
- *          blocks into one ascending block list (with a per-block mask of the
- *          queries attending to it) in the workspace, so each listed block's
- *          K/V is gathered once per tile and kv head; masked keys contribute
- *          exactly zero.  The workspace is capped near 512 MiB: longer
- *          prompts run as several launches of whole query tiles.  Results of a
- *          chunk starting at a row that is a multiple of 16 equal those of the
- *          same rows in one call bit for bit.  Too small: QSA_ERR_WORKSPACE.
+ *          Hq = 8 Hkv and Hkv = 2 or 4 runs on the tensor cores over tiles of
+ *          8 consecutive query rows: a pre-pass merges the tile's 8 selections
+ *          and tail blocks into one ascending block list (with a per-block
+ *          mask of the queries attending to it) in the workspace, so each
+ *          listed block's K/V (a pair of kv heads) is gathered once per tile;
+ *          masked keys contribute exactly zero.  The workspace is capped near
+ *          512 MiB: longer prompts run as several launches of whole query
+ *          tiles.  Results of a chunk starting at a row that is a multiple of
+ *          8 equal those of the same rows in one call bit for bit.  Too
+ *          small: QSA_ERR_WORKSPACE.
  */
 /* Kernels one qsa_sparse_attn_prefill call with these sizes launches: 1 (the
  * gather kernels: fp32, d = 256, other GQA ratios) or 2 per launch of query

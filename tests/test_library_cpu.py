@@ -150,18 +150,20 @@ def test_binding_constants_match_the_header(qsa):
 
 
 def test_prefill_attention_workspace_sizes(qsa):
-    """The tensor-core prefill (BF16, d = 128, 8 q heads per kv head) keeps
-    the merged block lists of its 16-query tiles in the workspace: 16 * (top_k
-    + 1) entries of 6 bytes per tile, capped near 512 MiB (longer prompts run
-    as several launches); the other shapes need none."""
+    """The tensor-core prefill (BF16, d = 128, 8 q heads per kv head, an even
+    number of kv heads) keeps the merged block lists of its 8-query tiles in
+    the workspace: 8 * (top_k + 1) entries of 6 bytes per tile (rounded to a
+    key tile of 16), capped near 512 MiB (longer prompts run as several
+    launches); the other shapes need none."""
     ws = qsa.qsa_sparse_attn_prefill_workspace
-    cap = (16 * 513 + 31) // 32 * 32
-    tiles = 131072 // 16
+    cap = (8 * 513 + 15) // 16 * 16
+    tiles = 131072 // 8
     r256 = lambda x: (x + 255) // 256 * 256
     assert ws(1, 131072, 512, 16, 2, 128, qsa.QSA_BF16) == r256(tiles * 4) + r256(tiles * cap * 4) + r256(tiles * cap * 2)
     assert ws(1, 1, 512, 16, 2, 128, qsa.QSA_BF16) > 0
     assert 0 < ws(1, 1 << 20, 2048, 16, 2, 128, qsa.QSA_BF16) <= (512 << 20) + 4096
     assert ws(1, 4096, 512, 24, 2, 256, qsa.QSA_BF16) == 0      # released shape: the gather kernel
+    assert ws(1, 4096, 512, 8, 1, 128, qsa.QSA_BF16) == 0       # one kv head: the gather kernel
     assert ws(1, 4096, 512, 8, 1, 128, qsa.QSA_FP32) == 0       # fp32: the SIMT kernel
     assert ws(0, 4096, 512, 16, 2, 128, qsa.QSA_BF16) == 0      # invalid
 
@@ -174,4 +176,5 @@ def test_prefill_kernel_counts(qsa):
     assert qsa.qsa_index_topk_prefill_kernels(1, 32768, 0, 0, qsa.QSA_BF16) == 1 + 2 * 1
     assert qsa.qsa_sparse_attn_prefill_kernels(1, 131072, 512, 16, 2, 128, qsa.QSA_BF16) == 2
     assert qsa.qsa_sparse_attn_prefill_kernels(1, 131072, 512, 24, 2, 256, qsa.QSA_BF16) == 1
+    assert qsa.qsa_sparse_attn_prefill_kernels(1, 131072, 512, 8, 1, 128, qsa.QSA_BF16) == 1
     assert qsa.qsa_sparse_attn_prefill_kernels(1, 1 << 20, 2048, 16, 2, 128, qsa.QSA_BF16) > 2
