@@ -118,6 +118,7 @@ struct AttnParams {
     unsigned *status;
     float k_scale, v_scale;  // KV8: K = k_scale * stored E4M3 value, V = v_scale * stored value
     Paging pg;               // pg.table: K/V are paged caches [slots][Hkv][D] (kv_stride = table capacity)
+    int no_tail;             // prefill: no tail entries (the listed blocks only)
 };
 
 // The key list of one work item: positions lbeg..lend of
@@ -169,7 +170,7 @@ __device__ __forceinline__ Item get_item(const AttnParams &p, int64_t i) {
         }
     }
     it.nb = (t_sel + 1) / kBlock;
-    it.tail = (int)(it.t + 1 - kBlock * it.nb);
+    it.tail = p.no_tail ? 0 : (int)(it.t + 1 - kBlock * it.nb);
     it.nsel = p.dense ? (int)it.nb : max(0, min(it.nsel, p.top_k));
     const int len = it.nsel + (it.tail + kBlock - 1) / kBlock;
     if (!p.decode) {
@@ -433,6 +434,19 @@ __global__ void __launch_bounds__(AttnCfg<HKV, KV8, D, G>::kThreads, AttnCfg<HKV
             }
             sl2 = p.scale_log2 * p.k_scale * ldexpf(1.0f, -qexp);
         }
+        // The query buffer is refilled by a bulk copy (async proxy) once every
+        // consumer has released it.  Its fragments must have arrived in
+        // registers first: plain shared loads may still be in flight at the
+        // release, and nothing reads them until the first key stage.  Reading
+        // every fragment here waits for the loads; the proxy fence orders these
+        // reads before the copy's writes.
+        {
+            uint32_t all = 0;
+#pragma unroll
+            for (int kk = 0; kk < kMT; ++kk) all ^= qf[kk][0] ^ qf[kk][1];
+            asm volatile("" ::"r"(all));
+        }
+        fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.qempty[qs]);
         float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
@@ -572,6 +586,7 @@ __global__ void __launch_bounds__(AttnCfg<HKV, KV8, D, G>::kThreads, AttnCfg<HKV
                     }
                 }
             }
+            fence_proxy_async_smem();   // this stage's shared reads before the next bulk copies into it
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.empty[s]);
         }
@@ -917,6 +932,7 @@ cudaError_t run_bf16(const AttnArgs &a, void *ws, unsigned *status, cudaStream_t
     p.pg = a.pg;
     p.k_scale = a.k_scale;
     p.v_scale = a.v_scale;
+    p.no_tail = (!a.decode && a.no_tail) ? 1 : 0;
     // entries of one item's list: top_k blocks + the tail blocks (dense: every block of the cache)
     const int list_max = p.dense ? (int)(a.kv_stride / kBlock + 1)
                                  : a.top_k + attn_tail_blocks(a.decode && a.cap_len, a.max_draft);
