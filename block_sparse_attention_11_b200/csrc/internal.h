@@ -145,17 +145,21 @@ struct AttnArgs {
     Paging pg;                          // pg.table: paged K/V caches (bf16 kernels), kv_stride = its capacity
     bool kv8 = false;                   // K/V caches of FP8 E4M3 (bf16 q/out): K = k_scale * k8, V = v_scale * v8
     float k_scale = 1.f, v_scale = 1.f;
+    bool no_tail = false;               // prefill: the rows attend to their listed blocks only (the split prefill
+                                        // gives each query's tail to the tile kernel)
 };
 int attn_tail_blocks(bool indexshare, int max_draft);
 size_t attn_decode_ws_bytes(int B, int Hq, int d, int top_k, int tail_blocks = 1);
 size_t attn_dense_decode_ws_bytes(int B, int Hq, int d, int64_t kv_stride);
 cudaError_t launch_attn_bf16(const AttnArgs &a, void *ws, unsigned *status, cudaStream_t s);
-// Prefill on the tensor cores over tiles of 16 queries (k_attn_tc.cu): BF16,
-// d = 128, 8 q heads per kv head, contiguous BF16 K/V.  Its workspace holds
-// the merged block lists of the query tiles.
+// Prefill split by sharing (k_attn_tc.cu): BF16, d = 128, 8 q heads per kv
+// head, contiguous BF16 K/V.  Blocks that several queries of a tile of 8
+// attend to run on the tensor cores once per tile; the rest run in the gather
+// kernel (launch_attn_bf16) per query; the tile kernel merges the two.  Its
+// workspace holds the block lists, the per-query lists and their lse.
 bool attn_union_supported(const AttnArgs &a);
-size_t attn_union_ws_bytes(int B, int64_t n_q, int top_k);
-int attn_union_launches(int B, int64_t n_q, int top_k);   // launches of query tiles per call
+size_t attn_union_ws_bytes(int B, int64_t n_q, int top_k, int Hq);
+int attn_union_launches(int B, int64_t n_q, int top_k, int Hq);   // chunks per call (3 kernels each)
 cudaError_t launch_attn_union(const AttnArgs &a, void *ws, unsigned *status, cudaStream_t s);
 cudaError_t launch_attn_f32(const AttnArgs &a, unsigned *status, cudaStream_t s);
 

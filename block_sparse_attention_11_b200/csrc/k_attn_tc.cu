@@ -71,6 +71,10 @@ constexpr int UBPW = (UB + UPW - 1) / UPW;   // blocks per producer warp per til
 #endif
 constexpr int UNS = QSA_UT_STAGES;     // key tiles in flight
 constexpr int UPRE = 4;                // key tiles whose block ids the producers hold ahead
+#ifndef QSA_UT_SHARE
+#define QSA_UT_SHARE 2
+#endif
+constexpr int kShare = QSA_UT_SHARE;   // queries of a tile that must attend to a block for the tile list
 constexpr int UW_MMA = UPW;            // warp index of the MMA issuer
 constexpr int USW = 8;                 // softmax warps: two per TMEM lane quarter, one per column half
 constexpr int UT_THREADS = (UPW + 1 + USW) * 32;
@@ -116,7 +120,8 @@ struct UtParams {
     const uint32_t *u_id;    // [B][n_qt][cap]
     const uint16_t *u_mask;  // [B][n_qt][cap]
     float scale_log2;
-    __nv_bfloat16 *out;
+    __nv_bfloat16 *out;      // in: the gather kernel's result over each query's own blocks; out: the total
+    const float *lse_q;      // [B][n_q][Hq] its log-sum-exp (natural log)
     float *lse;
     unsigned *status;
     int64_t items;
@@ -148,92 +153,139 @@ __device__ __forceinline__ UtItem ut_item(const UtParams &p, int64_t i) {
 }
 
 // ---------------------------------------------------------------- pre-pass
-// One CTA per (query tile, sequence).  Block ids of the tile's selections
-// (validated: 0 <= b < nb(t)) and each query's tail block (when it holds 1-3
-// tokens) set bit q in a mask word per id; the non-zero words are compacted
-// in id order.  Ids are processed UCHUNK at a time.
+// One CTA per query tile of a one-sequence view.  Block ids of the tile's
+// selections (validated: 0 <= b < nb(t)) and each query's tail block (when it
+// holds 1-3 tokens) set bit q in a mask word per id.  Ids are processed
+// UCHUNK at a time, in id order; each non-zero word goes
+//   * to the tile's block list (id, mask) when at least kShare queries of the
+//     tile attend to it, or it is some query's tail block (the tile kernel
+//     masks the tail's later positions): its K/V is gathered once for all;
+//   * otherwise to the own list of its one query (sel1 [rows][top_k],
+//     ascending ids, counts in nsel1), which the per-query gather kernel
+//     attends to (full blocks only).
+// Thread tid owns words [tid W, tid W + W) of a chunk, so block-wide
+// exclusive scans of its counts give every destination position.
+__device__ __forceinline__ int block_exclusive_scan(int v, int *s_w, int &total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) s_w[warp] = incl;
+    __syncthreads();
+    int before = 0;
+    total = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+        before += (w < warp) ? s_w[w] : 0;
+        total += s_w[w];
+    }
+    __syncthreads();
+    return before + incl - v;
+}
+
 __global__ void __launch_bounds__(256) union_build_kernel(const int32_t *__restrict__ sel,
                                                           const int32_t *__restrict__ nsel, int64_t n_q, int64_t q0,
-                                                          int top_k, int64_t row0, int64_t row_end, int64_t n_qt,
-                                                          int cap, int32_t *__restrict__ u_count,
-                                                          uint32_t *__restrict__ u_id, uint16_t *__restrict__ u_mask,
-                                                          unsigned *status) {
+                                                          int top_k, int64_t n_qt, int cap,
+                                                          int32_t *__restrict__ u_count, uint32_t *__restrict__ u_id,
+                                                          uint16_t *__restrict__ u_mask, int32_t *__restrict__ sel1,
+                                                          int32_t *__restrict__ nsel1, unsigned *status) {
     extern __shared__ uint32_t ub_bits[];
     __shared__ int s_nsel[UQ];
-    __shared__ int s_wsum[8];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int seq = blockIdx.y;
+    __shared__ int64_t s_tail[UQ];   // the query's tail block, or -1
+    __shared__ int s_w[8];
+    const int tid = threadIdx.x;
     const int64_t qt = blockIdx.x;
-    const int64_t r0 = row0 + qt * UQ;
-    const int nrows = (int)(row_end - r0 < UQ ? row_end - r0 : UQ);
+    const int64_t r0 = qt * UQ;
+    const int nrows = (int)(n_q - r0 < UQ ? n_q - r0 : UQ);
     pdl_wait();       // the selection comes from the previous kernel
     pdl_trigger();
-    if (tid < UQ) s_nsel[tid] = tid < nrows ? max(0, min(nsel[(int64_t)seq * n_q + r0 + tid], top_k)) : 0;
+    if (tid < UQ) {
+        s_nsel[tid] = tid < nrows ? max(0, min(nsel[r0 + tid], top_k)) : 0;
+        const int64_t t = q0 + r0 + tid;
+        s_tail[tid] = (tid < nrows && (t + 1) % kBlock != 0) ? (t + 1) / kBlock : -1;
+    }
     __syncthreads();
     const int64_t t_last = q0 + r0 + nrows - 1;
     const int64_t id_end = t_last / kBlock + 1;            // the last query's tail block, exclusive
-    const int64_t ti = (int64_t)seq * n_qt + qt;
-    uint32_t *oid = u_id + ti * cap;
-    uint16_t *om = u_mask + ti * cap;
+    uint32_t *oid = u_id + qt * cap;
+    uint16_t *om = u_mask + qt * cap;
     int count = 0;
+    int qcount[UQ];
+#pragma unroll
+    for (int q = 0; q < UQ; ++q) qcount[q] = 0;
     for (int64_t c0 = 0; c0 < id_end; c0 += UCHUNK) {
         const int span = (int)(id_end - c0 < UCHUNK ? id_end - c0 : UCHUNK);
         for (int i = tid; i < span; i += 256) ub_bits[i] = 0;
         __syncthreads();
-        for (int e = tid; e < UQ * top_k; e += 256) {
-            const int q = e / top_k, k = e - q * top_k;
+        for (int i = tid; i < nrows * top_k; i += 256) {
+            const int q = i / top_k, k = i % top_k;
             if (k >= s_nsel[q]) continue;
             const int64_t t = q0 + r0 + q;
-            const int32_t b = sel[((int64_t)seq * n_q + r0 + q) * top_k + k];
+            const int32_t b = sel[(r0 + q) * top_k + k];
             if (b < 0 || (int64_t)b >= (t + 1) / kBlock) {
                 if (c0 == 0) flag(status, QSA_DEV_BAD_INDEX);
                 continue;
             }
             if (b >= c0 && b < c0 + span) atomicOr(&ub_bits[b - c0], 1u << q);
         }
-        if (tid < nrows) {
-            const int64_t t = q0 + r0 + tid;
-            const int64_t nb = (t + 1) / kBlock;
-            if (t + 1 > kBlock * nb && nb >= c0 && nb < c0 + span) atomicOr(&ub_bits[nb - c0], 1u << tid);
-        }
+        if (tid < UQ && s_tail[tid] >= c0 && s_tail[tid] < c0 + span) atomicOr(&ub_bits[s_tail[tid] - c0], 1u << tid);
         __syncthreads();
-        // compaction in id order: thread tid owns words [tid * W, tid * W + W)
         const int W = (span + 255) / 256;
-        int mine = 0;
+        int mine = 0, qm[UQ];
+#pragma unroll
+        for (int q = 0; q < UQ; ++q) qm[q] = 0;
+        auto listed = [&](uint32_t m, int64_t id) {
+            bool tl = false;
+#pragma unroll
+            for (int q = 0; q < UQ; ++q) tl |= s_tail[q] == id;
+            return m != 0u && (__popc(m) >= kShare || tl);
+        };
         for (int i = 0; i < W; ++i) {
             const int w = tid * W + i;
-            if (w < span && ub_bits[w]) ++mine;
-        }
-        int incl = mine;
+            const uint32_t m = w < span ? ub_bits[w] : 0u;
+            if (listed(m, c0 + w)) ++mine;
+            else if (m)
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += v;
+                for (int q = 0; q < UQ; ++q) qm[q] += (m >> q) & 1u;
         }
-        if (lane == 31) s_wsum[warp] = incl;
-        __syncthreads();
-        int before = 0, total = 0;
+        int total;
+        int pos = count + block_exclusive_scan(mine, s_w, total);
+        count += total;
+        int qpos[UQ];
 #pragma unroll
-        for (int w = 0; w < 8; ++w) {
-            before += (w < warp) ? s_wsum[w] : 0;
-            total += s_wsum[w];
+        for (int q = 0; q < UQ; ++q) {
+            int tq;
+            qpos[q] = qcount[q] + block_exclusive_scan(qm[q], s_w, tq);
+            qcount[q] += tq;
         }
-        int pos = count + before + incl - mine;
         for (int i = 0; i < W; ++i) {
             const int w = tid * W + i;
-            if (w < span) {
-                const uint32_t m = ub_bits[w];
-                if (m && pos < cap) {
+            if (w >= span) break;
+            const uint32_t m = ub_bits[w];
+            if (listed(m, c0 + w)) {
+                if (pos < cap) {
                     oid[pos] = (uint32_t)(c0 + w);
                     om[pos] = (uint16_t)m;
-                    ++pos;
                 }
+                ++pos;
+            } else if (m) {
+#pragma unroll
+                for (int q = 0; q < UQ; ++q)
+                    if ((m >> q) & 1u) {
+                        if (qpos[q] < top_k) sel1[(r0 + q) * top_k + qpos[q]] = (int32_t)(c0 + w);
+                        ++qpos[q];
+                    }
             }
         }
-        count += total;
         __syncthreads();
     }
-    if (tid == 0) u_count[ti] = min(count, cap);
+    if (tid == 0) u_count[qt] = min(count, cap);
+#pragma unroll
+    for (int q = 0; q < UQ; ++q)
+        if (tid == q && q < nrows) nsel1[r0 + q] = min(qcount[q], top_k);
 }
 
 // ---------------------------------------------------------------- attention
@@ -600,40 +652,51 @@ __global__ void __launch_bounds__(UT_THREADS, 1)
             tmem_ld4(lane_base + TM_S + 4 * (hf ^ 1), yv);
             tc_wait_ld();
             const float m_oth = __uint_as_float(yv[0]), l_oth = __uint_as_float(yv[1]);
-            const float m_all = fmaxf(m_run, m_oth);
-            const bool any = ntile > 0 && m_all != -INFINITY;
-            const float a_own = any ? ex2_approx(m_run - m_all) : 0.f;
-            const float a_oth = any ? ex2_approx(m_oth - m_all) : 0.f;
-            const float l_tot = a_own * l_run + a_oth * l_oth;
-            const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
-            const float c_own = a_own * inv, c_oth = a_oth * inv;
+            // merge three partial softmaxes of the row: the two column halves of the listed
+            // blocks, and the gather kernel's (its own blocks and tail; out_q normalised, so its
+            // weight is 2^lse_q)
             const bool live = qi < it.nrows;
-            __nv_bfloat16 *dst = p.out + (((int64_t)it.seq * p.n_q + it.r0 + qi) * p.Hq + head) * UD + 64 * hf;
+            const int64_t orow = ((int64_t)it.seq * p.n_q + it.r0 + qi) * p.Hq + head;
+            const float lq = live ? p.lse_q[orow] * kLog2e : -INFINITY;
+            const bool tile = ntile > 0;
+            const float m_all = fmaxf(tile ? fmaxf(m_run, m_oth) : -INFINITY, lq);
+            const bool any = m_all != -INFINITY;
+            const float a_own = (any && tile) ? ex2_approx(m_run - m_all) : 0.f;
+            const float a_oth = (any && tile) ? ex2_approx(m_oth - m_all) : 0.f;
+            const float a_q = any ? ex2_approx(lq - m_all) : 0.f;
+            const float l_tot = a_own * l_run + a_oth * l_oth + a_q;
+            const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
+            const float c_own = a_own * inv, c_oth = a_oth * inv, c_q = a_q * inv;
+            __nv_bfloat16 *dst = p.out + orow * UD + 64 * hf;
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch) {
                 uint32_t o0[16], o1[16];
                 tmem_ld16(o_own + 64 * hf + 16 * ch, o0);
                 tmem_ld16(o_oth + 64 * hf + 16 * ch, o1);
+                uint4 q4[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+                if (live) {
+                    q4[0] = *reinterpret_cast<const uint4 *>(dst + 16 * ch);
+                    q4[1] = *reinterpret_cast<const uint4 *>(dst + 16 * ch + 8);
+                }
                 tc_wait_ld();
                 if (live) {
+                    const uint32_t *qw = reinterpret_cast<const uint32_t *>(q4);
                     uint32_t w[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        // no position at all (ntile = 0): nothing was accumulated, the output is zero
-                        const float v0 = any ? __uint_as_float(o0[2 * e]) * c_own + __uint_as_float(o1[2 * e]) * c_oth
-                                             : 0.f;
-                        const float v1 = any ? __uint_as_float(o0[2 * e + 1]) * c_own +
-                                                   __uint_as_float(o1[2 * e + 1]) * c_oth
-                                             : 0.f;
-                        w[e] = pack_bf16(v0, v1);
+                        // nothing was accumulated without a listed block: TMEM holds no values then
+                        const float x0 = tile ? __uint_as_float(o0[2 * e]) * c_own + __uint_as_float(o1[2 * e]) * c_oth : 0.f;
+                        const float x1 = tile ? __uint_as_float(o0[2 * e + 1]) * c_own +
+                                                    __uint_as_float(o1[2 * e + 1]) * c_oth
+                                              : 0.f;
+                        const float y0 = __uint_as_float(qw[e] << 16), y1 = __uint_as_float(qw[e] & 0xFFFF0000u);
+                        w[e] = pack_bf16(fmaf(y0, c_q, x0), fmaf(y1, c_q, x1));
                     }
                     *reinterpret_cast<uint4 *>(dst + 16 * ch) = make_uint4(w[0], w[1], w[2], w[3]);
                     *reinterpret_cast<uint4 *>(dst + 16 * ch + 8) = make_uint4(w[4], w[5], w[6], w[7]);
                 }
             }
-            if (live && hf == 0 && p.lse)
-                p.lse[((int64_t)it.seq * p.n_q + it.r0 + qi) * p.Hq + head] =
-                    l_tot > 0.f ? (m_all + log2f(l_tot)) / kLog2e : -INFINITY;
+            if (live && hf == 0 && p.lse) p.lse[orow] = l_tot > 0.f ? (m_all + log2f(l_tot)) / kLog2e : -INFINITY;
             tc_fence_before();
         }
     }
@@ -658,27 +721,32 @@ EncodeTiledFn get_encode_fn() {
     return fn;
 }
 
-// Rows of one launch and the list capacity of a query tile.
+// Rows of one chunk and the layout of its workspace.
 struct UnionPlan {
     int cap;             // list entries per query tile
-    int64_t rows;        // query rows per launch (a multiple of UQ)
-    size_t count_bytes, id_bytes, mask_bytes;
+    int64_t rows;        // query rows per chunk (a multiple of UQ)
+    size_t count_bytes, id_bytes, mask_bytes, sel1_bytes, nsel1_bytes, lse_bytes;
+    size_t total() const { return count_bytes + id_bytes + mask_bytes + sel1_bytes + nsel1_bytes + lse_bytes; }
 };
 
-constexpr size_t kUnionBudget = (size_t)512 << 20;   // workspace cap; longer prompts run in several launches
+constexpr size_t kUnionBudget = (size_t)1 << 30;   // workspace cap; longer prompts run in several chunks
 
-UnionPlan union_plan(int B, int64_t n_q, int top_k) {
+UnionPlan union_plan(int64_t n_q, int top_k, int Hq) {
     UnionPlan u{};
-    u.cap = (UQ * (top_k + 1) + UB - 1) / UB * UB;
-    const size_t per_tile = (size_t)u.cap * 6 + 4;
-    const int64_t want_tiles = (n_q + UQ - 1) / UQ;
-    const int64_t max_tiles = std::max<int64_t>(1, (int64_t)(kUnionBudget / (per_tile * std::max(B, 1))));
-    const int64_t tiles = std::max<int64_t>(1, std::min(want_tiles, max_tiles));
-    u.rows = tiles * UQ;
+    // each listed block holds >= kShare of the 8 x top_k selections, or is one of the <= 3 tail blocks
+    u.cap = (UQ * top_k / kShare + 3 + UB) / UB * UB;
+    const size_t per_row = (size_t)u.cap * 6 / UQ + 4 + (size_t)top_k * 4 + 4 + (size_t)Hq * 4;
+    const int64_t want = (n_q + UQ - 1) / UQ * UQ;
+    const int64_t fit = std::max<int64_t>(UQ, (int64_t)(kUnionBudget / per_row) / UQ * UQ);
+    u.rows = std::min(want, fit);
+    const int64_t tiles = u.rows / UQ;
     auto r256 = [](size_t x) { return (x + 255) / 256 * 256; };
-    u.count_bytes = r256((size_t)B * tiles * 4);
-    u.id_bytes = r256((size_t)B * tiles * u.cap * 4);
-    u.mask_bytes = r256((size_t)B * tiles * u.cap * 2);
+    u.count_bytes = r256((size_t)tiles * 4);
+    u.id_bytes = r256((size_t)tiles * u.cap * 4);
+    u.mask_bytes = r256((size_t)tiles * u.cap * 2);
+    u.sel1_bytes = r256((size_t)u.rows * top_k * 4);
+    u.nsel1_bytes = r256((size_t)u.rows * 4);
+    u.lse_bytes = r256((size_t)u.rows * Hq * 4);
     return u;
 }
 
@@ -688,78 +756,115 @@ bool attn_union_supported(const AttnArgs &a) {
     return !a.decode && !a.kv8 && a.d == UD && a.Hq == UG * a.Hkv && (a.Hkv == 2 || a.Hkv == 4) && !a.pg.table;
 }
 
-size_t attn_union_ws_bytes(int B, int64_t n_q, int top_k) {
+size_t attn_union_ws_bytes(int B, int64_t n_q, int top_k, int Hq) {
     if (B < 1 || n_q < 1) return 0;
-    const UnionPlan u = union_plan(B, n_q, top_k);
-    return u.count_bytes + u.id_bytes + u.mask_bytes;
+    return union_plan(n_q, top_k, Hq).total();
 }
 
-int attn_union_launches(int B, int64_t n_q, int top_k) {
+int attn_union_launches(int B, int64_t n_q, int top_k, int Hq) {
     if (B < 1 || n_q < 1) return 0;
-    const UnionPlan u = union_plan(B, n_q, top_k);
-    return (int)((n_q + u.rows - 1) / u.rows);
+    const UnionPlan u = union_plan(n_q, top_k, Hq);
+    return B * (int)((n_q + u.rows - 1) / u.rows);
 }
 
 cudaError_t launch_attn_union(const AttnArgs &a, void *ws, unsigned *status, cudaStream_t s) {
     if (a.n_q <= 0) return cudaSuccess;
     const DeviceInfo *di = device_info();
     const int sms = di ? di->sm_count : 148;
-    const UnionPlan u = union_plan(a.B, a.n_q, a.top_k);
+    const UnionPlan u = union_plan(a.n_q, a.top_k, a.Hq);
     uint8_t *w = static_cast<uint8_t *>(ws);
     int32_t *u_count = reinterpret_cast<int32_t *>(w);
-    uint32_t *u_id = reinterpret_cast<uint32_t *>(w + u.count_bytes);
-    uint16_t *u_mask = reinterpret_cast<uint16_t *>(w + u.count_bytes + u.id_bytes);
+    w += u.count_bytes;
+    uint32_t *u_id = reinterpret_cast<uint32_t *>(w);
+    w += u.id_bytes;
+    uint16_t *u_mask = reinterpret_cast<uint16_t *>(w);
+    w += u.mask_bytes;
+    int32_t *sel1 = reinterpret_cast<int32_t *>(w);
+    w += u.sel1_bytes;
+    int32_t *nsel1 = reinterpret_cast<int32_t *>(w);
+    w += u.nsel1_bytes;
+    float *lse_q = reinterpret_cast<float *>(w);
 
     auto enc = get_encode_fn();
     if (!enc) return cudaErrorInvalidValue;
-    CUtensorMap mk, mv;
-    // k, v: [B][kv_stride][Hkv][128] seen as (64 dims, token, kv head, dim half, sequence); a box of
-    // 64 dims x 4 tokens x 2 heads x 2 halves x 1 sequence lands as [half][head][token][64 dims]
-    for (int t = 0; t < 2; ++t) {
-        const cuuint64_t row = (cuuint64_t)a.Hkv * UD * 2;
-        cuuint64_t dims[5] = {64, (cuuint64_t)a.kv_stride, (cuuint64_t)a.Hkv, 2, (cuuint64_t)a.B};
-        cuuint64_t strides[4] = {row, UD * 2, 128, (cuuint64_t)a.kv_stride * row};
-        cuuint32_t box[5] = {64, kBlock, 2, 2, 1};
-        cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-        if (enc(t ? &mv : &mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(t ? a.v : a.k), dims, strides,
-                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return cudaErrorInvalidValue;
-    }
     const size_t smem = sizeof(UtSmem) + 1024;
     if (di && smem > di->smem_optin) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(attn_union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(union_build_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, UCHUNK * 4);
     if (e != cudaSuccess) return e;
-    for (int64_t r = 0; r < a.n_q; r += u.rows) {
-        const int64_t rows = std::min(u.rows, a.n_q - r);
-        const int64_t n_qt = (rows + UQ - 1) / UQ;
-        e = launch_pdl(union_build_kernel, dim3((unsigned)n_qt, (unsigned)a.B), dim3(256), (size_t)UCHUNK * 4, s,
-                       a.sel, a.nsel, a.n_q, a.q0, a.top_k, r, r + rows, n_qt, u.cap, u_count, u_id, u_mask, status);
-        if (e != cudaSuccess) return e;
-        UtParams p{};
-        p.q = static_cast<const __nv_bfloat16 *>(a.q);
-        p.B = a.B;
-        p.n_q = a.n_q;
-        p.q0 = a.q0;
-        p.Hq = a.Hq;
-        p.Hkv = a.Hkv;
-        p.row0 = r;
-        p.row_end = r + rows;
-        p.n_qt = n_qt;
-        p.cap = u.cap;
-        p.u_count = u_count;
-        p.u_id = u_id;
-        p.u_mask = u_mask;
-        p.scale_log2 = a.scale * kLog2e;
-        p.out = static_cast<__nv_bfloat16 *>(a.out);
-        p.lse = a.lse;
-        p.status = status;
-        p.items = (int64_t)a.B * n_qt * (a.Hkv / 2);
-        const int64_t grid = std::min<int64_t>(p.items, sms);
-        e = launch_pdl(attn_union_kernel, dim3((unsigned)grid), dim3(UT_THREADS), smem, s, mk, mv, p);
-        if (e != cudaSuccess) return e;
+    const size_t qrow = (size_t)a.Hq * UD;                 // elements of one query row of q / out
+    const size_t kvseq = (size_t)a.kv_stride * a.Hkv * UD;  // elements of one sequence's cache
+    for (int b = 0; b < a.B; ++b) {
+        CUtensorMap mk, mv;
+        // the sequence's k, v: [kv_stride][Hkv][128] seen as (64 dims, token, kv head, dim half); a box of
+        // 64 dims x 4 tokens x 2 heads x 2 halves lands as [half][head][token][64 dims]
+        for (int t = 0; t < 2; ++t) {
+            const cuuint64_t row = (cuuint64_t)a.Hkv * UD * 2;
+            cuuint64_t dims[5] = {64, (cuuint64_t)a.kv_stride, (cuuint64_t)a.Hkv, 2, 1};
+            cuuint64_t strides[4] = {row, UD * 2, 128, (cuuint64_t)a.kv_stride * row};
+            cuuint32_t box[5] = {64, kBlock, 2, 2, 1};
+            cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+            const __nv_bfloat16 *base = static_cast<const __nv_bfloat16 *>(t ? a.v : a.k) + (size_t)b * kvseq;
+            if (enc(t ? &mv : &mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<__nv_bfloat16 *>(base), dims,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+                return cudaErrorInvalidValue;
+        }
+        for (int64_t r = 0; r < a.n_q; r += u.rows) {
+            // rows [r, r + rows) of sequence b as a one-sequence problem
+            const int64_t rows = std::min(u.rows, a.n_q - r);
+            const int64_t n_qt = (rows + UQ - 1) / UQ;
+            const int64_t row_g = (int64_t)b * a.n_q + r;       // first row in the [B][n_q] layouts
+            const int32_t *sel_c = a.sel + row_g * a.top_k;
+            const int32_t *nsel_c = a.nsel + row_g;
+            const __nv_bfloat16 *q_c = static_cast<const __nv_bfloat16 *>(a.q) + row_g * qrow;
+            __nv_bfloat16 *out_c = static_cast<__nv_bfloat16 *>(a.out) + row_g * qrow;
+            // 1. block lists of the shared blocks, own lists of the others
+            e = launch_pdl(union_build_kernel, dim3((unsigned)n_qt), dim3(256), (size_t)UCHUNK * 4, s, sel_c,
+                           nsel_c, rows, a.q0 + r, a.top_k, n_qt, u.cap, u_count, u_id, u_mask, sel1, nsel1,
+                           status);
+            if (e != cudaSuccess) return e;
+            // 2. each query over its own blocks and its tail (gather kernel): out, lse_q
+            AttnArgs g = a;
+            g.q = q_c;
+            g.k = static_cast<const __nv_bfloat16 *>(a.k) + (size_t)b * kvseq;
+            g.v = static_cast<const __nv_bfloat16 *>(a.v) + (size_t)b * kvseq;
+            g.sel = sel1;
+            g.nsel = nsel1;
+            g.B = 1;
+            g.n_q = rows;
+            g.q0 = a.q0 + r;
+            g.out = out_c;
+            g.lse = lse_q;
+            g.no_tail = true;
+            e = launch_attn_bf16(g, nullptr, status, s);
+            if (e != cudaSuccess) return e;
+            // 3. the tiles over their shared blocks, merged with step 2
+            UtParams p{};
+            p.q = q_c;
+            p.B = 1;
+            p.n_q = rows;
+            p.q0 = a.q0 + r;
+            p.Hq = a.Hq;
+            p.Hkv = a.Hkv;
+            p.row0 = 0;
+            p.row_end = rows;
+            p.n_qt = n_qt;
+            p.cap = u.cap;
+            p.u_count = u_count;
+            p.u_id = u_id;
+            p.u_mask = u_mask;
+            p.scale_log2 = a.scale * kLog2e;
+            p.out = out_c;
+            p.lse_q = lse_q;
+            p.lse = a.lse ? a.lse + row_g * a.Hq : nullptr;
+            p.status = status;
+            p.items = n_qt * (a.Hkv / 2);
+            const int64_t grid = std::min<int64_t>(p.items, sms);
+            e = launch_pdl(attn_union_kernel, dim3((unsigned)grid), dim3(UT_THREADS), smem, s, mk, mv, p);
+            if (e != cudaSuccess) return e;
+        }
     }
     return cudaSuccess;
 }

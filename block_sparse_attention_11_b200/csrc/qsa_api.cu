@@ -325,7 +325,7 @@ size_t qsa_sparse_attn_prefill_workspace(int32_t B, int64_t n_q, int32_t top_k, 
     a.Hkv = Hkv;
     a.d = d;
     if (dtype != QSA_BF16 || !attn_union_supported(a)) return 0;
-    return attn_union_ws_bytes(B, n_q, top_k);
+    return attn_union_ws_bytes(B, n_q, top_k, Hq);
 }
 
 int qsa_sparse_attn_prefill_kernels(int32_t B, int64_t n_q, int32_t top_k, int32_t Hq, int32_t Hkv, int32_t d,
@@ -336,7 +336,7 @@ int qsa_sparse_attn_prefill_kernels(int32_t B, int64_t n_q, int32_t top_k, int32
     a.Hkv = Hkv;
     a.d = d;
     if (dtype != QSA_BF16 || !attn_union_supported(a)) return 1;
-    return 2 * attn_union_launches(B, n_q, top_k);   // per launch of query tiles: block lists, attention
+    return 3 * attn_union_launches(B, n_q, top_k, Hq);   // per chunk: block lists, gather kernel, tiles
 }
 
 int qsa_sparse_attn_prefill(const void *q, const void *k, const void *v, const int32_t *sel, const int32_t *nsel,
@@ -353,7 +353,7 @@ int qsa_sparse_attn_prefill(const void *q, const void *k, const void *v, const i
     AttnArgs a{q, k, v, sel, nsel, nullptr, B, n_q, q0, kv_stride, Hq, Hkv, d, top_k, scale, out, lse, false};
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (dtype == QSA_BF16 && attn_union_supported(a)) {
-        const size_t need = attn_union_ws_bytes(B, n_q, top_k);
+        const size_t need = attn_union_ws_bytes(B, n_q, top_k, Hq);
         if (!workspace || ws_bytes < need) return QSA_ERR_WORKSPACE;
         if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return QSA_ERR_INVALID_ARG;
         return cuda_status(launch_attn_union(a, workspace, di->status, s));

@@ -150,18 +150,24 @@ def test_binding_constants_match_the_header(qsa):
 
 
 def test_prefill_attention_workspace_sizes(qsa):
-    """The tensor-core prefill (BF16, d = 128, 8 q heads per kv head, an even
-    number of kv heads) keeps the merged block lists of its 8-query tiles in
-    the workspace: 8 * (top_k + 1) entries of 6 bytes per tile (rounded to a
-    key tile of 16), capped near 512 MiB (longer prompts run as several
-    launches); the other shapes need none."""
+    """The split prefill (BF16, d = 128, 8 q heads per kv head, 2 or 4 kv
+    heads) keeps in the workspace, per chunk of rows: the lists of blocks
+    shared within each 8-query tile (8 * top_k / 2 entries of 6 bytes, rounded
+    up to a key tile of 16; each listed block holds at least 2 of the tile's
+    selections), every query's own list (top_k ids and a count) and the lse of
+    the gather kernel's part (Hq floats a row); chunks are capped near 1 GiB;
+    the other shapes need none."""
     ws = qsa.qsa_sparse_attn_prefill_workspace
-    cap = (8 * 513 + 15) // 16 * 16
-    tiles = 131072 // 8
+    cap = (8 * 512 // 2 + 3 + 16) // 16 * 16
+    rows = 131072
+    tiles = rows // 8
     r256 = lambda x: (x + 255) // 256 * 256
-    assert ws(1, 131072, 512, 16, 2, 128, qsa.QSA_BF16) == r256(tiles * 4) + r256(tiles * cap * 4) + r256(tiles * cap * 2)
+    assert ws(1, rows, 512, 16, 2, 128, qsa.QSA_BF16) == (
+        r256(tiles * 4) + r256(tiles * cap * 4) + r256(tiles * cap * 2) + r256(rows * 512 * 4) + r256(rows * 4)
+        + r256(rows * 16 * 4))
     assert ws(1, 1, 512, 16, 2, 128, qsa.QSA_BF16) > 0
-    assert 0 < ws(1, 1 << 20, 2048, 16, 2, 128, qsa.QSA_BF16) <= (512 << 20) + 4096
+    assert 0 < ws(1, 1 << 20, 2048, 16, 2, 128, qsa.QSA_BF16) <= (1 << 30) + 8192
+    assert ws(4, 4096, 512, 16, 2, 128, qsa.QSA_BF16) == ws(1, 4096, 512, 16, 2, 128, qsa.QSA_BF16)  # per sequence
     assert ws(1, 4096, 512, 24, 2, 256, qsa.QSA_BF16) == 0      # released shape: the gather kernel
     assert ws(1, 4096, 512, 8, 1, 128, qsa.QSA_BF16) == 0       # one kv head: the gather kernel
     assert ws(1, 4096, 512, 8, 1, 128, qsa.QSA_FP32) == 0       # fp32: the SIMT kernel
@@ -171,10 +177,12 @@ def test_prefill_attention_workspace_sizes(qsa):
 def test_prefill_kernel_counts(qsa):
     """Launch counts the benchmark reports: the indexer at 128K runs its score
     kernel and row select in 8 chunks of 16384 rows (scores under 2 GiB); the
-    tensor-core attention is one block-list pre-pass and one attention launch."""
+    split attention runs three kernels per sequence and chunk of rows (lists,
+    gather kernel, tiles)."""
     assert qsa.qsa_index_topk_prefill_kernels(1, 131072, 0, 0, qsa.QSA_BF16) == 1 + 2 * 8
     assert qsa.qsa_index_topk_prefill_kernels(1, 32768, 0, 0, qsa.QSA_BF16) == 1 + 2 * 1
-    assert qsa.qsa_sparse_attn_prefill_kernels(1, 131072, 512, 16, 2, 128, qsa.QSA_BF16) == 2
+    assert qsa.qsa_sparse_attn_prefill_kernels(1, 131072, 512, 16, 2, 128, qsa.QSA_BF16) == 3
+    assert qsa.qsa_sparse_attn_prefill_kernels(2, 4096, 512, 16, 2, 128, qsa.QSA_BF16) == 6
     assert qsa.qsa_sparse_attn_prefill_kernels(1, 131072, 512, 24, 2, 256, qsa.QSA_BF16) == 1
     assert qsa.qsa_sparse_attn_prefill_kernels(1, 131072, 512, 8, 1, 128, qsa.QSA_BF16) == 1
-    assert qsa.qsa_sparse_attn_prefill_kernels(1, 1 << 20, 2048, 16, 2, 128, qsa.QSA_BF16) > 2
+    assert qsa.qsa_sparse_attn_prefill_kernels(1, 1 << 20, 2048, 16, 2, 128, qsa.QSA_BF16) > 3
