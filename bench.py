@@ -52,7 +52,7 @@ CSRC = os.path.join(ROOT, "block_sparse_attention_11_b200", "csrc")
 # ncu summary holding the DRAM traffic of each roofline kernel, and the sources it was built from
 _DECODE_SRC = ["k_decode_index.cu", "select.cuh", "common.cuh", "internal.h"]
 TRAFFIC_PROFILE = {
-    "prefill": [("attn_bf16_prefill_t32k.md", ["k_attn.cu", "common.cuh", "internal.h"])],
+    "prefill": [("attn_split_prefill_t128k.md", ["k_attn_tc.cu", "k_attn.cu", "common.cuh", "internal.h"])],
     "decode": [("decode_indexer_b64_l128k.md", _DECODE_SRC), ("decode_indexer_b64_l128k_fp8keys.md", _DECODE_SRC)],
 }
 
@@ -90,28 +90,6 @@ def profiled_traffic(kind, workload):
         except (KeyError, ValueError, OSError):
             return None
     return None
-
-
-def measure_l2_read(dev, reps=40):
-    """L2 read bandwidth (GB/s) measured here with CUDA events: a float32
-    buffer far smaller than L2 (48 MiB of the 126 MB) is read repeatedly by a
-    sum reduction after one warm-up pass, so every read after the first is
-    served by L2; the best of three sizes' rates is reported."""
-    best = 0.0
-    for mib in (24, 48, 64):
-        x = torch.ones(mib * (1 << 20) // 4, dtype=torch.float32, device=dev)
-        for _ in range(3):
-            x.sum()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(reps):
-            x.sum()
-        e1.record()
-        torch.cuda.synchronize()
-        best = max(best, x.numel() * 4 * reps / (e0.elapsed_time(e1) / 1e3) / 1e9)
-        del x
-    return best
 
 
 def peaks():
@@ -846,17 +824,9 @@ def run_ours(args, rank, world):
                                unit="TFLOP/s", frac=attn_tf / peak_tf,
                                traffic=profiled_traffic("prefill", w.name), peak_kind=pk_kind + " (sustained bf16)",
                                note="algorithmic flops = 4*d*Hq per selected position (4*nsel + tail per query) "
-                                    "over the attention stage's CUDA-event time; the bf16 sustained peak (a step "
-                                    "of tens of ms)")
-        l2 = measure_l2_read(torch.device("cuda", torch.cuda.current_device()))
-        gb = alg["attn_bytes"] / (attn_ms / 1e3) / 1e9
-        res["l2_roofline"] = dict(kernel="sparse_attn_prefill", achieved=gb, peak=l2, unit="GB/s", frac=gb / l2,
-                                  peak_kind="L2 read rate measured in this run (sum over a 24-64 MiB L2-resident "
-                                            "buffer, CUDA events)",
-                                  note="algorithmic bytes = the K/V rows each query attends to (4*nsel+tail "
-                                       "positions x Hkv x d x 2 B x 2) + q read + out write, as if every query "
-                                       "gathered its own; a kernel that shares a gathered block between the "
-                                       "queries selecting it moves fewer bytes than this")
+                                    "over the attention stage's CUDA-event time (its three kernels: block lists, "
+                                    "gather kernel, tensor-core tiles); the bf16 sustained peak (a step of tens "
+                                    "of ms)")
         flops = alg["attn_flops"] + alg["idx_flops"]
         tf = flops / (ms_per_step / 1e3) / 1e12
         res["tensor_roofline"] = dict(achieved=tf, peak=pk["bf16_tflops"], unit="TFLOP/s",
@@ -870,11 +840,15 @@ def run_ours(args, rank, world):
         el = 2 if w.dtype == "bf16" else 4
         pool_b = w.B * w.T * 128 * el * 1.25
         idx_b = w.B * w.T * (4 * 128 * el + w.top_k * 4 + 4) + w.B * (w.T // 4) * 128 * el
+        # the attention must read each K/V row of the sequence once from HBM (repeat gathers of a
+        # block by other queries can be served by L2 or shared within a tile), plus q, out and sel
+        attn_unique_b = w.B * w.T * (w.Hkv * w.d * el * 2 + 2 * w.Hq * w.d * 2 + w.top_k * 4)
         t_bound = (pool_b / hbm + max(alg["idx_flops"] / tens, idx_b / hbm)
-                   + max(alg["attn_flops"] / tens, alg["attn_bytes"] / hbm))
+                   + max(alg["attn_flops"] / tens, attn_unique_b / hbm))
         res["bound_aware"] = dict(bound_ms=t_bound * 1e3, frac=t_bound * 1e3 / ms_per_step,
-                                  note="sum over pool, indexer, attention of max(flops / bf16 peak, algorithmic "
-                                       "bytes / HBM peak), over the measured step time")
+                                  note="sum over pool, indexer, attention of max(flops / bf16 peak, bytes that "
+                                       "must cross HBM / HBM peak), over the measured step time; the attention's "
+                                       "HBM bytes are its unique inputs and outputs (each K/V row once)")
         res["config"] = dict(workload=w.name, B=w.B, T=w.T, top_k=w.top_k, Hq=w.Hq, Hkv=w.Hkv, d=w.d,
                              needles=w.needles, chunk=w.extra.get("chunk"),
                              l2="flushed between timed steps (256 MB write)",

@@ -82,7 +82,7 @@ constexpr int UQH = UM * 128;          // Q in shared memory: one 64-dim half of
 constexpr uint32_t TM_S = 0;           // S / P, two buffers of 128 columns
 constexpr uint32_t TM_O = 256;         // O_0, O_1: 128 columns each
 constexpr uint32_t TM_COLS = 512;
-constexpr int UCHUNK = 16384;          // pre-pass: block ids per pass (one 32-bit mask word each)
+constexpr int UCHUNK = 32768;          // pre-pass: block ids per pass (a one-byte query mask each: 32 KB)
 constexpr float kLog2e = 1.4426950408889634f;
 #ifndef QSA_UT_RESCALE
 #define QSA_UT_RESCALE 64.f
@@ -155,35 +155,49 @@ __device__ __forceinline__ UtItem ut_item(const UtParams &p, int64_t i) {
 // ---------------------------------------------------------------- pre-pass
 // One CTA per query tile of a one-sequence view.  Block ids of the tile's
 // selections (validated: 0 <= b < nb(t)) and each query's tail block (when it
-// holds 1-3 tokens) set bit q in a mask word per id.  Ids are processed
-// UCHUNK at a time, in id order; each non-zero word goes
+// holds 1-3 tokens) set bit q of a one-byte mask per id (four ids to a 32-bit
+// word).  Ids are processed UCHUNK at a time, in id order; each non-zero mask
+// goes
 //   * to the tile's block list (id, mask) when at least kShare queries of the
 //     tile attend to it, or it is some query's tail block (the tile kernel
 //     masks the tail's later positions): its K/V is gathered once for all;
 //   * otherwise to the own list of its one query (sel1 [rows][top_k],
 //     ascending ids, counts in nsel1), which the per-query gather kernel
 //     attends to (full blocks only).
-// Thread tid owns words [tid W, tid W + W) of a chunk, so block-wide
-// exclusive scans of its counts give every destination position.
-__device__ __forceinline__ int block_exclusive_scan(int v, int *s_w, int &total) {
+// Thread tid owns words [tid W, tid W + W) of a chunk; one block-wide
+// exclusive scan of its nine counts (list entries, and own-list entries per
+// query) gives every destination position.
+constexpr int kScanN = UQ + 1;
+
+__device__ __forceinline__ void block_exclusive_scan9(int (&v)[kScanN], int (*s_w)[8], int (&total)[kScanN]) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int incl = v;
+    int incl[kScanN];
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-    }
-    if (lane == 31) s_w[warp] = incl;
-    __syncthreads();
-    int before = 0;
-    total = 0;
+    for (int j = 0; j < kScanN; ++j) incl[j] = v[j];
 #pragma unroll
-    for (int w = 0; w < 8; ++w) {
-        before += (w < warp) ? s_w[w] : 0;
-        total += s_w[w];
+    for (int o = 1; o < 32; o <<= 1)
+#pragma unroll
+        for (int j = 0; j < kScanN; ++j) {
+            const int y = __shfl_up_sync(0xffffffffu, incl[j], o);
+            if (lane >= o) incl[j] += y;
+        }
+    if (lane == 31)
+#pragma unroll
+        for (int j = 0; j < kScanN; ++j) s_w[j][warp] = incl[j];
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < kScanN; ++j) {
+        int before = 0, tot = 0;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+            const int x = s_w[j][w];
+            before += (w < warp) ? x : 0;
+            tot += x;
+        }
+        total[j] = tot;
+        v[j] = before + incl[j] - v[j];
     }
     __syncthreads();
-    return before + incl - v;
 }
 
 __global__ void __launch_bounds__(256) union_build_kernel(const int32_t *__restrict__ sel,
@@ -192,10 +206,10 @@ __global__ void __launch_bounds__(256) union_build_kernel(const int32_t *__restr
                                                           int32_t *__restrict__ u_count, uint32_t *__restrict__ u_id,
                                                           uint16_t *__restrict__ u_mask, int32_t *__restrict__ sel1,
                                                           int32_t *__restrict__ nsel1, unsigned *status) {
-    extern __shared__ uint32_t ub_bits[];
+    extern __shared__ uint32_t ub_words[];   // UCHUNK / 4 words: byte j of word w = mask of id 4 w + j
     __shared__ int s_nsel[UQ];
-    __shared__ int64_t s_tail[UQ];   // the query's tail block, or -1
-    __shared__ int s_w[8];
+    __shared__ int64_t s_tail[UQ];           // the query's tail block, or -1
+    __shared__ int s_w[kScanN][8];
     const int tid = threadIdx.x;
     const int64_t qt = blockIdx.x;
     const int64_t r0 = qt * UQ;
@@ -210,6 +224,14 @@ __global__ void __launch_bounds__(256) union_build_kernel(const int32_t *__restr
     __syncthreads();
     const int64_t t_last = q0 + r0 + nrows - 1;
     const int64_t id_end = t_last / kBlock + 1;            // the last query's tail block, exclusive
+    // the tile's tail blocks are consecutive: [tail_lo, tail_hi]
+    int64_t tail_lo = INT64_MAX, tail_hi = -1;
+#pragma unroll
+    for (int q = 0; q < UQ; ++q)
+        if (s_tail[q] >= 0) {
+            tail_lo = min(tail_lo, s_tail[q]);
+            tail_hi = max(tail_hi, s_tail[q]);
+        }
     uint32_t *oid = u_id + qt * cap;
     uint16_t *om = u_mask + qt * cap;
     int count = 0;
@@ -218,66 +240,83 @@ __global__ void __launch_bounds__(256) union_build_kernel(const int32_t *__restr
     for (int q = 0; q < UQ; ++q) qcount[q] = 0;
     for (int64_t c0 = 0; c0 < id_end; c0 += UCHUNK) {
         const int span = (int)(id_end - c0 < UCHUNK ? id_end - c0 : UCHUNK);
-        for (int i = tid; i < span; i += 256) ub_bits[i] = 0;
+        const int nw = (span + 3) / 4;
+        for (int i = tid; i < nw; i += 256) ub_words[i] = 0;
         __syncthreads();
-        for (int i = tid; i < nrows * top_k; i += 256) {
-            const int q = i / top_k, k = i % top_k;
-            if (k >= s_nsel[q]) continue;
+        for (int q = 0; q < nrows; ++q) {
             const int64_t t = q0 + r0 + q;
-            const int32_t b = sel[(r0 + q) * top_k + k];
-            if (b < 0 || (int64_t)b >= (t + 1) / kBlock) {
-                if (c0 == 0) flag(status, QSA_DEV_BAD_INDEX);
-                continue;
+            const int32_t *row = sel + (r0 + q) * top_k;
+            for (int k = tid; k < s_nsel[q]; k += 256) {
+                const int32_t b = row[k];
+                if (b < 0 || (int64_t)b >= (t + 1) / kBlock) {
+                    if (c0 == 0) flag(status, QSA_DEV_BAD_INDEX);
+                    continue;
+                }
+                if (b >= c0 && b < c0 + span) {
+                    const int rel = (int)(b - c0);
+                    atomicOr(&ub_words[rel >> 2], 1u << (8 * (rel & 3) + q));
+                }
             }
-            if (b >= c0 && b < c0 + span) atomicOr(&ub_bits[b - c0], 1u << q);
         }
-        if (tid < UQ && s_tail[tid] >= c0 && s_tail[tid] < c0 + span) atomicOr(&ub_bits[s_tail[tid] - c0], 1u << tid);
+        if (tid < UQ && s_tail[tid] >= c0 && s_tail[tid] < c0 + span) {
+            const int rel = (int)(s_tail[tid] - c0);
+            atomicOr(&ub_words[rel >> 2], 1u << (8 * (rel & 3) + tid));
+        }
         __syncthreads();
-        const int W = (span + 255) / 256;
-        int mine = 0, qm[UQ];
-#pragma unroll
-        for (int q = 0; q < UQ; ++q) qm[q] = 0;
+        const int W = (nw + 255) / 256;
         auto listed = [&](uint32_t m, int64_t id) {
-            bool tl = false;
-#pragma unroll
-            for (int q = 0; q < UQ; ++q) tl |= s_tail[q] == id;
-            return m != 0u && (__popc(m) >= kShare || tl);
+            return __popc(m) >= kShare || (id >= tail_lo && id <= tail_hi);
         };
+        int cnt[kScanN];
+#pragma unroll
+        for (int j = 0; j < kScanN; ++j) cnt[j] = 0;
         for (int i = 0; i < W; ++i) {
             const int w = tid * W + i;
-            const uint32_t m = w < span ? ub_bits[w] : 0u;
-            if (listed(m, c0 + w)) ++mine;
-            else if (m)
+            const uint32_t word = w < nw ? ub_words[w] : 0u;
+            if (!word) continue;
 #pragma unroll
-                for (int q = 0; q < UQ; ++q) qm[q] += (m >> q) & 1u;
+            for (int j = 0; j < 4; ++j) {
+                const uint32_t m = (word >> (8 * j)) & 0xFFu;
+                if (!m) continue;
+                if (listed(m, c0 + 4 * w + j)) ++cnt[UQ];
+                else
+#pragma unroll
+                    for (int q = 0; q < UQ; ++q) cnt[q] += (m >> q) & 1u;
+            }
         }
-        int total;
-        int pos = count + block_exclusive_scan(mine, s_w, total);
-        count += total;
+        int total[kScanN];
+        block_exclusive_scan9(cnt, s_w, total);   // cnt: this thread's first positions
+        int pos = count + cnt[UQ];
+        count += total[UQ];
         int qpos[UQ];
 #pragma unroll
         for (int q = 0; q < UQ; ++q) {
-            int tq;
-            qpos[q] = qcount[q] + block_exclusive_scan(qm[q], s_w, tq);
-            qcount[q] += tq;
+            qpos[q] = qcount[q] + cnt[q];
+            qcount[q] += total[q];
         }
         for (int i = 0; i < W; ++i) {
             const int w = tid * W + i;
-            if (w >= span) break;
-            const uint32_t m = ub_bits[w];
-            if (listed(m, c0 + w)) {
-                if (pos < cap) {
-                    oid[pos] = (uint32_t)(c0 + w);
-                    om[pos] = (uint16_t)m;
-                }
-                ++pos;
-            } else if (m) {
+            const uint32_t word = w < nw ? ub_words[w] : 0u;
+            if (!word) continue;
 #pragma unroll
-                for (int q = 0; q < UQ; ++q)
-                    if ((m >> q) & 1u) {
-                        if (qpos[q] < top_k) sel1[(r0 + q) * top_k + qpos[q]] = (int32_t)(c0 + w);
-                        ++qpos[q];
+            for (int j = 0; j < 4; ++j) {
+                const uint32_t m = (word >> (8 * j)) & 0xFFu;
+                if (!m) continue;
+                const int64_t id = c0 + 4 * w + j;
+                if (listed(m, id)) {
+                    if (pos < cap) {
+                        oid[pos] = (uint32_t)id;
+                        om[pos] = (uint16_t)m;
                     }
+                    ++pos;
+                } else {
+#pragma unroll
+                    for (int q = 0; q < UQ; ++q)
+                        if ((m >> q) & 1u) {
+                            if (qpos[q] < top_k) sel1[(r0 + q) * top_k + qpos[q]] = (int32_t)id;
+                            ++qpos[q];
+                        }
+                }
             }
         }
         __syncthreads();
@@ -791,7 +830,7 @@ cudaError_t launch_attn_union(const AttnArgs &a, void *ws, unsigned *status, cud
     if (di && smem > di->smem_optin) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(attn_union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(union_build_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, UCHUNK * 4);
+    e = cudaFuncSetAttribute(union_build_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, UCHUNK);
     if (e != cudaSuccess) return e;
     const size_t qrow = (size_t)a.Hq * UD;                 // elements of one query row of q / out
     const size_t kvseq = (size_t)a.kv_stride * a.Hkv * UD;  // elements of one sequence's cache
@@ -821,7 +860,7 @@ cudaError_t launch_attn_union(const AttnArgs &a, void *ws, unsigned *status, cud
             const __nv_bfloat16 *q_c = static_cast<const __nv_bfloat16 *>(a.q) + row_g * qrow;
             __nv_bfloat16 *out_c = static_cast<__nv_bfloat16 *>(a.out) + row_g * qrow;
             // 1. block lists of the shared blocks, own lists of the others
-            e = launch_pdl(union_build_kernel, dim3((unsigned)n_qt), dim3(256), (size_t)UCHUNK * 4, s, sel_c,
+            e = launch_pdl(union_build_kernel, dim3((unsigned)n_qt), dim3(256), (size_t)UCHUNK, s, sel_c,
                            nsel_c, rows, a.q0 + r, a.top_k, n_qt, u.cap, u_count, u_id, u_mask, sel1, nsel1,
                            status);
             if (e != cudaSuccess) return e;
