@@ -104,6 +104,7 @@ struct ScoreGemmArgs {
     int relu;
     const float *head_w;  // [B][n_q][4] or null
     float *scores;        // [B][row_count][ld]
+    uint16_t *keys = nullptr;   // BF16 modes: [B][row_count][ld] 16-bit order keys, written instead of scores
 };
 cudaError_t launch_score_gemm(const ScoreGemmArgs &a, const void *qa0, const void *qa1, const void *k_pool,
                               unsigned *status, cudaStream_t s);
@@ -112,6 +113,13 @@ cudaError_t launch_score_simt_f32(const ScoreGemmArgs &a, const float *q_hat, co
 cudaError_t launch_select_rows(const float *scores, int B, int64_t row_begin, int64_t row_count, int64_t n_q,
                                int64_t q0, int64_t ld, int top_k, int32_t *sel, int32_t *nsel,
                                unsigned *status, cudaStream_t s);
+// Row top-k over 16-bit keys (BF16 modes): keys that tie with the threshold at
+// 16 bits are re-scored in fp32 from the query operand (qa0/qa1 as the
+// rotation wrote them: mode 0 hi/lo planes, mode 1 per-head) and k_pool.
+cudaError_t launch_select_keys(const uint16_t *keys, int B, int64_t row_begin, int64_t row_count, int64_t n_q,
+                               int64_t q0, int64_t ld, int top_k, int mode, int relu, const void *qa0, const void *qa1,
+                               const void *k_pool, int64_t pool_stride, const float *head_w, int32_t *sel,
+                               int32_t *nsel, cudaStream_t s);
 
 // ---- decode indexer (k_decode_index.cu)
 struct DecodePlan {

@@ -61,6 +61,7 @@ struct GemmParams {
     unsigned *status;
     int nsplit;           // CTAs per row tile, each over `span` key tiles
     int span;
+    uint16_t *keys;       // non-null: write the 16-bit order key of each score (ld per row) instead of scores
 };
 
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
@@ -189,6 +190,34 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                         x += __shfl_xor_sync(0xffffffffu, x, 2);
                         v[i] = x;
                     }
+                }
+                if (p.keys) {
+                    // the top 16 bits of the order key (sign, exponent, 7 mantissa bits): the
+                    // selection ranks by them and re-scores the keys that tie at 16 bits
+                    uint16_t(*t16)[40] = reinterpret_cast<uint16_t(*)[40]>(&sm.epi[quarter][0][0]);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        uint32_t w4[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            w4[e] = (score_key(v[8 * i + 2 * e]) >> 16) | (score_key(v[8 * i + 2 * e + 1]) & 0xFFFF0000u);
+                        *reinterpret_cast<uint4 *>(&t16[lane][8 * i]) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                    }
+                    __syncwarp();
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int rr = 8 * i + (lane >> 2);
+                        const int lr = quarter * 32 + rr;
+                        const int64_t q = p.per_head ? r0 + lr / kIdxHeads : r0 + lr;
+                        const bool writer = q < r_end && (!p.per_head || (lr % kIdxHeads) == 0);
+                        if (writer) {
+                            uint16_t *d = p.keys + ((int64_t)seq * p.row_count + (q - p.row_begin)) * p.ld +
+                                          (int64_t)(j0 + j) * GN + c * 32 + 8 * (lane & 3);
+                            *reinterpret_cast<uint4 *>(d) = *reinterpret_cast<const uint4 *>(&t16[rr][8 * (lane & 3)]);
+                        }
+                    }
+                    __syncwarp();
+                    continue;
                 }
                 // stage the 32 x 32 block in smem and store it row-contiguously
                 float(*tile)[36] = sm.epi[quarter];
@@ -492,6 +521,385 @@ __global__ void __launch_bounds__(SR_THREADS)
     if (tid == 0) *cnt_out = k;
 }
 
+// ---- rows of 16-bit keys (BF16 modes): one CTA per row
+//
+// The score GEMM stores the top 16 bits of each score's order key.  Ranking
+// by them is exact except among the keys equal to the threshold key; those
+// are re-scored in fp32 from the query operand and the compressed keys:
+//   pass 1  histogram of the key's high byte; the bin d1 holding the k-th
+//           largest key, and k1, the picks it supplies;
+//   pass 2  histogram of the low byte within bin d1: the threshold key
+//           T = (d1, d2) and k2, the picks among the keys equal to T;
+//   pass 3  ids of keys > T (exactly k - k2) and of keys == T, each list in
+//           ascending id order (per 2048-element tile a block scan orders
+//           the writes);
+//   rank    the keys == T are re-scored; the k2 best (score descending, id
+//           ascending: the ranking's tie rule) join the picks;
+//   merge   both ascending lists merge into the row's ascending selection.
+// More than SK_AMB_CAP keys equal to T (massive ties) take an exact radix
+// select over the re-scored 32-bit keys of those entries instead.  A row is
+// 2 bytes per visible block, so the CTAs resident at once hold a few tens of
+// MB of rows: passes 2 and 3 read L2.
+constexpr int SK_THREADS = 256;
+constexpr int SK_TILE = SK_THREADS * 8;    // elements per tile: one 16-byte load per thread
+constexpr int SK_AMB_CAP = 2048;
+
+struct KeySelSmem {
+    uint32_t h1[256], h2[256];
+    uint32_t sure[2048];                  // ids with key > T, ascending
+    uint32_t amb[SK_AMB_CAP];             // ids with key == T, ascending
+    float amb_s[SK_AMB_CAP];              // their re-scored values
+    uint32_t chosen[2048];                // the picked ids among them, ascending (also rank scratch)
+    float q[kIdxHeads * kIdxDim];         // the row's query operand in fp32 (mode 0: the head sum)
+    float w[kIdxHeads];
+    int wsum[2][SK_THREADS / 32];
+    uint32_t d1, k1, d2, k2, n_amb, prefix, need;
+};
+
+struct KeySelParams {
+    const uint16_t *keys;
+    int64_t row_begin, row_count, n_q, q0, ld, pool_stride;
+    int top_k, mode, relu;
+    const __nv_bfloat16 *qa0, *qa1;      // mode 0: hi, lo planes [B][n_q][128]; mode 1: [B][n_q][4][128]
+    const __nv_bfloat16 *k_pool;         // [B][pool_stride][128]
+    const float *head_w;                 // [B][n_q][4] or null
+    int32_t *sel, *nsel;
+};
+
+// The k-th largest of 256 bins counted from the top: bin d and the number of
+// picks it supplies (k minus the count above it).  Warp 0; lane l owns bins
+// 255 - 8 l .. 248 - 8 l.
+__device__ __forceinline__ void sk_find_bin(const uint32_t *h, uint32_t k, uint32_t *d_out, uint32_t *k_out) {
+    const int lane = threadIdx.x & 31;
+    uint32_t mine = 0;
+#pragma unroll
+    for (int b = 0; b < 8; ++b) mine += h[255 - 8 * lane - b];
+    uint32_t incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    uint32_t cum = incl - mine;
+    if (cum < k && cum + mine >= k) {
+        for (int b = 0; b < 8; ++b) {
+            const uint32_t c = h[255 - 8 * lane - b];
+            if (cum + c >= k) {
+                *d_out = (uint32_t)(255 - 8 * lane - b);
+                *k_out = k - cum;
+                break;
+            }
+            cum += c;
+        }
+    }
+}
+
+// Exclusive block scan of two counts; returns this thread's offsets and the totals.
+__device__ __forceinline__ void sk_scan2(int a, int b, int (*wsum)[SK_THREADS / 32], int &oa, int &ob, int &ta,
+                                         int &tb) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int ia = a, ib = b;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int x = __shfl_up_sync(0xffffffffu, ia, o), y = __shfl_up_sync(0xffffffffu, ib, o);
+        if (lane >= o) {
+            ia += x;
+            ib += y;
+        }
+    }
+    if (lane == 31) {
+        wsum[0][warp] = ia;
+        wsum[1][warp] = ib;
+    }
+    __syncthreads();
+    int pa = 0, pb = 0;
+    ta = tb = 0;
+#pragma unroll
+    for (int w = 0; w < SK_THREADS / 32; ++w) {
+        pa += (w < warp) ? wsum[0][w] : 0;
+        pb += (w < warp) ? wsum[1][w] : 0;
+        ta += wsum[0][w];
+        tb += wsum[1][w];
+    }
+    __syncthreads();
+    oa = pa + ia - a;
+    ob = pb + ib - b;
+}
+
+// The fp32 score of block b for the row whose operand is in sm.q (one thread).
+__device__ __forceinline__ float sk_score(const KeySelSmem &sm, const __nv_bfloat16 *kb, int mode, int relu) {
+    const __nv_bfloat162 *k2 = reinterpret_cast<const __nv_bfloat162 *>(kb);
+    if (mode == 0) {
+        float acc = 0.f;
+#pragma unroll 8
+        for (int i = 0; i < kIdxDim / 2; ++i) {
+            const float2 kv = __bfloat1622float2(k2[i]);
+            acc = fmaf(sm.q[2 * i], kv.x, acc);
+            acc = fmaf(sm.q[2 * i + 1], kv.y, acc);
+        }
+        return acc;
+    }
+    float tot = 0.f;
+    for (int h = 0; h < kIdxHeads; ++h) {
+        float acc = 0.f;
+#pragma unroll 8
+        for (int i = 0; i < kIdxDim / 2; ++i) {
+            const float2 kv = __bfloat1622float2(k2[i]);
+            acc = fmaf(sm.q[h * kIdxDim + 2 * i], kv.x, acc);
+            acc = fmaf(sm.q[h * kIdxDim + 2 * i + 1], kv.y, acc);
+        }
+        if (relu) acc = fmaxf(acc, 0.f);
+        tot = fmaf(sm.w[h], acc, tot);
+    }
+    return tot;
+}
+
+__global__ void __launch_bounds__(SK_THREADS) select_keys_kernel(KeySelParams p) {
+    extern __shared__ __align__(16) uint8_t ksm_raw[];
+    KeySelSmem &sm = *reinterpret_cast<KeySelSmem *>(ksm_raw);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int seq = blockIdx.y;
+    const int64_t rloc = blockIdx.x;
+    const int64_t row = p.row_begin + rloc;
+    const int64_t qrow = (int64_t)seq * p.n_q + row;
+    const int n = (int)((p.q0 + row + 1) / kBlock);
+    const uint32_t k = (uint32_t)p.top_k;
+    int32_t *out = p.sel + qrow * p.top_k;
+    pdl_wait();
+    pdl_trigger();
+    if (n <= (int)k) {
+        for (int i = tid; i < (int)k; i += SK_THREADS) out[i] = i < n ? i : -1;
+        if (tid == 0) p.nsel[qrow] = n;
+        return;
+    }
+    const uint16_t *src = p.keys + ((int64_t)seq * p.row_count + rloc) * p.ld;
+    const __nv_bfloat16 *kp = p.k_pool + (int64_t)seq * p.pool_stride * kIdxDim;
+    // the row's query operand (fp32) and head weights
+    if (p.mode == 0) {
+        for (int i = tid; i < kIdxDim; i += SK_THREADS)
+            sm.q[i] = __bfloat162float(p.qa0[qrow * kIdxDim + i]) + __bfloat162float(p.qa1[qrow * kIdxDim + i]);
+    } else {
+        for (int i = tid; i < kIdxHeads * kIdxDim; i += SK_THREADS)
+            sm.q[i] = __bfloat162float(p.qa0[qrow * kIdxHeads * kIdxDim + i]);
+        if (tid < kIdxHeads) sm.w[tid] = p.head_w ? p.head_w[qrow * kIdxHeads + tid] : 1.f;
+    }
+    for (int i = tid; i < 256; i += SK_THREADS) sm.h1[i] = sm.h2[i] = 0;
+    __syncthreads();
+
+    // 8 keys of a tile (thread tid: elements base + 8 tid ..), zero past the row (never counted)
+    auto load8 = [&](int base, uint16_t (&kk)[8]) {
+        const int i = base + 8 * tid;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (i < n) v = *reinterpret_cast<const uint4 *>(src + i);   // ld is a multiple of 128: in the row
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            kk[2 * e] = (uint16_t)(w4[e] & 0xFFFFu);
+            kk[2 * e + 1] = (uint16_t)(w4[e] >> 16);
+        }
+    };
+    // ---- pass 1: high byte
+    for (int base = 0; base < n; base += SK_TILE) {
+        uint16_t kk[8];
+        load8(base, kk);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            if (base + 8 * tid + e < n) atomicAdd(&sm.h1[kk[e] >> 8], 1u);
+    }
+    __syncthreads();
+    if (warp == 0) sk_find_bin(sm.h1, k, &sm.d1, &sm.k1);
+    __syncthreads();
+    const uint32_t d1 = sm.d1;
+    // ---- pass 2: low byte within bin d1
+    for (int base = 0; base < n; base += SK_TILE) {
+        uint16_t kk[8];
+        load8(base, kk);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            if (base + 8 * tid + e < n && (uint32_t)(kk[e] >> 8) == d1) atomicAdd(&sm.h2[kk[e] & 0xFFu], 1u);
+    }
+    __syncthreads();
+    if (warp == 0) {
+        sk_find_bin(sm.h2, sm.k1, &sm.d2, &sm.k2);
+        __syncwarp();
+        if (lane == 0) sm.n_amb = sm.h2[sm.d2];
+    }
+    __syncthreads();
+    const uint32_t T = (d1 << 8) | sm.d2;
+    const uint32_t k2 = sm.k2, n_amb = sm.n_amb;
+    const int n_sure = (int)(k - k2);
+    // ---- pass 3: ids above T and equal to T, ascending
+    {
+        int pos_s = 0, pos_a = 0;
+        for (int base = 0; base < n; base += SK_TILE) {
+            uint16_t kk[8];
+            load8(base, kk);
+            int cs = 0, ca = 0;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const bool live = base + 8 * tid + e < n;
+                cs += (live && kk[e] > T) ? 1 : 0;
+                ca += (live && kk[e] == T) ? 1 : 0;
+            }
+            int os, oa, ts, ta;
+            sk_scan2(cs, ca, sm.wsum, os, oa, ts, ta);
+            os += pos_s;
+            oa += pos_a;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const bool live = base + 8 * tid + e < n;
+                const uint32_t id = (uint32_t)(base + 8 * tid + e);
+                if (live && kk[e] > T) {
+                    if (os < 2048) sm.sure[os] = id;
+                    ++os;
+                }
+                if (live && kk[e] == T) {
+                    if (oa < SK_AMB_CAP) sm.amb[oa] = id;
+                    ++oa;
+                }
+            }
+            pos_s += ts;
+            pos_a += ta;
+        }
+    }
+    __syncthreads();
+    if (n_amb <= (uint32_t)SK_AMB_CAP) {
+        // ---- re-score the keys equal to T (one thread each), rank, pick the k2 best
+        for (uint32_t i = tid; i < n_amb; i += SK_THREADS)
+            sm.amb_s[i] = sk_score(sm, kp + (int64_t)sm.amb[i] * kIdxDim, p.mode, p.relu);
+        __syncthreads();
+        for (uint32_t i = tid; i < n_amb; i += SK_THREADS) {
+            const float si = sm.amb_s[i];
+            uint32_t r = 0;
+            for (uint32_t j = 0; j < n_amb; ++j) {
+                const float sj = sm.amb_s[j];
+                r += (sj > si || (sj == si && j < i)) ? 1u : 0u;   // the list is in id order
+            }
+            sm.chosen[i < 2048 ? i : 0] = r;   // n_amb <= SK_AMB_CAP = 2048
+        }
+        __syncthreads();
+        // compact the picked ones in id order
+        int pos = 0;
+        for (uint32_t base = 0; base < n_amb; base += SK_THREADS) {
+            const uint32_t i = base + tid;
+            const bool pick = i < n_amb && sm.chosen[i] < k2;
+            int o, dummy, t, td;
+            sk_scan2(pick ? 1 : 0, 0, sm.wsum, o, dummy, t, td);
+            // the ranks of this window are read before any write below (scan barrier)
+            if (pick) sm.amb_s[pos + o] = __uint_as_float(sm.amb[i]);
+            pos += t;
+        }
+        __syncthreads();
+        for (uint32_t i = tid; i < k2; i += SK_THREADS) sm.chosen[i] = __float_as_uint(sm.amb_s[i]);
+        __syncthreads();
+    } else {
+        // ---- massive ties: exact radix select over the re-scored 32-bit keys of the entries equal to T
+        if (tid == 0) {
+            sm.prefix = 0;
+            sm.need = k2;
+        }
+        for (int byte = 3; byte >= 0; --byte) {
+            for (int i = tid; i < 256; i += SK_THREADS) sm.h1[i] = 0;
+            __syncthreads();
+            const uint32_t prefix = sm.prefix;
+            for (int base = 0; base < n; base += SK_TILE) {
+                uint16_t kk[8];
+                load8(base, kk);
+#pragma unroll 1
+                for (int e = 0; e < 8; ++e) {
+                    if (base + 8 * tid + e >= n || kk[e] != T) continue;
+                    const uint32_t ek = score_key(sk_score(sm, kp + (int64_t)(base + 8 * tid + e) * kIdxDim, p.mode,
+                                                           p.relu));
+                    const bool match = byte == 3 || (ek >> (8 * (byte + 1))) == prefix;
+                    if (match) atomicAdd(&sm.h1[(ek >> (8 * byte)) & 0xFFu], 1u);
+                }
+            }
+            __syncthreads();
+            if (warp == 0) {
+                sk_find_bin(sm.h1, sm.need, &sm.d2, &sm.k1);   // (d2, k1 reused as scratch: T is kept above)
+                __syncwarp();
+                if (lane == 0) {
+                    sm.prefix = (prefix << 8) | sm.d2;
+                    sm.need = sm.k1;
+                }
+            }
+            __syncthreads();
+        }
+        const uint32_t tx = sm.prefix, need = sm.need;   // exact threshold key; picks among keys == tx
+        int pos = 0, peq = 0;
+        for (int base = 0; base < n; base += SK_TILE) {
+            uint16_t kk[8];
+            load8(base, kk);
+            uint32_t ek[8];
+            int cg = 0, ce = 0;
+#pragma unroll 1
+            for (int e = 0; e < 8; ++e) {
+                ek[e] = 0;
+                if (base + 8 * tid + e >= n || kk[e] != T) continue;
+                ek[e] = score_key(sk_score(sm, kp + (int64_t)(base + 8 * tid + e) * kIdxDim, p.mode, p.relu));
+                cg += ek[e] > tx ? 1 : 0;
+                ce += ek[e] == tx ? 1 : 0;
+            }
+            int og, oe, tg, te;
+            sk_scan2(cg, ce, sm.wsum, og, oe, tg, te);
+            // picks of this tile: every key > tx, and keys == tx while fewer than `need` were taken
+            int taken_eq = peq + oe;
+            int mine = 0;
+#pragma unroll 1
+            for (int e = 0; e < 8; ++e) {
+                if (base + 8 * tid + e >= n || kk[e] != T) continue;
+                if (ek[e] > tx) ++mine;
+                else if (ek[e] == tx && taken_eq < (int)need) {
+                    ++mine;
+                    ++taken_eq;
+                }
+            }
+            int om, dummy, tm, td;
+            sk_scan2(mine, 0, sm.wsum, om, dummy, tm, td);
+            om += pos;
+            taken_eq = peq + oe;
+#pragma unroll 1
+            for (int e = 0; e < 8; ++e) {
+                if (base + 8 * tid + e >= n || kk[e] != T) continue;
+                bool pick = ek[e] > tx;
+                if (!pick && ek[e] == tx && taken_eq < (int)need) {
+                    pick = true;
+                    ++taken_eq;
+                }
+                if (pick) {
+                    if (om < 2048) sm.chosen[om] = (uint32_t)(base + 8 * tid + e);
+                    ++om;
+                }
+            }
+            pos += tm;
+            peq += te;
+        }
+        __syncthreads();
+    }
+    // ---- merge the two ascending lists: sure (n_sure) and chosen (k2)
+    for (int i = tid; i < n_sure; i += SK_THREADS) {
+        const uint32_t id = sm.sure[i];
+        int lo = 0, hi = (int)k2;   // chosen ids below id
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (sm.chosen[mid] < id) lo = mid + 1;
+            else hi = mid;
+        }
+        out[i + lo] = (int32_t)id;
+    }
+    for (int j = tid; j < (int)k2; j += SK_THREADS) {
+        const uint32_t id = sm.chosen[j];
+        int lo = 0, hi = n_sure;
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (sm.sure[mid] < id) lo = mid + 1;
+            else hi = mid;
+        }
+        out[j + lo] = (int32_t)id;
+    }
+    if (tid == 0) p.nsel[qrow] = (int)k;
+}
+
 // Driver-API tensor-map encoder obtained through the runtime (no -lcuda).
 using EncodeTiledFn = decltype(&cuTensorMapEncodeTiled);
 EncodeTiledFn get_encode() {
@@ -532,7 +940,7 @@ cudaError_t launch_score_gemm(const ScoreGemmArgs &a, const void *qa0, const voi
     if (!make_map(&ma1, a.per_head ? qa0 : qa1, a_rows, GM)) return cudaErrorInvalidValue;
     if (!make_map(&mb, k_pool, (uint64_t)a.B * a.pool_stride, GN)) return cudaErrorInvalidValue;
     GemmParams p{a.n_q, a.q0, a.row_begin, a.row_count, a.pool_stride, a.ld, a.per_head, a.relu, a.head_w,
-                 a.scores, status, 1, 0};
+                 a.scores, status, 1, 0, a.keys};
     // Split each row tile's key tiles over several CTAs so that the grid holds
     // about four CTAs per SM whatever the row count (a 2048-row chunk of a
     // 1M-token context has 16 row tiles of 2048 key tiles each).
@@ -564,6 +972,34 @@ cudaError_t launch_score_simt_f32(const ScoreGemmArgs &a, const float *q_hat, co
     dim3 grid((unsigned)((nb_max + 127) / 128), (unsigned)a.row_count, (unsigned)a.B);
     score_simt_kernel<<<grid, 128, 0, s>>>(q_hat, k_pool, p);
     return cudaGetLastError();
+}
+
+cudaError_t launch_select_keys(const uint16_t *keys, int B, int64_t row_begin, int64_t row_count, int64_t n_q,
+                               int64_t q0, int64_t ld, int top_k, int mode, int relu, const void *qa0, const void *qa1,
+                               const void *k_pool, int64_t pool_stride, const float *head_w, int32_t *sel,
+                               int32_t *nsel, cudaStream_t s) {
+    if (row_count <= 0) return cudaSuccess;
+    KeySelParams p{};
+    p.keys = keys;
+    p.row_begin = row_begin;
+    p.row_count = row_count;
+    p.n_q = n_q;
+    p.q0 = q0;
+    p.ld = ld;
+    p.pool_stride = pool_stride;
+    p.top_k = top_k;
+    p.mode = mode;
+    p.relu = relu;
+    p.qa0 = static_cast<const __nv_bfloat16 *>(qa0);
+    p.qa1 = static_cast<const __nv_bfloat16 *>(qa1);
+    p.k_pool = static_cast<const __nv_bfloat16 *>(k_pool);
+    p.head_w = head_w;
+    p.sel = sel;
+    p.nsel = nsel;
+    const size_t smem = sizeof(KeySelSmem);
+    cudaError_t e = cudaFuncSetAttribute(select_keys_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(select_keys_kernel, dim3((unsigned)row_count, (unsigned)B), dim3(SK_THREADS), smem, s, p);
 }
 
 cudaError_t launch_select_rows(const float *scores, int B, int64_t row_begin, int64_t row_count, int64_t n_q,

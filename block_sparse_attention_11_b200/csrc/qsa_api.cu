@@ -102,10 +102,12 @@ PrefillPlan prefill_plan(int B, int64_t n_q, int64_t q0, uint32_t flags, int dty
     else p.q_bytes = round256(rows * kIdxHeads * kIdxDim * 4);
     const int64_t nb_max = (q0 + n_q) / kBlock;
     p.ld = std::max<int64_t>(128, (nb_max + 127) / 128 * 128);
-    // keep one chunk of scores under 2 GiB; chunks are multiples of 128 rows
-    const int64_t budget_rows = std::max<int64_t>(128, ((int64_t)1 << 31) / (p.ld * 4 * std::max(B, 1)) / 128 * 128);
+    // BF16 modes store 16-bit order keys, fp32 mode the scores; keep one chunk under 2 GiB;
+    // chunks are multiples of 128 rows
+    const int64_t el = p.mode == 2 ? 4 : 2;
+    const int64_t budget_rows = std::max<int64_t>(128, ((int64_t)1 << 31) / (p.ld * el * std::max(B, 1)) / 128 * 128);
     p.chunk = std::min<int64_t>(std::max<int64_t>(n_q, 1), budget_rows);
-    p.score_bytes = round256((size_t)B * p.chunk * p.ld * 4);
+    p.score_bytes = round256((size_t)B * p.chunk * p.ld * el);
     return p;
 }
 
@@ -259,10 +261,17 @@ int qsa_index_topk_prefill(const void *q_idx, const void *k_pool, const float *h
         a.relu = (flags & QSA_SCORE_RELU) ? 1 : 0;
         a.head_w = head_w;
         a.scores = scores;
-        if (pl.mode == 2) e = launch_score_simt_f32(a, static_cast<const float *>(q0buf), static_cast<const float *>(k_pool), s);
-        else e = launch_score_gemm(a, q0buf, q1buf, k_pool, di->status, s);
-        if (e != cudaSuccess) return QSA_ERR_CUDA;
-        e = launch_select_rows(scores, B, r, a.row_count, n_q, q0, pl.ld, top_k, sel, nsel, di->status, s);
+        if (pl.mode == 2) {
+            e = launch_score_simt_f32(a, static_cast<const float *>(q0buf), static_cast<const float *>(k_pool), s);
+            if (e != cudaSuccess) return QSA_ERR_CUDA;
+            e = launch_select_rows(scores, B, r, a.row_count, n_q, q0, pl.ld, top_k, sel, nsel, di->status, s);
+        } else {
+            a.keys = reinterpret_cast<uint16_t *>(scores);
+            e = launch_score_gemm(a, q0buf, q1buf, k_pool, di->status, s);
+            if (e != cudaSuccess) return QSA_ERR_CUDA;
+            e = launch_select_keys(a.keys, B, r, a.row_count, n_q, q0, pl.ld, top_k, pl.mode, a.relu, q0buf, q1buf,
+                                   k_pool, pool_stride, head_w, sel, nsel, s);
+        }
         if (e != cudaSuccess) return QSA_ERR_CUDA;
     }
     return QSA_OK;

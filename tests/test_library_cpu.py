@@ -176,10 +176,11 @@ def test_prefill_attention_workspace_sizes(qsa):
 
 def test_prefill_kernel_counts(qsa):
     """Launch counts the benchmark reports: the indexer at 128K runs its score
-    kernel and row select in 8 chunks of 16384 rows (scores under 2 GiB); the
+    kernel and row select in 4 chunks of 32768 rows (16-bit keys under 2 GiB); the
     split attention runs three kernels per sequence and chunk of rows (lists,
     gather kernel, tiles)."""
-    assert qsa.qsa_index_topk_prefill_kernels(1, 131072, 0, 0, qsa.QSA_BF16) == 1 + 2 * 8
+    assert qsa.qsa_index_topk_prefill_kernels(1, 131072, 0, 0, qsa.QSA_BF16) == 1 + 2 * 4
+    assert qsa.qsa_index_topk_prefill_kernels(1, 131072, 0, 0, qsa.QSA_FP32) == 1 + 2 * 8   # fp32 scores
     assert qsa.qsa_index_topk_prefill_kernels(1, 32768, 0, 0, qsa.QSA_BF16) == 1 + 2 * 1
     assert qsa.qsa_sparse_attn_prefill_kernels(1, 131072, 512, 16, 2, 128, qsa.QSA_BF16) == 3
     assert qsa.qsa_sparse_attn_prefill_kernels(2, 4096, 512, 16, 2, 128, qsa.QSA_BF16) == 6
