@@ -203,17 +203,21 @@ QSA_API int qsa_pool_keys_decode(const void *k_new, void *ring, void *k_pool, co
  * sel      device, [B][n_q][top_k] int32.   nsel  device, [B][n_q] int32.
  * workspace device scratch of at least qsa_index_topk_prefill_workspace()
  *          bytes, 256-byte aligned; contents on entry are ignored.  The
- *          scores of a group of rows are materialised there in fp32 (groups
- *          of at most 2 GiB: 2048 rows at a 1M-token context), so the size
- *          grows with q0 + n_q up to that cap.
+ *          scores of a group of rows are materialised there (groups of at
+ *          most 2 GiB), so the size grows with q0 + n_q up to that cap.
+ *          QSA_BF16 stores each score as the top 16 bits of its
+ *          order-preserving key (4096 rows a group at a 1M-token context);
+ *          the select ranks by them and re-scores in fp32 the blocks whose
+ *          16-bit key equals the k-th largest one, so the ranking is that of
+ *          the fp32 scores up to their rounding.  QSA_FP32 stores fp32 scores.
  * top_k    1..2048.
  * Chunked prefill: one call per chunk of rows with q0 = the chunk's first
  * position, after that chunk's keys were pooled into k_pool; the selections
  * equal those of one call over all rows (tested to 1,048,576 positions).
  */
 /* Kernels one qsa_index_topk_prefill call with these sizes launches: the
- * query rotation, then a score kernel and a row select per chunk of query rows
- * (chunks keep the score block under 2 GiB); 0 for invalid arguments. */
+ * query rotation, then a score kernel and a row select per group of query rows
+ * (groups keep the score block under 2 GiB); 0 for invalid arguments. */
 QSA_API int qsa_index_topk_prefill_kernels(int32_t B, int64_t n_q, int64_t q0, uint32_t flags, int32_t dtype);
 QSA_API size_t qsa_index_topk_prefill_workspace(int32_t B, int64_t n_q, int64_t q0, int32_t top_k,
                                         uint32_t flags, int32_t dtype);
@@ -290,20 +294,24 @@ QSA_API int qsa_index_topk_decode(const void *q_idx, const void *k_pool, const f
  * workspace: device, 256-byte aligned, at least qsa_sparse_attn_prefill_workspace()
  *          bytes, caller-owned and needing no initialisation; 0 bytes (pass
  *          NULL) for the shapes that run without one.  QSA_BF16 with d = 128,
- *          Hq = 8 Hkv and Hkv = 2 or 4 runs on the tensor cores over tiles of
- *          8 consecutive query rows: a pre-pass merges the tile's 8 selections
- *          and tail blocks into one ascending block list (with a per-block
- *          mask of the queries attending to it) in the workspace, so each
- *          listed block's K/V (a pair of kv heads) is gathered once per tile;
- *          masked keys contribute exactly zero.  The workspace is capped near
- *          512 MiB: longer prompts run as several launches of whole query
- *          tiles.  Results of a chunk starting at a row that is a multiple of
- *          8 equal those of the same rows in one call bit for bit.  Too
- *          small: QSA_ERR_WORKSPACE.
+ *          Hq = 8 Hkv and Hkv = 2 or 4 splits the work by sharing over tiles
+ *          of 8 consecutive query rows: a pre-pass lists, per tile, the
+ *          blocks that 2 or more of its queries select and the tail blocks
+ *          (with a mask of the queries attending to each), and per query the
+ *          blocks only it selects; the tile's listed blocks run on the tensor
+ *          cores, their K/V (a pair of kv heads) gathered once per tile
+ *          (masked keys contribute exactly zero), the own blocks in the
+ *          per-query gather kernel, and the two partial softmaxes are merged
+ *          by their log-sum-exp.  The workspace holds both lists and the
+ *          gather part's lse; it is capped near 1 GiB per sequence: longer
+ *          prompts run as several chunks of whole query tiles.  Results of a
+ *          chunk starting at a row that is a multiple of 8 equal those of the
+ *          same rows in one call bit for bit.  Too small: QSA_ERR_WORKSPACE.
  */
 /* Kernels one qsa_sparse_attn_prefill call with these sizes launches: 1 (the
- * gather kernels: fp32, d = 256, other GQA ratios) or 2 per launch of query
- * tiles (block lists, attention); 0 for invalid arguments. */
+ * gather kernels: fp32, d = 256, other GQA ratios) or 3 per sequence and
+ * chunk of query tiles (lists, gather kernel, tiles); 0 for invalid
+ * arguments. */
 QSA_API int qsa_sparse_attn_prefill_kernels(int32_t B, int64_t n_q, int32_t top_k, int32_t Hq, int32_t Hkv, int32_t d,
                                             int32_t dtype);
 QSA_API size_t qsa_sparse_attn_prefill_workspace(int32_t B, int64_t n_q, int32_t top_k, int32_t Hq, int32_t Hkv,
