@@ -189,9 +189,10 @@ class PrefillRunner:
         ws = max(qsa.qsa_index_topk_prefill_workspace(B, c1 - c0, c0, w.top_k, 0, self.dt_code)
                  for c0, c1 in self.chunks)
         self.ws = torch.empty(ws, dtype=torch.uint8, device=dev)
-        # the attention's workspace (block lists of its 16-query tiles), allocated once
+        # the attention's workspace (the split's lists), allocated once
         wa = 0 if self.kv8 else max(qsa.qsa_sparse_attn_prefill_workspace(B, c1 - c0, w.top_k, w.Hq, w.Hkv, w.d,
-                                                                          self.dt_code) for c0, c1 in self.chunks)
+                                                                          self.dt_code, q0=c0)
+                                    for c0, c1 in self.chunks)
         self.ws_a = torch.empty(max(wa, 1), dtype=torch.uint8, device=dev)
         # the step's inputs (~200 MB at T=32K) do not all stay in L2, but the
         # flush keeps every timed step cold
@@ -266,13 +267,13 @@ class PrefillRunner:
 
     def launches_per_step(self):
         # per chunk: pooling, the indexer's kernels (query rotation, then scores + row select per row
-        # chunk), the attention's kernels (block lists + attention per launch of query tiles, or one)
+        # chunk), the attention's kernels (lists + gather kernel + tiles per sequence and chunk of rows, or one)
         qsa, w = self.qsa, self.w
         n = 0
         for c0, c1 in self.chunks:
             n += 1 + qsa.qsa_index_topk_prefill_kernels(w.B, c1 - c0, c0, 0, self.dt_code)
             n += 1 if self.kv8 else qsa.qsa_sparse_attn_prefill_kernels(w.B, c1 - c0, w.top_k, w.Hq, w.Hkv, w.d,
-                                                                        self.dt_code)
+                                                                        self.dt_code, q0=c0)
         return n
 
     def units(self):

@@ -103,8 +103,8 @@ _sig("qsa_index_topk_decode", ctypes.c_int, _vp, _vp, _vp, _vp, _i32, _i64, _i64
 _sig("qsa_sparse_attn_prefill", ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i64, _i64, _i32, _i32, _i32,
      _i32, _f32, _vp, _vp, _vp, _sz, _i32, _vp)
 _sig("qsa_sparse_attn_decode_workspace", _sz, _i32, _i32, _i32, _i32, _i32)
-_sig("qsa_sparse_attn_prefill_workspace", _sz, _i32, _i64, _i32, _i32, _i32, _i32, _i32)
-_sig("qsa_sparse_attn_prefill_kernels", ctypes.c_int, _i32, _i64, _i32, _i32, _i32, _i32, _i32)
+_sig("qsa_sparse_attn_prefill_workspace", _sz, _i32, _i64, _i64, _i32, _i32, _i32, _i32, _i32)
+_sig("qsa_sparse_attn_prefill_kernels", ctypes.c_int, _i32, _i64, _i64, _i32, _i32, _i32, _i32, _i32)
 _sig("qsa_index_topk_prefill_kernels", ctypes.c_int, _i32, _i64, _i64, _u32, _i32)
 _sig("qsa_sparse_attn_decode", ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32, _i32,
      _f32, _vp, _vp, _vp, _sz, _i32, _vp)
@@ -261,16 +261,16 @@ def qsa_index_topk_decode(q_idx, k_pool, seq_len, sel, nsel, max_blocks=None, to
     _check(st, "qsa_index_topk_decode")
 
 
-def qsa_sparse_attn_prefill_kernels(B, n_q, top_k, Hq, Hkv, d, dtype=QSA_BF16) -> int:
-    return lib.qsa_sparse_attn_prefill_kernels(B, n_q, top_k, Hq, Hkv, d, dtype)
+def qsa_sparse_attn_prefill_kernels(B, n_q, top_k, Hq, Hkv, d, dtype=QSA_BF16, q0=0) -> int:
+    return lib.qsa_sparse_attn_prefill_kernels(B, n_q, q0, top_k, Hq, Hkv, d, dtype)
 
 
 def qsa_index_topk_prefill_kernels(B, n_q, q0=0, flags=0, dtype=QSA_BF16) -> int:
     return lib.qsa_index_topk_prefill_kernels(B, n_q, q0, flags, dtype)
 
 
-def qsa_sparse_attn_prefill_workspace(B, n_q, top_k, Hq, Hkv, d, dtype=QSA_BF16) -> int:
-    return lib.qsa_sparse_attn_prefill_workspace(B, n_q, top_k, Hq, Hkv, d, dtype)
+def qsa_sparse_attn_prefill_workspace(B, n_q, top_k, Hq, Hkv, d, dtype=QSA_BF16, q0=0) -> int:
+    return lib.qsa_sparse_attn_prefill_workspace(B, n_q, q0, top_k, Hq, Hkv, d, dtype)
 
 
 def qsa_sparse_attn_prefill(q, k, v, sel, nsel, out, q0=0, top_k=None, scale=None, lse=None, workspace=None,
@@ -282,7 +282,7 @@ def qsa_sparse_attn_prefill(q, k, v, sel, nsel, out, q0=0, top_k=None, scale=Non
     Hkv = k.shape[2]
     top_k = sel.shape[-1] if top_k is None else top_k
     scale = (1.0 / d ** 0.5) if scale is None else scale
-    need = qsa_sparse_attn_prefill_workspace(B, max(n_q, 1), top_k, Hq, Hkv, d, dt)
+    need = qsa_sparse_attn_prefill_workspace(B, max(n_q, 1), top_k, Hq, Hkv, d, dt, q0=q0)
     wp, wb = _ws(need, q.device, workspace) if need else (None, 0)
     st = lib.qsa_sparse_attn_prefill(_ptr(q, None, "q"), _ptr(k, q.dtype, "k"), _ptr(v, q.dtype, "v"),
                                      _ptr(sel, torch.int32, "sel"), _ptr(nsel, torch.int32, "nsel"), B, n_q, q0,

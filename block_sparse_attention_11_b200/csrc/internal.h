@@ -164,7 +164,8 @@ cudaError_t launch_attn_bf16(const AttnArgs &a, void *ws, unsigned *status, cuda
 // head, contiguous BF16 K/V.  Blocks that several queries of a tile of 8
 // attend to run on the tensor cores once per tile; the rest run in the gather
 // kernel (launch_attn_bf16) per query; the tile kernel merges the two.  Its
-// workspace holds the block lists, the per-query lists and their lse.
+// workspace holds the block lists, the per-query lists and their lse.  Used
+// for contexts of at most 32768 blocks (q0 + n_q <= 131075 positions).
 bool attn_union_supported(const AttnArgs &a);
 size_t attn_union_ws_bytes(int B, int64_t n_q, int top_k, int Hq);
 int attn_union_launches(int B, int64_t n_q, int top_k, int Hq);   // chunks per call (3 kernels each)

@@ -792,7 +792,11 @@ UnionPlan union_plan(int64_t n_q, int top_k, int Hq) {
 }  // namespace
 
 bool attn_union_supported(const AttnArgs &a) {
-    return !a.decode && !a.kv8 && a.d == UD && a.Hq == UG * a.Hkv && (a.Hkv == 2 || a.Hkv == 4) && !a.pg.table;
+    // Longer contexts take the gather kernel alone: their block ids no longer fit one
+    // pre-pass chunk, and measured at 1M tokens in 16,000-token chunks the split was slower
+    // (attention 193 vs 160 ms).
+    return !a.decode && !a.kv8 && a.d == UD && a.Hq == UG * a.Hkv && (a.Hkv == 2 || a.Hkv == 4) && !a.pg.table &&
+           (a.q0 + a.n_q) / kBlock <= UCHUNK;
 }
 
 size_t attn_union_ws_bytes(int B, int64_t n_q, int top_k, int Hq) {

@@ -205,11 +205,13 @@ QSA_API int qsa_pool_keys_decode(const void *k_new, void *ring, void *k_pool, co
  *          bytes, 256-byte aligned; contents on entry are ignored.  The
  *          scores of a group of rows are materialised there (groups of at
  *          most 2 GiB), so the size grows with q0 + n_q up to that cap.
- *          QSA_BF16 stores each score as the top 16 bits of its
- *          order-preserving key (4096 rows a group at a 1M-token context);
- *          the select ranks by them and re-scores in fp32 the blocks whose
- *          16-bit key equals the k-th largest one, so the ranking is that of
- *          the fp32 scores up to their rounding.  QSA_FP32 stores fp32 scores.
+ *          QSA_BF16 with rows of at most 32768 blocks ((q0 + n_q) / 4 <=
+ *          32768) stores each score as the top 16 bits of its
+ *          order-preserving key; the select ranks by them and re-scores in
+ *          fp32 the blocks whose 16-bit key equals the k-th largest one, so
+ *          the ranking is that of the fp32 scores up to their rounding.
+ *          Longer rows (2048 rows a group at a 1M-token context) and
+ *          QSA_FP32 store fp32 scores.
  * top_k    1..2048.
  * Chunked prefill: one call per chunk of rows with q0 = the chunk's first
  * position, after that chunk's keys were pooled into k_pool; the selections
@@ -294,7 +296,8 @@ QSA_API int qsa_index_topk_decode(const void *q_idx, const void *k_pool, const f
  * workspace: device, 256-byte aligned, at least qsa_sparse_attn_prefill_workspace()
  *          bytes, caller-owned and needing no initialisation; 0 bytes (pass
  *          NULL) for the shapes that run without one.  QSA_BF16 with d = 128,
- *          Hq = 8 Hkv and Hkv = 2 or 4 splits the work by sharing over tiles
+ *          Hq = 8 Hkv, Hkv = 2 or 4 and contexts of at most 32768 blocks
+ *          ((q0 + n_q) / 4 <= 32768) splits the work by sharing over tiles
  *          of 8 consecutive query rows: a pre-pass lists, per tile, the
  *          blocks that 2 or more of its queries select and the tail blocks
  *          (with a mask of the queries attending to each), and per query the
@@ -306,15 +309,17 @@ QSA_API int qsa_index_topk_decode(const void *q_idx, const void *k_pool, const f
  *          gather part's lse; it is capped near 1 GiB per sequence: longer
  *          prompts run as several chunks of whole query tiles.  Results of a
  *          chunk starting at a row that is a multiple of 8 equal those of the
- *          same rows in one call bit for bit.  Too small: QSA_ERR_WORKSPACE.
+ *          same rows in one call bit for bit when both calls split (the gather
+ *          kernel alone is chunk-independent too).  Too small:
+ *          QSA_ERR_WORKSPACE.
  */
 /* Kernels one qsa_sparse_attn_prefill call with these sizes launches: 1 (the
  * gather kernels: fp32, d = 256, other GQA ratios) or 3 per sequence and
  * chunk of query tiles (lists, gather kernel, tiles); 0 for invalid
  * arguments. */
-QSA_API int qsa_sparse_attn_prefill_kernels(int32_t B, int64_t n_q, int32_t top_k, int32_t Hq, int32_t Hkv, int32_t d,
-                                            int32_t dtype);
-QSA_API size_t qsa_sparse_attn_prefill_workspace(int32_t B, int64_t n_q, int32_t top_k, int32_t Hq, int32_t Hkv,
+QSA_API int qsa_sparse_attn_prefill_kernels(int32_t B, int64_t n_q, int64_t q0, int32_t top_k, int32_t Hq,
+                                            int32_t Hkv, int32_t d, int32_t dtype);
+QSA_API size_t qsa_sparse_attn_prefill_workspace(int32_t B, int64_t n_q, int64_t q0, int32_t top_k, int32_t Hq, int32_t Hkv,
                                                  int32_t d, int32_t dtype);
 QSA_API int qsa_sparse_attn_prefill(const void *q, const void *k, const void *v, const int32_t *sel,
                             const int32_t *nsel, int32_t B, int64_t n_q, int64_t q0, int64_t kv_stride,

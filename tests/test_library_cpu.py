@@ -166,7 +166,8 @@ def test_prefill_attention_workspace_sizes(qsa):
         r256(tiles * 4) + r256(tiles * cap * 4) + r256(tiles * cap * 2) + r256(rows * 512 * 4) + r256(rows * 4)
         + r256(rows * 16 * 4))
     assert ws(1, 1, 512, 16, 2, 128, qsa.QSA_BF16) > 0
-    assert 0 < ws(1, 1 << 20, 2048, 16, 2, 128, qsa.QSA_BF16) <= (1 << 30) + 8192
+    assert 0 < ws(1, 131072, 2048, 16, 2, 128, qsa.QSA_BF16) <= (1 << 30) + 8192
+    assert ws(1, 16000, 512, 16, 2, 128, qsa.QSA_BF16, q0=1032576) == 0   # contexts past 32768 blocks: gather kernel
     assert ws(4, 4096, 512, 16, 2, 128, qsa.QSA_BF16) == ws(1, 4096, 512, 16, 2, 128, qsa.QSA_BF16)  # per sequence
     assert ws(1, 4096, 512, 24, 2, 256, qsa.QSA_BF16) == 0      # released shape: the gather kernel
     assert ws(1, 4096, 512, 8, 1, 128, qsa.QSA_BF16) == 0       # one kv head: the gather kernel
@@ -186,4 +187,6 @@ def test_prefill_kernel_counts(qsa):
     assert qsa.qsa_sparse_attn_prefill_kernels(2, 4096, 512, 16, 2, 128, qsa.QSA_BF16) == 6
     assert qsa.qsa_sparse_attn_prefill_kernels(1, 131072, 512, 24, 2, 256, qsa.QSA_BF16) == 1
     assert qsa.qsa_sparse_attn_prefill_kernels(1, 131072, 512, 8, 1, 128, qsa.QSA_BF16) == 1
-    assert qsa.qsa_sparse_attn_prefill_kernels(1, 1 << 20, 2048, 16, 2, 128, qsa.QSA_BF16) > 3
+    assert qsa.qsa_sparse_attn_prefill_kernels(1, 131072, 2048, 16, 2, 128, qsa.QSA_BF16) >= 3
+    assert qsa.qsa_sparse_attn_prefill_kernels(1, 16000, 512, 16, 2, 128, qsa.QSA_BF16, q0=1032576) == 1
+    assert qsa.qsa_index_topk_prefill_kernels(1, 16000, 1032576, 0, qsa.QSA_BF16) == 1 + 2 * 8   # fp32 scores
