@@ -937,9 +937,10 @@ def _overlapping_selection(T, top_k, seed, hot=64, short_every=5):
                                            (16, 2, 9000, 2048), (16, 2, 5, 4)])
 def test_tile_attention_on_overlapping_selections(qsa, Hq, Hkv, T, top_k):
     """Hand-built overlapping selections (hot blocks shared by many rows, rows
-    with fewer than min(top_k, nb) blocks, a last partial 16-row tile): the
-    tensor-core prefill equals the oracle's attention over the same selections,
-    B = 2 sequences with different selections."""
+    with fewer than min(top_k, nb) blocks, a last partial 8-row tile): the
+    split prefill (shared blocks on the tensor cores, the rest in the gather
+    kernel) equals the oracle's attention over the same selections, B = 2
+    sequences with different selections."""
     w = W(T, top_k=top_k, Hq=Hq, Hkv=Hkv, B=2, seed=90 + Hq)
     x = workloads.make_prefill(w, device=DEV)
     sels, nsels = zip(*[_overlapping_selection(T, top_k, seed=7 + b) for b in range(2)])
@@ -959,8 +960,9 @@ def test_tile_attention_on_overlapping_selections(qsa, Hq, Hkv, T, top_k):
 
 
 def test_tile_attention_chunks_off_the_tile_grid(qsa):
-    """Chunks that start off the 16-row tile grid (q0 = 1000, 1001) form other
-    tiles than one call does; every row still matches the oracle."""
+    """Chunks that start off the 8-row tile grid (q0 = 1000, 1001 are not both
+    multiples of 8) form other tiles than one call does; every row still
+    matches the oracle."""
     T, top_k = 1700, 64
     w = W(T, top_k=top_k, seed=95)
     x = workloads.make_prefill(w, device=DEV)
@@ -981,8 +983,8 @@ def test_tile_attention_chunks_off_the_tile_grid(qsa):
 
 
 def test_tile_attention_aligned_chunks_are_bit_exact(qsa):
-    """Chunks starting on the 16-row tile grid reproduce one call bit for bit
-    (same tiles, same block lists, same order of accumulation)."""
+    """Chunks starting on the 8-row tile grid reproduce one call bit for bit
+    (same tiles, same lists, same order of accumulation)."""
     T, top_k = 2000, 96
     w = W(T, top_k=top_k, seed=96)
     x = workloads.make_prefill(w, device=DEV)
@@ -999,3 +1001,82 @@ def test_tile_attention_aligned_chunks_are_bit_exact(qsa):
         out[:, c0:c1] = o
     qsa.qsa_check_status()
     assert torch.equal(out, one)
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(16, 2), (32, 4)])
+def test_split_attention_repeats_bit_identically(qsa, Hq, Hkv):
+    """The split prefill on the oracle's selection: four calls give the same
+    bits (output and lse), and match the oracle.  (A race in the gather
+    kernel's query buffer once made rare rows differ from run to run when
+    its lists were short, as the split's own lists are.)"""
+    T = 2500
+    w = W(T, top_k=96, Hq=Hq, Hkv=Hkv, seed=33)
+    x = workloads.make_prefill(w, device=DEV)
+    rows = list(range(T))
+    kp = oracle.pool_keys(np32(x["k_idx"][0]), store_bf16=True)
+    ref = oracle.prefill_rows(rows, q_idx=np32(x["q_idx"][0]), k_pool=kp, top_k=96, store_bf16=True,
+                              q=np32(x["q"][0]), k=np32(x["k"][0]), v=np32(x["v"][0]), Hq=Hq, Hkv=Hkv, d=128)
+    sel = torch.from_numpy(ref["sel"][None]).to(DEV)
+    nsel = torch.from_numpy(ref["nsel"][None]).to(DEV)
+    outs = []
+    for _ in range(4):
+        out = torch.empty_like(x["q"])
+        lse = torch.empty(1, T, Hq, dtype=torch.float32, device=DEV)
+        qsa.qsa_sparse_attn_prefill(x["q"], x["k"], x["v"], sel, nsel, out, lse=lse)
+        outs.append((out, lse))
+    qsa.qsa_check_status()
+    for out, lse in outs[1:]:
+        assert torch.equal(out, outs[0][0]) and torch.equal(lse, outs[0][1])
+    assert np.abs(np32(outs[0][0][0]) - ref["out"]).max() <= TOL["bf16"]
+    assert np.abs(outs[0][1][0].cpu().numpy() - ref["lse"]).max() <= 1e-3
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(16, 2), (32, 4), (8, 1)])
+def test_attention_tail_only_rows(qsa, Hq, Hkv):
+    """Selections of no block at all (nsel = 0): each row attends to its own
+    0-3 tail tokens only, rows whose position ends a block attend to nothing
+    (zero output, lse = -inf); three calls give the same bits."""
+    T = 2500
+    w = W(T, top_k=96, Hq=Hq, Hkv=Hkv, seed=34)
+    x = workloads.make_prefill(w, device=DEV)
+    sel = torch.full((1, T, 96), -1, dtype=torch.int32, device=DEV)
+    nsel = torch.zeros(1, T, dtype=torch.int32, device=DEV)
+    outs = []
+    for _ in range(3):
+        out = torch.full_like(x["q"], 5.0)
+        lse = torch.empty(1, T, Hq, dtype=torch.float32, device=DEV)
+        qsa.qsa_sparse_attn_prefill(x["q"], x["k"], x["v"], sel, nsel, out, lse=lse)
+        outs.append((out, lse))
+    qsa.qsa_check_status()
+    for out, lse in outs[1:]:
+        assert torch.equal(out, outs[0][0]) and torch.equal(lse, outs[0][1])
+    rows = list(range(T))
+    ref = oracle.prefill_rows(rows, sel_in=sel[0].cpu().numpy(), nsel_in=nsel[0].cpu().numpy(), top_k=96,
+                              q=np32(x["q"][0]), k=np32(x["k"][0]), v=np32(x["v"][0]), Hq=Hq, Hkv=Hkv, d=128)
+    assert np.abs(np32(outs[0][0][0]) - ref["out"]).max() <= TOL["bf16"]
+    g, r = outs[0][1][0].cpu().numpy(), ref["lse"]
+    assert np.array_equal(np.isinf(g), np.isinf(r))
+    fin = np.isfinite(r)
+    assert np.abs(g[fin] - r[fin]).max() <= 1e-3
+
+
+@pytest.mark.parametrize("flags", [0, 1])
+def test_prefill_select_massive_16bit_ties(qsa, flags):
+    """Zero compressed keys: every score is exactly 0, so all keys of a row
+    tie at 16 bits (more than 2048 of them from position 8192 on) and the
+    select takes its exact radix over re-scored keys; the ties go to the
+    lowest ids, as in the oracle (bit-exact), for the linear and the ReLU
+    per-head scores."""
+    T, top_k = 40000, 512
+    g = torch.Generator(device=DEV).manual_seed(41)
+    q_idx = torch.randn(1, T, 4, 128, generator=g, device=DEV).to(torch.bfloat16)
+    k_pool = torch.zeros(1, T // 4, 128, dtype=torch.bfloat16, device=DEV)
+    sel = torch.full((1, T, top_k), -7, dtype=torch.int32, device=DEV)
+    nsel = torch.full((1, T), -7, dtype=torch.int32, device=DEV)
+    qsa.qsa_index_topk_prefill(q_idx, k_pool, sel, nsel, top_k=top_k, rope=qsa.Rope(), flags=flags)
+    qsa.qsa_check_status()
+    rows = [0, 3, 2047, 2048, 2051, 8191, 8200, 20000, 39999]
+    ref = oracle.prefill_rows(rows, q_idx=np32(q_idx[0]), k_pool=np32(k_pool[0]), top_k=top_k, store_bf16=True,
+                              relu=bool(flags & qsa.QSA_SCORE_RELU))
+    assert np.array_equal(nsel[0].cpu().numpy()[rows], ref["nsel"])
+    assert np.array_equal(sel[0].cpu().numpy()[rows], ref["sel"])
