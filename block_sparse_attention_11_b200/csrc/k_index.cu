@@ -22,7 +22,8 @@
 // CTA and stays in shared memory; key tiles stream through a 4-stage TMA
 // ring; two TMEM accumulators (128 columns each) let the epilogue of tile j
 // overlap the MMAs of tile j+1.  Warp roles: 0 = TMA producer, 1 = MMA issuer
-// and TMEM owner, 2..5 = epilogue (warp w reads TMEM lanes 32*(w%4)..+31).
+// and TMEM owner, 2..9 = epilogue: two warps per TMEM lane quarter (warp w
+// reads lanes 32*(w%4)..+31), one per half of the tile's 128 columns.
 #include "internal.h"
 #include "select.cuh"
 
@@ -32,12 +33,13 @@ namespace {
 
 constexpr int GM = 128;
 constexpr int GN = 128;
-constexpr int NST = 4;
+constexpr int NST = 3;
 constexpr int KATOM_BYTES_A = GM * 128;            // 128 rows x 128 bytes
 constexpr int KATOM_BYTES_B = GN * 128;
 constexpr int A_BYTES = 2 * KATOM_BYTES_A;         // one operand plane, both k-atoms
 constexpr int B_STAGE_BYTES = 2 * KATOM_BYTES_B;
-constexpr int GEMM_THREADS = 192;
+constexpr int GEMM_EPI = 8;                        // epilogue warps
+constexpr int GEMM_THREADS = (2 + GEMM_EPI) * 32;
 constexpr int TMEM_COLS = 2 * GN;
 
 struct GemmSmem {
@@ -50,7 +52,7 @@ struct GemmSmem {
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
     uint32_t tmem_base;
-    alignas(16) float epi[4][32][36];   // per epilogue warp: 32 rows x 32 scores, transposed for stores
+    alignas(16) float epi[GEMM_EPI][32][36];   // per epilogue warp: 32 rows x 32 scores, transposed for stores
 };
 
 struct GemmParams {
@@ -85,7 +87,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     if (threadIdx.x == 0) {
         mbar_init(&sm.a_full, 1);
         for (int s = 0; s < NST; ++s) { mbar_init(&sm.b_full[s], 1); mbar_init(&sm.b_empty[s], 1); }
-        for (int s = 0; s < 2; ++s) { mbar_init(&sm.acc_full[s], 1); mbar_init(&sm.acc_empty[s], 4); }
+        for (int s = 0; s < 2; ++s) { mbar_init(&sm.acc_full[s], 1); mbar_init(&sm.acc_empty[s], GEMM_EPI); }
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -160,6 +162,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     } else {
         // ---------------- epilogue: TMEM -> registers -> global scores
         const int quarter = warp & 3;
+        const int ew = warp - 2;                // epilogue warp: staging buffer
+        const int chalf = ew >> 2;              // columns [64 chalf, 64 chalf + 64) of each tile
         const int lrow = quarter * 32 + lane;   // TMEM lane = operand row in the tile
         int64_t qrow;                           // query row (within the sequence)
         int head = 0;
@@ -173,7 +177,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             if (!mbar_wait(&sm.acc_full[ab], (j >> 1) & 1, p.status)) break;
             tc_fence_after();
 #pragma unroll 1
-            for (int c = 0; c < GN / 32; ++c) {
+            for (int c = 2 * chalf; c < 2 * chalf + 2; ++c) {
                 uint32_t r[32];
                 tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(ab * GN + c * 32), r);
                 tc_wait_ld();
@@ -194,7 +198,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 if (p.keys) {
                     // the top 16 bits of the order key (sign, exponent, 7 mantissa bits): the
                     // selection ranks by them and re-scores the keys that tie at 16 bits
-                    uint16_t(*t16)[40] = reinterpret_cast<uint16_t(*)[40]>(&sm.epi[quarter][0][0]);
+                    uint16_t(*t16)[40] = reinterpret_cast<uint16_t(*)[40]>(&sm.epi[ew][0][0]);
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         uint32_t w4[4];
@@ -220,7 +224,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     continue;
                 }
                 // stage the 32 x 32 block in smem and store it row-contiguously
-                float(*tile)[36] = sm.epi[quarter];
+                float(*tile)[36] = sm.epi[ew];
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
                     *reinterpret_cast<float4 *>(&tile[lane][4 * i]) = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2],
