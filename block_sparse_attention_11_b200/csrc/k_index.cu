@@ -176,14 +176,21 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             const int ab = j & 1;
             if (!mbar_wait(&sm.acc_full[ab], (j >> 1) & 1, p.status)) break;
             tc_fence_after();
-#pragma unroll 1
-            for (int c = 2 * chalf; c < 2 * chalf + 2; ++c) {
-                uint32_t r[32];
-                tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(ab * GN + c * 32), r);
-                tc_wait_ld();
+            // both 32-column chunks into registers, then the accumulator is released at once:
+            // the MMAs of tile j + 2 need not wait for this tile's stores
+            uint32_t r2[2][32];
+            tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(ab * GN + 64 * chalf), r2[0]);
+            tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(ab * GN + 64 * chalf + 32), r2[1]);
+            tc_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.acc_empty[ab]);
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+                const int c = 2 * chalf + cc;
                 float v[32];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+                for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r2[cc][i]);
                 if (p.per_head) {
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
@@ -244,9 +251,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 }
                 __syncwarp();
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.acc_empty[ab]);
         }
     }
     tc_fence_before();
