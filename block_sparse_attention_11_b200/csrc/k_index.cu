@@ -534,9 +534,12 @@ __global__ void __launch_bounds__(SR_THREADS)
 // The score GEMM stores the top 16 bits of each score's order key.  Ranking
 // by them is exact except among the keys equal to the threshold key; those
 // are re-scored in fp32 from the query operand and the compressed keys:
-//   pass 1  histogram of the key's high byte; the bin d1 holding the k-th
-//           largest key, and k1, the picks it supplies;
-//   pass 2  histogram of the low byte within bin d1: the threshold key
+//   pass 1  histogram of the key's top 12 bits (sign, exponent and three
+//           significand bits: 8 bins per binade, so the few binades a row's
+//           scores crowd into spread over many bins and the shared-memory
+//           atomics rarely collide); the bin d1 holding the k-th largest key,
+//           and k1, the picks it supplies;
+//   pass 2  histogram of the low 4 bits within bin d1: the threshold key
 //           T = (d1, d2) and k2, the picks among the keys equal to T;
 //   pass 3  ids of keys > T (exactly k - k2) and of keys == T, each list in
 //           ascending id order (per 2048-element tile a block scan orders
@@ -549,15 +552,22 @@ __global__ void __launch_bounds__(SR_THREADS)
 // 2 bytes per visible block, so the CTAs resident at once hold a few tens of
 // MB of rows: passes 2 and 3 read L2.
 constexpr int SK_THREADS = 256;
-constexpr int SK_TILE = SK_THREADS * 8;    // elements per tile: one 16-byte load per thread
+constexpr int SK_TILE = SK_THREADS * 8;    // elements per tile: one 16-byte load per thread (massive ties)
+constexpr int SK_PER = 32;                 // passes 1-3: contiguous keys per thread (four 16-byte loads in flight)
+constexpr int SK_STILE = SK_THREADS * SK_PER;
 constexpr int SK_AMB_CAP = 2048;
 
 struct KeySelSmem {
-    uint32_t h1[256], h2[256];
+    uint32_t h2[256];                     // pass 2 (16 bins); the massive-tie radix select (256 bins)
     uint32_t sure[2048];                  // ids with key > T, ascending
     uint32_t amb[SK_AMB_CAP];             // ids with key == T, ascending
-    float amb_s[SK_AMB_CAP];              // their re-scored values
-    uint32_t chosen[2048];                // the picked ids among them, ascending (also rank scratch)
+    union {
+        uint32_t h1[4096];                // pass 1: counts of the keys' top 12 bits
+        struct {                          // after pass 3
+            float amb_s[SK_AMB_CAP];      // the re-scored values of the keys == T
+            uint32_t chosen[2048];        // the picked ids among them, ascending (also rank scratch)
+        };
+    };
     float q[kIdxHeads * kIdxDim];         // the row's query operand in fp32 (mode 0: the head sum)
     float w[kIdxHeads];
     int wsum[2][SK_THREADS / 32];
@@ -600,6 +610,44 @@ __device__ __forceinline__ void sk_find_bin(const uint32_t *h, uint32_t k, uint3
             cum += c;
         }
     }
+}
+
+// Exclusive block scan of two counts; returns this thread's offsets and the totals.
+__device__ __forceinline__ void sk_scan2(int a, int b, int (*wsum)[SK_THREADS / 32], int &oa, int &ob, int &ta,
+                                         int &tb);
+
+// The k-th largest of 4096 bins counted from the top (the whole CTA): bin d
+// and the picks it supplies.  Thread t owns bins 4095 - 16 t .. 4080 - 16 t.
+// Ends with a barrier.
+__device__ __forceinline__ void sk_find_bin4096(const uint32_t *h, uint32_t k, int (*wsum)[SK_THREADS / 32],
+                                                uint32_t *d_out, uint32_t *k_out) {
+    static_assert(SK_THREADS * 16 == 4096, "16 bins per thread");
+    const int tid = threadIdx.x;
+    const int lo = 16 * (SK_THREADS - 1 - tid);   // this thread's lowest bin
+    const uint4 *src = reinterpret_cast<const uint4 *>(h + lo);
+    uint32_t c[16];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint4 v = src[j];
+        c[4 * j] = v.x; c[4 * j + 1] = v.y; c[4 * j + 2] = v.z; c[4 * j + 3] = v.w;
+    }
+    uint32_t mine = 0;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) mine += c[j];
+    int above, unused, ta, tb;   // keys in the bins above this thread's (threads of lower index)
+    sk_scan2((int)mine, 0, wsum, above, unused, ta, tb);
+    uint32_t cum = (uint32_t)above;
+    if (cum < k && cum + mine >= k) {
+#pragma unroll
+        for (int j = 15; j >= 0; --j) {
+            if (cum < k && cum + c[j] >= k) {
+                *d_out = (uint32_t)(lo + j);
+                *k_out = k - cum;
+            }
+            cum += c[j];
+        }
+    }
+    __syncthreads();
 }
 
 // Exclusive block scan of two counts; returns this thread's offsets and the totals.
@@ -691,7 +739,8 @@ __global__ void __launch_bounds__(SK_THREADS) select_keys_kernel(KeySelParams p)
             sm.q[i] = __bfloat162float(p.qa0[qrow * kIdxHeads * kIdxDim + i]);
         if (tid < kIdxHeads) sm.w[tid] = p.head_w ? p.head_w[qrow * kIdxHeads + tid] : 1.f;
     }
-    for (int i = tid; i < 256; i += SK_THREADS) sm.h1[i] = sm.h2[i] = 0;
+    for (int i = tid; i < 4096 / 4; i += SK_THREADS) reinterpret_cast<uint4 *>(sm.h1)[i] = make_uint4(0, 0, 0, 0);
+    for (int i = tid; i < 256; i += SK_THREADS) sm.h2[i] = 0;
     __syncthreads();
 
     // 8 keys of a tile (thread tid: elements base + 8 tid ..), zero past the row (never counted)
@@ -706,65 +755,80 @@ __global__ void __launch_bounds__(SK_THREADS) select_keys_kernel(KeySelParams p)
             kk[2 * e + 1] = (uint16_t)(w4[e] >> 16);
         }
     };
-    // ---- pass 1: high byte
-    for (int base = 0; base < n; base += SK_TILE) {
-        uint16_t kk[8];
-        load8(base, kk);
+    // Passes 1-3 walk the row in tiles of SK_STILE keys, thread tid holding keys
+    // [base + 32 tid, base + 32 tid + 32): four 16-byte loads in flight per thread,
+    // and in pass 3 one ordered block scan per tile.  Returns the live keys held.
+    auto load32 = [&](int base, uint32_t (&w)[16]) -> int {
+        const int i = base + SK_PER * tid;
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
-            if (base + 8 * tid + e < n) atomicAdd(&sm.h1[kk[e] >> 8], 1u);
+        for (int j = 0; j < 4; ++j) {
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (i + 8 * j < n) v = *reinterpret_cast<const uint4 *>(src + i + 8 * j);   // ld: a multiple of 128
+            w[4 * j] = v.x; w[4 * j + 1] = v.y; w[4 * j + 2] = v.z; w[4 * j + 3] = v.w;
+        }
+        return max(0, min(SK_PER, n - i));
+    };
+    auto key_of = [](const uint32_t (&w)[16], int e) -> uint32_t { return (w[e >> 1] >> (16 * (e & 1))) & 0xFFFFu; };
+    // ---- pass 1: top 12 bits
+    for (int base = 0; base < n; base += SK_STILE) {
+        uint32_t w[16];
+        const int live = load32(base, w);
+#pragma unroll
+        for (int e = 0; e < SK_PER; ++e)
+            if (e < live) atomicAdd(&sm.h1[key_of(w, e) >> 4], 1u);
     }
     __syncthreads();
-    if (warp == 0) sk_find_bin(sm.h1, k, &sm.d1, &sm.k1);
-    __syncthreads();
+    sk_find_bin4096(sm.h1, k, sm.wsum, &sm.d1, &sm.k1);
     const uint32_t d1 = sm.d1;
-    // ---- pass 2: low byte within bin d1
-    for (int base = 0; base < n; base += SK_TILE) {
-        uint16_t kk[8];
-        load8(base, kk);
+    // ---- pass 2: low 4 bits within bin d1
+    for (int base = 0; base < n; base += SK_STILE) {
+        uint32_t w[16];
+        const int live = load32(base, w);
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
-            if (base + 8 * tid + e < n && (uint32_t)(kk[e] >> 8) == d1) atomicAdd(&sm.h2[kk[e] & 0xFFu], 1u);
+        for (int e = 0; e < SK_PER; ++e) {
+            const uint32_t key = key_of(w, e);
+            if (e < live && (key >> 4) == d1) atomicAdd(&sm.h2[key & 0xFu], 1u);
+        }
     }
     __syncthreads();
     if (warp == 0) {
-        sk_find_bin(sm.h2, sm.k1, &sm.d2, &sm.k2);
+        sk_find_bin(sm.h2, sm.k1, &sm.d2, &sm.k2);   // bins 16-255 are empty
         __syncwarp();
         if (lane == 0) sm.n_amb = sm.h2[sm.d2];
     }
     __syncthreads();
-    const uint32_t T = (d1 << 8) | sm.d2;
+    const uint32_t T = (d1 << 4) | sm.d2;
     const uint32_t k2 = sm.k2, n_amb = sm.n_amb;
     const int n_sure = (int)(k - k2);
     // ---- pass 3: ids above T and equal to T, ascending
     {
         int pos_s = 0, pos_a = 0;
-        for (int base = 0; base < n; base += SK_TILE) {
-            uint16_t kk[8];
-            load8(base, kk);
-            int cs = 0, ca = 0;
+        for (int base = 0; base < n; base += SK_STILE) {
+            uint32_t w[16];
+            const int live = load32(base, w);
+            uint32_t gt = 0, eq = 0;   // bit e: key e lies above T / equals T
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const bool live = base + 8 * tid + e < n;
-                cs += (live && kk[e] > T) ? 1 : 0;
-                ca += (live && kk[e] == T) ? 1 : 0;
+            for (int e = 0; e < SK_PER; ++e) {
+                const uint32_t key = key_of(w, e);
+                gt |= (e < live && key > T) ? (1u << e) : 0u;
+                eq |= (e < live && key == T) ? (1u << e) : 0u;
             }
             int os, oa, ts, ta;
-            sk_scan2(cs, ca, sm.wsum, os, oa, ts, ta);
+            sk_scan2(__popc(gt), __popc(eq), sm.wsum, os, oa, ts, ta);
             os += pos_s;
             oa += pos_a;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const bool live = base + 8 * tid + e < n;
-                const uint32_t id = (uint32_t)(base + 8 * tid + e);
-                if (live && kk[e] > T) {
-                    if (os < 2048) sm.sure[os] = id;
-                    ++os;
-                }
-                if (live && kk[e] == T) {
-                    if (oa < SK_AMB_CAP) sm.amb[oa] = id;
-                    ++oa;
-                }
+            const uint32_t id0 = (uint32_t)(base + SK_PER * tid);
+            while (gt) {   // few keys per row pass: walk the set bits
+                const int e = __ffs(gt) - 1;
+                gt &= gt - 1u;
+                if (os < 2048) sm.sure[os] = id0 + (uint32_t)e;
+                ++os;
+            }
+            while (eq) {
+                const int e = __ffs(eq) - 1;
+                eq &= eq - 1u;
+                if (oa < SK_AMB_CAP) sm.amb[oa] = id0 + (uint32_t)e;
+                ++oa;
             }
             pos_s += ts;
             pos_a += ta;
@@ -807,7 +871,7 @@ __global__ void __launch_bounds__(SK_THREADS) select_keys_kernel(KeySelParams p)
             sm.need = k2;
         }
         for (int byte = 3; byte >= 0; --byte) {
-            for (int i = tid; i < 256; i += SK_THREADS) sm.h1[i] = 0;
+            for (int i = tid; i < 256; i += SK_THREADS) sm.h2[i] = 0;
             __syncthreads();
             const uint32_t prefix = sm.prefix;
             for (int base = 0; base < n; base += SK_TILE) {
@@ -819,12 +883,12 @@ __global__ void __launch_bounds__(SK_THREADS) select_keys_kernel(KeySelParams p)
                     const uint32_t ek = score_key(sk_score(sm, kp + (int64_t)(base + 8 * tid + e) * kIdxDim, p.mode,
                                                            p.relu));
                     const bool match = byte == 3 || (ek >> (8 * (byte + 1))) == prefix;
-                    if (match) atomicAdd(&sm.h1[(ek >> (8 * byte)) & 0xFFu], 1u);
+                    if (match) atomicAdd(&sm.h2[(ek >> (8 * byte)) & 0xFFu], 1u);
                 }
             }
             __syncthreads();
             if (warp == 0) {
-                sk_find_bin(sm.h1, sm.need, &sm.d2, &sm.k1);   // (d2, k1 reused as scratch: T is kept above)
+                sk_find_bin(sm.h2, sm.need, &sm.d2, &sm.k1);   // (d2, k1 reused as scratch: T is kept above)
                 __syncwarp();
                 if (lane == 0) {
                     sm.prefix = (prefix << 8) | sm.d2;
