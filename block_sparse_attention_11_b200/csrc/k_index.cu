@@ -625,26 +625,24 @@ __device__ __forceinline__ void sk_find_bin4096(const uint32_t *h, uint32_t k, i
     const int tid = threadIdx.x;
     const int lo = 16 * (SK_THREADS - 1 - tid);   // this thread's lowest bin
     const uint4 *src = reinterpret_cast<const uint4 *>(h + lo);
-    uint32_t c[16];
+    uint32_t mine = 0;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const uint4 v = src[j];
-        c[4 * j] = v.x; c[4 * j + 1] = v.y; c[4 * j + 2] = v.z; c[4 * j + 3] = v.w;
+        mine += (v.x + v.y) + (v.z + v.w);
     }
-    uint32_t mine = 0;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) mine += c[j];
     int above, unused, ta, tb;   // keys in the bins above this thread's (threads of lower index)
     sk_scan2((int)mine, 0, wsum, above, unused, ta, tb);
     uint32_t cum = (uint32_t)above;
     if (cum < k && cum + mine >= k) {
-#pragma unroll
         for (int j = 15; j >= 0; --j) {
-            if (cum < k && cum + c[j] >= k) {
+            const uint32_t c = h[lo + j];
+            if (cum + c >= k) {
                 *d_out = (uint32_t)(lo + j);
                 *k_out = k - cum;
+                break;
             }
-            cum += c[j];
+            cum += c;
         }
     }
     __syncthreads();
@@ -710,7 +708,36 @@ __device__ __forceinline__ float sk_score(const KeySelSmem &sm, const __nv_bfloa
     return tot;
 }
 
-__global__ void __launch_bounds__(SK_THREADS) select_keys_kernel(KeySelParams p) {
+// The same score by one warp: lane l multiplies dims 4 l .. 4 l + 3 (one 8-byte
+// load of the key), a butterfly sum adds the lanes (every lane ends with the
+// same value).
+__device__ __forceinline__ float sk_score_warp(const KeySelSmem &sm, const __nv_bfloat16 *kb, int mode, int relu) {
+    const int lane = threadIdx.x & 31;
+    const uint2 raw = __ldg(reinterpret_cast<const uint2 *>(kb) + lane);
+    const float2 k01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
+    const float2 k23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));
+    auto dot = [&](const float *q) {
+        const float4 qv = reinterpret_cast<const float4 *>(q)[lane];
+        float a = qv.x * k01.x;
+        a = fmaf(qv.y, k01.y, a);
+        a = fmaf(qv.z, k23.x, a);
+        a = fmaf(qv.w, k23.y, a);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+        return a;
+    };
+    if (mode == 0) return dot(sm.q);
+    float tot = 0.f;
+#pragma unroll
+    for (int h = 0; h < kIdxHeads; ++h) {
+        float acc = dot(sm.q + h * kIdxDim);
+        if (relu) acc = fmaxf(acc, 0.f);
+        tot = fmaf(sm.w[h], acc, tot);
+    }
+    return tot;
+}
+
+__global__ void __launch_bounds__(SK_THREADS, 6) select_keys_kernel(KeySelParams p) {
     extern __shared__ __align__(16) uint8_t ksm_raw[];
     KeySelSmem &sm = *reinterpret_cast<KeySelSmem *>(ksm_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -730,14 +757,17 @@ __global__ void __launch_bounds__(SK_THREADS) select_keys_kernel(KeySelParams p)
     }
     const uint16_t *src = p.keys + ((int64_t)seq * p.row_count + rloc) * p.ld;
     const __nv_bfloat16 *kp = p.k_pool + (int64_t)seq * p.pool_stride * kIdxDim;
-    // the row's query operand (fp32) and head weights
+    // the row's query operand (fp32) and head weights: loaded now, stored to shared
+    // memory after pass 3 (only the re-score reads them), so no pass waits for them
+    static_assert(kIdxDim <= SK_THREADS && kIdxHeads * kIdxDim == 2 * SK_THREADS, "operand staging");
+    float qv0 = 0.f, qv1 = 0.f, wv = 1.f;
     if (p.mode == 0) {
-        for (int i = tid; i < kIdxDim; i += SK_THREADS)
-            sm.q[i] = __bfloat162float(p.qa0[qrow * kIdxDim + i]) + __bfloat162float(p.qa1[qrow * kIdxDim + i]);
+        if (tid < kIdxDim)
+            qv0 = __bfloat162float(p.qa0[qrow * kIdxDim + tid]) + __bfloat162float(p.qa1[qrow * kIdxDim + tid]);
     } else {
-        for (int i = tid; i < kIdxHeads * kIdxDim; i += SK_THREADS)
-            sm.q[i] = __bfloat162float(p.qa0[qrow * kIdxHeads * kIdxDim + i]);
-        if (tid < kIdxHeads) sm.w[tid] = p.head_w ? p.head_w[qrow * kIdxHeads + tid] : 1.f;
+        qv0 = __bfloat162float(p.qa0[qrow * kIdxHeads * kIdxDim + tid]);
+        qv1 = __bfloat162float(p.qa0[qrow * kIdxHeads * kIdxDim + SK_THREADS + tid]);
+        if (tid < kIdxHeads && p.head_w) wv = p.head_w[qrow * kIdxHeads + tid];
     }
     for (int i = tid; i < 4096 / 4; i += SK_THREADS) reinterpret_cast<uint4 *>(sm.h1)[i] = make_uint4(0, 0, 0, 0);
     for (int i = tid; i < 256; i += SK_THREADS) sm.h2[i] = 0;
@@ -777,19 +807,27 @@ __global__ void __launch_bounds__(SK_THREADS) select_keys_kernel(KeySelParams p)
         for (int e = 0; e < SK_PER; ++e)
             if (e < live) atomicAdd(&sm.h1[key_of(w, e) >> 4], 1u);
     }
+    // the next pass's first tile is loaded while the bin is searched (likewise before pass 3)
+    uint32_t wpre[16];
+    int lpre = load32(0, wpre);
     __syncthreads();
     sk_find_bin4096(sm.h1, k, sm.wsum, &sm.d1, &sm.k1);
     const uint32_t d1 = sm.d1;
     // ---- pass 2: low 4 bits within bin d1
-    for (int base = 0; base < n; base += SK_STILE) {
-        uint32_t w[16];
-        const int live = load32(base, w);
+    auto pass2_tile = [&](const uint32_t (&w)[16], int live) {
 #pragma unroll
         for (int e = 0; e < SK_PER; ++e) {
             const uint32_t key = key_of(w, e);
             if (e < live && (key >> 4) == d1) atomicAdd(&sm.h2[key & 0xFu], 1u);
         }
+    };
+    pass2_tile(wpre, lpre);
+    for (int base = SK_STILE; base < n; base += SK_STILE) {
+        uint32_t w[16];
+        const int live = load32(base, w);
+        pass2_tile(w, live);
     }
+    lpre = load32(0, wpre);
     __syncthreads();
     if (warp == 0) {
         sk_find_bin(sm.h2, sm.k1, &sm.d2, &sm.k2);   // bins 16-255 are empty
@@ -803,9 +841,7 @@ __global__ void __launch_bounds__(SK_THREADS) select_keys_kernel(KeySelParams p)
     // ---- pass 3: ids above T and equal to T, ascending
     {
         int pos_s = 0, pos_a = 0;
-        for (int base = 0; base < n; base += SK_STILE) {
-            uint32_t w[16];
-            const int live = load32(base, w);
+        auto pass3_tile = [&](const uint32_t (&w)[16], int live, int base) {
             uint32_t gt = 0, eq = 0;   // bit e: key e lies above T / equals T
 #pragma unroll
             for (int e = 0; e < SK_PER; ++e) {
@@ -832,13 +868,28 @@ __global__ void __launch_bounds__(SK_THREADS) select_keys_kernel(KeySelParams p)
             }
             pos_s += ts;
             pos_a += ta;
+        };
+        pass3_tile(wpre, lpre, 0);
+        for (int base = SK_STILE; base < n; base += SK_STILE) {
+            uint32_t w[16];
+            const int live = load32(base, w);
+            pass3_tile(w, live, base);
         }
+    }
+    if (p.mode == 0) {
+        if (tid < kIdxDim) sm.q[tid] = qv0;
+    } else {
+        sm.q[tid] = qv0;
+        sm.q[SK_THREADS + tid] = qv1;
+        if (tid < kIdxHeads) sm.w[tid] = wv;
     }
     __syncthreads();
     if (n_amb <= (uint32_t)SK_AMB_CAP) {
-        // ---- re-score the keys equal to T (one thread each), rank, pick the k2 best
-        for (uint32_t i = tid; i < n_amb; i += SK_THREADS)
-            sm.amb_s[i] = sk_score(sm, kp + (int64_t)sm.amb[i] * kIdxDim, p.mode, p.relu);
+        // ---- re-score the keys equal to T (a warp each), rank, pick the k2 best
+        for (uint32_t i = warp; i < n_amb; i += SK_THREADS / 32) {
+            const float sc = sk_score_warp(sm, kp + (int64_t)sm.amb[i] * kIdxDim, p.mode, p.relu);
+            if (lane == 0) sm.amb_s[i] = sc;
+        }
         __syncthreads();
         for (uint32_t i = tid; i < n_amb; i += SK_THREADS) {
             const float si = sm.amb_s[i];
