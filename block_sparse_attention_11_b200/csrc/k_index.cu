@@ -542,8 +542,10 @@ __global__ void __launch_bounds__(SR_THREADS)
 //   pass 2  histogram of the low 4 bits within bin d1: the threshold key
 //           T = (d1, d2) and k2, the picks among the keys equal to T;
 //   pass 3  ids of keys > T (exactly k - k2) and of keys == T, each list in
-//           ascending id order (per 2048-element tile a block scan orders
-//           the writes);
+//           ascending id order (per 8192-element tile a block scan orders
+//           the writes).  Rows of several tiles whose keys above bin d1 and
+//           in it number at most SK_LIST skip it: pass 2 lists those keys in
+//           id order with their low 4 bits, and the list is split instead;
 //   rank    the keys == T are re-scored; the k2 best (score descending, id
 //           ascending: the ranking's tie rule) join the picks;
 //   merge   both ascending lists merge into the row's ascending selection.
@@ -555,6 +557,7 @@ constexpr int SK_THREADS = 256;
 constexpr int SK_TILE = SK_THREADS * 8;    // elements per tile: one 16-byte load per thread (massive ties)
 constexpr int SK_PER = 32;                 // passes 1-3: contiguous keys per thread (four 16-byte loads in flight)
 constexpr int SK_STILE = SK_THREADS * SK_PER;
+constexpr int SK_LIST = 4096;              // one-read rows: keys above bin d1 and in it, listed in pass 2
 constexpr int SK_AMB_CAP = 2048;
 
 struct KeySelSmem {
@@ -571,7 +574,7 @@ struct KeySelSmem {
     float q[kIdxHeads * kIdxDim];         // the row's query operand in fp32 (mode 0: the head sum)
     float w[kIdxHeads];
     int wsum[2][SK_THREADS / 32];
-    uint32_t d1, k1, d2, k2, n_amb, prefix, need;
+    uint32_t d1, k1, n_d1, d2, k2, n_amb, prefix, need;
 };
 
 struct KeySelParams {
@@ -616,11 +619,11 @@ __device__ __forceinline__ void sk_find_bin(const uint32_t *h, uint32_t k, uint3
 __device__ __forceinline__ void sk_scan2(int a, int b, int (*wsum)[SK_THREADS / 32], int &oa, int &ob, int &ta,
                                          int &tb);
 
-// The k-th largest of 4096 bins counted from the top (the whole CTA): bin d
-// and the picks it supplies.  Thread t owns bins 4095 - 16 t .. 4080 - 16 t.
+// The k-th largest of 4096 bins counted from the top (the whole CTA): bin d,
+// the picks it supplies and its count.  Thread t owns bins 4095 - 16 t .. 4080 - 16 t.
 // Ends with a barrier.
 __device__ __forceinline__ void sk_find_bin4096(const uint32_t *h, uint32_t k, int (*wsum)[SK_THREADS / 32],
-                                                uint32_t *d_out, uint32_t *k_out) {
+                                                uint32_t *d_out, uint32_t *k_out, uint32_t *n_out) {
     static_assert(SK_THREADS * 16 == 4096, "16 bins per thread");
     const int tid = threadIdx.x;
     const int lo = 16 * (SK_THREADS - 1 - tid);   // this thread's lowest bin
@@ -640,6 +643,7 @@ __device__ __forceinline__ void sk_find_bin4096(const uint32_t *h, uint32_t k, i
             if (cum + c >= k) {
                 *d_out = (uint32_t)(lo + j);
                 *k_out = k - cum;
+                *n_out = c;
                 break;
             }
             cum += c;
@@ -811,71 +815,153 @@ __global__ void __launch_bounds__(SK_THREADS, 6) select_keys_kernel(KeySelParams
     uint32_t wpre[16];
     int lpre = load32(0, wpre);
     __syncthreads();
-    sk_find_bin4096(sm.h1, k, sm.wsum, &sm.d1, &sm.k1);
-    const uint32_t d1 = sm.d1;
-    // ---- pass 2: low 4 bits within bin d1
-    auto pass2_tile = [&](const uint32_t (&w)[16], int live) {
-#pragma unroll
-        for (int e = 0; e < SK_PER; ++e) {
-            const uint32_t key = key_of(w, e);
-            if (e < live && (key >> 4) == d1) atomicAdd(&sm.h2[key & 0xFu], 1u);
-        }
-    };
-    pass2_tile(wpre, lpre);
-    for (int base = SK_STILE; base < n; base += SK_STILE) {
-        uint32_t w[16];
-        const int live = load32(base, w);
-        pass2_tile(w, live);
-    }
-    lpre = load32(0, wpre);
-    __syncthreads();
-    if (warp == 0) {
-        sk_find_bin(sm.h2, sm.k1, &sm.d2, &sm.k2);   // bins 16-255 are empty
-        __syncwarp();
-        if (lane == 0) sm.n_amb = sm.h2[sm.d2];
-    }
-    __syncthreads();
-    const uint32_t T = (d1 << 4) | sm.d2;
-    const uint32_t k2 = sm.k2, n_amb = sm.n_amb;
-    const int n_sure = (int)(k - k2);
-    // ---- pass 3: ids above T and equal to T, ascending
-    {
-        int pos_s = 0, pos_a = 0;
-        auto pass3_tile = [&](const uint32_t (&w)[16], int live, int base) {
-            uint32_t gt = 0, eq = 0;   // bit e: key e lies above T / equals T
+    sk_find_bin4096(sm.h1, k, sm.wsum, &sm.d1, &sm.k1, &sm.n_d1);
+    const uint32_t d1 = sm.d1, k1 = sm.k1;
+    uint32_t T, k2, n_amb;
+    if (n > SK_STILE && (k - k1) + sm.n_d1 <= (uint32_t)SK_LIST) {
+        // ---- pass 2, rows of several tiles whose keys above bin d1 (k - k1 of
+        // them, all picked) and in it fit the list: pass 2 writes them in id
+        // order (entry: id | low 4 bits << 16 | above bin d1 << 20) beside the
+        // low-4-bit histogram of bin d1, and the row is not read again.  (A
+        // one-tile row re-reads its tile from L2 for less than the list costs.)
+        uint32_t *list = sm.h1;   // the pass-1 counts are no longer read
+        int pos = 0;
+        auto tile = [&](const uint32_t (&w)[16], int live, int base) {
+            uint32_t am = 0, cm = 0;
+            uint32_t nib[4] = {0u, 0u, 0u, 0u};   // low 4 bits of key e at bits 4 (e & 7) of nib[e >> 3]
 #pragma unroll
             for (int e = 0; e < SK_PER; ++e) {
-                const uint32_t key = key_of(w, e);
-                gt |= (e < live && key > T) ? (1u << e) : 0u;
-                eq |= (e < live && key == T) ? (1u << e) : 0u;
+                const uint32_t key = key_of(w, e), b = key >> 4;
+                const bool in = e < live && b == d1;
+                am |= (e < live && b > d1) ? (1u << e) : 0u;
+                cm |= in ? (1u << e) : 0u;
+                nib[e >> 3] |= (key & 0xFu) << (4 * (e & 7));
+                if (in) atomicAdd(&sm.h2[key & 0xFu], 1u);
             }
-            int os, oa, ts, ta;
-            sk_scan2(__popc(gt), __popc(eq), sm.wsum, os, oa, ts, ta);
-            os += pos_s;
-            oa += pos_a;
+            uint32_t all = am | cm;
+            int o, ob, t, tb;
+            sk_scan2(__popc(all), 0, sm.wsum, o, ob, t, tb);
+            o += pos;
             const uint32_t id0 = (uint32_t)(base + SK_PER * tid);
-            while (gt) {   // few keys per row pass: walk the set bits
-                const int e = __ffs(gt) - 1;
-                gt &= gt - 1u;
-                if (os < 2048) sm.sure[os] = id0 + (uint32_t)e;
-                ++os;
+            while (all) {   // a few keys per thread and tile
+                const int e = __ffs(all) - 1;
+                all &= all - 1u;
+                const uint32_t nw = e < 16 ? (e < 8 ? nib[0] : nib[1]) : (e < 24 ? nib[2] : nib[3]);
+                if (o < SK_LIST) list[o] = (id0 + (uint32_t)e) | (((nw >> (4 * (e & 7))) & 0xFu) << 16) | (((am >> e) & 1u) << 20);
+                ++o;
             }
-            while (eq) {
-                const int e = __ffs(eq) - 1;
-                eq &= eq - 1u;
-                if (oa < SK_AMB_CAP) sm.amb[oa] = id0 + (uint32_t)e;
-                ++oa;
-            }
-            pos_s += ts;
-            pos_a += ta;
+            pos += t;
         };
-        pass3_tile(wpre, lpre, 0);
+        tile(wpre, lpre, 0);
         for (int base = SK_STILE; base < n; base += SK_STILE) {
             uint32_t w[16];
             const int live = load32(base, w);
-            pass3_tile(w, live, base);
+            tile(w, live, base);
+        }
+        __syncthreads();
+        if (warp == 0) {
+            sk_find_bin(sm.h2, k1, &sm.d2, &sm.k2);   // bins 16-255 are empty
+            __syncwarp();
+            if (lane == 0) sm.n_amb = sm.h2[sm.d2];
+        }
+        __syncthreads();
+        const uint32_t d2 = sm.d2;
+        T = (d1 << 4) | d2;
+        k2 = sm.k2;
+        n_amb = sm.n_amb;
+        // ---- the list split in id order: keys above T and keys equal to T
+        static_assert(SK_LIST == 16 * SK_THREADS, "16 list entries per thread");
+        const int nl = min(pos, SK_LIST);
+        const int j0 = 16 * tid;
+        uint32_t gt = 0, eq = 0;   // bit j: entry j0 + j lies above T / equals T
+        for (int j = 0; j < 16 && j0 + j < nl; ++j) {
+            const uint32_t ent = list[j0 + j];
+            const uint32_t nib = (ent >> 16) & 0xFu;
+            const bool above = (ent >> 20) & 1u;
+            gt |= (above || nib > d2) ? (1u << j) : 0u;
+            eq |= (!above && nib == d2) ? (1u << j) : 0u;
+        }
+        int os, oa, ts, ta;
+        sk_scan2(__popc(gt), __popc(eq), sm.wsum, os, oa, ts, ta);
+        // the list is read again below; nothing writes over it before the barrier after this split
+        while (gt) {
+            const int j = __ffs(gt) - 1;
+            gt &= gt - 1u;
+            if (os < 2048) sm.sure[os] = list[j0 + j] & 0xFFFFu;
+            ++os;
+        }
+        while (eq) {
+            const int j = __ffs(eq) - 1;
+            eq &= eq - 1u;
+            if (oa < SK_AMB_CAP) sm.amb[oa] = list[j0 + j] & 0xFFFFu;
+            ++oa;
+        }
+    } else {
+        // ---- pass 2: low 4 bits within bin d1
+        auto pass2_tile = [&](const uint32_t (&w)[16], int live) {
+#pragma unroll
+            for (int e = 0; e < SK_PER; ++e) {
+                const uint32_t key = key_of(w, e);
+                if (e < live && (key >> 4) == d1) atomicAdd(&sm.h2[key & 0xFu], 1u);
+            }
+        };
+        pass2_tile(wpre, lpre);
+        for (int base = SK_STILE; base < n; base += SK_STILE) {
+            uint32_t w[16];
+            const int live = load32(base, w);
+            pass2_tile(w, live);
+        }
+        lpre = load32(0, wpre);
+        __syncthreads();
+        if (warp == 0) {
+            sk_find_bin(sm.h2, sm.k1, &sm.d2, &sm.k2);   // bins 16-255 are empty
+            __syncwarp();
+            if (lane == 0) sm.n_amb = sm.h2[sm.d2];
+        }
+        __syncthreads();
+        T = (d1 << 4) | sm.d2;
+        k2 = sm.k2;
+        n_amb = sm.n_amb;
+        // ---- pass 3: ids above T and equal to T, ascending
+        {
+            int pos_s = 0, pos_a = 0;
+            auto pass3_tile = [&](const uint32_t (&w)[16], int live, int base) {
+                uint32_t gt = 0, eq = 0;   // bit e: key e lies above T / equals T
+#pragma unroll
+                for (int e = 0; e < SK_PER; ++e) {
+                    const uint32_t key = key_of(w, e);
+                    gt |= (e < live && key > T) ? (1u << e) : 0u;
+                    eq |= (e < live && key == T) ? (1u << e) : 0u;
+                }
+                int os, oa, ts, ta;
+                sk_scan2(__popc(gt), __popc(eq), sm.wsum, os, oa, ts, ta);
+                os += pos_s;
+                oa += pos_a;
+                const uint32_t id0 = (uint32_t)(base + SK_PER * tid);
+                while (gt) {   // few keys per row pass: walk the set bits
+                    const int e = __ffs(gt) - 1;
+                    gt &= gt - 1u;
+                    if (os < 2048) sm.sure[os] = id0 + (uint32_t)e;
+                    ++os;
+                }
+                while (eq) {
+                    const int e = __ffs(eq) - 1;
+                    eq &= eq - 1u;
+                    if (oa < SK_AMB_CAP) sm.amb[oa] = id0 + (uint32_t)e;
+                    ++oa;
+                }
+                pos_s += ts;
+                pos_a += ta;
+            };
+            pass3_tile(wpre, lpre, 0);
+            for (int base = SK_STILE; base < n; base += SK_STILE) {
+                uint32_t w[16];
+                const int live = load32(base, w);
+                pass3_tile(w, live, base);
+            }
         }
     }
+    const int n_sure = (int)(k - k2);
     if (p.mode == 0) {
         if (tid < kIdxDim) sm.q[tid] = qv0;
     } else {
