@@ -10,7 +10,7 @@ import torch
 
 import workloads
 from qsa_testlib import (TOL, check_prefill_workload, decode_selection_matches, np32, rope_of,
-                         stage_isolated_decode)
+                         selection_report, stage_isolated_decode)
 
 pytestmark = pytest.mark.gpu
 
@@ -1080,3 +1080,31 @@ def test_prefill_select_massive_16bit_ties(qsa, flags):
                               relu=bool(flags & qsa.QSA_SCORE_RELU))
     assert np.array_equal(nsel[0].cpu().numpy()[rows], ref["nsel"])
     assert np.array_equal(sel[0].cpu().numpy()[rows], ref["sel"])
+
+
+@pytest.mark.parametrize("eps", [0.02, 0.03])
+def test_prefill_select_crowded_bins_multi_tile(qsa, eps):
+    """Compressed keys 1 + U(-eps, eps): every score of a row is close to the
+    same value, so a row's keys crowd into one or two 12-bit bins and tie in
+    the hundreds at 16 bits.  Rows of more than 8192 blocks whose keys above
+    and in the threshold's 12-bit bin exceed the select's 4096-entry list
+    (eps 0.02: about 6900 and 10000 at rows 36000 and 39999) read the row a
+    third time; the others (eps 0.03, row 39999: about 1070) are listed in
+    pass 2.  Both agree with the oracle under the 1e-4 gap rule."""
+    T, top_k = 40000, 512
+    g = torch.Generator().manual_seed(43)
+    q_idx = torch.randn(1, T, 4, 128, generator=g).to(torch.bfloat16)
+    k_pool = (1.0 + eps * (2 * torch.rand(1, T // 4, 128, generator=g) - 1)).to(torch.bfloat16)
+    q_idx, k_pool = q_idx.to(DEV), k_pool.to(DEV)
+    sel = torch.full((1, T, top_k), -7, dtype=torch.int32, device=DEV)
+    nsel = torch.full((1, T), -7, dtype=torch.int32, device=DEV)
+    qsa.qsa_index_topk_prefill(q_idx, k_pool, sel, nsel, top_k=top_k, rope=qsa.Rope())
+    qsa.qsa_check_status()
+    rows = [32775, 36000, 38000, 39999]
+    qi, kp = np32(q_idx[0]), np32(k_pool[0])
+    ref = oracle.prefill_rows(rows, q_idx=qi, k_pool=kp, top_k=top_k, store_bf16=True)
+
+    def score_fn(rr):
+        return oracle.prefill_rows(rr, q_idx=qi, k_pool=kp, top_k=top_k, store_bf16=True, want_scores=True)["scores"]
+
+    selection_report(sel[0].cpu().numpy()[rows], nsel[0].cpu().numpy()[rows], ref, score_fn, rows)
