@@ -19,7 +19,7 @@
 //
 // Tile shape: M = 128 (TMEM lanes), N = 128 key blocks, K = 128 (two
 // 64-element 128-byte-swizzled k-atoms).  The query tile is loaded once per
-// CTA and stays in shared memory; key tiles stream through a 4-stage TMA
+// CTA and stays in shared memory; key tiles stream through a 3-stage TMA
 // ring; two TMEM accumulators (128 columns each) let the epilogue of tile j
 // overlap the MMAs of tile j+1.  Warp roles: 0 = TMA producer, 1 = MMA issuer
 // and TMEM owner, 2..9 = epilogue: two warps per TMEM lane quarter (warp w
